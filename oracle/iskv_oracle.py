@@ -1,0 +1,314 @@
+"""Float64 CPU oracle of the iS-KV hot path: block-incremental truncated SVD of a growing row set
+plus decode attention over the reconstructed cache.
+
+TEST INFRASTRUCTURE ONLY. The product package never imports, links or runs anything here; only
+``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` do. It shares no
+code with the CUDA path: the two meet only in the seeded inputs of ``iskv_synth``.
+
+Source: "iS-KV: Online Low-Rank KV Cache Compression via Block-Incremental SVD" (summary page).
+
+* section "Theoretical Foundation": the rank-budgeted objective and the truncated SVD ``SVD_r``,
+  which keeps ``k = min(r, n, d)`` singular triplets with orthonormal ``U``, ``B``;
+* section "Architecture Overview": per K/V path an exact window of the most recent tokens plus a
+  low-rank history;
+* section "Block-Incremental Decoding Updates": steps 1-3 (residual ``E = F - (F B) B^T``, residual
+  basis ``P`` via QR and SVD, augmented core ``Z = [[Sigma, 0], [F B, F P]]``, core SVD
+  ``(G, Sigma+, H) = SVD_r(Z)``, ``U+ = diag(U, I_b) G``, ``B+ = [B P] H``);
+* section "Reconstruction and Storage": compressed rows are ``(U Sigma B^T)[j]``, the others the
+  exact rows; persistent storage ``k (n + d + 1)`` factor scalars per path plus ``d e`` exact
+  scalars.
+
+Readings taken where the page is silent (each also stated at its definition):
+
+* fold trigger: rows are appended one at a time; whenever the exact window holds ``window +
+  block`` rows, its oldest ``block`` rows are folded, so ``n_c(t) = block * floor(max(0, t -
+  window) / block)`` and decode at ``t`` tokens sees positions ``0 .. t-1``;
+* the residual is projected twice (classical Gram-Schmidt, twice);
+* ``P`` spans the numerical row space of ``E`` (singular values above ``1e-12 max(1, ||F||_2)``),
+  re-orthogonalised against ``B``; ``p`` is that numerical rank;
+* the retained rank after a fold is ``min(r, k + p)``; zero singular values are kept;
+* RoPE pairs channel ``j`` with ``j + d/2`` at angle ``pos * theta^(-2j/d)``; keys are stored
+  before RoPE and rotated at attention time, queries arrive rotated; scale ``1/sqrt(d)``; q-head
+  ``g`` reads kv-head ``g // (n_q / n_kv)``;
+* the "stale coordinates" variant (``rotate=False``) updates ``Sigma`` and ``B`` exactly as above
+  but keeps the old rows' coordinates ``U Sigma`` unrotated (zero-padded or truncated to the new
+  rank) and reconstructs them against the new basis; new rows get ``F B+``.
+
+Parity: every function here is pinned by ``tests/test_oracle_*.py`` (closed forms, library special
+cases, invariants and brute force); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "svd_r",
+    "n_compressed",
+    "residual_basis",
+    "fold",
+    "fold_from_coords",
+    "OracleUnit",
+    "OracleCache",
+    "rope",
+    "attention",
+]
+
+
+# ----------------------------------------------------------------------------------------------
+# Theoretical Foundation
+# ----------------------------------------------------------------------------------------------
+def svd_r(X: np.ndarray, r: int):
+    """Truncated SVD ``SVD_r(X) = (U, sigma, B)`` keeping ``k = min(r, n, d)`` components.
+
+    iS-KV summary, section "Theoretical Foundation": the optimum of the rank-``r`` objective.
+    """
+    U, s, Vt = np.linalg.svd(np.asarray(X, dtype=np.float64), full_matrices=False)
+    k = min(r, X.shape[0], X.shape[1])
+    return U[:, :k], s[:k], Vt[:k].T
+
+
+def n_compressed(t: int, block: int, window: int) -> int:
+    """Rows in the low-rank history after ``t`` tokens (fold when window + block rows are exact).
+
+    iS-KV summary, section "Architecture Overview" (exact window of the most recent ``w`` tokens)
+    with the reading that a fold consumes the oldest ``block`` rows as soon as ``window + block``
+    rows are exact.
+    """
+    return block * (max(0, t - window) // block)
+
+
+# ----------------------------------------------------------------------------------------------
+# Block-Incremental Decoding Updates
+# ----------------------------------------------------------------------------------------------
+def residual_basis(F: np.ndarray, B: np.ndarray):
+    """Step 1: residual ``E = F - (F B) B^T`` and an orthonormal residual basis ``P``.
+
+    The projection is applied twice (the page gives it once; twice keeps ``E`` orthogonal to ``B``
+    to rounding). ``P`` is found "via QR and SVD": QR of ``E^T``, then the SVD of the R factor
+    keeps the directions with singular value above ``1e-12 max(1, ||F||_2)``; ``P`` is finally
+    re-orthogonalised against ``B``. Returns ``(E, P)`` with ``P`` of shape ``d x p``.
+    """
+    F = np.asarray(F, dtype=np.float64)
+    d = F.shape[1]
+    k = B.shape[1]
+    if k:
+        E = F - (F @ B) @ B.T
+        E = E - (E @ B) @ B.T
+    else:
+        E = F.copy()
+    Q, R = np.linalg.qr(E.T)                 # d x m, m x b   (m = min(d, b))
+    Ur, sr, _ = np.linalg.svd(R)
+    tol = 1e-12 * max(1.0, float(np.linalg.norm(F, 2)))
+    p = int(np.count_nonzero(sr > tol))
+    P = Q @ Ur[:, :p]
+    if k and p:
+        P = P - B @ (B.T @ P)
+        P = np.linalg.qr(P)[0]
+    return E, P.reshape(d, p)
+
+
+def fold(U: np.ndarray, sigma: np.ndarray, B: np.ndarray, F: np.ndarray, r: int):
+    """One block-incremental update of ``A = U diag(sigma) B^T`` with the pending block ``F``.
+
+    iS-KV summary, section "Block-Incremental Decoding Updates", steps 1-3:
+    ``Z = [[Sigma, 0], [F B, F P]]`` of size ``(k+b) x (k+p)``, ``(G, Sigma+, H) = SVD_r(Z)``,
+    ``U+ = diag(U, I_b) G`` and ``B+ = [B P] H``. The retained rank is ``min(r, k + p)``.
+
+    Returns ``(U+, sigma+, B+, H, P)``.
+    """
+    F = np.asarray(F, dtype=np.float64)
+    b, d = F.shape
+    n, k = U.shape[0], sigma.size
+    _, P = residual_basis(F, B)
+    p = P.shape[1]
+    Z = np.zeros((k + b, k + p))
+    Z[:k, :k] = np.diag(sigma)
+    Z[k:, :k] = F @ B
+    Z[k:, k:] = F @ P
+    G, s, Ht = np.linalg.svd(Z, full_matrices=False)
+    kp = min(r, k + p)
+    G, s, H = G[:, :kp], s[:kp], Ht[:kp].T
+    Ublk = np.zeros((n + b, k + b))
+    Ublk[:n, :k] = U
+    Ublk[n:, k:] = np.eye(b)
+    U_new = Ublk @ G
+    B_new = np.hstack([B, P]) @ H
+    return U_new, s, B_new, H, P
+
+
+def fold_from_coords(C: np.ndarray, sigma: np.ndarray, B: np.ndarray, F: np.ndarray, r: int):
+    """One fold started from stored coordinates ``C = U diag(sigma)`` (e.g. a GPU state).
+
+    ``U`` is recovered as ``C diag(1/sigma)`` on the columns with ``sigma > 0`` (zero columns
+    otherwise), then :func:`fold` runs. Returns ``(C+, sigma+, B+, H_top)`` where ``C+ = U+
+    diag(sigma+)`` and ``H_top = H[:k]`` maps old coordinates to new ones.
+    """
+    sigma = np.asarray(sigma, dtype=np.float64)
+    k = sigma.size
+    U = np.zeros_like(np.asarray(C, dtype=np.float64)[:, :k])
+    nz = sigma > 0
+    U[:, nz] = np.asarray(C, dtype=np.float64)[:, :k][:, nz] / sigma[nz]
+    U_new, s, B_new, H, _ = fold(U, sigma, np.asarray(B, dtype=np.float64)[:, :k], F, r)
+    return U_new * s, s, B_new, H[:k]
+
+
+class OracleUnit:
+    """One (sequence, layer, kv-head, path) of the cache: exact window plus low-rank history.
+
+    iS-KV summary, section "Architecture Overview" (two components per K/V path) and section
+    "Reconstruction and Storage".
+    """
+
+    def __init__(self, d: int, rank: int, block: int, window: int, rotate: bool = True):
+        self.d, self.rank, self.block, self.window, self.rotate = d, rank, block, window, rotate
+        self.U = np.zeros((0, 0))
+        self.sigma = np.zeros(0)
+        self.B = np.zeros((d, 0))
+        self.C_stale = np.zeros((0, 0))      # stored coordinates when rotate=False
+        self._exact: list[np.ndarray] = []
+        self.t = 0
+        self.n = 0
+        self.folds = 0
+
+    # -- state ---------------------------------------------------------------------------------
+    @property
+    def k(self) -> int:
+        return self.sigma.size
+
+    @property
+    def exact(self) -> np.ndarray:
+        return np.asarray(self._exact, dtype=np.float64).reshape(len(self._exact), self.d)
+
+    def coords(self) -> np.ndarray:
+        """Stored history coordinates ``U Sigma`` (``n x k``)."""
+        if not self.rotate:
+            return self.C_stale
+        return self.U * self.sigma
+
+    def storage_scalars(self) -> int:
+        """Persistent scalars of this path: ``k (n + d + 1)`` factors plus ``d e`` exact values.
+
+        iS-KV summary, section "Reconstruction and Storage" (storage formula, per path).
+        """
+        return self.k * (self.n + self.d + 1) + self.d * len(self._exact)
+
+    # -- updates -------------------------------------------------------------------------------
+    def append(self, rows: np.ndarray) -> int:
+        """Append rows one by one; fold the oldest ``block`` exact rows whenever the window holds
+        ``window + block`` rows. Returns the number of folds done."""
+        done = 0
+        for row in np.atleast_2d(np.asarray(rows, dtype=np.float64)):
+            self._exact.append(row.copy())
+            self.t += 1
+            while len(self._exact) >= self.window + self.block:
+                F = np.asarray(self._exact[: self.block])
+                del self._exact[: self.block]
+                self._fold(F)
+                done += 1
+        return done
+
+    def _fold(self, F: np.ndarray) -> None:
+        k_old = self.k
+        U_new, s, B_new, H, _ = fold(self.U, self.sigma, self.B, F, self.rank)
+        if not self.rotate:
+            kp = s.size
+            C = np.zeros((self.n, kp))
+            m = min(k_old, kp)
+            C[:, :m] = self.C_stale[:, :m]
+            self.C_stale = np.vstack([C, F @ B_new])
+        self.U, self.sigma, self.B = U_new, s, B_new
+        self.n += F.shape[0]
+        self.folds += 1
+
+    # -- reading -------------------------------------------------------------------------------
+    def reconstruct(self) -> np.ndarray:
+        """``X~``: compressed rows ``(U Sigma B^T)[i]`` for ``i < n``, exact rows after."""
+        hist = self.coords() @ self.B.T if self.n else np.zeros((0, self.d))
+        return np.vstack([hist, self.exact])
+
+
+# ----------------------------------------------------------------------------------------------
+# Decode attention over the reconstructed cache
+# ----------------------------------------------------------------------------------------------
+def rope(X: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
+    """Rotary embedding, half-split pairs ``(j, j + d/2)`` at angle ``pos * theta^(-2j/d)``."""
+    X = np.asarray(X, dtype=np.float64)
+    d = X.shape[-1]
+    h = d // 2
+    omega = theta ** (-2.0 * np.arange(h, dtype=np.float64) / d)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * omega[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = X[..., :h], X[..., h:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """Softmax attention of one query over rows of ``K``/``V``, scale ``1/sqrt(d)``, float64."""
+    q = np.asarray(q, dtype=np.float64)
+    s = (np.asarray(K, dtype=np.float64) @ q) / math.sqrt(q.size)
+    s = s - s.max()
+    p = np.exp(s)
+    p /= p.sum()
+    return p @ np.asarray(V, dtype=np.float64)
+
+
+class OracleCache:
+    """All units of a cache: ``[layer][sequence][kv-head]`` for the K and V paths."""
+
+    def __init__(self, batch: int, n_layers: int, n_kv_heads: int, n_q_heads: int,
+                 head_dim: int, rank_k: int, rank_v: int, block: int, window: int,
+                 rope: bool = False, rope_theta: float = 5e5, rotate: bool = True):
+        self.batch, self.n_layers, self.n_kv, self.n_q = batch, n_layers, n_kv_heads, n_q_heads
+        self.d, self.rope, self.theta = head_dim, rope, rope_theta
+        self.units = [[[[OracleUnit(head_dim, rank_k if w == 0 else rank_v, block, window, rotate)
+                         for w in range(2)] for _ in range(n_kv_heads)] for _ in range(batch)]
+                      for _ in range(n_layers)]
+
+    def unit(self, layer: int, seq: int, head: int, which: int) -> OracleUnit:
+        return self.units[layer][seq][head][which]
+
+    def tokens(self, layer: int) -> int:
+        return self.units[layer][0][0][0].t
+
+    def append(self, layer: int, K: np.ndarray, V: np.ndarray) -> None:
+        """``K``, ``V``: ``[batch][n_kv][m][d]`` rows (pre-RoPE keys)."""
+        for s in range(self.batch):
+            for h in range(self.n_kv):
+                self.units[layer][s][h][0].append(K[s, h])
+                self.units[layer][s][h][1].append(V[s, h])
+
+    def keys_values(self, layer: int, seq: int, head: int):
+        """Reconstructed keys (RoPE applied when enabled) and values of one kv-head."""
+        K = self.units[layer][seq][head][0].reconstruct()
+        V = self.units[layer][seq][head][1].reconstruct()
+        if self.rope:
+            K = rope(K, np.arange(K.shape[0]), self.theta)
+        return K, V
+
+    def decode(self, layer: int, q: np.ndarray) -> np.ndarray:
+        """``q``: ``[batch][n_q][d]`` (already rotated) -> ``[batch][n_q][d]`` attention output."""
+        if self.tokens(layer) == 0:
+            raise ValueError("decode over an empty cache")
+        G = self.n_q // self.n_kv
+        out = np.zeros((self.batch, self.n_q, self.d))
+        for s in range(self.batch):
+            for h in range(self.n_kv):
+                K, V = self.keys_values(layer, s, h)
+                for g in range(h * G, (h + 1) * G):
+                    out[s, g] = attention(q[s, g], K, V)
+        return out
+
+    def reconstruct(self, layer: int, which: int, apply_rope: bool = False) -> np.ndarray:
+        """``[batch][n_kv][t][d]`` reconstructed rows of the K (0) or V (1) path."""
+        out = []
+        for s in range(self.batch):
+            row = []
+            for h in range(self.n_kv):
+                X = self.units[layer][s][h][which].reconstruct()
+                if apply_rope and which == 0:
+                    X = rope(X, np.arange(X.shape[0]), self.theta)
+                row.append(X)
+            out.append(row)
+        return np.asarray(out)

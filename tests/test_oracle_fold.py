@@ -1,0 +1,236 @@
+"""Pins of the float64 oracle's block-incremental SVD (no GPU).
+
+Each test ties the oracle to something other than itself: the library SVD of the stacked matrix
+that the page says every fold optimises (iS-KV summary, "Block-Incremental Decoding Updates"),
+Eckart-Young, exactness without truncation, invariants, and closed forms of the schedule and of
+the storage formula ("Reconstruction and Storage").
+"""
+import numpy as np
+import pytest
+
+import iskv_synth as syn
+from oracle import OracleUnit, fold, fold_from_coords, n_compressed, residual_basis, svd_r
+
+
+def _stream(T, d, seed, decay=1.0, noise=1e-3):
+    rng = np.random.default_rng(seed)
+    G = np.linalg.qr(rng.standard_normal((T, d)))[0] * np.sqrt(T)
+    H = np.linalg.qr(rng.standard_normal((d, d)))[0]
+    s = np.arange(1, d + 1, dtype=float) ** -decay
+    return (G * s) @ H.T + noise * rng.standard_normal((T, d))
+
+
+def _projector(B):
+    return B @ B.T
+
+
+# ---------------------------------------------------------------------------------------------
+# T1: the first fold (k = 0) is the plain truncated SVD of the block
+# ---------------------------------------------------------------------------------------------
+def test_first_fold_is_truncated_svd_of_block():
+    F = _stream(12, 10, 1)
+    r = 4
+    U, s, B, H, P = fold(np.zeros((0, 0)), np.zeros(0), np.zeros((10, 0)), F, r)
+    Ur, sr, Br = svd_r(F, r)
+    np.testing.assert_allclose(s, sr, rtol=1e-12)
+    np.testing.assert_allclose(_projector(B), _projector(Br), atol=1e-10)
+    np.testing.assert_allclose((U * s) @ B.T, (Ur * sr) @ Br.T, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# T2: every fold equals SVD_r([previous reconstruction; F])
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("d,r,b", [(16, 4, 3), (16, 6, 8), (8, 3, 7), (12, 12, 5)])
+def test_every_fold_is_svd_of_stacked_rows(d, r, b):
+    X = _stream(10 * b, d, 2 + d + r + b, decay=0.7)
+    U, s, B = np.zeros((0, 0)), np.zeros(0), np.zeros((d, 0))
+    for f in range(10):
+        F = X[f * b:(f + 1) * b]
+        A = (U * s) @ B.T if U.shape[0] else np.zeros((0, d))
+        M = np.vstack([A, F])
+        U, s, B, H, P = fold(U, s, B, F, r)
+        Um, sm, Bm = svd_r(M, r)
+        kp = s.size
+        np.testing.assert_allclose(s, sm[:kp], rtol=1e-10, atol=1e-13)
+        full = np.linalg.svd(M, compute_uv=False)
+        if kp < full.size and (full[kp - 1] - full[kp]) / full[0] > 1e-3:
+            np.testing.assert_allclose(_projector(B), _projector(Bm[:, :kp]), atol=1e-9)
+        np.testing.assert_allclose((U * s) @ B.T, (Um[:, :kp] * sm[:kp]) @ Bm[:, :kp].T,
+                                   atol=1e-9 * max(1.0, full[0]))
+
+
+def test_unit_schedule_matches_manual_folds():
+    d, r, b, w = 8, 3, 4, 6
+    X = _stream(50, d, 7)
+    unit = OracleUnit(d, r, b, w)
+    U, s, B = np.zeros((0, 0)), np.zeros(0), np.zeros((d, 0))
+    nf = 0
+    for t in range(1, 51):
+        unit.append(X[t - 1:t])
+        assert unit.n == n_compressed(t, b, w)
+        while nf * b < n_compressed(t, b, w):
+            U, s, B, _, _ = fold(U, s, B, X[nf * b:(nf + 1) * b], r)
+            nf += 1
+        np.testing.assert_allclose(unit.sigma, s, rtol=1e-12)
+        rec = unit.reconstruct()
+        assert rec.shape == (t, d)
+        np.testing.assert_array_equal(rec[unit.n:], X[unit.n:t])     # exact window rows
+
+
+# ---------------------------------------------------------------------------------------------
+# T3: Eckart-Young on a single block, and optimality against random rank-r subspaces
+# ---------------------------------------------------------------------------------------------
+def test_eckart_young_tail_energy_single_block():
+    F = _stream(20, 12, 3, decay=0.5, noise=0.05)
+    r = 5
+    U, s, B, _, _ = fold(np.zeros((0, 0)), np.zeros(0), np.zeros((12, 0)), F, r)
+    Fh = (U * s) @ B.T
+    err2 = np.linalg.norm(F - Fh) ** 2
+    # orthogonal projection: ||F - F^||^2 = ||F||^2 - sum of kept sigma^2
+    assert err2 == pytest.approx(np.linalg.norm(F) ** 2 - np.sum(s ** 2), rel=1e-10)
+    # tail energy equals the discarded squared singular values (computed from the Gram matrix)
+    lam = np.sort(np.linalg.eigvalsh(F.T @ F))[::-1]
+    assert err2 == pytest.approx(lam[r:].sum(), rel=1e-8)
+    # no random rank-r right subspace does better
+    rng = np.random.default_rng(0)
+    for _ in range(2000):
+        Q = np.linalg.qr(rng.standard_normal((12, r)))[0]
+        assert np.linalg.norm(F - F @ Q @ Q.T) ** 2 >= err2 * (1 - 1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# T4: no truncation -> the factorisation is the full SVD of all folded rows
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("b,w", [(3, 4), (5, 0), (16, 2)])
+def test_no_truncation_is_exact_full_svd(b, w):
+    d = 8
+    X = _stream(41, d, 11, noise=0.1)
+    unit = OracleUnit(d, d, b, w)
+    unit.append(X)
+    n = unit.n
+    assert n == n_compressed(41, b, w)
+    np.testing.assert_allclose(unit.reconstruct(), X, atol=1e-12)
+    sv = np.linalg.svd(X[:n], compute_uv=False)
+    np.testing.assert_allclose(unit.sigma, sv[:unit.k], rtol=1e-11)
+    Vt = np.linalg.svd(X[:n], full_matrices=False)[2]
+    np.testing.assert_allclose(_projector(unit.B), _projector(Vt[:unit.k].T), atol=1e-10)
+
+
+# ---------------------------------------------------------------------------------------------
+# T5: data of exact rank q <= r reconstructs exactly
+# ---------------------------------------------------------------------------------------------
+def test_exact_low_rank_reconstructs():
+    wl = syn.WORKLOADS[0]
+    X = syn.kv_rows(300, 32, 5, 1.0, variant="lowrank", rank=3)
+    unit = OracleUnit(32, 5, 16, 20)
+    unit.append(X)
+    rel = np.linalg.norm(unit.reconstruct() - X) / np.linalg.norm(X)
+    assert rel <= 1e-12
+    assert wl.head_dim == 128
+    # the residual basis of a block that lies inside span(B) is empty
+    E, P = residual_basis(X[:16] @ unit.B @ unit.B.T, unit.B)
+    assert P.shape[1] == 0 and np.linalg.norm(E) <= 1e-12 * np.linalg.norm(X[:16])
+
+
+# ---------------------------------------------------------------------------------------------
+# T6: orthonormal factors; C^T C = Sigma^2
+# ---------------------------------------------------------------------------------------------
+def test_factors_orthonormal():
+    d = 32
+    X = _stream(400, d, 13, decay=0.8, noise=0.01)
+    unit = OracleUnit(d, 7, 16, 24)
+    unit.append(X)
+    I = np.eye(unit.k)
+    assert np.abs(unit.B.T @ unit.B - I).max() <= 1e-12
+    assert np.abs(unit.U.T @ unit.U - I).max() <= 1e-12
+    C = unit.coords()
+    np.testing.assert_allclose(C.T @ C, np.diag(unit.sigma ** 2), atol=1e-10 * unit.sigma[0] ** 2)
+    assert np.all(np.diff(unit.sigma) <= 0)
+
+
+# ---------------------------------------------------------------------------------------------
+# T7: drift of stale coordinates vs none with rotated coordinates; global error bounds
+# ---------------------------------------------------------------------------------------------
+def test_drift_stale_vs_rotated():
+    d, r, b, w = 32, 6, 16, 16
+    X = _stream(16 * 24 + w, d, 17, decay=0.4, noise=0.05)
+    sync = OracleUnit(d, r, b, w, rotate=True)
+    stale = OracleUnit(d, r, b, w, rotate=False)
+    drifts = []
+    for f in range(24):
+        rows = X[: b + w] if f == 0 else X[b + w + (f - 1) * b: b + w + f * b]
+        sync.append(rows)
+        stale.append(rows)
+        a = sync.reconstruct()[: sync.n]
+        s_ = stale.reconstruct()[: stale.n]
+        drifts.append(np.linalg.norm(s_ - a) / np.linalg.norm(a))
+    # identical basis trajectory
+    np.testing.assert_allclose(stale.sigma, sync.sigma, rtol=1e-12)
+    np.testing.assert_allclose(stale.B, sync.B, atol=1e-12)
+    assert drifts[0] <= 1e-12            # one fold: nothing old to rotate yet
+    assert drifts[1] > 1e-3              # second fold: old coordinates are in the old basis
+    assert drifts[-1] > drifts[1]        # and the stale history keeps drifting
+    n = sync.n
+    err = np.linalg.norm(X[:n] - sync.reconstruct()[:n])
+    u, s, v = svd_r(X[:n], r)
+    opt = np.linalg.norm(X[:n] - (u * s) @ v.T)
+    assert err >= opt * (1 - 1e-12)      # no streaming result beats the global SVD_r
+
+
+def test_error_bounded_by_sum_of_discarded_energy():
+    d, r, b = 16, 4, 6
+    X = _stream(60, d, 19, decay=0.6, noise=0.05)
+    U, s, B = np.zeros((0, 0)), np.zeros(0), np.zeros((d, 0))
+    bound = 0.0
+    for f in range(10):
+        F = X[f * b:(f + 1) * b]
+        A = (U * s) @ B.T if U.shape[0] else np.zeros((0, d))
+        M2 = np.linalg.norm(A) ** 2 + np.linalg.norm(F) ** 2
+        U, s, B, _, _ = fold(U, s, B, F, r)
+        bound += np.sqrt(max(M2 - np.sum(s ** 2), 0.0))
+        n = (f + 1) * b
+        err = np.linalg.norm(X[:n] - (U * s) @ B.T)
+        assert err <= bound * (1 + 1e-10) + 1e-12
+
+
+# ---------------------------------------------------------------------------------------------
+# one fold started from stored coordinates equals the fold of the (U, Sigma, B) state
+# ---------------------------------------------------------------------------------------------
+def test_fold_from_coords_matches_fold():
+    d, r, b = 16, 5, 4
+    X = _stream(40, d, 23)
+    U, s, B = np.zeros((0, 0)), np.zeros(0), np.zeros((d, 0))
+    for f in range(6):
+        U, s, B, _, _ = fold(U, s, B, X[f * b:(f + 1) * b], r)
+    F = X[24:28]
+    C1, s1, B1, Ht = fold_from_coords(U * s, s, B, F, r)
+    U2, s2, B2, H2, _ = fold(U, s, B, F, r)
+    np.testing.assert_allclose(C1, U2 * s2, atol=1e-12)
+    np.testing.assert_allclose(s1, s2, rtol=1e-13)
+    # history rotation identity: old coordinates times H[:k] are the top rows of U+ Sigma+
+    np.testing.assert_allclose((U * s) @ Ht, (U2 * s2)[: U.shape[0]], atol=1e-12)
+    # new-row coordinates are F B+
+    np.testing.assert_allclose(F @ B2, (U2 * s2)[U.shape[0]:], atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# schedule and storage closed forms
+# ---------------------------------------------------------------------------------------------
+def test_schedule_closed_forms():
+    assert n_compressed(4096, 64, 256) == 3840               # Llama-3-8B layer workload
+    assert n_compressed(65536, 512, 512) == 65024            # long-context prefill
+    assert n_compressed(65536 + 2048, 512, 512) == 65024 + 2048
+    assert n_compressed(1088, 32, 64) == 1024                # single-head workload
+    for t in range(0, 2000, 7):
+        n = n_compressed(t, 64, 256)
+        e = t - n
+        assert n % 64 == 0 and (e == t if t < 256 else 256 <= e <= 256 + 63)
+
+
+def test_storage_formula_counts_stored_scalars():
+    d = 16
+    unit = OracleUnit(d, 4, 5, 7)
+    unit.append(_stream(53, d, 29))
+    stored = unit.coords().size + unit.B.size + unit.sigma.size + unit.exact.size
+    assert unit.storage_scalars() == stored
+    assert stored == unit.k * (unit.n + d + 1) + d * (53 - unit.n)
