@@ -30,6 +30,9 @@ Readings taken where the page is silent (each also stated at its definition):
 * RoPE pairs channel ``j`` with ``j + d/2`` at angle ``pos * theta^(-2j/d)``; keys are stored
   before RoPE and rotated at attention time, queries arrive rotated; scale ``1/sqrt(d)``; q-head
   ``g`` reads kv-head ``g // (n_q / n_kv)``;
+* singular vectors are sign-ambiguous; each fold orients new basis vector ``c`` along old basis
+  vector ``c`` (``H[c, c] >= 0`` for ``c < k``). Reconstructions and attention do not depend on
+  it; the stale-coordinate variant does;
 * the "stale coordinates" variant (``rotate=False``) updates ``Sigma`` and ``B`` exactly as above
   but keeps the old rows' coordinates ``U Sigma`` unrotated (zero-padded or truncated to the new
   rank) and reconstructs them against the new basis; new rows get ``F B+``.
@@ -129,7 +132,15 @@ def fold(U: np.ndarray, sigma: np.ndarray, B: np.ndarray, F: np.ndarray, r: int)
     Z[k:, k:] = F @ P
     G, s, Ht = np.linalg.svd(Z, full_matrices=False)
     kp = min(r, k + p)
-    G, s, H = G[:, :kp], s[:kp], Ht[:kp].T
+    G, s, H = G[:, :kp], s[:kp], Ht[:kp].T.copy()
+    G = G.copy()
+    # sign convention (the page fixes none; singular vectors are sign-ambiguous): new basis
+    # vector c points along old basis vector c, i.e. H[c, c] >= 0 for c < k. Reconstructions do
+    # not depend on it; the stale-coordinate variant does.
+    for c in range(min(k, kp)):
+        if H[c, c] < 0:
+            H[:, c] = -H[:, c]
+            G[:, c] = -G[:, c]
     Ublk = np.zeros((n + b, k + b))
     Ublk[:n, :k] = U
     Ublk[n:, k:] = np.eye(b)
