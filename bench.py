@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark of the iS-KV hot path on B200: streamed decode over a block-incrementally compressed
+KV cache (Llama-3-8B-shaped layer: 8 kv / 32 q heads, d=128, 4096 generated tokens, b=64, w=256,
+r_K=32, r_V=48, RoPE theta=5e5, bf16 rows, batch 1 per GPU).
+
+One step = one pass of the whole hot path over one sequence batch: for each of the 4096 tokens,
+append its K/V rows (window append, and a block-incremental fold of every path whenever the window
+releases a block: 60 folds x 8 heads x 2 paths = 960 head-block updates) and run decode attention
+of the 32 q-heads over the compressed history plus the exact window. The step's C-ABI calls are
+captured once into a CUDA graph and replayed; inputs (rows and queries of all 4096 tokens) are
+resident in HBM when the timed region starts; L2 is flushed (256 MiB write) before every timed
+step.
+
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the same workload.
+Multi-GPU (torchrun): every rank streams its own independent sequence batch (weak scaling, no
+collective on the data path); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import iskv_synth as syn  # noqa: E402
+
+WL = syn.WORKLOADS[1]
+METRIC = "decode tok/s over compressed KV"
+UNIT = "tok/s"
+D = 128
+
+
+# ---------------------------------------------------------------------------------------------
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=5)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--sample-every", type=int, default=16,
+                   help="decode calls between event-timed samples inside the graph")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def workload_inputs(seq: int):
+    """Token-major device-layout rows [T][1][H][D] for K and V, float64 values, queries."""
+    T, H = WL.tokens, WL.n_kv_heads
+    kd = np.empty((T, 1, H, D), np.uint16)
+    vd = np.empty((T, 1, H, D), np.uint16)
+    for h in range(H):
+        kd[:, 0, h], _ = syn.workload_rows(WL, seq, 0, h, 0)
+        vd[:, 0, h], _ = syn.workload_rows(WL, seq, 0, h, 1)
+    q = syn.queries(syn.unit_seed(WL.cfg_id, seq, 0, 0, 0), (T, 1, WL.n_q_heads, D))
+    return kd, vd, q
+
+
+def decode_bytes(t: int) -> int:
+    """Algorithmic bytes of one decode call at t tokens (all kv-heads of the layer): fp32
+    coordinates of the compressed rows, bf16 window rows (K and V), fp32 bases, q and out."""
+    n = WL.n_c(t)
+    e = t - n
+    kK = kV = 0
+    if n:
+        f = n // WL.block
+        k = [0, 0]
+        for _ in range(f):
+            for x, r in ((0, WL.rank_k), (1, WL.rank_v)):
+                k[x] = min(r, k[x] + min(WL.block, D - k[x]))
+        kK, kV = k
+    per_unit = 4 * n * (kK + kV) + 2 * 2 * e * D + 4 * D * (kK + kV) + 2 * 4 * WL.group * D
+    return WL.n_kv_heads * per_unit
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except Exception:
+                self.p.kill()
+
+    def summary(self):
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+        sm = [num(r[1]) for r in rows]
+        mx = [num(r[2]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": float(np.nanmedian(sm)), "sm_max_mhz": float(np.nanmax(mx)),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------------
+def oracle_sample(seq: int = 0, heads: int = 2, decodes: int = 256):
+    """Times the float64 oracle on a bounded sample of the workload and extrapolates to tok/s:
+    ``heads`` of the 8 kv-heads (their K and V paths and q-heads), all 4096 appends with their
+    folds, and ``decodes`` of the 4096 decode steps evenly spaced in t."""
+    from threadpoolctl import threadpool_info
+
+    from oracle import OracleCache
+    T, G = WL.tokens, WL.group
+    kv = np.empty((1, heads, T, D))
+    vv = np.empty((1, heads, T, D))
+    for h in range(heads):
+        kv[0, h] = syn.workload_rows(WL, seq, 0, h, 0)[1]
+        vv[0, h] = syn.workload_rows(WL, seq, 0, h, 1)[1]
+    q = syn.queries(syn.unit_seed(WL.cfg_id, seq, 0, 0, 0), (T, 1, WL.n_q_heads, D))
+    q = q[:, :, : heads * G].astype(np.float64)
+    orc = OracleCache(1, 1, heads, heads * G, D, WL.rank_k, WL.rank_v, WL.block, WL.window,
+                      rope=True, rope_theta=WL.rope_theta)
+    marks = sorted(set(np.linspace(1, T, decodes).round().astype(int).tolist()))
+    t_app = t_dec = 0.0
+    t = 0
+    for m in marks:
+        a = time.perf_counter()
+        orc.append(0, kv[:, :, t:m], vv[:, :, t:m])
+        b = time.perf_counter()
+        orc.decode(0, q[m - 1])
+        c = time.perf_counter()
+        t_app += b - a
+        t_dec += c - b
+        t = m
+    full = (t_app + t_dec * T / len(marks)) * (WL.n_kv_heads / heads)
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {
+        "value": T / full,
+        "unit": UNIT,
+        "cores": int(threads),
+        "host_cores": len(os.sched_getaffinity(0)),
+        "kind": "oracle",
+        "sample": (f"{heads} of {WL.n_kv_heads} kv-heads (K+V paths, {heads * G} q-heads): all "
+                   f"{T} appends with their folds and {len(marks)} of {T} decode steps evenly "
+                   f"spaced in t; extrapolated linearly to all heads and steps"),
+        "sample_seconds": t_app + t_dec,
+    }
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(heads=1, decodes=48)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        s = oracle_sample(heads=1, decodes=48)
+        vals.append(s["value"])
+        secs.append(s["sample_seconds"])
+    v = float(np.mean(vals))
+    s["value"] = v
+    out = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * WL.tokens / v, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WL.name, "global_batch": WL.batch * args.gpus,
+                   "seq_len": WL.tokens, "parallelism": f"replicas{args.gpus}"},
+        "cpu_baseline": {k: s[k] for k in ("kind", "cores", "sample", "value", "unit")},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "sample_seconds_per_step": float(np.mean(secs)),
+    }
+    print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    from cuda.bindings import runtime as rt
+
+    import rank_kv_cache_isvd_b200 as iskv
+    from rank_kv_cache_isvd_b200.cache import IsKVCache
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    T, H, QH = WL.tokens, WL.n_kv_heads, WL.n_q_heads
+    kd, vd, q = workload_inputs(seq=rank)
+    K = torch.from_numpy(kd.view(np.int16)).to(dev).view(torch.bfloat16)   # [T][1][H][D]
+    V = torch.from_numpy(vd.view(np.int16)).to(dev).view(torch.bfloat16)
+    Q = torch.from_numpy(q).to(dev)                                          # [T][1][QH][D]
+    OUT = torch.empty_like(Q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    cache = IsKVCache(batch=1, n_layers=1, n_kv_heads=H, n_q_heads=QH, rank_k=WL.rank_k,
+                      rank_v=WL.rank_v, block=WL.block, window=WL.window, max_tokens=T,
+                      kv_dtype="bf16", rope=True, rope_theta=WL.rope_theta)
+    h = cache.handle
+    kb, vb, qb, ob = K.data_ptr(), V.data_ptr(), Q.data_ptr(), OUT.data_ptr()
+    krow = H * D * 2
+    qrow = QH * D * 4
+
+    def ev():
+        err, e = rt.cudaEventCreate()
+        assert err == rt.cudaError_t.cudaSuccess
+        return e
+
+    def rec(e, s):
+        err, = rt.cudaEventRecordWithFlags(e, s, rt.cudaEventRecordExternal)
+        assert err == rt.cudaError_t.cudaSuccess
+
+    dec_marks = [(t, ev(), ev()) for t in range(args.sample_every - 1, T, args.sample_every)]
+    dec_set = {t: (a, b) for t, a, b in dec_marks}
+    fold_ts = [t for t in range(T) if WL.n_c(t + 1) > WL.n_c(t)]
+    fold_marks = {t: (ev(), ev()) for t in fold_ts}
+
+    def step(stream_handle: int, timed_events: bool):
+        iskv.check(iskv.iskv_reset(h, stream_handle))
+        for t in range(T):
+            fm = fold_marks.get(t) if timed_events else None
+            if fm:
+                rec(fm[0], stream_handle)
+            iskv.check(iskv.iskv_append_block(h, 0, kb + t * krow, vb + t * krow, 1, stream_handle))
+            if fm:
+                rec(fm[1], stream_handle)
+            dm = dec_set.get(t) if timed_events else None
+            if dm:
+                rec(dm[0], stream_handle)
+            iskv.check(iskv.iskv_decode_attn(h, 0, qb + t * qrow, ob + t * qrow, stream_handle))
+            if dm:
+                rec(dm[1], stream_handle)
+
+    s = torch.cuda.Stream(device=dev)
+    sh = s.cuda_stream
+    # eager warm-up (function attributes, first-touch), then parity-relevant status check
+    with torch.cuda.stream(s):
+        step(sh, False)
+    assert iskv.iskv_sync_status(h, sh) == 0, "device status after eager step"
+    n0 = cache.launches()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step(sh, True)
+    launches_per_step = cache.launches() - n0
+    for _ in range(args.warmup):
+        with torch.cuda.stream(s):
+            g.replay()
+    torch.cuda.synchronize(dev)
+
+    def elapsed(a, b):
+        err, ms = rt.cudaEventElapsedTime(a, b)
+        assert err == rt.cudaError_t.cudaSuccess
+        return ms
+
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    torch.cuda.synchronize(dev)
+    step_ms, dec_ms, dec_bytes, fold_ms = [], [], [], []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local_rank) as clk:
+        for _ in range(args.steps):
+            with torch.cuda.stream(s):
+                flush.zero_()
+                e0.record(s)
+                g.replay()
+                e1.record(s)
+            s.synchronize()
+            step_ms.append(e0.elapsed_time(e1))
+            for t, a, b in dec_marks:
+                dec_ms.append(elapsed(a, b))
+                dec_bytes.append(decode_bytes(t + 1))
+            fold_ms.append(sum(elapsed(a, b) for a, b in fold_marks.values()))
+    torch.cuda.synchronize(dev)
+    clocks = clk.summary()
+    total_ms = float(np.sum(step_ms))
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    value = world * WL.batch * T / (ms_per_step / 1e3)
+
+    # ---- end to end through the public API with host buffers --------------------------------
+    kh = torch.from_numpy(kd.view(np.int16)).view(torch.bfloat16).pin_memory()
+    vh = torch.from_numpy(vd.view(np.int16)).view(torch.bfloat16).pin_memory()
+    qh = torch.from_numpy(q).pin_memory()
+    oh = torch.empty(OUT.shape, dtype=OUT.dtype).pin_memory()
+    e2e_ms = []
+    for i in range(args.steps + 1):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0.record(s)
+            K.copy_(kh, non_blocking=True)
+            V.copy_(vh, non_blocking=True)
+            Q.copy_(qh, non_blocking=True)
+            g.replay()
+            oh.copy_(OUT, non_blocking=True)
+            e1.record(s)
+        s.synchronize()
+        if i:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = float(np.sum(e2e_ms))
+    if world > 1:
+        tt = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_total = float(tt.item())
+    e2e_value = world * WL.batch * T / (e2e_total / args.steps / 1e3)
+    h2d = (kh.numel() + vh.numel()) * 2 + qh.numel() * 4
+    d2h = oh.numel() * 4
+    status = iskv.iskv_sync_status(h, sh)
+    assert status == 0, f"device status {status}"
+
+    # ---- roofline of the dominant kernel class --------------------------------------------------
+    hbm, which = peaks()
+    dec_total = float(np.mean(dec_ms)) * T          # per step, from the sampled launches
+    fold_total = float(np.mean(fold_ms))
+    achieved = float(np.sum(dec_bytes)) / (float(np.sum(dec_ms)) / 1e3) / 1e9
+    updates = len(fold_ts) * H * 2
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WL.name, "global_batch": world * WL.batch, "seq_len": T,
+                   "kv_heads": H, "q_heads": QH, "block": WL.block, "window": WL.window,
+                   "rank_k": WL.rank_k, "rank_v": WL.rank_v, "kv_dtype": "bf16",
+                   "parallelism": f"replicas{world}", "l2": "flushed (256 MiB write) before each step",
+                   "graph": "the step's C-ABI calls captured once into a CUDA graph"},
+        "roofline": {"bound": "hbm", "kernel": "decode attention (split + combine)",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "peak_source": f"{which} MEASURED_PEAKS hbm_gbs",
+                     "bytes_per_launch_mean": float(np.mean(dec_bytes)),
+                     "launch_us_mean": 1e3 * float(np.mean(dec_ms))},
+        "fold": {"head_block_updates_per_s": updates / (fold_total / 1e3),
+                 "updates_per_step": updates, "fold_ms_per_step": fold_total,
+                 "us_per_fold_call": 1e3 * fold_total / len(fold_ts)},
+        "decode_ms_per_step": dec_total,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h),
+                "how": "pinned host rows+queries copied in, graph replay, outputs copied out"},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample()
+        out["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        out["cpu_baseline"]["host_cores"] = cb["host_cores"]
+    del g
+    cache.close()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

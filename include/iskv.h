@@ -1,0 +1,183 @@
+/*
+ * iskv.h - C ABI of the iS-KV hot path on one B200 (sm_100a): block-incremental truncated SVD of
+ * each (layer, sequence, kv-head) key and value stream, plus decode attention over the compressed
+ * history and an exact recent window.
+ *
+ * Method: "iS-KV: Online Low-Rank KV Cache Compression via Block-Incremental SVD" (summary page).
+ *   - "Architecture Overview": per K/V path an exact window of the most recent tokens and a
+ *     low-rank history of rank at most r.
+ *   - "Block-Incremental Decoding Updates": each fold takes the pending block F (b rows), forms the
+ *     residual E = F - (F B) B^T and an orthonormal residual basis P, the core
+ *     Z = [[Sigma, 0], [F B, F P]], its truncated SVD (G, Sigma+, H), and the updated factors
+ *     U+ = diag(U, I_b) G, B+ = [B P] H. Old rows' coordinates move with the basis.
+ *   - "Reconstruction and Storage": compressed row i is (U Sigma B^T)[i]; window rows are exact;
+ *     storage k (n + d + 1) factor scalars per path plus d e exact scalars.
+ *
+ * Conventions shared by every entry point:
+ *   - Return value: ISKV_OK (0) or a negative ISKV_ERR_* code; no C++ exception crosses the ABI.
+ *     Argument errors are detected on the host before anything is enqueued.
+ *   - Pointers named *_dev are device pointers owned by the caller; they must stay valid until
+ *     the work enqueued on `stream` has completed. Pointers to host scalars are written before
+ *     the call returns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). All device work is enqueued on
+ *     it asynchronously; nothing synchronises except iskv_sync_status().
+ *   - The handle owns all persistent device state, allocated once by iskv_create() and sized by
+ *     max_tokens; it is never reallocated. A handle is not thread-safe.
+ *   - Each layer keeps its own token count t; layer = -1 addresses all layers at once (they must
+ *     then hold the same t).
+ *   - Device-side failures (a core SVD that did not converge, a non-finite singular value) set a
+ *     sticky status word that iskv_sync_status() returns.
+ */
+#ifndef ISKV_H
+#define ISKV_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct iskv_handle iskv_handle;
+/* Layout-compatible with cudaStream_t. */
+typedef struct CUstream_st *iskv_stream_t;
+
+enum {
+    ISKV_OK = 0,
+    ISKV_ERR_INVALID_ARG = -1,  /* bad config, NULL pointer, layer out of range, ...        */
+    ISKV_ERR_CAPACITY = -2,     /* t + m > max_tokens                                        */
+    ISKV_ERR_CUDA = -3,         /* a CUDA runtime call failed (allocation, launch, copy)     */
+    ISKV_ERR_NOT_CONVERGED = -4,/* a core SVD hit its sweep cap (sticky, device side)        */
+    ISKV_ERR_NONFINITE = -5,    /* a non-finite singular value appeared (sticky, device side) */
+    ISKV_ERR_UNSUPPORTED = -6   /* valid request outside what this build implements          */
+};
+
+enum { ISKV_BF16 = 0, ISKV_F32 = 1 };
+
+typedef struct {
+    int batch;            /* sequences decoded in lock-step                                  */
+    int n_layers;
+    int n_kv_heads;
+    int n_q_heads;        /* multiple of n_kv_heads; q-head g reads kv-head g / (n_q/n_kv)    */
+    int head_dim;         /* d; must be 128                                                  */
+    int rank_k, rank_v;   /* rank budgets r_K, r_V (1 .. head_dim)                           */
+    int block;            /* b: rows folded per update (1 .. 128)                            */
+    int window;           /* w: exact rows kept before a fold may take them (>= 0)           */
+    long long max_tokens; /* capacity per sequence and layer                                 */
+    int kv_dtype;         /* ISKV_BF16 or ISKV_F32: dtype of appended rows and of the window  */
+    int rope;             /* 1: rotate keys by RoPE (pairs j, j+d/2) after reconstruction     */
+    double rope_theta;    /* RoPE base; angle of pair j at position i is i * theta^(-2j/d)    */
+    int rotate_history;   /* 1: iS-KV (old coordinates rotate with the basis).               */
+                          /* 0: stale-coordinate ablation (drift study only).                */
+} iskv_config;
+
+/*
+ * Creates a cache for `cfg` on the current CUDA device. Allocates every device buffer
+ * (coordinates C = U Sigma [max compressed rows x r] in fp32, bases B [d x r] fp32 (two copies
+ * for in-place updates), Sigma [r] fp32, exact ring of window + block rows per path in kv_dtype,
+ * a RoPE table [max_tokens x d/2] of (cos, sin), decode split partials and a status word).
+ * Errors: ISKV_ERR_INVALID_ARG (cfg out of range), ISKV_ERR_CUDA (allocation failed; nothing
+ * leaks). On success *out owns the handle; release it with iskv_destroy().
+ */
+int iskv_create(const iskv_config *cfg, iskv_handle **out);
+
+/* Frees every device buffer of the handle (synchronises the device first). NULL is a no-op. */
+int iskv_destroy(iskv_handle *h);
+
+/*
+ * Appends m >= 1 new rows per (sequence, kv-head) to the key and value streams of `layer` and
+ * folds every block that the window releases ("Block-Incremental Decoding Updates"): rows enter
+ * the exact window one by one; whenever it holds window + block rows its oldest block is folded,
+ * so after t tokens n_c(t) = block * floor(max(0, t - window) / block) rows are compressed.
+ *   k_rows_dev, v_rows_dev: kv_dtype, row-major [batch][n_kv_heads][m][head_dim] for layer >= 0,
+ *                           [n_layers][batch][n_kv_heads][m][head_dim] for layer == -1.
+ *                           Keys are pre-RoPE.
+ * Errors: ISKV_ERR_INVALID_ARG (NULL rows, m < 1, bad layer, layers with different t for -1),
+ *         ISKV_ERR_CAPACITY (t + m > max_tokens), ISKV_ERR_CUDA (launch failed).
+ */
+int iskv_append_block(iskv_handle *h, int layer, const void *k_rows_dev, const void *v_rows_dev,
+                      int m, iskv_stream_t stream);
+
+/*
+ * Decode attention of `layer` over all t cached positions 0 .. t-1: compressed rows are
+ * reconstructed as C B^T ("Reconstruction and Storage"), keys are then rotated by RoPE at their
+ * position (when cfg.rope), scores use scale 1/sqrt(d), softmax is exact (fp32, log-sum-exp
+ * merge of position splits).
+ *   q_dev:   fp32 [batch][n_q_heads][head_dim], already rotated for the query position.
+ *   out_dev: fp32 [batch][n_q_heads][head_dim].
+ * Errors: ISKV_ERR_INVALID_ARG (NULL pointers, bad layer, t == 0), ISKV_ERR_CUDA.
+ */
+int iskv_decode_attn(iskv_handle *h, int layer, const float *q_dev, float *out_dev,
+                     iskv_stream_t stream);
+
+/*
+ * Writes the reconstructed cache of one path of `layer` ("Reconstruction and Storage"): row i is
+ * (C B^T)[i] for i < n_c and the exact window row otherwise; keys are rotated by RoPE when
+ * apply_rope != 0 (ignored for values).
+ *   which:   0 = keys, 1 = values.
+ *   out_dev: fp32 [batch][n_kv_heads][t][head_dim].
+ * Errors: ISKV_ERR_INVALID_ARG, ISKV_ERR_CUDA.
+ */
+int iskv_reconstruct(iskv_handle *h, int layer, int which, int apply_rope, float *out_dev,
+                     iskv_stream_t stream);
+
+/*
+ * Copies the factors of one unit (layer, seq, kv_head, path) into caller buffers (device to
+ * device, on `stream`) and reports its current rank and compressed-row count.
+ *   coords_dev: fp32 [n_c][rank] (row stride = rank budget of the path), may be NULL;
+ *   basis_dev:  fp32 [head_dim][rank], may be NULL;
+ *   sigma_dev:  fp32 [rank], may be NULL (entries >= *k_out are zero);
+ *   k_out, n_c_out: host pointers, may be NULL.
+ * Errors: ISKV_ERR_INVALID_ARG, ISKV_ERR_CUDA.
+ */
+int iskv_get_factors(iskv_handle *h, int layer, int seq, int kv_head, int which,
+                     float *coords_dev, float *basis_dev, float *sigma_dev, int *k_out,
+                     long long *n_c_out, iskv_stream_t stream);
+
+/*
+ * Empties every layer (t = n_c = 0, rank 0) and clears the sticky status, keeping all device
+ * allocations, so a handle can serve a new batch of sequences. Host bookkeeping plus one
+ * asynchronous device write on `stream`; later calls must be ordered after it on a stream.
+ * Errors: ISKV_ERR_INVALID_ARG, ISKV_ERR_CUDA.
+ */
+int iskv_reset(iskv_handle *h, iskv_stream_t stream);
+
+/*
+ * Number of kernel launches this handle has enqueued since creation (host counter; launches
+ * captured into a CUDA graph are counted once, at capture). Errors: ISKV_ERR_INVALID_ARG.
+ */
+int iskv_launch_count(const iskv_handle *h, long long *count_out);
+
+/* Tokens cached in `layer` (host value). Errors: ISKV_ERR_INVALID_ARG. */
+int iskv_num_tokens(const iskv_handle *h, int layer, long long *t_out);
+
+/*
+ * Persistent bytes of one layer per the storage formula of "Reconstruction and Storage":
+ * beta_f * sum_X k_X (n_X + d + 1) + beta_e * d * sum_X e_X, summed over sequences and kv-heads,
+ * with beta_f = 4 (fp32 factors) and beta_e = bytes of kv_dtype. Host only.
+ */
+int iskv_storage_bytes(const iskv_handle *h, int layer, long long *bytes_out);
+
+/*
+ * Host-only schedule of the fold trigger ("Architecture Overview" window, read as: fold the
+ * oldest block whenever window + block rows are exact). For a stream holding t tokens, appending
+ * m rows leaves *n_c_out compressed rows and performs *folds_out folds. Needs no GPU.
+ * Errors: ISKV_ERR_INVALID_ARG (block < 1, window < 0, t < 0, m < 0).
+ */
+int iskv_schedule(int block, int window, long long t, long long m, long long *n_c_out,
+                  long long *folds_out);
+
+/*
+ * Synchronises `stream` and returns the sticky device status: ISKV_OK, ISKV_ERR_NOT_CONVERGED or
+ * ISKV_ERR_NONFINITE (the first error seen since creation), or ISKV_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+int iskv_sync_status(iskv_handle *h, iskv_stream_t stream);
+
+/* Static description of an error code. */
+const char *iskv_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISKV_H */

@@ -1,0 +1,100 @@
+"""Convenience wrapper over the C ABI: owns an ``iskv_handle`` and allocates caller-side buffers
+with torch (device memory and streams only; all arithmetic runs in ``libiskv.so``)."""
+from __future__ import annotations
+
+import torch
+
+from .binding import (ISKV_BF16, ISKV_F32, check, iskv_append_block, iskv_config, iskv_create,
+                      iskv_decode_attn, iskv_destroy, iskv_get_factors, iskv_launch_count,
+                      iskv_num_tokens, iskv_reconstruct, iskv_reset, iskv_storage_bytes,
+                      iskv_sync_status)
+
+
+class IsKVCache:
+    """iS-KV cache of ``n_layers`` layers x ``batch`` sequences x ``n_kv_heads`` kv-heads."""
+
+    def __init__(self, *, batch: int, n_layers: int, n_kv_heads: int, n_q_heads: int,
+                 rank_k: int, rank_v: int, block: int, window: int, max_tokens: int,
+                 kv_dtype: str = "bf16", rope: bool = True, rope_theta: float = 5e5,
+                 rotate_history: bool = True, head_dim: int = 128):
+        self.cfg = iskv_config(batch, n_layers, n_kv_heads, n_q_heads, head_dim, rank_k, rank_v,
+                               block, window, max_tokens,
+                               ISKV_BF16 if kv_dtype == "bf16" else ISKV_F32, int(rope),
+                               float(rope_theta), int(rotate_history))
+        self.dtype = torch.bfloat16 if kv_dtype == "bf16" else torch.float32
+        self.handle = 0
+        code, h = iskv_create(self.cfg)
+        check(code, "iskv_create")
+        self.handle = h
+
+    # -- lifetime ----------------------------------------------------------------------------
+    def close(self) -> None:
+        if self.handle:
+            iskv_destroy(self.handle)
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- calls ---------------------------------------------------------------------------------
+    def append(self, layer: int, k_rows: torch.Tensor, v_rows: torch.Tensor, stream=None) -> None:
+        """``k_rows``/``v_rows``: ``[batch][n_kv][m][d]`` (or ``[L][batch][n_kv][m][d]`` with
+        ``layer=-1``), contiguous, on the device, in the cache's kv dtype."""
+        assert k_rows.dtype == self.dtype and v_rows.dtype == self.dtype
+        assert k_rows.is_contiguous() and v_rows.is_contiguous()
+        check(iskv_append_block(self.handle, layer, k_rows, v_rows, k_rows.shape[-2], stream),
+              "iskv_append_block")
+
+    def decode(self, layer: int, q: torch.Tensor, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+        assert q.dtype == torch.float32 and q.is_contiguous()
+        if out is None:
+            out = torch.empty_like(q)
+        check(iskv_decode_attn(self.handle, layer, q, out, stream), "iskv_decode_attn")
+        return out
+
+    def reconstruct(self, layer: int, which: int, apply_rope: bool = False,
+                    stream=None) -> torch.Tensor:
+        t = self.tokens(layer)
+        out = torch.empty((self.cfg.batch, self.cfg.n_kv_heads, t, self.cfg.head_dim),
+                          dtype=torch.float32, device="cuda")
+        check(iskv_reconstruct(self.handle, layer, which, int(apply_rope), out, stream),
+              "iskv_reconstruct")
+        return out
+
+    def factors(self, layer: int, seq: int, kv_head: int, which: int, stream=None):
+        """``(coords [n_c][r], basis [d][r], sigma [r], k, n_c)`` copies of one unit."""
+        r = self.cfg.rank_k if which == 0 else self.cfg.rank_v
+        code, k, n_c = iskv_get_factors(self.handle, layer, seq, kv_head, which)
+        check(code, "iskv_get_factors")
+        coords = torch.empty((max(n_c, 1), r), dtype=torch.float32, device="cuda")
+        basis = torch.empty((self.cfg.head_dim, r), dtype=torch.float32, device="cuda")
+        sigma = torch.empty((r,), dtype=torch.float32, device="cuda")
+        code, k, n_c = iskv_get_factors(self.handle, layer, seq, kv_head, which, coords, basis,
+                                        sigma, stream)
+        check(code, "iskv_get_factors")
+        return coords[:n_c], basis, sigma, k, n_c
+
+    def tokens(self, layer: int) -> int:
+        code, t = iskv_num_tokens(self.handle, layer)
+        check(code, "iskv_num_tokens")
+        return t
+
+    def storage_bytes(self, layer: int) -> int:
+        code, b = iskv_storage_bytes(self.handle, layer)
+        check(code, "iskv_storage_bytes")
+        return b
+
+    def reset(self, stream=None) -> None:
+        check(iskv_reset(self.handle, stream), "iskv_reset")
+
+    def launches(self) -> int:
+        code, n = iskv_launch_count(self.handle)
+        check(code, "iskv_launch_count")
+        return n
+
+    def status(self, stream=None) -> int:
+        return iskv_sync_status(self.handle, stream)

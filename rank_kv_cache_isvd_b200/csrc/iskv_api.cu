@@ -1,0 +1,439 @@
+// Host side of the C ABI declared in include/iskv.h: configuration checks, device allocation,
+// per-layer counters (tokens t, compressed rows n_c, current ranks, basis buffer), the fold
+// schedule and launch sequencing. No device work happens outside the kernels in this directory.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "iskv_internal.cuh"
+
+using namespace iskv;
+
+struct iskv_handle {
+    iskv_config cfg;
+    int device = 0;
+    int sms = 148;
+    int U = 0;            // units per path: n_layers * batch * n_kv_heads
+    int UL = 0;           // units per layer
+    int R = 0;            // ring rows per unit
+    int G = 1;
+    long long n_max = 0;  // coordinate rows per unit
+    int max_splits = 0;
+    size_t esz = 2;
+    float *coords[2] = {nullptr, nullptr};
+    float *basis[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+    float *sigma[2] = {nullptr, nullptr};
+    void *ring[2] = {nullptr, nullptr};
+    float *htop[2] = {nullptr, nullptr};
+    float2 *rope_cs = nullptr;
+    float *ws = nullptr;
+    int *status = nullptr;
+    std::vector<long long> t, nc;
+    std::vector<int> kcur[2];
+    std::vector<int> cur;  // which basis buffer is current, per layer
+    long long launches = 0;
+};
+
+namespace {
+
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int now = -1;
+        if (prev >= 0 && cudaGetDevice(&now) == cudaSuccess && now != prev) cudaSetDevice(prev);
+    }
+};
+
+int rank_of(const iskv_handle *h, int which) { return which ? h->cfg.rank_v : h->cfg.rank_k; }
+
+long long ncomp(long long t, int block, int window) {
+    const long long x = t - window;
+    return x > 0 ? (long long)block * (x / block) : 0;
+}
+
+void free_all(iskv_handle *h) {
+    for (int x = 0; x < 2; ++x) {
+        cudaFree(h->coords[x]);
+        cudaFree(h->basis[x][0]);
+        cudaFree(h->basis[x][1]);
+        cudaFree(h->sigma[x]);
+        cudaFree(h->ring[x]);
+        cudaFree(h->htop[x]);
+    }
+    cudaFree(h->rope_cs);
+    cudaFree(h->ws);
+    cudaFree(h->status);
+}
+
+bool valid_layer(const iskv_handle *h, int layer) {
+    return layer >= 0 && layer < h->cfg.n_layers;
+}
+
+int fold_layers(iskv_handle *h, int l0, int nl, cudaStream_t s) {
+    const iskv_config &c = h->cfg;
+    const long long nc = h->nc[l0];
+    FoldArgs fa;
+    RotArgs ra;
+    memset(&fa, 0, sizeof(fa));
+    memset(&ra, 0, sizeof(ra));
+    const int cur = h->cur[l0];
+    for (int x = 0; x < 2; ++x) {
+        const int r = rank_of(h, x);
+        const int k = h->kcur[x][l0];
+        const int p = c.block < D - k ? c.block : D - k;
+        const int kp = r < k + p ? r : k + p;
+        FoldPath &fp = fa.path[x];
+        fp.ring = h->ring[x];
+        fp.basis_in = h->basis[x][cur];
+        fp.basis_out = h->basis[x][cur ^ 1];
+        fp.sigma = h->sigma[x];
+        fp.coords = h->coords[x];
+        fp.htop = h->htop[x];
+        fp.r = r;
+        fp.k = k;
+        fp.p = p;
+        fp.kp = kp;
+        RotPath &rp = ra.path[x];
+        rp.coords = h->coords[x];
+        rp.htop = h->htop[x];
+        rp.r = r;
+        rp.k = k;
+        rp.kp = kp;
+    }
+    fa.unit0 = l0 * h->UL;
+    fa.n_c = nc;
+    fa.n_max = h->n_max;
+    fa.slot0 = (int)(nc % h->R);
+    fa.R = h->R;
+    fa.b = c.block;
+    fa.kv_dtype = c.kv_dtype;
+    fa.status = h->status;
+    if (launch_fold(fa, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+    h->launches += 1 + (nc > 0 ? 1 : 0);
+    ra.unit0 = l0 * h->UL;
+    ra.n_old = nc;
+    ra.n_max = h->n_max;
+    ra.stale = c.rotate_history ? 0 : 1;
+    if (launch_rotate(ra, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+    for (int l = l0; l < l0 + nl; ++l) {
+        h->nc[l] += c.block;
+        h->cur[l] ^= 1;
+        for (int x = 0; x < 2; ++x) h->kcur[x][l] = fa.path[x].kp;
+    }
+    return ISKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *iskv_strerror(int code) {
+    switch (code) {
+        case ISKV_OK: return "ok";
+        case ISKV_ERR_INVALID_ARG: return "invalid argument";
+        case ISKV_ERR_CAPACITY: return "capacity exceeded (t + m > max_tokens)";
+        case ISKV_ERR_CUDA: return "CUDA runtime error";
+        case ISKV_ERR_NOT_CONVERGED: return "core SVD did not converge within the sweep cap";
+        case ISKV_ERR_NONFINITE: return "non-finite singular value";
+        case ISKV_ERR_UNSUPPORTED: return "unsupported configuration";
+        default: return "unknown error";
+    }
+}
+
+int iskv_schedule(int block, int window, long long t, long long m, long long *n_c_out,
+                  long long *folds_out) {
+    if (block < 1 || window < 0 || t < 0 || m < 0) return ISKV_ERR_INVALID_ARG;
+    const long long a = ncomp(t, block, window), b = ncomp(t + m, block, window);
+    if (n_c_out) *n_c_out = b;
+    if (folds_out) *folds_out = (b - a) / block;
+    return ISKV_OK;
+}
+
+int iskv_create(const iskv_config *cfg, iskv_handle **out) {
+    if (!cfg || !out) return ISKV_ERR_INVALID_ARG;
+    *out = nullptr;
+    const iskv_config &c = *cfg;
+    if (c.batch < 1 || c.n_layers < 1 || c.n_kv_heads < 1 || c.n_q_heads < c.n_kv_heads ||
+        c.n_q_heads % c.n_kv_heads != 0 || c.n_q_heads / c.n_kv_heads > GMAX || c.head_dim != D ||
+        c.rank_k < 1 || c.rank_k > D || c.rank_v < 1 || c.rank_v > D || c.block < 1 ||
+        c.window < 0 || c.max_tokens < 1 || (c.kv_dtype != ISKV_BF16 && c.kv_dtype != ISKV_F32) ||
+        (c.rope && !(c.rope_theta > 0.0)))
+        return ISKV_ERR_INVALID_ARG;
+    if (c.block > BMAX) return ISKV_ERR_UNSUPPORTED;
+    iskv_handle *h = new (std::nothrow) iskv_handle();
+    if (!h) return ISKV_ERR_CUDA;
+    try {
+        h->cfg = c;
+        if (cudaGetDevice(&h->device) != cudaSuccess) {
+            delete h;
+            return ISKV_ERR_CUDA;
+        }
+        cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
+        h->UL = c.batch * c.n_kv_heads;
+        h->U = c.n_layers * h->UL;
+        h->R = c.window + c.block;
+        h->G = c.n_q_heads / c.n_kv_heads;
+        h->n_max = ncomp(c.max_tokens, c.block, c.window);
+        h->esz = c.kv_dtype == ISKV_BF16 ? 2 : 4;
+        const long long ctiles = (h->n_max + DEC_TILE - 1) / DEC_TILE;
+        h->max_splits = (int)(ctiles + (h->R + DEC_TILE - 1) / DEC_TILE + 1);
+        h->t.assign(c.n_layers, 0);
+        h->nc.assign(c.n_layers, 0);
+        h->cur.assign(c.n_layers, 0);
+        h->kcur[0].assign(c.n_layers, 0);
+        h->kcur[1].assign(c.n_layers, 0);
+    } catch (...) {
+        delete h;
+        return ISKV_ERR_CUDA;
+    }
+    bool ok = true;
+    auto alloc = [&](void **p, size_t bytes) {
+        if (!ok) return;
+        if (bytes == 0) bytes = 16;
+        if (cudaMalloc(p, bytes) != cudaSuccess) {
+            ok = false;
+            *p = nullptr;
+        }
+    };
+    const size_t U = (size_t)h->U;
+    for (int x = 0; x < 2; ++x) {
+        const size_t r = (size_t)rank_of(h, x);
+        alloc((void **)&h->coords[x], U * (size_t)h->n_max * r * sizeof(float));
+        alloc((void **)&h->basis[x][0], U * D * r * sizeof(float));
+        alloc((void **)&h->basis[x][1], U * D * r * sizeof(float));
+        alloc((void **)&h->sigma[x], U * r * sizeof(float));
+        alloc(&h->ring[x], U * (size_t)h->R * D * h->esz);
+        alloc((void **)&h->htop[x], U * r * r * sizeof(float));
+    }
+    if (c.rope) alloc((void **)&h->rope_cs, (size_t)c.max_tokens * DH * sizeof(float2));
+    alloc((void **)&h->ws, (size_t)h->UL * h->max_splits * h->G * (2 + D) * sizeof(float));
+    alloc((void **)&h->status, sizeof(int));
+    if (ok) {
+        for (int x = 0; x < 2; ++x) {
+            const size_t r = (size_t)rank_of(h, x);
+            ok = ok && cudaMemset(h->basis[x][0], 0, U * D * r * sizeof(float)) == cudaSuccess;
+            ok = ok && cudaMemset(h->basis[x][1], 0, U * D * r * sizeof(float)) == cudaSuccess;
+            ok = ok && cudaMemset(h->sigma[x], 0, U * r * sizeof(float)) == cudaSuccess;
+        }
+        ok = ok && cudaMemset(h->status, 0, sizeof(int)) == cudaSuccess;
+        if (ok && c.rope)
+            ok = launch_rope_table(h->rope_cs, c.max_tokens, c.rope_theta, 0) == cudaSuccess;
+        ok = ok && cudaDeviceSynchronize() == cudaSuccess;
+    }
+    if (!ok) {
+        free_all(h);
+        delete h;
+        cudaGetLastError();
+        return ISKV_ERR_CUDA;
+    }
+    *out = h;
+    return ISKV_OK;
+}
+
+int iskv_destroy(iskv_handle *h) {
+    if (!h) return ISKV_OK;
+    DeviceGuard g(h->device);
+    cudaDeviceSynchronize();
+    free_all(h);
+    delete h;
+    return ISKV_OK;
+}
+
+int iskv_append_block(iskv_handle *h, int layer, const void *k_rows, const void *v_rows, int m,
+                      iskv_stream_t stream) {
+    if (!h || !k_rows || !v_rows || m < 1) return ISKV_ERR_INVALID_ARG;
+    const iskv_config &c = h->cfg;
+    if (layer != -1 && !valid_layer(h, layer)) return ISKV_ERR_INVALID_ARG;
+    const int l0 = layer < 0 ? 0 : layer;
+    const int nl = layer < 0 ? c.n_layers : 1;
+    for (int l = l0; l < l0 + nl; ++l)
+        if (h->t[l] != h->t[l0] || h->nc[l] != h->nc[l0] || h->cur[l] != h->cur[l0])
+            return ISKV_ERR_INVALID_ARG;
+    if (h->t[l0] + m > c.max_tokens) return ISKV_ERR_CAPACITY;
+    DeviceGuard g(h->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    long long t = h->t[l0];
+    int done = 0;
+    while (done < m) {
+        const long long e = t - h->nc[l0];
+        const long long room = (long long)h->R - e;   // rows until the window holds w + b
+        const int chunk = (int)((long long)(m - done) < room ? (m - done) : room);
+        AppendArgs aa;
+        aa.src[0] = k_rows;
+        aa.src[1] = v_rows;
+        aa.ring[0] = h->ring[0];
+        aa.ring[1] = h->ring[1];
+        aa.unit0 = l0 * h->UL;
+        aa.m_total = m;
+        aa.row0 = done;
+        aa.rows = chunk;
+        aa.pos0 = t;
+        aa.R = h->R;
+        aa.kv_dtype = c.kv_dtype;
+        if (launch_append(aa, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+        h->launches += 1;
+        t += chunk;
+        done += chunk;
+        for (int l = l0; l < l0 + nl; ++l) h->t[l] = t;
+        if (t - h->nc[l0] >= (long long)h->R) {
+            const int rc = fold_layers(h, l0, nl, s);
+            if (rc != ISKV_OK) return rc;
+        }
+    }
+    return ISKV_OK;
+}
+
+int iskv_decode_attn(iskv_handle *h, int layer, const float *q, float *out, iskv_stream_t stream) {
+    if (!h || !q || !out || !valid_layer(h, layer)) return ISKV_ERR_INVALID_ARG;
+    if (h->t[layer] < 1) return ISKV_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    const iskv_config &c = h->cfg;
+    DecodeArgs da;
+    memset(&da, 0, sizeof(da));
+    const int cur = h->cur[layer];
+    for (int x = 0; x < 2; ++x) {
+        const size_t r = (size_t)rank_of(h, x);
+        const size_t u0 = (size_t)layer * h->UL;
+        da.coords[x] = h->coords[x] + u0 * (size_t)h->n_max * r;
+        da.basis[x] = h->basis[x][cur] + u0 * D * r;
+        da.ring[x] = static_cast<const char *>(h->ring[x]) + u0 * (size_t)h->R * D * h->esz;
+        da.r[x] = (int)r;
+        da.k[x] = h->kcur[x][layer];
+    }
+    da.rope_cs = c.rope ? h->rope_cs : nullptr;
+    da.q = q;
+    da.out = out;
+    da.ws = h->ws;
+    da.n_c = h->nc[layer];
+    da.t = h->t[layer];
+    da.n_max = h->n_max;
+    da.R = h->R;
+    da.H = c.n_kv_heads;
+    da.G = h->G;
+    const long long ctiles = (da.n_c + DEC_TILE - 1) / DEC_TILE;
+    const long long target = 2LL * h->sms;
+    long long tps = (ctiles * h->UL + target - 1) / target;
+    if (tps < 1) tps = 1;
+    da.split_rows = (int)(tps * DEC_TILE);
+    da.n_split_c = (int)((ctiles + tps - 1) / tps);
+    const long long e = da.t - da.n_c;
+    da.n_split = da.n_split_c + (int)((e + DEC_TILE - 1) / DEC_TILE);
+    da.max_splits = h->max_splits;
+    da.kv_dtype = c.kv_dtype;
+    da.scale = 1.0f / sqrtf((float)D);
+    if (da.n_split > h->max_splits) return ISKV_ERR_INVALID_ARG;
+    if (launch_decode(da, h->UL, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ISKV_ERR_CUDA;
+    h->launches += 2;
+    return ISKV_OK;
+}
+
+int iskv_reconstruct(iskv_handle *h, int layer, int which, int apply_rope, float *out,
+                     iskv_stream_t stream) {
+    if (!h || !out || !valid_layer(h, layer) || (which != 0 && which != 1))
+        return ISKV_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    const size_t r = (size_t)rank_of(h, which);
+    const size_t u0 = (size_t)layer * h->UL;
+    ReconArgs ra;
+    ra.coords = h->coords[which] + u0 * (size_t)h->n_max * r;
+    ra.basis = h->basis[which][h->cur[layer]] + u0 * D * r;
+    ra.ring = static_cast<const char *>(h->ring[which]) + u0 * (size_t)h->R * D * h->esz;
+    ra.rope_cs = h->rope_cs;
+    ra.out = out;
+    ra.r = (int)r;
+    ra.k = h->kcur[which][layer];
+    ra.n_c = h->nc[layer];
+    ra.t = h->t[layer];
+    ra.n_max = h->n_max;
+    ra.R = h->R;
+    ra.kv_dtype = h->cfg.kv_dtype;
+    ra.apply_rope = (which == 0 && apply_rope && h->cfg.rope) ? 1 : 0;
+    if (launch_reconstruct(ra, h->UL, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ISKV_ERR_CUDA;
+    h->launches += ra.t > 0 ? 1 : 0;
+    return ISKV_OK;
+}
+
+int iskv_get_factors(iskv_handle *h, int layer, int seq, int kv_head, int which, float *coords,
+                     float *basis, float *sigma, int *k_out, long long *n_c_out,
+                     iskv_stream_t stream) {
+    if (!h || !valid_layer(h, layer) || seq < 0 || seq >= h->cfg.batch || kv_head < 0 ||
+        kv_head >= h->cfg.n_kv_heads || (which != 0 && which != 1))
+        return ISKV_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t r = (size_t)rank_of(h, which);
+    const size_t u = ((size_t)layer * h->cfg.batch + seq) * h->cfg.n_kv_heads + kv_head;
+    const long long nc = h->nc[layer];
+    if (coords && nc > 0 &&
+        cudaMemcpyAsync(coords, h->coords[which] + u * (size_t)h->n_max * r,
+                        (size_t)nc * r * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return ISKV_ERR_CUDA;
+    if (basis && cudaMemcpyAsync(basis, h->basis[which][h->cur[layer]] + u * D * r,
+                                 D * r * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return ISKV_ERR_CUDA;
+    if (sigma && cudaMemcpyAsync(sigma, h->sigma[which] + u * r, r * sizeof(float),
+                                 cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return ISKV_ERR_CUDA;
+    if (k_out) *k_out = h->kcur[which][layer];
+    if (n_c_out) *n_c_out = nc;
+    return ISKV_OK;
+}
+
+int iskv_reset(iskv_handle *h, iskv_stream_t stream) {
+    if (!h) return ISKV_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    for (int l = 0; l < h->cfg.n_layers; ++l) {
+        h->t[l] = 0;
+        h->nc[l] = 0;
+        h->cur[l] = 0;
+        h->kcur[0][l] = 0;
+        h->kcur[1][l] = 0;
+    }
+    if (cudaMemsetAsync(h->status, 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return ISKV_ERR_CUDA;
+    return ISKV_OK;
+}
+
+int iskv_launch_count(const iskv_handle *h, long long *count_out) {
+    if (!h || !count_out) return ISKV_ERR_INVALID_ARG;
+    *count_out = h->launches;
+    return ISKV_OK;
+}
+
+int iskv_num_tokens(const iskv_handle *h, int layer, long long *t_out) {
+    if (!h || !t_out || !valid_layer(h, layer)) return ISKV_ERR_INVALID_ARG;
+    *t_out = h->t[layer];
+    return ISKV_OK;
+}
+
+int iskv_storage_bytes(const iskv_handle *h, int layer, long long *bytes_out) {
+    if (!h || !bytes_out || !valid_layer(h, layer)) return ISKV_ERR_INVALID_ARG;
+    const long long n = h->nc[layer], e = h->t[layer] - n;
+    long long f = 0;
+    for (int x = 0; x < 2; ++x) f += (long long)h->kcur[x][layer] * (n + D + 1);
+    *bytes_out = (long long)h->UL * (4LL * f + (long long)h->esz * D * 2LL * e);
+    return ISKV_OK;
+}
+
+int iskv_sync_status(iskv_handle *h, iskv_stream_t stream) {
+    if (!h) return ISKV_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    int st = 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&st, h->status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return ISKV_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ISKV_ERR_CUDA;
+    return st;
+}
+
+}  // extern "C"

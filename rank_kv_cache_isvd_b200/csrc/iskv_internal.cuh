@@ -1,0 +1,121 @@
+// Internal declarations of the iS-KV CUDA path (kernels + launchers). Not part of the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "iskv.h"
+
+namespace iskv {
+
+constexpr int D = 128;        // head_dim (fixed by the build)
+constexpr int DH = D / 2;     // RoPE pairs (j, j + 64)
+constexpr int BMAX = 128;     // largest block folded by the in-shared-memory fold kernel
+constexpr int LDS = D + 1;    // padded stride of 128-float rows/columns in shared memory
+constexpr int GMAX = 8;       // largest GQA group (q-heads per kv-head)
+constexpr int DEC_TILE = 128; // decode rows per tile
+constexpr int JACOBI_MAX_SWEEPS = 30;
+
+// ---- fold: projection/residual/QR + core SVD + basis update (one CTA per unit and path) ------
+struct FoldPath {
+    const void *ring;       // [units][R][D] kv dtype
+    const float *basis_in;  // [units][D][r]
+    float *basis_out;       // [units][D][r]
+    float *sigma;           // [units][r]
+    float *coords;          // [units][n_max][r]
+    float *htop;            // [units][r][r]
+    int r, k, p, kp;        // rank budget, rank before, residual basis size, rank after
+};
+
+struct FoldArgs {
+    FoldPath path[2];
+    int unit0;              // first unit of the folded set
+    long long n_c;          // rows compressed before this fold
+    long long n_max;        // coordinate rows per unit
+    int slot0;              // ring slot of the oldest exact row (n_c mod R)
+    int R;                  // ring capacity (window + block)
+    int b;                  // block
+    int kv_dtype;
+    int *status;
+};
+
+// ---- history rotation C[0:n] <- C[0:n] H_top (or stale zero-padding) ---------------------------
+struct RotPath {
+    float *coords;          // [units][n_max][r]
+    const float *htop;      // [units][r][r]
+    int r, k, kp;
+};
+struct RotArgs {
+    RotPath path[2];
+    int unit0;
+    long long n_old;        // rows to rotate
+    long long n_max;
+    int stale;              // 1: keep old coordinates (zero columns k..kp-1)
+};
+
+// ---- window append ----------------------------------------------------------------------------
+struct AppendArgs {
+    const void *src[2];     // [units][m_total][D] rows of K and V
+    void *ring[2];          // [units][R][D]
+    int unit0;
+    int m_total;            // rows per unit in the caller's array
+    int row0;               // first row of this chunk in the caller's array
+    int rows;               // rows in this chunk
+    long long pos0;         // token position of the chunk's first row
+    int R;
+    int kv_dtype;
+};
+
+// ---- decode -------------------------------------------------------------------------------------
+struct DecodeArgs {
+    const float *coords[2]; // [units][n_max][r] (units offset to the layer)
+    const float *basis[2];  // [units][D][r]
+    const void *ring[2];    // [units][R][D]
+    const float2 *rope_cs;  // [max_tokens][DH] (cos, sin) or nullptr
+    const float *q;         // [S][QH][D]
+    float *out;             // [S][QH][D]
+    float *ws;              // [units_in_layer][max_splits][G][2 + D]
+    int r[2], k[2];
+    long long n_c, t, n_max;
+    int R;
+    int H, G;               // kv heads, group size
+    int split_rows;         // compressed rows per split (multiple of DEC_TILE)
+    int n_split_c;          // compressed splits
+    int n_split;            // total splits (compressed + window)
+    int max_splits;
+    int kv_dtype;
+    float scale;
+};
+
+// ---- reconstruct ------------------------------------------------------------------------------
+struct ReconArgs {
+    const float *coords;
+    const float *basis;
+    const void *ring;
+    const float2 *rope_cs;
+    float *out;             // [units][t][D]
+    int r, k;
+    long long n_c, t, n_max;
+    int R, kv_dtype, apply_rope;
+};
+
+cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s);
+cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s);
+cudaError_t launch_append(const AppendArgs &a, int n_units, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs &a, int n_units, cudaStream_t s);
+cudaError_t launch_reconstruct(const ReconArgs &a, int n_units, cudaStream_t s);
+cudaError_t launch_rope_table(float2 *table, long long max_tokens, double theta, cudaStream_t s);
+size_t fold_smem_bytes();
+
+__device__ __forceinline__ float load_row_elem(const void *base, size_t idx, int kv_dtype) {
+    if (kv_dtype == ISKV_BF16)
+        return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[idx]);
+    return reinterpret_cast<const float *>(base)[idx];
+}
+
+__device__ __forceinline__ void set_status(int *status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+}  // namespace iskv

@@ -1,0 +1,105 @@
+// Exact recent window (ring buffer of window + block rows per unit and path), cache
+// reconstruction, and the RoPE angle table.
+//
+// iS-KV summary, "Architecture Overview": the most recent tokens stay exact; "Reconstruction and
+// Storage": compressed row i is (U Sigma B^T)[i] = (C B^T)[i], other rows are the exact rows.
+#include "iskv_internal.cuh"
+
+namespace iskv {
+
+// One CTA per (row of the chunk, unit); blockIdx.z = path. Copies 128 elements (16-byte vectors).
+__global__ void append_kernel(AppendArgs a) {
+    const int path = blockIdx.z;
+    const int i = blockIdx.x;            // row within the chunk
+    const int unit = a.unit0 + blockIdx.y;
+    const long long pos = a.pos0 + i;
+    const int slot = (int)(pos % a.R);
+    const size_t esz = a.kv_dtype == ISKV_BF16 ? 2 : 4;
+    const char *src = static_cast<const char *>(a.src[path]) +
+                      ((size_t)blockIdx.y * a.m_total + a.row0 + i) * D * esz;
+    char *dst = static_cast<char *>(a.ring[path]) + ((size_t)unit * a.R + slot) * D * esz;
+    const int nvec = (int)(D * esz / 16);
+    if (threadIdx.x < nvec)
+        reinterpret_cast<uint4 *>(dst)[threadIdx.x] = reinterpret_cast<const uint4 *>(src)[threadIdx.x];
+}
+
+cudaError_t launch_append(const AppendArgs &a, int n_units, cudaStream_t s) {
+    if (a.rows <= 0) return cudaSuccess;
+    append_kernel<<<dim3(a.rows, n_units, 2), 32, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+// (cos, sin) of pos * theta^(-2j/d) for every position and pair j, computed in double and
+// rounded once to float (the angle of a far position is too large for a float product).
+__global__ void rope_table_kernel(float2 *table, long long max_tokens, double theta) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= max_tokens * DH) return;
+    const long long pos = idx / DH;
+    const int j = (int)(idx % DH);
+    const double omega = pow(theta, -2.0 * j / (double)D);
+    double sn, cs;
+    sincos((double)pos * omega, &sn, &cs);
+    table[idx] = make_float2((float)cs, (float)sn);
+}
+
+cudaError_t launch_rope_table(float2 *table, long long max_tokens, double theta, cudaStream_t s) {
+    const long long n = max_tokens * DH;
+    const unsigned grid = (unsigned)((n + 255) / 256);
+    rope_table_kernel<<<grid, 256, 0, s>>>(table, max_tokens, theta);
+    return cudaGetLastError();
+}
+
+// One CTA per (tile of 64 positions, unit); 128 threads (one per channel).
+__global__ void reconstruct_kernel(ReconArgs a) {
+    extern __shared__ float sB[];        // basis row j, column c at [j * ks + c]
+    const int unit = blockIdx.y;
+    const int j = threadIdx.x;
+    const int k = a.k, r = a.r, ks = k | 1;
+    const float *B = a.basis + (size_t)unit * D * r;
+    for (int o = threadIdx.x; o < D * k; o += blockDim.x) sB[(o / k) * ks + o % k] = B[(size_t)(o / k) * r + o % k];
+    __syncthreads();
+    const long long p0 = (long long)blockIdx.x * 64;
+    for (int i = 0; i < 64; ++i) {
+        const long long pos = p0 + i;
+        if (pos >= a.t) break;
+        float x;
+        if (pos < a.n_c) {
+            const float *c = a.coords + ((size_t)unit * a.n_max + pos) * r;
+            float s = 0.f;
+            for (int l = 0; l < k; ++l) s = fmaf(c[l], sB[j * ks + l], s);
+            x = s;
+        } else {
+            const int slot = (int)(pos % a.R);
+            x = load_row_elem(a.ring, ((size_t)unit * a.R + slot) * D + j, a.kv_dtype);
+        }
+        float *o = a.out + ((size_t)unit * a.t + pos) * D;
+        if (a.apply_rope) {
+            // pair (j, j + 64) lives in two threads: exchange through shared memory
+            __shared__ float sx[D];
+            sx[j] = x;
+            __syncthreads();
+            const float2 cs = a.rope_cs[pos * DH + (j & (DH - 1))];
+            x = (j < DH) ? x * cs.x - sx[j + DH] * cs.y : x * cs.x + sx[j - DH] * cs.y;
+            __syncthreads();
+        }
+        o[j] = x;
+    }
+}
+
+cudaError_t launch_reconstruct(const ReconArgs &a, int n_units, cudaStream_t s) {
+    if (a.t <= 0) return cudaSuccess;
+    const size_t smem = (size_t)D * ((a.k | 1)) * sizeof(float);
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)(D * 129 * sizeof(float)));
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const unsigned gx = (unsigned)((a.t + 63) / 64);
+    reconstruct_kernel<<<dim3(gx, n_units), D, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace iskv

@@ -1,0 +1,274 @@
+"""GPU parity of the CUDA path (through the C ABI) against the float64 oracle on the same seeded
+inputs.
+
+Tolerances: singular values relative error <= 1e-4; subspace projector error
+||B B^T - B0 B0^T||_F <= 1e-3 where the relative spectral gap at the kept rank exceeds 1e-2;
+attention output relative error <= 2e-3 per q-head (max over heads); window rows, token counts,
+compressed-row counts and ranks bit-exact.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import iskv_synth as syn  # noqa: E402
+from gpu_harness import (max_head_rel_err, projector_err, rel_err, to_device,  # noqa: E402
+                         workload_arrays)
+from oracle import OracleCache, fold_from_coords, n_compressed  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+SIG_TOL, PROJ_TOL, ATTN_TOL, GAP = 1e-4, 1e-3, 2e-3, 1e-2
+W0, W1 = syn.WORKLOADS[0], syn.WORKLOADS[1]
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def make_cache(wl, **kw):
+    from rank_kv_cache_isvd_b200.cache import IsKVCache
+    args = dict(batch=wl.batch, n_layers=wl.n_layers, n_kv_heads=wl.n_kv_heads,
+                n_q_heads=wl.n_q_heads, rank_k=wl.rank_k, rank_v=wl.rank_v, block=wl.block,
+                window=wl.window, max_tokens=wl.tokens, kv_dtype=wl.kv_dtype, rope=wl.rope,
+                rope_theta=wl.rope_theta)
+    args.update(kw)
+    return IsKVCache(**args)
+
+
+def make_oracle(wl, rotate=True):
+    return OracleCache(wl.batch, wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim,
+                       wl.rank_k, wl.rank_v, wl.block, wl.window, rope=wl.rope,
+                       rope_theta=wl.rope_theta, rotate=rotate)
+
+
+def sub(wl, **kw):
+    return dataclasses.replace(wl, **kw)
+
+
+def append_both(cache, orc, layer, kd, kv, vd, vv, t0, t1):
+    K = to_device(kd[:, :, t0:t1])
+    V = to_device(vd[:, :, t0:t1])
+    cache.append(layer, K, V)
+    orc.append(layer, kv[:, :, t0:t1], vv[:, :, t0:t1])
+
+
+# ------------------------------------------------------------------------------------------------
+def test_window_rows_bit_exact_and_decode_before_any_fold():
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=300)
+    kd, kv, vd, vv = workload_arrays(wl)
+    cache, orc = make_cache(wl), make_oracle(wl)
+    append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], 0, 200)
+    assert cache.tokens(0) == 200
+    rk = cache.reconstruct(0, 0).cpu().numpy()
+    rv = cache.reconstruct(0, 1).cpu().numpy()
+    assert np.array_equal(rk, kv[0][:, :, :200].astype(np.float32))
+    assert np.array_equal(rv, vv[0][:, :, :200].astype(np.float32))
+    q = syn.queries(7, (1, 8, 128))
+    out = cache.decode(0, torch.from_numpy(q).cuda()).cpu().numpy()
+    assert max_head_rel_err(out, orc.decode(0, q.astype(np.float64))) <= ATTN_TOL
+    assert cache.status() == 0
+
+
+# ------------------------------------------------------------------------------------------------
+def _snapshot(cache, wl):
+    snap = {}
+    for s in range(wl.batch):
+        for h in range(wl.n_kv_heads):
+            for x in (0, 1):
+                C, B, S, k, n = cache.factors(0, s, h, x)
+                snap[s, h, x] = (C.cpu().numpy().astype(np.float64), B.cpu().numpy().astype(np.float64),
+                                 S.cpu().numpy().astype(np.float64), k, n)
+    return snap
+
+
+@pytest.mark.parametrize("variant", ["gapped", "literal"])
+def test_fold_one_step_parity(variant):
+    """Each GPU fold, started from the GPU's own state, matches the oracle's fold."""
+    wl = sub(W1, n_kv_heads=3, n_q_heads=12, tokens=1100)
+    kd, kv, vd, vv = workload_arrays(wl, variant=variant)
+    cache = make_cache(wl)
+    t, folds, worst = 0, 0, {"sigma": 0.0, "proj": 0.0, "recon": 0.0}
+    while True:
+        nc = n_compressed(t, wl.block, wl.window)
+        t_fold = nc + wl.window + wl.block           # the append that reaches it folds
+        if t_fold > wl.tokens:
+            break
+        before = _snapshot(cache, wl)
+        cache.append(0, to_device(kd[0][:, :, t:t_fold]), to_device(vd[0][:, :, t:t_fold]))
+        t = t_fold
+        after = _snapshot(cache, wl)
+        folds += 1
+        for (s, h, x), (C0, B0, S0, k0, n0) in before.items():
+            r = wl.rank_k if x == 0 else wl.rank_v
+            F = (kv if x == 0 else vv)[0][s, h, n0:n0 + wl.block]
+            Cr, Sr, Br, _ = fold_from_coords(C0[:, :k0], S0[:k0], B0[:, :k0], F, r)
+            C1, B1, S1, k1, n1 = after[s, h, x]
+            assert n1 == n0 + wl.block and k1 == Sr.size
+            sig = np.abs(S1[:k1] - Sr) / Sr
+            worst["sigma"] = max(worst["sigma"], float(sig.max()))
+            M = np.vstack([C0[:, :k0] @ B0[:, :k0].T, F]) if n0 else F
+            sv = np.linalg.svd(M, compute_uv=False)
+            gapped = k1 < sv.size and (sv[k1 - 1] - sv[k1]) / sv[0] > GAP
+            rec = rel_err(C1[:, :k1] @ B1[:, :k1].T, Cr @ Br.T)
+            if gapped:
+                worst["proj"] = max(worst["proj"], projector_err(B1[:, :k1], Br))
+                worst["recon"] = max(worst["recon"], rec)
+            assert np.abs(B1[:, :k1].T @ B1[:, :k1] - np.eye(k1)).max() <= 5e-5
+    print(f"\n{variant}: {folds} folds, worst {worst}")
+    assert folds == n_compressed(wl.tokens, wl.block, wl.window) // wl.block
+    assert worst["sigma"] <= SIG_TOL
+    assert worst["proj"] <= PROJ_TOL
+    assert worst["recon"] <= SIG_TOL
+    assert cache.status() == 0
+
+
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("key_scale", [1.0, 8.0])
+def test_decode_parity_llama_layer_full(key_scale):
+    """Llama-3-8B-shaped layer (8 kv / 32 q heads, 4096 tokens, b=64, w=256, rK=32, rV=48)."""
+    wl = W1
+    kd, kv, vd, vv = workload_arrays(wl, key_scale=key_scale)
+    cache, orc = make_cache(wl), make_oracle(wl)
+    checkpoints = [1, 255, 256, 319, 320, 321, 700, 2048, 4095, 4096]
+    t, worst = 0, 0.0
+    for i, tc in enumerate(checkpoints):
+        append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], t, tc)
+        t = tc
+        assert cache.tokens(0) == t
+        q = syn.queries(100 + i, (1, wl.n_q_heads, 128))
+        out = cache.decode(0, torch.from_numpy(q).cuda()).cpu().numpy()
+        err = max_head_rel_err(out, orc.decode(0, q.astype(np.float64)))
+        worst = max(worst, err)
+    print(f"\nkey_scale={key_scale}: worst attention rel err {worst:.3e}")
+    assert worst <= ATTN_TOL
+    for x in (0, 1):
+        _, B, S, k, n = cache.factors(0, 0, 0, x)
+        assert n == 3840 and k == (32 if x == 0 else 48)
+    assert cache.status() == 0
+
+
+def test_single_head_f32_no_rope_full():
+    """Single head, d=128, fp32 rows, n=1024 compressed + 64 window, b=32, r=32, one query."""
+    wl = W0
+    kd, kv, vd, vv = workload_arrays(wl)
+    cache, orc = make_cache(wl), make_oracle(wl)
+    append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], 0, wl.tokens)
+    q = syn.queries(5, (1, 1, 128))
+    out = cache.decode(0, torch.from_numpy(q).cuda()).cpu().numpy()
+    assert max_head_rel_err(out, orc.decode(0, q.astype(np.float64))) <= ATTN_TOL
+    _, _, S, k, n = cache.factors(0, 0, 0, 0)
+    assert n == 1024 and k == 32
+    assert cache.status() == 0
+
+
+def test_gapped_end_to_end_sigma_and_projector():
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=2000)
+    kd, kv, vd, vv = workload_arrays(wl, variant="gapped")
+    cache, orc = make_cache(wl), make_oracle(wl)
+    append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], 0, wl.tokens)
+    for h in range(2):
+        for x in (0, 1):
+            C, B, S, k, n = cache.factors(0, 0, h, x)
+            u = orc.unit(0, 0, h, x)
+            S, B = S.cpu().numpy(), B.cpu().numpy()
+            assert k == u.k and n == u.n
+            assert np.max(np.abs(S[:k] - u.sigma) / u.sigma) <= SIG_TOL
+            assert projector_err(B[:, :k], u.B) <= PROJ_TOL
+    q = syn.queries(9, (1, 8, 128))
+    out = cache.decode(0, torch.from_numpy(q).cuda()).cpu().numpy()
+    assert max_head_rel_err(out, orc.decode(0, q.astype(np.float64))) <= ATTN_TOL
+
+
+def test_stale_coordinates_mode_matches_oracle():
+    wl = sub(W1, n_kv_heads=1, n_q_heads=4, tokens=900)
+    kd, kv, vd, vv = workload_arrays(wl, variant="gapped")
+    cache, orc = make_cache(wl, rotate_history=False), make_oracle(wl, rotate=False)
+    sync = make_oracle(wl)
+    append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], 0, wl.tokens)
+    sync.append(0, kv[0], vv[0])
+    for x in (0, 1):
+        rec = cache.reconstruct(0, x).cpu().numpy()[0, 0]
+        ref = orc.unit(0, 0, 0, x).reconstruct()
+        n = orc.unit(0, 0, 0, x).n
+        assert rel_err(rec[:n], ref[:n]) <= 1e-3
+        drift = rel_err(ref[:n], sync.unit(0, 0, 0, x).reconstruct()[:n])
+        assert drift > 1e-2          # stale coordinates do drift
+
+
+def test_all_layers_batched_equals_per_layer():
+    wl = sub(W1, n_layers=3, n_kv_heads=2, n_q_heads=8, tokens=700)
+    kd, kv, vd, vv = workload_arrays(wl)
+    a, b = make_cache(wl), make_cache(wl)
+    for t0, t1 in [(0, 1), (1, 333), (333, 700)]:
+        a.append(-1, to_device(kd[:, :, :, t0:t1]), to_device(vd[:, :, :, t0:t1]))
+        for l in range(3):
+            b.append(l, to_device(kd[l, :, :, t0:t1]), to_device(vd[l, :, :, t0:t1]))
+    for l in range(3):
+        for x in (0, 1):
+            assert torch.equal(a.reconstruct(l, x), b.reconstruct(l, x))
+
+
+def test_bulk_append_equals_streaming():
+    wl = sub(W1, n_kv_heads=1, n_q_heads=4, tokens=800)
+    kd, kv, vd, vv = workload_arrays(wl)
+    a, b = make_cache(wl), make_cache(wl)
+    a.append(0, to_device(kd[0]), to_device(vd[0]))
+    for t in range(800):
+        b.append(0, to_device(kd[0][:, :, t:t + 1]), to_device(vd[0][:, :, t:t + 1]))
+    for x in (0, 1):
+        assert torch.equal(a.reconstruct(0, x), b.reconstruct(0, x))
+    q = torch.from_numpy(syn.queries(3, (1, 4, 128))).cuda()
+    assert torch.equal(a.decode(0, q), b.decode(0, q))
+
+
+def test_no_truncation_reconstructs_exactly():
+    """r = d: every fold keeps all directions (after the first fold p = 0)."""
+    wl = sub(W0, rank_k=128, rank_v=128, tokens=500, block=32, window=40)
+    kd, kv, vd, vv = workload_arrays(wl)
+    cache = make_cache(wl)
+    cache.append(0, to_device(kd[0]), to_device(vd[0]))
+    for x, vals in ((0, kv), (1, vv)):
+        rec = cache.reconstruct(0, x).cpu().numpy()[0, 0]
+        assert rel_err(rec, vals[0][0, 0]) <= 1e-5
+        _, B, _, k, _ = cache.factors(0, 0, 0, x)
+        B = B.cpu().numpy()
+        assert k == 128 and np.abs(B.T @ B - np.eye(128)).max() <= 5e-5
+
+
+def test_exact_low_rank_and_zero_rows():
+    """Rank-3 rows with r = 8: exact reconstruction and orthonormal bases even though most
+    singular values are zero; an all-zero block keeps the factors finite."""
+    wl = sub(W0, rank_k=8, rank_v=8, tokens=400, block=16, window=16)
+    X = syn.kv_rows(400, 128, 3, 1.0, variant="lowrank", rank=3).astype(np.float32)
+    X[200:232] = 0.0
+    Xd = X[None, None].copy()
+    cache = make_cache(wl)
+    cache.append(0, to_device(Xd), to_device(Xd))
+    for x in (0, 1):
+        rec = cache.reconstruct(0, x).cpu().numpy()[0, 0]
+        assert rel_err(rec, X) <= 1e-5
+        _, B, S, k, _ = cache.factors(0, 0, 0, x)
+        B = B.cpu().numpy()[:, :k]
+        assert np.all(np.isfinite(S.cpu().numpy()))
+        assert np.abs(B.T @ B - np.eye(k)).max() <= 1e-4
+    assert cache.status() == 0
+
+
+def test_block_of_one_row_and_capacity_error():
+    from rank_kv_cache_isvd_b200 import ISKV_ERR_CAPACITY, IsKVError
+    wl = sub(W1, n_kv_heads=1, n_q_heads=2, tokens=150, block=1, window=5, rank_k=4, rank_v=6)
+    kd, kv, vd, vv = workload_arrays(wl)
+    cache, orc = make_cache(wl), make_oracle(wl)
+    append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], 0, 150)
+    q = syn.queries(11, (1, 2, 128))
+    out = cache.decode(0, torch.from_numpy(q).cuda()).cpu().numpy()
+    assert max_head_rel_err(out, orc.decode(0, q.astype(np.float64))) <= ATTN_TOL
+    with pytest.raises(IsKVError) as e:
+        cache.append(0, to_device(kd[0][:, :, :1]), to_device(vd[0][:, :, :1]))
+    assert e.value.code == ISKV_ERR_CAPACITY
+    assert cache.tokens(0) == 150
