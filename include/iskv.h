@@ -48,7 +48,8 @@ enum {
     ISKV_ERR_CUDA = -3,         /* a CUDA runtime call failed (allocation, launch, copy)     */
     ISKV_ERR_NOT_CONVERGED = -4,/* a core SVD hit its sweep cap (sticky, device side)        */
     ISKV_ERR_NONFINITE = -5,    /* a non-finite singular value appeared (sticky, device side) */
-    ISKV_ERR_UNSUPPORTED = -6   /* valid request outside what this build implements          */
+    ISKV_ERR_UNSUPPORTED = -6,  /* valid request outside what this build implements          */
+    ISKV_ERR_TIMEOUT = -7       /* a device-side wait hit its bound (sticky, device side)    */
 };
 
 enum { ISKV_BF16 = 0, ISKV_F32 = 1 };
@@ -147,6 +148,15 @@ int iskv_reset(iskv_handle *h, iskv_stream_t stream);
  */
 int iskv_launch_count(const iskv_handle *h, long long *count_out);
 
+/*
+ * Statistics of the core SVDs run since creation or the last iskv_reset(): the largest number of
+ * Jacobi sweeps one core needed, the total number of sweeps, and the number of cores solved.
+ * Synchronises `stream` (a device-to-host copy). Any output pointer may be NULL.
+ * Errors: ISKV_ERR_INVALID_ARG, ISKV_ERR_CUDA.
+ */
+int iskv_fold_stats(iskv_handle *h, iskv_stream_t stream, int *max_sweeps_out,
+                    long long *total_sweeps_out, long long *cores_out);
+
 /* Tokens cached in `layer` (host value). Errors: ISKV_ERR_INVALID_ARG. */
 int iskv_num_tokens(const iskv_handle *h, int layer, long long *t_out);
 
@@ -167,9 +177,9 @@ int iskv_schedule(int block, int window, long long t, long long m, long long *n_
                   long long *folds_out);
 
 /*
- * Synchronises `stream` and returns the sticky device status: ISKV_OK, ISKV_ERR_NOT_CONVERGED or
- * ISKV_ERR_NONFINITE (the first error seen since creation), or ISKV_ERR_CUDA if the
- * synchronisation itself failed.
+ * Synchronises `stream` and returns the sticky device status: ISKV_OK, ISKV_ERR_NOT_CONVERGED,
+ * ISKV_ERR_NONFINITE or ISKV_ERR_TIMEOUT (the first error seen since creation or the last
+ * iskv_reset()), or ISKV_ERR_CUDA if the synchronisation itself failed.
  */
 int iskv_sync_status(iskv_handle *h, iskv_stream_t stream);
 

@@ -16,10 +16,10 @@ import os
 __all__ = [
     "IsKVError", "iskv_config", "lib", "check", "ISKV_OK", "ISKV_ERR_INVALID_ARG",
     "ISKV_ERR_CAPACITY", "ISKV_ERR_CUDA", "ISKV_ERR_NOT_CONVERGED", "ISKV_ERR_NONFINITE",
-    "ISKV_ERR_UNSUPPORTED", "ISKV_BF16", "ISKV_F32", "LIB_PATH",
+    "ISKV_ERR_UNSUPPORTED", "ISKV_ERR_TIMEOUT", "ISKV_BF16", "ISKV_F32", "LIB_PATH",
     "iskv_create", "iskv_destroy", "iskv_append_block", "iskv_decode_attn", "iskv_reconstruct",
     "iskv_get_factors", "iskv_num_tokens", "iskv_storage_bytes", "iskv_schedule",
-    "iskv_sync_status", "iskv_strerror", "iskv_reset", "iskv_launch_count",
+    "iskv_sync_status", "iskv_strerror", "iskv_reset", "iskv_launch_count", "iskv_fold_stats",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libiskv.so")
@@ -31,6 +31,7 @@ ISKV_ERR_CUDA = -3
 ISKV_ERR_NOT_CONVERGED = -4
 ISKV_ERR_NONFINITE = -5
 ISKV_ERR_UNSUPPORTED = -6
+ISKV_ERR_TIMEOUT = -7
 ISKV_BF16 = 0
 ISKV_F32 = 1
 
@@ -80,6 +81,8 @@ _SIGNATURES = {
     "iskv_strerror": (ctypes.c_char_p, [_i]),
     "iskv_reset": (_i, [_vp, _vp]),
     "iskv_launch_count": (_i, [_vp, ctypes.POINTER(_ll)]),
+    "iskv_fold_stats": (_i, [_vp, _vp, ctypes.POINTER(_i), ctypes.POINTER(_ll),
+                             ctypes.POINTER(_ll)]),
 }
 
 
@@ -190,6 +193,16 @@ def iskv_launch_count(handle):
     n = _ll(0)
     code = lib.iskv_launch_count(handle, ctypes.byref(n))
     return code, n.value
+
+
+def iskv_fold_stats(handle, stream=None):
+    """Returns ``(code, max_sweeps, total_sweeps, cores)``; synchronises the stream."""
+    m = _i(0)
+    t = _ll(0)
+    c = _ll(0)
+    code = lib.iskv_fold_stats(handle, _stream(stream), ctypes.byref(m), ctypes.byref(t),
+                               ctypes.byref(c))
+    return code, m.value, t.value, c.value
 
 
 def iskv_sync_status(handle, stream=None) -> int:

@@ -5,7 +5,8 @@ from __future__ import annotations
 import torch
 
 from .binding import (ISKV_BF16, ISKV_F32, check, iskv_append_block, iskv_config, iskv_create,
-                      iskv_decode_attn, iskv_destroy, iskv_get_factors, iskv_launch_count,
+                      iskv_decode_attn, iskv_destroy, iskv_fold_stats, iskv_get_factors,
+                      iskv_launch_count,
                       iskv_num_tokens, iskv_reconstruct, iskv_reset, iskv_storage_bytes,
                       iskv_sync_status)
 
@@ -95,6 +96,12 @@ class IsKVCache:
         code, n = iskv_launch_count(self.handle)
         check(code, "iskv_launch_count")
         return n
+
+    def fold_stats(self, stream=None):
+        """``(max_sweeps, total_sweeps, cores)`` of the core SVDs since creation/reset."""
+        code, m, t, c = iskv_fold_stats(self.handle, stream)
+        check(code, "iskv_fold_stats")
+        return m, t, c
 
     def status(self, stream=None) -> int:
         return iskv_sync_status(self.handle, stream)

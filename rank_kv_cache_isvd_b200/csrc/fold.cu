@@ -203,7 +203,9 @@ __global__ void __launch_bounds__(FOLD_THREADS, 1) fold_core_kernel(FoldArgs a) 
         const int gid = tid / JG, gl = tid % JG;
         const unsigned gmask = 0xffu << ((lane / JG) * JG);
         bool converged = false;
+        int sweeps = 0;
         for (int sweep = 0; sweep < JACOBI_MAX_SWEEPS; ++sweep) {
+            ++sweeps;
             if (tid == 0) sFlag[0] = 0;
             __syncthreads();
             for (int round = 0; round < Np - 1; ++round) {
@@ -231,12 +233,17 @@ __global__ void __launch_bounds__(FOLD_THREADS, 1) fold_core_kernel(FoldArgs a) 
                         const float az = fabsf(zeta);
                         const float t = (az > 1e18f ? 0.5f / az : 1.f / (az + sqrtf(fmaf(az, az, 1.f))));
                         const float tt = zeta < 0.f ? -t : t;
-                        const float c = 1.f / sqrtf(fmaf(tt, tt, 1.f));
-                        const float s = c * tt;
+                        // rotation [[c, s], [-s, c]] with c = 1/rr, s = t/rr applied as a
+                        // correction: dc = 1 - c is formed directly, because for |t| < sqrt(eps)
+                        // c rounds to 1 while s = t, and the rounded rotation would inflate column
+                        // norms by t^2/2 each time (a systematic bias over thousands of rotations)
+                        const float rr = sqrtf(fmaf(tt, tt, 1.f));
+                        const float dc = (tt * tt) / (rr * (1.f + rr));
+                        const float s = tt / rr;
                         for (int m = gl; m < n; m += JG) {
                             const float u = xa[m], v = xb[m];
-                            xa[m] = c * u - s * v;
-                            xb[m] = s * u + c * v;
+                            xa[m] = u - fmaf(dc, u, s * v);
+                            xb[m] = v - fmaf(dc, v, -s * u);
                         }
                         if (gl == 0 && t != 0.f) sFlag[0] = 1;
                     }
@@ -250,6 +257,11 @@ __global__ void __launch_bounds__(FOLD_THREADS, 1) fold_core_kernel(FoldArgs a) 
             __syncthreads();
         }
         if (!converged && tid == 0) set_status(a.status, ISKV_ERR_NOT_CONVERGED);
+        if (tid == 0 && a.stats) {
+            atomicMax(a.stats, (unsigned long long)sweeps);
+            atomicAdd(a.stats + 1, (unsigned long long)sweeps);
+            atomicAdd(a.stats + 2, 1ull);
+        }
     }
 
     // ---- singular values = column norms; select the top kp (descending, ties by index) -------

@@ -31,6 +31,11 @@ struct iskv_handle {
     float2 *rope_cs = nullptr;
     float *ws = nullptr;
     int *status = nullptr;
+    unsigned long long *stats = nullptr;  // fold statistics (3 counters)
+    int *counters = nullptr;              // decode split arrival counters [units per layer]
+    bool tc = false;                      // tensor-core decode available for this shape
+    CUtensorMap tmC;                      // key coordinates [U * n_max][r_K], 32 x 128 boxes
+    CUtensorMap tmB[2];                   // key bases (two buffers) [U * D][r_K]
     std::vector<long long> t, nc;
     std::vector<int> kcur[2];
     std::vector<int> cur;  // which basis buffer is current, per layer
@@ -70,6 +75,44 @@ void free_all(iskv_handle *h) {
     cudaFree(h->rope_cs);
     cudaFree(h->ws);
     cudaFree(h->status);
+    cudaFree(h->stats);
+    cudaFree(h->counters);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D fp32 tensor [rows][cols] (row stride cols), boxes of 32 columns x 128 rows, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const float *base, int cols, long long rows) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn || rows < 1 || rows > 0x7fffffffLL) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(float)};
+    cuuint32_t box[2] = {32, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool valid_layer(const iskv_handle *h, int layer) {
@@ -115,6 +158,7 @@ int fold_layers(iskv_handle *h, int l0, int nl, cudaStream_t s) {
     fa.b = c.block;
     fa.kv_dtype = c.kv_dtype;
     fa.status = h->status;
+    fa.stats = h->stats;
     if (launch_fold(fa, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
     h->launches += 1 + (nc > 0 ? 1 : 0);
     ra.unit0 = l0 * h->UL;
@@ -143,6 +187,7 @@ const char *iskv_strerror(int code) {
         case ISKV_ERR_NOT_CONVERGED: return "core SVD did not converge within the sweep cap";
         case ISKV_ERR_NONFINITE: return "non-finite singular value";
         case ISKV_ERR_UNSUPPORTED: return "unsupported configuration";
+        case ISKV_ERR_TIMEOUT: return "a device-side wait exceeded its bound";
         default: return "unknown error";
     }
 }
@@ -215,6 +260,8 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
     if (c.rope) alloc((void **)&h->rope_cs, (size_t)c.max_tokens * DH * sizeof(float2));
     alloc((void **)&h->ws, (size_t)h->UL * h->max_splits * h->G * (2 + D) * sizeof(float));
     alloc((void **)&h->status, sizeof(int));
+    alloc((void **)&h->stats, 4 * sizeof(unsigned long long));
+    alloc((void **)&h->counters, (size_t)h->UL * sizeof(int));
     if (ok) {
         for (int x = 0; x < 2; ++x) {
             const size_t r = (size_t)rank_of(h, x);
@@ -223,6 +270,8 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
             ok = ok && cudaMemset(h->sigma[x], 0, U * r * sizeof(float)) == cudaSuccess;
         }
         ok = ok && cudaMemset(h->status, 0, sizeof(int)) == cudaSuccess;
+        ok = ok && cudaMemset(h->stats, 0, 4 * sizeof(unsigned long long)) == cudaSuccess;
+        ok = ok && cudaMemset(h->counters, 0, (size_t)h->UL * sizeof(int)) == cudaSuccess;
         if (ok && c.rope)
             ok = launch_rope_table(h->rope_cs, c.max_tokens, c.rope_theta, 0) == cudaSuccess;
         ok = ok && cudaDeviceSynchronize() == cudaSuccess;
@@ -232,6 +281,21 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         delete h;
         cudaGetLastError();
         return ISKV_ERR_CUDA;
+    }
+    // tensor-core decode: key coordinates in 32-column TMA boxes (r_K <= 64, rows 16-byte
+    // aligned), value rows copied in bulk (r_V multiple of 4), compute capability 10.x
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, h->device);
+    memset(&h->tmC, 0, sizeof(h->tmC));
+    memset(h->tmB, 0, sizeof(h->tmB));
+    if (major == 10 && c.rank_k % 4 == 0 && c.rank_k <= 64 && c.rank_v % 4 == 0) {
+        bool m_ok = true;
+        if (h->n_max > 0) {
+            m_ok = make_map(&h->tmC, h->coords[0], c.rank_k, (long long)h->U * h->n_max) &&
+                   make_map(&h->tmB[0], h->basis[0][0], c.rank_k, (long long)h->U * D) &&
+                   make_map(&h->tmB[1], h->basis[0][1], c.rank_k, (long long)h->U * D);
+        }
+        h->tc = m_ok;
     }
     *out = h;
     return ISKV_OK;
@@ -329,8 +393,20 @@ int iskv_decode_attn(iskv_handle *h, int layer, const float *q, float *out, iskv
     da.kv_dtype = c.kv_dtype;
     da.scale = 1.0f / sqrtf((float)D);
     if (da.n_split > h->max_splits) return ISKV_ERR_INVALID_ARG;
-    if (launch_decode(da, h->UL, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return ISKV_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (h->tc) {
+        TcExtra x;
+        x.kblocks = (c.rank_k + 31) / 32;
+        x.row0 = (long long)layer * h->UL * h->n_max;
+        x.brow0 = layer * h->UL * D;
+        x.counters = h->counters;
+        x.status = h->status;
+        if (launch_decode_tc(&h->tmC, &h->tmB[cur], da, x, h->UL, s) != cudaSuccess)
+            return ISKV_ERR_CUDA;
+        h->launches += 1;
+        return ISKV_OK;
+    }
+    if (launch_decode(da, h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
     h->launches += 2;
     return ISKV_OK;
 }
@@ -401,6 +477,24 @@ int iskv_reset(iskv_handle *h, iskv_stream_t stream) {
     if (cudaMemsetAsync(h->status, 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)) !=
         cudaSuccess)
         return ISKV_ERR_CUDA;
+    if (cudaMemsetAsync(h->stats, 0, 4 * sizeof(unsigned long long),
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ISKV_ERR_CUDA;
+    return ISKV_OK;
+}
+
+int iskv_fold_stats(iskv_handle *h, iskv_stream_t stream, int *max_sweeps_out,
+                    long long *total_sweeps_out, long long *cores_out) {
+    if (!h) return ISKV_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    unsigned long long v[4] = {0, 0, 0, 0};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(v, h->stats, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return ISKV_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ISKV_ERR_CUDA;
+    if (max_sweeps_out) *max_sweeps_out = (int)v[0];
+    if (total_sweeps_out) *total_sweeps_out = (long long)v[1];
+    if (cores_out) *cores_out = (long long)v[2];
     return ISKV_OK;
 }
 

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cuda.h>
+
 #include "iskv.h"
 
 namespace iskv {
@@ -38,6 +40,7 @@ struct FoldArgs {
     int b;                  // block
     int kv_dtype;
     int *status;
+    unsigned long long *stats;  // [0] max sweeps, [1] total sweeps, [2] cores solved
 };
 
 // ---- history rotation C[0:n] <- C[0:n] H_top (or stale zero-padding) ---------------------------
@@ -100,13 +103,25 @@ struct ReconArgs {
     int R, kv_dtype, apply_rope;
 };
 
+// extra state of the tensor-core decode kernel
+struct TcExtra {
+    int kblocks;            // 32-column K-blocks of the key coordinates (ceil(r_K / 32))
+    long long row0;         // first coordinate row of this layer in the coordinate tensor map
+    int brow0;              // first basis row of this layer in the basis tensor map
+    int *counters;          // [units of the layer] split arrival counters (self-resetting)
+    int *status;
+};
+
 cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_append(const AppendArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_reconstruct(const ReconArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_rope_table(float2 *table, long long max_tokens, double theta, cudaStream_t s);
+cudaError_t launch_decode_tc(const CUtensorMap *tmC, const CUtensorMap *tmB, const DecodeArgs &a,
+                             const TcExtra &x, int n_units, cudaStream_t s);
 size_t fold_smem_bytes();
+size_t tc_smem_bytes(int kblocks, int rV, int esz);
 
 __device__ __forceinline__ float load_row_elem(const void *base, size_t idx, int kv_dtype) {
     if (kv_dtype == ISKV_BF16)

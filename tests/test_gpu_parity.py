@@ -272,3 +272,42 @@ def test_block_of_one_row_and_capacity_error():
         cache.append(0, to_device(kd[0][:, :, :1]), to_device(vd[0][:, :, :1]))
     assert e.value.code == ISKV_ERR_CAPACITY
     assert cache.tokens(0) == 150
+
+
+def test_fma_decode_path_for_ranks_outside_the_tensor_core_layout():
+    """r_K = 30 is not a multiple of 4, so decode runs on the CUDA-core kernel; same parity."""
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=900, rank_k=30, rank_v=42)
+    kd, kv, vd, vv = workload_arrays(wl)
+    cache, orc = make_cache(wl), make_oracle(wl)
+    append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], 0, wl.tokens)
+    q = syn.queries(13, (1, 8, 128))
+    out = cache.decode(0, torch.from_numpy(q).cuda()).cpu().numpy()
+    assert max_head_rel_err(out, orc.decode(0, q.astype(np.float64))) <= ATTN_TOL
+    assert cache.status() == 0
+
+
+def test_decode_is_repeatable_and_graph_capturable():
+    """The same decode twice gives identical output (the split-merge counters re-arm), also
+    when captured into a CUDA graph and replayed."""
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=1500)
+    kd, kv, vd, vv = workload_arrays(wl)
+    cache = make_cache(wl)
+    cache.append(0, to_device(kd[0]), to_device(vd[0]))
+    q = torch.from_numpy(syn.queries(17, (1, 8, 128))).cuda()
+    o1 = cache.decode(0, q).clone()
+    o2 = cache.decode(0, q).clone()
+    assert torch.equal(o1, o2)
+    out = torch.empty_like(q)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        cache.decode(0, q, out, stream=s)       # warm-up on the capture stream
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        cache.decode(0, q, out, stream=s)
+    out.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, o1)
+    assert cache.status() == 0

@@ -76,7 +76,7 @@ def test_null_handle_and_strerror():
     assert iskv.iskv_append_block(None, 0, 1, 1, 1, 0) == iskv.ISKV_ERR_INVALID_ARG
     assert iskv.iskv_decode_attn(None, 0, 1, 1, 0) == iskv.ISKV_ERR_INVALID_ARG
     assert iskv.iskv_sync_status(None, 0) == iskv.ISKV_ERR_INVALID_ARG
-    for code in range(-6, 1):
+    for code in range(-7, 1):
         assert iskv.iskv_strerror(code) != "unknown error"
     assert iskv.iskv_strerror(-99) == "unknown error"
 
