@@ -108,7 +108,7 @@ __device__ __forceinline__ void load_row32(const void *ring, size_t base, int kv
     }
 }
 
-__global__ void __launch_bounds__(TC_THREADS, 1) decode_tc_kernel(
+__global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmB,
     DecodeArgs a, TcExtra x) {
     extern __shared__ uint8_t smem_raw[];
@@ -141,8 +141,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1) decode_tc_kernel(
         p0 = a.n_c + (long long)(split - a.n_split_c) * DEC_TILE;
         p1 = min(a.t, p0 + DEC_TILE);
     }
-    for (int o = tid; o < G * D; o += TC_THREADS)
-        sQ[o] = a.q[((size_t)seq * a.H * G + (size_t)h * G) * D + o] * a.scale;
+    {
+        const float4 *q4 = reinterpret_cast<const float4 *>(a.q + ((size_t)seq * a.H * G + (size_t)h * G) * D);
+        float4 *s4 = reinterpret_cast<float4 *>(sQ);
+        const float sc = a.scale;
+        float4 v[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int o = tid + TC_THREADS * u;
+            v[u] = o < G * D / 4 ? q4[o] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int o = tid + TC_THREADS * u;
+            if (o < G * D / 4) s4[o] = make_float4(v[u].x * sc, v[u].y * sc, v[u].z * sc, v[u].w * sc);
+        }
+    }
     if (tid < G) {
         sM[tid] = -CUDART_INF_F;
         sL[tid] = 0.f;
@@ -164,15 +178,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1) decode_tc_kernel(
     const float *Cv = a.coords[1] + (size_t)ul * a.n_max * rV;
     const uint32_t idesc = idesc_tf32(128, 128);
 
-    if (comp) {
-        if (tid == 0) {
-            mbar_arrive_expect_tx(bar_load, x.kblocks * KBLK_BYTES);
+    // thread 0: loads of one tile (key coordinates by TMA, value coordinates or exact window
+    // value rows by bulk copy); the caller has posted the expected byte count
+    auto issue_tile = [&](long long t0, int rows) {
+        if (comp) {
+            for (int kb = 0; kb < x.kblocks; ++kb)
+                tma_load_2d(bAh + kb * KBLK_BYTES, &tmC, kb * 32,
+                            (int)(x.row0 + (long long)ul * a.n_max + t0), bar_load);
+            bulk_load(bV, Cv + (size_t)t0 * rV, (uint32_t)rows * rV * 4, bar_load);
+        } else {
+            const int s0 = (int)(t0 % a.R);
+            const int n1 = min(rows, a.R - s0);
+            const uint32_t rb = D * esz;
+            const char *ring = static_cast<const char *>(a.ring[1]);
+            bulk_load(bV, ring + (ring_base + (size_t)s0 * D) * esz, (uint32_t)n1 * rb, bar_load);
+            if (n1 < rows)
+                bulk_load(bV + (size_t)n1 * rb, ring + ring_base * esz, (uint32_t)(rows - n1) * rb,
+                          bar_load);
+        }
+    };
+    auto tile_bytes = [&](int rows) -> uint32_t {
+        return comp ? x.kblocks * KBLK_BYTES + (uint32_t)rows * rV * 4 : (uint32_t)rows * D * esz;
+    };
+    if (tid == 0 && p0 < p1) {
+        const int rows0 = (int)min((long long)DEC_TILE, p1 - p0);
+        mbar_arrive_expect_tx(bar_load, tile_bytes(rows0) + (comp ? x.kblocks * KBLK_BYTES : 0u));
+        if (comp)
             for (int kb = 0; kb < x.kblocks; ++kb)
                 tma_load_2d(bBh + kb * KBLK_BYTES, &tmB, kb * 32, x.brow0 + ul * D, bar_load);
-        }
-        ok = __syncthreads_and(mbar_wait(bar_load, ph_load)) != 0;
-        ph_load ^= 1;
-        if (ok) split_tf32(bBh, bBl, x.kblocks * KBLK_BYTES);
+        issue_tile(p0, rows0);
     }
 
     float vacc[8];
@@ -182,35 +216,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1) decode_tc_kernel(
 
     for (long long t0 = p0; t0 < p1 && ok; t0 += DEC_TILE) {
         const int rows = (int)min((long long)DEC_TILE, p1 - t0);
-        tc_fence_before();
-        __syncthreads();                     // previous tile fully consumed (smem and TMEM)
-        if (tid == 0) {
-            if (comp) {
-                const uint32_t vbytes = (uint32_t)rows * rV * 4;
-                mbar_arrive_expect_tx(bar_load, x.kblocks * KBLK_BYTES + vbytes);
-                for (int kb = 0; kb < x.kblocks; ++kb)
-                    tma_load_2d(bAh + kb * KBLK_BYTES, &tmC, kb * 32,
-                                (int)(x.row0 + (long long)ul * a.n_max + t0), bar_load);
-                bulk_load(bV, Cv + (size_t)t0 * rV, vbytes, bar_load);
-            } else {
-                const int s0 = (int)(t0 % a.R);
-                const int n1 = min(rows, a.R - s0);
-                const uint32_t rb = D * esz;
-                mbar_arrive_expect_tx(bar_load, (uint32_t)rows * rb);
-                const char *ring = static_cast<const char *>(a.ring[1]);
-                bulk_load(bV, ring + (ring_base + (size_t)s0 * D) * esz, (uint32_t)n1 * rb, bar_load);
-                if (n1 < rows)
-                    bulk_load(bV + (size_t)n1 * rb, ring + ring_base * esz, (uint32_t)(rows - n1) * rb,
-                              bar_load);
+        if (t0 != p0) {
+            tc_fence_before();
+            __syncthreads();                 // previous tile fully consumed (smem and TMEM)
+            if (tid == 0) {
+                mbar_arrive_expect_tx(bar_load, tile_bytes(rows));
+                issue_tile(t0, rows);
             }
         }
         ok = __syncthreads_and(mbar_wait(bar_load, ph_load)) != 0;
         ph_load ^= 1;
         if (!ok) break;
+        if (comp && t0 == p0) split_tf32(bBh, bBl, x.kblocks * KBLK_BYTES);
 
         const int row = tid;
         const bool valid = row < rows;
         const long long pos = t0 + row;
+        const bool rope = valid && a.rope_cs != nullptr;
+        float4 cs0[16];
         float part[GMAX];
 #pragma unroll
         for (int g = 0; g < GMAX; ++g) part[g] = 0.f;
@@ -235,12 +258,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1) decode_tc_kernel(
                     }
                 mma_commit(bar_mma);
             }
+            if (rope) {                       // RoPE angles of pass 0 load while the MMA runs
+                const float4 *cs = reinterpret_cast<const float4 *>(a.rope_cs + pos * DH);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) cs0[q] = cs[q];
+            }
             ok = __syncthreads_and(mbar_wait(bar_mma, ph_mma)) != 0;
             ph_mma ^= 1;
             tc_fence_after();
             if (!ok) break;
         }
 
+        if (!comp && rope) {
+            const float4 *cs = reinterpret_cast<const float4 *>(a.rope_cs + pos * DH);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) cs0[q] = cs[q];
+        }
         // ---- this row's key (two passes: channel pairs (j, j+64), j in [32hp, 32hp+32)) -------
         const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
 #pragma unroll
@@ -258,11 +291,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) decode_tc_kernel(
 #pragma unroll
                 for (int j = 0; j < 32; ++j) lo[j] = hi[j] = 0.f;
             }
-            if (valid && a.rope_cs) {
+            if (rope) {
                 const float4 *cs = reinterpret_cast<const float4 *>(a.rope_cs + pos * DH + hp * 32);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
-                    const float4 w = cs[q];
+                    const float4 w = hp == 0 ? cs0[q] : cs[q];
                     const float x0 = lo[2 * q], y0 = hi[2 * q], x1 = lo[2 * q + 1], y1 = hi[2 * q + 1];
                     lo[2 * q] = x0 * w.x - y0 * w.y;
                     hi[2 * q] = y0 * w.x + x0 * w.y;
@@ -335,33 +368,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1) decode_tc_kernel(
             if (o < G * nacc) {
                 const int g = o / nacc, c = o % nacc;
                 const float *pg = sP + g * DEC_TILE;
-                float s0 = 0.f, s1 = 0.f;
-                if (comp) {
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                const int ld = comp ? rV : D;
+                int i = 0;
+                if (comp || esz == 4) {
                     const float *vv = reinterpret_cast<const float *>(bV) + c;
-                    int i = 0;
-                    for (; i + 1 < rows; i += 2) {
-                        s0 = fmaf(pg[i], vv[i * rV], s0);
-                        s1 = fmaf(pg[i + 1], vv[(i + 1) * rV], s1);
-                    }
-                    if (i < rows) s0 = fmaf(pg[i], vv[i * rV], s0);
-                } else if (esz == 2) {
-                    const __nv_bfloat16 *vv = reinterpret_cast<const __nv_bfloat16 *>(bV) + c;
-                    int i = 0;
-                    for (; i + 1 < rows; i += 2) {
-                        s0 = fmaf(pg[i], __bfloat162float(vv[i * D]), s0);
-                        s1 = fmaf(pg[i + 1], __bfloat162float(vv[(i + 1) * D]), s1);
-                    }
-                    if (i < rows) s0 = fmaf(pg[i], __bfloat162float(vv[i * D]), s0);
+                    for (; i + 3 < rows; i += 4)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) s4[u] = fmaf(pg[i + u], vv[(i + u) * ld], s4[u]);
+                    for (; i < rows; ++i) s4[0] = fmaf(pg[i], vv[i * ld], s4[0]);
                 } else {
-                    const float *vv = reinterpret_cast<const float *>(bV) + c;
-                    int i = 0;
-                    for (; i + 1 < rows; i += 2) {
-                        s0 = fmaf(pg[i], vv[i * D], s0);
-                        s1 = fmaf(pg[i + 1], vv[(i + 1) * D], s1);
-                    }
-                    if (i < rows) s0 = fmaf(pg[i], vv[i * D], s0);
+                    const __nv_bfloat16 *vv = reinterpret_cast<const __nv_bfloat16 *>(bV) + c;
+                    for (; i + 3 < rows; i += 4)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            s4[u] = fmaf(pg[i + u], __bfloat162float(vv[(i + u) * D]), s4[u]);
+                    for (; i < rows; ++i) s4[0] = fmaf(pg[i], __bfloat162float(vv[i * D]), s4[0]);
                 }
-                vacc[w] = fmaf(vacc[w], sAl[g], s0 + s1);
+                vacc[w] = fmaf(vacc[w], sAl[g], (s4[0] + s4[1]) + (s4[2] + s4[3]));
             }
         }
     }
@@ -394,46 +418,114 @@ __global__ void __launch_bounds__(TC_THREADS, 1) decode_tc_kernel(
     __syncthreads();
     if (!sFlag[0]) return;
     __threadfence();
-    float *sW = reinterpret_cast<float *>(bV);          // [n_split] split weights
-    float *sAcc = sP;                                    // [D] rank-space sum
-    const float *wsu = a.ws + (size_t)ul * a.max_splits * G * (2 + D);
-    const float *BV = a.basis[1] + (size_t)ul * D * rV;
-    for (int g = 0; g < G; ++g) {
-        float m = -CUDART_INF_F;
-        for (int s = tid; s < a.n_split; s += TC_THREADS)
-            m = fmaxf(m, __ldcg(wsu + ((size_t)s * G + g) * (2 + D)));
-        m = warp_max_f(m);
-        __syncthreads();
-        if (lane == 0) sRed[warp] = m;
-        __syncthreads();
-        const float M = fmaxf(fmaxf(sRed[0], sRed[1]), fmaxf(sRed[2], sRed[3]));
-        float lsum = 0.f;
-        for (int s = tid; s < a.n_split; s += TC_THREADS) {
-            const float *pw = wsu + ((size_t)s * G + g) * (2 + D);
-            const float w = expf(__ldcg(pw) - M);
-            sW[s] = w;
-            lsum = fmaf(w, __ldcg(pw + 1), lsum);
+    float *sBV = reinterpret_cast<float *>(bV);         // B_V rows [D][rV] (bulk copy)
+    const bool bv_smem = ok;
+    if (bv_smem && tid == 0) {
+        mbar_arrive_expect_tx(bar_load, (uint32_t)(D * rV * 4));
+        bulk_load(sBV, a.basis[1] + (size_t)ul * D * rV, (uint32_t)(D * rV * 4), bar_load);
+    }
+    // all q-heads at once: split maxima and sums, per-head weights, then each thread (one channel
+    // j) sums its channel over the splits with several independent loads in flight, and the
+    // rank-space part is expanded through row j of B_V (read as float4 from L2)
+    const int ns = a.n_split, nsc = a.n_split_c;
+    const int stride = G * (2 + D);
+    const float *wsu = a.ws + (size_t)ul * a.max_splits * stride;
+    float *sMw = reinterpret_cast<float *>(bBh);        // [ns][G] maxima, then weights
+    float *sLs = sMw + ns * G;                          // [ns][G] sums
+    float *sAcc = sP;                                   // [G][D] rank-space sums
+    for (int i0 = tid; i0 < ns * G; i0 += 4 * TC_THREADS) {
+        float mv[4], lv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * TC_THREADS;
+            const float *pw = wsu + (size_t)(i / G) * stride + (i % G) * (2 + D);
+            mv[u] = i < ns * G ? __ldcg(pw) : 0.f;
+            lv[u] = i < ns * G ? __ldcg(pw + 1) : 0.f;
         }
-        lsum = warp_sum_f(lsum);
-        if (lane == 0) sRed[4 + warp] = lsum;
-        __syncthreads();
-        const float Lsum = sRed[4] + sRed[5] + sRed[6] + sRed[7];
-        const int j = tid;
-        float accr = 0.f, accw = 0.f;
-        for (int s = 0; s < a.n_split; ++s) {
-            const float v = __ldcg(wsu + ((size_t)s * G + g) * (2 + D) + 2 + j);
-            if (s < a.n_split_c) {
-                if (j < kV) accr = fmaf(sW[s], v, accr);
-            } else {
-                accw = fmaf(sW[s], v, accw);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * TC_THREADS;
+            if (i < ns * G) {
+                sMw[i] = mv[u];
+                sLs[i] = lv[u];
             }
         }
-        sAcc[j] = accr;
+    }
+    __syncthreads();
+    for (int g = warp; g < G; g += 4) {
+        float m = -CUDART_INF_F;
+        for (int s2 = lane; s2 < ns; s2 += 32) m = fmaxf(m, sMw[s2 * G + g]);
+        m = warp_max_f(m);
+        float lsum = 0.f;
+        for (int s2 = lane; s2 < ns; s2 += 32) {
+            const float w = expf(sMw[s2 * G + g] - m);
+            sMw[s2 * G + g] = w;
+            lsum = fmaf(w, sLs[s2 * G + g], lsum);
+        }
+        lsum = warp_sum_f(lsum);
+        if (lane == 0) sRed[g] = lsum;
+    }
+    __syncthreads();
+    {
+        const int j = tid;
+        float accr[GMAX], accw[GMAX];
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) accr[g] = accw[g] = 0.f;
+        for (int s0 = 0; s0 < ns; s0 += 16) {
+            float v[16][GMAX];
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+#pragma unroll
+                for (int g = 0; g < GMAX; ++g) {
+                    const int s2 = s0 + u;
+                    v[u][g] = (g < G && s2 < ns && (s2 >= nsc || j < kV))
+                                  ? __ldcg(wsu + (size_t)s2 * stride + g * (2 + D) + 2 + j)
+                                  : 0.f;
+                }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int s2 = s0 + u;
+                if (s2 < ns) {
+#pragma unroll
+                    for (int g = 0; g < GMAX; ++g)
+                        if (g < G) {
+                            const float w = sMw[s2 * G + g];
+                            if (s2 < nsc) accr[g] = fmaf(w, v[u][g], accr[g]);
+                            else accw[g] = fmaf(w, v[u][g], accw[g]);
+                        }
+                }
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g)
+            if (g < G) sAcc[g * D + j] = accr[g];
         __syncthreads();
-        float o = accw;
-        for (int c = 0; c < kV; ++c) o = fmaf(sAcc[c], __ldg(BV + (size_t)j * rV + c), o);
-        a.out[((size_t)seq * a.H * G + (size_t)h * G + g) * D + j] = o / Lsum;
-        __syncthreads();
+        float o[GMAX];
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) o[g] = accw[g];
+        const bool bv_ok = bv_smem && __syncthreads_and(mbar_wait(bar_load, ph_load)) != 0;
+        const float *bvrow = bv_ok ? sBV + j * rV : a.basis[1] + ((size_t)ul * D + j) * rV;
+        for (int c4 = 0; c4 < kV / 4; ++c4) {
+            const float4 b4 = reinterpret_cast<const float4 *>(bvrow)[c4];
+#pragma unroll
+            for (int g = 0; g < GMAX; ++g)
+                if (g < G) {
+                    const float *ac = sAcc + g * D + 4 * c4;
+                    o[g] = fmaf(ac[0], b4.x, o[g]);
+                    o[g] = fmaf(ac[1], b4.y, o[g]);
+                    o[g] = fmaf(ac[2], b4.z, o[g]);
+                    o[g] = fmaf(ac[3], b4.w, o[g]);
+                }
+        }
+        for (int c = kV & ~3; c < kV; ++c) {
+            const float b1 = bvrow[c];
+#pragma unroll
+            for (int g = 0; g < GMAX; ++g)
+                if (g < G) o[g] = fmaf(sAcc[g * D + c], b1, o[g]);
+        }
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g)
+            if (g < G) a.out[((size_t)seq * a.H * G + (size_t)h * G + g) * D + j] = o[g] / sRed[g];
     }
     if (tid == 0) x.counters[ul] = 0;
 }

@@ -2,30 +2,45 @@
 //
 // iS-KV summary, "Block-Incremental Decoding Updates", steps 1-3, for history A = U Sigma B^T
 // (k components, coordinates C = U Sigma stored) and pending block F (b rows of the window):
-//   1. S = F B, E = F - S B^T (projected twice); orthonormal residual basis P (d x p) from a
-//      Householder QR of [B, E^T] (its columns after the first k), p = min(b, d - k);
+//   1. S = F B, E = F - S B^T; orthonormal residual basis P (d x p) from a Householder QR of
+//      [B, E^T] (its columns after the first k), p = min(b, d - k). The QR runs over B's columns
+//      first, which re-orthogonalises E against B to rounding (the oracle's second projection pass).
 //   2. Z = [[Sigma, 0], [S, F P]], (k + b) x (k + p); with P from that QR, F P = E P is the
-//      transpose of the QR's trailing R block for the rows that entered it;
+//      transpose of the QR's trailing R block for the rows that entered it.
 //   3. (G, Sigma+, H) = SVD_r(Z) by one-sided (Hestenes) Jacobi on the columns of Z^T: at
 //      convergence the columns of Z^T J are orthogonal, their norms are the singular values and
 //      the normalised columns are the right singular vectors H of Z, so J is never accumulated;
-//      B+ = [B P] H, the old coordinates move by H[:k] (kernel rotate_kernel) and the new rows'
+//      B+ = [B P] H, the old coordinates move by H[:k] (rotate_kernel) and the new rows'
 //      coordinates are F B+ (bottom block of U+ Sigma+, since Z H = G Sigma+).
-// One CTA per unit and path (blockIdx.y = path), everything in shared memory (b <= 128).
+// One CTA (256 threads) per unit and path (blockIdx.y = path), everything on chip (b <= 128).
 #include "iskv_internal.cuh"
 
 namespace iskv {
 
-constexpr int FOLD_THREADS = 512;
-constexpr int FOLD_WARPS = FOLD_THREADS / 32;
-constexpr int JG = 8;                         // lanes per Jacobi pair group
-constexpr int JGROUPS = FOLD_THREADS / JG;    // pair groups per CTA
+constexpr int FT = 256;                       // threads
+constexpr int FW = FT / 32;                   // warps
+constexpr int JL = 16;                        // lanes per Jacobi column group
+constexpr int JGRP = FT / JL;                 // column groups
+constexpr int NSLOT = 2 * JGRP;               // Jacobi slots (two per group)
+constexpr int SS = 132;                       // column stride of the Jacobi staging area
 constexpr float JACOBI_TOL = 4e-6f;           // rotate while |a.b| > tol |a| |b|
 
-size_t fold_smem_bytes() {
-    return (size_t)(3 * 128 * LDS + 128 + 128 + 256 + FOLD_WARPS * 128) * sizeof(float) +
-           (size_t)(128 + 4) * sizeof(int);
-}
+// shared memory (floats)
+constexpr int OFF_A = 0;                                  // F/E rows -> [P | B_old] -> F rows
+constexpr int OFF_B = OFF_A + 128 * LDS;                  // Y = [S | T] rows
+constexpr int STAGE_FLOATS = NSLOT * 8 * SS;              // Jacobi staging (overlays B and C)
+constexpr int C_FLOATS = STAGE_FLOATS - 128 * LDS;        // QR columns -> Sigma columns
+constexpr int OFF_C = OFF_B + 128 * LDS;
+constexpr int OFF_TAU = OFF_C + C_FLOATS;
+constexpr int OFF_SIG = OFF_TAU + 128;
+constexpr int OFF_NRM = OFF_SIG + 128;                    // [256] column norms
+constexpr int OFF_SNRM = OFF_NRM + 256;                   // [256] staged squared norms
+constexpr int OFF_SCR = OFF_SNRM + 256;                   // per-warp scratch, 128 floats each
+constexpr int OFF_INT = OFF_SCR + FW * 128;               // ints: sel[256], flags[4]
+constexpr int SMEM_FLOATS = OFF_INT + 256 + 4;
+static_assert(C_FLOATS >= 128 * LDS, "QR matrix must fit");
+
+size_t fold_smem_bytes() { return (size_t)SMEM_FLOATS * sizeof(float); }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -33,91 +48,371 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Round-robin (circle) schedule over Np players: in each of the Np - 1 rounds every player meets
-// one other; over a sweep every pair meets once.
-__device__ __forceinline__ void rr_pair(int Np, int round, int i, int &a, int &b) {
-    const int M = Np - 1;
-    if (i == 0) {
-        a = 0;
-        b = 1 + round % M;
-    } else {
-        a = 1 + (round + i) % M;
-        b = 1 + (round - i + M) % M;
+__device__ __forceinline__ float group_sum(float v) {   // over the 16 lanes of a Jacobi group
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    return v;
+}
+
+// Rotation parameters of one Hestenes step for columns with squared norms nx, ny and inner
+// product g: t = tan(theta) of the rotation [[c, s], [-s, c]] that makes the pair orthogonal, or
+// t = 0 (identity) when |g| <= tol |x| |y|. Returns (s, dc) with dc = 1 - c formed directly: for
+// |t| < sqrt(eps) c rounds to 1 while s = t, and a rounded rotation would inflate the norms by
+// t^2/2 every time (a systematic bias over thousands of rotations). With dc and s derived from
+// the same 1/sqrt(1 + t^2), c^2 + s^2 - 1 = O(eps t^2), so approximate reciprocals and square
+// roots keep tiny rotations norm-preserving.
+__device__ __forceinline__ void jparams(float g, float nx, float ny, float &t, float &s, float &dc) {
+    const bool doit = g * g > (JACOBI_TOL * JACOBI_TOL) * nx * ny;
+    const float gg = doit ? g : 1.f;
+    const float zeta = __fdividef(ny - nx, 2.f * gg);
+    const float az = fminf(fabsf(zeta), 1e18f);
+    const float q = fmaf(az, az, 1.f);
+    const float t0 = __fdividef(1.f, az + q * rsqrtf(q));
+    t = doit ? copysignf(t0, zeta) : 0.f;
+    const float ri = rsqrtf(fmaf(t, t, 1.f));           // c = 1 / sqrt(1 + t^2)
+    s = t * ri;
+    dc = __fdividef(t * t * ri * ri, 1.f + ri);          // 1 - c
+}
+
+// Rotates HC disjoint column pairs (x_j, y_(j+S) mod HC) of a lane group at once: the dot
+// products, their reductions and the rotation parameters of all pairs overlap (no branches).
+template <int HC, int RPL, int S>
+__device__ __forceinline__ void jcross(float (&xa)[HC][RPL], float (&xb)[HC][RPL], float (&na)[HC],
+                                       float (&nb)[HC], int &rotated) {
+    float g[HC];
+#pragma unroll
+    for (int j = 0; j < HC; ++j) {
+        g[j] = 0.f;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) g[j] = fmaf(xa[j][i], xb[(j + S) % HC][i], g[j]);
+    }
+#pragma unroll
+    for (int o = 1; o < JL; o <<= 1)
+#pragma unroll
+        for (int j = 0; j < HC; ++j) g[j] += __shfl_xor_sync(0xffffffffu, g[j], o);
+#pragma unroll
+    for (int j = 0; j < HC; ++j) {
+        const int jb = (j + S) % HC;
+        float t, sn, dc;
+        jparams(g[j], na[j], nb[jb], t, sn, dc);
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            const float xi = xa[j][i], yi = xb[jb][i];
+            xa[j][i] = fmaf(-sn, yi, fmaf(-dc, xi, xi));
+            xb[jb][i] = fmaf(sn, xi, fmaf(-dc, yi, yi));
+        }
+        na[j] = fmaxf(na[j] - t * g[j], 0.f);
+        nb[jb] = fmaxf(nb[jb] + t * g[j], 0.f);
+        rotated |= (t != 0.f);
     }
 }
 
-__global__ void __launch_bounds__(FOLD_THREADS, 1) fold_core_kernel(FoldArgs a) {
-    extern __shared__ float smem[];
-    float *sA = smem;                    // F/E rows -> [P | B_old] columns -> F rows
-    float *sB = sA + 128 * LDS;          // Y = [S | T] rows = Z^T columns k .. k+b-1
-    float *sC = sB + 128 * LDS;          // QR columns -> Z^T columns 0 .. k-1 -> B+ columns
-    float *sTau = sC + 128 * LDS;        // Householder tau
-    float *sSig = sTau + 128;            // Sigma (old)
-    float *sNrm = sSig + 128;            // column norms of Z^T J (up to 256 columns)
-    float *sScr = sNrm + 256;            // per-warp scratch (128 floats each)
-    int *sSel = reinterpret_cast<int *>(sScr + FOLD_WARPS * 128);
-    int *sFlag = sSel + 128;
-
-    const FoldPath P = blockIdx.y ? a.path[1] : a.path[0];
-    const int unit = a.unit0 + blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int k = P.k, r = P.r, p = P.p, kp = P.kp, b = a.b;
-    const int n = k + p;                 // rows of Z^T (columns of Z)
-    const int N = k + b;                 // columns of Z^T
-
-    const size_t ring_base = (size_t)unit * a.R * D;
-    const float *Bin = P.basis_in + (size_t)unit * D * r;
-
-    // ---- load F (b x D) and B (as k columns), Sigma ------------------------------------------
-    for (int o = tid; o < b * D; o += FOLD_THREADS) {
-        const int i = o / D, j = o % D;
-        const int slot = (a.slot0 + i) % a.R;
-        sA[i * LDS + j] = load_row_elem(P.ring, ring_base + (size_t)slot * D + j, a.kv_dtype);
+// One rotation of the pair (x, y) within a slot (used in round 0 of a sweep).
+template <int RPL>
+__device__ __forceinline__ void jrot(float (&x)[RPL], float (&y)[RPL], float &nx, float &ny,
+                                     int &rotated) {
+    float g = 0.f;
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) g = fmaf(x[i], y[i], g);
+    g = group_sum(g);
+    float t, sn, dc;
+    jparams(g, nx, ny, t, sn, dc);
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+        const float xi = x[i], yi = y[i];
+        x[i] = fmaf(-sn, yi, fmaf(-dc, xi, xi));
+        y[i] = fmaf(sn, xi, fmaf(-dc, yi, yi));
     }
-    for (int o = tid; o < D * k; o += FOLD_THREADS) {
-        const int j = o / k, c = o % k;
-        sC[c * LDS + j] = Bin[(size_t)j * r + c];
-    }
-    if (tid < k) sSig[tid] = P.sigma[(size_t)unit * r + tid];
-    if (tid == 0) sFlag[1] = 0;
-    __syncthreads();
+    nx = fmaxf(nx - t * g, 0.f);
+    ny = fmaxf(ny + t * g, 0.f);
+    rotated |= (t != 0.f);
+}
 
-    // ---- step 1: S = F B (into Y[:, :k]); E = F - S B^T, twice (one warp per row) -------------
-    if (k > 0) {
-        float *scr = sScr + warp * 128;
-        for (int i = warp; i < b; i += FOLD_WARPS) {
-            float *f = sA + i * LDS;
-            for (int c = lane; c < k; c += 32) {
-                const float *bc = sC + c * LDS;
-                float s = 0.f;
-                for (int j = 0; j < D; ++j) s = fmaf(f[j], bc[j], s);
-                sB[i * LDS + c] = s;
-                scr[c] = s;
-            }
-            __syncwarp();
-            for (int pass = 0; pass < 2; ++pass) {
-                for (int j = lane; j < D; j += 32) {
-                    float e = f[j];
-                    for (int c = 0; c < k; ++c) e = fmaf(-scr[c], sC[c * LDS + j], e);
-                    f[j] = e;
+template <int HC, int RPL, int S>
+struct JCrossAll {
+    __device__ __forceinline__ static void run(float (&xa)[HC][RPL], float (&xb)[HC][RPL],
+                                               float (&na)[HC], float (&nb)[HC], int &rotated) {
+        jcross<HC, RPL, S>(xa, xb, na, nb, rotated);
+        JCrossAll<HC, RPL, S + 1>::run(xa, xb, na, nb, rotated);
+    }
+};
+template <int HC, int RPL>
+struct JCrossAll<HC, RPL, HC> {
+    __device__ __forceinline__ static void run(float (&)[HC][RPL], float (&)[HC][RPL],
+                                               float (&)[HC], float (&)[HC], int &) {}
+};
+
+// Register-resident one-sided Jacobi on N <= 2 ng HC columns of length n <= 16 RPL, where
+// ng = ceil(N / (2 HC)) <= 16 column groups are active. Group g (16 lanes) holds slots top[g] and
+// bottom[g] of HC columns each; lane l holds rows [RPL l, RPL l + RPL). Each sweep is the
+// round-robin (circle) tournament on the 2 ng slots: 2 ng - 1 rounds, every slot pair meets once;
+// columns within a slot are rotated in round 0. Between rounds the slots move through the
+// staging area: top[0] stays, top[i] -> top[i+1], top[ng-1] -> bottom[ng-1],
+// bottom[i] -> bottom[i-1], bottom[0] -> top[1].
+// On return the final columns are in `stage` (column (pos*HC + j), stride SS, 2 ng HC columns)
+// with their norms in nrm_out; returns the number of sweeps (negative if the cap was reached).
+template <int HC, int RPL>
+__device__ __noinline__ int jacobi_regs(const float *sB, const float *sC, int k, int N, int n,
+                                        float *stage, float *stage_n, float *nrm_out) {
+    const int tid = threadIdx.x;
+    const int grp = tid / JL, gl = tid % JL;
+    const int r0 = gl * RPL;
+    const int ng = (N + 2 * HC - 1) / (2 * HC);
+    const bool active = grp < ng;
+    const bool warp_active = (tid & ~31) / JL < ng;     // the warp's first group is active
+    float xa[HC][RPL], xb[HC][RPL], na[HC], nb[HC];
+#pragma unroll
+    for (int j = 0; j < HC; ++j) {
+        const int ca = grp * HC + j, cb = (grp + ng) * HC + j;
+        const float *pa = (active && ca < N) ? (ca < k ? sC + ca * LDS : sB + (ca - k) * LDS) : nullptr;
+        const float *pb = (active && cb < N) ? (cb < k ? sC + cb * LDS : sB + (cb - k) * LDS) : nullptr;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            const int row = r0 + i;
+            xa[j][i] = (pa != nullptr && row < n) ? pa[row] : 0.f;
+            xb[j][i] = (pb != nullptr && row < n) ? pb[row] : 0.f;
+        }
+    }
+    __syncthreads();                          // inputs consumed: the staging area is free
+    const int destA = grp == 0 ? 0 : (grp < ng - 1 ? grp + 1 : 2 * ng - 1);
+    const int destB = grp == 0 ? 1 : ng + grp - 1;
+    int sweeps = 0;
+    bool converged = false;
+    while (sweeps < JACOBI_MAX_SWEEPS) {
+        ++sweeps;
+        int rotated = 0;
+        if (warp_active) {
+#pragma unroll
+            for (int j = 0; j < HC; ++j) {
+                float sa = 0.f, sb = 0.f;
+#pragma unroll
+                for (int i = 0; i < RPL; ++i) {
+                    sa = fmaf(xa[j][i], xa[j][i], sa);
+                    sb = fmaf(xb[j][i], xb[j][i], sb);
                 }
-                __syncwarp();
-                if (pass == 0) {
-                    for (int c = lane; c < k; c += 32) {
-                        const float *bc = sC + c * LDS;
-                        float s = 0.f;
-                        for (int j = 0; j < D; ++j) s = fmaf(f[j], bc[j], s);
-                        scr[c] = s;
+                na[j] = group_sum(sa);
+                nb[j] = group_sum(sb);
+            }
+        }
+#pragma unroll 1
+        for (int round = 0; round < 2 * ng - 1; ++round) {
+            if (warp_active) {
+                if (round == 0) {
+#pragma unroll
+                    for (int j1 = 0; j1 < HC; ++j1)
+#pragma unroll
+                        for (int j2 = j1 + 1; j2 < HC; ++j2) {
+                            jrot<RPL>(xa[j1], xa[j2], na[j1], na[j2], rotated);
+                            jrot<RPL>(xb[j1], xb[j2], nb[j1], nb[j2], rotated);
+                        }
+                }
+                JCrossAll<HC, RPL, 0>::run(xa, xb, na, nb, rotated);
+            }
+            if (ng > 1) {                     // move the slots for the next round
+                if (active) {
+#pragma unroll
+                    for (int j = 0; j < HC; ++j) {
+                        float *da = stage + (destA * HC + j) * SS + r0;
+                        float *db = stage + (destB * HC + j) * SS + r0;
+#pragma unroll
+                        for (int i = 0; i < RPL; ++i) {
+                            da[i] = xa[j][i];
+                            db[i] = xb[j][i];
+                        }
+                        if (gl == 0) {
+                            stage_n[destA * HC + j] = na[j];
+                            stage_n[destB * HC + j] = nb[j];
+                        }
                     }
-                    __syncwarp();
+                }
+                __syncthreads();
+                if (active) {
+#pragma unroll
+                    for (int j = 0; j < HC; ++j) {
+                        const float *sa = stage + (grp * HC + j) * SS + r0;
+                        const float *sb = stage + ((ng + grp) * HC + j) * SS + r0;
+#pragma unroll
+                        for (int i = 0; i < RPL; ++i) {
+                            xa[j][i] = sa[i];
+                            xb[j][i] = sb[i];
+                        }
+                        na[j] = stage_n[grp * HC + j];
+                        nb[j] = stage_n[(ng + grp) * HC + j];
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        if (__syncthreads_or(rotated) == 0) {
+            converged = true;
+            break;
+        }
+    }
+    // final columns (position order) and their exact norms
+    if (warp_active) {
+#pragma unroll
+        for (int j = 0; j < HC; ++j) {
+            float sa = 0.f, sb = 0.f;
+#pragma unroll
+            for (int i = 0; i < RPL; ++i) {
+                sa = fmaf(xa[j][i], xa[j][i], sa);
+                sb = fmaf(xb[j][i], xb[j][i], sb);
+            }
+            sa = group_sum(sa);
+            sb = group_sum(sb);
+            if (active) {
+                float *da = stage + (grp * HC + j) * SS + r0;
+                float *db = stage + ((ng + grp) * HC + j) * SS + r0;
+#pragma unroll
+                for (int i = 0; i < RPL; ++i) {
+                    da[i] = xa[j][i];
+                    db[i] = xb[j][i];
+                }
+                if (gl == 0) {
+                    nrm_out[grp * HC + j] = sqrtf(sa);
+                    nrm_out[(ng + grp) * HC + j] = sqrtf(sb);
                 }
             }
         }
     }
     __syncthreads();
+    return converged ? sweeps : -sweeps;
+}
+
+__global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
+    extern __shared__ float smem[];
+    float *sA = smem + OFF_A;
+    float *sB = smem + OFF_B;
+    float *sC = smem + OFF_C;
+    float *sTau = smem + OFF_TAU;
+    float *sSig = smem + OFF_SIG;
+    float *sNrm = smem + OFF_NRM;
+    float *sSN = smem + OFF_SNRM;
+    float *sScr = smem + OFF_SCR;
+    int *sSel = reinterpret_cast<int *>(smem + OFF_INT);
+    float *stage = sB;                    // Jacobi staging overlays B and C
+
+    const FoldPath P = blockIdx.y ? a.path[1] : a.path[0];
+    const int unit = a.unit0 + blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int k = P.k, r = P.r, p = P.p, kp = P.kp, b = a.b;
+    const int n = k + p;                  // rows of Z^T (columns of Z)
+    const int N = k + b;                  // columns of Z^T
+    const size_t ring_base = (size_t)unit * a.R * D;
+    const float *Bin = P.basis_in + (size_t)unit * D * r;
+
+    // ---- load F (b x D) from the exact window ring, B (as k columns) and Sigma ---------------
+    auto load_F = [&]() {
+        if (a.kv_dtype == ISKV_BF16) {
+            const __nv_bfloat16 *ring = reinterpret_cast<const __nv_bfloat16 *>(P.ring);
+            const int nv = b * (D / 8);
+            for (int v0 = tid; v0 < nv; v0 += 4 * FT) {
+                uint4 u[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int v = v0 + q * FT;
+                    if (v < nv) {
+                        const int i = v >> 4, j8 = (v & 15) * 8;
+                        const int slot = (a.slot0 + i) % a.R;
+                        u[q] = *reinterpret_cast<const uint4 *>(ring + ring_base + (size_t)slot * D + j8);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int v = v0 + q * FT;
+                    if (v < nv) {
+                        const int i = v >> 4, j8 = (v & 15) * 8;
+                        const uint32_t w[4] = {u[q].x, u[q].y, u[q].z, u[q].w};
+                        float *dst = sA + i * LDS + j8;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            dst[2 * e] = __uint_as_float(w[e] << 16);
+                            dst[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+                        }
+                    }
+                }
+            }
+        } else {
+            const float *ring = reinterpret_cast<const float *>(P.ring);
+            const int nv = b * (D / 4);
+            for (int v0 = tid; v0 < nv; v0 += 4 * FT) {
+                float4 u[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int v = v0 + q * FT;
+                    if (v < nv) {
+                        const int i = v >> 5, j4 = (v & 31) * 4;
+                        const int slot = (a.slot0 + i) % a.R;
+                        u[q] = *reinterpret_cast<const float4 *>(ring + ring_base + (size_t)slot * D + j4);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int v = v0 + q * FT;
+                    if (v < nv) {
+                        const int i = v >> 5, j4 = (v & 31) * 4;
+                        float *dst = sA + i * LDS + j4;
+                        dst[0] = u[q].x;
+                        dst[1] = u[q].y;
+                        dst[2] = u[q].z;
+                        dst[3] = u[q].w;
+                    }
+                }
+            }
+        }
+    };
+    load_F();
+    for (int o0 = tid; o0 < D * k; o0 += 4 * FT) {
+        float v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int o = o0 + q * FT;
+            v[q] = o < D * k ? Bin[(size_t)(o / k) * r + o % k] : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int o = o0 + q * FT;
+            if (o < D * k) sC[(o % k) * LDS + o / k] = v[q];
+        }
+    }
+    if (tid < k) sSig[tid] = P.sigma[(size_t)unit * r + tid];
+    __syncthreads();
+
+    // ---- step 1: S = F B (into Y[:, :k]) and the residual E = F - S B^T (in place) -----------
+    if (k > 0) {
+        for (int o = tid; o < b * k; o += FT) {
+            const int i = o / k, c = o % k;
+            const float *f = sA + i * LDS, *bc = sC + c * LDS;
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll 4
+            for (int j = 0; j < D; j += 4) {
+                s0 = fmaf(f[j], bc[j], s0);
+                s1 = fmaf(f[j + 1], bc[j + 1], s1);
+                s2 = fmaf(f[j + 2], bc[j + 2], s2);
+                s3 = fmaf(f[j + 3], bc[j + 3], s3);
+            }
+            sB[i * LDS + c] = (s0 + s1) + (s2 + s3);
+        }
+        __syncthreads();
+        for (int o = tid; o < b * D; o += FT) {
+            const int i = o / D, j = o % D;
+            const float *srow = sB + i * LDS;
+            float e0 = sA[i * LDS + j], e1 = 0.f;
+            int c = 0;
+            for (; c + 1 < k; c += 2) {
+                e0 = fmaf(-srow[c], sC[c * LDS + j], e0);
+                e1 = fmaf(-srow[c + 1], sC[(c + 1) * LDS + j], e1);
+            }
+            if (c < k) e0 = fmaf(-srow[c], sC[c * LDS + j], e0);
+            sA[i * LDS + j] = e0 + e1;
+        }
+        __syncthreads();
+    }
 
     // ---- residual basis: Householder QR of [B, E^T(rows 0..p-1)] (D x n, columns in sC) ------
-    for (int o = tid; o < p * D; o += FOLD_THREADS) {
+    for (int o = tid; o < p * D; o += FT) {
         const int i = o / D, j = o % D;
         sC[(k + i) * LDS + j] = sA[i * LDS + j];
     }
@@ -125,8 +420,13 @@ __global__ void __launch_bounds__(FOLD_THREADS, 1) fold_core_kernel(FoldArgs a) 
     for (int jc = 0; jc < n; ++jc) {
         float *col = sC + jc * LDS;
         if (warp == 0) {
-            float s2 = 0.f;
-            for (int i = jc + 1 + lane; i < D; i += 32) s2 = fmaf(col[i], col[i], s2);
+            float xv[4], s2 = 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = lane + 32 * u;
+                xv[u] = col[i];
+                s2 = fmaf(i > jc ? xv[u] : 0.f, xv[u], s2);
+            }
             s2 = warp_sum(s2);
             const float alpha = col[jc];
             float tau = 0.f, beta = alpha, scale = 0.f;
@@ -136,7 +436,11 @@ __global__ void __launch_bounds__(FOLD_THREADS, 1) fold_core_kernel(FoldArgs a) 
                 scale = 1.f / (alpha - beta);
             }
             __syncwarp();
-            for (int i = jc + 1 + lane; i < D; i += 32) col[i] *= scale;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = lane + 32 * u;
+                if (i > jc) col[i] = xv[u] * scale;
+            }
             if (lane == 0) {
                 col[jc] = beta;
                 sTau[jc] = tau;
@@ -145,143 +449,164 @@ __global__ void __launch_bounds__(FOLD_THREADS, 1) fold_core_kernel(FoldArgs a) 
         __syncthreads();
         const float tau = sTau[jc];
         if (tau != 0.f) {
-            for (int c = jc + 1 + warp; c < n; c += FOLD_WARPS) {
-                float *x = sC + c * LDS;
-                float w = 0.f;
-                for (int i = jc + 1 + lane; i < D; i += 32) w = fmaf(col[i], x[i], w);
-                w = (warp_sum(w) + x[jc]) * tau;
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = lane + 32 * u;
+                v[u] = i > jc ? col[i] : 0.f;
+            }
+            // trailing columns c = jc + 1 + warp + FW m, eight per batch (overlapped reductions)
+            for (int cb = jc + 1 + warp; cb < n; cb += 8 * FW) {
+                float w[8], xq[8][4];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int c = min(cb + q * FW, n - 1);
+                    const float *x = sC + c * LDS;
+                    w[q] = 0.f;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        xq[q][u] = x[lane + 32 * u];
+                        w[q] = fmaf(v[u], xq[q][u], w[q]);
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) w[q] += __shfl_xor_sync(0xffffffffu, w[q], o);
+                float xj[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) xj[q] = sC[min(cb + q * FW, n - 1) * LDS + jc];
                 __syncwarp();
-                if (lane == 0) x[jc] -= w;
-                for (int i = jc + 1 + lane; i < D; i += 32) x[i] = fmaf(-w, col[i], x[i]);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int c = cb + q * FW;
+                    if (c < n) {
+                        float *x = sC + c * LDS;
+                        const float wq = (w[q] + xj[q]) * tau;
+                        if (lane == 0) x[jc] = xj[q] - wq;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int i = lane + 32 * u;
+                            if (i > jc) x[i] = fmaf(-wq, v[u], xq[q][u]);
+                        }
+                    }
+                }
+                __syncwarp();
             }
         }
         __syncthreads();
     }
 
     // ---- T = F P for the rows in the QR: T[i][l] = R[k+l][k+i] (l <= i) ----------------------
-    for (int o = tid; o < p * p; o += FOLD_THREADS) {
+    for (int o = tid; o < p * p; o += FT) {
         const int i = o / p, l = o % p;
         sB[i * LDS + k + l] = (l <= i) ? sC[(k + i) * LDS + k + l] : 0.f;
     }
     // ---- P = Q[:, k:k+p] into sA columns 0..p-1 (over E rows 0..p-1, no longer needed) -------
-    for (int l = warp; l < p; l += FOLD_WARPS) {
-        float *x = sA + l * LDS;
-        for (int i = lane; i < D; i += 32) x[i] = (i == k + l) ? 1.f : 0.f;
-        __syncwarp();
-        for (int jc = min(n - 1, k + l); jc >= 0; --jc) {
+    //      warp w builds columns l = w + FW q, eight at a time (overlapped reductions)
+    for (int lb = warp; lb < p; lb += 8 * FW) {
+        float xr[8][4];
+        int lmax = lb;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int l = lb + q * FW;
+            if (l < p) lmax = l;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) xr[q][u] = (lane + 32 * u == k + l) ? 1.f : 0.f;
+        }
+        for (int jc = min(n - 1, k + lmax); jc >= 0; --jc) {
             const float tau = sTau[jc];
             if (tau == 0.f) continue;
             const float *v = sC + jc * LDS;
-            float w = 0.f;
-            for (int i = jc + 1 + lane; i < D; i += 32) w = fmaf(v[i], x[i], w);
-            w = (warp_sum(w) + x[jc]) * tau;
-            __syncwarp();
-            if (lane == 0) x[jc] -= w;
-            for (int i = jc + 1 + lane; i < D; i += 32) x[i] = fmaf(-w, v[i], x[i]);
-            __syncwarp();
+            float vv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = lane + 32 * u;
+                vv[u] = i > jc ? v[i] : (i == jc ? 1.f : 0.f);
+            }
+            float w[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                w[q] = 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) w[q] = fmaf(vv[u], xr[q][u], w[q]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) w[q] += __shfl_xor_sync(0xffffffffu, w[q], o);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) xr[q][u] = fmaf(-w[q] * tau, vv[u], xr[q][u]);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int l = lb + q * FW;
+            if (l < p)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) sA[l * LDS + lane + 32 * u] = xr[q][u];
         }
     }
     __syncthreads();
     // ---- rows that did not enter the QR (p < b): T[i] = E[i] P ---------------------------------
-    for (int o = tid; o < (b - p) * p; o += FOLD_THREADS) {
+    for (int o = tid; o < (b - p) * p; o += FT) {
         const int i = p + o / p, l = o % p;
         const float *e = sA + i * LDS, *pc = sA + l * LDS;
-        float s = 0.f;
-        for (int j = 0; j < D; ++j) s = fmaf(e[j], pc[j], s);
-        sB[i * LDS + k + l] = s;
+        float s0 = 0.f, s1 = 0.f;
+        for (int j = 0; j < D; j += 2) {
+            s0 = fmaf(e[j], pc[j], s0);
+            s1 = fmaf(e[j + 1], pc[j + 1], s1);
+        }
+        sB[i * LDS + k + l] = s0 + s1;
     }
     // ---- Z^T columns 0..k-1: Sigma_c e_c (length n) -------------------------------------------
-    for (int o = tid; o < k * n; o += FOLD_THREADS) {
+    for (int o = tid; o < k * n; o += FT) {
         const int c = o / n, m = o % n;
         sC[c * LDS + m] = (m == c) ? sSig[c] : 0.f;
     }
     __syncthreads();
 
-    // ---- one-sided Jacobi on the N columns (length n) of Z^T ----------------------------------
+    // ---- one-sided Jacobi on the N columns (length n) of Z^T, register resident --------------
+    int sweeps;
+    const int HC = N <= 96 ? 3 : (N <= 128 ? 4 : 8);
     {
-        const int Np = N + (N & 1);
-        const int gid = tid / JG, gl = tid % JG;
-        const unsigned gmask = 0xffu << ((lane / JG) * JG);
-        bool converged = false;
-        int sweeps = 0;
-        for (int sweep = 0; sweep < JACOBI_MAX_SWEEPS; ++sweep) {
-            ++sweeps;
-            if (tid == 0) sFlag[0] = 0;
-            __syncthreads();
-            for (int round = 0; round < Np - 1; ++round) {
-                for (int i = gid; i < Np / 2; i += JGROUPS) {
-                    int ca, cb;
-                    rr_pair(Np, round, i, ca, cb);
-                    if (ca >= N || cb >= N) continue;
-                    float *xa = ca < k ? sC + ca * LDS : sB + (ca - k) * LDS;
-                    float *xb = cb < k ? sC + cb * LDS : sB + (cb - k) * LDS;
-                    float al = 0.f, be = 0.f, ga = 0.f;
-                    for (int m = gl; m < n; m += JG) {
-                        const float u = xa[m], v = xb[m];
-                        al = fmaf(u, u, al);
-                        be = fmaf(v, v, be);
-                        ga = fmaf(u, v, ga);
-                    }
-#pragma unroll
-                    for (int o = JG / 2; o > 0; o >>= 1) {
-                        al += __shfl_xor_sync(gmask, al, o);
-                        be += __shfl_xor_sync(gmask, be, o);
-                        ga += __shfl_xor_sync(gmask, ga, o);
-                    }
-                    if (fabsf(ga) > JACOBI_TOL * sqrtf(al) * sqrtf(be)) {
-                        const float zeta = (be - al) / (2.f * ga);
-                        const float az = fabsf(zeta);
-                        const float t = (az > 1e18f ? 0.5f / az : 1.f / (az + sqrtf(fmaf(az, az, 1.f))));
-                        const float tt = zeta < 0.f ? -t : t;
-                        // rotation [[c, s], [-s, c]] with c = 1/rr, s = t/rr applied as a
-                        // correction: dc = 1 - c is formed directly, because for |t| < sqrt(eps)
-                        // c rounds to 1 while s = t, and the rounded rotation would inflate column
-                        // norms by t^2/2 each time (a systematic bias over thousands of rotations)
-                        const float rr = sqrtf(fmaf(tt, tt, 1.f));
-                        const float dc = (tt * tt) / (rr * (1.f + rr));
-                        const float s = tt / rr;
-                        for (int m = gl; m < n; m += JG) {
-                            const float u = xa[m], v = xb[m];
-                            xa[m] = u - fmaf(dc, u, s * v);
-                            xb[m] = v - fmaf(dc, v, -s * u);
-                        }
-                        if (gl == 0 && t != 0.f) sFlag[0] = 1;
-                    }
-                }
-                __syncthreads();
-            }
-            if (sFlag[0] == 0) {
-                converged = true;
-                break;
-            }
-            __syncthreads();
+        const int rpl = n <= 96 ? 6 : (n <= 112 ? 7 : 8);
+        switch (HC * 16 + rpl) {
+            case 3 * 16 + 6: sweeps = jacobi_regs<3, 6>(sB, sC, k, N, n, stage, sSN, sNrm); break;
+            case 3 * 16 + 7: sweeps = jacobi_regs<3, 7>(sB, sC, k, N, n, stage, sSN, sNrm); break;
+            case 3 * 16 + 8: sweeps = jacobi_regs<3, 8>(sB, sC, k, N, n, stage, sSN, sNrm); break;
+            case 4 * 16 + 6: sweeps = jacobi_regs<4, 6>(sB, sC, k, N, n, stage, sSN, sNrm); break;
+            case 4 * 16 + 7: sweeps = jacobi_regs<4, 7>(sB, sC, k, N, n, stage, sSN, sNrm); break;
+            case 4 * 16 + 8: sweeps = jacobi_regs<4, 8>(sB, sC, k, N, n, stage, sSN, sNrm); break;
+            case 8 * 16 + 6: sweeps = jacobi_regs<8, 6>(sB, sC, k, N, n, stage, sSN, sNrm); break;
+            case 8 * 16 + 7: sweeps = jacobi_regs<8, 7>(sB, sC, k, N, n, stage, sSN, sNrm); break;
+            default: sweeps = jacobi_regs<8, 8>(sB, sC, k, N, n, stage, sSN, sNrm); break;
         }
-        if (!converged && tid == 0) set_status(a.status, ISKV_ERR_NOT_CONVERGED);
-        if (tid == 0 && a.stats) {
-            atomicMax(a.stats, (unsigned long long)sweeps);
-            atomicAdd(a.stats + 1, (unsigned long long)sweeps);
+    }
+    const int NC = 2 * ((N + 2 * HC - 1) / (2 * HC)) * HC;   // staged columns (NC - N zero)
+    if (tid == 0) {
+        if (sweeps < 0) set_status(a.status, ISKV_ERR_NOT_CONVERGED);
+        if (a.stats) {
+            const unsigned long long sw = (unsigned long long)(sweeps < 0 ? -sweeps : sweeps);
+            atomicMax(a.stats, sw);
+            atomicAdd(a.stats + 1, sw);
             atomicAdd(a.stats + 2, 1ull);
         }
     }
 
     // ---- singular values = column norms; select the top kp (descending, ties by index) -------
-    for (int c = tid; c < N; c += FOLD_THREADS) {
-        const float *x = c < k ? sC + c * LDS : sB + (c - k) * LDS;
-        float s = 0.f;
-        for (int m = 0; m < n; ++m) s = fmaf(x[m], x[m], s);
-        s = sqrtf(s);
-        if (!isfinite(s)) {
+    for (int c = tid; c < NC; c += FT) {
+        if (!isfinite(sNrm[c])) {
             set_status(a.status, ISKV_ERR_NONFINITE);
-            s = -1.f;
+            sNrm[c] = -1.f;
         }
-        sNrm[c] = s;
     }
-    if (tid < 128) sSel[tid] = 0;
     __syncthreads();
-    for (int c = tid; c < N; c += FOLD_THREADS) {
+    for (int c = tid; c < NC; c += FT) {
         const float s = sNrm[c];
         int rank = 0;
-        for (int c2 = 0; c2 < N; ++c2) {
+        for (int c2 = 0; c2 < NC; ++c2) {
             const float s2 = sNrm[c2];
             rank += (s2 > s) || (s2 == s && c2 < c);
         }
@@ -289,29 +614,27 @@ __global__ void __launch_bounds__(FOLD_THREADS, 1) fold_core_kernel(FoldArgs a) 
     }
     __syncthreads();
     // normalise the selected columns in place: they become the columns of H (length n)
-    for (int o = tid; o < kp * n; o += FOLD_THREADS) {
+    for (int o = tid; o < kp * n; o += FT) {
         const int c = o / n, m = o % n;
         const int cs = sSel[c];
         const float s = sNrm[cs];
-        float *x = cs < k ? sC + cs * LDS : sB + (cs - k) * LDS;
-        if (s > 1e-30f) x[m] = x[m] / s;
+        if (s > 1e-30f) stage[cs * SS + m] /= s;
     }
     __syncthreads();
-    // exactly-zero singular values: complete H with orthonormal directions (rare; rank-deficient
-    // input); keeps B+ orthonormal
+    // exactly-zero singular values: complete H with orthonormal directions (rank-deficient input)
     if (warp == 0) {
         float *v = sScr;
         for (int c = 0; c < kp; ++c) {
             const int cs = sSel[c];
             if (sNrm[cs] > 1e-30f) continue;
-            float *x = cs < k ? sC + cs * LDS : sB + (cs - k) * LDS;
+            float *x = stage + cs * SS;
             for (int e = 0; e < n; ++e) {
                 for (int m = lane; m < n; m += 32) v[m] = (m == e) ? 1.f : 0.f;
                 __syncwarp();
                 for (int c2 = 0; c2 < kp; ++c2) {
                     const int cs2 = sSel[c2];
                     if (c2 == c || (sNrm[cs2] <= 1e-30f && c2 > c)) continue;
-                    const float *y = cs2 < k ? sC + cs2 * LDS : sB + (cs2 - k) * LDS;
+                    const float *y = stage + cs2 * SS;
                     float d = 0.f;
                     for (int m = lane; m < n; m += 32) d = fmaf(y[m], v[m], d);
                     d = warp_sum(d);
@@ -333,118 +656,121 @@ __global__ void __launch_bounds__(FOLD_THREADS, 1) fold_core_kernel(FoldArgs a) 
         }
     }
     // ---- W = [P | B_old] as columns of sA (B_old at columns p .. p+k-1) ------------------------
-    for (int o = tid; o < D * k; o += FOLD_THREADS) {
-        const int j = o / k, l = o % k;
-        sA[(p + l) * LDS + j] = Bin[(size_t)j * r + l];
+    for (int o0 = tid; o0 < D * k; o0 += 4 * FT) {
+        float v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int o = o0 + q * FT;
+            v[q] = o < D * k ? Bin[(size_t)(o / k) * r + o % k] : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int o = o0 + q * FT;
+            if (o < D * k) sA[(p + o % k) * LDS + o / k] = v[q];
+        }
     }
     __syncthreads();
     // ---- sign convention: new basis vector c points along old basis vector c (H[c][c] >= 0) ----
-    const int ks = k < kp ? k : kp;
-    for (int c = tid; c < ks; c += FOLD_THREADS) {
-        const int cs = sSel[c];
-        const float *x = cs < k ? sC + cs * LDS : sB + (cs - k) * LDS;
-        sTau[c] = x[c] < 0.f ? -1.f : 1.f;
-    }
+    const int ksg = k < kp ? k : kp;
+    for (int c = tid; c < ksg; c += FT) sTau[c] = stage[sSel[c] * SS + c] < 0.f ? -1.f : 1.f;
     __syncthreads();
-    for (int o = tid; o < ks * n; o += FOLD_THREADS) {
+    for (int o = tid; o < ksg * n; o += FT) {
         const int c = o / n, m = o % n;
-        if (sTau[c] < 0.f) {
-            const int cs = sSel[c];
-            float *x = cs < k ? sC + cs * LDS : sB + (cs - k) * LDS;
-            x[m] = -x[m];
-        }
+        if (sTau[c] < 0.f) stage[sSel[c] * SS + m] = -stage[sSel[c] * SS + m];
     }
     __syncthreads();
 
     // ---- outputs: Sigma+, H_top, B+ = [B P] H ------------------------------------------------
     float *sig_out = P.sigma + (size_t)unit * r;
-    for (int c = tid; c < r; c += FOLD_THREADS) sig_out[c] = c < kp ? sNrm[sSel[c]] : 0.f;
+    for (int c = tid; c < r; c += FT) sig_out[c] = c < kp ? sNrm[sSel[c]] : 0.f;
     float *ht = P.htop + (size_t)unit * r * r;
-    for (int o = tid; o < k * kp; o += FOLD_THREADS) {
+    for (int o = tid; o < k * kp; o += FT) {
         const int l = o / kp, c = o % kp;
-        const int cs = sSel[c];
-        const float *x = cs < k ? sC + cs * LDS : sB + (cs - k) * LDS;
-        ht[(size_t)l * r + c] = x[l];
+        ht[(size_t)l * r + c] = stage[sSel[c] * SS + l];
     }
+    float *Bout = P.basis_out + (size_t)unit * D * r;
     const int j = tid & (D - 1);
-    const int c0 = tid >> 7;             // 0..3
-    float bp[32];
+    const int c0 = tid >> 7;               // 0..1
+    for (int cb = 0; cb < r; cb += 64) {
+        float bp[32];
 #pragma unroll
-    for (int q = 0; q < 32; ++q) {
-        const int c = c0 + 4 * q;
-        float s = 0.f;
-        if (c < kp) {
-            const int cs = sSel[c];
-            const float *h = cs < k ? sC + cs * LDS : sB + (cs - k) * LDS;
-            for (int l = 0; l < p; ++l) s = fmaf(sA[l * LDS + j], h[k + l], s);
-            for (int l = 0; l < k; ++l) s = fmaf(sA[(p + l) * LDS + j], h[l], s);
+        for (int q = 0; q < 32; ++q) {
+            const int c = cb + c0 + 2 * q;
+            float s0 = 0.f, s1 = 0.f;
+            if (c < kp) {
+                const float *hv = stage + sSel[c] * SS;
+                int l = 0;
+                for (; l + 1 < p; l += 2) {
+                    s0 = fmaf(sA[l * LDS + j], hv[k + l], s0);
+                    s1 = fmaf(sA[(l + 1) * LDS + j], hv[k + l + 1], s1);
+                }
+                if (l < p) s0 = fmaf(sA[l * LDS + j], hv[k + l], s0);
+                for (l = 0; l + 1 < k; l += 2) {
+                    s0 = fmaf(sA[(p + l) * LDS + j], hv[l], s0);
+                    s1 = fmaf(sA[(p + l + 1) * LDS + j], hv[l + 1], s1);
+                }
+                if (l < k) s0 = fmaf(sA[(p + l) * LDS + j], hv[l], s0);
+            }
+            bp[q] = s0 + s1;
         }
-        bp[q] = s;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const int c = cb + c0 + 2 * q;
+            if (c < r) Bout[(size_t)j * r + c] = bp[q];
+        }
     }
-    __syncthreads();                     // H and W consumed
+    __syncthreads();                       // H, W consumed; B+ (uncorrected) and H_top written
     // ---- one Newton-Schulz step towards the nearest orthonormal basis, B+ <- B+ (3I - M) / 2 with
     //      M = B+^T B+ (the Jacobi stops at a relative orthogonality threshold, and without this
     //      the loss of orthonormality would add up over folds); H_top gets the same right factor so
     //      old coordinates stay consistent with the corrected basis.
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-        const int c = c0 + 4 * q;
-        if (c < kp) sC[c * LDS + j] = bp[q];
-    }
+    float *sBp = sC;                       // B+ columns [kp][LDS]
+    float *sM = sB;                        // M [kp][kp]
+    float *sH = sA;                        // H_top [k][kp]
+    for (int o = tid; o < D * kp; o += FT) sBp[(o % kp) * LDS + o / kp] = Bout[(size_t)(o / kp) * r + o % kp];
+    for (int o = tid; o < k * kp; o += FT) sH[o] = ht[(size_t)(o / kp) * r + o % kp];
     __syncthreads();
-    for (int o = tid; o < kp * kp; o += FOLD_THREADS) {
+    for (int o = tid; o < kp * kp; o += FT) {
         const int c = o / kp, c2 = o % kp;
-        const float *x = sC + c * LDS, *y = sC + c2 * LDS;
-        float s = 0.f;
-        for (int jj = 0; jj < D; ++jj) s = fmaf(x[jj], y[jj], s);
-        sB[o] = s;
-    }
-    for (int o = tid; o < k * kp; o += FOLD_THREADS) sA[o] = ht[(size_t)(o / kp) * r + o % kp];
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-        const int c = c0 + 4 * q;
-        if (c < kp) {
-            float s = 0.f;
-            for (int c2 = 0; c2 < kp; ++c2) s = fmaf(sC[c2 * LDS + j], sB[c2 * kp + c], s);
-            bp[q] = 1.5f * bp[q] - 0.5f * s;
+        const float *x = sBp + c * LDS, *y = sBp + c2 * LDS;
+        float s0 = 0.f, s1 = 0.f;
+        for (int jj = 0; jj < D; jj += 2) {
+            s0 = fmaf(x[jj], y[jj], s0);
+            s1 = fmaf(x[jj + 1], y[jj + 1], s1);
         }
+        sM[o] = s0 + s1;
     }
-    for (int o = tid; o < k * kp; o += FOLD_THREADS) {
+    __syncthreads();
+    for (int o = tid; o < D * kp; o += FT) {
+        const int c = o / D, jj = o % D;
+        float s = 0.f;
+        for (int c2 = 0; c2 < kp; ++c2) s = fmaf(sBp[c2 * LDS + jj], sM[c2 * kp + c], s);
+        Bout[(size_t)jj * r + c] = 1.5f * sBp[c * LDS + jj] - 0.5f * s;
+    }
+    for (int o = tid; o < k * kp; o += FT) {
         const int l = o / kp, c = o % kp;
         float s = 0.f;
-        for (int c2 = 0; c2 < kp; ++c2) s = fmaf(sA[l * kp + c2], sB[c2 * kp + c], s);
-        ht[(size_t)l * r + c] = 1.5f * sA[o] - 0.5f * s;
-    }
-    float *Bout = P.basis_out + (size_t)unit * D * r;
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-        const int c = c0 + 4 * q;
-        if (c < r) Bout[(size_t)j * r + c] = bp[q];
+        for (int c2 = 0; c2 < kp; ++c2) s = fmaf(sH[l * kp + c2], sM[c2 * kp + c], s);
+        ht[(size_t)l * r + c] = 1.5f * sH[o] - 0.5f * s;
     }
     __syncthreads();
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-        const int c = c0 + 4 * q;
-        if (c < kp) sC[c * LDS + j] = bp[q];
-    }
-    // reload F for the new rows' coordinates
-    for (int o = tid; o < b * D; o += FOLD_THREADS) {
-        const int i = o / D, jj = o % D;
-        const int slot = (a.slot0 + i) % a.R;
-        sA[i * LDS + jj] = load_row_elem(P.ring, ring_base + (size_t)slot * D + jj, a.kv_dtype);
-    }
+    // corrected B+ columns back into shared memory; reload F for the new rows' coordinates
+    for (int o = tid; o < D * kp; o += FT) sBp[(o % kp) * LDS + o / kp] = Bout[(size_t)(o / kp) * r + o % kp];
+    load_F();
     __syncthreads();
     // ---- new rows' coordinates C[n_c + i] = F[i] B+ --------------------------------------------
     float *Cn = P.coords + ((size_t)unit * a.n_max + a.n_c) * r;
-    for (int o = tid; o < b * r; o += FOLD_THREADS) {
+    for (int o = tid; o < b * r; o += FT) {
         const int i = o / r, c = o % r;
-        float s = 0.f;
+        float s0 = 0.f, s1 = 0.f;
         if (c < kp) {
-            const float *f = sA + i * LDS, *bc = sC + c * LDS;
-            for (int jj = 0; jj < D; ++jj) s = fmaf(f[jj], bc[jj], s);
+            const float *f = sA + i * LDS, *bc = sBp + c * LDS;
+            for (int jj = 0; jj < D; jj += 2) {
+                s0 = fmaf(f[jj], bc[jj], s0);
+                s1 = fmaf(f[jj + 1], bc[jj + 1], s1);
+            }
         }
-        Cn[(size_t)i * r + c] = s;
+        Cn[(size_t)i * r + c] = s0 + s1;
     }
 }
 
@@ -499,7 +825,7 @@ cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    fold_core_kernel<<<dim3(n_units, 2), FOLD_THREADS, smem, s>>>(a);
+    fold_core_kernel<<<dim3(n_units, 2), FT, smem, s>>>(a);
     return cudaGetLastError();
 }
 
