@@ -183,6 +183,54 @@ int iskv_schedule(int block, int window, long long t, long long m, long long *n_
  */
 int iskv_sync_status(iskv_handle *h, iskv_stream_t stream);
 
+/*
+ * Decode attention over caller-owned buffers that allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine, no handle). The paper has no counterpart: this entry point exists
+ * for callers that cannot allocate device memory on their decode path - code running inside CUDA
+ * stream capture (cudaMalloc is not capturable), engines whose device memory is entirely owned by
+ * their own pool allocator, and latency-critical loops where cudaMalloc's implicit device
+ * synchronisation is not acceptable.
+ *
+ * The computation is that of iskv_decode_attn() for one layer, on the CUDA-core decode kernels,
+ * with the cache described by `view` instead of a handle. The split partials that
+ * iskv_decode_attn() keeps in handle-owned memory live here in a file-scope device array of
+ * ISKV_NOALLOC_SCRATCH_FLOATS floats (4 MiB) that every GPU which loads the library holds until the
+ * process exits. Required scratch: batch * n_kv_heads * splits * (n_q_heads / n_kv_heads) *
+ * (head_dim + 2) floats, with splits = ceil(n_c / 128) + ceil((t - n_c) / 128) at most; larger
+ * requests return ISKV_ERR_CAPACITY before anything is enqueued.
+ *
+ * All calls share that array and it keeps the last call's contents; nothing in it has to start at
+ * zero (every split writes its partials before the merge reads them). Calls whose work overlaps
+ * on the GPU (different streams, or different host threads) race on the array: order them on one
+ * stream. The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and keeps it; make that first call before any
+ * stream capture.
+ *   view:    cache description (layouts below), all pointers device pointers owned by the caller;
+ *   q_dev:   fp32 [batch][n_q_heads][head_dim], already rotated for the query position;
+ *   out_dev: fp32 [batch][n_q_heads][head_dim].
+ * Errors: ISKV_ERR_INVALID_ARG (NULL pointer, inconsistent sizes), ISKV_ERR_CAPACITY (scratch
+ * too small), ISKV_ERR_CUDA (address lookup or launch failed).
+ */
+#define ISKV_NOALLOC_SCRATCH_FLOATS (1 << 20)
+
+typedef struct {
+    long long n_c;        /* compressed rows per unit (positions 0 .. n_c-1)                   */
+    long long t;          /* tokens: positions 0 .. t-1 are attended (t >= 1)                  */
+    long long n_max;      /* coordinate rows per unit in coords_k / coords_v (>= n_c)          */
+    int batch, n_kv_heads, n_q_heads, head_dim;    /* head_dim must be 128                  */
+    int rank_k, rank_v;   /* row stride of the coordinate arrays = columns of the bases        */
+    int k_k, k_v;         /* ranks in use (1 .. rank) when n_c > 0                             */
+    int ring_rows;        /* R: exact row of position i (n_c <= i < t) sits at slot i mod R   */
+    int kv_dtype;         /* ISKV_BF16 or ISKV_F32 (exact rows)                                */
+    const float *coords_k, *coords_v;  /* [batch*n_kv_heads][n_max][rank] fp32                */
+    const float *basis_k, *basis_v;    /* [batch*n_kv_heads][head_dim][rank] fp32             */
+    const void *ring_k, *ring_v;       /* [batch*n_kv_heads][R][head_dim] kv_dtype, pre-RoPE */
+    const float *rope_cs;              /* [t][head_dim/2] (cos, sin) pairs, or NULL: no RoPE */
+} iskv_decode_view;
+
+int iskv_decode_attn_noalloc(const iskv_decode_view *view, const float *q_dev, float *out_dev,
+                             iskv_stream_t stream);
+
 /* Static description of an error code. */
 const char *iskv_strerror(int code);
 

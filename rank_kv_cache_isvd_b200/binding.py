@@ -20,6 +20,7 @@ __all__ = [
     "iskv_create", "iskv_destroy", "iskv_append_block", "iskv_decode_attn", "iskv_reconstruct",
     "iskv_get_factors", "iskv_num_tokens", "iskv_storage_bytes", "iskv_schedule",
     "iskv_sync_status", "iskv_strerror", "iskv_reset", "iskv_launch_count", "iskv_fold_stats",
+    "iskv_decode_view", "iskv_decode_attn_noalloc", "ISKV_NOALLOC_SCRATCH_FLOATS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libiskv.so")
@@ -55,6 +56,35 @@ class iskv_config(ctypes.Structure):
     ]
 
 
+ISKV_NOALLOC_SCRATCH_FLOATS = 1 << 20
+
+
+class iskv_decode_view(ctypes.Structure):
+    """Cache description for iskv_decode_attn_noalloc (mirrors the C struct)."""
+    _fields_ = [
+        ("n_c", ctypes.c_longlong),
+        ("t", ctypes.c_longlong),
+        ("n_max", ctypes.c_longlong),
+        ("batch", ctypes.c_int),
+        ("n_kv_heads", ctypes.c_int),
+        ("n_q_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("rank_k", ctypes.c_int),
+        ("rank_v", ctypes.c_int),
+        ("k_k", ctypes.c_int),
+        ("k_v", ctypes.c_int),
+        ("ring_rows", ctypes.c_int),
+        ("kv_dtype", ctypes.c_int),
+        ("coords_k", ctypes.c_void_p),
+        ("coords_v", ctypes.c_void_p),
+        ("basis_k", ctypes.c_void_p),
+        ("basis_v", ctypes.c_void_p),
+        ("ring_k", ctypes.c_void_p),
+        ("ring_v", ctypes.c_void_p),
+        ("rope_cs", ctypes.c_void_p),
+    ]
+
+
 class IsKVError(RuntimeError):
     def __init__(self, code: int, what: str = ""):
         self.code = code
@@ -83,6 +113,7 @@ _SIGNATURES = {
     "iskv_launch_count": (_i, [_vp, ctypes.POINTER(_ll)]),
     "iskv_fold_stats": (_i, [_vp, _vp, ctypes.POINTER(_i), ctypes.POINTER(_ll),
                              ctypes.POINTER(_ll)]),
+    "iskv_decode_attn_noalloc": (_i, [ctypes.POINTER(iskv_decode_view), _vp, _vp, _vp]),
 }
 
 
@@ -203,6 +234,11 @@ def iskv_fold_stats(handle, stream=None):
     code = lib.iskv_fold_stats(handle, _stream(stream), ctypes.byref(m), ctypes.byref(t),
                                ctypes.byref(c))
     return code, m.value, t.value, c.value
+
+
+def iskv_decode_attn_noalloc(view: iskv_decode_view, q, out, stream=None) -> int:
+    return lib.iskv_decode_attn_noalloc(None if view is None else ctypes.byref(view), _ptr(q),
+                                        _ptr(out), _stream(stream))
 
 
 def iskv_sync_status(handle, stream=None) -> int:

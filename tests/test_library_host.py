@@ -87,3 +87,26 @@ def test_create_without_gpu_fails_cleanly():
         pytest.skip("a GPU is visible")
     code, h = iskv.iskv_create(_cfg())
     assert code == iskv.ISKV_ERR_CUDA and h == 0
+
+
+def _view(**kw):
+    base = dict(n_c=0, t=8192, n_max=0, batch=8, n_kv_heads=8, n_q_heads=32, head_dim=128,
+                rank_k=32, rank_v=48, k_k=0, k_v=0, ring_rows=8192, kv_dtype=iskv.ISKV_BF16)
+    base.update(kw)
+    return iskv.iskv_decode_view(**base)
+
+
+def test_no_alloc_decode_refuses_oversize_requests_before_any_cuda_call():
+    # 64 window splits x 64 kv-heads x GQA 4 x 130 floats > the fixed scratch: refused on the host
+    # (the pointers are never read: the size check comes first)
+    need = 8 * 8 * (8192 // 128) * 4 * 130
+    assert need > iskv.ISKV_NOALLOC_SCRATCH_FLOATS
+    v = _view(ring_k=256, ring_v=256)
+    assert iskv.iskv_decode_attn_noalloc(v, 256, 256) == iskv.ISKV_ERR_CAPACITY
+    assert iskv.iskv_decode_attn_noalloc(None, 256, 256) == iskv.ISKV_ERR_INVALID_ARG
+    assert iskv.iskv_decode_attn_noalloc(_view(), 256, 256) == iskv.ISKV_ERR_INVALID_ARG  # no ring
+    assert iskv.iskv_decode_attn_noalloc(_view(head_dim=64, ring_k=256, ring_v=256), 256,
+                                         256) == iskv.ISKV_ERR_INVALID_ARG
+    assert iskv.iskv_decode_attn_noalloc(_view(n_c=128, t=200, n_max=128, ring_rows=72,
+                                               ring_k=256, ring_v=256), 256,
+                                         256) == iskv.ISKV_ERR_INVALID_ARG  # n_c > 0, no factors
