@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--sample-every", type=int, default=16,
                    help="decode calls between event-timed samples inside the graph")
+    p.add_argument("--profile-case", action="store_true",
+                   help="run the short program used for profiler captures instead of the bench")
     return p.parse_args()
 
 
@@ -394,8 +396,36 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         print(json.dumps(out), flush=True)
 
 
+def run_profile_case():
+    """Short program for profiler captures of the bench workload's kernels with few launches
+    before them: one bulk append of all 4096 tokens (60 folds per head and path, each followed by
+    the history rotation), then three decode calls at t = 4096."""
+    import torch
+
+    from rank_kv_cache_isvd_b200.cache import IsKVCache
+    T, H, QH = WL.tokens, WL.n_kv_heads, WL.n_q_heads
+    kd, vd, q = workload_inputs(seq=0)
+    K = torch.from_numpy(kd.view(np.int16)).cuda().view(torch.bfloat16)[:, 0].transpose(0, 1)
+    V = torch.from_numpy(vd.view(np.int16)).cuda().view(torch.bfloat16)[:, 0].transpose(0, 1)
+    Q = torch.from_numpy(q[T - 1]).cuda()
+    cache = IsKVCache(batch=1, n_layers=1, n_kv_heads=H, n_q_heads=QH, rank_k=WL.rank_k,
+                      rank_v=WL.rank_v, block=WL.block, window=WL.window, max_tokens=T,
+                      kv_dtype="bf16", rope=True, rope_theta=WL.rope_theta)
+    cache.append(0, K.contiguous()[None], V.contiguous()[None])
+    for _ in range(3):
+        out = cache.decode(0, Q)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": WL.name, "tokens": cache.tokens(0),
+                      "status": cache.status(), "launches": cache.launches(),
+                      "out_norm": float(out.norm())}))
+    cache.close()
+
+
 def main():
     args = parse()
+    if args.profile_case:
+        run_profile_case()
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
