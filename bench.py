@@ -6,10 +6,14 @@ r_K=32, r_V=48, RoPE theta=5e5, bf16 rows, batch 1 per GPU).
 One step = one pass of the whole hot path over one sequence batch: for each of the 4096 tokens,
 append its K/V rows (window append, and a block-incremental fold of every path whenever the window
 releases a block: 60 folds x 8 heads x 2 paths = 960 head-block updates) and run decode attention
-of the 32 q-heads over the compressed history plus the exact window. The step's C-ABI calls are
-captured once into a CUDA graph and replayed; inputs (rows and queries of all 4096 tokens) are
-resident in HBM when the timed region starts; L2 is flushed (256 MiB write) before every timed
-step.
+of the 32 q-heads over the compressed history plus the exact window. Folds start on an internal
+stream as soon as their block is complete and join the decode stream when the window releases the
+block (every decode sees the same state as with folds at the trigger); the four folds of blocks
+still inside the window at the end of the stream are joined at the end of the step. The step's
+C-ABI calls are captured once into a CUDA graph and replayed; inputs (rows and queries of all 4096
+tokens) are resident in HBM when the timed region starts; L2 is flushed (256 MiB write) before
+every timed step. The fold throughput is timed separately: one append of all 4096 rows, whose 60
+folds then run back to back on the caller's stream.
 
 ``--impl reference`` times the float64 CPU oracle on a bounded sample of the same workload.
 Multi-GPU (torchrun): every rank streams its own independent sequence batch (weak scaling, no
@@ -76,21 +80,23 @@ def workload_inputs(seq: int):
     return kd, vd, q
 
 
-def decode_bytes(t: int) -> int:
-    """Algorithmic bytes of one decode call at t tokens (all kv-heads of the layer): fp32
-    coordinates of the compressed rows, bf16 window rows (K and V), fp32 bases, q and out."""
-    n = WL.n_c(t)
+def decode_bytes(t: int, wl=None) -> int:
+    """Algorithmic bytes of one decode call at t tokens (all sequences and kv-heads of the
+    layer): fp32 coordinates of the compressed rows, bf16 window rows (K and V), fp32 bases, q and
+    out."""
+    wl = WL if wl is None else wl
+    n = wl.n_c(t)
     e = t - n
     kK = kV = 0
     if n:
-        f = n // WL.block
+        f = n // wl.block
         k = [0, 0]
         for _ in range(f):
-            for x, r in ((0, WL.rank_k), (1, WL.rank_v)):
-                k[x] = min(r, k[x] + min(WL.block, D - k[x]))
+            for x, r in ((0, wl.rank_k), (1, wl.rank_v)):
+                k[x] = min(r, k[x] + min(wl.block, D - k[x]))
         kK, kV = k
-    per_unit = 4 * n * (kK + kV) + 2 * 2 * e * D + 4 * D * (kK + kV) + 2 * 4 * WL.group * D
-    return WL.n_kv_heads * per_unit
+    per_unit = 4 * n * (kK + kV) + 2 * 2 * e * D + 4 * D * (kK + kV) + 2 * 4 * wl.group * D
+    return wl.batch * wl.n_kv_heads * per_unit
 
 
 class Clocks:
@@ -220,6 +226,110 @@ def run_reference(args, rank: int):
 
 
 # ---------------------------------------------------------------------------------------------
+WL_LONG = syn.WORKLOADS[3]
+
+
+def long_context_decode(args, dev, flush, calls: int = 10):
+    """Decode over a long compressed history: one layer of the Qwen3-8B-shaped workload (batch 8
+    x 8 kv-heads, 32 q-heads, b=128, w=256, r_K=32, r_V=64) filled to 32768 tokens in one append
+    (rows drawn on the GPU with the same recipe), then ``calls`` decode calls, each after an L2
+    flush, timed with CUDA events: about 0.8 GB of coordinates per call, the HBM-bound regime of
+    the decode kernels. Returns (microseconds per call, bytes per call)."""
+    import torch
+
+    from rank_kv_cache_isvd_b200.cache import IsKVCache
+    wl = WL_LONG
+    S, H, T, QH = wl.batch, wl.n_kv_heads, wl.tokens, wl.n_q_heads
+    cache = IsKVCache(batch=S, n_layers=1, n_kv_heads=H, n_q_heads=QH, rank_k=wl.rank_k,
+                      rank_v=wl.rank_v, block=wl.block, window=wl.window, max_tokens=T,
+                      kv_dtype="bf16", rope=True, rope_theta=wl.rope_theta)
+    s = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(s):
+        Kr = torch.empty((S, H, T, D), dtype=torch.bfloat16, device=dev)
+        Vr = torch.empty_like(Kr)
+        for sq in range(S):
+            for h in range(H):
+                Kr[sq, h] = syn.device_rows(wl, sq, 0, h, 0, device=dev)
+                Vr[sq, h] = syn.device_rows(wl, sq, 0, h, 1, device=dev)
+        cache.append(0, Kr, Vr, s.cuda_stream)
+        del Kr, Vr
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(12345)
+        q = torch.randn((S, QH, D), generator=gen, device=dev)
+        out = torch.empty_like(q)
+    s.synchronize()
+    st = cache.status(s.cuda_stream)
+    assert st == 0, f"device status {st} after filling the long-context layer"
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for i in range(args.warmup + calls):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0.record(s)
+            cache.decode(0, q, out, s.cuda_stream)
+            e1.record(s)
+        s.synchronize()
+        if i >= args.warmup:
+            ms.append(e0.elapsed_time(e1))
+    assert cache.status(s.cuda_stream) == 0 and bool(torch.isfinite(out).all())
+    cache.close()
+    return 1e3 * float(np.median(ms)), decode_bytes(T, wl)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of the ranks' values: a multi-GPU step lasts as long as its slowest rank."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, total_ms: float, steps: int) -> float:
+    """Whole-job tokens/s: every rank streams its own sequence batch (weak scaling)."""
+    return world * WL.batch * WL.tokens / (total_ms / steps / 1e3)
+
+
+def fold_timing(args, dev, K, V, s, flush):
+    """Milliseconds of one append of the whole stream in a single call (every fold back to back
+    on the caller's stream), per replay of a captured graph."""
+    import torch
+
+    from rank_kv_cache_isvd_b200.cache import IsKVCache
+    T, H = WL.tokens, WL.n_kv_heads
+    fc = IsKVCache(batch=1, n_layers=1, n_kv_heads=H, n_q_heads=WL.n_q_heads, rank_k=WL.rank_k,
+                   rank_v=WL.rank_v, block=WL.block, window=WL.window, max_tokens=T,
+                   kv_dtype="bf16", rope=True, rope_theta=WL.rope_theta)
+    Kb = K[:, 0].transpose(0, 1).contiguous()[None]                 # [1][H][T][D]
+    Vb = V[:, 0].transpose(0, 1).contiguous()[None]
+    sh = s.cuda_stream
+    with torch.cuda.stream(s):
+        fc.reset(sh)
+        fc.append(0, Kb, Vb, sh)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fc.reset(sh)
+        fc.append(0, Kb, Vb, sh)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = []
+    for i in range(args.warmup + args.steps):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0.record(s)
+            g.replay()
+            e1.record(s)
+        s.synchronize()
+        if i >= args.warmup:
+            out.append(e0.elapsed_time(e1))
+    assert fc.status(sh) == 0
+    del g
+    fc.close()
+    return out
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -240,7 +350,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     cache = IsKVCache(batch=1, n_layers=1, n_kv_heads=H, n_q_heads=QH, rank_k=WL.rank_k,
                       rank_v=WL.rank_v, block=WL.block, window=WL.window, max_tokens=T,
-                      kv_dtype="bf16", rope=True, rope_theta=WL.rope_theta)
+                      kv_dtype="bf16", rope=True, rope_theta=WL.rope_theta, lookahead_folds=True)
     h = cache.handle
     kb, vb, qb, ob = K.data_ptr(), V.data_ptr(), Q.data_ptr(), OUT.data_ptr()
     krow = H * D * 2
@@ -258,23 +368,19 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     dec_marks = [(t, ev(), ev()) for t in range(args.sample_every - 1, T, args.sample_every)]
     dec_set = {t: (a, b) for t, a, b in dec_marks}
     fold_ts = [t for t in range(T) if WL.n_c(t + 1) > WL.n_c(t)]
-    fold_marks = {t: (ev(), ev()) for t in fold_ts}
 
     def step(stream_handle: int, timed_events: bool):
         iskv.check(iskv.iskv_reset(h, stream_handle))
         for t in range(T):
-            fm = fold_marks.get(t) if timed_events else None
-            if fm:
-                rec(fm[0], stream_handle)
             iskv.check(iskv.iskv_append_block(h, 0, kb + t * krow, vb + t * krow, 1, stream_handle))
-            if fm:
-                rec(fm[1], stream_handle)
             dm = dec_set.get(t) if timed_events else None
             if dm:
                 rec(dm[0], stream_handle)
             iskv.check(iskv.iskv_decode_attn(h, 0, qb + t * qrow, ob + t * qrow, stream_handle))
             if dm:
                 rec(dm[1], stream_handle)
+        # folds started ahead for blocks the window has not released yet join the step here
+        iskv.check(iskv.iskv_join(h, stream_handle))
 
     s = torch.cuda.Stream(device=dev)
     sh = s.cuda_stream
@@ -300,7 +406,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if world > 1:
         dist.barrier(device_ids=[local_rank])
     torch.cuda.synchronize(dev)
-    step_ms, dec_ms, dec_bytes, fold_ms = [], [], [], []
+    step_ms, dec_ms, dec_bytes = [], [], []
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with Clocks(local_rank) as clk:
         for _ in range(args.steps):
@@ -314,16 +420,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             for t, a, b in dec_marks:
                 dec_ms.append(elapsed(a, b))
                 dec_bytes.append(decode_bytes(t + 1))
-            fold_ms.append(sum(elapsed(a, b) for a, b in fold_marks.values()))
     torch.cuda.synchronize(dev)
     clocks = clk.summary()
-    total_ms = float(np.sum(step_ms))
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(float(np.sum(step_ms)), world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * WL.batch * T / (ms_per_step / 1e3)
+    value = job_throughput(world, total_ms, args.steps)
 
     # ---- end to end through the public API with host buffers --------------------------------
     kh = torch.from_numpy(kd.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -344,16 +445,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         s.synchronize()
         if i:
             e2e_ms.append(e0.elapsed_time(e1))
-    e2e_total = float(np.sum(e2e_ms))
-    if world > 1:
-        tt = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_total = float(tt.item())
-    e2e_value = world * WL.batch * T / (e2e_total / args.steps / 1e3)
+    e2e_total = max_over_ranks(float(np.sum(e2e_ms)), world, dev)
+    e2e_value = job_throughput(world, e2e_total, args.steps)
     h2d = (kh.numel() + vh.numel()) * 2 + qh.numel() * 4
     d2h = oh.numel() * 4
     status = iskv.iskv_sync_status(h, sh)
     assert status == 0, f"device status {status}"
+
+    # ---- fold throughput: the same 4096 rows appended in one call (60 folds back to back) ------
+    fold_ms = fold_timing(args, dev, K, V, s, flush)
+    # ---- decode over a long history (HBM-bound regime), rank 0 of a single-GPU run only --------
+    long_us, long_bytes = (long_context_decode(args, dev, flush) if world == 1 and rank == 0
+                           else (None, None))
 
     # ---- roofline of the dominant kernel class --------------------------------------------------
     hbm, which = peaks()
@@ -377,9 +480,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      "bytes_per_launch_mean": float(np.mean(dec_bytes)),
                      "launch_us_mean": 1e3 * float(np.mean(dec_ms))},
         "fold": {"head_block_updates_per_s": updates / (fold_total / 1e3),
-                 "updates_per_step": updates, "fold_ms_per_step": fold_total,
-                 "us_per_fold_call": 1e3 * fold_total / len(fold_ts)},
+                 "updates_per_call": updates, "ms_per_call": fold_total,
+                 "us_per_fold": 1e3 * fold_total / len(fold_ts),
+                 "how": (f"one append of all {T} rows (folds on the caller's stream, with the "
+                         f"history rotations and window appends), graph replay, L2 flushed; in "
+                         f"the decode step the folds run ahead on an internal stream")},
         "decode_ms_per_step": dec_total,
+        "roofline_long_context": None if long_us is None else {
+            "bound": "hbm", "kernel": "decode attention (split + combine)",
+            "workload": f"{WL_LONG.name}: one layer at t = {WL_LONG.tokens}",
+            "achieved": long_bytes / (long_us / 1e6) / 1e9, "peak": hbm, "unit": "GB/s",
+            "frac": long_bytes / (long_us / 1e6) / 1e9 / hbm, "traffic": None,
+            "bytes_per_launch": long_bytes, "launch_us": long_us},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h),
                 "how": "pinned host rows+queries copied in, graph replay, outputs copied out"},

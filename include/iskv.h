@@ -69,13 +69,23 @@ typedef struct {
     double rope_theta;    /* RoPE base; angle of pair j at position i is i * theta^(-2j/d)    */
     int rotate_history;   /* 1: iS-KV (old coordinates rotate with the basis).               */
                           /* 0: stale-coordinate ablation (drift study only).                */
+    int lookahead_folds;  /* 0: each fold runs on the caller's stream when the window releases  */
+                          /*    its block.                                                     */
+                          /* 1: each fold starts on an internal stream as soon as its block is */
+                          /*    complete (up to window / block + 1 folds ahead) and is joined  */
+                          /*    into the caller's stream when the window releases the block;   */
+                          /*    every decode sees exactly the state of mode 0. Call            */
+                          /*    iskv_join() before ending a stream capture that contains       */
+                          /*    appends.                                                       */
 } iskv_config;
 
 /*
  * Creates a cache for `cfg` on the current CUDA device. Allocates every device buffer
- * (coordinates C = U Sigma [max compressed rows x r] in fp32, bases B [d x r] fp32 (two copies
- * for in-place updates), Sigma [r] fp32, exact ring of window + block rows per path in kv_dtype,
- * a RoPE table [max_tokens x d/2] of (cos, sin), decode split partials and a status word).
+ * (coordinates C = U Sigma [max compressed rows x r] in fp32; bases B [d x r], Sigma [r] and the
+ * fold's H_top [r x r] in fp32, each in a ring of 2 buffers, or window / block + 3 with
+ * lookahead_folds; the exact ring of window + block rows per path in kv_dtype; a RoPE table
+ * [max_tokens x d/2] of (cos, sin); decode split partials; a status word) and, with
+ * lookahead_folds, the internal streams and events of the early folds.
  * Errors: ISKV_ERR_INVALID_ARG (cfg out of range), ISKV_ERR_CUDA (allocation failed; nothing
  * leaks). On success *out owns the handle; release it with iskv_destroy().
  */
@@ -102,7 +112,7 @@ int iskv_append_block(iskv_handle *h, int layer, const void *k_rows_dev, const v
  * Decode attention of `layer` over all t cached positions 0 .. t-1: compressed rows are
  * reconstructed as C B^T ("Reconstruction and Storage"), keys are then rotated by RoPE at their
  * position (when cfg.rope), scores use scale 1/sqrt(d), softmax is exact (fp32, log-sum-exp
- * merge of position splits).
+ * merge of position splits). Two kernels (position splits, then their merge) on `stream`.
  *   q_dev:   fp32 [batch][n_q_heads][head_dim], already rotated for the query position.
  *   out_dev: fp32 [batch][n_q_heads][head_dim].
  * Errors: ISKV_ERR_INVALID_ARG (NULL pointers, bad layer, t == 0), ISKV_ERR_CUDA.
@@ -136,8 +146,9 @@ int iskv_get_factors(iskv_handle *h, int layer, int seq, int kv_head, int which,
 
 /*
  * Empties every layer (t = n_c = 0, rank 0) and clears the sticky status, keeping all device
- * allocations, so a handle can serve a new batch of sequences. Host bookkeeping plus one
- * asynchronous device write on `stream`; later calls must be ordered after it on a stream.
+ * allocations, so a handle can serve a new batch of sequences. Joins pending early folds into
+ * `stream` first (iskv_join); then host bookkeeping plus asynchronous device writes on `stream`;
+ * later calls must be ordered after it on a stream.
  * Errors: ISKV_ERR_INVALID_ARG, ISKV_ERR_CUDA.
  */
 int iskv_reset(iskv_handle *h, iskv_stream_t stream);
@@ -177,7 +188,16 @@ int iskv_schedule(int block, int window, long long t, long long m, long long *n_
                   long long *folds_out);
 
 /*
- * Synchronises `stream` and returns the sticky device status: ISKV_OK, ISKV_ERR_NOT_CONVERGED,
+ * Makes `stream` wait for every fold that lookahead_folds started on an internal stream and that
+ * no later call has joined yet (those whose blocks the window has not released). Required before
+ * ending a stream capture that contains iskv_append_block() calls, so that the capture holds no
+ * unjoined work; a no-op without lookahead_folds. Enqueues only event waits.
+ * Errors: ISKV_ERR_INVALID_ARG, ISKV_ERR_CUDA.
+ */
+int iskv_join(iskv_handle *h, iskv_stream_t stream);
+
+/*
+ * Joins pending early folds (iskv_join), synchronises `stream` and returns the sticky status: ISKV_OK, ISKV_ERR_NOT_CONVERGED,
  * ISKV_ERR_NONFINITE or ISKV_ERR_TIMEOUT (the first error seen since creation or the last
  * iskv_reset()), or ISKV_ERR_CUDA if the synchronisation itself failed.
  */

@@ -36,6 +36,7 @@ __all__ = [
     "to_bf16",
     "queries",
     "workload_rows",
+    "device_rows",
 ]
 
 
@@ -177,3 +178,31 @@ def workload_rows(wl: Workload, seq: int, layer: int, head: int, kv: int, T: int
         return to_bf16(X)
     f = X.astype(np.float32)
     return f, f.astype(np.float64)
+
+
+def device_rows(wl: Workload, seq: int, layer: int, head: int, kv: int, T: int | None = None,
+                device="cuda"):
+    """The literal recipe of :func:`kv_rows` drawn with torch on a GPU, for timing workloads too
+    large to generate on the host in reasonable time (tens of thousands of rows per unit).
+
+    Same distribution and structure (orthonormal ``G`` and ``H`` from QR of Gaussians, spectrum
+    ``i^-a`` with the workload's exponent for this unit, noise 0.01, lognormal channel scales),
+    but a different random stream: the values do not equal :func:`workload_rows`. Returns a
+    ``T x d`` tensor in the workload's dtype on ``device``.
+    """
+    import torch
+    T = wl.tokens if T is None else T
+    d = wl.head_dim
+    seed = unit_seed(wl.cfg_id, seq, layer, head, kv)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    g = torch.randn(T, d, generator=gen, device=device, dtype=torch.float32)
+    h = torch.randn(d, d, generator=gen, device=device, dtype=torch.float32)
+    G = torch.linalg.qr(g)[0]
+    H = torch.linalg.qr(h)[0]
+    a = _decay(wl, seed, kv)
+    s = torch.arange(1, d + 1, device=device, dtype=torch.float32) ** (-a)
+    X = (G * s) @ H.T + 0.01 * torch.randn(T, d, generator=gen, device=device)
+    if wl.channel_sigma:
+        X = X * torch.exp(wl.channel_sigma * torch.randn(d, generator=gen, device=device))
+    return X.to(torch.bfloat16 if wl.kv_dtype == "bf16" else torch.float32)

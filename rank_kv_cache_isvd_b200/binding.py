@@ -20,6 +20,7 @@ __all__ = [
     "iskv_create", "iskv_destroy", "iskv_append_block", "iskv_decode_attn", "iskv_reconstruct",
     "iskv_get_factors", "iskv_num_tokens", "iskv_storage_bytes", "iskv_schedule",
     "iskv_sync_status", "iskv_strerror", "iskv_reset", "iskv_launch_count", "iskv_fold_stats",
+    "iskv_join",
     "iskv_decode_view", "iskv_decode_attn_noalloc", "ISKV_NOALLOC_SCRATCH_FLOATS",
 ]
 
@@ -53,6 +54,7 @@ class iskv_config(ctypes.Structure):
         ("rope", ctypes.c_int),
         ("rope_theta", ctypes.c_double),
         ("rotate_history", ctypes.c_int),
+        ("lookahead_folds", ctypes.c_int),
     ]
 
 
@@ -108,6 +110,7 @@ _SIGNATURES = {
     "iskv_storage_bytes": (_i, [_vp, _i, ctypes.POINTER(_ll)]),
     "iskv_schedule": (_i, [_i, _i, _ll, _ll, ctypes.POINTER(_ll), ctypes.POINTER(_ll)]),
     "iskv_sync_status": (_i, [_vp, _vp]),
+    "iskv_join": (_i, [_vp, _vp]),
     "iskv_strerror": (ctypes.c_char_p, [_i]),
     "iskv_reset": (_i, [_vp, _vp]),
     "iskv_launch_count": (_i, [_vp, ctypes.POINTER(_ll)]),
@@ -239,6 +242,10 @@ def iskv_fold_stats(handle, stream=None):
 def iskv_decode_attn_noalloc(view: iskv_decode_view, q, out, stream=None) -> int:
     return lib.iskv_decode_attn_noalloc(None if view is None else ctypes.byref(view), _ptr(q),
                                         _ptr(out), _stream(stream))
+
+
+def iskv_join(handle, stream=None) -> int:
+    return lib.iskv_join(handle, _stream(stream))
 
 
 def iskv_sync_status(handle, stream=None) -> int:

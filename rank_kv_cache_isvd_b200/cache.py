@@ -6,7 +6,7 @@ import torch
 
 from .binding import (ISKV_BF16, ISKV_F32, check, iskv_append_block, iskv_config, iskv_create,
                       iskv_decode_attn, iskv_destroy, iskv_fold_stats, iskv_get_factors,
-                      iskv_launch_count,
+                      iskv_join, iskv_launch_count,
                       iskv_num_tokens, iskv_reconstruct, iskv_reset, iskv_storage_bytes,
                       iskv_sync_status)
 
@@ -17,11 +17,12 @@ class IsKVCache:
     def __init__(self, *, batch: int, n_layers: int, n_kv_heads: int, n_q_heads: int,
                  rank_k: int, rank_v: int, block: int, window: int, max_tokens: int,
                  kv_dtype: str = "bf16", rope: bool = True, rope_theta: float = 5e5,
-                 rotate_history: bool = True, head_dim: int = 128):
+                 rotate_history: bool = True, head_dim: int = 128,
+                 lookahead_folds: bool = False):
         self.cfg = iskv_config(batch, n_layers, n_kv_heads, n_q_heads, head_dim, rank_k, rank_v,
                                block, window, max_tokens,
                                ISKV_BF16 if kv_dtype == "bf16" else ISKV_F32, int(rope),
-                               float(rope_theta), int(rotate_history))
+                               float(rope_theta), int(rotate_history), int(lookahead_folds))
         self.dtype = torch.bfloat16 if kv_dtype == "bf16" else torch.float32
         self.handle = 0
         code, h = iskv_create(self.cfg)
@@ -88,6 +89,10 @@ class IsKVCache:
         code, b = iskv_storage_bytes(self.handle, layer)
         check(code, "iskv_storage_bytes")
         return b
+
+    def join(self, stream=None) -> None:
+        """Joins folds started ahead of time into ``stream`` (needed before ending a capture)."""
+        check(iskv_join(self.handle, stream), "iskv_join")
 
     def reset(self, stream=None) -> None:
         check(iskv_reset(self.handle, stream), "iskv_reset")

@@ -2,18 +2,22 @@
 //
 // iS-KV summary, "Reconstruction and Storage": compressed rows are (C B^T)[i]; keys were
 // compressed before RoPE, so a key tile K~ = C_K[tile] B_K^T (128 rows x 128 channels) is formed on
-// the tensor cores and rotated afterwards, row by row. One CTA (4 warps) serves one split of one
-// kv-head; thread i owns row i of the tile, which is TMEM lane i of the accumulator.
+// the tensor cores and rotated afterwards, row by row.
 //
-// Per compressed tile: a TMA load of the coordinate tile (128-byte swizzle, 32 fp32 per row and
-// K-block) and a bulk load of the value coordinates; the key coordinates are split into tf32
-// hi + lo parts in place and three kind::tf32 MMAs (hi*hi + hi*lo + lo*hi) give fp32-level keys in
-// TMEM; the epilogue reads the row (tcgen05.ld), applies RoPE at the row's position, takes the dot
-// products with the G pre-scaled queries, updates the online softmax and accumulates
-// sum_i p_i C_V[i] in rank space. Window tiles read the exact bf16/fp32 rows instead.
-// The last CTA of a kv-head to finish merges all splits (log-sum-exp) and expands the rank-space
-// value sum once through B_V^T; an arrival counter, reset by that CTA, decides who is last, so no
-// CTA ever waits for another.
+// Split kernel: one CTA (8 warps) serves one split of one kv-head. Row i of a 128-row tile is TMEM
+// lane i of the accumulator; warps w and w + 4 both read lanes 32 (w mod 4) .. +31 and take half of
+// the RoPE channel pairs (j, j + 64) each, so every row has two threads. Per compressed tile: a
+// TMA load of the key-coordinate tile (128-byte swizzle, 32 fp32 per row and K-block) and a bulk
+// load of the value coordinates; the key coordinates are split into tf32 hi + lo parts and three
+// kind::tf32 MMAs (hi*hi + hi*lo + lo*hi) give fp32-level keys in TMEM; the epilogue rotates the
+// row at its position, forms the dot products with the G pre-scaled queries, updates the online
+// softmax and accumulates sum_i p_i C_V[i] in rank space. The next tile's key coordinates are
+// loaded while this tile's epilogue runs, its value coordinates while the softmax runs. Window
+// tiles read the exact bf16/fp32 rows instead. Each split writes (max, sum, accumulator) partials.
+//
+// Merge kernel: one CTA per (q-head, kv-head) combines the splits (log-sum-exp weights) and
+// expands the rank-space value sum once through B_V^T. It is launched as a programmatic dependent
+// of the split kernel, so its prologue (staging B_V) overlaps the split kernel's tail.
 #include <math_constants.h>
 
 #include "iskv_internal.cuh"
@@ -21,13 +25,17 @@
 
 namespace iskv {
 
-constexpr int TC_THREADS = 128;
+constexpr int TC_THREADS = 256;
+constexpr int MERGE_THREADS = 128;
+constexpr int MERGE_REG = 48;             // splits whose partials a merge thread keeps in registers
 constexpr int KBLK_BYTES = 128 * 128;     // one K-block: 128 rows x 32 fp32
 
 struct TcLayout {
-    uint32_t b_hi, b_lo, a_hi, a_lo, v, q, p, red, stat, bars, total;
+    uint32_t b_hi, b_lo, a_hi, a_lo, v, q, x, red, acc, bars, total;
 };
 
+// Shared-memory plan of the split kernel. Window tiles stage their exact value rows from a_hi
+// onwards (a_hi, a_lo and v are contiguous and unused by window tiles otherwise).
 __host__ __device__ inline TcLayout tc_layout(int kblocks, int rV, int esz) {
     TcLayout L;
     uint32_t o = 0;
@@ -36,12 +44,16 @@ __host__ __device__ inline TcLayout tc_layout(int kblocks, int rV, int esz) {
     L.a_hi = o; o += kblocks * KBLK_BYTES;
     L.a_lo = o; o += kblocks * KBLK_BYTES;
     L.v = o;
-    const uint32_t vb = (uint32_t)(128 * rV * 4) > (uint32_t)(128 * D * esz) ? 128 * rV * 4 : 128 * D * esz;
+    const uint32_t vcomp = 128u * rV * 4u;
+    const uint32_t vwin = 128u * D * esz;
+    const uint32_t span = 2u * kblocks * KBLK_BYTES;      // a_hi + a_lo
+    uint32_t vb = vcomp;
+    if (vwin > span + vb) vb = vwin - span;
     o += (vb + 1023) & ~1023u;
     L.q = o; o += GMAX * D * 4;
-    L.p = o; o += GMAX * 128 * 4;
+    L.x = o; o += 2 * GMAX * 128 * 4;        // score halves, then (aliased) probabilities
     L.red = o; o += 2 * 4 * GMAX * 4;
-    L.stat = o; o += 4 * GMAX * 4;
+    L.acc = o; o += GMAX * D * 4;
     L.bars = o; o += 64;
     L.total = o + 1024;                    // slack for aligning the base to 1024 bytes
     return L;
@@ -58,6 +70,28 @@ __device__ __forceinline__ float warp_sum_f(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Split fp32 values into a tf32 "hi" part (top 19 bits, exact in tf32) kept in place and the
@@ -80,13 +114,14 @@ __device__ __forceinline__ void split_tf32(uint8_t *hi, uint8_t *lo, int bytes) 
     }
 }
 
-__device__ __forceinline__ void load_row32(const void *ring, size_t base, int kv_dtype,
-                                           float (&v)[32]) {
+// 16 consecutive channels of an exact row (bf16 or fp32) as fp32.
+__device__ __forceinline__ void load_row16(const void *ring, size_t base, int kv_dtype,
+                                           float (&v)[16]) {
     if (kv_dtype == ISKV_BF16) {
         const uint4 *p = reinterpret_cast<const uint4 *>(
             reinterpret_cast<const __nv_bfloat16 *>(ring) + base);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
             const uint4 u = p[q];
             const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -98,7 +133,7 @@ __device__ __forceinline__ void load_row32(const void *ring, size_t base, int kv
     } else {
         const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(ring) + base);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < 4; ++q) {
             const float4 f = p[q];
             v[4 * q] = f.x;
             v[4 * q + 1] = f.y;
@@ -108,6 +143,17 @@ __device__ __forceinline__ void load_row32(const void *ring, size_t base, int kv
     }
 }
 
+// Four consecutive channels of a value row staged in shared memory.
+__device__ __forceinline__ float4 load_v4(const uint8_t *row, int c, int fmt) {
+    if (fmt == 2) {                                   // bf16 row
+        const uint2 u = *reinterpret_cast<const uint2 *>(row + 2 * c);
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                           __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+    }
+    return *reinterpret_cast<const float4 *>(row + 4 * c);
+}
+
+template <int GT>
 __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmB,
     DecodeArgs a, TcExtra x) {
@@ -118,21 +164,25 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
     const int esz = a.kv_dtype == ISKV_BF16 ? 2 : 4;
     const TcLayout L = tc_layout(x.kblocks, rV, esz);
     uint8_t *bBh = sm + L.b_hi, *bBl = sm + L.b_lo, *bAh = sm + L.a_hi, *bAl = sm + L.a_lo;
-    uint8_t *bV = sm + L.v;
     float *sQ = reinterpret_cast<float *>(sm + L.q);
-    float *sP = reinterpret_cast<float *>(sm + L.p);
-    float *sRed = reinterpret_cast<float *>(sm + L.red);        // [2][4 warps][GMAX]
-    float *sM = reinterpret_cast<float *>(sm + L.stat);         // [GMAX] running max
-    float *sL = sM + GMAX, *sAl = sL + GMAX;
-    int *sFlag = reinterpret_cast<int *>(sAl + GMAX);
-    uint64_t *bar_load = reinterpret_cast<uint64_t *>(sm + L.bars);
-    uint64_t *bar_mma = bar_load + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_load + 2);
+    float *sX = reinterpret_cast<float *>(sm + L.x);            // [2 halves][GMAX][128]
+    float *sP = sX;                                             // [GMAX][128] (after the scores)
+    float *sRed = reinterpret_cast<float *>(sm + L.red);        // [2][4][GMAX]
+    float *sAcc = reinterpret_cast<float *>(sm + L.acc);        // [GMAX][D] running value sums
+    uint64_t *bar_a = reinterpret_cast<uint64_t *>(sm + L.bars);
+    uint64_t *bar_v = bar_a + 1;
+    uint64_t *bar_mma = bar_a + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_a + 3);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, half = warp >> 2;
     const int ul = blockIdx.y, split = blockIdx.x;
     const int seq = ul / a.H, h = ul % a.H;
     const bool comp = split < a.n_split_c;
+    uint8_t *bV = comp ? sm + L.v : bAh;                        // value rows of the tile
+    const int vfmt = comp ? 4 : esz;
+    const int vld = comp ? rV * 4 : D * esz;                    // bytes per staged value row
+    const int nacc = comp ? kV : D;
     long long p0, p1;
     if (comp) {
         p0 = (long long)split * a.split_rows;
@@ -141,105 +191,108 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
         p0 = a.n_c + (long long)(split - a.n_split_c) * DEC_TILE;
         p1 = min(a.t, p0 + DEC_TILE);
     }
-    {
-        const float4 *q4 = reinterpret_cast<const float4 *>(a.q + ((size_t)seq * a.H * G + (size_t)h * G) * D);
-        float4 *s4 = reinterpret_cast<float4 *>(sQ);
-        const float sc = a.scale;
-        float4 v[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int o = tid + TC_THREADS * u;
-            v[u] = o < G * D / 4 ? q4[o] : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int o = tid + TC_THREADS * u;
-            if (o < G * D / 4) s4[o] = make_float4(v[u].x * sc, v[u].y * sc, v[u].z * sc, v[u].w * sc);
-        }
-    }
-    if (tid < G) {
-        sM[tid] = -CUDART_INF_F;
-        sL[tid] = 0.f;
-    }
-    if (tid == 0) {
-        mbar_init(bar_load, 1);
-        mbar_init(bar_mma, 1);
-        fence_mbar_init();
-    }
-    if (comp && warp == 0) tmem_alloc(tmem_slot, 128);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = comp ? *tmem_slot : 0u;
-    uint32_t ph_load = 0, ph_mma = 0;
-    bool ok = true;
 
     const size_t ring_base = (size_t)ul * a.R * D;
     const float *Cv = a.coords[1] + (size_t)ul * a.n_max * rV;
     const uint32_t idesc = idesc_tf32(128, 128);
+    const uint32_t abytes = x.kblocks * KBLK_BYTES;
 
-    // thread 0: loads of one tile (key coordinates by TMA, value coordinates or exact window
-    // value rows by bulk copy); the caller has posted the expected byte count
-    auto issue_tile = [&](long long t0, int rows) {
+    // thread 0: key-coordinate tile (TMA) and value rows (bulk copies) of the tile at t0; each
+    // barrier phase gets exactly one arrival, which posts all bytes of that phase
+    auto tma_a = [&](long long t0) {
+        for (int kb = 0; kb < x.kblocks; ++kb)
+            tma_load_2d(bAh + kb * KBLK_BYTES, &tmC, kb * 32,
+                        (int)(x.row0 + (long long)ul * a.n_max + t0), bar_a);
+    };
+    auto issue_v = [&](long long t0, int rows) {
         if (comp) {
-            for (int kb = 0; kb < x.kblocks; ++kb)
-                tma_load_2d(bAh + kb * KBLK_BYTES, &tmC, kb * 32,
-                            (int)(x.row0 + (long long)ul * a.n_max + t0), bar_load);
-            bulk_load(bV, Cv + (size_t)t0 * rV, (uint32_t)rows * rV * 4, bar_load);
+            mbar_arrive_expect_tx(bar_v, (uint32_t)rows * rV * 4);
+            bulk_load(bV, Cv + (size_t)t0 * rV, (uint32_t)rows * rV * 4, bar_v);
         } else {
             const int s0 = (int)(t0 % a.R);
             const int n1 = min(rows, a.R - s0);
             const uint32_t rb = D * esz;
             const char *ring = static_cast<const char *>(a.ring[1]);
-            bulk_load(bV, ring + (ring_base + (size_t)s0 * D) * esz, (uint32_t)n1 * rb, bar_load);
+            mbar_arrive_expect_tx(bar_v, (uint32_t)rows * rb);
+            bulk_load(bV, ring + (ring_base + (size_t)s0 * D) * esz, (uint32_t)n1 * rb, bar_v);
             if (n1 < rows)
                 bulk_load(bV + (size_t)n1 * rb, ring + ring_base * esz, (uint32_t)(rows - n1) * rb,
-                          bar_load);
+                          bar_v);
         }
     };
-    auto tile_bytes = [&](int rows) -> uint32_t {
-        return comp ? x.kblocks * KBLK_BYTES + (uint32_t)rows * rV * 4 : (uint32_t)rows * D * esz;
-    };
-    if (tid == 0 && p0 < p1) {
-        const int rows0 = (int)min((long long)DEC_TILE, p1 - p0);
-        mbar_arrive_expect_tx(bar_load, tile_bytes(rows0) + (comp ? x.kblocks * KBLK_BYTES : 0u));
-        if (comp)
-            for (int kb = 0; kb < x.kblocks; ++kb)
-                tma_load_2d(bBh + kb * KBLK_BYTES, &tmB, kb * 32, x.brow0 + ul * D, bar_load);
-        issue_tile(p0, rows0);
-    }
 
-    float vacc[8];
+    if (comp && warp == 0) tmem_alloc(tmem_slot, 128);
+    // everything the previous kernel in the stream writes (rows, factors, queries) is read only
+    // after this point; dependents may start once every CTA got here
+    griddep_wait();
+    griddep_launch_dependents();
+    // outstanding phases (the same in every thread: issue conditions are uniform)
+    bool pend_a = comp && p0 < p1, pend_v = p0 < p1, pend_m = false;
+    uint32_t ph_a = 0, ph_v = 0, ph_m = 0;
+    if (tid == 0) {
+        mbar_init(bar_a, 1);
+        mbar_init(bar_v, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+        if (p0 < p1) {
+            if (comp) {
+                mbar_arrive_expect_tx(bar_a, 2 * abytes);
+                for (int kb = 0; kb < x.kblocks; ++kb)
+                    tma_load_2d(bBh + kb * KBLK_BYTES, &tmB, kb * 32, x.brow0 + ul * D, bar_a);
+                tma_a(p0);
+            }
+            issue_v(p0, (int)min((long long)DEC_TILE, p1 - p0));
+        }
+    }
+    {
+        const float4 *q4 = reinterpret_cast<const float4 *>(a.q + ((size_t)seq * a.H * G + (size_t)h * G) * D);
+        float4 *s4 = reinterpret_cast<float4 *>(sQ);
+        const float sc = a.scale;
+        if (tid < G * D / 4) {
+            const float4 v = q4[tid];
+            s4[tid] = make_float4(v.x * sc, v.y * sc, v.z * sc, v.w * sc);
+        }
+        for (int o = tid; o < G * D; o += TC_THREADS) sAcc[o] = 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = comp ? *tmem_slot : 0u;
+    bool ok = true;
+
+    float mrun[GT], lrun[GT];
 #pragma unroll
-    for (int w = 0; w < 8; ++w) vacc[w] = 0.f;
-    const int nacc = comp ? kV : D;
+    for (int g = 0; g < GT; ++g) {
+        mrun[g] = -CUDART_INF_F;
+        lrun[g] = 0.f;
+    }
+    const int row = 32 * wq + lane;
 
     for (long long t0 = p0; t0 < p1 && ok; t0 += DEC_TILE) {
         const int rows = (int)min((long long)DEC_TILE, p1 - t0);
-        if (t0 != p0) {
-            tc_fence_before();
-            __syncthreads();                 // previous tile fully consumed (smem and TMEM)
-            if (tid == 0) {
-                mbar_arrive_expect_tx(bar_load, tile_bytes(rows));
-                issue_tile(t0, rows);
-            }
-        }
-        ok = __syncthreads_and(mbar_wait(bar_load, ph_load)) != 0;
-        ph_load ^= 1;
-        if (!ok) break;
-        if (comp && t0 == p0) split_tf32(bBh, bBl, x.kblocks * KBLK_BYTES);
-
-        const int row = tid;
         const bool valid = row < rows;
         const long long pos = t0 + row;
         const bool rope = valid && a.rope_cs != nullptr;
-        float4 cs0[16];
-        float part[GMAX];
+        const int jb = 32 * half;               // this thread's first channel pair
+        float part[GT];
 #pragma unroll
-        for (int g = 0; g < GMAX; ++g) part[g] = 0.f;
+        for (int g = 0; g < GT; ++g) part[g] = 0.f;
+        // RoPE angles of this thread's 32 pairs: the first half is loaded before anything waits,
+        // the second half while the MMA runs, so their latency hides under the tile loads
+        float4 cs[16];
+        const float4 *c4 = reinterpret_cast<const float4 *>(a.rope_cs + pos * DH + jb);
+        if (rope) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) cs[q] = c4[q];
+        }
 
         if (comp) {
-            split_tf32(bAh, bAl, x.kblocks * KBLK_BYTES);
+            ok = __syncthreads_and(mbar_wait(bar_a, ph_a)) != 0;
+            if (!ok) break;
+            pend_a = false;
+            ph_a ^= 1;
+            if (t0 == p0) split_tf32(bBh, bBl, abytes);
+            split_tf32(bAh, bAl, abytes);
             fence_proxy_async_smem();
             __syncthreads();
             if (tid == 0) {
@@ -258,44 +311,52 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
                     }
                 mma_commit(bar_mma);
             }
-            if (rope) {                       // RoPE angles of pass 0 load while the MMA runs
-                const float4 *cs = reinterpret_cast<const float4 *>(a.rope_cs + pos * DH);
+            pend_m = true;
+            if (rope) {
 #pragma unroll
-                for (int q = 0; q < 16; ++q) cs0[q] = cs[q];
+                for (int q = 8; q < 16; ++q) cs[q] = c4[q];
             }
-            ok = __syncthreads_and(mbar_wait(bar_mma, ph_mma)) != 0;
-            ph_mma ^= 1;
+            ok = __syncthreads_and(mbar_wait(bar_mma, ph_m)) != 0;
             tc_fence_after();
             if (!ok) break;
+            pend_m = false;
+            ph_m ^= 1;
+            // the key-coordinate buffers are free again: fetch the next tile's under this epilogue
+            if (t0 + DEC_TILE < p1) {
+                pend_a = true;
+                if (tid == 0) {
+                    mbar_arrive_expect_tx(bar_a, abytes);
+                    tma_a(t0 + DEC_TILE);
+                }
+            }
         }
 
-        if (!comp && rope) {
-            const float4 *cs = reinterpret_cast<const float4 *>(a.rope_cs + pos * DH);
+        // ---- this row's key, channel pairs (j, j + 64) for j in [jb, jb + 32), two chunks -------
+        const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) cs0[q] = cs[q];
-        }
-        // ---- this row's key (two passes: channel pairs (j, j+64), j in [32hp, 32hp+32)) -------
-        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll
-        for (int hp = 0; hp < 2; ++hp) {
-            float lo[32], hi[32];
+        for (int ch = 0; ch < 2; ++ch) {
+            const int j0 = jb + 16 * ch;
+            float lo[16], hi[16];
             if (comp) {
-                tmem_ld32(trow + hp * 32, lo);
-                tmem_ld32(trow + 64 + hp * 32, hi);
+                tmem_ld16(trow + j0, lo);
+                tmem_ld16(trow + 64 + j0, hi);
                 tmem_wait_ld();
             } else if (valid) {
                 const size_t rb = ring_base + (size_t)(pos % a.R) * D;
-                load_row32(a.ring[0], rb + hp * 32, a.kv_dtype, lo);
-                load_row32(a.ring[0], rb + 64 + hp * 32, a.kv_dtype, hi);
+                load_row16(a.ring[0], rb + j0, a.kv_dtype, lo);
+                load_row16(a.ring[0], rb + 64 + j0, a.kv_dtype, hi);
             } else {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) lo[j] = hi[j] = 0.f;
+                for (int j = 0; j < 16; ++j) lo[j] = hi[j] = 0.f;
+            }
+            if (rope && !comp && ch == 1) {
+#pragma unroll
+                for (int q = 8; q < 16; ++q) cs[q] = c4[q];
             }
             if (rope) {
-                const float4 *cs = reinterpret_cast<const float4 *>(a.rope_cs + pos * DH + hp * 32);
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const float4 w = hp == 0 ? cs0[q] : cs[q];
+                for (int q = 0; q < 8; ++q) {
+                    const float4 w = cs[8 * ch + q];
                     const float x0 = lo[2 * q], y0 = hi[2 * q], x1 = lo[2 * q + 1], y1 = hi[2 * q + 1];
                     lo[2 * q] = x0 * w.x - y0 * w.y;
                     hi[2 * q] = y0 * w.x + x0 * w.y;
@@ -304,13 +365,13 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
                 }
             }
 #pragma unroll
-            for (int g = 0; g < GMAX; ++g) {
+            for (int g = 0; g < GT; ++g) {
                 if (g < G) {
-                    const float4 *ql = reinterpret_cast<const float4 *>(sQ + g * D + hp * 32);
-                    const float4 *qh = reinterpret_cast<const float4 *>(sQ + g * D + 64 + hp * 32);
+                    const float4 *ql = reinterpret_cast<const float4 *>(sQ + g * D + j0);
+                    const float4 *qh = reinterpret_cast<const float4 *>(sQ + g * D + 64 + j0);
                     float s = part[g];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
+                    for (int q = 0; q < 4; ++q) {
                         const float4 u = ql[q], v = qh[q];
                         s = fmaf(u.x, lo[4 * q], s);
                         s = fmaf(u.y, lo[4 * q + 1], s);
@@ -325,71 +386,123 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
                 }
             }
         }
-        // ---- online softmax over the tile's rows -------------------------------------------------
+        // ---- the two halves of each row meet; both threads hold the same score ------------------
 #pragma unroll
-        for (int g = 0; g < GMAX; ++g) {
+        for (int g = 0; g < GT; ++g)
+            if (g < G) sX[(half * GMAX + g) * 128 + row] = part[g];
+        __syncthreads();
+#pragma unroll
+        for (int g = 0; g < GT; ++g)
             if (g < G) {
+                part[g] = sX[g * 128 + row] + sX[(GMAX + g) * 128 + row];
                 const float m = warp_max_f(valid ? part[g] : -CUDART_INF_F);
-                if (lane == 0) sRed[warp * GMAX + g] = m;
+                if (half == 0 && lane == 0) sRed[wq * GMAX + g] = m;
             }
-        }
         __syncthreads();
+        // ---- online softmax: every thread keeps the same running max and sum -------------------
+        float alpha[GT];
 #pragma unroll
-        for (int g = 0; g < GMAX; ++g) {
+        for (int g = 0; g < GT; ++g) {
+            alpha[g] = 1.f;
             if (g < G) {
-                float mt = sRed[g];
-#pragma unroll
-                for (int w = 1; w < 4; ++w) mt = fmaxf(mt, sRed[w * GMAX + g]);
-                const float m_new = fmaxf(sM[g], mt);
+                const float mt = fmaxf(fmaxf(sRed[g], sRed[GMAX + g]),
+                                       fmaxf(sRed[2 * GMAX + g], sRed[3 * GMAX + g]));
+                const float m_new = fmaxf(mrun[g], mt);
                 const float pr = valid ? expf(part[g] - m_new) : 0.f;
-                sP[g * DEC_TILE + row] = pr;
-                const float s = warp_sum_f(pr);
-                if (lane == 0) sRed[4 * GMAX + warp * GMAX + g] = s;
-                part[g] = m_new;                 // keep m_new for the stats update
-            }
-        }
-        __syncthreads();
-        if (tid < G) {
-            const int g = tid;
-            const float m_new = part[g];
-            const float alpha = expf(sM[g] - m_new);
-            float s = 0.f;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) s += sRed[4 * GMAX + w * GMAX + g];
-            sL[g] = sL[g] * alpha + s;
-            sM[g] = m_new;
-            sAl[g] = alpha;
-        }
-        __syncthreads();
-        // ---- value accumulation: acc[g][c] = acc * alpha_g + sum_i p[g][i] V[i][c] ------------------
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            const int o = tid + TC_THREADS * w;
-            if (o < G * nacc) {
-                const int g = o / nacc, c = o % nacc;
-                const float *pg = sP + g * DEC_TILE;
-                float s4[4] = {0.f, 0.f, 0.f, 0.f};
-                const int ld = comp ? rV : D;
-                int i = 0;
-                if (comp || esz == 4) {
-                    const float *vv = reinterpret_cast<const float *>(bV) + c;
-                    for (; i + 3 < rows; i += 4)
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) s4[u] = fmaf(pg[i + u], vv[(i + u) * ld], s4[u]);
-                    for (; i < rows; ++i) s4[0] = fmaf(pg[i], vv[i * ld], s4[0]);
-                } else {
-                    const __nv_bfloat16 *vv = reinterpret_cast<const __nv_bfloat16 *>(bV) + c;
-                    for (; i + 3 < rows; i += 4)
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            s4[u] = fmaf(pg[i + u], __bfloat162float(vv[(i + u) * D]), s4[u]);
-                    for (; i < rows; ++i) s4[0] = fmaf(pg[i], __bfloat162float(vv[i * D]), s4[0]);
+                if ((g & 1) == half) {
+                    sP[g * 128 + row] = pr;
+                    const float s = warp_sum_f(pr);
+                    if (lane == 0) sRed[4 * GMAX + wq * GMAX + g] = s;
                 }
-                vacc[w] = fmaf(vacc[w], sAl[g], (s4[0] + s4[1]) + (s4[2] + s4[3]));
+                alpha[g] = expf(mrun[g] - m_new);
+                mrun[g] = m_new;
             }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int g = 0; g < GT; ++g)
+            if (g < G) {
+                const float s = (sRed[4 * GMAX + g] + sRed[5 * GMAX + g]) +
+                                (sRed[6 * GMAX + g] + sRed[7 * GMAX + g]);
+                lrun[g] = fmaf(lrun[g], alpha[g], s);
+            }
+        // ---- value accumulation: sAcc[g][c] = sAcc * alpha_g + sum_i p[g][i] V[i][c] ------------
+        // thread = (channel quad qd, row slice sl): quads vary fastest, so the lanes of a
+        // shared-memory phase read consecutive 16-byte (8-byte for bf16) pieces of one staged row
+        // (no bank conflicts); slice sl takes rows sl, sl + nsl, ... Quads past the row's end
+        // (nqp is a power of two) read the next row's values and are never used. The slices'
+        // sums meet in shared memory: first within the warp (shuffles), then across the 8 warps
+        // in `red` (a_lo for compressed tiles: free once the MMA is done; b_hi for window tiles).
+        ok = __syncthreads_and(mbar_wait(bar_v, ph_v)) != 0;
+        if (!ok) break;
+        pend_v = false;
+        ph_v ^= 1;
+        {
+            const int nq = (nacc + 3) >> 2;
+            const int nqp = nq <= 8 ? 8 : nq <= 16 ? 16 : 32;
+            const int nsl = TC_THREADS / nqp;
+            const int qd = tid & (nqp - 1), sl = tid / nqp;
+            float *red = reinterpret_cast<float *>(comp ? bAl : bBh);   // [8 warps][G][4 nqp]
+            float4 acc4[GT];
+#pragma unroll
+            for (int g = 0; g < GT; ++g) acc4[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int i = sl; i < rows; i += nsl) {
+                const float4 v = load_v4(bV + (size_t)i * vld, 4 * qd, vfmt);
+#pragma unroll
+                for (int g = 0; g < GT; ++g)
+                    if (g < G) {
+                        const float pg = sP[g * 128 + i];
+                        acc4[g].x = fmaf(pg, v.x, acc4[g].x);
+                        acc4[g].y = fmaf(pg, v.y, acc4[g].y);
+                        acc4[g].z = fmaf(pg, v.z, acc4[g].z);
+                        acc4[g].w = fmaf(pg, v.w, acc4[g].w);
+                    }
+            }
+            // slices that share a warp: lanes nqp, 2 nqp, ... apart
+#pragma unroll
+            for (int g = 0; g < GT; ++g)
+                if (g < G) {
+                    for (int o = nqp; o < 32; o <<= 1) {
+                        acc4[g].x += __shfl_xor_sync(0xffffffffu, acc4[g].x, o);
+                        acc4[g].y += __shfl_xor_sync(0xffffffffu, acc4[g].y, o);
+                        acc4[g].z += __shfl_xor_sync(0xffffffffu, acc4[g].z, o);
+                        acc4[g].w += __shfl_xor_sync(0xffffffffu, acc4[g].w, o);
+                    }
+                }
+            if (lane < nqp) {
+#pragma unroll
+                for (int g = 0; g < GT; ++g)
+                    if (g < G)
+                        reinterpret_cast<float4 *>(red)[(warp * G + g) * nqp + qd] = acc4[g];
+            }
+            __syncthreads();
+            for (int o = tid; o < G * nacc; o += TC_THREADS) {
+                const int g = o / nacc, c = o % nacc;
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) sum += red[((w * G + g) * nqp) * 4 + c];
+                float al = 1.f;
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg)
+                    if (gg == g) al = alpha[gg];
+                sAcc[g * D + c] = fmaf(sAcc[g * D + c], al, sum);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();                       // value rows, probabilities and TMEM consumed
+        if (t0 + DEC_TILE < p1) {
+            pend_v = true;
+            if (tid == 0) issue_v(t0 + DEC_TILE, (int)min((long long)DEC_TILE, p1 - t0 - DEC_TILE));
         }
     }
-    if (!ok && tid == 0) set_status(x.status, ISKV_ERR_TIMEOUT);
+    if (!ok && tid == 0) {
+        // a wait gave up: record it, then let this CTA's own copies and MMAs drain (bounded)
+        set_status(x.status, ISKV_ERR_TIMEOUT);
+        if (pend_a) mbar_wait(bar_a, ph_a);
+        if (pend_v) mbar_wait(bar_v, ph_v);
+        if (pend_m) mbar_wait(bar_mma, ph_m);
+    }
 
     // ---- release tensor memory -------------------------------------------------------------------
     tc_fence_before();
@@ -401,149 +514,144 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
 
     // ---- partials: [m, l, acc[nacc]] per q-head ------------------------------------------------
     float *ws = a.ws + ((size_t)ul * a.max_splits + split) * G * (2 + D);
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        const int o = tid + TC_THREADS * w;
-        if (o < G * nacc) ws[(o / nacc) * (2 + D) + 2 + o % nacc] = vacc[w];
+    for (int o = tid; o < G * nacc; o += TC_THREADS) {
+        const int g = o / nacc, c = o % nacc;
+        ws[g * (2 + D) + 2 + c] = sAcc[g * D + c];
     }
     if (tid < G) {
-        ws[tid * (2 + D)] = sM[tid];
-        ws[tid * (2 + D) + 1] = sL[tid];
+#pragma unroll
+        for (int g = 0; g < GT; ++g)
+            if (g == tid) {
+                ws[g * (2 + D)] = mrun[g];
+                ws[g * (2 + D) + 1] = lrun[g];
+            }
     }
+}
 
-    // ---- the last split of this kv-head merges all splits ------------------------------------
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) sFlag[0] = (atomicAdd(x.counters + ul, 1) == a.n_split - 1);
-    __syncthreads();
-    if (!sFlag[0]) return;
-    __threadfence();
-    float *sBV = reinterpret_cast<float *>(bV);         // B_V rows [D][rV] (bulk copy)
-    const bool bv_smem = ok;
-    if (bv_smem && tid == 0) {
-        mbar_arrive_expect_tx(bar_load, (uint32_t)(D * rV * 4));
-        bulk_load(sBV, a.basis[1] + (size_t)ul * D * rV, (uint32_t)(D * rV * 4), bar_load);
-    }
-    // all q-heads at once: split maxima and sums, per-head weights, then each thread (one channel
-    // j) sums its channel over the splits with several independent loads in flight, and the
-    // rank-space part is expanded through row j of B_V (read as float4 from L2)
+// One CTA per (q-head g, kv-head unit): log-sum-exp merge of the splits and the expansion of the
+// rank-space value sum through B_V^T. Thread j owns output channel j.
+__global__ void __launch_bounds__(MERGE_THREADS) decode_merge_kernel(DecodeArgs a) {
+    extern __shared__ float msm[];
+    const int G = a.G, rV = a.r[1], kV = a.k[1];
+    const int ldb = kV | 1;
+    float *sBV = msm;                                   // [D][ldb]
+    float *sW = sBV + D * ldb;                          // [max_splits] maxima, then weights
+    float *sL = sW + a.max_splits;                      // [max_splits] sums
+    float *sAcc = sL + a.max_splits;                    // [D]
+    float *sRed = sAcc + D;                             // [8]
+    const int g = blockIdx.x, ul = blockIdx.y;
+    const int seq = ul / a.H, h = ul % a.H;
+    const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
+    // B_V was written before the split kernel started: stage it while the splits finish
+    const float *B = a.basis[1] + (size_t)ul * D * rV;
+    for (int o = j; o < D * kV; o += MERGE_THREADS) sBV[(o / kV) * ldb + o % kV] = B[(size_t)(o / kV) * rV + o % kV];
+    griddep_wait();
+
+    // every load this thread needs is issued at once: the maxima and sums of splits j, j + 128,
+    // ... and its channel of the first MERGE_REG splits (one L2 round trip)
     const int ns = a.n_split, nsc = a.n_split_c;
-    const int stride = G * (2 + D);
-    const float *wsu = a.ws + (size_t)ul * a.max_splits * stride;
-    float *sMw = reinterpret_cast<float *>(bBh);        // [ns][G] maxima, then weights
-    float *sLs = sMw + ns * G;                          // [ns][G] sums
-    float *sAcc = sP;                                   // [G][D] rank-space sums
-    for (int i0 = tid; i0 < ns * G; i0 += 4 * TC_THREADS) {
-        float mv[4], lv[4];
+    const size_t stride = (size_t)G * (2 + D);
+    const float *wsu = a.ws + (size_t)ul * a.max_splits * stride + (size_t)g * (2 + D);
+    const float *col = wsu + 2 + j;
+    float v[MERGE_REG];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * TC_THREADS;
-            const float *pw = wsu + (size_t)(i / G) * stride + (i % G) * (2 + D);
-            mv[u] = i < ns * G ? __ldcg(pw) : 0.f;
-            lv[u] = i < ns * G ? __ldcg(pw + 1) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * TC_THREADS;
-            if (i < ns * G) {
-                sMw[i] = mv[u];
-                sLs[i] = lv[u];
-            }
-        }
+    for (int u = 0; u < MERGE_REG; ++u)
+        v[u] = (u < ns && (u >= nsc || j < kV)) ? __ldcg(col + u * stride) : 0.f;
+    float m = -CUDART_INF_F;
+    for (int s = j; s < ns; s += MERGE_THREADS) {
+        const float ms = __ldcg(wsu + s * stride);
+        sW[s] = ms;
+        sL[s] = __ldcg(wsu + s * stride + 1);
+        m = fmaxf(m, ms);
     }
+    m = warp_max_f(m);
+    if (lane == 0) sRed[warp] = m;
     __syncthreads();
-    for (int g = warp; g < G; g += 4) {
-        float m = -CUDART_INF_F;
-        for (int s2 = lane; s2 < ns; s2 += 32) m = fmaxf(m, sMw[s2 * G + g]);
-        m = warp_max_f(m);
-        float lsum = 0.f;
-        for (int s2 = lane; s2 < ns; s2 += 32) {
-            const float w = expf(sMw[s2 * G + g] - m);
-            sMw[s2 * G + g] = w;
-            lsum = fmaf(w, sLs[s2 * G + g], lsum);
-        }
-        lsum = warp_sum_f(lsum);
-        if (lane == 0) sRed[g] = lsum;
+    const float M = fmaxf(fmaxf(sRed[0], sRed[1]), fmaxf(sRed[2], sRed[3]));
+    float l = 0.f;
+    for (int s = j; s < ns; s += MERGE_THREADS) {
+        const float w = expf(sW[s] - M);
+        sW[s] = w;
+        l = fmaf(w, sL[s], l);
     }
+    l = warp_sum_f(l);
+    if (lane == 0) sRed[4 + warp] = l;
     __syncthreads();
-    {
-        const int j = tid;
-        float accr[GMAX], accw[GMAX];
+    const float lsum = (sRed[4] + sRed[5]) + (sRed[6] + sRed[7]);
+
+    float accr = 0.f, accw = 0.f;
 #pragma unroll
-        for (int g = 0; g < GMAX; ++g) accr[g] = accw[g] = 0.f;
-        for (int s0 = 0; s0 < ns; s0 += 16) {
-            float v[16][GMAX];
-#pragma unroll
-            for (int u = 0; u < 16; ++u)
-#pragma unroll
-                for (int g = 0; g < GMAX; ++g) {
-                    const int s2 = s0 + u;
-                    v[u][g] = (g < G && s2 < ns && (s2 >= nsc || j < kV))
-                                  ? __ldcg(wsu + (size_t)s2 * stride + g * (2 + D) + 2 + j)
-                                  : 0.f;
-                }
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int s2 = s0 + u;
-                if (s2 < ns) {
-#pragma unroll
-                    for (int g = 0; g < GMAX; ++g)
-                        if (g < G) {
-                            const float w = sMw[s2 * G + g];
-                            if (s2 < nsc) accr[g] = fmaf(w, v[u][g], accr[g]);
-                            else accw[g] = fmaf(w, v[u][g], accw[g]);
-                        }
-                }
-            }
+    for (int u = 0; u < MERGE_REG; ++u)
+        if (u < ns) {
+            if (u < nsc) accr = fmaf(sW[u], v[u], accr);
+            else accw = fmaf(sW[u], v[u], accw);
         }
-#pragma unroll
-        for (int g = 0; g < GMAX; ++g)
-            if (g < G) sAcc[g * D + j] = accr[g];
-        __syncthreads();
-        float o[GMAX];
-#pragma unroll
-        for (int g = 0; g < GMAX; ++g) o[g] = accw[g];
-        const bool bv_ok = bv_smem && __syncthreads_and(mbar_wait(bar_load, ph_load)) != 0;
-        const float *bvrow = bv_ok ? sBV + j * rV : a.basis[1] + ((size_t)ul * D + j) * rV;
-        for (int c4 = 0; c4 < kV / 4; ++c4) {
-            const float4 b4 = reinterpret_cast<const float4 *>(bvrow)[c4];
-#pragma unroll
-            for (int g = 0; g < GMAX; ++g)
-                if (g < G) {
-                    const float *ac = sAcc + g * D + 4 * c4;
-                    o[g] = fmaf(ac[0], b4.x, o[g]);
-                    o[g] = fmaf(ac[1], b4.y, o[g]);
-                    o[g] = fmaf(ac[2], b4.z, o[g]);
-                    o[g] = fmaf(ac[3], b4.w, o[g]);
-                }
+    for (int s = MERGE_REG; s < ns; ++s) {
+        if (s < nsc) {
+            if (j < kV) accr = fmaf(sW[s], __ldcg(col + s * stride), accr);
+        } else {
+            accw = fmaf(sW[s], __ldcg(col + s * stride), accw);
         }
-        for (int c = kV & ~3; c < kV; ++c) {
-            const float b1 = bvrow[c];
-#pragma unroll
-            for (int g = 0; g < GMAX; ++g)
-                if (g < G) o[g] = fmaf(sAcc[g * D + c], b1, o[g]);
-        }
-#pragma unroll
-        for (int g = 0; g < GMAX; ++g)
-            if (g < G) a.out[((size_t)seq * a.H * G + (size_t)h * G + g) * D + j] = o[g] / sRed[g];
     }
-    if (tid == 0) x.counters[ul] = 0;
+    sAcc[j] = accr;
+    __syncthreads();
+    float o = accw;
+    const float *br = sBV + j * ldb;
+    for (int c = 0; c < kV; ++c) o = fmaf(sAcc[c], br[c], o);
+    a.out[((size_t)seq * a.H * G + (size_t)h * G + g) * D + j] = o / lsum;
+}
+
+size_t merge_smem_bytes(int kV, int max_splits) {
+    return ((size_t)D * (kV | 1) + 2 * (size_t)max_splits + D + 8) * sizeof(float);
 }
 
 cudaError_t launch_decode_tc(const CUtensorMap *tmC, const CUtensorMap *tmB, const DecodeArgs &a,
                              const TcExtra &x, int n_units, cudaStream_t s) {
     const int esz = a.kv_dtype == ISKV_BF16 ? 2 : 4;
     const size_t smem = tc_smem_bytes(x.kblocks, a.r[1], esz);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)tc_smem_bytes(2, 128, 4));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
+    const size_t msmem = merge_smem_bytes(a.k[1], a.max_splits);
+    // opt-in dynamic shared memory, raised per device whenever a launch needs more
+    static size_t attr_tc[64] = {0}, attr_merge[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (smem > attr_tc[dev]) {
+        const void *fns[4] = {(const void *)decode_tc_kernel<1>, (const void *)decode_tc_kernel<2>,
+                              (const void *)decode_tc_kernel<4>, (const void *)decode_tc_kernel<8>};
+        for (const void *f : fns) {
+            e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        attr_tc[dev] = smem;
     }
-    decode_tc_kernel<<<dim3(a.n_split, n_units), TC_THREADS, smem, s>>>(*tmC, *tmB, a, x);
-    return cudaGetLastError();
+    if (msmem > attr_merge[dev]) {
+        e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)msmem);
+        if (e != cudaSuccess) return e;
+        attr_merge[dev] = msmem;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.n_split, n_units);
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    switch (a.G <= 1 ? 1 : a.G <= 2 ? 2 : a.G <= 4 ? 4 : 8) {
+    case 1: e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<1>, *tmC, *tmB, a, x); break;
+    case 2: e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<2>, *tmC, *tmB, a, x); break;
+    case 4: e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<4>, *tmC, *tmB, a, x); break;
+    default: e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<8>, *tmC, *tmB, a, x); break;
+    }
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(a.G, n_units);
+    cfg.blockDim = dim3(MERGE_THREADS);
+    cfg.dynamicSmemBytes = msmem;
+    return cudaLaunchKernelEx(&cfg, decode_merge_kernel, a);
 }
 
 }  // namespace iskv

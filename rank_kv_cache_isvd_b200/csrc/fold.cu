@@ -24,6 +24,7 @@ constexpr int JGRP = FT / JL;                 // column groups
 constexpr int NSLOT = 2 * JGRP;               // Jacobi slots (two per group)
 constexpr int SS = 132;                       // column stride of the Jacobi staging area
 constexpr float JACOBI_TOL = 4e-6f;           // rotate while |a.b| > tol |a| |b|
+constexpr float JACOBI_ZERO = 1e-10f;         // columns with |a|^2 <= this * ||Z||_F^2 are noise
 
 // shared memory (floats)
 constexpr int OFF_A = 0;                                  // F/E rows -> [P | B_old] -> F rows
@@ -62,9 +63,13 @@ __device__ __forceinline__ float group_sum(float v) {   // over the 16 lanes of 
 // |t| < sqrt(eps) c rounds to 1 while s = t, and a rounded rotation would inflate the norms by
 // t^2/2 every time (a systematic bias over thousands of rotations). With dc and s derived from
 // the same 1/sqrt(1 + t^2), c^2 + s^2 - 1 = O(eps t^2), so approximate reciprocals and square
-// roots keep tiny rotations norm-preserving.
-__device__ __forceinline__ void jparams(float g, float nx, float ny, float &t, float &s, float &dc) {
-    const bool doit = g * g > (JACOBI_TOL * JACOBI_TOL) * nx * ny;
+// roots keep tiny rotations norm-preserving. Pairs with a column whose squared norm is at most
+// `floor2` are left alone: such columns hold rounding noise only (when the core has more rows
+// than columns, Z^T has more columns than dimensions and the surplus converges to zero), and
+// their normalised inner products would otherwise stay O(1) for ever.
+__device__ __forceinline__ void jparams(float g, float nx, float ny, float floor2, float &t,
+                                        float &s, float &dc) {
+    const bool doit = g * g > (JACOBI_TOL * JACOBI_TOL) * nx * ny && fminf(nx, ny) > floor2;
     const float gg = doit ? g : 1.f;
     const float zeta = __fdividef(ny - nx, 2.f * gg);
     const float az = fminf(fabsf(zeta), 1e18f);
@@ -80,7 +85,7 @@ __device__ __forceinline__ void jparams(float g, float nx, float ny, float &t, f
 // products, their reductions and the rotation parameters of all pairs overlap (no branches).
 template <int HC, int RPL, int S>
 __device__ __forceinline__ void jcross(float (&xa)[HC][RPL], float (&xb)[HC][RPL], float (&na)[HC],
-                                       float (&nb)[HC], int &rotated) {
+                                       float (&nb)[HC], float floor2, int &rotated) {
     float g[HC];
 #pragma unroll
     for (int j = 0; j < HC; ++j) {
@@ -96,7 +101,7 @@ __device__ __forceinline__ void jcross(float (&xa)[HC][RPL], float (&xb)[HC][RPL
     for (int j = 0; j < HC; ++j) {
         const int jb = (j + S) % HC;
         float t, sn, dc;
-        jparams(g[j], na[j], nb[jb], t, sn, dc);
+        jparams(g[j], na[j], nb[jb], floor2, t, sn, dc);
 #pragma unroll
         for (int i = 0; i < RPL; ++i) {
             const float xi = xa[j][i], yi = xb[jb][i];
@@ -112,13 +117,13 @@ __device__ __forceinline__ void jcross(float (&xa)[HC][RPL], float (&xb)[HC][RPL
 // One rotation of the pair (x, y) within a slot (used in round 0 of a sweep).
 template <int RPL>
 __device__ __forceinline__ void jrot(float (&x)[RPL], float (&y)[RPL], float &nx, float &ny,
-                                     int &rotated) {
+                                     float floor2, int &rotated) {
     float g = 0.f;
 #pragma unroll
     for (int i = 0; i < RPL; ++i) g = fmaf(x[i], y[i], g);
     g = group_sum(g);
     float t, sn, dc;
-    jparams(g, nx, ny, t, sn, dc);
+    jparams(g, nx, ny, floor2, t, sn, dc);
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
         const float xi = x[i], yi = y[i];
@@ -133,15 +138,16 @@ __device__ __forceinline__ void jrot(float (&x)[RPL], float (&y)[RPL], float &nx
 template <int HC, int RPL, int S>
 struct JCrossAll {
     __device__ __forceinline__ static void run(float (&xa)[HC][RPL], float (&xb)[HC][RPL],
-                                               float (&na)[HC], float (&nb)[HC], int &rotated) {
-        jcross<HC, RPL, S>(xa, xb, na, nb, rotated);
-        JCrossAll<HC, RPL, S + 1>::run(xa, xb, na, nb, rotated);
+                                               float (&na)[HC], float (&nb)[HC], float floor2,
+                                               int &rotated) {
+        jcross<HC, RPL, S>(xa, xb, na, nb, floor2, rotated);
+        JCrossAll<HC, RPL, S + 1>::run(xa, xb, na, nb, floor2, rotated);
     }
 };
 template <int HC, int RPL>
 struct JCrossAll<HC, RPL, HC> {
     __device__ __forceinline__ static void run(float (&)[HC][RPL], float (&)[HC][RPL],
-                                               float (&)[HC], float (&)[HC], int &) {}
+                                               float (&)[HC], float (&)[HC], float, int &) {}
 };
 
 // Register-resident one-sided Jacobi on N <= 2 ng HC columns of length n <= 16 RPL, where
@@ -175,7 +181,23 @@ __device__ __noinline__ int jacobi_regs(const float *sB, const float *sC, int k,
             xb[j][i] = (pb != nullptr && row < n) ? pb[row] : 0.f;
         }
     }
+    // ||Z||_F^2 (invariant under the rotations) sets the level below which a column is noise
+    {
+        float f = 0.f;
+#pragma unroll
+        for (int j = 0; j < HC; ++j)
+#pragma unroll
+            for (int i = 0; i < RPL; ++i) f = fmaf(xa[j][i], xa[j][i], fmaf(xb[j][i], xb[j][i], f));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
+        if ((tid & 31) == 0) stage_n[tid >> 5] = f;
+    }
     __syncthreads();                          // inputs consumed: the staging area is free
+    float fro2 = 0.f;
+#pragma unroll
+    for (int w = 0; w < FW; ++w) fro2 += stage_n[w];
+    const float floor2 = JACOBI_ZERO * fro2;
+    __syncthreads();                          // the staged norms area is free again
     const int destA = grp == 0 ? 0 : (grp < ng - 1 ? grp + 1 : 2 * ng - 1);
     const int destB = grp == 0 ? 1 : ng + grp - 1;
     int sweeps = 0;
@@ -204,11 +226,11 @@ __device__ __noinline__ int jacobi_regs(const float *sB, const float *sC, int k,
                     for (int j1 = 0; j1 < HC; ++j1)
 #pragma unroll
                         for (int j2 = j1 + 1; j2 < HC; ++j2) {
-                            jrot<RPL>(xa[j1], xa[j2], na[j1], na[j2], rotated);
-                            jrot<RPL>(xb[j1], xb[j2], nb[j1], nb[j2], rotated);
+                            jrot<RPL>(xa[j1], xa[j2], na[j1], na[j2], floor2, rotated);
+                            jrot<RPL>(xb[j1], xb[j2], nb[j1], nb[j2], floor2, rotated);
                         }
                 }
-                JCrossAll<HC, RPL, 0>::run(xa, xb, na, nb, rotated);
+                JCrossAll<HC, RPL, 0>::run(xa, xb, na, nb, floor2, rotated);
             }
             if (ng > 1) {                     // move the slots for the next round
                 if (active) {
@@ -377,7 +399,7 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
             if (o < D * k) sC[(o % k) * LDS + o / k] = v[q];
         }
     }
-    if (tid < k) sSig[tid] = P.sigma[(size_t)unit * r + tid];
+    if (tid < k) sSig[tid] = P.sigma_in[(size_t)unit * r + tid];
     __syncthreads();
 
     // ---- step 1: S = F B (into Y[:, :k]) and the residual E = F - S B^T (in place) -----------
@@ -603,6 +625,13 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
         }
     }
     __syncthreads();
+    // columns at or below the Jacobi's noise level (it leaves them unrotated) count as zero
+    float zthr;
+    {
+        float f = 0.f;
+        for (int c = lane; c < NC; c += 32) f = fmaf(fmaxf(sNrm[c], 0.f), fmaxf(sNrm[c], 0.f), f);
+        zthr = sqrtf(JACOBI_ZERO * warp_sum(f));
+    }
     for (int c = tid; c < NC; c += FT) {
         const float s = sNrm[c];
         int rank = 0;
@@ -618,7 +647,7 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
         const int c = o / n, m = o % n;
         const int cs = sSel[c];
         const float s = sNrm[cs];
-        if (s > 1e-30f) stage[cs * SS + m] /= s;
+        if (s > zthr) stage[cs * SS + m] /= s;
     }
     __syncthreads();
     // exactly-zero singular values: complete H with orthonormal directions (rank-deficient input)
@@ -626,14 +655,14 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
         float *v = sScr;
         for (int c = 0; c < kp; ++c) {
             const int cs = sSel[c];
-            if (sNrm[cs] > 1e-30f) continue;
+            if (sNrm[cs] > zthr) continue;
             float *x = stage + cs * SS;
             for (int e = 0; e < n; ++e) {
                 for (int m = lane; m < n; m += 32) v[m] = (m == e) ? 1.f : 0.f;
                 __syncwarp();
                 for (int c2 = 0; c2 < kp; ++c2) {
                     const int cs2 = sSel[c2];
-                    if (c2 == c || (sNrm[cs2] <= 1e-30f && c2 > c)) continue;
+                    if (c2 == c || (sNrm[cs2] <= zthr && c2 > c)) continue;
                     const float *y = stage + cs2 * SS;
                     float d = 0.f;
                     for (int m = lane; m < n; m += 32) d = fmaf(y[m], v[m], d);
@@ -681,7 +710,7 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
     __syncthreads();
 
     // ---- outputs: Sigma+, H_top, B+ = [B P] H ------------------------------------------------
-    float *sig_out = P.sigma + (size_t)unit * r;
+    float *sig_out = P.sigma_out + (size_t)unit * r;
     for (int c = tid; c < r; c += FT) sig_out[c] = c < kp ? sNrm[sSel[c]] : 0.f;
     float *ht = P.htop + (size_t)unit * r * r;
     for (int o = tid; o < k * kp; o += FT) {

@@ -20,25 +20,34 @@ struct iskv_handle {
     int UL = 0;           // units per layer
     int R = 0;            // ring rows per unit
     int G = 1;
+    int NB = 2;           // buffers of basis / Sigma / H_top per path (ring indexed by fold number)
     long long n_max = 0;  // coordinate rows per unit
     int max_splits = 0;
     size_t esz = 2;
     float *coords[2] = {nullptr, nullptr};
-    float *basis[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
-    float *sigma[2] = {nullptr, nullptr};
+    float *basis[2] = {nullptr, nullptr};   // [NB][U][D][r]
+    float *sigma[2] = {nullptr, nullptr};   // [NB][U][r]
+    float *htop[2] = {nullptr, nullptr};    // [NB][U][r][r]
     void *ring[2] = {nullptr, nullptr};
-    float *htop[2] = {nullptr, nullptr};
     float2 *rope_cs = nullptr;
     float *ws = nullptr;
     int *status = nullptr;
     unsigned long long *stats = nullptr;  // fold statistics (3 counters)
-    int *counters = nullptr;              // decode split arrival counters [units per layer]
     bool tc = false;                      // tensor-core decode available for this shape
     CUtensorMap tmC;                      // key coordinates [U * n_max][r_K], 32 x 128 boxes
-    CUtensorMap tmB[2];                   // key bases (two buffers) [U * D][r_K]
+    CUtensorMap tmB;                      // key bases [NB * U * D][r_K]
+    // per layer
     std::vector<long long> t, nc;
-    std::vector<int> kcur[2];
-    std::vector<int> cur;  // which basis buffer is current, per layer
+    std::vector<int> kcur[2];             // ranks as of the last applied fold (what decode reads)
+    std::vector<long long> nf;            // folds launched (applied folds: nc / block)
+    std::vector<int> kf[2];               // ranks after the last launched fold
+    std::vector<int> fk;                  // [layer][NB][4]: k_K, kp_K, k_V, kp_V of fold j % NB
+    std::vector<unsigned char> on_side;   // [layer][NB]: fold j % NB ran on an internal stream
+    // look-ahead folding: internal streams and completion events
+    static constexpr int NS = 4;
+    cudaStream_t side[NS] = {nullptr, nullptr, nullptr, nullptr};
+    std::vector<cudaEvent_t> done;        // [layer][NB]
+    cudaEvent_t fork = nullptr;
     long long launches = 0;
 };
 
@@ -66,8 +75,7 @@ long long ncomp(long long t, int block, int window) {
 void free_all(iskv_handle *h) {
     for (int x = 0; x < 2; ++x) {
         cudaFree(h->coords[x]);
-        cudaFree(h->basis[x][0]);
-        cudaFree(h->basis[x][1]);
+        cudaFree(h->basis[x]);
         cudaFree(h->sigma[x]);
         cudaFree(h->ring[x]);
         cudaFree(h->htop[x]);
@@ -76,7 +84,11 @@ void free_all(iskv_handle *h) {
     cudaFree(h->ws);
     cudaFree(h->status);
     cudaFree(h->stats);
-    cudaFree(h->counters);
+    for (cudaEvent_t e : h->done)
+        if (e) cudaEventDestroy(e);
+    if (h->fork) cudaEventDestroy(h->fork);
+    for (int i = 0; i < iskv_handle::NS; ++i)
+        if (h->side[i]) cudaStreamDestroy(h->side[i]);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -119,37 +131,53 @@ bool valid_layer(const iskv_handle *h, int layer) {
     return layer >= 0 && layer < h->cfg.n_layers;
 }
 
-int fold_layers(iskv_handle *h, int l0, int nl, cudaStream_t s) {
+float *basis_buf(const iskv_handle *h, int x, int i) {
+    return h->basis[x] + (size_t)i * h->U * D * rank_of(h, x);
+}
+float *sigma_buf(const iskv_handle *h, int x, int i) {
+    return h->sigma[x] + (size_t)i * h->U * rank_of(h, x);
+}
+float *htop_buf(const iskv_handle *h, int x, int i) {
+    const size_t r = (size_t)rank_of(h, x);
+    return h->htop[x] + (size_t)i * h->U * r * r;
+}
+// buffer of the basis / Sigma produced by the last applied fold
+int current_buffer(const iskv_handle *h, int layer) {
+    return (int)((h->nc[layer] / h->cfg.block) % h->NB);
+}
+int *fold_ranks(iskv_handle *h, int layer, long long j) {
+    return &h->fk[((size_t)layer * h->NB + (size_t)(j % h->NB)) * 4];
+}
+
+// Launches fold j (rows j*b .. j*b+b-1) of layers l0 .. l0+nl-1 on stream s: projection,
+// residual basis, core SVD, basis update into buffer (j+1) % NB, Sigma into (j+1) % NB, H_top
+// into j % NB and the new rows' coordinates. The history is rotated when the fold is applied.
+int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
     const iskv_config &c = h->cfg;
-    const long long nc = h->nc[l0];
+    // the new rows' coordinates go to rows j*b .. j*b+b-1, which must lie within n_max
+    if ((j + 1) * c.block > h->n_max) return ISKV_ERR_CAPACITY;
+    const int bi = (int)(j % h->NB), bo = (int)((j + 1) % h->NB);
     FoldArgs fa;
-    RotArgs ra;
     memset(&fa, 0, sizeof(fa));
-    memset(&ra, 0, sizeof(ra));
-    const int cur = h->cur[l0];
     for (int x = 0; x < 2; ++x) {
         const int r = rank_of(h, x);
-        const int k = h->kcur[x][l0];
+        const int k = h->kf[x][l0];
         const int p = c.block < D - k ? c.block : D - k;
         const int kp = r < k + p ? r : k + p;
         FoldPath &fp = fa.path[x];
         fp.ring = h->ring[x];
-        fp.basis_in = h->basis[x][cur];
-        fp.basis_out = h->basis[x][cur ^ 1];
-        fp.sigma = h->sigma[x];
+        fp.basis_in = basis_buf(h, x, bi);
+        fp.basis_out = basis_buf(h, x, bo);
+        fp.sigma_in = sigma_buf(h, x, bi);
+        fp.sigma_out = sigma_buf(h, x, bo);
         fp.coords = h->coords[x];
-        fp.htop = h->htop[x];
+        fp.htop = htop_buf(h, x, bi);
         fp.r = r;
         fp.k = k;
         fp.p = p;
         fp.kp = kp;
-        RotPath &rp = ra.path[x];
-        rp.coords = h->coords[x];
-        rp.htop = h->htop[x];
-        rp.r = r;
-        rp.k = k;
-        rp.kp = kp;
     }
+    const long long nc = j * c.block;
     fa.unit0 = l0 * h->UL;
     fa.n_c = nc;
     fa.n_max = h->n_max;
@@ -160,17 +188,103 @@ int fold_layers(iskv_handle *h, int l0, int nl, cudaStream_t s) {
     fa.status = h->status;
     fa.stats = h->stats;
     if (launch_fold(fa, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
-    h->launches += 1 + (nc > 0 ? 1 : 0);
-    ra.unit0 = l0 * h->UL;
-    ra.n_old = nc;
-    ra.n_max = h->n_max;
-    ra.stale = c.rotate_history ? 0 : 1;
-    if (launch_rotate(ra, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+    h->launches += 1;
+    for (int l = l0; l < l0 + nl; ++l) {
+        int *f = fold_ranks(h, l, j);
+        f[0] = fa.path[0].k;
+        f[1] = fa.path[0].kp;
+        f[2] = fa.path[1].k;
+        f[3] = fa.path[1].kp;
+        h->kf[0][l] = fa.path[0].kp;
+        h->kf[1][l] = fa.path[1].kp;
+        h->nf[l] = j + 1;
+    }
+    return ISKV_OK;
+}
+
+// Applies the oldest pending fold of layers l0 .. l0+nl-1 on stream s: launches it here if no
+// earlier call did, else makes s wait for it; then rotates the history C[0:n_c] <- C H_top and
+// advances n_c, the ranks and the current buffer.
+int apply_fold(iskv_handle *h, int l0, int nl, cudaStream_t s) {
+    const iskv_config &c = h->cfg;
+    const long long j = h->nc[l0] / c.block;
+    const int bi = (int)(j % h->NB);
+    if (h->nf[l0] <= j) {
+        const int rc = launch_fold_j(h, l0, nl, j, s);
+        if (rc != ISKV_OK) return rc;
+        for (int l = l0; l < l0 + nl; ++l) h->on_side[(size_t)l * h->NB + bi] = 0;
+    } else if (h->on_side[(size_t)l0 * h->NB + bi]) {
+        if (cudaStreamWaitEvent(s, h->done[(size_t)l0 * h->NB + bi], 0) != cudaSuccess)
+            return ISKV_ERR_CUDA;
+        for (int l = l0; l < l0 + nl; ++l) h->on_side[(size_t)l * h->NB + bi] = 0;
+    }
+    const int *f = fold_ranks(h, l0, j);
+    const long long nc = h->nc[l0];
+    if (nc > 0) {
+        RotArgs ra;
+        memset(&ra, 0, sizeof(ra));
+        for (int x = 0; x < 2; ++x) {
+            RotPath &rp = ra.path[x];
+            rp.coords = h->coords[x];
+            rp.htop = htop_buf(h, x, bi);
+            rp.r = rank_of(h, x);
+            rp.k = f[2 * x];
+            rp.kp = f[2 * x + 1];
+        }
+        ra.unit0 = l0 * h->UL;
+        ra.n_old = nc;
+        ra.n_max = h->n_max;
+        ra.stale = c.rotate_history ? 0 : 1;
+        if (launch_rotate(ra, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+        h->launches += 1;
+    }
     for (int l = l0; l < l0 + nl; ++l) {
         h->nc[l] += c.block;
-        h->cur[l] ^= 1;
-        for (int x = 0; x < 2; ++x) h->kcur[x][l] = fa.path[x].kp;
+        h->kcur[0][l] = f[1];
+        h->kcur[1][l] = f[3];
     }
+    return ISKV_OK;
+}
+
+// Look-ahead: starts every fold whose block is complete on an internal stream (forked from s),
+// as far as the buffer ring allows and only for blocks that the window can still release within
+// max_tokens (the others are never applied, and their coordinates would not fit in n_max rows);
+// apply_fold() later joins it back.
+int launch_ahead(iskv_handle *h, int l0, int nl, cudaStream_t s) {
+    const iskv_config &c = h->cfg;
+    cudaStream_t side = h->side[l0 % iskv_handle::NS];
+    bool forked = false;
+    while ((h->nf[l0] + 1) * c.block <= h->t[l0] && (h->nf[l0] + 1) * c.block <= h->n_max &&
+           h->nf[l0] <= h->nc[l0] / c.block + h->NB - 2) {
+        const long long j = h->nf[l0];
+        const int bi = (int)(j % h->NB);
+        if (!forked) {
+            if (cudaEventRecord(h->fork, s) != cudaSuccess ||
+                cudaStreamWaitEvent(side, h->fork, 0) != cudaSuccess)
+                return ISKV_ERR_CUDA;
+            forked = true;
+        }
+        const int rc = launch_fold_j(h, l0, nl, j, side);
+        if (rc != ISKV_OK) return rc;
+        for (int l = l0; l < l0 + nl; ++l) {
+            if (cudaEventRecord(h->done[(size_t)l * h->NB + bi], side) != cudaSuccess)
+                return ISKV_ERR_CUDA;
+            h->on_side[(size_t)l * h->NB + bi] = 1;
+        }
+    }
+    return ISKV_OK;
+}
+
+// Makes s wait for every fold still running on an internal stream.
+int join_all(iskv_handle *h, cudaStream_t s) {
+    for (int l = 0; l < h->cfg.n_layers; ++l)
+        for (int i = 0; i < h->NB; ++i) {
+            unsigned char &f = h->on_side[(size_t)l * h->NB + i];
+            if (!f) continue;
+            if (cudaStreamWaitEvent(s, h->done[(size_t)l * h->NB + i], 0) != cudaSuccess)
+                return ISKV_ERR_CUDA;
+            f = 0;
+        }
     return ISKV_OK;
 }
 
@@ -229,11 +343,18 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         h->esz = c.kv_dtype == ISKV_BF16 ? 2 : 4;
         const long long ctiles = (h->n_max + DEC_TILE - 1) / DEC_TILE;
         h->max_splits = (int)(ctiles + (h->R + DEC_TILE - 1) / DEC_TILE + 1);
+        // folds in flight ahead of their trigger: at most window / block + 1 (look-ahead only)
+        h->NB = c.lookahead_folds ? c.window / c.block + 3 : 2;
         h->t.assign(c.n_layers, 0);
         h->nc.assign(c.n_layers, 0);
-        h->cur.assign(c.n_layers, 0);
-        h->kcur[0].assign(c.n_layers, 0);
-        h->kcur[1].assign(c.n_layers, 0);
+        h->nf.assign(c.n_layers, 0);
+        for (int x = 0; x < 2; ++x) {
+            h->kcur[x].assign(c.n_layers, 0);
+            h->kf[x].assign(c.n_layers, 0);
+        }
+        h->fk.assign((size_t)c.n_layers * h->NB * 4, 0);
+        h->on_side.assign((size_t)c.n_layers * h->NB, 0);
+        h->done.assign((size_t)c.n_layers * h->NB, nullptr);
     } catch (...) {
         delete h;
         return ISKV_ERR_CUDA;
@@ -250,28 +371,30 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
     const size_t U = (size_t)h->U;
     for (int x = 0; x < 2; ++x) {
         const size_t r = (size_t)rank_of(h, x);
+        const size_t nb = (size_t)h->NB;
         alloc((void **)&h->coords[x], U * (size_t)h->n_max * r * sizeof(float));
-        alloc((void **)&h->basis[x][0], U * D * r * sizeof(float));
-        alloc((void **)&h->basis[x][1], U * D * r * sizeof(float));
-        alloc((void **)&h->sigma[x], U * r * sizeof(float));
+        alloc((void **)&h->basis[x], nb * U * D * r * sizeof(float));
+        alloc((void **)&h->sigma[x], nb * U * r * sizeof(float));
         alloc(&h->ring[x], U * (size_t)h->R * D * h->esz);
-        alloc((void **)&h->htop[x], U * r * r * sizeof(float));
+        alloc((void **)&h->htop[x], nb * U * r * r * sizeof(float));
     }
     if (c.rope) alloc((void **)&h->rope_cs, (size_t)c.max_tokens * DH * sizeof(float2));
     alloc((void **)&h->ws, (size_t)h->UL * h->max_splits * h->G * (2 + D) * sizeof(float));
     alloc((void **)&h->status, sizeof(int));
     alloc((void **)&h->stats, 4 * sizeof(unsigned long long));
-    alloc((void **)&h->counters, (size_t)h->UL * sizeof(int));
     if (ok) {
         for (int x = 0; x < 2; ++x) {
-            const size_t r = (size_t)rank_of(h, x);
-            ok = ok && cudaMemset(h->basis[x][0], 0, U * D * r * sizeof(float)) == cudaSuccess;
-            ok = ok && cudaMemset(h->basis[x][1], 0, U * D * r * sizeof(float)) == cudaSuccess;
-            ok = ok && cudaMemset(h->sigma[x], 0, U * r * sizeof(float)) == cudaSuccess;
+            const size_t r = (size_t)rank_of(h, x), nb = (size_t)h->NB;
+            ok = ok && cudaMemset(h->basis[x], 0, nb * U * D * r * sizeof(float)) == cudaSuccess;
+            ok = ok && cudaMemset(h->sigma[x], 0, nb * U * r * sizeof(float)) == cudaSuccess;
         }
         ok = ok && cudaMemset(h->status, 0, sizeof(int)) == cudaSuccess;
         ok = ok && cudaMemset(h->stats, 0, 4 * sizeof(unsigned long long)) == cudaSuccess;
-        ok = ok && cudaMemset(h->counters, 0, (size_t)h->UL * sizeof(int)) == cudaSuccess;
+        for (int i = 0; ok && i < iskv_handle::NS; ++i)
+            ok = cudaStreamCreateWithFlags(&h->side[i], cudaStreamNonBlocking) == cudaSuccess;
+        ok = ok && cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming) == cudaSuccess;
+        for (size_t i = 0; ok && i < h->done.size(); ++i)
+            ok = cudaEventCreateWithFlags(&h->done[i], cudaEventDisableTiming) == cudaSuccess;
         if (ok && c.rope)
             ok = launch_rope_table(h->rope_cs, c.max_tokens, c.rope_theta, 0) == cudaSuccess;
         ok = ok && cudaDeviceSynchronize() == cudaSuccess;
@@ -287,13 +410,16 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
     int major = 0;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, h->device);
     memset(&h->tmC, 0, sizeof(h->tmC));
-    memset(h->tmB, 0, sizeof(h->tmB));
-    if (major == 10 && c.rank_k % 4 == 0 && c.rank_k <= 64 && c.rank_v % 4 == 0) {
+    memset(&h->tmB, 0, sizeof(h->tmB));
+    // (the value-sum reduction of a compressed tile lives in the key-coordinate lo buffer:
+    //  G x next-power-of-two(r_V / 4) quads must fit in it)
+    const int nq_v = c.rank_v / 4, nqp_v = nq_v <= 8 ? 8 : nq_v <= 16 ? 16 : 32;
+    if (major == 10 && c.rank_k % 4 == 0 && c.rank_k <= 64 && c.rank_v % 4 == 0 &&
+        h->G * nqp_v <= 128 * ((c.rank_k + 31) / 32)) {
         bool m_ok = true;
         if (h->n_max > 0) {
             m_ok = make_map(&h->tmC, h->coords[0], c.rank_k, (long long)h->U * h->n_max) &&
-                   make_map(&h->tmB[0], h->basis[0][0], c.rank_k, (long long)h->U * D) &&
-                   make_map(&h->tmB[1], h->basis[0][1], c.rank_k, (long long)h->U * D);
+                   make_map(&h->tmB, h->basis[0], c.rank_k, (long long)h->NB * h->U * D);
         }
         h->tc = m_ok;
     }
@@ -318,7 +444,7 @@ int iskv_append_block(iskv_handle *h, int layer, const void *k_rows, const void 
     const int l0 = layer < 0 ? 0 : layer;
     const int nl = layer < 0 ? c.n_layers : 1;
     for (int l = l0; l < l0 + nl; ++l)
-        if (h->t[l] != h->t[l0] || h->nc[l] != h->nc[l0] || h->cur[l] != h->cur[l0])
+        if (h->t[l] != h->t[l0] || h->nc[l] != h->nc[l0] || h->nf[l] != h->nf[l0])
             return ISKV_ERR_INVALID_ARG;
     if (h->t[l0] + m > c.max_tokens) return ISKV_ERR_CAPACITY;
     DeviceGuard g(h->device);
@@ -347,7 +473,11 @@ int iskv_append_block(iskv_handle *h, int layer, const void *k_rows, const void 
         done += chunk;
         for (int l = l0; l < l0 + nl; ++l) h->t[l] = t;
         if (t - h->nc[l0] >= (long long)h->R) {
-            const int rc = fold_layers(h, l0, nl, s);
+            const int rc = apply_fold(h, l0, nl, s);
+            if (rc != ISKV_OK) return rc;
+        }
+        if (c.lookahead_folds) {
+            const int rc = launch_ahead(h, l0, nl, s);
             if (rc != ISKV_OK) return rc;
         }
     }
@@ -361,12 +491,12 @@ int iskv_decode_attn(iskv_handle *h, int layer, const float *q, float *out, iskv
     const iskv_config &c = h->cfg;
     DecodeArgs da;
     memset(&da, 0, sizeof(da));
-    const int cur = h->cur[layer];
+    const int cur = current_buffer(h, layer);
     for (int x = 0; x < 2; ++x) {
         const size_t r = (size_t)rank_of(h, x);
         const size_t u0 = (size_t)layer * h->UL;
         da.coords[x] = h->coords[x] + u0 * (size_t)h->n_max * r;
-        da.basis[x] = h->basis[x][cur] + u0 * D * r;
+        da.basis[x] = basis_buf(h, x, cur) + u0 * D * r;
         da.ring[x] = static_cast<const char *>(h->ring[x]) + u0 * (size_t)h->R * D * h->esz;
         da.r[x] = (int)r;
         da.k[x] = h->kcur[x][layer];
@@ -398,12 +528,11 @@ int iskv_decode_attn(iskv_handle *h, int layer, const float *q, float *out, iskv
         TcExtra x;
         x.kblocks = (c.rank_k + 31) / 32;
         x.row0 = (long long)layer * h->UL * h->n_max;
-        x.brow0 = layer * h->UL * D;
-        x.counters = h->counters;
+        x.brow0 = (cur * h->U + layer * h->UL) * D;
         x.status = h->status;
-        if (launch_decode_tc(&h->tmC, &h->tmB[cur], da, x, h->UL, s) != cudaSuccess)
+        if (launch_decode_tc(&h->tmC, &h->tmB, da, x, h->UL, s) != cudaSuccess)
             return ISKV_ERR_CUDA;
-        h->launches += 1;
+        h->launches += 2;
         return ISKV_OK;
     }
     if (launch_decode(da, h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
@@ -420,7 +549,7 @@ int iskv_reconstruct(iskv_handle *h, int layer, int which, int apply_rope, float
     const size_t u0 = (size_t)layer * h->UL;
     ReconArgs ra;
     ra.coords = h->coords[which] + u0 * (size_t)h->n_max * r;
-    ra.basis = h->basis[which][h->cur[layer]] + u0 * D * r;
+    ra.basis = basis_buf(h, which, current_buffer(h, layer)) + u0 * D * r;
     ra.ring = static_cast<const char *>(h->ring[which]) + u0 * (size_t)h->R * D * h->esz;
     ra.rope_cs = h->rope_cs;
     ra.out = out;
@@ -453,10 +582,11 @@ int iskv_get_factors(iskv_handle *h, int layer, int seq, int kv_head, int which,
         cudaMemcpyAsync(coords, h->coords[which] + u * (size_t)h->n_max * r,
                         (size_t)nc * r * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
         return ISKV_ERR_CUDA;
-    if (basis && cudaMemcpyAsync(basis, h->basis[which][h->cur[layer]] + u * D * r,
+    const int cur = current_buffer(h, layer);
+    if (basis && cudaMemcpyAsync(basis, basis_buf(h, which, cur) + u * D * r,
                                  D * r * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
         return ISKV_ERR_CUDA;
-    if (sigma && cudaMemcpyAsync(sigma, h->sigma[which] + u * r, r * sizeof(float),
+    if (sigma && cudaMemcpyAsync(sigma, sigma_buf(h, which, cur) + u * r, r * sizeof(float),
                                  cudaMemcpyDeviceToDevice, s) != cudaSuccess)
         return ISKV_ERR_CUDA;
     if (k_out) *k_out = h->kcur[which][layer];
@@ -464,15 +594,22 @@ int iskv_get_factors(iskv_handle *h, int layer, int seq, int kv_head, int which,
     return ISKV_OK;
 }
 
+int iskv_join(iskv_handle *h, iskv_stream_t stream) {
+    if (!h) return ISKV_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    return join_all(h, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int iskv_reset(iskv_handle *h, iskv_stream_t stream) {
     if (!h) return ISKV_ERR_INVALID_ARG;
     DeviceGuard g(h->device);
+    const int rc = join_all(h, reinterpret_cast<cudaStream_t>(stream));
+    if (rc != ISKV_OK) return rc;
     for (int l = 0; l < h->cfg.n_layers; ++l) {
         h->t[l] = 0;
         h->nc[l] = 0;
-        h->cur[l] = 0;
-        h->kcur[0][l] = 0;
-        h->kcur[1][l] = 0;
+        h->nf[l] = 0;
+        for (int x = 0; x < 2; ++x) h->kcur[x][l] = h->kf[x][l] = 0;
     }
     if (cudaMemsetAsync(h->status, 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)) !=
         cudaSuccess)
@@ -489,6 +626,7 @@ int iskv_fold_stats(iskv_handle *h, iskv_stream_t stream, int *max_sweeps_out,
     DeviceGuard g(h->device);
     unsigned long long v[4] = {0, 0, 0, 0};
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (join_all(h, s) != ISKV_OK) return ISKV_ERR_CUDA;
     if (cudaMemcpyAsync(v, h->stats, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return ISKV_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return ISKV_ERR_CUDA;
@@ -524,6 +662,7 @@ int iskv_sync_status(iskv_handle *h, iskv_stream_t stream) {
     DeviceGuard g(h->device);
     int st = 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (join_all(h, s) != ISKV_OK) return ISKV_ERR_CUDA;
     if (cudaMemcpyAsync(&st, h->status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return ISKV_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return ISKV_ERR_CUDA;

@@ -24,7 +24,8 @@ struct FoldPath {
     const void *ring;       // [units][R][D] kv dtype
     const float *basis_in;  // [units][D][r]
     float *basis_out;       // [units][D][r]
-    float *sigma;           // [units][r]
+    const float *sigma_in;  // [units][r] Sigma before the fold (read when k > 0)
+    float *sigma_out;       // [units][r] Sigma after the fold
     float *coords;          // [units][n_max][r]
     float *htop;            // [units][r][r]
     int r, k, p, kp;        // rank budget, rank before, residual basis size, rank after
@@ -107,8 +108,7 @@ struct ReconArgs {
 struct TcExtra {
     int kblocks;            // 32-column K-blocks of the key coordinates (ceil(r_K / 32))
     long long row0;         // first coordinate row of this layer in the coordinate tensor map
-    int brow0;              // first basis row of this layer in the basis tensor map
-    int *counters;          // [units of the layer] split arrival counters (self-resetting)
+    int brow0;              // first basis row of this layer (current buffer) in the basis map
     int *status;
 };
 

@@ -86,10 +86,14 @@ def _snapshot(cache, wl):
     return snap
 
 
-@pytest.mark.parametrize("variant", ["gapped", "literal"])
-def test_fold_one_step_parity(variant):
-    """Each GPU fold, started from the GPU's own state, matches the oracle's fold."""
-    wl = sub(W1, n_kv_heads=3, n_q_heads=12, tokens=1100)
+@pytest.mark.parametrize("variant,wl_id", [("gapped", 1), ("literal", 1), ("gapped", 3),
+                                            ("literal", 3)])
+def test_fold_one_step_parity(variant, wl_id):
+    """Each GPU fold, started from the GPU's own state, matches the oracle's fold. With the
+    Qwen3-shaped schedule (b=128, r_K=32, r_V=64) the core has more rows than columns once k > 0
+    (k + b > k + p = d), so its transpose has surplus columns that converge to zero."""
+    base = syn.WORKLOADS[wl_id]
+    wl = sub(base, batch=1, n_layers=1, n_kv_heads=3, n_q_heads=12, tokens=1100)
     kd, kv, vd, vv = workload_arrays(wl, variant=variant)
     cache = make_cache(wl)
     t, folds, worst = 0, 0, {"sigma": 0.0, "proj": 0.0, "recon": 0.0}
@@ -311,3 +315,101 @@ def test_decode_is_repeatable_and_graph_capturable():
     torch.cuda.synchronize()
     assert torch.equal(out, o1)
     assert cache.status() == 0
+
+
+def _stream_tokens(cache, K, V, Q, t0, t1, out, stream=None):
+    for t in range(t0, t1):
+        cache.append(0, K[:, :, t:t + 1].contiguous(), V[:, :, t:t + 1].contiguous(), stream)
+        cache.decode(0, Q[t], out[t], stream)
+
+
+def test_lookahead_folds_match_synchronous_folds_bitwise():
+    """Folds started early on internal streams give exactly the decode outputs and factors of
+    folds run at the trigger: every token's decode is compared bit for bit."""
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=1200)
+    kd, kv, vd, vv = workload_arrays(wl)
+    K, V = to_device(kd[0]), to_device(vd[0])
+    Q = torch.from_numpy(syn.queries(23, (wl.tokens, 1, 8, 128))).cuda()
+    outs = []
+    for la in (False, True):
+        cache = make_cache(wl, lookahead_folds=la)
+        out = torch.empty_like(Q)
+        _stream_tokens(cache, K, V, Q, 0, wl.tokens, out)
+        assert cache.status() == 0
+        fac = [cache.factors(0, 0, h, x) for h in range(2) for x in (0, 1)]
+        outs.append((out, fac, cache.launches()))
+        cache.close()
+    (o0, f0, n0), (o1, f1, n1) = outs
+    assert torch.equal(o0, o1)
+    for a, b in zip(f0, f1):
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+        assert a[3:] == b[3:]
+    # the early folds of blocks the window never released ran too
+    assert n1 >= n0
+
+
+def test_lookahead_stream_captures_into_a_graph():
+    """A reset + 700-token append/decode segment with early folds, captured once (joined before
+    the capture ends) and replayed twice, reproduces the eager synchronous outputs."""
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=700)
+    kd, kv, vd, vv = workload_arrays(wl)
+    K, V = to_device(kd[0]), to_device(vd[0])
+    Q = torch.from_numpy(syn.queries(29, (wl.tokens, 1, 8, 128))).cuda()
+    ref_cache = make_cache(wl)
+    ref = torch.empty_like(Q)
+    _stream_tokens(ref_cache, K, V, Q, 0, wl.tokens, ref)
+    torch.cuda.synchronize()
+    cache = make_cache(wl, lookahead_folds=True)
+    out = torch.empty_like(Q)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        _stream_tokens(cache, K, V, Q, 0, wl.tokens, out, s)    # eager warm-up
+        cache.reset(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        cache.reset(s)
+        _stream_tokens(cache, K, V, Q, 0, wl.tokens, out, s)
+        cache.join(s)
+    for _ in range(2):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    assert cache.status(s) == 0
+
+
+def test_long_context_layer_sampled_units():
+    """Full-size Qwen3-8B-shaped layer as the benchmark's long-context decode runs it (batch 8 x
+    8 kv-heads, 32 q-heads, b=128, w=256, r_K=32, r_V=64, 32768 tokens in one append, rows drawn
+    on the GPU): every output is finite and the q-heads of three sampled (sequence, kv-head)
+    units match the oracle run on those units' rows alone."""
+    wl = syn.WORKLOADS[3]
+    S, H, T, QH, G = wl.batch, wl.n_kv_heads, wl.tokens, wl.n_q_heads, wl.group
+    cache = make_cache(sub(wl, n_layers=1))
+    K = torch.empty((S, H, T, 128), dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+    for sq in range(S):
+        for h in range(H):
+            K[sq, h] = syn.device_rows(wl, sq, 0, h, 0)
+            V[sq, h] = syn.device_rows(wl, sq, 0, h, 1)
+    cache.append(0, K, V)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(12345)
+    q = torch.randn((S, QH, 128), generator=gen, device="cuda")
+    out = cache.decode(0, q)
+    assert cache.status() == 0 and bool(torch.isfinite(out).all())
+    assert cache.tokens(0) == T
+    for sq, h in ((0, 0), (3, 5), (7, 7)):
+        orc = OracleCache(1, 1, 1, G, 128, wl.rank_k, wl.rank_v, wl.block, wl.window, rope=True,
+                          rope_theta=wl.rope_theta)
+        kv = K[sq, h].float().cpu().numpy().astype(np.float64)[None, None]
+        vv = V[sq, h].float().cpu().numpy().astype(np.float64)[None, None]
+        orc.append(0, kv, vv)
+        qs = q[sq, h * G:(h + 1) * G].cpu().numpy().astype(np.float64)[None]
+        ref = orc.decode(0, qs)
+        got = out[sq, h * G:(h + 1) * G].cpu().numpy()[None]
+        err = max_head_rel_err(got, ref)
+        print(f"\nunit (seq {sq}, kv-head {h}): attention rel err {err:.3e}")
+        assert err <= ATTN_TOL
+    cache.close()
