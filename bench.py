@@ -6,7 +6,8 @@ r_K=32, r_V=48, RoPE theta=5e5, bf16 rows, batch 1 per GPU).
 One step = one pass of the whole hot path over one sequence batch: for each of the 4096 tokens,
 append its K/V rows (window append, and a block-incremental fold of every path whenever the window
 releases a block: 60 folds x 8 heads x 2 paths = 960 head-block updates) and run decode attention
-of the 32 q-heads over the compressed history plus the exact window. Folds start on an internal
+of the 32 q-heads over the compressed history plus the exact window (one iskv_append_decode call
+per token: the decode kernel stores the new rows in the window itself). Folds start on an internal
 stream as soon as their block is complete and join the decode stream when the window releases the
 block (every decode sees the same state as with folds at the trigger); the four folds of blocks
 still inside the window at the end of the stream are joined at the end of the step. The step's
@@ -54,8 +55,9 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--sample-every", type=int, default=16,
                    help="decode calls between event-timed samples inside the graph")
-    p.add_argument("--profile-case", action="store_true",
-                   help="run the short program used for profiler captures instead of the bench")
+    p.add_argument("--profile-case", choices=["short", "long"], nargs="?", const="short",
+                   help="run a short program for profiler captures instead of the bench: "
+                        "'short' = the bench workload, 'long' = the long-context layer")
     return p.parse_args()
 
 
@@ -228,6 +230,12 @@ def run_reference(args, rank: int):
 # ---------------------------------------------------------------------------------------------
 WL_LONG = syn.WORKLOADS[3]
 
+# DRAM bytes (read + write) of one launch of the split kernel as ncu counted them for the current
+# kernel: the t = 4096 launch of the bench workload (--profile-case) and the long-context launch
+# (--profile-case long). Set to None whenever the kernel changes until it is captured again.
+TRAFFIC_T4096 = 13_208_064
+TRAFFIC_LONG = 832_619_264
+
 
 def long_context_decode(args, dev, flush, calls: int = 10):
     """Decode over a long compressed history: one layer of the Qwen3-8B-shaped workload (batch 8
@@ -372,11 +380,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     def step(stream_handle: int, timed_events: bool):
         iskv.check(iskv.iskv_reset(h, stream_handle))
         for t in range(T):
-            iskv.check(iskv.iskv_append_block(h, 0, kb + t * krow, vb + t * krow, 1, stream_handle))
             dm = dec_set.get(t) if timed_events else None
             if dm:
                 rec(dm[0], stream_handle)
-            iskv.check(iskv.iskv_decode_attn(h, 0, qb + t * qrow, ob + t * qrow, stream_handle))
+            # one decode step: append token t's rows (the decode kernel stores them) and attend
+            iskv.check(iskv.iskv_append_decode(h, 0, kb + t * krow, vb + t * krow, qb + t * qrow,
+                                               ob + t * qrow, stream_handle))
             if dm:
                 rec(dm[1], stream_handle)
         # folds started ahead for blocks the window has not released yet join the step here
@@ -475,7 +484,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "graph": "the step's C-ABI calls captured once into a CUDA graph"},
         "roofline": {"bound": "hbm", "kernel": "decode attention (split + combine)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
+                     "frac": achieved / hbm, "traffic": TRAFFIC_T4096,
+                     "traffic_launch": ("ncu count of the t = 4096 launch (--profile-case); its "
+                                        f"algorithmic bytes are {decode_bytes(WL.tokens)}"),
                      "peak_source": f"{which} MEASURED_PEAKS hbm_gbs",
                      "bytes_per_launch_mean": float(np.mean(dec_bytes)),
                      "launch_us_mean": 1e3 * float(np.mean(dec_ms))},
@@ -490,7 +501,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "bound": "hbm", "kernel": "decode attention (split + combine)",
             "workload": f"{WL_LONG.name}: one layer at t = {WL_LONG.tokens}",
             "achieved": long_bytes / (long_us / 1e6) / 1e9, "peak": hbm, "unit": "GB/s",
-            "frac": long_bytes / (long_us / 1e6) / 1e9 / hbm, "traffic": None,
+            "frac": long_bytes / (long_us / 1e6) / 1e9 / hbm, "traffic": TRAFFIC_LONG,
             "bytes_per_launch": long_bytes, "launch_us": long_us},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h),
@@ -535,6 +546,14 @@ def run_profile_case():
 
 def main():
     args = parse()
+    if args.profile_case == "long":
+        import torch
+        dev = torch.device("cuda", 0)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        args.warmup = 1
+        us, nbytes = long_context_decode(args, dev, flush, calls=2)
+        print(json.dumps({"profile_case": "long", "us": us, "bytes": nbytes}))
+        return
     if args.profile_case:
         run_profile_case()
         return

@@ -121,6 +121,20 @@ int iskv_decode_attn(iskv_handle *h, int layer, const float *q_dev, float *out_d
                      iskv_stream_t stream);
 
 /*
+ * One decode step of `layer`: appends one new row per (sequence, kv-head) to the key and value
+ * streams (with any fold the window releases, as iskv_append_block() with m = 1) and then runs
+ * iskv_decode_attn() over positions 0 .. t (the new row included). Same results as those two
+ * calls. With the tensor-core decode and window >= 1 the new rows are read by the decode kernel
+ * itself, which also stores them in the exact ring, so the step needs no separate append launch;
+ * otherwise the two calls are made in turn.
+ *   k_row_dev, v_row_dev: kv_dtype [batch][n_kv_heads][1][head_dim] (keys pre-RoPE);
+ *   q_dev, out_dev: as iskv_decode_attn().
+ * Errors: those of iskv_append_block() and iskv_decode_attn().
+ */
+int iskv_append_decode(iskv_handle *h, int layer, const void *k_row_dev, const void *v_row_dev,
+                       const float *q_dev, float *out_dev, iskv_stream_t stream);
+
+/*
  * Writes the reconstructed cache of one path of `layer` ("Reconstruction and Storage"): row i is
  * (C B^T)[i] for i < n_c and the exact window row otherwise; keys are rotated by RoPE when
  * apply_rope != 0 (ignored for values).

@@ -20,7 +20,7 @@ __all__ = [
     "iskv_create", "iskv_destroy", "iskv_append_block", "iskv_decode_attn", "iskv_reconstruct",
     "iskv_get_factors", "iskv_num_tokens", "iskv_storage_bytes", "iskv_schedule",
     "iskv_sync_status", "iskv_strerror", "iskv_reset", "iskv_launch_count", "iskv_fold_stats",
-    "iskv_join",
+    "iskv_join", "iskv_append_decode",
     "iskv_decode_view", "iskv_decode_attn_noalloc", "ISKV_NOALLOC_SCRATCH_FLOATS",
 ]
 
@@ -111,6 +111,7 @@ _SIGNATURES = {
     "iskv_schedule": (_i, [_i, _i, _ll, _ll, ctypes.POINTER(_ll), ctypes.POINTER(_ll)]),
     "iskv_sync_status": (_i, [_vp, _vp]),
     "iskv_join": (_i, [_vp, _vp]),
+    "iskv_append_decode": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "iskv_strerror": (ctypes.c_char_p, [_i]),
     "iskv_reset": (_i, [_vp, _vp]),
     "iskv_launch_count": (_i, [_vp, ctypes.POINTER(_ll)]),
@@ -242,6 +243,11 @@ def iskv_fold_stats(handle, stream=None):
 def iskv_decode_attn_noalloc(view: iskv_decode_view, q, out, stream=None) -> int:
     return lib.iskv_decode_attn_noalloc(None if view is None else ctypes.byref(view), _ptr(q),
                                         _ptr(out), _stream(stream))
+
+
+def iskv_append_decode(handle, layer: int, k_row, v_row, q, out, stream=None) -> int:
+    return lib.iskv_append_decode(handle, layer, _ptr(k_row), _ptr(v_row), _ptr(q), _ptr(out),
+                                  _stream(stream))
 
 
 def iskv_join(handle, stream=None) -> int:

@@ -6,7 +6,7 @@ import torch
 
 from .binding import (ISKV_BF16, ISKV_F32, check, iskv_append_block, iskv_config, iskv_create,
                       iskv_decode_attn, iskv_destroy, iskv_fold_stats, iskv_get_factors,
-                      iskv_join, iskv_launch_count,
+                      iskv_append_decode, iskv_join, iskv_launch_count,
                       iskv_num_tokens, iskv_reconstruct, iskv_reset, iskv_storage_bytes,
                       iskv_sync_status)
 
@@ -56,6 +56,18 @@ class IsKVCache:
         if out is None:
             out = torch.empty_like(q)
         check(iskv_decode_attn(self.handle, layer, q, out, stream), "iskv_decode_attn")
+        return out
+
+    def append_decode(self, layer: int, k_row: torch.Tensor, v_row: torch.Tensor, q: torch.Tensor,
+                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """One decode step: append one row per (sequence, kv-head) (``[batch][n_kv][1][d]``) and
+        attend over every position including it."""
+        assert k_row.dtype == self.dtype and k_row.is_contiguous() and v_row.is_contiguous()
+        assert q.dtype == torch.float32 and q.is_contiguous()
+        if out is None:
+            out = torch.empty_like(q)
+        check(iskv_append_decode(self.handle, layer, k_row, v_row, q, out, stream),
+              "iskv_append_decode")
         return out
 
     def reconstruct(self, layer: int, which: int, apply_rope: bool = False,

@@ -36,7 +36,7 @@ struct TcLayout {
 
 // Shared-memory plan of the split kernel. Window tiles stage their exact value rows from a_hi
 // onwards (a_hi, a_lo and v are contiguous and unused by window tiles otherwise).
-__host__ __device__ inline TcLayout tc_layout(int kblocks, int rV, int esz) {
+__host__ __device__ inline TcLayout tc_layout(int kblocks, int rV, int esz, int G) {
     TcLayout L;
     uint32_t o = 0;
     L.b_hi = o; o += kblocks * KBLK_BYTES;
@@ -47,19 +47,24 @@ __host__ __device__ inline TcLayout tc_layout(int kblocks, int rV, int esz) {
     const uint32_t vcomp = 128u * rV * 4u;
     const uint32_t vwin = 128u * D * esz;
     const uint32_t span = 2u * kblocks * KBLK_BYTES;      // a_hi + a_lo
-    uint32_t vb = vcomp;
+    const int nq = (rV + 3) / 4, nqp = nq <= 8 ? 8 : nq <= 16 ? 16 : 32;
+    const uint32_t redv = 8u * G * nqp * 16u;             // value-sum reduction in the stage
+    uint32_t vb = vcomp > redv ? vcomp : redv;
     if (vwin > span + vb) vb = vwin - span;
+    if (8u * G * 32u * 16u > span + vb) vb = 8u * G * 32u * 16u - span;   // window reduction
     o += (vb + 1023) & ~1023u;
-    L.q = o; o += GMAX * D * 4;
-    L.x = o; o += 2 * GMAX * 128 * 4;        // score halves, then (aliased) probabilities
+    L.q = o; o += G * D * 4;
+    L.x = o; o += 2 * G * 128 * 4;           // score halves, then (aliased) probabilities
     L.red = o; o += 2 * 4 * GMAX * 4;
-    L.acc = o; o += GMAX * D * 4;
+    L.acc = o; o += G * D * 4;
     L.bars = o; o += 64;
     L.total = o + 1024;                    // slack for aligning the base to 1024 bytes
     return L;
 }
 
-size_t tc_smem_bytes(int kblocks, int rV, int esz) { return tc_layout(kblocks, rV, esz).total; }
+size_t tc_smem_bytes(int kblocks, int rV, int esz, int G) {
+    return tc_layout(kblocks, rV, esz, G).total;
+}
 
 __device__ __forceinline__ float warp_max_f(float v) {
 #pragma unroll
@@ -162,13 +167,13 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int G = a.G, rV = a.r[1], kV = a.k[1];
     const int esz = a.kv_dtype == ISKV_BF16 ? 2 : 4;
-    const TcLayout L = tc_layout(x.kblocks, rV, esz);
+    const TcLayout L = tc_layout(x.kblocks, rV, esz, G);
     uint8_t *bBh = sm + L.b_hi, *bBl = sm + L.b_lo, *bAh = sm + L.a_hi, *bAl = sm + L.a_lo;
     float *sQ = reinterpret_cast<float *>(sm + L.q);
-    float *sX = reinterpret_cast<float *>(sm + L.x);            // [2 halves][GMAX][128]
-    float *sP = sX;                                             // [GMAX][128] (after the scores)
+    float *sX = reinterpret_cast<float *>(sm + L.x);            // [2 halves][G][128]
+    float *sP = sX;                                             // [G][128] (after the scores)
     float *sRed = reinterpret_cast<float *>(sm + L.red);        // [2][4][GMAX]
-    float *sAcc = reinterpret_cast<float *>(sm + L.acc);        // [GMAX][D] running value sums
+    float *sAcc = reinterpret_cast<float *>(sm + L.acc);        // [G][D] running value sums
     uint64_t *bar_a = reinterpret_cast<uint64_t *>(sm + L.bars);
     uint64_t *bar_v = bar_a + 1;
     uint64_t *bar_mma = bar_a + 2;
@@ -176,7 +181,22 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, half = warp >> 2;
-    const int ul = blockIdx.y, split = blockIdx.x;
+    // one-dimensional grid: all window splits first (short), then the compressed splits, so the
+    // long compressed CTAs start in the first wave
+    int ul, split;
+    {
+        const int nsw = a.n_split - a.n_split_c;
+        const int W = (int)(gridDim.x / a.n_split) * nsw;
+        int idx = blockIdx.x;
+        if (idx < W) {
+            ul = idx / nsw;
+            split = a.n_split_c + idx % nsw;
+        } else {
+            idx -= W;
+            ul = idx / a.n_split_c;
+            split = idx % a.n_split_c;
+        }
+    }
     const int seq = ul / a.H, h = ul % a.H;
     const bool comp = split < a.n_split_c;
     uint8_t *bV = comp ? sm + L.v : bAh;                        // value rows of the tile
@@ -221,7 +241,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
         }
     };
 
-    if (comp && warp == 0) tmem_alloc(tmem_slot, 128);
+    if (comp && warp == 0) tmem_alloc(tmem_slot, 256);
     // everything the previous kernel in the stream writes (rows, factors, queries) is read only
     // after this point; dependents may start once every CTA got here
     griddep_wait();
@@ -267,62 +287,69 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
         lrun[g] = 0.f;
     }
     const int row = 32 * wq + lane;
+    const int jb = 32 * half;                   // this thread's first channel pair
 
-    for (long long t0 = p0; t0 < p1 && ok; t0 += DEC_TILE) {
-        const int rows = (int)min((long long)DEC_TILE, p1 - t0);
-        const bool valid = row < rows;
-        const long long pos = t0 + row;
-        const bool rope = valid && a.rope_cs != nullptr;
-        const int jb = 32 * half;               // this thread's first channel pair
-        float part[GT];
+    // thread 0 issues the three-term tf32 product of the staged key-coordinate tile into TMEM
+    // accumulator `buf` (columns 128 buf .. 128 buf + 127)
+    auto issue_mma = [&](int buf) {
+        tc_fence_after();
+        const uint32_t aH = smem_u32(bAh), aL = smem_u32(bAl);
+        const uint32_t bH = smem_u32(bBh), bL = smem_u32(bBl);
+        const uint32_t d = tmem + 128u * buf;
+        uint32_t acc = 0;
+        for (int kb = 0; kb < x.kblocks; ++kb)
 #pragma unroll
-        for (int g = 0; g < GT; ++g) part[g] = 0.f;
-        // RoPE angles of this thread's 32 pairs: the first half is loaded before anything waits,
-        // the second half while the MMA runs, so their latency hides under the tile loads
-        float4 cs[16];
-        const float4 *c4 = reinterpret_cast<const float4 *>(a.rope_cs + pos * DH + jb);
-        if (rope) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) cs[q] = c4[q];
-        }
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t off = kb * KBLK_BYTES + kk * 32;
+                mma_tf32(d, sw128_kmajor_desc(aH + off), sw128_kmajor_desc(bH + off), idesc, acc);
+                acc = 1;
+                mma_tf32(d, sw128_kmajor_desc(aH + off), sw128_kmajor_desc(bL + off), idesc, 1);
+                mma_tf32(d, sw128_kmajor_desc(aL + off), sw128_kmajor_desc(bH + off), idesc, 1);
+            }
+        mma_commit(bar_mma);
+    };
 
-        if (comp) {
-            ok = __syncthreads_and(mbar_wait(bar_a, ph_a)) != 0;
-            if (!ok) break;
+    // first compressed tile: split B and A, start its product
+    if (comp && p0 < p1) {
+        ok = __syncthreads_and(mbar_wait(bar_a, ph_a)) != 0;
+        if (ok) {
             pend_a = false;
             ph_a ^= 1;
-            if (t0 == p0) split_tf32(bBh, bBl, abytes);
+            split_tf32(bBh, bBl, abytes);
             split_tf32(bAh, bAl, abytes);
             fence_proxy_async_smem();
             __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
-                const uint32_t aH = smem_u32(bAh), aL = smem_u32(bAl);
-                const uint32_t bH = smem_u32(bBh), bL = smem_u32(bBl);
-                uint32_t acc = 0;
-                for (int kb = 0; kb < x.kblocks; ++kb)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t off = kb * KBLK_BYTES + kk * 32;
-                        mma_tf32(tmem, sw128_kmajor_desc(aH + off), sw128_kmajor_desc(bH + off), idesc, acc);
-                        acc = 1;
-                        mma_tf32(tmem, sw128_kmajor_desc(aH + off), sw128_kmajor_desc(bL + off), idesc, 1);
-                        mma_tf32(tmem, sw128_kmajor_desc(aL + off), sw128_kmajor_desc(bH + off), idesc, 1);
-                    }
-                mma_commit(bar_mma);
-            }
+            if (tid == 0) issue_mma(0);
             pend_m = true;
-            if (rope) {
+        }
+    }
+
+    int it = 0;
+    for (long long t0 = p0; t0 < p1 && ok; t0 += DEC_TILE, ++it) {
+        const int rows = (int)min((long long)DEC_TILE, p1 - t0);
+        const bool valid = row < rows;
+        const long long pos = t0 + row;
+        const bool rope = valid && x.rope_t != nullptr;
+        const bool more = t0 + DEC_TILE < p1;
+        float part[GT];
 #pragma unroll
-                for (int q = 8; q < 16; ++q) cs[q] = c4[q];
-            }
+        for (int g = 0; g < GT; ++g) part[g] = 0.f;
+        // RoPE angles of this thread's 32 pairs, first half now (under the MMA wait)
+        float4 cs[16];
+        // (transposed table: float4 q of this row is entry (jb/2 + q) * rope_rows + pos)
+        const float4 *c4 = x.rope_t + (size_t)(jb / 2) * x.rope_rows + pos;
+        if (rope) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) cs[q] = c4[(size_t)q * x.rope_rows];
+        }
+        if (comp) {
             ok = __syncthreads_and(mbar_wait(bar_mma, ph_m)) != 0;
             tc_fence_after();
             if (!ok) break;
             pend_m = false;
             ph_m ^= 1;
             // the key-coordinate buffers are free again: fetch the next tile's under this epilogue
-            if (t0 + DEC_TILE < p1) {
+            if (more) {
                 pend_a = true;
                 if (tid == 0) {
                     mbar_arrive_expect_tx(bar_a, abytes);
@@ -331,8 +358,9 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
             }
         }
 
-        // ---- this row's key, channel pairs (j, j + 64) for j in [jb, jb + 32), two chunks -------
-        const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
+        // ---- this row's key, channel pairs (j, j + 64) for j in [jb, jb + 32), two chunks;
+        //      RoPE and the dot products in packed fp32 pairs ----------------------------------
+        const uint32_t trow = tmem + 128u * (it & 1) + ((uint32_t)(wq * 32) << 16);
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
             const int j0 = jb + 16 * ch;
@@ -342,26 +370,34 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
                 tmem_ld16(trow + 64 + j0, hi);
                 tmem_wait_ld();
             } else if (valid) {
-                const size_t rb = ring_base + (size_t)(pos % a.R) * D;
-                load_row16(a.ring[0], rb + j0, a.kv_dtype, lo);
-                load_row16(a.ring[0], rb + 64 + j0, a.kv_dtype, hi);
+                const bool fresh = pos == a.new_pos;      // appended by this call
+                const void *src = fresh ? a.new_row[0] : a.ring[0];
+                const size_t rb = fresh ? (size_t)ul * D : ring_base + (size_t)(pos % a.R) * D;
+                load_row16(src, rb + j0, a.kv_dtype, lo);
+                load_row16(src, rb + 64 + j0, a.kv_dtype, hi);
             } else {
 #pragma unroll
                 for (int j = 0; j < 16; ++j) lo[j] = hi[j] = 0.f;
             }
-            if (rope && !comp && ch == 1) {
+            float2 L2[8], H2[8];
 #pragma unroll
-                for (int q = 8; q < 16; ++q) cs[q] = c4[q];
+            for (int q = 0; q < 8; ++q) {
+                L2[q] = make_float2(lo[2 * q], lo[2 * q + 1]);
+                H2[q] = make_float2(hi[2 * q], hi[2 * q + 1]);
             }
             if (rope) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const float4 w = cs[8 * ch + q];
-                    const float x0 = lo[2 * q], y0 = hi[2 * q], x1 = lo[2 * q + 1], y1 = hi[2 * q + 1];
-                    lo[2 * q] = x0 * w.x - y0 * w.y;
-                    hi[2 * q] = y0 * w.x + x0 * w.y;
-                    lo[2 * q + 1] = x1 * w.z - y1 * w.w;
-                    hi[2 * q + 1] = y1 * w.z + x1 * w.w;
+                    const float4 w = cs[8 * ch + q];              // (cos, sin) of two pairs
+                    const float2 c = make_float2(w.x, w.z), sn = make_float2(w.y, w.w);
+                    const float2 ys = __fmul2_rn(H2[q], sn), xs = __fmul2_rn(L2[q], sn);
+                    const float2 xl = __ffma2_rn(L2[q], c, make_float2(-ys.x, -ys.y));
+                    H2[q] = __ffma2_rn(H2[q], c, xs);
+                    L2[q] = xl;
+                }
+                if (ch == 0) {                   // second half of the angles, under this chunk
+#pragma unroll
+                    for (int q = 8; q < 16; ++q) cs[q] = c4[(size_t)q * x.rope_rows];
                 }
             }
 #pragma unroll
@@ -369,36 +405,47 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
                 if (g < G) {
                     const float4 *ql = reinterpret_cast<const float4 *>(sQ + g * D + j0);
                     const float4 *qh = reinterpret_cast<const float4 *>(sQ + g * D + 64 + j0);
-                    float s = part[g];
+                    float2 s2 = make_float2(part[g], 0.f);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const float4 u = ql[q], v = qh[q];
-                        s = fmaf(u.x, lo[4 * q], s);
-                        s = fmaf(u.y, lo[4 * q + 1], s);
-                        s = fmaf(u.z, lo[4 * q + 2], s);
-                        s = fmaf(u.w, lo[4 * q + 3], s);
-                        s = fmaf(v.x, hi[4 * q], s);
-                        s = fmaf(v.y, hi[4 * q + 1], s);
-                        s = fmaf(v.z, hi[4 * q + 2], s);
-                        s = fmaf(v.w, hi[4 * q + 3], s);
+                        s2 = __ffma2_rn(make_float2(u.x, u.y), L2[2 * q], s2);
+                        s2 = __ffma2_rn(make_float2(u.z, u.w), L2[2 * q + 1], s2);
+                        s2 = __ffma2_rn(make_float2(v.x, v.y), H2[2 * q], s2);
+                        s2 = __ffma2_rn(make_float2(v.z, v.w), H2[2 * q + 1], s2);
                     }
-                    part[g] = s;
+                    part[g] = s2.x + s2.y;
                 }
             }
         }
         // ---- the two halves of each row meet; both threads hold the same score ------------------
 #pragma unroll
         for (int g = 0; g < GT; ++g)
-            if (g < G) sX[(half * GMAX + g) * 128 + row] = part[g];
+            if (g < G) sX[(half * G + g) * 128 + row] = part[g];
         __syncthreads();
 #pragma unroll
         for (int g = 0; g < GT; ++g)
             if (g < G) {
-                part[g] = sX[g * 128 + row] + sX[(GMAX + g) * 128 + row];
+                part[g] = sX[g * 128 + row] + sX[(G + g) * 128 + row];
                 const float m = warp_max_f(valid ? part[g] : -CUDART_INF_F);
                 if (half == 0 && lane == 0) sRed[wq * GMAX + g] = m;
             }
-        __syncthreads();
+        // ---- next tile: split its key coordinates and start its product into the other
+        //      accumulator, so the tensor cores work under this tile's softmax and values -------
+        bool okn = true;
+        if (comp && more) {
+            okn = mbar_wait(bar_a, ph_a);
+            if (okn) split_tf32(bAh, bAl, abytes);
+            fence_proxy_async_smem();
+        }
+        ok = __syncthreads_and(okn) != 0;
+        if (!ok) break;
+        if (comp && more) {
+            pend_a = false;
+            ph_a ^= 1;
+            if (tid == 0) issue_mma((it + 1) & 1);
+            pend_m = true;
+        }
         // ---- online softmax: every thread keeps the same running max and sum -------------------
         float alpha[GT];
 #pragma unroll
@@ -432,31 +479,61 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
         // (no bank conflicts); slice sl takes rows sl, sl + nsl, ... Quads past the row's end
         // (nqp is a power of two) read the next row's values and are never used. The slices'
         // sums meet in shared memory: first within the warp (shuffles), then across the 8 warps
-        // in `red` (a_lo for compressed tiles: free once the MMA is done; b_hi for window tiles).
+        // in the value stage itself once every warp is done reading it.
         ok = __syncthreads_and(mbar_wait(bar_v, ph_v)) != 0;
         if (!ok) break;
         pend_v = false;
         ph_v ^= 1;
+        if (!comp && a.new_pos >= t0 && a.new_pos < t0 + rows) {
+            // fused append: the staged copy of this slot is stale; take the caller's row and
+            // store K and V in the ring for later calls (one CTA owns this position)
+            const int i = (int)(a.new_pos - t0);
+            const size_t slot = ring_base + (size_t)(a.new_pos % a.R) * D;
+            if (a.kv_dtype == ISKV_BF16) {
+                const __nv_bfloat16 *nk = static_cast<const __nv_bfloat16 *>(a.new_row[0]) + (size_t)ul * D;
+                const __nv_bfloat16 *nv = static_cast<const __nv_bfloat16 *>(a.new_row[1]) + (size_t)ul * D;
+                __nv_bfloat16 *rk = const_cast<__nv_bfloat16 *>(static_cast<const __nv_bfloat16 *>(a.ring[0])) + slot;
+                __nv_bfloat16 *rv = const_cast<__nv_bfloat16 *>(static_cast<const __nv_bfloat16 *>(a.ring[1])) + slot;
+                if (tid < D) {
+                    const __nv_bfloat16 v = nv[tid];
+                    reinterpret_cast<__nv_bfloat16 *>(bV + (size_t)i * vld)[tid] = v;
+                    rv[tid] = v;
+                    rk[tid] = nk[tid];
+                }
+            } else {
+                const float *nk = static_cast<const float *>(a.new_row[0]) + (size_t)ul * D;
+                const float *nv = static_cast<const float *>(a.new_row[1]) + (size_t)ul * D;
+                float *rk = const_cast<float *>(static_cast<const float *>(a.ring[0])) + slot;
+                float *rv = const_cast<float *>(static_cast<const float *>(a.ring[1])) + slot;
+                if (tid < D) {
+                    const float v = nv[tid];
+                    reinterpret_cast<float *>(bV + (size_t)i * vld)[tid] = v;
+                    rv[tid] = v;
+                    rk[tid] = nk[tid];
+                }
+            }
+            __syncthreads();
+        }
         {
             const int nq = (nacc + 3) >> 2;
             const int nqp = nq <= 8 ? 8 : nq <= 16 ? 16 : 32;
             const int nsl = TC_THREADS / nqp;
             const int qd = tid & (nqp - 1), sl = tid / nqp;
-            float *red = reinterpret_cast<float *>(comp ? bAl : bBh);   // [8 warps][G][4 nqp]
             float4 acc4[GT];
 #pragma unroll
             for (int g = 0; g < GT; ++g) acc4[g] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
             for (int i = sl; i < rows; i += nsl) {
                 const float4 v = load_v4(bV + (size_t)i * vld, 4 * qd, vfmt);
+                const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
 #pragma unroll
                 for (int g = 0; g < GT; ++g)
                     if (g < G) {
                         const float pg = sP[g * 128 + i];
-                        acc4[g].x = fmaf(pg, v.x, acc4[g].x);
-                        acc4[g].y = fmaf(pg, v.y, acc4[g].y);
-                        acc4[g].z = fmaf(pg, v.z, acc4[g].z);
-                        acc4[g].w = fmaf(pg, v.w, acc4[g].w);
+                        const float2 p2 = make_float2(pg, pg);
+                        const float2 a01 = __ffma2_rn(p2, v01, make_float2(acc4[g].x, acc4[g].y));
+                        const float2 a23 = __ffma2_rn(p2, v23, make_float2(acc4[g].z, acc4[g].w));
+                        acc4[g] = make_float4(a01.x, a01.y, a23.x, a23.y);
                     }
             }
             // slices that share a warp: lanes nqp, 2 nqp, ... apart
@@ -470,18 +547,20 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
                         acc4[g].w += __shfl_xor_sync(0xffffffffu, acc4[g].w, o);
                     }
                 }
+            float *sRedV = reinterpret_cast<float *>(bV);       // [8 warps][G][4 nqp]
+            __syncthreads();                                    // value stage consumed
             if (lane < nqp) {
 #pragma unroll
                 for (int g = 0; g < GT; ++g)
                     if (g < G)
-                        reinterpret_cast<float4 *>(red)[(warp * G + g) * nqp + qd] = acc4[g];
+                        reinterpret_cast<float4 *>(sRedV)[(warp * G + g) * nqp + qd] = acc4[g];
             }
             __syncthreads();
             for (int o = tid; o < G * nacc; o += TC_THREADS) {
-                const int g = o / nacc, c = o % nacc;
+                const int g = o / nacc, c = o - g * nacc;
                 float sum = 0.f;
 #pragma unroll
-                for (int w = 0; w < 8; ++w) sum += red[((w * G + g) * nqp) * 4 + c];
+                for (int w = 0; w < 8; ++w) sum += sRedV[((w * G + g) * nqp) * 4 + c];
                 float al = 1.f;
 #pragma unroll
                 for (int gg = 0; gg < GT; ++gg)
@@ -489,9 +568,10 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
                 sAcc[g * D + c] = fmaf(sAcc[g * D + c], al, sum);
             }
         }
+        fence_proxy_async_smem();              // the stage was written through the generic proxy
         tc_fence_before();
         __syncthreads();                       // value rows, probabilities and TMEM consumed
-        if (t0 + DEC_TILE < p1) {
+        if (more) {
             pend_v = true;
             if (tid == 0) issue_v(t0 + DEC_TILE, (int)min((long long)DEC_TILE, p1 - t0 - DEC_TILE));
         }
@@ -509,7 +589,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
     __syncthreads();
     if (comp && warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 128);
+        tmem_dealloc(tmem, 256);
     }
 
     // ---- partials: [m, l, acc[nacc]] per q-head ------------------------------------------------
@@ -608,7 +688,7 @@ size_t merge_smem_bytes(int kV, int max_splits) {
 cudaError_t launch_decode_tc(const CUtensorMap *tmC, const CUtensorMap *tmB, const DecodeArgs &a,
                              const TcExtra &x, int n_units, cudaStream_t s) {
     const int esz = a.kv_dtype == ISKV_BF16 ? 2 : 4;
-    const size_t smem = tc_smem_bytes(x.kblocks, a.r[1], esz);
+    const size_t smem = tc_smem_bytes(x.kblocks, a.r[1], esz, a.G);
     const size_t msmem = merge_smem_bytes(a.k[1], a.max_splits);
     // opt-in dynamic shared memory, raised per device whenever a launch needs more
     static size_t attr_tc[64] = {0}, attr_merge[64] = {0};
@@ -635,7 +715,7 @@ cudaError_t launch_decode_tc(const CUtensorMap *tmC, const CUtensorMap *tmB, con
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.n_split, n_units);
+    cfg.gridDim = dim3(a.n_split * n_units);
     cfg.blockDim = dim3(TC_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;

@@ -30,6 +30,7 @@ struct iskv_handle {
     float *htop[2] = {nullptr, nullptr};    // [NB][U][r][r]
     void *ring[2] = {nullptr, nullptr};
     float2 *rope_cs = nullptr;
+    float4 *rope_t = nullptr;             // transposed copy for the tensor-core decode
     float *ws = nullptr;
     int *status = nullptr;
     unsigned long long *stats = nullptr;  // fold statistics (3 counters)
@@ -81,6 +82,7 @@ void free_all(iskv_handle *h) {
         cudaFree(h->htop[x]);
     }
     cudaFree(h->rope_cs);
+    cudaFree(h->rope_t);
     cudaFree(h->ws);
     cudaFree(h->status);
     cudaFree(h->stats);
@@ -379,6 +381,7 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         alloc((void **)&h->htop[x], nb * U * r * r * sizeof(float));
     }
     if (c.rope) alloc((void **)&h->rope_cs, (size_t)c.max_tokens * DH * sizeof(float2));
+    if (c.rope) alloc((void **)&h->rope_t, (size_t)c.max_tokens * DH * sizeof(float2));
     alloc((void **)&h->ws, (size_t)h->UL * h->max_splits * h->G * (2 + D) * sizeof(float));
     alloc((void **)&h->status, sizeof(int));
     alloc((void **)&h->stats, 4 * sizeof(unsigned long long));
@@ -396,7 +399,8 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         for (size_t i = 0; ok && i < h->done.size(); ++i)
             ok = cudaEventCreateWithFlags(&h->done[i], cudaEventDisableTiming) == cudaSuccess;
         if (ok && c.rope)
-            ok = launch_rope_table(h->rope_cs, c.max_tokens, c.rope_theta, 0) == cudaSuccess;
+            ok = launch_rope_table(h->rope_cs, c.max_tokens, c.rope_theta, 0) == cudaSuccess &&
+                 launch_rope_table_t(h->rope_t, c.max_tokens, c.rope_theta, 0) == cudaSuccess;
         ok = ok && cudaDeviceSynchronize() == cudaSuccess;
     }
     if (!ok) {
@@ -411,11 +415,8 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, h->device);
     memset(&h->tmC, 0, sizeof(h->tmC));
     memset(&h->tmB, 0, sizeof(h->tmB));
-    // (the value-sum reduction of a compressed tile lives in the key-coordinate lo buffer:
-    //  G x next-power-of-two(r_V / 4) quads must fit in it)
-    const int nq_v = c.rank_v / 4, nqp_v = nq_v <= 8 ? 8 : nq_v <= 16 ? 16 : 32;
     if (major == 10 && c.rank_k % 4 == 0 && c.rank_k <= 64 && c.rank_v % 4 == 0 &&
-        h->G * nqp_v <= 128 * ((c.rank_k + 31) / 32)) {
+        tc_smem_bytes((c.rank_k + 31) / 32, c.rank_v, (int)h->esz, h->G) <= 227 * 1024) {
         bool m_ok = true;
         if (h->n_max > 0) {
             m_ok = make_map(&h->tmC, h->coords[0], c.rank_k, (long long)h->U * h->n_max) &&
@@ -484,10 +485,14 @@ int iskv_append_block(iskv_handle *h, int layer, const void *k_rows, const void 
     return ISKV_OK;
 }
 
-int iskv_decode_attn(iskv_handle *h, int layer, const float *q, float *out, iskv_stream_t stream) {
-    if (!h || !q || !out || !valid_layer(h, layer)) return ISKV_ERR_INVALID_ARG;
-    if (h->t[layer] < 1) return ISKV_ERR_INVALID_ARG;
-    DeviceGuard g(h->device);
+}  // extern "C"
+
+namespace {
+
+// Decode attention of one layer over positions 0 .. t-1. With new_k/new_v (tensor-core path),
+// the row of position t-1 is taken from the caller's arrays and stored in the ring by the kernel.
+int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStream_t s,
+                 const void *new_k, const void *new_v) {
     const iskv_config &c = h->cfg;
     DecodeArgs da;
     memset(&da, 0, sizeof(da));
@@ -511,10 +516,16 @@ int iskv_decode_attn(iskv_handle *h, int layer, const float *q, float *out, iskv
     da.R = h->R;
     da.H = c.n_kv_heads;
     da.G = h->G;
+    da.new_row[0] = new_k;
+    da.new_row[1] = new_v;
+    da.new_pos = new_k ? da.t - 1 : -1;
+    // compressed splits: at most one wave of CTAs (two per SM) over all units of the layer, the
+    // compressed tiles of a unit spread evenly over its splits
     const long long ctiles = (da.n_c + DEC_TILE - 1) / DEC_TILE;
-    const long long target = 2LL * h->sms;
-    long long tps = (ctiles * h->UL + target - 1) / target;
-    if (tps < 1) tps = 1;
+    long long per_unit = 2LL * h->sms / h->UL;
+    if (per_unit < 1) per_unit = 1;
+    const long long nsc = ctiles < per_unit ? ctiles : per_unit;
+    const long long tps = nsc > 0 ? (ctiles + nsc - 1) / nsc : 1;
     da.split_rows = (int)(tps * DEC_TILE);
     da.n_split_c = (int)((ctiles + tps - 1) / tps);
     const long long e = da.t - da.n_c;
@@ -523,21 +534,59 @@ int iskv_decode_attn(iskv_handle *h, int layer, const float *q, float *out, iskv
     da.kv_dtype = c.kv_dtype;
     da.scale = 1.0f / sqrtf((float)D);
     if (da.n_split > h->max_splits) return ISKV_ERR_INVALID_ARG;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (h->tc) {
         TcExtra x;
         x.kblocks = (c.rank_k + 31) / 32;
         x.row0 = (long long)layer * h->UL * h->n_max;
         x.brow0 = (cur * h->U + layer * h->UL) * D;
+        x.rope_t = c.rope ? h->rope_t : nullptr;
+        x.rope_rows = c.max_tokens;
         x.status = h->status;
         if (launch_decode_tc(&h->tmC, &h->tmB, da, x, h->UL, s) != cudaSuccess)
             return ISKV_ERR_CUDA;
         h->launches += 2;
         return ISKV_OK;
     }
+    if (new_k) return ISKV_ERR_UNSUPPORTED;     // callers fall back to a separate append
     if (launch_decode(da, h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
     h->launches += 2;
     return ISKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int iskv_decode_attn(iskv_handle *h, int layer, const float *q, float *out, iskv_stream_t stream) {
+    if (!h || !q || !out || !valid_layer(h, layer)) return ISKV_ERR_INVALID_ARG;
+    if (h->t[layer] < 1) return ISKV_ERR_INVALID_ARG;
+    DeviceGuard g(h->device);
+    return decode_layer(h, layer, q, out, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+int iskv_append_decode(iskv_handle *h, int layer, const void *k_row, const void *v_row,
+                       const float *q, float *out, iskv_stream_t stream) {
+    if (!h || !k_row || !v_row || !q || !out || !valid_layer(h, layer)) return ISKV_ERR_INVALID_ARG;
+    const iskv_config &c = h->cfg;
+    // the fused form needs the tensor-core decode, and a window of at least one row (so that a
+    // fold released by this token never needs the token's own row)
+    if (!h->tc || c.window < 1) {
+        int rc = iskv_append_block(h, layer, k_row, v_row, 1, stream);
+        if (rc != ISKV_OK) return rc;
+        return iskv_decode_attn(h, layer, q, out, stream);
+    }
+    if (h->t[layer] + 1 > c.max_tokens) return ISKV_ERR_CAPACITY;
+    DeviceGuard g(h->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    h->t[layer] += 1;
+    if (h->t[layer] - h->nc[layer] >= (long long)h->R) {
+        const int rc = apply_fold(h, layer, 1, s);
+        if (rc != ISKV_OK) return rc;
+    }
+    int rc = decode_layer(h, layer, q, out, s, k_row, v_row);
+    if (rc != ISKV_OK) return rc;
+    if (c.lookahead_folds) rc = launch_ahead(h, layer, 1, s);
+    return rc;
 }
 
 int iskv_reconstruct(iskv_handle *h, int layer, int which, int apply_rope, float *out,

@@ -90,6 +90,10 @@ struct DecodeArgs {
     int max_splits;
     int kv_dtype;
     float scale;
+    // fused append (tensor-core path only): the row of position new_pos is not yet in the ring;
+    // its K and V come from new_row[] ([units][D] kv dtype) and the kernel stores them in the ring
+    const void *new_row[2];
+    long long new_pos;      // -1: no fused append
 };
 
 // ---- reconstruct ------------------------------------------------------------------------------
@@ -109,6 +113,8 @@ struct TcExtra {
     int kblocks;            // 32-column K-blocks of the key coordinates (ceil(r_K / 32))
     long long row0;         // first coordinate row of this layer in the coordinate tensor map
     int brow0;              // first basis row of this layer (current buffer) in the basis map
+    const float4 *rope_t;   // [DH/2][rope_rows] (cos, sin) of pair pairs, or nullptr
+    long long rope_rows;
     int *status;
 };
 
@@ -118,10 +124,12 @@ cudaError_t launch_append(const AppendArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_reconstruct(const ReconArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_rope_table(float2 *table, long long max_tokens, double theta, cudaStream_t s);
+cudaError_t launch_rope_table_t(float4 *table_t, long long max_tokens, double theta,
+                                cudaStream_t s);
 cudaError_t launch_decode_tc(const CUtensorMap *tmC, const CUtensorMap *tmB, const DecodeArgs &a,
                              const TcExtra &x, int n_units, cudaStream_t s);
 size_t fold_smem_bytes();
-size_t tc_smem_bytes(int kblocks, int rV, int esz);
+size_t tc_smem_bytes(int kblocks, int rV, int esz, int G);
 
 __device__ __forceinline__ float load_row_elem(const void *base, size_t idx, int kv_dtype) {
     if (kv_dtype == ISKV_BF16)

@@ -107,6 +107,7 @@ extern "C" int iskv_decode_attn_noalloc(const iskv_decode_view *v, const float *
     da.G = G;
     da.kv_dtype = v->kv_dtype;
     da.scale = 1.0f / sqrtf((float)D);
+    da.new_pos = -1;
     return launch_decode(da, units, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? ISKV_OK
                : ISKV_ERR_CUDA;

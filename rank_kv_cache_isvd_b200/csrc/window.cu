@@ -42,6 +42,27 @@ __global__ void rope_table_kernel(float2 *table, long long max_tokens, double th
     table[idx] = make_float2((float)cs, (float)sn);
 }
 
+// Transposed copy for the tensor-core decode: table_t[q][pos] = (cos, sin) of pairs 2q and 2q+1
+// at position pos, so that the 32 rows of a warp read 32 consecutive float4 (one coalesced line)
+// instead of 32 rows 512 bytes apart.
+__global__ void rope_table_t_kernel(float4 *table_t, long long max_tokens, double theta) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= max_tokens * (DH / 2)) return;
+    const int q = (int)(idx / max_tokens);
+    const long long pos = idx % max_tokens;
+    double s0, c0, s1, c1;
+    sincos((double)pos * pow(theta, -2.0 * (2 * q) / (double)D), &s0, &c0);
+    sincos((double)pos * pow(theta, -2.0 * (2 * q + 1) / (double)D), &s1, &c1);
+    table_t[idx] = make_float4((float)c0, (float)s0, (float)c1, (float)s1);
+}
+
+cudaError_t launch_rope_table_t(float4 *table_t, long long max_tokens, double theta,
+                                cudaStream_t s) {
+    const long long n = max_tokens * (DH / 2);
+    rope_table_t_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(table_t, max_tokens, theta);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_rope_table(float2 *table, long long max_tokens, double theta, cudaStream_t s) {
     const long long n = max_tokens * DH;
     const unsigned grid = (unsigned)((n + 255) / 256);

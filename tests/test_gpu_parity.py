@@ -413,3 +413,33 @@ def test_long_context_layer_sampled_units():
         print(f"\nunit (seq {sq}, kv-head {h}): attention rel err {err:.3e}")
         assert err <= ATTN_TOL
     cache.close()
+
+
+@pytest.mark.parametrize("lookahead,window", [(False, 256), (True, 256), (False, 0)])
+def test_fused_append_decode_equals_separate_calls(lookahead, window):
+    """iskv_append_decode (the decode kernel reads the new rows itself and stores them in the
+    ring) gives bit-for-bit the outputs, factors and reconstructions of iskv_append_block +
+    iskv_decode_attn, across fold triggers; with window 0 it falls back to the two calls."""
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=900, window=window)
+    kd, kv, vd, vv = workload_arrays(wl)
+    K, V = to_device(kd[0]), to_device(vd[0])
+    Q = torch.from_numpy(syn.queries(31, (wl.tokens, 1, 8, 128))).cuda()
+    outs = []
+    for fused in (False, True):
+        cache = make_cache(wl, lookahead_folds=lookahead)
+        out = torch.empty_like(Q)
+        for t in range(wl.tokens):
+            kr = K[:, :, t:t + 1].contiguous()
+            vr = V[:, :, t:t + 1].contiguous()
+            if fused:
+                cache.append_decode(0, kr, vr, Q[t], out[t])
+            else:
+                cache.append(0, kr, vr)
+                cache.decode(0, Q[t], out[t])
+        assert cache.status() == 0 and cache.tokens(0) == wl.tokens
+        rec = [cache.reconstruct(0, x) for x in (0, 1)]
+        outs.append((out, rec))
+        cache.close()
+    (o0, r0), (o1, r1) = outs
+    assert torch.equal(o0, o1)
+    assert torch.equal(r0[0], r1[0]) and torch.equal(r0[1], r1[1])
