@@ -284,6 +284,63 @@ def long_context_decode(args, dev, flush, calls: int = 10):
     return 1e3 * float(np.median(ms)), decode_bytes(T, wl)
 
 
+WL_LAYERS = syn.WORKLOADS[2]
+
+
+def all_layers_decode_step(args, dev, flush, steps: int = 5):
+    """One decode step of a 32-layer model: the 32-layer x 8 kv-head workload (batch 1, b=64,
+    w=128, r_K=24, r_V=40) filled to 16384 tokens with one append of all layers (rows drawn on the
+    GPU), then the 32 per-layer decode calls of one step captured in a CUDA graph and replayed,
+    each replay after an L2 flush. Returns (microseconds per step, bytes per step)."""
+    import torch
+
+    from rank_kv_cache_isvd_b200.cache import IsKVCache
+    wl = WL_LAYERS
+    L, S, H, T, QH = wl.n_layers, wl.batch, wl.n_kv_heads, wl.tokens, wl.n_q_heads
+    cache = IsKVCache(batch=S, n_layers=L, n_kv_heads=H, n_q_heads=QH, rank_k=wl.rank_k,
+                      rank_v=wl.rank_v, block=wl.block, window=wl.window, max_tokens=T,
+                      kv_dtype="bf16", rope=True, rope_theta=wl.rope_theta)
+    s = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(s):
+        Kr = torch.empty((L, S, H, T, D), dtype=torch.bfloat16, device=dev)
+        Vr = torch.empty_like(Kr)
+        for l in range(L):
+            for sq in range(S):
+                for h in range(H):
+                    Kr[l, sq, h] = syn.device_rows(wl, sq, l, h, 0, device=dev)
+                    Vr[l, sq, h] = syn.device_rows(wl, sq, l, h, 1, device=dev)
+        cache.append(-1, Kr, Vr, s.cuda_stream)
+        del Kr, Vr
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(2024)
+        q = torch.randn((L, S, QH, D), generator=gen, device=dev)
+        out = torch.empty_like(q)
+        for l in range(L):
+            cache.decode(l, q[l], out[l], s.cuda_stream)
+    s.synchronize()
+    st = cache.status(s.cuda_stream)
+    assert st == 0, f"device status {st} after filling the 32-layer cache"
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for l in range(L):
+            cache.decode(l, q[l], out[l], s.cuda_stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for i in range(args.warmup + steps):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0.record(s)
+            g.replay()
+            e1.record(s)
+        s.synchronize()
+        if i >= args.warmup:
+            ms.append(e0.elapsed_time(e1))
+    assert cache.status(s.cuda_stream) == 0 and bool(torch.isfinite(out).all())
+    del g
+    cache.close()
+    return 1e3 * float(np.median(ms)), L * decode_bytes(T, wl)
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     """The largest of the ranks' values: a multi-GPU step lasts as long as its slowest rank."""
     if world == 1:
@@ -466,6 +523,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # ---- decode over a long history (HBM-bound regime), rank 0 of a single-GPU run only --------
     long_us, long_bytes = (long_context_decode(args, dev, flush) if world == 1 and rank == 0
                            else (None, None))
+    step_us, step_bytes = (all_layers_decode_step(args, dev, flush) if world == 1 and rank == 0
+                           else (None, None))
 
     # ---- roofline of the dominant kernel class --------------------------------------------------
     hbm, which = peaks()
@@ -503,6 +562,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "achieved": long_bytes / (long_us / 1e6) / 1e9, "peak": hbm, "unit": "GB/s",
             "frac": long_bytes / (long_us / 1e6) / 1e9 / hbm, "traffic": TRAFFIC_LONG,
             "bytes_per_launch": long_bytes, "launch_us": long_us},
+        "roofline_32_layer_step": None if step_us is None else {
+            "bound": "hbm", "kernel": "decode attention (split + combine), 32 calls",
+            "workload": f"{WL_LAYERS.name}: one decode step of all layers at t = {WL_LAYERS.tokens}",
+            "achieved": step_bytes / (step_us / 1e6) / 1e9, "peak": hbm, "unit": "GB/s",
+            "frac": step_bytes / (step_us / 1e6) / 1e9 / hbm, "traffic": None,
+            "bytes_per_step": step_bytes, "step_us": step_us,
+            "tok_per_s_one_sequence": 1e6 / step_us},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h),
                 "how": "pinned host rows+queries copied in, graph replay, outputs copied out"},

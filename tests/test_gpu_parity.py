@@ -443,3 +443,23 @@ def test_fused_append_decode_equals_separate_calls(lookahead, window):
     (o0, r0), (o1, r1) = outs
     assert torch.equal(o0, o1)
     assert torch.equal(r0[0], r1[0]) and torch.equal(r0[1], r1[1])
+
+
+def test_decode_parity_ranks_below_one_tensor_map_box():
+    """32-layer-workload ranks (r_K = 24, r_V = 40, b = 64, w = 128): the key-coordinate boxes of
+    the tensor-core decode are 32 columns wide, so the last 8 come from outside the 24-column
+    tensor (zero fill); decode matches the oracle at several lengths."""
+    base = syn.WORKLOADS[2]
+    wl = sub(base, n_layers=1, n_kv_heads=2, n_q_heads=8, tokens=1500)
+    kd, kv, vd, vv = workload_arrays(wl)
+    cache, orc = make_cache(wl, lookahead_folds=True), make_oracle(wl)
+    t, worst = 0, 0.0
+    for i, tc in enumerate([100, 129, 200, 700, 1500]):
+        append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], t, tc)
+        t = tc
+        q = syn.queries(200 + i, (1, wl.n_q_heads, 128))
+        out = cache.decode(0, torch.from_numpy(q).cuda()).cpu().numpy()
+        worst = max(worst, max_head_rel_err(out, orc.decode(0, q.astype(np.float64))))
+    print(f"\nr_K=24/r_V=40: worst attention rel err {worst:.3e}")
+    assert worst <= ATTN_TOL
+    assert cache.status() == 0
