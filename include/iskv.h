@@ -113,9 +113,11 @@ int iskv_append_block(iskv_handle *h, int layer, const void *k_rows_dev, const v
  * reconstructed as C B^T ("Reconstruction and Storage"), keys are then rotated by RoPE at their
  * position (when cfg.rope), scores use scale 1/sqrt(d), softmax is exact (fp32, log-sum-exp
  * merge of position splits). Two kernels (position splits, then their merge) on `stream`.
- *   q_dev:   fp32 [batch][n_q_heads][head_dim], already rotated for the query position.
+ *   q_dev:   fp32 [batch][n_q_heads][head_dim], already rotated for the query position,
+ *            16-byte aligned (the kernels copy it in 16-byte units).
  *   out_dev: fp32 [batch][n_q_heads][head_dim].
- * Errors: ISKV_ERR_INVALID_ARG (NULL pointers, bad layer, t == 0), ISKV_ERR_CUDA.
+ * Errors: ISKV_ERR_INVALID_ARG (NULL pointers, bad layer, t == 0, misaligned q_dev),
+ *         ISKV_ERR_CUDA.
  */
 int iskv_decode_attn(iskv_handle *h, int layer, const float *q_dev, float *out_dev,
                      iskv_stream_t stream);

@@ -256,7 +256,10 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
         fence_mbar_init();
         if (p0 < p1) {
             if (comp) {
-                mbar_arrive_expect_tx(bar_a, 2 * abytes);
+                // the queries of this kv-head ride on the first key-tile barrier
+                mbar_arrive_expect_tx(bar_a, 2 * abytes + (uint32_t)(G * D * 4));
+                bulk_load(sQ, a.q + ((size_t)seq * a.H * G + (size_t)h * G) * D,
+                          (uint32_t)(G * D * 4), bar_a);
                 for (int kb = 0; kb < x.kblocks; ++kb)
                     tma_load_2d(bBh + kb * KBLK_BYTES, &tmB, kb * 32, x.brow0 + ul * D, bar_a);
                 tma_a(p0);
@@ -265,13 +268,10 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
         }
     }
     {
+        // window CTAs load the queries through registers (compressed CTAs got them by bulk copy)
         const float4 *q4 = reinterpret_cast<const float4 *>(a.q + ((size_t)seq * a.H * G + (size_t)h * G) * D);
         float4 *s4 = reinterpret_cast<float4 *>(sQ);
-        const float sc = a.scale;
-        if (tid < G * D / 4) {
-            const float4 v = q4[tid];
-            s4[tid] = make_float4(v.x * sc, v.y * sc, v.z * sc, v.w * sc);
-        }
+        if (!comp && tid < G * D / 4) s4[tid] = q4[tid];
         for (int o = tid; o < G * D; o += TC_THREADS) sAcc[o] = 0.f;
     }
     tc_fence_before();
@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
 #pragma unroll
         for (int g = 0; g < GT; ++g)
             if (g < G) {
-                part[g] = sX[g * 128 + row] + sX[(G + g) * 128 + row];
+                part[g] = (sX[g * 128 + row] + sX[(G + g) * 128 + row]) * a.scale;
                 const float m = warp_max_f(valid ? part[g] : -CUDART_INF_F);
                 if (half == 0 && lane == 0) sRed[wq * GMAX + g] = m;
             }
@@ -584,15 +584,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
         if (pend_m) mbar_wait(bar_mma, ph_m);
     }
 
-    // ---- release tensor memory -------------------------------------------------------------------
-    tc_fence_before();
-    __syncthreads();
-    if (comp && warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 256);
-    }
-
-    // ---- partials: [m, l, acc[nacc]] per q-head ------------------------------------------------
+    // ---- partials: [m, l, acc[nacc]] per q-head (sAcc is final after the last tile's barrier) ---
     float *ws = a.ws + ((size_t)ul * a.max_splits + split) * G * (2 + D);
     for (int o = tid; o < G * nacc; o += TC_THREADS) {
         const int g = o / nacc, c = o % nacc;
@@ -605,6 +597,14 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
                 ws[g * (2 + D)] = mrun[g];
                 ws[g * (2 + D) + 1] = lrun[g];
             }
+    }
+
+    // ---- release tensor memory -------------------------------------------------------------------
+    tc_fence_before();
+    __syncthreads();
+    if (comp && warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
     }
 }
 

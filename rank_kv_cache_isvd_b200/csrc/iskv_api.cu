@@ -535,6 +535,7 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
     da.scale = 1.0f / sqrtf((float)D);
     if (da.n_split > h->max_splits) return ISKV_ERR_INVALID_ARG;
     if (h->tc) {
+        if (reinterpret_cast<uintptr_t>(q) % 16 != 0) return ISKV_ERR_INVALID_ARG;
         TcExtra x;
         x.kblocks = (c.rank_k + 31) / 32;
         x.row0 = (long long)layer * h->UL * h->n_max;
