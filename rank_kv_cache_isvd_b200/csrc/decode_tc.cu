@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
     uint8_t *bBh = sm + L.b_hi, *bBl = sm + L.b_lo, *bAh = sm + L.a_hi, *bAl = sm + L.a_lo;
     float *sQ = reinterpret_cast<float *>(sm + L.q);
     float *sX = reinterpret_cast<float *>(sm + L.x);            // [2 halves][G][128]
-    float *sP = sX;                                             // [G][128] (after the scores)
+    float *sP = sX;                                             // [128][GT] (after the scores)
     float *sRed = reinterpret_cast<float *>(sm + L.red);        // [2][4][GMAX]
     float *sAcc = reinterpret_cast<float *>(sm + L.acc);        // [G][D] running value sums
     uint64_t *bar_a = reinterpret_cast<uint64_t *>(sm + L.bars);
@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
                 const float m_new = fmaxf(mrun[g], mt);
                 const float pr = valid ? expf(part[g] - m_new) : 0.f;
                 if ((g & 1) == half) {
-                    sP[g * 128 + row] = pr;
+                    sP[row * GT + g] = pr;
                     const float s = warp_sum_f(pr);
                     if (lane == 0) sRed[4 * GMAX + wq * GMAX + g] = s;
                 }
@@ -526,10 +526,24 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
             for (int i = sl; i < rows; i += nsl) {
                 const float4 v = load_v4(bV + (size_t)i * vld, 4 * qd, vfmt);
                 const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
+                float pv[GT];                   // this row's probabilities, one vector load
+                if (GT >= 4) {
+#pragma unroll
+                    for (int g4 = 0; g4 < GT / 4; ++g4) {
+                        const float4 p4 = reinterpret_cast<const float4 *>(sP + i * GT)[g4];
+                        pv[4 * g4] = p4.x;
+                        pv[4 * g4 + 1] = p4.y;
+                        pv[4 * g4 + 2] = p4.z;
+                        pv[4 * g4 + 3] = p4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int g = 0; g < GT; ++g) pv[g] = sP[i * GT + g];
+                }
 #pragma unroll
                 for (int g = 0; g < GT; ++g)
                     if (g < G) {
-                        const float pg = sP[g * 128 + i];
+                        const float pg = pv[g];
                         const float2 p2 = make_float2(pg, pg);
                         const float2 a01 = __ffma2_rn(p2, v01, make_float2(acc4[g].x, acc4[g].y));
                         const float2 a23 = __ffma2_rn(p2, v23, make_float2(acc4[g].z, acc4[g].w));
@@ -622,6 +636,9 @@ __global__ void __launch_bounds__(MERGE_THREADS) decode_merge_kernel(DecodeArgs 
     const int g = blockIdx.x, ul = blockIdx.y;
     const int seq = ul / a.H, h = ul % a.H;
     const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
+    // the next kernel in the stream (the next decode's split kernel) may start its prologue
+    // now; it reads nothing this kernel writes before its own dependency wait
+    griddep_launch_dependents();
     // B_V was written before the split kernel started: stage it while the splits finish
     const float *B = a.basis[1] + (size_t)ul * D * rV;
     for (int o = j; o < D * kV; o += MERGE_THREADS) sBV[(o / kV) * ldb + o % kV] = B[(size_t)(o / kV) * rV + o % kV];
