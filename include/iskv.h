@@ -61,7 +61,8 @@ typedef struct {
     int n_q_heads;        /* multiple of n_kv_heads; q-head g reads kv-head g / (n_q/n_kv)    */
     int head_dim;         /* d; must be 128                                                  */
     int rank_k, rank_v;   /* rank budgets r_K, r_V (1 .. head_dim)                           */
-    int block;            /* b: rows folded per update (1 .. 128)                            */
+    int block;            /* b: rows folded per update (1 .. 1024; blocks above 128 rows are  */
+                          /*    folded through their 128-row triangular factor)              */
     int window;           /* w: exact rows kept before a fold may take them (>= 0)           */
     long long max_tokens; /* capacity per sequence and layer                                 */
     int kv_dtype;         /* ISKV_BF16 or ISKV_F32: dtype of appended rows and of the window  */

@@ -788,6 +788,7 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
     load_F();
     __syncthreads();
     // ---- new rows' coordinates C[n_c + i] = F[i] B+ --------------------------------------------
+    if (a.skip_new_rows) return;
     float *Cn = P.coords + ((size_t)unit * a.n_max + a.n_c) * r;
     for (int o = tid; o < b * r; o += FT) {
         const int i = o / r, c = o % r;

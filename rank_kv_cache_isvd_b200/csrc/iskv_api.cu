@@ -28,6 +28,7 @@ struct iskv_handle {
     float *basis[2] = {nullptr, nullptr};   // [NB][U][D][r]
     float *sigma[2] = {nullptr, nullptr};   // [NB][U][r]
     float *htop[2] = {nullptr, nullptr};    // [NB][U][r][r]
+    float *rbig[2] = {nullptr, nullptr};    // [U][128][D] triangular factor of a large block
     void *ring[2] = {nullptr, nullptr};
     float2 *rope_cs = nullptr;
     float4 *rope_t = nullptr;             // transposed copy for the tensor-core decode
@@ -80,6 +81,7 @@ void free_all(iskv_handle *h) {
         cudaFree(h->sigma[x]);
         cudaFree(h->ring[x]);
         cudaFree(h->htop[x]);
+        cudaFree(h->rbig[x]);
     }
     cudaFree(h->rope_cs);
     cudaFree(h->rope_t);
@@ -189,8 +191,50 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
     fa.kv_dtype = c.kv_dtype;
     fa.status = h->status;
     fa.stats = h->stats;
-    if (launch_fold(fa, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
-    h->launches += 1;
+    if (c.block > BMAX) {
+        // large block: fold the 128-row triangular factor of the block (same Sigma+, H and basis),
+        // then the coordinates of the block's real rows
+        RFactorArgs rf;
+        memset(&rf, 0, sizeof(rf));
+        for (int x = 0; x < 2; ++x) {
+            rf.path[x].ring = h->ring[x];
+            rf.path[x].rout = h->rbig[x];
+            fa.path[x].ring = h->rbig[x];
+        }
+        rf.unit0 = fa.unit0;
+        rf.slot0 = fa.slot0;
+        rf.R = h->R;
+        rf.b = c.block;
+        rf.kv_dtype = c.kv_dtype;
+        if (launch_rfactor(rf, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+        fa.slot0 = 0;
+        fa.R = DEC_TILE;
+        fa.b = DEC_TILE;
+        fa.kv_dtype = ISKV_F32;
+        fa.skip_new_rows = 1;
+        if (launch_fold(fa, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+        NewRowsArgs nr;
+        memset(&nr, 0, sizeof(nr));
+        for (int x = 0; x < 2; ++x) {
+            nr.path[x].ring = h->ring[x];
+            nr.path[x].basis = fa.path[x].basis_out;
+            nr.path[x].coords = h->coords[x];
+            nr.path[x].r = fa.path[x].r;
+            nr.path[x].kp = fa.path[x].kp;
+        }
+        nr.unit0 = rf.unit0;
+        nr.slot0 = rf.slot0;
+        nr.R = h->R;
+        nr.b = c.block;
+        nr.kv_dtype = c.kv_dtype;
+        nr.n_c = nc;
+        nr.n_max = h->n_max;
+        if (launch_newrows(nr, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+        h->launches += 3;
+    } else {
+        if (launch_fold(fa, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+        h->launches += 1;
+    }
     for (int l = l0; l < l0 + nl; ++l) {
         int *f = fold_ranks(h, l, j);
         f[0] = fa.path[0].k;
@@ -327,7 +371,7 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         c.window < 0 || c.max_tokens < 1 || (c.kv_dtype != ISKV_BF16 && c.kv_dtype != ISKV_F32) ||
         (c.rope && !(c.rope_theta > 0.0)))
         return ISKV_ERR_INVALID_ARG;
-    if (c.block > BMAX) return ISKV_ERR_UNSUPPORTED;
+    if (c.block > BMAX_LARGE) return ISKV_ERR_UNSUPPORTED;
     iskv_handle *h = new (std::nothrow) iskv_handle();
     if (!h) return ISKV_ERR_CUDA;
     try {
@@ -379,6 +423,7 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         alloc((void **)&h->sigma[x], nb * U * r * sizeof(float));
         alloc(&h->ring[x], U * (size_t)h->R * D * h->esz);
         alloc((void **)&h->htop[x], nb * U * r * r * sizeof(float));
+        if (c.block > BMAX) alloc((void **)&h->rbig[x], U * DEC_TILE * D * sizeof(float));
     }
     if (c.rope) alloc((void **)&h->rope_cs, (size_t)c.max_tokens * DH * sizeof(float2));
     if (c.rope) alloc((void **)&h->rope_t, (size_t)c.max_tokens * DH * sizeof(float2));

@@ -14,6 +14,7 @@ namespace iskv {
 constexpr int D = 128;        // head_dim (fixed by the build)
 constexpr int DH = D / 2;     // RoPE pairs (j, j + 64)
 constexpr int BMAX = 128;     // largest block folded by the in-shared-memory fold kernel
+constexpr int BMAX_LARGE = 1024;  // largest block (folded through its triangular factor)
 constexpr int LDS = D + 1;    // padded stride of 128-float rows/columns in shared memory
 constexpr int GMAX = 8;       // largest GQA group (q-heads per kv-head)
 constexpr int DEC_TILE = 128; // decode rows per tile
@@ -42,6 +43,28 @@ struct FoldArgs {
     int kv_dtype;
     int *status;
     unsigned long long *stats;  // [0] max sweeps, [1] total sweeps, [2] cores solved
+    int skip_new_rows;      // 1: leave the new rows' coordinates to newrows_kernel (large blocks)
+};
+
+// ---- large blocks (b > BMAX): triangular factor of the block, then the real rows' coordinates -
+struct RFactorPath {
+    const void *ring;       // [units][R][D] kv dtype
+    float *rout;            // [units][128][D] fp32 pseudo-block (R of the block)
+};
+struct RFactorArgs {
+    RFactorPath path[2];
+    int unit0, slot0, R, b, kv_dtype;
+};
+struct NewRowsPath {
+    const void *ring;       // [units][R][D] kv dtype
+    const float *basis;     // [units][D][r] basis after the fold
+    float *coords;          // [units][n_max][r]
+    int r, kp;
+};
+struct NewRowsArgs {
+    NewRowsPath path[2];
+    int unit0, slot0, R, b, kv_dtype;
+    long long n_c, n_max;
 };
 
 // ---- history rotation C[0:n] <- C[0:n] H_top (or stale zero-padding) ---------------------------
@@ -119,6 +142,8 @@ struct TcExtra {
 };
 
 cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s);
+cudaError_t launch_rfactor(const RFactorArgs &a, int n_units, cudaStream_t s);
+cudaError_t launch_newrows(const NewRowsArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_append(const AppendArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int n_units, cudaStream_t s);

@@ -463,3 +463,65 @@ def test_decode_parity_ranks_below_one_tensor_map_box():
     print(f"\nr_K=24/r_V=40: worst attention rel err {worst:.3e}")
     assert worst <= ATTN_TOL
     assert cache.status() == 0
+
+
+def test_two_sequences_two_layers_fused_steps_with_lookahead():
+    """Batch 2 x 2 layers x 2 kv-heads, every token one fused step per layer with look-ahead
+    folds (one internal stream per layer): every layer's decode matches the oracle at several
+    lengths, and reconstructed keys with RoPE match the oracle's rotated keys."""
+    wl = sub(W1, batch=2, n_layers=2, n_kv_heads=2, n_q_heads=8, tokens=700)
+    kd, kv, vd, vv = workload_arrays(wl, variant="gapped")  # well-defined subspaces
+    cache, orc = make_cache(wl, lookahead_folds=True), make_oracle(wl)
+    K, V = to_device(kd), to_device(vd)                     # [L][S][H][T][D]
+    checkpoints, worst = {321, 450, 700}, 0.0
+    for t in range(wl.tokens):
+        for l in range(wl.n_layers):
+            q = syn.queries(1000 + 10 * t + l, (wl.batch, wl.n_q_heads, 128))
+            out = cache.append_decode(l, K[l][:, :, t:t + 1].contiguous(),
+                                      V[l][:, :, t:t + 1].contiguous(), torch.from_numpy(q).cuda())
+            orc.append(l, kv[l][:, :, t:t + 1], vv[l][:, :, t:t + 1])
+            if t + 1 in checkpoints:
+                err = max_head_rel_err(out.cpu().numpy(), orc.decode(l, q.astype(np.float64)))
+                worst = max(worst, err)
+    print(f"\nbatch 2 x 2 layers, fused steps: worst attention rel err {worst:.3e}")
+    assert worst <= ATTN_TOL
+    for l in range(wl.n_layers):
+        rk = cache.reconstruct(l, 0, apply_rope=True).cpu().numpy()
+        for s in range(wl.batch):
+            for h in range(wl.n_kv_heads):
+                kref, _ = orc.keys_values(l, s, h)
+                assert rel_err(rk[s, h], kref) <= 1e-3
+    assert cache.status() == 0
+
+
+@pytest.mark.parametrize("variant", ["gapped", "literal"])
+def test_large_blocks_fold_through_their_triangular_factor(variant):
+    """Long-context shapes (b = 512, w = 512, r_K = 64, r_V = 96): blocks above 128 rows are
+    folded through the 128-row triangular factor of the block. A 2048-row prefill (3 folds) plus
+    100 streamed tokens: Sigma, projectors (gapped rows) and decode match the oracle."""
+    base = syn.WORKLOADS[4]
+    wl = sub(base, batch=1, n_layers=1, n_kv_heads=2, n_q_heads=8, tokens=2148, prefill=2048)
+    kd, kv, vd, vv = workload_arrays(wl, variant=variant)
+    cache, orc = make_cache(wl, lookahead_folds=True), make_oracle(wl)
+    append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], 0, 2048)
+    K, V = to_device(kd[0]), to_device(vd[0])
+    worst = 0.0
+    for t in range(2048, wl.tokens):
+        q = syn.queries(3000 + t, (1, wl.n_q_heads, 128))
+        out = cache.append_decode(0, K[:, :, t:t + 1].contiguous(), V[:, :, t:t + 1].contiguous(),
+                                  torch.from_numpy(q).cuda())
+        orc.append(0, kv[0][:, :, t:t + 1], vv[0][:, :, t:t + 1])
+        if t % 25 == 0 or t == wl.tokens - 1:
+            worst = max(worst, max_head_rel_err(out.cpu().numpy(), orc.decode(0, q.astype(np.float64))))
+    print(f"\nb=512 {variant}: worst attention rel err {worst:.3e}")
+    assert worst <= ATTN_TOL
+    for h in range(2):
+        for x in (0, 1):
+            C, B, S, k, n = cache.factors(0, 0, h, x)
+            u = orc.unit(0, 0, h, x)
+            assert k == u.k and n == u.n == 1536
+            if variant == "gapped":
+                S, B = S.cpu().numpy(), B.cpu().numpy()
+                assert np.max(np.abs(S[:k] - u.sigma) / u.sigma) <= SIG_TOL
+                assert projector_err(B[:, :k], u.B) <= PROJ_TOL
+    assert cache.status() == 0

@@ -67,7 +67,7 @@ def test_create_rejects_invalid_config(bad):
 
 
 def test_create_reports_unsupported_block():
-    code, h = iskv.iskv_create(_cfg(block=256))
+    code, h = iskv.iskv_create(_cfg(block=2048))
     assert code == iskv.ISKV_ERR_UNSUPPORTED and h == 0
 
 
