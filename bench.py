@@ -233,8 +233,8 @@ WL_LONG = syn.WORKLOADS[3]
 # DRAM bytes (read + write) of one launch of the split kernel as ncu counted them for the current
 # kernel: the t = 4096 launch of the bench workload (--profile-case) and the long-context launch
 # (--profile-case long). Set to None whenever the kernel changes until it is captured again.
-TRAFFIC_T4096 = 13_208_064
-TRAFFIC_LONG = 832_619_264
+TRAFFIC_T4096 = 13_452_800
+TRAFFIC_LONG = 833_116_928
 
 
 def long_context_decode(args, dev, flush, calls: int = 10):
@@ -282,6 +282,71 @@ def long_context_decode(args, dev, flush, calls: int = 10):
     assert cache.status(s.cuda_stream) == 0 and bool(torch.isfinite(out).all())
     cache.close()
     return 1e3 * float(np.median(ms)), decode_bytes(T, wl)
+
+
+WL_PREFILL = syn.WORKLOADS[4]
+
+
+def prefill_and_decode(args, dev, flush, calls: int = 5):
+    """One layer of the long-context workload (batch 4 x 8 kv-heads, 32 q-heads, b = 512, w = 512,
+    r_K = 64, r_V = 96): the 65536-row prefill appended in one call (127 folds of 512-row blocks
+    per head and path; rows drawn on the GPU), timed as a graph replay, then decode calls over
+    the 65024 compressed rows. Returns (prefill ms, head-block updates, decode us, decode bytes)."""
+    import torch
+
+    from rank_kv_cache_isvd_b200.cache import IsKVCache
+    wl = WL_PREFILL
+    S, H, T0, QH = wl.batch, wl.n_kv_heads, wl.prefill, wl.n_q_heads
+    cache = IsKVCache(batch=S, n_layers=1, n_kv_heads=H, n_q_heads=QH, rank_k=wl.rank_k,
+                      rank_v=wl.rank_v, block=wl.block, window=wl.window, max_tokens=wl.tokens,
+                      kv_dtype="bf16", rope=True, rope_theta=wl.rope_theta)
+    s = torch.cuda.Stream(device=dev)
+    sh = s.cuda_stream
+    with torch.cuda.stream(s):
+        Kr = torch.empty((S, H, T0, D), dtype=torch.bfloat16, device=dev)
+        Vr = torch.empty_like(Kr)
+        for sq in range(S):
+            for h in range(H):
+                Kr[sq, h] = syn.device_rows(wl, sq, 0, h, 0, T=T0, device=dev)
+                Vr[sq, h] = syn.device_rows(wl, sq, 0, h, 1, T=T0, device=dev)
+        cache.append(0, Kr, Vr, sh)
+    s.synchronize()
+    st = cache.status(sh)
+    assert st == 0, f"device status {st} after the long prefill"
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        cache.reset(sh)
+        cache.append(0, Kr, Vr, sh)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pre = []
+    for i in range(2):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0.record(s)
+            g.replay()
+            e1.record(s)
+        s.synchronize()
+        pre.append(e0.elapsed_time(e1))
+    del g, Kr, Vr
+    folds = wl.n_c(T0) // wl.block
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4242)
+    q = torch.randn((S, QH, D), generator=gen, device=dev)
+    out = torch.empty_like(q)
+    ms = []
+    for i in range(args.warmup + calls):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0.record(s)
+            cache.decode(0, q, out, sh)
+            e1.record(s)
+        s.synchronize()
+        if i >= args.warmup:
+            ms.append(e0.elapsed_time(e1))
+    assert cache.status(sh) == 0 and bool(torch.isfinite(out).all())
+    cache.close()
+    return (float(min(pre)), folds * S * H * 2, 1e3 * float(np.median(ms)),
+            decode_bytes(T0, wl))
 
 
 WL_LAYERS = syn.WORKLOADS[2]
@@ -525,6 +590,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                            else (None, None))
     step_us, step_bytes = (all_layers_decode_step(args, dev, flush) if world == 1 and rank == 0
                            else (None, None))
+    pre_ms, pre_updates, pre_dec_us, pre_dec_bytes = (
+        prefill_and_decode(args, dev, flush) if world == 1 and rank == 0
+        else (None, None, None, None))
 
     # ---- roofline of the dominant kernel class --------------------------------------------------
     hbm, which = peaks()
@@ -569,6 +637,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "frac": step_bytes / (step_us / 1e6) / 1e9 / hbm, "traffic": None,
             "bytes_per_step": step_bytes, "step_us": step_us,
             "tok_per_s_one_sequence": 1e6 / step_us},
+        "long_prefill": None if pre_ms is None else {
+            "workload": (f"{WL_PREFILL.name}: one layer, {WL_PREFILL.prefill}-row prefill in one "
+                         "append, then decode at that length"),
+            "prefill_ms": pre_ms, "head_block_updates": pre_updates,
+            "head_block_updates_per_s": pre_updates / (pre_ms / 1e3),
+            "decode_us": pre_dec_us, "decode_bytes": pre_dec_bytes,
+            "decode_achieved_gbs": pre_dec_bytes / (pre_dec_us / 1e6) / 1e9,
+            "decode_frac_of_hbm": pre_dec_bytes / (pre_dec_us / 1e6) / 1e9 / hbm},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h),
                 "how": "pinned host rows+queries copied in, graph replay, outputs copied out"},

@@ -564,10 +564,12 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
     da.new_row[0] = new_k;
     da.new_row[1] = new_v;
     da.new_pos = new_k ? da.t - 1 : -1;
-    // compressed splits: at most one wave of CTAs (two per SM) over all units of the layer, the
-    // compressed tiles of a unit spread evenly over its splits
+    // compressed splits: at most one wave of CTAs over all units of the layer (two per SM when
+    // two fit in shared memory), the compressed tiles of a unit spread evenly over its splits
     const long long ctiles = (da.n_c + DEC_TILE - 1) / DEC_TILE;
-    long long per_unit = 2LL * h->sms / h->UL;
+    const int per_sm = (!h->tc || tc_smem_bytes((c.rank_k + 31) / 32, c.rank_v, (int)h->esz, h->G) +
+                                          1024 <= 114u * 1024u) ? 2 : 1;
+    long long per_unit = (long long)per_sm * h->sms / h->UL;
     if (per_unit < 1) per_unit = 1;
     const long long nsc = ctiles < per_unit ? ctiles : per_unit;
     const long long tps = nsc > 0 ? (ctiles + nsc - 1) / nsc : 1;
