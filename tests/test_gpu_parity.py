@@ -525,3 +525,72 @@ def test_large_blocks_fold_through_their_triangular_factor(variant):
                 assert np.max(np.abs(S[:k] - u.sigma) / u.sigma) <= SIG_TOL
                 assert projector_err(B[:, :k], u.B) <= PROJ_TOL
     assert cache.status() == 0
+
+
+def _sampled_unit_check(wl, q, out, units):
+    """Oracle run on single (sequence, kv-head) units of a full-size cache, compared on their
+    q-heads; rows come back from the device (bf16 values, exact in float64)."""
+    G = wl.group
+    worst = 0.0
+    for sq, h, K, V in units:
+        orc = OracleCache(1, 1, 1, G, 128, wl.rank_k, wl.rank_v, wl.block, wl.window, rope=True,
+                          rope_theta=wl.rope_theta)
+        orc.append(0, K.float().cpu().numpy().astype(np.float64)[None, None],
+                   V.float().cpu().numpy().astype(np.float64)[None, None])
+        qs = q[sq, h * G:(h + 1) * G].cpu().numpy().astype(np.float64)[None]
+        err = max_head_rel_err(out[sq, h * G:(h + 1) * G].cpu().numpy()[None], orc.decode(0, qs))
+        worst = max(worst, err)
+    return worst
+
+
+def test_32_layer_workload_full_size_sampled_units():
+    """The 32-layer x 8 kv-head workload at its full length (16384 tokens, b=64, w=128, r_K=24,
+    r_V=40), all layers appended in one call as the benchmark does; two sampled (layer, kv-head)
+    units of the decode match the oracle run on their rows alone."""
+    wl = syn.WORKLOADS[2]
+    L, S, H, T = wl.n_layers, wl.batch, wl.n_kv_heads, wl.tokens
+    cache = make_cache(wl)
+    K = torch.empty((L, S, H, T, 128), dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+    for l in range(L):
+        for h in range(H):
+            K[l, 0, h] = syn.device_rows(wl, 0, l, h, 0)
+            V[l, 0, h] = syn.device_rows(wl, 0, l, h, 1)
+    cache.append(-1, K, V)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(2024)
+    worst = 0.0
+    for l, h in ((0, 3), (31, 6)):
+        q = torch.randn((S, wl.n_q_heads, 128), generator=gen, device="cuda")
+        out = cache.decode(l, q)
+        assert bool(torch.isfinite(out).all())
+        worst = max(worst, _sampled_unit_check(wl, q, out, [(0, h, K[l, 0, h], V[l, 0, h])]))
+    print(f"\n32-layer workload, sampled units: worst attention rel err {worst:.3e}")
+    assert worst <= ATTN_TOL
+    assert cache.status() == 0
+    cache.close()
+
+
+def test_long_prefill_full_size_sampled_unit():
+    """The long-context layer at its full prefill (batch 4 x 8 kv-heads, 65536 rows in one
+    append, b = 512, w = 512, r_K = 64, r_V = 96): one sampled unit of the decode matches the
+    oracle run on its rows alone."""
+    wl = syn.WORKLOADS[4]
+    S, H, T0 = wl.batch, wl.n_kv_heads, wl.prefill
+    cache = make_cache(sub(wl, n_layers=1))
+    K = torch.empty((S, H, T0, 128), dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+    for sq in range(S):
+        for h in range(H):
+            K[sq, h] = syn.device_rows(wl, sq, 0, h, 0, T=T0)
+            V[sq, h] = syn.device_rows(wl, sq, 0, h, 1, T=T0)
+    cache.append(0, K, V)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(4242)
+    q = torch.randn((S, wl.n_q_heads, 128), generator=gen, device="cuda")
+    out = cache.decode(0, q)
+    assert cache.status() == 0 and bool(torch.isfinite(out).all())
+    err = _sampled_unit_check(wl, q, out, [(2, 5, K[2, 5], V[2, 5])])
+    print(f"\nlong prefill, sampled unit: attention rel err {err:.3e}")
+    assert err <= ATTN_TOL
+    cache.close()
