@@ -7,9 +7,10 @@
 //      first, which re-orthogonalises E against B to rounding (the oracle's second projection pass).
 //   2. Z = [[Sigma, 0], [S, F P]], (k + b) x (k + p); with P from that QR, F P = E P is the
 //      transpose of the QR's trailing R block for the rows that entered it.
-//   3. (G, Sigma+, H) = SVD_r(Z) by one-sided (Hestenes) Jacobi on the columns of Z^T: at
-//      convergence the columns of Z^T J are orthogonal, their norms are the singular values and
-//      the normalised columns are the right singular vectors H of Z, so J is never accumulated;
+//   3. (G, Sigma+, H) = SVD_r(Z): Z is first reduced to its triangular factor R (Householder,
+//      Q discarded; R^T R = Z^T Z), then one-sided (Hestenes) Jacobi runs on the columns of R^T:
+//      at convergence the columns of R^T J are orthogonal, their norms are the singular values
+//      and the normalised columns are the right singular vectors H of Z, so J is never accumulated;
 //      B+ = [B P] H, the old coordinates move by H[:k] (rotate_kernel) and the new rows'
 //      coordinates are F B+ (bottom block of U+ Sigma+, since Z H = G Sigma+).
 // One CTA (256 threads) per unit and path (blockIdx.y = path), everything on chip (b <= 128).
@@ -20,8 +21,6 @@ namespace iskv {
 constexpr int FT = 256;                       // threads
 constexpr int FW = FT / 32;                   // warps
 constexpr int JL = 16;                        // lanes per Jacobi column group
-constexpr int JGRP = FT / JL;                 // column groups
-constexpr int NSLOT = 2 * JGRP;               // Jacobi slots (two per group)
 constexpr int SS = 132;                       // column stride of the Jacobi staging area
 constexpr float JACOBI_TOL = 4e-6f;           // rotate while |a.b| > tol |a| |b|
 constexpr float JACOBI_ZERO = 1e-10f;         // columns with |a|^2 <= this * ||Z||_F^2 are noise
@@ -29,13 +28,14 @@ constexpr float JACOBI_ZERO = 1e-10f;         // columns with |a|^2 <= this * ||
 // shared memory (floats)
 constexpr int OFF_A = 0;                                  // F/E rows -> [P | B_old] -> F rows
 constexpr int OFF_B = OFF_A + 128 * LDS;                  // Y = [S | T] rows
-constexpr int STAGE_FLOATS = NSLOT * 8 * SS;              // Jacobi staging (overlays B and C)
+constexpr int STAGE_FLOATS = 2 * 128 * SS;                // two Jacobi staging buffers of 128
+                                                          // columns (overlay B and C)
 constexpr int C_FLOATS = STAGE_FLOATS - 128 * LDS;        // QR columns -> Sigma columns
 constexpr int OFF_C = OFF_B + 128 * LDS;
 constexpr int OFF_TAU = OFF_C + C_FLOATS;
 constexpr int OFF_SIG = OFF_TAU + 128;
 constexpr int OFF_NRM = OFF_SIG + 128;                    // [256] column norms
-constexpr int OFF_SNRM = OFF_NRM + 256;                   // [256] staged squared norms
+constexpr int OFF_SNRM = OFF_NRM + 256;                   // [2][128] staged squared norms
 constexpr int OFF_SCR = OFF_SNRM + 256;                   // per-warp scratch, 128 floats each
 constexpr int OFF_INT = OFF_SCR + FW * 128;               // ints: sel[256], flags[4]
 constexpr int SMEM_FLOATS = OFF_INT + 256 + 4;
@@ -233,19 +233,23 @@ __device__ __noinline__ int jacobi_regs(const float *sB, const float *sC, int k,
                 JCrossAll<HC, RPL, 0>::run(xa, xb, na, nb, floor2, rotated);
             }
             if (ng > 1) {                     // move the slots for the next round
+                // two staging buffers, alternating by round: a round's writes never meet the
+                // previous round's reads, so one barrier per round suffices
+                float *stg = stage + (round & 1) * (2 * ng * HC * SS);
+                float *stn = stage_n + (round & 1) * (2 * ng * HC);
                 if (active) {
 #pragma unroll
                     for (int j = 0; j < HC; ++j) {
-                        float *da = stage + (destA * HC + j) * SS + r0;
-                        float *db = stage + (destB * HC + j) * SS + r0;
+                        float *da = stg + (destA * HC + j) * SS + r0;
+                        float *db = stg + (destB * HC + j) * SS + r0;
 #pragma unroll
                         for (int i = 0; i < RPL; ++i) {
                             da[i] = xa[j][i];
                             db[i] = xb[j][i];
                         }
                         if (gl == 0) {
-                            stage_n[destA * HC + j] = na[j];
-                            stage_n[destB * HC + j] = nb[j];
+                            stn[destA * HC + j] = na[j];
+                            stn[destB * HC + j] = nb[j];
                         }
                     }
                 }
@@ -253,18 +257,17 @@ __device__ __noinline__ int jacobi_regs(const float *sB, const float *sC, int k,
                 if (active) {
 #pragma unroll
                     for (int j = 0; j < HC; ++j) {
-                        const float *sa = stage + (grp * HC + j) * SS + r0;
-                        const float *sb = stage + ((ng + grp) * HC + j) * SS + r0;
+                        const float *sa = stg + (grp * HC + j) * SS + r0;
+                        const float *sb = stg + ((ng + grp) * HC + j) * SS + r0;
 #pragma unroll
                         for (int i = 0; i < RPL; ++i) {
                             xa[j][i] = sa[i];
                             xb[j][i] = sb[i];
                         }
-                        na[j] = stage_n[grp * HC + j];
-                        nb[j] = stage_n[(ng + grp) * HC + j];
+                        na[j] = stn[grp * HC + j];
+                        nb[j] = stn[(ng + grp) * HC + j];
                     }
                 }
-                __syncthreads();
             }
         }
         if (__syncthreads_or(rotated) == 0) {
@@ -303,6 +306,201 @@ __device__ __noinline__ int jacobi_regs(const float *sB, const float *sC, int k,
     return converged ? sweeps : -sweeps;
 }
 
+// Register-tiled product over shared-memory operands: out(i, j, sum_l A(i, l) B(l, j)) for
+// i < M, j < N, l < K, each thread accumulating TI x TJ outputs (rows ib + MS ii, columns
+// TJ jb + jj). Lanes of a warp take consecutive ib, so row-strided A loads fall in distinct banks
+// (odd row stride) and B loads are shared by the lanes of a column block.
+template <int TI, int TJ, class LA, class LB, class ST>
+__device__ __forceinline__ void tile_gemm(int M, int N, int K, LA la, LB lb, ST st) {
+    const int MS = (M + TI - 1) / TI, NSB = (N + TJ - 1) / TJ;
+    for (int t = threadIdx.x; t < MS * NSB; t += FT) {
+        const int ib = t % MS, jb = t / MS;
+        int ii_[TI], jj_[TJ];
+#pragma unroll
+        for (int a = 0; a < TI; ++a) ii_[a] = min(ib + MS * a, M - 1);
+#pragma unroll
+        for (int b = 0; b < TJ; ++b) jj_[b] = min(TJ * jb + b, N - 1);
+        float acc[TI][TJ];
+#pragma unroll
+        for (int a = 0; a < TI; ++a)
+#pragma unroll
+            for (int b = 0; b < TJ; ++b) acc[a][b] = 0.f;
+#pragma unroll 2
+        for (int l = 0; l < K; ++l) {
+            float av[TI], bv[TJ];
+#pragma unroll
+            for (int a = 0; a < TI; ++a) av[a] = la(ii_[a], l);
+#pragma unroll
+            for (int b = 0; b < TJ; ++b) bv[b] = lb(l, jj_[b]);
+#pragma unroll
+            for (int a = 0; a < TI; ++a)
+#pragma unroll
+                for (int b = 0; b < TJ; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
+        }
+#pragma unroll
+        for (int a = 0; a < TI; ++a)
+#pragma unroll
+            for (int b = 0; b < TJ; ++b) {
+                const int i = ib + MS * a, j = TJ * jb + b;
+                if (i < M && j < N) st(i, j, acc[a][b]);
+            }
+    }
+}
+
+// Householder QR in shared memory (R in place, reflectors kept below it).
+//
+// Step j reflects the pivot row j and the body rows y0(j) .. y1 - 1 of column j: lane l holds
+// body rows y0 + l + 32 u (u < 4) of the reflector in registers, each warp updates trailing
+// columns j + 1 + warp + FW m, eight at a time with overlapped reductions. Warp 0's first batch
+// holds column j + 1, so it forms the next reflector right after that column's update (norm from
+// the updated values in its registers); each step therefore ends with a single barrier.
+// Reflectors are stored scaled in the body rows of their column (v_i below the pivot, v_pivot = 1
+// implicit) with tau_j in sTau[j]; R's diagonal entries replace the pivots.
+//
+// Storage policies: element (i, c) of a body row is at(i, c); the pivot row of step j is the
+// vector pivot(j) with stride pstride; body rows number at most 128.
+struct CoreRows {               // the fold core Z: Sigma rows in sC, block rows in sY (row-major)
+    float *sY, *sC;
+    int k, b;
+    __device__ float *pivot(int j) const { return j < k ? sC + j * LDS : sY + (j - k) * LDS; }
+    __device__ int pstride() const { return 1; }
+    __device__ int y0(int j) const { return j < k ? 0 : j - k + 1; }
+    __device__ int y1() const { return b; }
+    __device__ float &at(int i, int c) const { return sY[i * LDS + c]; }
+};
+struct ColumnRows {             // a D-row matrix stored by columns in sC (column c at sC + c LDS)
+    float *sC;
+    __device__ float *pivot(int j) const { return sC + j; }
+    __device__ int pstride() const { return LDS; }
+    __device__ int y0(int j) const { return j + 1; }
+    __device__ int y1() const { return D; }
+    __device__ float &at(int i, int c) const { return sC[c * LDS + i]; }
+};
+
+// Reflector of column j from its body values x[u] (rows y0 + lane + 32 u, those below `from`
+// taking part) and the pivot entry `alpha`: stores v = x * scale below the pivot, beta at the
+// pivot and tau. Called by one full warp.
+template <class M>
+__device__ __forceinline__ void qr_reflector(const M &m, int j, int y0, int from, float alpha,
+                                             const float (&x)[4], float *sTau) {
+    const int lane = threadIdx.x & 31, y1 = m.y1();
+    float s2 = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int i = y0 + lane + 32 * u;
+        if (i < y1 && i >= from) s2 = fmaf(x[u], x[u], s2);
+    }
+    s2 = warp_sum(s2);
+    float tau = 0.f, beta = alpha, scale = 0.f;
+    if (s2 > 0.f) {
+        beta = -copysignf(sqrtf(fmaf(alpha, alpha, s2)), alpha);
+        tau = (beta - alpha) / beta;
+        scale = 1.f / (alpha - beta);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int i = y0 + lane + 32 * u;
+        if (i < y1 && i >= from) m.at(i, j) = x[u] * scale;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        m.pivot(j)[j * m.pstride()] = beta;
+        sTau[j] = tau;
+    }
+}
+
+template <class M>
+__device__ void householder_qr(const M &m, int n, float *sTau) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int ps = m.pstride(), y1 = m.y1();
+    if (warp == 0 && n > 0) {                        // reflector of column 0
+        const int y0 = m.y0(0);
+        float x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = y0 + lane + 32 * u;
+            x[u] = i < y1 ? m.at(i, 0) : 0.f;
+        }
+        qr_reflector(m, 0, y0, y0, m.pivot(0)[0], x, sTau);
+    }
+    __syncthreads();
+    for (int j = 0; j < n; ++j) {
+        const float tau = sTau[j];
+        const int y0 = m.y0(j);
+        const int y0n = j + 1 < n ? m.y0(j + 1) : y1;  // body of the next step
+        float *pr = m.pivot(j);
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = y0 + lane + 32 * u;
+            v[u] = i < y1 ? m.at(i, j) : 0.f;
+        }
+        for (int cb = j + 1 + warp; cb < n; cb += 8 * FW) {
+            float w[8], xq[8][4], pj[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int c = min(cb + q * FW, n - 1);
+                w[q] = 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = y0 + lane + 32 * u;
+                    xq[q][u] = i < y1 ? m.at(i, c) : 0.f;
+                    w[q] = fmaf(v[u], xq[q][u], w[q]);
+                }
+                pj[q] = pr[c * ps];
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) w[q] += __shfl_xor_sync(0xffffffffu, w[q], o);
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int c = cb + q * FW;
+                if (c < n) {
+                    const float wq = (w[q] + pj[q]) * tau;
+                    if (lane == 0) pr[c * ps] = pj[q] - wq;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = y0 + lane + 32 * u;
+                        xq[q][u] = fmaf(-wq, v[u], xq[q][u]);
+                        if (i < y1) m.at(i, c) = xq[q][u];
+                    }
+                }
+            }
+            if (cb == j + 1 && j + 1 < n) {            // warp 0: column j + 1 is final for step j
+                float al = 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (y0 + lane + 32 * u == y0n - 1) al = xq[0][u];
+                al = warp_sum(al);                     // (at most one lane holds the pivot)
+                if (y0n - 1 < y0) al = m.pivot(j + 1)[(j + 1) * ps];   // untouched by step j
+                __syncwarp();
+                qr_reflector(m, j + 1, y0, y0n, al, xq[0], sTau);
+            }
+            __syncwarp();
+        }
+        __syncthreads();
+    }
+}
+
+// Triangular factor of the core, in place: Z = Q R, keeping R only. R^T R = Z^T Z, so R has the
+// singular values and the right singular vectors H of Z, and the one-sided Jacobi on the rows of
+// R converges in fewer sweeps than on the rows of Z (triangular preconditioning of the Hestenes
+// method). Z's rows are vectors of length n: row c < k (Sigma_c e_c) at sC + c LDS, row k + i (the
+// block's [S | T] row i) at sY + i LDS; the Sigma rows are diagonal, so the reflector of column
+// j < k involves only row j and the b block rows, and column j >= k pivots on block row j - k. On
+// return R's row c is stored where Z's row c was, entries below the diagonal cleared (block rows
+// p .. b - 1 become zero).
+__device__ void core_triangular_factor(float *sY, float *sC, float *sTau, int k, int b, int n) {
+    householder_qr(CoreRows{sY, sC, k, b}, n, sTau);
+    for (int o = threadIdx.x; o < b * n; o += FT) {
+        const int i = o / n, c = o % n;
+        if (c < k + i) sY[i * LDS + c] = 0.f;
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
     extern __shared__ float smem[];
     float *sA = smem + OFF_A;
@@ -321,7 +519,6 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = P.k, r = P.r, p = P.p, kp = P.kp, b = a.b;
     const int n = k + p;                  // rows of Z^T (columns of Z)
-    const int N = k + b;                  // columns of Z^T
     const size_t ring_base = (size_t)unit * a.R * D;
     const float *Bin = P.basis_in + (size_t)unit * D * r;
 
@@ -404,32 +601,13 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
 
     // ---- step 1: S = F B (into Y[:, :k]) and the residual E = F - S B^T (in place) -----------
     if (k > 0) {
-        for (int o = tid; o < b * k; o += FT) {
-            const int i = o / k, c = o % k;
-            const float *f = sA + i * LDS, *bc = sC + c * LDS;
-            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll 4
-            for (int j = 0; j < D; j += 4) {
-                s0 = fmaf(f[j], bc[j], s0);
-                s1 = fmaf(f[j + 1], bc[j + 1], s1);
-                s2 = fmaf(f[j + 2], bc[j + 2], s2);
-                s3 = fmaf(f[j + 3], bc[j + 3], s3);
-            }
-            sB[i * LDS + c] = (s0 + s1) + (s2 + s3);
-        }
+        tile_gemm<2, 4>(b, k, D, [&](int i, int l) { return sA[i * LDS + l]; },
+                        [&](int l, int c) { return sC[c * LDS + l]; },
+                        [&](int i, int c, float v) { sB[i * LDS + c] = v; });
         __syncthreads();
-        for (int o = tid; o < b * D; o += FT) {
-            const int i = o / D, j = o % D;
-            const float *srow = sB + i * LDS;
-            float e0 = sA[i * LDS + j], e1 = 0.f;
-            int c = 0;
-            for (; c + 1 < k; c += 2) {
-                e0 = fmaf(-srow[c], sC[c * LDS + j], e0);
-                e1 = fmaf(-srow[c + 1], sC[(c + 1) * LDS + j], e1);
-            }
-            if (c < k) e0 = fmaf(-srow[c], sC[c * LDS + j], e0);
-            sA[i * LDS + j] = e0 + e1;
-        }
+        tile_gemm<2, 4>(b, D, k, [&](int i, int c) { return sB[i * LDS + c]; },
+                        [&](int c, int j) { return sC[c * LDS + j]; },
+                        [&](int i, int j, float v) { sA[i * LDS + j] -= v; });
         __syncthreads();
     }
 
@@ -439,85 +617,7 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
         sC[(k + i) * LDS + j] = sA[i * LDS + j];
     }
     __syncthreads();
-    for (int jc = 0; jc < n; ++jc) {
-        float *col = sC + jc * LDS;
-        if (warp == 0) {
-            float xv[4], s2 = 0.f;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = lane + 32 * u;
-                xv[u] = col[i];
-                s2 = fmaf(i > jc ? xv[u] : 0.f, xv[u], s2);
-            }
-            s2 = warp_sum(s2);
-            const float alpha = col[jc];
-            float tau = 0.f, beta = alpha, scale = 0.f;
-            if (s2 > 0.f) {
-                beta = -copysignf(sqrtf(fmaf(alpha, alpha, s2)), alpha);
-                tau = (beta - alpha) / beta;
-                scale = 1.f / (alpha - beta);
-            }
-            __syncwarp();
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = lane + 32 * u;
-                if (i > jc) col[i] = xv[u] * scale;
-            }
-            if (lane == 0) {
-                col[jc] = beta;
-                sTau[jc] = tau;
-            }
-        }
-        __syncthreads();
-        const float tau = sTau[jc];
-        if (tau != 0.f) {
-            float v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = lane + 32 * u;
-                v[u] = i > jc ? col[i] : 0.f;
-            }
-            // trailing columns c = jc + 1 + warp + FW m, eight per batch (overlapped reductions)
-            for (int cb = jc + 1 + warp; cb < n; cb += 8 * FW) {
-                float w[8], xq[8][4];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int c = min(cb + q * FW, n - 1);
-                    const float *x = sC + c * LDS;
-                    w[q] = 0.f;
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        xq[q][u] = x[lane + 32 * u];
-                        w[q] = fmaf(v[u], xq[q][u], w[q]);
-                    }
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) w[q] += __shfl_xor_sync(0xffffffffu, w[q], o);
-                float xj[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) xj[q] = sC[min(cb + q * FW, n - 1) * LDS + jc];
-                __syncwarp();
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int c = cb + q * FW;
-                    if (c < n) {
-                        float *x = sC + c * LDS;
-                        const float wq = (w[q] + xj[q]) * tau;
-                        if (lane == 0) x[jc] = xj[q] - wq;
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int i = lane + 32 * u;
-                            if (i > jc) x[i] = fmaf(-wq, v[u], xq[q][u]);
-                        }
-                    }
-                }
-                __syncwarp();
-            }
-        }
-        __syncthreads();
-    }
+    householder_qr(ColumnRows{sC}, n, sTau);
 
     // ---- T = F P for the rows in the QR: T[i][l] = R[k+l][k+i] (l <= i) ----------------------
     for (int o = tid; o < p * p; o += FT) {
@@ -589,24 +689,23 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
     }
     __syncthreads();
 
-    // ---- one-sided Jacobi on the N columns (length n) of Z^T, register resident --------------
+    // ---- Z -> R (same Z^T Z), then one-sided Jacobi on the n columns of R^T, register resident
+    core_triangular_factor(sB, sC, sTau, k, b, n);
+    const int NJ = n;                     // Jacobi columns: the rows of R
     int sweeps;
-    const int HC = N <= 96 ? 3 : (N <= 128 ? 4 : 8);
+    const int HC = NJ <= 96 ? 3 : 4;     // NJ = k + p <= D
     {
         const int rpl = n <= 96 ? 6 : (n <= 112 ? 7 : 8);
         switch (HC * 16 + rpl) {
-            case 3 * 16 + 6: sweeps = jacobi_regs<3, 6>(sB, sC, k, N, n, stage, sSN, sNrm); break;
-            case 3 * 16 + 7: sweeps = jacobi_regs<3, 7>(sB, sC, k, N, n, stage, sSN, sNrm); break;
-            case 3 * 16 + 8: sweeps = jacobi_regs<3, 8>(sB, sC, k, N, n, stage, sSN, sNrm); break;
-            case 4 * 16 + 6: sweeps = jacobi_regs<4, 6>(sB, sC, k, N, n, stage, sSN, sNrm); break;
-            case 4 * 16 + 7: sweeps = jacobi_regs<4, 7>(sB, sC, k, N, n, stage, sSN, sNrm); break;
-            case 4 * 16 + 8: sweeps = jacobi_regs<4, 8>(sB, sC, k, N, n, stage, sSN, sNrm); break;
-            case 8 * 16 + 6: sweeps = jacobi_regs<8, 6>(sB, sC, k, N, n, stage, sSN, sNrm); break;
-            case 8 * 16 + 7: sweeps = jacobi_regs<8, 7>(sB, sC, k, N, n, stage, sSN, sNrm); break;
-            default: sweeps = jacobi_regs<8, 8>(sB, sC, k, N, n, stage, sSN, sNrm); break;
+            case 3 * 16 + 6: sweeps = jacobi_regs<3, 6>(sB, sC, k, NJ, n, stage, sSN, sNrm); break;
+            case 3 * 16 + 7: sweeps = jacobi_regs<3, 7>(sB, sC, k, NJ, n, stage, sSN, sNrm); break;
+            case 3 * 16 + 8: sweeps = jacobi_regs<3, 8>(sB, sC, k, NJ, n, stage, sSN, sNrm); break;
+            case 4 * 16 + 6: sweeps = jacobi_regs<4, 6>(sB, sC, k, NJ, n, stage, sSN, sNrm); break;
+            case 4 * 16 + 7: sweeps = jacobi_regs<4, 7>(sB, sC, k, NJ, n, stage, sSN, sNrm); break;
+            default: sweeps = jacobi_regs<4, 8>(sB, sC, k, NJ, n, stage, sSN, sNrm); break;
         }
     }
-    const int NC = 2 * ((N + 2 * HC - 1) / (2 * HC)) * HC;   // staged columns (NC - N zero)
+    const int NC = 2 * ((NJ + 2 * HC - 1) / (2 * HC)) * HC;  // staged columns (NC - NJ zero)
     if (tid == 0) {
         if (sweeps < 0) set_status(a.status, ISKV_ERR_NOT_CONVERGED);
         if (a.stats) {
@@ -718,36 +817,18 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
         ht[(size_t)l * r + c] = stage[sSel[c] * SS + l];
     }
     float *Bout = P.basis_out + (size_t)unit * D * r;
-    const int j = tid & (D - 1);
-    const int c0 = tid >> 7;               // 0..1
-    for (int cb = 0; cb < r; cb += 64) {
-        float bp[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const int c = cb + c0 + 2 * q;
-            float s0 = 0.f, s1 = 0.f;
-            if (c < kp) {
-                const float *hv = stage + sSel[c] * SS;
-                int l = 0;
-                for (; l + 1 < p; l += 2) {
-                    s0 = fmaf(sA[l * LDS + j], hv[k + l], s0);
-                    s1 = fmaf(sA[(l + 1) * LDS + j], hv[k + l + 1], s1);
-                }
-                if (l < p) s0 = fmaf(sA[l * LDS + j], hv[k + l], s0);
-                for (l = 0; l + 1 < k; l += 2) {
-                    s0 = fmaf(sA[(p + l) * LDS + j], hv[l], s0);
-                    s1 = fmaf(sA[(p + l + 1) * LDS + j], hv[l + 1], s1);
-                }
-                if (l < k) s0 = fmaf(sA[(p + l) * LDS + j], hv[l], s0);
-            }
-            bp[q] = s0 + s1;
-        }
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const int c = cb + c0 + 2 * q;
-            if (c < r) Bout[(size_t)j * r + c] = bp[q];
-        }
+    // dense H rows in the order of W's columns: Hd[l][c] = H[k + l][c] (P part), H[l - p][c] (B)
+    float *Hd = sC + 512;                  // past the staged columns (NC SS <= 128 LDS + 384)
+    for (int o = tid; o < n * kp; o += FT) {
+        const int l = o / kp, c = o % kp;
+        Hd[o] = stage[sSel[c] * SS + (l < p ? k + l : l - p)];
     }
+    __syncthreads();
+    tile_gemm<4, 4>(D, kp, n, [&](int j, int l) { return sA[l * LDS + j]; },
+                    [&](int l, int c) { return Hd[l * kp + c]; },
+                    [&](int j, int c, float v) { Bout[(size_t)j * r + c] = v; });
+    for (int o = tid; o < D * (r - kp); o += FT)
+        Bout[(size_t)(o / (r - kp)) * r + kp + o % (r - kp)] = 0.f;
     __syncthreads();                       // H, W consumed; B+ (uncorrected) and H_top written
     // ---- one Newton-Schulz step towards the nearest orthonormal basis, B+ <- B+ (3I - M) / 2 with
     //      M = B+^T B+ (the Jacobi stops at a relative orthogonality threshold, and without this
@@ -755,33 +836,25 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
     //      old coordinates stay consistent with the corrected basis.
     float *sBp = sC;                       // B+ columns [kp][LDS]
     float *sM = sB;                        // M [kp][kp]
-    float *sH = sA;                        // H_top [k][kp]
+    float *sH = sA;                        // H_top [k][kp + 1]
+    const int hld = kp + 1;
     for (int o = tid; o < D * kp; o += FT) sBp[(o % kp) * LDS + o / kp] = Bout[(size_t)(o / kp) * r + o % kp];
-    for (int o = tid; o < k * kp; o += FT) sH[o] = ht[(size_t)(o / kp) * r + o % kp];
+    for (int o = tid; o < k * kp; o += FT) sH[(o / kp) * hld + o % kp] = ht[(size_t)(o / kp) * r + o % kp];
     __syncthreads();
-    for (int o = tid; o < kp * kp; o += FT) {
-        const int c = o / kp, c2 = o % kp;
-        const float *x = sBp + c * LDS, *y = sBp + c2 * LDS;
-        float s0 = 0.f, s1 = 0.f;
-        for (int jj = 0; jj < D; jj += 2) {
-            s0 = fmaf(x[jj], y[jj], s0);
-            s1 = fmaf(x[jj + 1], y[jj + 1], s1);
-        }
-        sM[o] = s0 + s1;
-    }
+    tile_gemm<2, 4>(kp, kp, D, [&](int c, int j) { return sBp[c * LDS + j]; },
+                    [&](int j, int c2) { return sBp[c2 * LDS + j]; },
+                    [&](int c, int c2, float v) { sM[c * kp + c2] = v; });
     __syncthreads();
-    for (int o = tid; o < D * kp; o += FT) {
-        const int c = o / D, jj = o % D;
-        float s = 0.f;
-        for (int c2 = 0; c2 < kp; ++c2) s = fmaf(sBp[c2 * LDS + jj], sM[c2 * kp + c], s);
-        Bout[(size_t)jj * r + c] = 1.5f * sBp[c * LDS + jj] - 0.5f * s;
-    }
-    for (int o = tid; o < k * kp; o += FT) {
-        const int l = o / kp, c = o % kp;
-        float s = 0.f;
-        for (int c2 = 0; c2 < kp; ++c2) s = fmaf(sH[l * kp + c2], sM[c2 * kp + c], s);
-        ht[(size_t)l * r + c] = 1.5f * sH[o] - 0.5f * s;
-    }
+    tile_gemm<4, 4>(D, kp, kp, [&](int j, int c2) { return sBp[c2 * LDS + j]; },
+                    [&](int c2, int c) { return sM[c2 * kp + c]; },
+                    [&](int j, int c, float v) {
+                        Bout[(size_t)j * r + c] = 1.5f * sBp[c * LDS + j] - 0.5f * v;
+                    });
+    tile_gemm<2, 4>(k, kp, kp, [&](int l, int c2) { return sH[l * hld + c2]; },
+                    [&](int c2, int c) { return sM[c2 * kp + c]; },
+                    [&](int l, int c, float v) {
+                        ht[(size_t)l * r + c] = 1.5f * sH[l * hld + c] - 0.5f * v;
+                    });
     __syncthreads();
     // corrected B+ columns back into shared memory; reload F for the new rows' coordinates
     for (int o = tid; o < D * kp; o += FT) sBp[(o % kp) * LDS + o / kp] = Bout[(size_t)(o / kp) * r + o % kp];
@@ -790,18 +863,11 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
     // ---- new rows' coordinates C[n_c + i] = F[i] B+ --------------------------------------------
     if (a.skip_new_rows) return;
     float *Cn = P.coords + ((size_t)unit * a.n_max + a.n_c) * r;
-    for (int o = tid; o < b * r; o += FT) {
-        const int i = o / r, c = o % r;
-        float s0 = 0.f, s1 = 0.f;
-        if (c < kp) {
-            const float *f = sA + i * LDS, *bc = sBp + c * LDS;
-            for (int jj = 0; jj < D; jj += 2) {
-                s0 = fmaf(f[jj], bc[jj], s0);
-                s1 = fmaf(f[jj + 1], bc[jj + 1], s1);
-            }
-        }
-        Cn[(size_t)i * r + c] = s0 + s1;
-    }
+    tile_gemm<2, 4>(b, kp, D, [&](int i, int jj) { return sA[i * LDS + jj]; },
+                    [&](int jj, int c) { return sBp[c * LDS + jj]; },
+                    [&](int i, int c, float v) { Cn[(size_t)i * r + c] = v; });
+    for (int o = tid; o < b * (r - kp); o += FT)
+        Cn[(size_t)(o / (r - kp)) * r + kp + o % (r - kp)] = 0.f;
 }
 
 // History rotation: old coordinates move with the basis, C[0:n] <- C[0:n] H[:k] (iS-KV summary,
