@@ -233,6 +233,7 @@ WL_LONG = syn.WORKLOADS[3]
 # DRAM bytes (read + write) of one launch of the split kernel as ncu counted them for the current
 # kernel: the t = 4096 launch of the bench workload (--profile-case) and the long-context launch
 # (--profile-case long). Set to None whenever the kernel changes until it is captured again.
+FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12    # fp32 FMA peak of the B200 at its max SM clock
 TRAFFIC_T4096 = 13_452_800
 TRAFFIC_LONG = 833_116_928
 
@@ -374,7 +375,10 @@ def all_layers_decode_step(args, dev, flush, steps: int = 5):
                 for h in range(H):
                     Kr[l, sq, h] = syn.device_rows(wl, sq, l, h, 0, device=dev)
                     Vr[l, sq, h] = syn.device_rows(wl, sq, l, h, 1, device=dev)
+        fa0, fa1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fa0.record(s)
         cache.append(-1, Kr, Vr, s.cuda_stream)
+        fa1.record(s)
         del Kr, Vr
         gen = torch.Generator(device=dev)
         gen.manual_seed(2024)
@@ -385,6 +389,7 @@ def all_layers_decode_step(args, dev, flush, steps: int = 5):
     s.synchronize()
     st = cache.status(s.cuda_stream)
     assert st == 0, f"device status {st} after filling the 32-layer cache"
+    append_ms = fa0.elapsed_time(fa1)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
         for l in range(L):
@@ -403,7 +408,27 @@ def all_layers_decode_step(args, dev, flush, steps: int = 5):
     assert cache.status(s.cuda_stream) == 0 and bool(torch.isfinite(out).all())
     del g
     cache.close()
-    return 1e3 * float(np.median(ms)), L * decode_bytes(T, wl)
+    return 1e3 * float(np.median(ms)), L * decode_bytes(T, wl), append_ms
+
+
+def fold_flops(wl, T: int) -> float:
+    """Algorithmic flops of all folds of one append of T rows per unit (all layers, sequences,
+    kv-heads, both paths): per fold 4 b d k (projection) + 4 d b^2 - 4 b^3 / 3 (residual QR, p = b)
+    + 2 m n^2 + 11 n^3 (core SVD, m = k + b, n = k + p) + 2 d (k + p) r (new basis)
+    + 2 n_c k r (history rotation) + 2 b d r (new rows' coordinates)."""
+    b, d = wl.block, D
+    units = wl.n_layers * wl.batch * wl.n_kv_heads
+    total = 0.0
+    for r in (wl.rank_k, wl.rank_v):
+        k, n_c = 0, 0
+        for _ in range(wl.n_c(T) // b):
+            p = min(b, d - k)
+            m, n = k + b, k + p
+            total += units * (4 * b * d * k + 4 * d * b * p - 4 * p ** 3 / 3 + 2 * m * n * n
+                              + 11 * n ** 3 + 2 * d * (k + p) * r + 2 * n_c * k * r + 2 * b * d * r)
+            k = min(r, k + p)
+            n_c += b
+    return total
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -588,8 +613,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # ---- decode over a long history (HBM-bound regime), rank 0 of a single-GPU run only --------
     long_us, long_bytes = (long_context_decode(args, dev, flush) if world == 1 and rank == 0
                            else (None, None))
-    step_us, step_bytes = (all_layers_decode_step(args, dev, flush) if world == 1 and rank == 0
-                           else (None, None))
+    step_us, step_bytes, append_ms = (all_layers_decode_step(args, dev, flush)
+                                      if world == 1 and rank == 0 else (None, None, None))
     pre_ms, pre_updates, pre_dec_us, pre_dec_bytes = (
         prefill_and_decode(args, dev, flush) if world == 1 and rank == 0
         else (None, None, None, None))
@@ -637,6 +662,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "frac": step_bytes / (step_us / 1e6) / 1e9 / hbm, "traffic": None,
             "bytes_per_step": step_bytes, "step_us": step_us,
             "tok_per_s_one_sequence": 1e6 / step_us},
+        "fold_all_layers": None if append_ms is None else {
+            "bound": "fp32 fma", "workload": (f"{WL_LAYERS.name}: one append of all {WL_LAYERS.tokens} "
+                                              f"rows of every layer (512 units per fold launch)"),
+            "folds_per_unit": WL_LAYERS.n_c(WL_LAYERS.tokens) // WL_LAYERS.block,
+            "append_ms": append_ms,
+            "head_block_updates_per_s": (2 * WL_LAYERS.n_layers * WL_LAYERS.n_kv_heads
+                                         * (WL_LAYERS.n_c(WL_LAYERS.tokens) // WL_LAYERS.block)
+                                         / (append_ms / 1e3)),
+            "achieved_tflops": fold_flops(WL_LAYERS, WL_LAYERS.tokens) / (append_ms / 1e3) / 1e12,
+            "peak_tflops": FMA_PEAK_TFLOPS,
+            "frac": fold_flops(WL_LAYERS, WL_LAYERS.tokens) / (append_ms / 1e3) / 1e12 / FMA_PEAK_TFLOPS,
+            "peak_source": "148 SMs x 128 fp32 lanes x 2 x 1.965 GHz (derived from the unit counts)"},
         "long_prefill": None if pre_ms is None else {
             "workload": (f"{WL_PREFILL.name}: one layer, {WL_PREFILL.prefill}-row prefill in one "
                          "append, then decode at that length"),
