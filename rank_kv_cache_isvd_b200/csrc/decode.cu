@@ -305,17 +305,11 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeArgs a) {
 cudaError_t launch_decode(const DecodeArgs &a, int n_units, cudaStream_t s) {
     const DecSmem L = dec_layout(a.r[0], a.G);
     const size_t smem = (size_t)L.total * sizeof(float);
-    static bool attr_set = false;
-    if (!attr_set) {
-        const DecSmem Lmax = dec_layout(128, GMAX);
-        cudaError_t e = cudaFuncSetAttribute(decode_split_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(Lmax.total * sizeof(float)));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static size_t attr[64] = {0};
+    cudaError_t e = ensure_smem((const void *)decode_split_kernel, smem, attr);
+    if (e != cudaSuccess) return e;
     decode_split_kernel<<<dim3(a.n_split, n_units), DEC_THREADS, smem, s>>>(a);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     decode_combine_kernel<<<n_units, D, 0, s>>>(a);
     return cudaGetLastError();

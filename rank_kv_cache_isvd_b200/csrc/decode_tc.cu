@@ -388,8 +388,8 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
             if (rope) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const float4 w = cs[8 * ch + q];              // (cos, sin) of two pairs
-                    const float2 c = make_float2(w.x, w.z), sn = make_float2(w.y, w.w);
+                    const float4 w = cs[8 * ch + q];              // (cos, cos, sin, sin)
+                    const float2 c = make_float2(w.x, w.y), sn = make_float2(w.z, w.w);
                     const float2 ys = __fmul2_rn(H2[q], sn), xs = __fmul2_rn(L2[q], sn);
                     const float2 xl = __ffma2_rn(L2[q], c, make_float2(-ys.x, -ys.y));
                     H2[q] = __ffma2_rn(H2[q], c, xs);

@@ -913,14 +913,10 @@ __global__ void __launch_bounds__(ROT_THREADS) rotate_kernel(RotArgs a) {
 }
 
 cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s) {
-    static bool attr_set = false;
+    static size_t attr[64] = {0};
     const size_t smem = fold_smem_bytes();
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(fold_core_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    const cudaError_t e = ensure_smem((const void *)fold_core_kernel, smem, attr);
+    if (e != cudaSuccess) return e;
     fold_core_kernel<<<dim3(n_units, 2), FT, smem, s>>>(a);
     return cudaGetLastError();
 }
@@ -929,14 +925,9 @@ cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s) {
     if (a.n_old <= 0) return cudaSuccess;
     const int rmax = a.path[0].r > a.path[1].r ? a.path[0].r : a.path[1].r;
     const size_t smem = (size_t)(rmax * rmax + ROT_ROWS * (rmax + 1)) * sizeof(float);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(rotate_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)((128 * 128 + ROT_ROWS * 129) * sizeof(float)));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static size_t attr[64] = {0};
+    const cudaError_t e = ensure_smem((const void *)rotate_kernel, smem, attr);
+    if (e != cudaSuccess) return e;
     const unsigned gx = (unsigned)((a.n_old + ROT_ROWS - 1) / ROT_ROWS);
     rotate_kernel<<<dim3(gx, n_units, 2), ROT_THREADS, smem, s>>>(a);
     return cudaGetLastError();

@@ -169,14 +169,9 @@ __global__ void __launch_bounds__(RF_THREADS) newrows_kernel(NewRowsArgs a) {
 size_t rfactor_smem_bytes() { return ((size_t)D * RF_LDM + D) * sizeof(float); }
 
 cudaError_t launch_rfactor(const RFactorArgs &a, int n_units, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(rfactor_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)rfactor_smem_bytes());
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static size_t attr[64] = {0};
+    const cudaError_t e = ensure_smem((const void *)rfactor_kernel, rfactor_smem_bytes(), attr);
+    if (e != cudaSuccess) return e;
     rfactor_kernel<<<dim3(n_units, 2), RF_THREADS, rfactor_smem_bytes(), s>>>(a);
     return cudaGetLastError();
 }
@@ -184,14 +179,9 @@ cudaError_t launch_rfactor(const RFactorArgs &a, int n_units, cudaStream_t s) {
 cudaError_t launch_newrows(const NewRowsArgs &a, int n_units, cudaStream_t s) {
     const int kpmax = a.path[0].kp > a.path[1].kp ? a.path[0].kp : a.path[1].kp;
     const size_t smem = ((size_t)D * (kpmax | 1) + 32 * (D + 1)) * sizeof(float);
-    static size_t attr = 0;
-    if (smem > attr) {
-        cudaError_t e = cudaFuncSetAttribute(newrows_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        attr = smem;
-    }
+    static size_t attr[64] = {0};
+    const cudaError_t e = ensure_smem((const void *)newrows_kernel, smem, attr);
+    if (e != cudaSuccess) return e;
     const int chunks = (a.b + DEC_TILE - 1) / DEC_TILE;
     newrows_kernel<<<dim3(chunks, n_units, 2), RF_THREADS, smem, s>>>(a);
     return cudaGetLastError();

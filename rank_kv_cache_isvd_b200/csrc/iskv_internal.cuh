@@ -136,7 +136,7 @@ struct TcExtra {
     int kblocks;            // 32-column K-blocks of the key coordinates (ceil(r_K / 32))
     long long row0;         // first coordinate row of this layer in the coordinate tensor map
     int brow0;              // first basis row of this layer (current buffer) in the basis map
-    const float4 *rope_t;   // [DH/2][rope_rows] (cos, sin) of pair pairs, or nullptr
+    const float4 *rope_t;   // [DH/2][rope_rows] (cos, cos, sin, sin) of pair pairs, or nullptr
     long long rope_rows;
     int *status;
 };
@@ -160,6 +160,20 @@ __device__ __forceinline__ float load_row_elem(const void *base, size_t idx, int
     if (kv_dtype == ISKV_BF16)
         return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[idx]);
     return reinterpret_cast<const float *>(base)[idx];
+}
+
+// Raises `fn`'s dynamic shared-memory limit on the current device to at least `bytes`. Function
+// attributes belong to a device, so the largest value set so far is remembered per device in
+// `done` (64 entries, zero-initialised by the caller).
+inline cudaError_t ensure_smem(const void *fn, size_t bytes, size_t *done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (bytes <= done[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done[dev] = bytes;
+    return e;
 }
 
 __device__ __forceinline__ void set_status(int *status, int code) {

@@ -42,9 +42,10 @@ __global__ void rope_table_kernel(float2 *table, long long max_tokens, double th
     table[idx] = make_float2((float)cs, (float)sn);
 }
 
-// Transposed copy for the tensor-core decode: table_t[q][pos] = (cos, sin) of pairs 2q and 2q+1
-// at position pos, so that the 32 rows of a warp read 32 consecutive float4 (one coalesced line)
-// instead of 32 rows 512 bytes apart.
+// Transposed copy for the tensor-core decode: table_t[q][pos] = (cos_2q, cos_2q+1, sin_2q,
+// sin_2q+1) of pairs 2q and 2q+1 at position pos, so that the 32 rows of a warp read 32
+// consecutive float4 (one coalesced line) instead of 32 rows 512 bytes apart, and the two cosines
+// (sines) form one packed fp32 operand.
 __global__ void rope_table_t_kernel(float4 *table_t, long long max_tokens, double theta) {
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= max_tokens * (DH / 2)) return;
@@ -53,7 +54,7 @@ __global__ void rope_table_t_kernel(float4 *table_t, long long max_tokens, doubl
     double s0, c0, s1, c1;
     sincos((double)pos * pow(theta, -2.0 * (2 * q) / (double)D), &s0, &c0);
     sincos((double)pos * pow(theta, -2.0 * (2 * q + 1) / (double)D), &s1, &c1);
-    table_t[idx] = make_float4((float)c0, (float)s0, (float)c1, (float)s1);
+    table_t[idx] = make_float4((float)c0, (float)c1, (float)s0, (float)s1);
 }
 
 cudaError_t launch_rope_table_t(float4 *table_t, long long max_tokens, double theta,
@@ -110,14 +111,9 @@ __global__ void reconstruct_kernel(ReconArgs a) {
 cudaError_t launch_reconstruct(const ReconArgs &a, int n_units, cudaStream_t s) {
     if (a.t <= 0) return cudaSuccess;
     const size_t smem = (size_t)D * ((a.k | 1)) * sizeof(float);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(D * 129 * sizeof(float)));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static size_t attr[64] = {0};
+    const cudaError_t e = ensure_smem((const void *)reconstruct_kernel, smem, attr);
+    if (e != cudaSuccess) return e;
     const unsigned gx = (unsigned)((a.t + 63) / 64);
     reconstruct_kernel<<<dim3(gx, n_units), D, smem, s>>>(a);
     return cudaGetLastError();
