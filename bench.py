@@ -230,12 +230,13 @@ def run_reference(args, rank: int):
 # ---------------------------------------------------------------------------------------------
 WL_LONG = syn.WORKLOADS[3]
 
+FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12    # fp32 FMA peak of the B200 at its max SM clock
+
 # DRAM bytes (read + write) of one launch of the split kernel as ncu counted them for the current
 # kernel: the t = 4096 launch of the bench workload (--profile-case) and the long-context launch
 # (--profile-case long). Set to None whenever the kernel changes until it is captured again.
-FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12    # fp32 FMA peak of the B200 at its max SM clock
-TRAFFIC_T4096 = None
-TRAFFIC_LONG = None
+TRAFFIC_T4096 = 13_451_520
+TRAFFIC_LONG = 834_641_408
 
 
 def long_context_decode(args, dev, flush, calls: int = 10):
