@@ -231,6 +231,7 @@ def run_reference(args, rank: int):
 WL_LONG = syn.WORKLOADS[3]
 
 FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12    # fp32 FMA peak of the B200 at its max SM clock
+HBM_NOMINAL_GBS = 7700.0                              # HBM3e nominal bandwidth (HGX figure), context
 
 # DRAM bytes (read + write) of one launch of the split kernel as ncu counted them for the current
 # kernel: the t = 4096 launch of the bench workload (--profile-case) and the long-context launch
@@ -637,7 +638,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "graph": "the step's C-ABI calls captured once into a CUDA graph"},
         "roofline": {"bound": "hbm", "kernel": "decode attention (split + combine)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": TRAFFIC_T4096,
+                     "frac": achieved / hbm, "frac_of_nominal": achieved / HBM_NOMINAL_GBS,
+                     "traffic": TRAFFIC_T4096,
                      "traffic_launch": ("ncu count of the t = 4096 launch (--profile-case); its "
                                         f"algorithmic bytes are {decode_bytes(WL.tokens)}"),
                      "peak_source": f"{which} MEASURED_PEAKS hbm_gbs",
@@ -654,13 +656,17 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "bound": "hbm", "kernel": "decode attention (split + combine)",
             "workload": f"{WL_LONG.name}: one layer at t = {WL_LONG.tokens}",
             "achieved": long_bytes / (long_us / 1e6) / 1e9, "peak": hbm, "unit": "GB/s",
-            "frac": long_bytes / (long_us / 1e6) / 1e9 / hbm, "traffic": TRAFFIC_LONG,
+            "frac": long_bytes / (long_us / 1e6) / 1e9 / hbm,
+            "frac_of_nominal": long_bytes / (long_us / 1e6) / 1e9 / HBM_NOMINAL_GBS,
+            "traffic": TRAFFIC_LONG,
             "bytes_per_launch": long_bytes, "launch_us": long_us},
         "roofline_32_layer_step": None if step_us is None else {
             "bound": "hbm", "kernel": "decode attention (split + combine), 32 calls",
             "workload": f"{WL_LAYERS.name}: one decode step of all layers at t = {WL_LAYERS.tokens}",
             "achieved": step_bytes / (step_us / 1e6) / 1e9, "peak": hbm, "unit": "GB/s",
-            "frac": step_bytes / (step_us / 1e6) / 1e9 / hbm, "traffic": None,
+            "frac": step_bytes / (step_us / 1e6) / 1e9 / hbm,
+            "frac_of_nominal": step_bytes / (step_us / 1e6) / 1e9 / HBM_NOMINAL_GBS,
+            "traffic": None,
             "bytes_per_step": step_bytes, "step_us": step_us,
             "tok_per_s_one_sequence": 1e6 / step_us},
         "fold_all_layers": None if append_ms is None else {
