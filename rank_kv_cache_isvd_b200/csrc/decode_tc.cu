@@ -31,7 +31,7 @@ constexpr int MERGE_REG = 48;             // splits whose partials a merge threa
 constexpr int KBLK_BYTES = 128 * 128;     // one K-block: 128 rows x 32 fp32
 
 struct TcLayout {
-    uint32_t b_hi, b_lo, a_hi, a_lo, v, q, x, red, acc, bars, total;
+    uint32_t b_hi, b_lo, a_hi, a_lo, v, q, x, red, bars, total;
 };
 
 // Shared-memory plan of the split kernel. Window tiles stage their exact value rows from a_hi
@@ -56,7 +56,6 @@ __host__ __device__ inline TcLayout tc_layout(int kblocks, int rV, int esz, int 
     L.q = o; o += G * D * 4;
     L.x = o; o += 2 * G * 128 * 4;           // score halves, then (aliased) probabilities
     L.red = o; o += 2 * 4 * GMAX * 4;
-    L.acc = o; o += G * D * 4;
     L.bars = o; o += 64;
     L.total = o + 1024;                    // slack for aligning the base to 1024 bytes
     return L;
@@ -173,7 +172,6 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
     float *sX = reinterpret_cast<float *>(sm + L.x);            // [2 halves][G][128]
     float *sP = sX;                                             // [128][GT] (after the scores)
     float *sRed = reinterpret_cast<float *>(sm + L.red);        // [2][4][GMAX]
-    float *sAcc = reinterpret_cast<float *>(sm + L.acc);        // [G][D] running value sums
     uint64_t *bar_a = reinterpret_cast<uint64_t *>(sm + L.bars);
     uint64_t *bar_v = bar_a + 1;
     uint64_t *bar_mma = bar_a + 2;
@@ -272,7 +270,6 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
         const float4 *q4 = reinterpret_cast<const float4 *>(a.q + ((size_t)seq * a.H * G + (size_t)h * G) * D);
         float4 *s4 = reinterpret_cast<float4 *>(sQ);
         if (!comp && tid < G * D / 4) s4[tid] = q4[tid];
-        for (int o = tid; o < G * D; o += TC_THREADS) sAcc[o] = 0.f;
     }
     tc_fence_before();
     __syncthreads();
@@ -288,6 +285,16 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
     }
     const int row = 32 * wq + lane;
     const int jb = 32 * half;                   // this thread's first channel pair
+    // value sums in rank space (or channels, window CTAs): thread = (channel quad qd, row slice
+    // sl); each thread keeps its slice's sums in registers over all tiles of the split, rescaled
+    // with the running max, and the slices are added once at the end
+    const int nq = (nacc + 3) >> 2;
+    const int nqp = nq <= 8 ? 8 : nq <= 16 ? 16 : 32;
+    const int nsl = TC_THREADS / nqp;
+    const int qd = tid & (nqp - 1), sl = tid / nqp;
+    float4 vacc[GT];
+#pragma unroll
+    for (int g = 0; g < GT; ++g) vacc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
 
     // thread 0 issues the three-term tf32 product of the staged key-coordinate tile into TMEM
     // accumulator `buf` (columns 128 buf .. 128 buf + 127)
@@ -473,13 +480,11 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
                                 (sRed[6 * GMAX + g] + sRed[7 * GMAX + g]);
                 lrun[g] = fmaf(lrun[g], alpha[g], s);
             }
-        // ---- value accumulation: sAcc[g][c] = sAcc * alpha_g + sum_i p[g][i] V[i][c] ------------
-        // thread = (channel quad qd, row slice sl): quads vary fastest, so the lanes of a
-        // shared-memory phase read consecutive 16-byte (8-byte for bf16) pieces of one staged row
-        // (no bank conflicts); slice sl takes rows sl, sl + nsl, ... Quads past the row's end
-        // (nqp is a power of two) read the next row's values and are never used. The slices'
-        // sums meet in shared memory: first within the warp (shuffles), then across the 8 warps
-        // in the value stage itself once every warp is done reading it.
+        // ---- value accumulation: vacc_g = vacc_g * alpha_g + sum_i p[g][i] V[i][quad] ------------
+        // quads vary fastest across a warp's lanes, so the lanes of a shared-memory phase read
+        // consecutive 16-byte (8-byte for bf16) pieces of one staged row (no bank conflicts);
+        // slice sl takes rows sl, sl + nsl, ... Quads past the row's end (nqp is a power of two)
+        // read the next row's values and are never used.
         ok = __syncthreads_and(mbar_wait(bar_v, ph_v)) != 0;
         if (!ok) break;
         pend_v = false;
@@ -514,73 +519,41 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
             }
             __syncthreads();
         }
-        {
-            const int nq = (nacc + 3) >> 2;
-            const int nqp = nq <= 8 ? 8 : nq <= 16 ? 16 : 32;
-            const int nsl = TC_THREADS / nqp;
-            const int qd = tid & (nqp - 1), sl = tid / nqp;
-            float4 acc4[GT];
 #pragma unroll
-            for (int g = 0; g < GT; ++g) acc4[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-            for (int i = sl; i < rows; i += nsl) {
-                const float4 v = load_v4(bV + (size_t)i * vld, 4 * qd, vfmt);
-                const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
-                float pv[GT];                   // this row's probabilities, one vector load
-                if (GT >= 4) {
-#pragma unroll
-                    for (int g4 = 0; g4 < GT / 4; ++g4) {
-                        const float4 p4 = reinterpret_cast<const float4 *>(sP + i * GT)[g4];
-                        pv[4 * g4] = p4.x;
-                        pv[4 * g4 + 1] = p4.y;
-                        pv[4 * g4 + 2] = p4.z;
-                        pv[4 * g4 + 3] = p4.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int g = 0; g < GT; ++g) pv[g] = sP[i * GT + g];
-                }
-#pragma unroll
-                for (int g = 0; g < GT; ++g)
-                    if (g < G) {
-                        const float pg = pv[g];
-                        const float2 p2 = make_float2(pg, pg);
-                        const float2 a01 = __ffma2_rn(p2, v01, make_float2(acc4[g].x, acc4[g].y));
-                        const float2 a23 = __ffma2_rn(p2, v23, make_float2(acc4[g].z, acc4[g].w));
-                        acc4[g] = make_float4(a01.x, a01.y, a23.x, a23.y);
-                    }
+        for (int g = 0; g < GT; ++g)
+            if (g < G) {
+                const float2 al2 = make_float2(alpha[g], alpha[g]);
+                const float2 a01 = __fmul2_rn(al2, make_float2(vacc[g].x, vacc[g].y));
+                const float2 a23 = __fmul2_rn(al2, make_float2(vacc[g].z, vacc[g].w));
+                vacc[g] = make_float4(a01.x, a01.y, a23.x, a23.y);
             }
-            // slices that share a warp: lanes nqp, 2 nqp, ... apart
+#pragma unroll 4
+        for (int i = sl; i < rows; i += nsl) {
+            const float4 v = load_v4(bV + (size_t)i * vld, 4 * qd, vfmt);
+            const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
+            float pv[GT];                       // this row's probabilities, one vector load
+            if (GT >= 4) {
+#pragma unroll
+                for (int g4 = 0; g4 < GT / 4; ++g4) {
+                    const float4 p4 = reinterpret_cast<const float4 *>(sP + i * GT)[g4];
+                    pv[4 * g4] = p4.x;
+                    pv[4 * g4 + 1] = p4.y;
+                    pv[4 * g4 + 2] = p4.z;
+                    pv[4 * g4 + 3] = p4.w;
+                }
+            } else {
+#pragma unroll
+                for (int g = 0; g < GT; ++g) pv[g] = sP[i * GT + g];
+            }
 #pragma unroll
             for (int g = 0; g < GT; ++g)
                 if (g < G) {
-                    for (int o = nqp; o < 32; o <<= 1) {
-                        acc4[g].x += __shfl_xor_sync(0xffffffffu, acc4[g].x, o);
-                        acc4[g].y += __shfl_xor_sync(0xffffffffu, acc4[g].y, o);
-                        acc4[g].z += __shfl_xor_sync(0xffffffffu, acc4[g].z, o);
-                        acc4[g].w += __shfl_xor_sync(0xffffffffu, acc4[g].w, o);
-                    }
+                    const float pg = pv[g];
+                    const float2 p2 = make_float2(pg, pg);
+                    const float2 a01 = __ffma2_rn(p2, v01, make_float2(vacc[g].x, vacc[g].y));
+                    const float2 a23 = __ffma2_rn(p2, v23, make_float2(vacc[g].z, vacc[g].w));
+                    vacc[g] = make_float4(a01.x, a01.y, a23.x, a23.y);
                 }
-            float *sRedV = reinterpret_cast<float *>(bV);       // [8 warps][G][4 nqp]
-            __syncthreads();                                    // value stage consumed
-            if (lane < nqp) {
-#pragma unroll
-                for (int g = 0; g < GT; ++g)
-                    if (g < G)
-                        reinterpret_cast<float4 *>(sRedV)[(warp * G + g) * nqp + qd] = acc4[g];
-            }
-            __syncthreads();
-            for (int o = tid; o < G * nacc; o += TC_THREADS) {
-                const int g = o / nacc, c = o - g * nacc;
-                float sum = 0.f;
-#pragma unroll
-                for (int w = 0; w < 8; ++w) sum += sRedV[((w * G + g) * nqp) * 4 + c];
-                float al = 1.f;
-#pragma unroll
-                for (int gg = 0; gg < GT; ++gg)
-                    if (gg == g) al = alpha[gg];
-                sAcc[g * D + c] = fmaf(sAcc[g * D + c], al, sum);
-            }
         }
         fence_proxy_async_smem();              // the stage was written through the generic proxy
         tc_fence_before();
@@ -598,11 +571,35 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
         if (pend_m) mbar_wait(bar_mma, ph_m);
     }
 
-    // ---- partials: [m, l, acc[nacc]] per q-head (sAcc is final after the last tile's barrier) ---
+    // ---- the slices' value sums meet once: within the warp (shuffles), then across the 8 warps
+    //      in the value stage (free: every copy into it has completed or drained) -------------------
+#pragma unroll
+    for (int g = 0; g < GT; ++g)
+        if (g < G) {
+            for (int o = nqp; o < 32; o <<= 1) {
+                vacc[g].x += __shfl_xor_sync(0xffffffffu, vacc[g].x, o);
+                vacc[g].y += __shfl_xor_sync(0xffffffffu, vacc[g].y, o);
+                vacc[g].z += __shfl_xor_sync(0xffffffffu, vacc[g].z, o);
+                vacc[g].w += __shfl_xor_sync(0xffffffffu, vacc[g].w, o);
+            }
+        }
+    float *sRedV = reinterpret_cast<float *>(bV);               // [8 warps][G][4 nqp]
+    __syncthreads();
+    if (lane < nqp) {
+#pragma unroll
+        for (int g = 0; g < GT; ++g)
+            if (g < G) reinterpret_cast<float4 *>(sRedV)[(warp * G + g) * nqp + qd] = vacc[g];
+    }
+    __syncthreads();
+
+    // ---- partials: [m, l, acc[nacc]] per q-head ---------------------------------------------------
     float *ws = a.ws + ((size_t)ul * a.max_splits + split) * G * (2 + D);
     for (int o = tid; o < G * nacc; o += TC_THREADS) {
         const int g = o / nacc, c = o % nacc;
-        ws[g * (2 + D) + 2 + c] = sAcc[g * D + c];
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) sum += sRedV[((w * G + g) * nqp) * 4 + c];
+        ws[g * (2 + D) + 2 + c] = sum;
     }
     if (tid < G) {
 #pragma unroll
