@@ -236,8 +236,8 @@ HBM_NOMINAL_GBS = 7700.0                              # HBM3e nominal bandwidth 
 # DRAM bytes (read + write) of one launch of the split kernel as ncu counted them for the current
 # kernel: the t = 4096 launch of the bench workload (--profile-case) and the long-context launch
 # (--profile-case long). Set to None whenever the kernel changes until it is captured again.
-TRAFFIC_T4096 = None
-TRAFFIC_LONG = None
+TRAFFIC_T4096 = 13_453_824
+TRAFFIC_LONG = 836_655_360
 
 
 def long_context_decode(args, dev, flush, calls: int = 10):
