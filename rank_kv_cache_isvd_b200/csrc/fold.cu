@@ -350,10 +350,10 @@ __device__ __forceinline__ void tile_gemm(int M, int N, int K, LA la, LB lb, ST 
 // Householder QR in shared memory (R in place, reflectors kept below it).
 //
 // Step j reflects the pivot row j and the body rows y0(j) .. y1 - 1 of column j: lane l holds
-// body rows y0 + l + 32 u (u < 4) of the reflector in registers, each warp updates trailing
-// columns j + 1 + warp + FW m, eight at a time with overlapped reductions. Warp 0's first batch
-// holds column j + 1, so it forms the next reflector right after that column's update (norm from
-// the updated values in its registers); each step therefore ends with a single barrier.
+// body rows y0 + l + 32 u (u < 4) of the reflector in registers. Warp 0 updates column j + 1
+// alone and forms the next reflector from the updated values in its registers; warps 1 .. FW - 1
+// update the other trailing columns, eight at a time with overlapped reductions. Each step
+// therefore ends with a single barrier, and the next reflector is off the other warps' path.
 // Reflectors are stored scaled in the body rows of their column (v_i below the pivot, v_pivot = 1
 // implicit) with tau_j in sTau[j]; R's diagonal entries replace the pivots.
 //
@@ -435,50 +435,78 @@ __device__ void householder_qr(const M &m, int n, float *sTau) {
             const int i = y0 + lane + 32 * u;
             v[u] = i < y1 ? m.at(i, j) : 0.f;
         }
-        for (int cb = j + 1 + warp; cb < n; cb += 8 * FW) {
-            float w[8], xq[8][4], pj[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int c = min(cb + q * FW, n - 1);
-                w[q] = 0.f;
+        if (warp == 0) {
+            // column j + 1 alone, then its reflector (the next step's), off the other warps' path
+            if (j + 1 < n) {
+                const int c = j + 1;
+                float x[4], w = 0.f;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int i = y0 + lane + 32 * u;
-                    xq[q][u] = i < y1 ? m.at(i, c) : 0.f;
-                    w[q] = fmaf(v[u], xq[q][u], w[q]);
+                    x[u] = i < y1 ? m.at(i, c) : 0.f;
+                    w = fmaf(v[u], x[u], w);
                 }
-                pj[q] = pr[c * ps];
+                w = warp_sum(w);
+                const float pj = pr[c * ps];
+                const float wq = (w + pj) * tau;
+                __syncwarp();
+                if (lane == 0) pr[c * ps] = pj - wq;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = y0 + lane + 32 * u;
+                    x[u] = fmaf(-wq, v[u], x[u]);
+                    if (i < y1) m.at(i, c) = x[u];
+                }
+                // the next pivot: a body row of this step (one lane holds it) or untouched
+                const int rel = y0n - 1 - y0;
+                float al;
+                if (rel >= 0) {
+                    const int ur = rel >> 5;
+                    const float cand = ur == 0 ? x[0] : ur == 1 ? x[1] : ur == 2 ? x[2] : x[3];
+                    al = __shfl_sync(0xffffffffu, cand, rel & 31);
+                } else {
+                    al = m.pivot(j + 1)[(j + 1) * ps];
+                }
+                __syncwarp();
+                qr_reflector(m, j + 1, y0, y0n, al, x, sTau);
             }
+        } else {
+            // columns j + 2 ... over warps 1 .. FW - 1, eight per batch (overlapped reductions)
+            constexpr int W1 = FW - 1;
+            for (int cb = j + 2 + (warp - 1); cb < n; cb += 8 * W1) {
+                float w[8], xq[8][4], pj[8];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-                for (int q = 0; q < 8; ++q) w[q] += __shfl_xor_sync(0xffffffffu, w[q], o);
-            __syncwarp();
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int c = cb + q * FW;
-                if (c < n) {
-                    const float wq = (w[q] + pj[q]) * tau;
-                    if (lane == 0) pr[c * ps] = pj[q] - wq;
+                for (int q = 0; q < 8; ++q) {
+                    const int c = min(cb + q * W1, n - 1);
+                    w[q] = 0.f;
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int i = y0 + lane + 32 * u;
-                        xq[q][u] = fmaf(-wq, v[u], xq[q][u]);
-                        if (i < y1) m.at(i, c) = xq[q][u];
+                        xq[q][u] = i < y1 ? m.at(i, c) : 0.f;
+                        w[q] = fmaf(v[u], xq[q][u], w[q]);
+                    }
+                    pj[q] = pr[c * ps];
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) w[q] += __shfl_xor_sync(0xffffffffu, w[q], o);
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int c = cb + q * W1;
+                    if (c < n) {
+                        const float wq = (w[q] + pj[q]) * tau;
+                        if (lane == 0) pr[c * ps] = pj[q] - wq;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int i = y0 + lane + 32 * u;
+                            if (i < y1) m.at(i, c) = fmaf(-wq, v[u], xq[q][u]);
+                        }
                     }
                 }
-            }
-            if (cb == j + 1 && j + 1 < n) {            // warp 0: column j + 1 is final for step j
-                float al = 0.f;
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    if (y0 + lane + 32 * u == y0n - 1) al = xq[0][u];
-                al = warp_sum(al);                     // (at most one lane holds the pivot)
-                if (y0n - 1 < y0) al = m.pivot(j + 1)[(j + 1) * ps];   // untouched by step j
                 __syncwarp();
-                qr_reflector(m, j + 1, y0, y0n, al, xq[0], sTau);
             }
-            __syncwarp();
         }
         __syncthreads();
     }
