@@ -201,6 +201,18 @@ def oracle_sample(seq: int = 0, heads: int = 2, decodes: int = 256):
     }
 
 
+def cpu_baseline() -> dict:
+    """The oracle timed on the host with the BLAS pool as configured and with one thread (the
+    oracle's matrices are small, so the pool's threads rarely help)."""
+    from threadpoolctl import threadpool_limits
+    cb = oracle_sample()
+    out = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    out["host_cores"] = cb["host_cores"]
+    with threadpool_limits(limits=1):
+        out["value_1_thread"] = oracle_sample()["value"]
+    return out
+
+
 def run_reference(args, rank: int):
     if rank != 0:
         return
@@ -696,9 +708,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = oracle_sample()
-        out["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
-        out["cpu_baseline"]["host_cores"] = cb["host_cores"]
+        out["cpu_baseline"] = cpu_baseline()
     del g
     cache.close()
     if rank == 0:
