@@ -35,7 +35,12 @@ Readings taken where the page is silent (each also stated at its definition):
   it; the stale-coordinate variant does;
 * the "stale coordinates" variant (``rotate=False``) updates ``Sigma`` and ``B`` exactly as above
   but keeps the old rows' coordinates ``U Sigma`` unrotated (zero-padded or truncated to the new
-  rank) and reconstructs them against the new basis; new rows get ``F B+``.
+  rank) and reconstructs them against the new basis; new rows get ``F B+``;
+* the "fixed basis" variant (``fixed_basis=True``, section "Ablation Study": bases kept fixed)
+  runs the regular update for the first ``ceil(min(r, d) / block)`` blocks, which fill the rank
+  budget, and then freezes ``B`` and ``Sigma``: every later block is stored as its coordinates
+  ``F B`` in the frozen basis (its orthogonal projection onto ``span B``) and old coordinates stay
+  as they are (the basis does not move, so nothing drifts).
 
 Parity: every function here is pinned by ``tests/test_oracle_*.py`` (closed forms, library special
 cases, invariants and brute force); none is "parity unpinned".
@@ -172,12 +177,16 @@ class OracleUnit:
     "Reconstruction and Storage".
     """
 
-    def __init__(self, d: int, rank: int, block: int, window: int, rotate: bool = True):
+    def __init__(self, d: int, rank: int, block: int, window: int, rotate: bool = True,
+                 fixed_basis: bool = False):
         self.d, self.rank, self.block, self.window, self.rotate = d, rank, block, window, rotate
+        self.fixed_basis = fixed_basis
+        # folds that run the regular update before a fixed basis freezes (fill the rank budget)
+        self.adapt_folds = -(-min(rank, d) // block)
         self.U = np.zeros((0, 0))
         self.sigma = np.zeros(0)
         self.B = np.zeros((d, 0))
-        self.C_stale = np.zeros((0, 0))      # stored coordinates when rotate=False
+        self.C_stale = np.zeros((0, 0))      # stored coordinates (stale or fixed-basis modes)
         self._exact: list[np.ndarray] = []
         self.t = 0
         self.n = 0
@@ -194,7 +203,7 @@ class OracleUnit:
 
     def coords(self) -> np.ndarray:
         """Stored history coordinates ``U Sigma`` (``n x k``)."""
-        if not self.rotate:
+        if not self.rotate or self.fixed_basis:
             return self.C_stale
         return self.U * self.sigma
 
@@ -222,8 +231,17 @@ class OracleUnit:
 
     def _fold(self, F: np.ndarray) -> None:
         k_old = self.k
+        if self.fixed_basis and self.folds >= self.adapt_folds:
+            # frozen basis: the block's rows are stored as their coordinates in it
+            self.C_stale = np.vstack([self.C_stale, F @ self.B])
+            self.n += F.shape[0]
+            self.folds += 1
+            return
         U_new, s, B_new, H, _ = fold(self.U, self.sigma, self.B, F, self.rank)
-        if not self.rotate:
+        if self.fixed_basis:
+            # still adapting: coordinates rotate with the basis, as in the regular update
+            self.C_stale = U_new * s
+        elif not self.rotate:
             kp = s.size
             C = np.zeros((self.n, kp))
             m = min(k_old, kp)
@@ -270,10 +288,12 @@ class OracleCache:
 
     def __init__(self, batch: int, n_layers: int, n_kv_heads: int, n_q_heads: int,
                  head_dim: int, rank_k: int, rank_v: int, block: int, window: int,
-                 rope: bool = False, rope_theta: float = 5e5, rotate: bool = True):
+                 rope: bool = False, rope_theta: float = 5e5, rotate: bool = True,
+                 fixed_basis: bool = False):
         self.batch, self.n_layers, self.n_kv, self.n_q = batch, n_layers, n_kv_heads, n_q_heads
         self.d, self.rope, self.theta = head_dim, rope, rope_theta
-        self.units = [[[[OracleUnit(head_dim, rank_k if w == 0 else rank_v, block, window, rotate)
+        self.units = [[[[OracleUnit(head_dim, rank_k if w == 0 else rank_v, block, window, rotate,
+                                    fixed_basis)
                          for w in range(2)] for _ in range(n_kv_heads)] for _ in range(batch)]
                       for _ in range(n_layers)]
 

@@ -234,3 +234,66 @@ def test_storage_formula_counts_stored_scalars():
     stored = unit.coords().size + unit.B.size + unit.sigma.size + unit.exact.size
     assert unit.storage_scalars() == stored
     assert stored == unit.k * (unit.n + d + 1) + d * (53 - unit.n)
+
+
+# ---------------------------------------------------------------------------------------------
+# stale coordinates, closed form: with r >= d nothing is truncated, so after the second fold the
+# basis spans all stacked rows and its first k1 columns are fixed by the sign convention
+# ---------------------------------------------------------------------------------------------
+def test_stale_rows_closed_form_two_folds():
+    d, b = 16, 4
+    X = _stream(d, d, 31, decay=0.5, noise=0.05)[:2 * b]
+    F1, F2 = X[:b], X[b:]
+    stale = OracleUnit(d, d, b, 0, rotate=False)
+    stale.append(F1)
+    B1 = stale.B.copy()
+    k1 = B1.shape[1]
+    # first fold: B1 spans the right singular vectors of F1 (library SVD), any signs
+    V1 = np.linalg.svd(F1, full_matrices=False)[2][:k1].T
+    np.testing.assert_allclose(np.abs(B1.T @ V1), np.eye(k1), atol=1e-10)
+    # its stored coordinates are F1 B1 (no truncation: F1 = U1 Sigma1 B1^T)
+    np.testing.assert_allclose(stale.coords(), F1 @ B1, atol=1e-12)
+    stale.append(F2)
+    assert stale.n == 2 * b and stale.k == 2 * b
+    # second basis: right singular vectors of the stacked rows (library SVD), column c < k1
+    # oriented along B1's column c (the sign convention)
+    V2 = np.linalg.svd(X, full_matrices=False)[2][:2 * b].T
+    for c in range(k1):
+        if V2[:, c] @ B1[:, c] < 0:
+            V2[:, c] = -V2[:, c]
+    rec = stale.reconstruct()
+    # old rows keep their first-fold coordinates, now read against the new basis' first k1
+    # columns; new rows are coded in the new basis, which spans them, so they come back exactly
+    np.testing.assert_allclose(rec[:b], (F1 @ B1) @ V2[:, :k1].T, atol=1e-10)
+    np.testing.assert_allclose(rec[b:], F2, atol=1e-10)
+    # and this differs from the synchronised history, which reproduces F1
+    assert np.linalg.norm(rec[:b] - F1) > 1e-3 * np.linalg.norm(F1)
+
+
+# ---------------------------------------------------------------------------------------------
+# fixed basis ("Ablation Study"): the update runs until the rank budget is filled, then every
+# block is stored as its projection onto the frozen basis
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("d,r,b,w", [(16, 4, 6, 3), (16, 6, 4, 5), (12, 5, 5, 0)])
+def test_fixed_basis_projects_later_blocks(d, r, b, w):
+    X = _stream(9 * b + w, d, 37 + r + b, decay=0.5, noise=0.05)
+    unit = OracleUnit(d, r, b, w, fixed_basis=True)
+    unit.append(X)
+    n = unit.n
+    f0 = -(-min(r, d) // b)                 # folds that fill the rank budget
+    # the frozen basis is the rank-r truncated SVD basis of the first f0 blocks (no truncation
+    # happens before the last of them, so the regular update is the SVD of their stacked rows)
+    A = X[:f0 * b]
+    Vt = np.linalg.svd(A, full_matrices=False)[2]
+    kf = min(r, A.shape[0], d)
+    P = Vt[:kf].T @ Vt[:kf]
+    np.testing.assert_allclose(unit.B @ unit.B.T, P, atol=1e-10)
+    rec = unit.reconstruct()
+    u, s, v = svd_r(A, r)
+    np.testing.assert_allclose(rec[:f0 * b], (u * s) @ v.T, atol=1e-10)
+    np.testing.assert_allclose(rec[f0 * b:n], X[f0 * b:n] @ P, atol=1e-10)
+    np.testing.assert_array_equal(rec[n:], X[n:])
+    # the adapting cache does better on the same rows
+    sync = OracleUnit(d, r, b, w)
+    sync.append(X)
+    assert np.linalg.norm(sync.reconstruct()[:n] - X[:n]) < np.linalg.norm(rec[:n] - X[:n])

@@ -79,7 +79,39 @@ def _pin_schedule(m):
             and m.n_compressed(320, 64, 256) == 64 and m.n_compressed(319, 64, 256) == 0)
 
 
-PINS = [_pin_stacked_svd, _pin_no_truncation, _pin_rope, _pin_attention, _pin_schedule]
+def _pin_stale_two_folds(m):
+    """Stale coordinates after two untruncated folds: old rows keep their first-fold coordinates
+    against the new basis' first columns, new rows come back exactly (library SVDs)."""
+    d, b = 16, 4
+    X = _stream(d, d, 31)[:2 * b]
+    unit = m.OracleUnit(d, d, b, 0, rotate=False)
+    unit.append(X[:b])
+    B1 = unit.B.copy()
+    k1 = B1.shape[1]
+    unit.append(X[b:])
+    V2 = np.linalg.svd(X, full_matrices=False)[2][:2 * b].T
+    for c in range(k1):
+        if V2[:, c] @ B1[:, c] < 0:
+            V2[:, c] = -V2[:, c]
+    rec = unit.reconstruct()
+    return (np.allclose(rec[:b], (X[:b] @ B1) @ V2[:, :k1].T, atol=1e-10)
+            and np.allclose(rec[b:], X[b:], atol=1e-10))
+
+
+def _pin_fixed_basis(m):
+    """Fixed basis: after the folds that fill the rank budget, blocks are projected onto the
+    rank-r right singular subspace of the rows folded so far (library SVD)."""
+    d, r, b = 16, 6, 4
+    X = _stream(40, d, 41)
+    unit = m.OracleUnit(d, r, b, 0, fixed_basis=True)
+    unit.append(X)
+    Vt = np.linalg.svd(X[:8], full_matrices=False)[2][:r]
+    P = Vt.T @ Vt
+    return unit.n == 40 and np.allclose(unit.reconstruct()[8:], X[8:] @ P, atol=1e-10)
+
+
+PINS = [_pin_stacked_svd, _pin_no_truncation, _pin_rope, _pin_attention, _pin_schedule,
+        _pin_stale_two_folds, _pin_fixed_basis]
 
 MUTANTS = {
     "new-row identity block negated": ("Ublk[n:, k:] = np.eye(b)", "Ublk[n:, k:] = -np.eye(b)"),
@@ -94,6 +126,16 @@ MUTANTS = {
                                 "theta ** (-1.0 * np.arange(h, dtype=np.float64) / d)"),
     "softmax scale 1/d": ("/ math.sqrt(q.size)", "/ q.size"),
     "fold one row early": ("max(0, t - window)", "max(0, t - window + 1)"),
+    "stale: new rows coded in the old basis": (
+        "self.C_stale = np.vstack([C, F @ B_new])",
+        "self.C_stale = np.vstack([C, np.hstack([F @ self.B, "
+        "np.zeros((F.shape[0], kp - k_old))])])"),
+    "stale: old coordinates in the wrong columns": ("C[:, :m] = self.C_stale[:, :m]",
+                                                    "C[:, kp - m:] = self.C_stale[:, :m]"),
+    "fixed basis: one adapting fold too few": ("self.adapt_folds = -(-min(rank, d) // block)",
+                                               "self.adapt_folds = min(rank, d) // block"),
+    "fixed basis: frozen one fold late": ("self.folds >= self.adapt_folds",
+                                          "self.folds > self.adapt_folds"),
 }
 
 
