@@ -78,6 +78,12 @@ typedef struct {
                           /*    every decode sees exactly the state of mode 0. Call            */
                           /*    iskv_join() before ending a stream capture that contains       */
                           /*    appends.                                                       */
+    int fixed_basis;      /* 1: fixed-basis ablation ("Ablation Study", bases kept fixed): the   */
+                          /*    regular update runs for the first ceil(min(r, d) / block) folds */
+                          /*    of a path (they fill its rank budget); after that the path's   */
+                          /*    basis and Sigma freeze and each later block is stored as its   */
+                          /*    coordinates F B in the frozen basis (old coordinates untouched). */
+                          /*    0: iS-KV. Cannot be combined with rotate_history = 0.           */
 } iskv_config;
 
 /*

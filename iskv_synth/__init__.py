@@ -37,6 +37,7 @@ __all__ = [
     "queries",
     "workload_rows",
     "device_rows",
+    "device_rows_batch",
 ]
 
 
@@ -206,3 +207,36 @@ def device_rows(wl: Workload, seq: int, layer: int, head: int, kv: int, T: int |
     if wl.channel_sigma:
         X = X * torch.exp(wl.channel_sigma * torch.randn(d, generator=gen, device=device))
     return X.to(torch.bfloat16 if wl.kv_dtype == "bf16" else torch.float32)
+
+
+def device_rows_batch(wl: Workload, seqs, layer: int, heads, kv: int, T: int | None = None,
+                      device="cuda"):
+    """:func:`device_rows` for several units at once: a ``[len(seqs)][len(heads)][T][d]`` tensor
+    in the workload's dtype, drawn with one generator per (layer, path) and batched QRs.
+
+    Same recipe as :func:`kv_rows` (orthonormal ``G``, orthogonal ``H``, spectrum ``i^-a`` with each
+    unit's own exponent, noise 0.01, lognormal channel scales), a different random stream again.
+    """
+    import torch
+    T = wl.tokens if T is None else T
+    d = wl.head_dim
+    seqs, heads = list(seqs), list(heads)
+    n = len(seqs) * len(heads)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(unit_seed(wl.cfg_id, seqs[0], layer, heads[0], kv) * 7919 + 13)
+    a = torch.tensor([_decay(wl, unit_seed(wl.cfg_id, s, layer, h, kv), kv)
+                      for s in seqs for h in heads], device=device, dtype=torch.float32)
+    i = torch.arange(1, d + 1, device=device, dtype=torch.float32)
+    s_ = i[None, :] ** (-a[:, None])                                   # [n][d]
+    out = torch.empty((n, T, d), device=device,
+                      dtype=torch.bfloat16 if wl.kv_dtype == "bf16" else torch.float32)
+    for u in range(n):
+        g = torch.randn(T, d, generator=gen, device=device, dtype=torch.float32)
+        h = torch.randn(d, d, generator=gen, device=device, dtype=torch.float32)
+        G = torch.linalg.qr(g)[0]
+        H = torch.linalg.qr(h)[0]
+        X = (G * s_[u]) @ H.T + 0.01 * torch.randn(T, d, generator=gen, device=device)
+        if wl.channel_sigma:
+            X = X * torch.exp(wl.channel_sigma * torch.randn(d, generator=gen, device=device))
+        out[u] = X.to(out.dtype)
+    return out.view(len(seqs), len(heads), T, d)

@@ -55,6 +55,7 @@ class iskv_config(ctypes.Structure):
         ("rope_theta", ctypes.c_double),
         ("rotate_history", ctypes.c_int),
         ("lookahead_folds", ctypes.c_int),
+        ("fixed_basis", ctypes.c_int),
     ]
 
 

@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
     int *sSel = reinterpret_cast<int *>(smem + OFF_INT);
     float *stage = sB;                    // Jacobi staging overlays B and C
 
-    const FoldPath P = blockIdx.y ? a.path[1] : a.path[0];
+    const FoldPath P = (a.path_lo + (int)blockIdx.y) ? a.path[1] : a.path[0];
     const int unit = a.unit0 + blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = P.k, r = P.r, p = P.p, kp = P.kp, b = a.b;
@@ -906,7 +906,7 @@ constexpr int ROT_THREADS = 256;
 
 __global__ void __launch_bounds__(ROT_THREADS) rotate_kernel(RotArgs a) {
     extern __shared__ float smem[];
-    const RotPath P = blockIdx.z ? a.path[1] : a.path[0];
+    const RotPath P = (a.path_lo + (int)blockIdx.z) ? a.path[1] : a.path[0];
     const int unit = a.unit0 + blockIdx.y;
     const long long row0 = (long long)blockIdx.x * ROT_ROWS;
     if (row0 >= a.n_old) return;
@@ -941,23 +941,24 @@ __global__ void __launch_bounds__(ROT_THREADS) rotate_kernel(RotArgs a) {
 }
 
 cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s) {
+    if (a.path_hi <= a.path_lo || n_units <= 0) return cudaSuccess;
     static size_t attr[64] = {0};
     const size_t smem = fold_smem_bytes();
     const cudaError_t e = ensure_smem((const void *)fold_core_kernel, smem, attr);
     if (e != cudaSuccess) return e;
-    fold_core_kernel<<<dim3(n_units, 2), FT, smem, s>>>(a);
+    fold_core_kernel<<<dim3(n_units, a.path_hi - a.path_lo), FT, smem, s>>>(a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s) {
-    if (a.n_old <= 0) return cudaSuccess;
+    if (a.n_old <= 0 || a.path_hi <= a.path_lo || n_units <= 0) return cudaSuccess;
     const int rmax = a.path[0].r > a.path[1].r ? a.path[0].r : a.path[1].r;
     const size_t smem = (size_t)(rmax * rmax + ROT_ROWS * (rmax + 1)) * sizeof(float);
     static size_t attr[64] = {0};
     const cudaError_t e = ensure_smem((const void *)rotate_kernel, smem, attr);
     if (e != cudaSuccess) return e;
     const unsigned gx = (unsigned)((a.n_old + ROT_ROWS - 1) / ROT_ROWS);
-    rotate_kernel<<<dim3(gx, n_units, 2), ROT_THREADS, smem, s>>>(a);
+    rotate_kernel<<<dim3(gx, n_units, a.path_hi - a.path_lo), ROT_THREADS, smem, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(RF_THREADS) rfactor_kernel(RFactorArgs a) {
     extern __shared__ float rsm[];
     float *M = rsm;                              // [128 columns][RF_LDM]: rows 0..127 = R, 128.. = chunk
     float *sTau = rsm + D * RF_LDM;
-    const RFactorPath P = blockIdx.y ? a.path[1] : a.path[0];
+    const RFactorPath P = (a.path_lo + (int)blockIdx.y) ? a.path[1] : a.path[0];
     const int unit = a.unit0 + blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int FW = RF_THREADS / 32;
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(RF_THREADS) rfactor_kernel(RFactorArgs a) {
 // One CTA per (128-row chunk, unit, path): C[n_c + i] = F[i] B+ for the block's real rows.
 __global__ void __launch_bounds__(RF_THREADS) newrows_kernel(NewRowsArgs a) {
     extern __shared__ float nsm[];
-    const NewRowsPath P = blockIdx.z ? a.path[1] : a.path[0];
+    const NewRowsPath P = (a.path_lo + (int)blockIdx.z) ? a.path[1] : a.path[0];
     const int unit = a.unit0 + blockIdx.y;
     const int r = P.r, kp = P.kp, ldb = kp | 1;
     float *sB = nsm;                                 // B+ [D][ldb]
@@ -169,21 +169,23 @@ __global__ void __launch_bounds__(RF_THREADS) newrows_kernel(NewRowsArgs a) {
 size_t rfactor_smem_bytes() { return ((size_t)D * RF_LDM + D) * sizeof(float); }
 
 cudaError_t launch_rfactor(const RFactorArgs &a, int n_units, cudaStream_t s) {
+    if (a.path_hi <= a.path_lo || n_units <= 0) return cudaSuccess;
     static size_t attr[64] = {0};
     const cudaError_t e = ensure_smem((const void *)rfactor_kernel, rfactor_smem_bytes(), attr);
     if (e != cudaSuccess) return e;
-    rfactor_kernel<<<dim3(n_units, 2), RF_THREADS, rfactor_smem_bytes(), s>>>(a);
+    rfactor_kernel<<<dim3(n_units, a.path_hi - a.path_lo), RF_THREADS, rfactor_smem_bytes(), s>>>(a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_newrows(const NewRowsArgs &a, int n_units, cudaStream_t s) {
+    if (a.path_hi <= a.path_lo || n_units <= 0) return cudaSuccess;
     const int kpmax = a.path[0].kp > a.path[1].kp ? a.path[0].kp : a.path[1].kp;
     const size_t smem = ((size_t)D * (kpmax | 1) + 32 * (D + 1)) * sizeof(float);
     static size_t attr[64] = {0};
     const cudaError_t e = ensure_smem((const void *)newrows_kernel, smem, attr);
     if (e != cudaSuccess) return e;
     const int chunks = (a.b + DEC_TILE - 1) / DEC_TILE;
-    newrows_kernel<<<dim3(chunks, n_units, 2), RF_THREADS, smem, s>>>(a);
+    newrows_kernel<<<dim3(chunks, n_units, a.path_hi - a.path_lo), RF_THREADS, smem, s>>>(a);
     return cudaGetLastError();
 }
 

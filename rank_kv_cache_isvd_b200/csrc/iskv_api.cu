@@ -145,6 +145,14 @@ float *htop_buf(const iskv_handle *h, int x, int i) {
     const size_t r = (size_t)rank_of(h, x);
     return h->htop[x] + (size_t)i * h->U * r * r;
 }
+// Fixed-basis mode: fold j of path x only stores the block's coordinates in the frozen basis once
+// the first ceil(min(r, d) / b) folds (which fill the rank budget) have run.
+bool frozen(const iskv_handle *h, int x, long long j) {
+    if (!h->cfg.fixed_basis) return false;
+    const int r = rank_of(h, x) < D ? rank_of(h, x) : D;
+    return j >= (r + h->cfg.block - 1) / h->cfg.block;
+}
+
 // buffer of the basis / Sigma produced by the last applied fold
 int current_buffer(const iskv_handle *h, int layer) {
     return (int)((h->nc[layer] / h->cfg.block) % h->NB);
@@ -161,12 +169,17 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
     // the new rows' coordinates go to rows j*b .. j*b+b-1, which must lie within n_max
     if ((j + 1) * c.block > h->n_max) return ISKV_ERR_CAPACITY;
     const int bi = (int)(j % h->NB), bo = (int)((j + 1) % h->NB);
+    // paths that run the regular update (a contiguous range: frozen paths are a prefix or suffix)
+    const bool fz[2] = {frozen(h, 0, j), frozen(h, 1, j)};
+    const int plo = fz[0] ? 1 : 0, phi = fz[1] ? 1 : 2;
     FoldArgs fa;
     memset(&fa, 0, sizeof(fa));
+    fa.path_lo = plo;
+    fa.path_hi = phi > plo ? phi : plo;
     for (int x = 0; x < 2; ++x) {
         const int r = rank_of(h, x);
         const int k = h->kf[x][l0];
-        const int p = c.block < D - k ? c.block : D - k;
+        const int p = fz[x] ? 0 : (c.block < D - k ? c.block : D - k);
         const int kp = r < k + p ? r : k + p;
         FoldPath &fp = fa.path[x];
         fp.ring = h->ring[x];
@@ -191,6 +204,24 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
     fa.kv_dtype = c.kv_dtype;
     fa.status = h->status;
     fa.stats = h->stats;
+    // coordinates of the block's real rows in the new basis (large blocks) or, for frozen paths,
+    // in the frozen basis
+    NewRowsArgs nr;
+    memset(&nr, 0, sizeof(nr));
+    for (int x = 0; x < 2; ++x) {
+        nr.path[x].ring = h->ring[x];
+        nr.path[x].basis = fz[x] ? fa.path[x].basis_in : fa.path[x].basis_out;
+        nr.path[x].coords = h->coords[x];
+        nr.path[x].r = fa.path[x].r;
+        nr.path[x].kp = fa.path[x].kp;
+    }
+    nr.unit0 = fa.unit0;
+    nr.slot0 = fa.slot0;
+    nr.R = h->R;
+    nr.b = c.block;
+    nr.kv_dtype = c.kv_dtype;
+    nr.n_c = nc;
+    nr.n_max = h->n_max;
     if (c.block > BMAX) {
         // large block: fold the 128-row triangular factor of the block (same Sigma+, H and basis),
         // then the coordinates of the block's real rows
@@ -206,6 +237,8 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
         rf.R = h->R;
         rf.b = c.block;
         rf.kv_dtype = c.kv_dtype;
+        rf.path_lo = fa.path_lo;
+        rf.path_hi = fa.path_hi;
         if (launch_rfactor(rf, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
         fa.slot0 = 0;
         fa.R = DEC_TILE;
@@ -213,27 +246,29 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
         fa.kv_dtype = ISKV_F32;
         fa.skip_new_rows = 1;
         if (launch_fold(fa, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
-        NewRowsArgs nr;
-        memset(&nr, 0, sizeof(nr));
-        for (int x = 0; x < 2; ++x) {
-            nr.path[x].ring = h->ring[x];
-            nr.path[x].basis = fa.path[x].basis_out;
-            nr.path[x].coords = h->coords[x];
-            nr.path[x].r = fa.path[x].r;
-            nr.path[x].kp = fa.path[x].kp;
-        }
-        nr.unit0 = rf.unit0;
-        nr.slot0 = rf.slot0;
-        nr.R = h->R;
-        nr.b = c.block;
-        nr.kv_dtype = c.kv_dtype;
-        nr.n_c = nc;
-        nr.n_max = h->n_max;
+        nr.path_lo = 0;
+        nr.path_hi = 2;
         if (launch_newrows(nr, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
-        h->launches += 3;
+        h->launches += (fa.path_hi > fa.path_lo ? 2 : 0) + 1;
     } else {
         if (launch_fold(fa, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
-        h->launches += 1;
+        h->launches += fa.path_hi > fa.path_lo ? 1 : 0;
+        if (fz[0] || fz[1]) {
+            nr.path_lo = fz[0] ? 0 : 1;
+            nr.path_hi = fz[1] ? 2 : 1;
+            if (launch_newrows(nr, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+            h->launches += 1;
+        }
+    }
+    // frozen paths carry their basis and Sigma over to the next fold's buffer
+    for (int x = 0; x < 2; ++x) {
+        if (!fz[x]) continue;
+        const size_t r = (size_t)rank_of(h, x), u0 = (size_t)l0 * h->UL, nu = (size_t)nl * h->UL;
+        if (cudaMemcpyAsync(basis_buf(h, x, bo) + u0 * D * r, basis_buf(h, x, bi) + u0 * D * r,
+                            nu * D * r * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(sigma_buf(h, x, bo) + u0 * r, sigma_buf(h, x, bi) + u0 * r,
+                            nu * r * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+            return ISKV_ERR_CUDA;
     }
     for (int l = l0; l < l0 + nl; ++l) {
         int *f = fold_ranks(h, l, j);
@@ -266,9 +301,13 @@ int apply_fold(iskv_handle *h, int l0, int nl, cudaStream_t s) {
     }
     const int *f = fold_ranks(h, l0, j);
     const long long nc = h->nc[l0];
-    if (nc > 0) {
+    // frozen paths (fixed-basis mode) keep their old coordinates: nothing to rotate
+    const bool fz[2] = {frozen(h, 0, j), frozen(h, 1, j)};
+    if (nc > 0 && !(fz[0] && fz[1])) {
         RotArgs ra;
         memset(&ra, 0, sizeof(ra));
+        ra.path_lo = fz[0] ? 1 : 0;
+        ra.path_hi = fz[1] ? 1 : 2;
         for (int x = 0; x < 2; ++x) {
             RotPath &rp = ra.path[x];
             rp.coords = h->coords[x];
@@ -369,7 +408,7 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         c.n_q_heads % c.n_kv_heads != 0 || c.n_q_heads / c.n_kv_heads > GMAX || c.head_dim != D ||
         c.rank_k < 1 || c.rank_k > D || c.rank_v < 1 || c.rank_v > D || c.block < 1 ||
         c.window < 0 || c.max_tokens < 1 || (c.kv_dtype != ISKV_BF16 && c.kv_dtype != ISKV_F32) ||
-        (c.rope && !(c.rope_theta > 0.0)))
+        (c.rope && !(c.rope_theta > 0.0)) || (c.fixed_basis && !c.rotate_history))
         return ISKV_ERR_INVALID_ARG;
     if (c.block > BMAX_LARGE) return ISKV_ERR_UNSUPPORTED;
     iskv_handle *h = new (std::nothrow) iskv_handle();

@@ -44,6 +44,7 @@ struct FoldArgs {
     int *status;
     unsigned long long *stats;  // [0] max sweeps, [1] total sweeps, [2] cores solved
     int skip_new_rows;      // 1: leave the new rows' coordinates to newrows_kernel (large blocks)
+    int path_lo, path_hi;   // paths folded: path_lo .. path_hi - 1 (0 = keys, 1 = values)
 };
 
 // ---- large blocks (b > BMAX): triangular factor of the block, then the real rows' coordinates -
@@ -54,6 +55,7 @@ struct RFactorPath {
 struct RFactorArgs {
     RFactorPath path[2];
     int unit0, slot0, R, b, kv_dtype;
+    int path_lo, path_hi;   // paths processed: path_lo .. path_hi - 1
 };
 struct NewRowsPath {
     const void *ring;       // [units][R][D] kv dtype
@@ -65,6 +67,7 @@ struct NewRowsArgs {
     NewRowsPath path[2];
     int unit0, slot0, R, b, kv_dtype;
     long long n_c, n_max;
+    int path_lo, path_hi;   // paths processed: path_lo .. path_hi - 1
 };
 
 // ---- history rotation C[0:n] <- C[0:n] H_top (or stale zero-padding) ---------------------------
@@ -79,6 +82,7 @@ struct RotArgs {
     long long n_old;        // rows to rotate
     long long n_max;
     int stale;              // 1: keep old coordinates (zero columns k..kp-1)
+    int path_lo, path_hi;   // paths rotated: path_lo .. path_hi - 1
 };
 
 // ---- window append ----------------------------------------------------------------------------

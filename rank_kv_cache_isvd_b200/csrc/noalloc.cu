@@ -17,7 +17,8 @@ namespace {
 // it until exit. Shared by all calls: overlapping calls on the GPU race.
 static __device__ __align__(256) float g_noalloc_scratch[ISKV_NOALLOC_SCRATCH_FLOATS];
 
-constexpr int kMaxDevices = 128;
+// Same device limit as the per-device function attributes of the decode launchers (64).
+constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 float *g_scratch_addr[kMaxDevices] = {nullptr};
 
@@ -65,9 +66,13 @@ extern "C" int iskv_decode_attn_noalloc(const iskv_decode_view *v, const float *
     const long long wsplits = (v->t - v->n_c + DEC_TILE - 1) / DEC_TILE + (v->n_c > 0 ? 1 : 0);
     if ((long long)units * wsplits * G * (2 + D) > ISKV_NOALLOC_SCRATCH_FLOATS)
         return ISKV_ERR_CAPACITY;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess) return ISKV_ERR_CUDA;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ISKV_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms < 1) {
+        cudaGetLastError();
+        return ISKV_ERR_CUDA;
+    }
 
     DecodeArgs da;
     memset(&da, 0, sizeof(da));

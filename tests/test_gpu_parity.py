@@ -7,6 +7,7 @@ attention output relative error <= 2e-3 per q-head (max over heads); window rows
 compressed-row counts and ranks bit-exact.
 """
 import dataclasses
+import math
 
 import numpy as np
 import pytest
@@ -40,10 +41,10 @@ def make_cache(wl, **kw):
     return IsKVCache(**args)
 
 
-def make_oracle(wl, rotate=True):
+def make_oracle(wl, rotate=True, fixed_basis=False):
     return OracleCache(wl.batch, wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim,
                        wl.rank_k, wl.rank_v, wl.block, wl.window, rope=wl.rope,
-                       rope_theta=wl.rope_theta, rotate=rotate)
+                       rope_theta=wl.rope_theta, rotate=rotate, fixed_basis=fixed_basis)
 
 
 def sub(wl, **kw):
@@ -202,6 +203,35 @@ def test_stale_coordinates_mode_matches_oracle():
         assert rel_err(rec[:n], ref[:n]) <= 1e-3
         drift = rel_err(ref[:n], sync.unit(0, 0, 0, x).reconstruct()[:n])
         assert drift > 1e-2          # stale coordinates do drift
+
+
+@pytest.mark.parametrize("block,window,rank_k,rank_v,tokens", [
+    (64, 256, 32, 48, 900),        # both paths freeze after the first fold
+    (32, 64, 32, 48, 700),         # keys freeze after one fold, values adapt for two
+    (256, 128, 64, 96, 1500),      # blocks above 128 rows (triangular-factor folds)
+])
+def test_fixed_basis_mode_matches_oracle(block, window, rank_k, rank_v, tokens):
+    """Fixed-basis ablation: after the folds that fill the rank budget, blocks are stored as their
+    coordinates in the frozen basis. Reconstructions, ranks and decode match the oracle's variant;
+    the frozen basis is the one the adapting folds produced."""
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=tokens, block=block, window=window,
+             rank_k=rank_k, rank_v=rank_v)
+    kd, kv, vd, vv = workload_arrays(wl, variant="gapped")
+    cache = make_cache(wl, fixed_basis=True, lookahead_folds=True)
+    orc = make_oracle(wl, fixed_basis=True)
+    append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], 0, wl.tokens)
+    for h in range(2):
+        for x in (0, 1):
+            u = orc.unit(0, 0, h, x)
+            C, B, S, k, n = cache.factors(0, 0, h, x)
+            assert k == u.k and n == u.n and n > 2 * block
+            rec = cache.reconstruct(0, x).cpu().numpy()[0, h]
+            assert rel_err(rec[:n], u.reconstruct()[:n]) <= 1e-3
+            assert projector_err(B.cpu().numpy()[:, :k], u.B) <= PROJ_TOL
+    q = syn.queries(41, (1, 8, 128))
+    out = cache.decode(0, torch.from_numpy(q).cuda()).cpu().numpy()
+    assert max_head_rel_err(out, orc.decode(0, q.astype(np.float64))) <= ATTN_TOL
+    assert cache.status() == 0
 
 
 def test_all_layers_batched_equals_per_layer():
@@ -400,18 +430,16 @@ def test_long_context_layer_sampled_units():
     out = cache.decode(0, q)
     assert cache.status() == 0 and bool(torch.isfinite(out).all())
     assert cache.tokens(0) == T
+    units = []
     for sq, h in ((0, 0), (3, 5), (7, 7)):
-        orc = OracleCache(1, 1, 1, G, 128, wl.rank_k, wl.rank_v, wl.block, wl.window, rope=True,
-                          rope_theta=wl.rope_theta)
-        kv = K[sq, h].float().cpu().numpy().astype(np.float64)[None, None]
-        vv = V[sq, h].float().cpu().numpy().astype(np.float64)[None, None]
-        orc.append(0, kv, vv)
-        qs = q[sq, h * G:(h + 1) * G].cpu().numpy().astype(np.float64)[None]
-        ref = orc.decode(0, qs)
-        got = out[sq, h * G:(h + 1) * G].cpu().numpy()[None]
-        err = max_head_rel_err(got, ref)
+        err, (orc,) = _sampled_unit_check(wl, q, out, [(sq, h, K[sq, h], V[sq, h])])
         print(f"\nunit (seq {sq}, kv-head {h}): attention rel err {err:.3e}")
         assert err <= ATTN_TOL
+        units.append((sq, h, K[sq, h], V[sq, h], orc))
+    # sharp attention (logit 20) on compressed rows early, mid and late, and a window row
+    sa, sb = _sharp_checks(cache, wl, 0, units, [1000, 20000, 32500, 32700], 999)
+    print(f"sharp: {sa:.3e} vs device state, {sb:.3e} vs oracle stream")
+    assert sa <= ATTN_TOL and sb <= ATTN_TOL
     cache.close()
 
 
@@ -527,20 +555,79 @@ def test_large_blocks_fold_through_their_triangular_factor(variant):
     assert cache.status() == 0
 
 
+def _unit_oracle(wl, K, V):
+    """Float64 oracle of one (sequence, kv-head) unit fed the unit's rows as they are on the device
+    (bf16 values, exact in float64)."""
+    orc = OracleCache(1, 1, 1, wl.group, 128, wl.rank_k, wl.rank_v, wl.block, wl.window,
+                      rope=True, rope_theta=wl.rope_theta)
+    orc.append(0, K.float().cpu().numpy().astype(np.float64)[None, None],
+               V.float().cpu().numpy().astype(np.float64)[None, None])
+    return orc
+
+
 def _sampled_unit_check(wl, q, out, units):
     """Oracle run on single (sequence, kv-head) units of a full-size cache, compared on their
-    q-heads; rows come back from the device (bf16 values, exact in float64)."""
+    q-heads. Returns (worst error, the units' oracles)."""
     G = wl.group
-    worst = 0.0
+    worst, oracles = 0.0, []
     for sq, h, K, V in units:
-        orc = OracleCache(1, 1, 1, G, 128, wl.rank_k, wl.rank_v, wl.block, wl.window, rope=True,
-                          rope_theta=wl.rope_theta)
-        orc.append(0, K.float().cpu().numpy().astype(np.float64)[None, None],
-                   V.float().cpu().numpy().astype(np.float64)[None, None])
+        orc = _unit_oracle(wl, K, V)
         qs = q[sq, h * G:(h + 1) * G].cpu().numpy().astype(np.float64)[None]
         err = max_head_rel_err(out[sq, h * G:(h + 1) * G].cpu().numpy()[None], orc.decode(0, qs))
         worst = max(worst, err)
-    return worst
+        oracles.append(orc)
+    return worst, oracles
+
+
+def _sharp(keys_rot, positions, logit=20.0):
+    """Queries aligned with the (rotated) keys at `positions`, scaled so that each one's own logit
+    q.k / sqrt(d) is `logit`: sharp attention that peaks on those positions."""
+    return np.stack([keys_rot[p] * (logit * math.sqrt(128) / float(keys_rot[p] @ keys_rot[p]))
+                     for p in positions])
+
+
+def _attention_over_device_state(cache, wl, layer, seq, head, K, V, qs):
+    """Float64 attention (the oracle's RoPE and softmax) over the cache's own state: compressed rows
+    C B^T from the device factors promoted to float64, window rows exact. Isolates the decode
+    kernels from the fold trajectory (one-step parity of the decode)."""
+    from oracle import attention, rope
+    t = cache.tokens(layer)
+    rows = []
+    for x, X in ((0, K), (1, V)):
+        C, B, _, k, n = cache.factors(layer, seq, head, x)
+        C = C.cpu().numpy().astype(np.float64)[:, :k]
+        B = B.cpu().numpy().astype(np.float64)[:, :k]
+        ex = X[n:t].float().cpu().numpy().astype(np.float64)
+        rows.append(np.vstack([C @ B.T, ex]) if n else ex)
+    Kr = rope(rows[0], np.arange(t), wl.rope_theta)
+    return np.stack([attention(qg, Kr, rows[1]) for qg in qs]), Kr
+
+
+def _sharp_checks(cache, wl, layer, units, positions, rng_seed):
+    """Sharp-softmax decode parity on sampled units of a full-size cache. Every q-head of a sampled
+    unit gets a query aligned with one of `positions` (logit 20); the other units get random
+    queries. Compares each sampled q-head with (a) float64 attention over the device state and
+    (b) the unit's own float64 oracle stream. Returns the worst errors (a, b)."""
+    S, QH, G = wl.batch, wl.n_q_heads, wl.group
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(rng_seed)
+    q = torch.randn((S, QH, 128), generator=gen, device="cuda")
+    refs = []
+    for sq, h, K, V, orc in units:
+        kref, _ = orc.keys_values(0, 0, 0)
+        qs = _sharp(kref, positions)
+        q[sq, h * G:(h + 1) * G] = torch.from_numpy(qs.astype(np.float32)).cuda()
+        refs.append(qs)
+    out = cache.decode(layer, q)
+    assert cache.status() == 0 and bool(torch.isfinite(out).all())
+    wa = wb = 0.0
+    for (sq, h, K, V, orc), qs in zip(units, refs):
+        qs32 = q[sq, h * G:(h + 1) * G].cpu().numpy().astype(np.float64)
+        got = out[sq, h * G:(h + 1) * G].cpu().numpy()[None]
+        ref_a, _ = _attention_over_device_state(cache, wl, layer, sq, h, K, V, qs32)
+        wa = max(wa, max_head_rel_err(got, ref_a[None]))
+        wb = max(wb, max_head_rel_err(got, orc.decode(0, qs32[None])))
+    return wa, wb
 
 
 def test_32_layer_workload_full_size_sampled_units():
@@ -559,14 +646,20 @@ def test_32_layer_workload_full_size_sampled_units():
     cache.append(-1, K, V)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(2024)
-    worst = 0.0
+    worst, sa, sb = 0.0, 0.0, 0.0
     for l, h in ((0, 3), (31, 6)):
         q = torch.randn((S, wl.n_q_heads, 128), generator=gen, device="cuda")
         out = cache.decode(l, q)
         assert bool(torch.isfinite(out).all())
-        worst = max(worst, _sampled_unit_check(wl, q, out, [(0, h, K[l, 0, h], V[l, 0, h])]))
-    print(f"\n32-layer workload, sampled units: worst attention rel err {worst:.3e}")
-    assert worst <= ATTN_TOL
+        err, (orc,) = _sampled_unit_check(wl, q, out, [(0, h, K[l, 0, h], V[l, 0, h])])
+        worst = max(worst, err)
+        # sharp attention (logit 20) on compressed rows early, mid and late, and a window row
+        a, b = _sharp_checks(cache, wl, l, [(0, h, K[l, 0, h], V[l, 0, h], orc)],
+                             [5, 9000, 16250, 16300], 77 + l)
+        sa, sb = max(sa, a), max(sb, b)
+    print(f"\n32-layer workload, sampled units: worst attention rel err {worst:.3e}; sharp: "
+          f"{sa:.3e} vs device state, {sb:.3e} vs oracle stream")
+    assert worst <= ATTN_TOL and sa <= ATTN_TOL and sb <= ATTN_TOL
     assert cache.status() == 0
     cache.close()
 
@@ -590,7 +683,11 @@ def test_long_prefill_full_size_sampled_unit():
     q = torch.randn((S, wl.n_q_heads, 128), generator=gen, device="cuda")
     out = cache.decode(0, q)
     assert cache.status() == 0 and bool(torch.isfinite(out).all())
-    err = _sampled_unit_check(wl, q, out, [(2, 5, K[2, 5], V[2, 5])])
-    print(f"\nlong prefill, sampled unit: attention rel err {err:.3e}")
-    assert err <= ATTN_TOL
+    err, (orc,) = _sampled_unit_check(wl, q, out, [(2, 5, K[2, 5], V[2, 5])])
+    # sharp attention on compressed rows past 60K (n_c = 65024) and on a window row
+    sa, sb = _sharp_checks(cache, wl, 0, [(2, 5, K[2, 5], V[2, 5], orc)],
+                           [60001, 62500, 64999, 65300], 4343)
+    print(f"\nlong prefill, sampled unit: attention rel err {err:.3e}; sharp: {sa:.3e} vs "
+          f"device state, {sb:.3e} vs oracle stream")
+    assert err <= ATTN_TOL and sa <= ATTN_TOL and sb <= ATTN_TOL
     cache.close()

@@ -59,7 +59,7 @@ def _cfg(**kw):
 @pytest.mark.parametrize("bad", [
     dict(head_dim=64), dict(rank_k=0), dict(rank_v=129), dict(block=0), dict(window=-1),
     dict(n_q_heads=12), dict(n_q_heads=128), dict(batch=0), dict(max_tokens=0), dict(kv_dtype=7),
-    dict(rope=1, rope_theta=0.0), dict(n_layers=0),
+    dict(rope=1, rope_theta=0.0), dict(n_layers=0), dict(fixed_basis=1, rotate_history=0),
 ])
 def test_create_rejects_invalid_config(bad):
     code, h = iskv.iskv_create(_cfg(**bad))

@@ -45,7 +45,7 @@ def test_step_time_is_max_over_ranks_and_value_counts_all_ranks():
         assert p.exitcode == 0
     for rank, total, value in res:
         assert total == 180.0
-        assert value == pytest.approx(2 * bench.WL.tokens / (60.0 / 1e3))
+        assert value == pytest.approx(2 * bench.WL.batch * bench.TOK_PER_STEP / (60.0 / 1e3))
 
 
 def test_single_rank_needs_no_process_group():
