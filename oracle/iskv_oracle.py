@@ -36,6 +36,12 @@ Readings taken where the page is silent (each also stated at its definition):
 * the "stale coordinates" variant (``rotate=False``) updates ``Sigma`` and ``B`` exactly as above
   but keeps the old rows' coordinates ``U Sigma`` unrotated (zero-padded or truncated to the new
   rank) and reconstructs them against the new basis; new rows get ``F B+``;
+* bf16 coordinates (``coord_bf16=True``; "Reconstruction and Storage" leaves the bytes per factor
+  scalar beta_f open and the "Conclusion" names quantisation as the next step): the stored
+  coordinates ``C = U Sigma`` (the ``k n`` scalars that grow with the history) are rounded to
+  bf16 (nearest even, through float32, as a kernel rounding its fp32 results) after every fold,
+  and the next fold starts from the rounded values; ``B`` and ``Sigma`` stay unrounded, because
+  the update's core assumes an orthonormal ``B``;
 * the "fixed basis" variant (``fixed_basis=True``, section "Ablation Study": bases kept fixed)
   runs the regular update for the first ``ceil(min(r, d) / block)`` blocks, which fill the rank
   budget, and then freezes ``B`` and ``Sigma``: every later block is stored as its coordinates
@@ -61,6 +67,7 @@ __all__ = [
     "OracleCache",
     "rope",
     "attention",
+    "round_bf16",
 ]
 
 
@@ -75,6 +82,15 @@ def svd_r(X: np.ndarray, r: int):
     U, s, Vt = np.linalg.svd(np.asarray(X, dtype=np.float64), full_matrices=False)
     k = min(r, X.shape[0], X.shape[1])
     return U[:, :k], s[:k], Vt[:k].T
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Values rounded to bfloat16 (8-bit significand, round to nearest even) through float32, as
+    a kernel that computes in fp32 and stores bf16 rounds them; returned as float64."""
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(f.shape)
 
 
 def n_compressed(t: int, block: int, window: int) -> int:
@@ -178,9 +194,9 @@ class OracleUnit:
     """
 
     def __init__(self, d: int, rank: int, block: int, window: int, rotate: bool = True,
-                 fixed_basis: bool = False):
+                 fixed_basis: bool = False, coord_bf16: bool = False):
         self.d, self.rank, self.block, self.window, self.rotate = d, rank, block, window, rotate
-        self.fixed_basis = fixed_basis
+        self.fixed_basis, self.coord_bf16 = fixed_basis, coord_bf16
         # folds that run the regular update before a fixed basis freezes (fill the rank budget)
         self.adapt_folds = -(-min(rank, d) // block)
         self.U = np.zeros((0, 0))
@@ -203,7 +219,7 @@ class OracleUnit:
 
     def coords(self) -> np.ndarray:
         """Stored history coordinates ``U Sigma`` (``n x k``)."""
-        if not self.rotate or self.fixed_basis:
+        if not self.rotate or self.fixed_basis or self.coord_bf16:
             return self.C_stale
         return self.U * self.sigma
 
@@ -213,6 +229,12 @@ class OracleUnit:
         iS-KV summary, section "Reconstruction and Storage" (storage formula, per path).
         """
         return self.k * (self.n + self.d + 1) + self.d * len(self._exact)
+
+    def storage_bytes(self, beta_e: int) -> int:
+        """Persistent bytes of this path: the storage formula with bf16 (2 bytes) or fp32 (4 bytes)
+        coordinates, fp32 basis and Sigma, and ``beta_e`` bytes per exact scalar."""
+        beta_c = 2 if self.coord_bf16 else 4
+        return beta_c * self.k * self.n + 4 * self.k * (self.d + 1) + beta_e * self.d * len(self._exact)
 
     # -- updates -------------------------------------------------------------------------------
     def append(self, rows: np.ndarray) -> int:
@@ -231,9 +253,27 @@ class OracleUnit:
 
     def _fold(self, F: np.ndarray) -> None:
         k_old = self.k
+        rnd = round_bf16 if self.coord_bf16 else (lambda x: x)
         if self.fixed_basis and self.folds >= self.adapt_folds:
             # frozen basis: the block's rows are stored as their coordinates in it
-            self.C_stale = np.vstack([self.C_stale, F @ self.B])
+            self.C_stale = np.vstack([self.C_stale, rnd(F @ self.B)])
+            self.n += F.shape[0]
+            self.folds += 1
+            return
+        if self.coord_bf16:
+            # the update starts from the stored (rounded) coordinates; its result is rounded
+            C_new, s, B_new, _ = fold_from_coords(self.C_stale.reshape(self.n, k_old),
+                                                  self.sigma, self.B, F, self.rank)
+            if self.rotate:
+                self.C_stale = rnd(C_new)
+            else:
+                kp = s.size
+                C = np.zeros((self.n, kp))
+                m = min(k_old, kp)
+                C[:, :m] = self.C_stale[:, :m]
+                self.C_stale = np.vstack([C, rnd(F @ B_new)])
+            self.U = np.zeros((self.n + F.shape[0], s.size))      # not kept: C is the state
+            self.sigma, self.B = s, B_new
             self.n += F.shape[0]
             self.folds += 1
             return
@@ -289,11 +329,11 @@ class OracleCache:
     def __init__(self, batch: int, n_layers: int, n_kv_heads: int, n_q_heads: int,
                  head_dim: int, rank_k: int, rank_v: int, block: int, window: int,
                  rope: bool = False, rope_theta: float = 5e5, rotate: bool = True,
-                 fixed_basis: bool = False):
+                 fixed_basis: bool = False, coord_bf16: bool = False):
         self.batch, self.n_layers, self.n_kv, self.n_q = batch, n_layers, n_kv_heads, n_q_heads
         self.d, self.rope, self.theta = head_dim, rope, rope_theta
         self.units = [[[[OracleUnit(head_dim, rank_k if w == 0 else rank_v, block, window, rotate,
-                                    fixed_basis)
+                                    fixed_basis, coord_bf16)
                          for w in range(2)] for _ in range(n_kv_heads)] for _ in range(batch)]
                       for _ in range(n_layers)]
 

@@ -297,3 +297,72 @@ def test_fixed_basis_projects_later_blocks(d, r, b, w):
     sync = OracleUnit(d, r, b, w)
     sync.append(X)
     assert np.linalg.norm(sync.reconstruct()[:n] - X[:n]) < np.linalg.norm(rec[:n] - X[:n])
+
+
+# ---------------------------------------------------------------------------------------------
+# bf16 coordinates: every fold is the update of the stored (rounded) state, rounded again
+# ---------------------------------------------------------------------------------------------
+def _bf16_grid_ok(x):
+    """Every value has at most 8 significant bits (a bf16 number)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return bool(np.all(m * 256.0 == np.round(m * 256.0)))
+
+
+def test_round_bf16_is_nearest_even_on_the_bf16_grid():
+    from oracle import round_bf16
+    # exact values stay, halfway cases go to the even neighbour, others to the nearest
+    assert round_bf16(np.array([1.0, -2.5, 0.0]))[0] == 1.0
+    one_ulp = 2.0 ** -7                       # bf16 spacing in [1, 2)
+    half = 1.0 + one_ulp / 2                  # halfway between 1 and 1 + ulp: even is 1
+    assert round_bf16(np.array([half]))[0] == 1.0
+    assert round_bf16(np.array([1.0 + 1.5 * one_ulp]))[0] == 1.0 + 2 * one_ulp
+    assert round_bf16(np.array([1.0 + 0.6 * one_ulp]))[0] == 1.0 + one_ulp
+    x = np.random.default_rng(0).standard_normal(10000)
+    y = round_bf16(x)
+    assert _bf16_grid_ok(y)
+    assert np.max(np.abs(y - x) / np.abs(x)) <= 2.0 ** -8 * (1 + 1e-6)
+
+
+@pytest.mark.parametrize("d,r,b,w", [(16, 4, 3, 2), (16, 6, 8, 0), (32, 8, 16, 5)])
+def test_bf16_coordinates_closed_form_per_fold(d, r, b, w):
+    X = _stream(12 * b + w, d, 43 + d + r, decay=0.6, noise=0.02)
+    unit = OracleUnit(d, r, b, w, coord_bf16=True)
+    ref = OracleUnit(d, r, b, w)
+    t = 0
+    while unit.folds < 10:
+        C0, s0, B0, n0 = unit.coords().copy(), unit.sigma.copy(), unit.B.copy(), unit.n
+        step = (w + b) if unit.folds == 0 else b
+        unit.append(X[t:t + step])
+        ref.append(X[t:t + step])
+        t += step
+        F = X[n0:n0 + b]
+        # library SVD of the history's rows Sigma B^T stacked on the block gives Sigma+ and B+
+        M = np.vstack([s0[:, None] * B0.T, F]) if s0.size else F
+        _, sv, Vt = np.linalg.svd(M, full_matrices=False)
+        kp = unit.k
+        V = Vt[:kp].T
+        for c in range(kp):
+            # columns c < k follow the sign convention; new directions have no fixed sign
+            ref_col = B0[:, c] if c < s0.size else unit.B[:, c]
+            if V[:, c] @ ref_col < 0:
+                V[:, c] = -V[:, c]
+        np.testing.assert_allclose(unit.sigma, sv[:kp], rtol=1e-10, atol=1e-12)
+        gap = kp < sv.size and (sv[kp - 1] - sv[kp]) / sv[0] > 1e-3
+        if gap:
+            np.testing.assert_allclose(unit.B, V, atol=1e-8)
+        C = unit.coords()
+        assert _bf16_grid_ok(C)
+        # stored coordinates: old rows moved by H[:k] = B^T B+, new rows F B+, then rounded
+        if gap:
+            expect = np.vstack([C0 @ (B0.T @ V), F @ V]) if n0 else F @ V
+            from oracle import round_bf16
+            diff = np.abs(C - round_bf16(expect))
+            ulp = np.abs(round_bf16(expect)) * 2.0 ** -7 + 1e-30
+            assert np.all(diff <= ulp)                       # at most one bf16 step apart
+            assert np.mean(diff > 0) <= 1e-2                 # and equal almost everywhere
+    # the rounded cache stays close to the unrounded one (rounding is 2^-8 relative per value)
+    n = unit.n
+    rel = np.linalg.norm(unit.reconstruct()[:n] - ref.reconstruct()[:n]) / np.linalg.norm(X[:n])
+    assert rel <= 2e-2
+    assert unit.storage_bytes(2) == 2 * unit.k * n + 4 * unit.k * (d + 1) + 2 * d * (t - n)

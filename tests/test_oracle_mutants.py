@@ -110,8 +110,36 @@ def _pin_fixed_basis(m):
     return unit.n == 40 and np.allclose(unit.reconstruct()[8:], X[8:] @ P, atol=1e-10)
 
 
+def _pin_bf16_coordinates(m):
+    """bf16 coordinates: stored values lie on the bf16 grid and each fold's coordinates are the
+    rounded [C H[:k]; F B+] of the stored state (library SVD of [Sigma B^T; F])."""
+    d, r, b = 16, 5, 6
+    X = _stream(60, d, 47)
+    unit = m.OracleUnit(d, r, b, 0, coord_bf16=True)
+    unit.append(X[:b])
+    for f in range(1, 6):
+        C0, s0, B0 = unit.coords().copy(), unit.sigma.copy(), unit.B.copy()
+        F = X[f * b:(f + 1) * b]
+        unit.append(F)
+        _, sv, Vt = np.linalg.svd(np.vstack([s0[:, None] * B0.T, F]), full_matrices=False)
+        V = Vt[:unit.k].T
+        for c in range(unit.k):
+            if V[:, c] @ (B0[:, c] if c < s0.size else unit.B[:, c]) < 0:
+                V[:, c] = -V[:, c]
+        C = unit.coords()
+        mant = np.frexp(C)[0] * 256.0
+        if not np.all(mant == np.round(mant)):
+            return False
+        expect = np.vstack([C0 @ (B0.T @ V), F @ V])
+        # nearest rounding to 8 significant bits moves a value by at most half a step
+        if np.any(np.abs(C - expect) > 2.0 ** -8 * np.abs(expect) * (1 + 1e-4)
+                  + 1e-9 * np.abs(expect).max()):
+            return False
+    return True
+
+
 PINS = [_pin_stacked_svd, _pin_no_truncation, _pin_rope, _pin_attention, _pin_schedule,
-        _pin_stale_two_folds, _pin_fixed_basis]
+        _pin_stale_two_folds, _pin_fixed_basis, _pin_bf16_coordinates]
 
 MUTANTS = {
     "new-row identity block negated": ("Ublk[n:, k:] = np.eye(b)", "Ublk[n:, k:] = -np.eye(b)"),
@@ -130,12 +158,17 @@ MUTANTS = {
         "self.C_stale = np.vstack([C, F @ B_new])",
         "self.C_stale = np.vstack([C, np.hstack([F @ self.B, "
         "np.zeros((F.shape[0], kp - k_old))])])"),
-    "stale: old coordinates in the wrong columns": ("C[:, :m] = self.C_stale[:, :m]",
-                                                    "C[:, kp - m:] = self.C_stale[:, :m]"),
+    "stale: old coordinates in the wrong columns": (
+        "C[:, :m] = self.C_stale[:, :m]\n            self.C_stale = np.vstack([C, F @ B_new])",
+        "C[:, kp - m:] = self.C_stale[:, :m]\n            self.C_stale = np.vstack([C, F @ B_new])"),
     "fixed basis: one adapting fold too few": ("self.adapt_folds = -(-min(rank, d) // block)",
                                                "self.adapt_folds = min(rank, d) // block"),
     "fixed basis: frozen one fold late": ("self.folds >= self.adapt_folds",
                                           "self.folds > self.adapt_folds"),
+    "bf16: rotated coordinates left unrounded": ("                self.C_stale = rnd(C_new)",
+                                                 "                self.C_stale = C_new"),
+    "bf16: rounding to 7 significant bits": ("u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16\n    return (u.astype(np.uint32) << 16)",
+                                             "u = (u + 0xFFFF + ((u >> 17) & 1)) >> 17\n    return (u.astype(np.uint32) << 17)"),
 }
 
 
