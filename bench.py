@@ -78,6 +78,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true", help="headline line only")
+    p.add_argument("--coords", choices=["bf16", "f32"], default="bf16",
+                   help="storage of the coordinates C = U Sigma (bases and Sigma stay fp32)")
     p.add_argument("--profile-case", choices=["short", "long", "prefill"], nargs="?",
                    const="short",
                    help="run a short program for profiler captures instead of the bench: "
@@ -105,15 +107,16 @@ def ranks_after(wl, t: int):
     return k
 
 
-def decode_bytes(t: int, wl=None) -> int:
+def decode_bytes(t: int, wl=None, csz: int = 4) -> int:
     """Algorithmic bytes of one decode call at t tokens (all sequences and kv-heads of a layer):
-    fp32 coordinates of the compressed rows, bf16 window rows (K and V), fp32 bases, q and out."""
+    coordinates of the compressed rows (csz bytes each: 4 fp32, 2 bf16), window rows (K and V),
+    fp32 bases, q and out."""
     wl = WL if wl is None else wl
     n = wl.n_c(t)
     e = t - n
     kK, kV = ranks_after(wl, t) if n else (0, 0)
     esz = 2 if wl.kv_dtype == "bf16" else 4
-    per_unit = 4 * n * (kK + kV) + 2 * esz * e * D + 4 * D * (kK + kV) + 2 * 4 * wl.group * D
+    per_unit = csz * n * (kK + kV) + 2 * esz * e * D + 4 * D * (kK + kV) + 2 * 4 * wl.group * D
     return wl.batch * wl.n_kv_heads * per_unit
 
 
@@ -326,6 +329,10 @@ def workload_inputs(seq: int, wl=None):
     return kd, vd, q
 
 
+def _csz(args) -> int:
+    return 2 if getattr(args, "coords", "bf16") == "bf16" else 4
+
+
 def _cache(wl, n_layers=None, **kw):
     from rank_kv_cache_isvd_b200.cache import IsKVCache
     args = dict(batch=wl.batch, n_layers=wl.n_layers if n_layers is None else n_layers,
@@ -351,7 +358,7 @@ def headline(args, dev, rank: int, world: int, local_rank: int):
     seqs = range(rank * S, rank * S + S)           # every rank streams its own sequences
     s = torch.cuda.Stream(device=dev)
     sh = s.cuda_stream
-    cache = _cache(wl, lookahead_folds=True)
+    cache = _cache(wl, lookahead_folds=True, coord_bf16=args.coords == "bf16")
     h = cache.handle
     SK = torch.empty((n_stream, L, S, H, D), dtype=torch.bfloat16, device=dev)
     SV = torch.empty_like(SK)
@@ -406,6 +413,7 @@ def headline(args, dev, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize(dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     with Clocks(local_rank) as clk:
+        torch.cuda.nvtx.range_push("timed")          # marks the timed steps for profilers
         with torch.cuda.stream(s):
             ev[0].record(s)
             for k in range(args.steps):
@@ -413,6 +421,7 @@ def headline(args, dev, rank: int, world: int, local_rank: int):
                 pos += TOK_PER_STEP
                 ev[k + 1].record(s)
         s.synchronize()
+        torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier(device_ids=[local_rank])
@@ -435,7 +444,7 @@ def headline(args, dev, rank: int, world: int, local_rank: int):
         s.synchronize()
         dec.append(e0.elapsed_time(e1) / L)
     dec_ms = float(np.median(dec))
-    dec_bytes = decode_bytes(t_now)
+    dec_bytes = decode_bytes(t_now, csz=_csz(args))
 
     # ---- end to end through the C ABI with host buffers ------------------------------------------
     lo = pos
@@ -515,7 +524,7 @@ def llama_layer_stream(args, dev, flush):
     V = torch.from_numpy(vd.view(np.int16)).to(dev).view(torch.bfloat16)
     Q = torch.from_numpy(q).to(dev)
     OUT = torch.empty_like(Q)
-    cache = _cache(wl, lookahead_folds=True)
+    cache = _cache(wl, lookahead_folds=True, coord_bf16=args.coords == "bf16")
     h = cache.handle
     kb, vb, qb, ob = K.data_ptr(), V.data_ptr(), Q.data_ptr(), OUT.data_ptr()
     krow, qrow = H * D * 2, QH * D * 4
@@ -551,7 +560,7 @@ def llama_layer_stream(args, dev, flush):
     # fold throughput: all 4096 rows in one append (60 folds per path back to back)
     Kb = K[:, 0].transpose(0, 1).contiguous()[None]
     Vb = V[:, 0].transpose(0, 1).contiguous()[None]
-    fc = _cache(wl)
+    fc = _cache(wl, coord_bf16=args.coords == "bf16")
     with torch.cuda.stream(s):
         fc.append(0, Kb, Vb, sh)
     s.synchronize()
@@ -589,7 +598,7 @@ def all_layers_decode_step(args, dev, flush, steps: int = 5):
     import torch
     wl = WL_LAYERS
     L, S, H, T, QH = wl.n_layers, wl.batch, wl.n_kv_heads, wl.tokens, wl.n_q_heads
-    cache = _cache(wl)
+    cache = _cache(wl, coord_bf16=args.coords == "bf16")
     s = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(s):
         Kr = torch.empty((L, S, H, T, D), dtype=torch.bfloat16, device=dev)
@@ -631,7 +640,7 @@ def all_layers_decode_step(args, dev, flush, steps: int = 5):
     cache.close()
     hbm, _ = peaks()
     step_us = 1e3 * float(np.median(ms))
-    nbytes = L * decode_bytes(T, wl)
+    nbytes = L * decode_bytes(T, wl, csz=_csz(args))
     folds = wl.n_c(T) // wl.block
     flops = fold_flops(wl, T)
     return {
@@ -659,7 +668,7 @@ def long_prefill(args, dev, flush, calls: int = 5):
     import torch
     wl = WL_PREFILL
     S, H, T0, QH = wl.batch, wl.n_kv_heads, wl.prefill, wl.n_q_heads
-    cache = _cache(wl, n_layers=1)
+    cache = _cache(wl, n_layers=1, coord_bf16=args.coords == "bf16")
     s = torch.cuda.Stream(device=dev)
     sh = s.cuda_stream
     with torch.cuda.stream(s):
@@ -703,7 +712,7 @@ def long_prefill(args, dev, flush, calls: int = 5):
     folds = wl.n_c(T0) // wl.block
     pre_ms = float(min(pre))
     dec_us = 1e3 * float(np.median(ms))
-    nbytes = decode_bytes(T0, wl)
+    nbytes = decode_bytes(T0, wl, csz=_csz(args))
     return {"workload": f"{wl.name}: one layer, {T0}-row prefill in one append, then decode",
             "prefill_ms": pre_ms, "head_block_updates": folds * S * H * 2,
             "head_block_updates_per_s": folds * S * H * 2 / (pre_ms / 1e3),
@@ -711,6 +720,48 @@ def long_prefill(args, dev, flush, calls: int = 5):
             "decode_us": dec_us, "decode_bytes": nbytes,
             "decode_achieved_gbs": nbytes / (dec_us / 1e6) / 1e9,
             "decode_frac_of_hbm": nbytes / (dec_us / 1e6) / 1e9 / hbm}
+
+
+def layer_decode(args, dev, flush, coords: str, calls: int = 10):
+    """One layer of the headline workload (batch 8 x 8 kv-heads, 32 q-heads) filled to 32768 tokens
+    in one append, then decode calls, each after an L2 flush (CUDA events, median): the per-call
+    decode of the headline at its end length, for bf16 and fp32 coordinates."""
+    import torch
+    wl = WL
+    S, H, T, QH = wl.batch, wl.n_kv_heads, wl.tokens, wl.n_q_heads
+    cache = _cache(wl, n_layers=1, coord_bf16=coords == "bf16")
+    s = torch.cuda.Stream(device=dev)
+    sh = s.cuda_stream
+    with torch.cuda.stream(s):
+        K = syn.device_rows_batch(wl, range(S), 0, range(H), 0, device=dev)
+        V = syn.device_rows_batch(wl, range(S), 0, range(H), 1, device=dev)
+        cache.append(0, K, V, sh)
+        del K, V
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(12345)
+        q = torch.randn((S, QH, D), generator=gen, device=dev)
+        out = torch.empty_like(q)
+    s.synchronize()
+    assert cache.status(sh) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for i in range(args.warmup + calls):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0.record(s)
+            cache.decode(0, q, out, sh)
+            e1.record(s)
+        s.synchronize()
+        if i >= args.warmup:
+            ms.append(e0.elapsed_time(e1))
+    assert cache.status(sh) == 0 and bool(torch.isfinite(out).all())
+    cache.close()
+    hbm, _ = peaks()
+    us = 1e3 * float(np.median(ms))
+    nbytes = decode_bytes(T, wl, csz=2 if coords == "bf16" else 4)
+    return {"coords": coords, "launch_us": us, "bytes": nbytes,
+            "achieved_gbs": nbytes / (us / 1e6) / 1e9, "frac": nbytes / (us / 1e6) / 1e9 / hbm,
+            "frac_of_nominal": nbytes / (us / 1e6) / 1e9 / HBM_NOMINAL_GBS}
 
 
 def single_head(args, dev, flush):
@@ -772,7 +823,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "config": {"workload": WL.name, "global_batch": world * WL.batch, "seq_len": WL.tokens,
                    "layers": WL.n_layers, "kv_heads": WL.n_kv_heads, "q_heads": WL.n_q_heads,
                    "block": WL.block, "window": WL.window, "rank_k": WL.rank_k,
-                   "rank_v": WL.rank_v, "kv_dtype": WL.kv_dtype, "factor_dtype": "f32",
+                   "rank_v": WL.rank_v, "kv_dtype": WL.kv_dtype,
+                   "coords": args.coords, "basis_sigma": "f32",
                    "tokens_per_step": TOK_PER_STEP, "tokens": head["tokens"],
                    "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (about 29 GB of compressed history per token)"},
@@ -784,6 +836,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     }
     if world == 1 and rank == 0 and not args.no_extras:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        out["layer_decode_t32768"] = {c: layer_decode(args, dev, flush, c) for c in ("bf16", "f32")}
         out["single_head"] = single_head(args, dev, flush)
         out["llama3_8b_layer_stream"] = llama_layer_stream(args, dev, flush)
         out.update(all_layers_decode_step(args, dev, flush))
@@ -795,7 +848,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         print(json.dumps(out), flush=True)
 
 
-def run_profile_case(which: str):
+def run_profile_case(which: str, coords: str = "bf16"):
     """Short programs for profiler captures, with few launches before the captured ones."""
     import torch
     dev = torch.device("cuda", 0)
@@ -806,12 +859,12 @@ def run_profile_case(which: str):
         K = torch.from_numpy(kd.view(np.int16)).cuda().view(torch.bfloat16)[:, 0].transpose(0, 1)
         V = torch.from_numpy(vd.view(np.int16)).cuda().view(torch.bfloat16)[:, 0].transpose(0, 1)
         Q = torch.from_numpy(q[T - 1]).cuda()
-        cache = _cache(wl)
+        cache = _cache(wl, coord_bf16=coords == "bf16")
         cache.append(0, K.contiguous()[None], V.contiguous()[None])
     else:
         wl = WL if which == "long" else WL_PREFILL
         T = wl.tokens if which == "long" else wl.prefill
-        cache = _cache(wl, n_layers=1)
+        cache = _cache(wl, n_layers=1, coord_bf16=coords == "bf16")
         K = syn.device_rows_batch(wl, range(wl.batch), 0, range(wl.n_kv_heads), 0, T=T, device=dev)
         V = syn.device_rows_batch(wl, range(wl.batch), 0, range(wl.n_kv_heads), 1, T=T, device=dev)
         cache.append(0, K, V)
@@ -823,7 +876,8 @@ def run_profile_case(which: str):
         out = cache.decode(0, Q)
     torch.cuda.synchronize()
     print(json.dumps({"profile_case": which, "workload": wl.name, "tokens": cache.tokens(0),
-                      "decode_bytes": decode_bytes(cache.tokens(0), wl),
+                      "coords": coords,
+                      "decode_bytes": decode_bytes(cache.tokens(0), wl, csz=2 if coords == "bf16" else 4),
                       "status": cache.status(), "launches": cache.launches(),
                       "out_norm": float(out.norm())}))
     cache.close()
@@ -832,7 +886,7 @@ def run_profile_case(which: str):
 def main():
     args = parse()
     if args.profile_case:
-        run_profile_case(args.profile_case)
+        run_profile_case(args.profile_case, args.coords)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -84,11 +84,18 @@ typedef struct {
                           /*    basis and Sigma freeze and each later block is stored as its   */
                           /*    coordinates F B in the frozen basis (old coordinates untouched). */
                           /*    0: iS-KV. Cannot be combined with rotate_history = 0.           */
+    int coord_bf16;       /* 1: store the coordinates C = U Sigma (the k n factor scalars that    */
+                          /*    grow with the history) in bf16, rounded to nearest even after   */
+                          /*    every fold and history rotation; arithmetic stays fp32 and B,    */
+                          /*    Sigma stay fp32 ("Reconstruction and Storage": beta_f = 2 for C). */
+                          /*    Needs rank_k <= 64, rank_k and rank_v multiples of 8 and a GQA   */
+                          /*    group of 1, 2 or 4 (else ISKV_ERR_UNSUPPORTED). 0: fp32.         */
 } iskv_config;
 
 /*
  * Creates a cache for `cfg` on the current CUDA device. Allocates every device buffer
- * (coordinates C = U Sigma [max compressed rows x r] in fp32; bases B [d x r], Sigma [r] and the
+ * (coordinates C = U Sigma [max compressed rows x r] in fp32, or bf16 with coord_bf16; bases
+ * B [d x r], Sigma [r] and the
  * fold's H_top [r x r] in fp32, each in a ring of 2 buffers, or window / block + 3 with
  * lookahead_folds; the exact ring of window + block rows per path in kv_dtype; a RoPE table
  * [max_tokens x d/2] of (cos, sin); decode split partials; a status word) and, with
@@ -157,7 +164,8 @@ int iskv_reconstruct(iskv_handle *h, int layer, int which, int apply_rope, float
 /*
  * Copies the factors of one unit (layer, seq, kv_head, path) into caller buffers (device to
  * device, on `stream`) and reports its current rank and compressed-row count.
- *   coords_dev: fp32 [n_c][rank] (row stride = rank budget of the path), may be NULL;
+ *   coords_dev: fp32 [n_c][rank] (row stride = rank budget of the path; bf16-stored coordinates
+ *               are widened to fp32 exactly), may be NULL;
  *   basis_dev:  fp32 [head_dim][rank], may be NULL;
  *   sigma_dev:  fp32 [rank], may be NULL (entries >= *k_out are zero);
  *   k_out, n_c_out: host pointers, may be NULL.
@@ -196,8 +204,9 @@ int iskv_num_tokens(const iskv_handle *h, int layer, long long *t_out);
 
 /*
  * Persistent bytes of one layer per the storage formula of "Reconstruction and Storage":
- * beta_f * sum_X k_X (n_X + d + 1) + beta_e * d * sum_X e_X, summed over sequences and kv-heads,
- * with beta_f = 4 (fp32 factors) and beta_e = bytes of kv_dtype. Host only.
+ * sum_X [beta_c k_X n_X + 4 k_X (d + 1)] + beta_e * d * sum_X e_X, summed over sequences and
+ * kv-heads, with beta_c = 2 (coord_bf16) or 4 bytes per coordinate, fp32 bases and Sigma, and
+ * beta_e = bytes of kv_dtype. Host only.
  */
 int iskv_storage_bytes(const iskv_handle *h, int layer, long long *bytes_out);
 

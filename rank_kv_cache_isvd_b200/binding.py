@@ -56,6 +56,7 @@ class iskv_config(ctypes.Structure):
         ("rotate_history", ctypes.c_int),
         ("lookahead_folds", ctypes.c_int),
         ("fixed_basis", ctypes.c_int),
+        ("coord_bf16", ctypes.c_int),
     ]
 
 

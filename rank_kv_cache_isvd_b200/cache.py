@@ -18,12 +18,13 @@ class IsKVCache:
                  rank_k: int, rank_v: int, block: int, window: int, max_tokens: int,
                  kv_dtype: str = "bf16", rope: bool = True, rope_theta: float = 5e5,
                  rotate_history: bool = True, head_dim: int = 128,
-                 lookahead_folds: bool = False, fixed_basis: bool = False):
+                 lookahead_folds: bool = False, fixed_basis: bool = False,
+                 coord_bf16: bool = False):
         self.cfg = iskv_config(batch, n_layers, n_kv_heads, n_q_heads, head_dim, rank_k, rank_v,
                                block, window, max_tokens,
                                ISKV_BF16 if kv_dtype == "bf16" else ISKV_F32, int(rope),
                                float(rope_theta), int(rotate_history), int(lookahead_folds),
-                               int(fixed_basis))
+                               int(fixed_basis), int(coord_bf16))
         self.dtype = torch.bfloat16 if kv_dtype == "bf16" else torch.float32
         self.handle = 0
         code, h = iskv_create(self.cfg)

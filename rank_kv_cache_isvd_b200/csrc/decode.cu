@@ -74,8 +74,8 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(DecodeArgs a)
     float vacc[4] = {0.f, 0.f, 0.f, 0.f};
 
     const int q4 = tid & 3, rp = tid >> 2;     // channel quarter, row pair
-    const float *Ck = a.coords[0] + (size_t)ul * a.n_max * rK;
-    const float *Cv = a.coords[1] + (size_t)ul * a.n_max * rV;
+    const float *Ck = static_cast<const float *>(a.coords[0]) + (size_t)ul * a.n_max * rK;
+    const float *Cv = static_cast<const float *>(a.coords[1]) + (size_t)ul * a.n_max * rV;
     const size_t ring_base = (size_t)ul * a.R * D;
 
     for (long long t0 = p0; t0 < p1; t0 += DEC_TILE) {

@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
     }
 
     const size_t ring_base = (size_t)ul * a.R * D;
-    const float *Cv = a.coords[1] + (size_t)ul * a.n_max * rV;
+    const float *Cv = static_cast<const float *>(a.coords[1]) + (size_t)ul * a.n_max * rV;
     const uint32_t idesc = idesc_tf32(128, 128);
     const uint32_t abytes = x.kblocks * KBLK_BYTES;
 

@@ -1,0 +1,993 @@
+// Decode attention over the compressed cache, warp-specialised and persistent (sm_100a: TMA,
+// tcgen05 tensor cores with TMEM accumulators, mbarrier pipelines).
+//
+// iS-KV summary, "Reconstruction and Storage": compressed row i is (C B^T)[i] (C = U Sigma), the
+// window rows are exact. Keys are compressed before RoPE, so a tile of 128 reconstructed keys
+// K~ = C_K[tile] B_K^T is formed on the tensor cores (three-term tf32 for fp32 factors) and rotated
+// afterwards. RoPE at position t0 + tau (tile start t0, row tau) is split into two rotations:
+//   score_g = sum_j Re( conj(Q_gj e^{-i w_j t0}) * (k_j e^{i w_j tau}) ),  k_j = K~_j + i K~_{j+64},
+// so the queries are rotated once per tile (by t0) and every row by an angle that depends only on
+// tau, whose cosines and sines each thread keeps in registers for the whole kernel (no per-row
+// table reads). Values are accumulated in rank space (sum_i p_i C_V[i]) and expanded once through
+// B_V^T by the merge kernel.
+//
+// Work split: the (unit, tile) pairs of all units of the layer - each unit's compressed tiles
+// followed by its window tiles - are cut into one contiguous range per CTA (one CTA per SM), so
+// every SM streams the same number of tiles. A CTA's range covers segments of one or more units;
+// each segment leaves one partial (running max, sum, rank-space and channel-space accumulators)
+// per q-head, and the merge kernel combines the partials of a unit with log-sum-exp weights.
+//
+// Warp roles (12 warps):
+//   warp 0      TMA producer: queries, B_K, key-coordinate tiles (K ring), value tiles (V ring);
+//   warps 1-3   split the fp32 key tiles into tf32 hi + lo parts; warp 1 issues the MMAs into one
+//               of two TMEM accumulators and commits them to the ring barriers;
+//   warps 4-11  epilogue: two threads per row (TMEM lane = row, each half of the RoPE pairs);
+//               rotation and dot products, online softmax, value sums, partial records.
+// Every wait is bounded: a wait that gives up raises a CTA-wide abort flag, the sticky device
+// status is set to ISKV_ERR_TIMEOUT, and the CTA drains its own copies and MMAs before it exits.
+#include <math_constants.h>
+
+#include "iskv_internal.cuh"
+#include "tc_util.cuh"
+
+namespace iskv {
+
+constexpr int WS_THREADS = 384;
+constexpr int WS_EPI = 256;                  // epilogue threads (warps 4 .. 11)
+constexpr int WS_NSK = 2;                    // key-coordinate stages
+constexpr int WS_MAXSV = 4;                  // value stages (at most)
+constexpr uint32_t WS_BLK = 128u * 128u;     // 128 rows x 128 bytes
+constexpr int BAR_EPI = 1, BAR_SPLIT = 2;    // named barriers
+constexpr float LOG2E = 1.4426950408889634f;
+// register split: producer/split warpgroup, epilogue warpgroups, and the per-thread count the
+// launch must grant for it (128 x 64 + 256 x 200 = 384 x 154.7)
+constexpr int WS_REG_LO = 64, WS_REG_HI = 200, WS_REG_LAUNCH = 160;
+static_assert(128 * WS_REG_LO + 256 * WS_REG_HI <= WS_THREADS * WS_REG_LAUNCH,
+              "register split exceeds the launch allocation");
+
+struct WsLayout {
+    uint32_t bh, bl, kst, vst, q, qt, ss, sp, smax, ssum, bars, total;
+    uint32_t kstage, vstage;
+    int nsv;
+};
+
+// Shared-memory plan. fp32 coordinates: a K stage holds the tile's tf32 hi part (in place) and its
+// lo part; bf16 coordinates: the tile only (exact bf16 operands). The reduction area of the partial records aliases the
+// per-tile buffers qt, ss and sp (free at the end of a segment).
+__host__ __device__ inline WsLayout ws_layout(int bf, int rV, int esz, int G, uint32_t limit) {
+    WsLayout L;
+    uint32_t o = 0;
+    // B_K terms: fp32 coordinates use tf32 (hi, lo); bf16 coordinates use three bf16 terms of the
+    // fp32 basis (hi, mid, lo: 24 significant bits), the third at bl + WS_BLK
+    L.bh = o; o += WS_BLK;
+    L.bl = o; o += bf ? 2u * WS_BLK : WS_BLK;
+    L.kstage = bf ? WS_BLK : 2u * WS_BLK;
+    L.kst = o; o += WS_NSK * L.kstage;
+    const uint32_t vc = 128u * rV * (bf ? 2u : 4u), vw = 128u * D * esz;
+    L.vstage = ((vc > vw ? vc : vw) + 1023u) & ~1023u;
+    L.vst = o;
+    const uint32_t misc = (uint32_t)G * 512u * 2u            // q, two segment slots
+                          + (uint32_t)G * 512u * 8u          // qt[2], ss[2][2], sp[2]
+                          + 2u * 2u * 4u * 4u * 4u           // smax, ssum
+                          + 256u + 1024u;                    // barriers, alignment slack
+    int nsv = WS_MAXSV;
+    while (nsv > 2 && o + nsv * L.vstage + misc > limit) --nsv;
+    L.nsv = nsv;
+    o += nsv * L.vstage;
+    L.q = o; o += G * 512u * 2u;
+    L.qt = o; o += G * 512u * 2u;
+    L.ss = o; o += G * 512u * 4u;
+    L.sp = o; o += G * 512u * 2u;
+    L.smax = o; o += 2u * 4u * 4u * 4u;
+    L.ssum = o; o += 2u * 4u * 4u * 4u;
+    L.bars = o; o += 256u;
+    L.total = o + 1024u;
+    return L;
+}
+
+size_t ws_smem_bytes(int bf, int rV, int esz, int G) {
+    return ws_layout(bf, rV, esz, G, 227u * 1024u).total;
+}
+
+// ---- small device helpers --------------------------------------------------------------------
+__device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait that also gives up as soon as another role raised the abort flag.
+__device__ __forceinline__ bool wait_ab(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    for (uint32_t i = 0; i < MBAR_SPIN_LIMIT; ++i) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void bar_named(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Named barrier that also returns the AND of `v` over the participating threads.
+__device__ __forceinline__ bool bar_and(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void ws_griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void ws_griddep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// 8 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld8x(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 with bf16 operands, one CTA.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor: D fp32, A and B bf16, both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+// fp32 values in place -> their tf32 "hi" part (top 19 bits); the exact remainder "lo" at the
+// same offset of `lo`. Threads t0 .. t0 + nt - 1 of the CTA share the work.
+__device__ __forceinline__ void split_tf32_range(uint8_t *hi, uint8_t *lo, int bytes, int t,
+                                                 int nt) {
+    float4 *h4 = reinterpret_cast<float4 *>(hi);
+    float4 *l4 = reinterpret_cast<float4 *>(lo);
+    for (int i = t; i < bytes / 16; i += nt) {
+        float4 x = h4[i], h, l;
+        h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
+        h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
+        h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u);
+        h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u);
+        l.x = x.x - h.x;
+        l.y = x.y - h.y;
+        l.z = x.z - h.z;
+        l.w = x.w - h.w;
+        h4[i] = h;
+        l4[i] = l;
+    }
+}
+
+// Three bf16 terms (hi + mid + lo, 24 significant bits) of a fp32 basis [D][rK] (rK <= 64, even),
+// written as 128 rows x 64 columns (zero beyond rK) in the 128-byte-swizzled K-major layout: the
+// 16-byte chunk c of row n sits at chunk c ^ (n mod 8). Threads t, t + nt, ... share the work.
+__device__ __forceinline__ void build_b_terms(uint8_t *bh, uint8_t *bm, uint8_t *bl,
+                                              const float *B, int rK, int t, int nt) {
+    for (int p = t; p < 128 * 32; p += nt) {
+        const int n = p >> 5, k = (p & 31) * 2;
+        float v0 = 0.f, v1 = 0.f;
+        if (k < rK) {
+            const float2 f = *reinterpret_cast<const float2 *>(B + (size_t)n * rK + k);
+            v0 = f.x;
+            v1 = f.y;
+        }
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+        const float r0 = v0 - __low2float(h), r1 = v1 - __high2float(h);
+        const __nv_bfloat162 m = __floats2bfloat162_rn(r0, r1);
+        const __nv_bfloat162 l = __floats2bfloat162_rn(r0 - __low2float(m), r1 - __high2float(m));
+        const uint32_t byte = (uint32_t)k * 2u;
+        const uint32_t off = (uint32_t)n * 128u + ((((byte >> 4) ^ (uint32_t)(n & 7)) << 4) | (byte & 15u));
+        *reinterpret_cast<__nv_bfloat162 *>(bh + off) = h;
+        *reinterpret_cast<__nv_bfloat162 *>(bm + off) = m;
+        *reinterpret_cast<__nv_bfloat162 *>(bl + off) = l;
+    }
+}
+
+// 8 consecutive channels of an exact row (bf16 or fp32) as fp32.
+__device__ __forceinline__ void load_row8(const void *base, size_t idx, int kv_dtype,
+                                          float (&v)[8]) {
+    if (kv_dtype == ISKV_BF16) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(
+            reinterpret_cast<const __nv_bfloat16 *>(base) + idx);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            v[2 * e] = __uint_as_float(w[e] << 16);
+            v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+    } else {
+        const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(base) + idx);
+        const float4 a = p[0], b = p[1];
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
+// Four consecutive values of a staged value row: fmt 2 = bf16, 4 = fp32.
+__device__ __forceinline__ float4 load_v4s(const uint8_t *row, int c, int fmt) {
+    if (fmt == 2) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(row + 2 * c);
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                           __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+    }
+    return *reinterpret_cast<const float4 *>(row + 4 * c);
+}
+
+// The CTA's tile range and the segment (unit, first tile, end tile) containing tile g.
+struct WsRange {
+    long long g0, g1;
+};
+__device__ __forceinline__ WsRange ws_range(const WsExtra &x, int c) {
+    WsRange r;
+    r.g0 = (long long)c * x.N / x.P;
+    r.g1 = (long long)(c + 1) * x.N / x.P;
+    return r;
+}
+
+// ---- the split kernel --------------------------------------------------------------------------
+template <bool BF, int GT>
+__global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
+    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmB,
+    DecodeArgs a, WsExtra x) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int G = GT;
+    const int rV = a.r[1];
+    const int esz = a.kv_dtype == ISKV_BF16 ? 2 : 4;
+    const WsLayout L = ws_layout(BF ? 1 : 0, rV, esz, G, 227u * 1024u);
+    const int NSV = L.nsv;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L.bars);
+    uint64_t *k_full = bars, *k_empty = bars + 2, *v_full = bars + 4, *v_empty = bars + 8;
+    uint64_t *b_full = bars + 12, *b_empty = bars + 13, *acc_full = bars + 14,
+             *acc_empty = bars + 16, *q_full = bars + 18, *q_empty = bars + 20;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 22);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 23);
+    int *counters = reinterpret_cast<int *>(bars + 24);    // [8] progress, read at teardown
+    float *sQ = reinterpret_cast<float *>(sm + L.q);        // [2 slots][G][128]
+    float *sQt = reinterpret_cast<float *>(sm + L.qt);      // [2][G][128] rotated, scaled
+    float *sS = reinterpret_cast<float *>(sm + L.ss);       // [2][2 halves][G][128]
+    float *sP = reinterpret_cast<float *>(sm + L.sp);       // [2][128][G]
+    float *sMax = reinterpret_cast<float *>(sm + L.smax);   // [2][4][4]
+    float *sSum = reinterpret_cast<float *>(sm + L.ssum);   // [2][4][4]
+    float4 *sRed = reinterpret_cast<float4 *>(sm + L.qt);   // [8 warps][G][32] (aliases qt..sp)
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const WsRange rg = ws_range(x, blockIdx.x);
+    const int Tc = x.Tc, Tu = x.Tu;
+    const long long u_first = rg.g0 / Tu;
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(k_full + i, 1);
+            mbar_init(k_empty + i, 1);
+            mbar_init(acc_full + i, 1);
+            mbar_init(acc_empty + i, 8);
+            mbar_init(q_full + i, 1);
+            mbar_init(q_empty + i, 8);
+        }
+        for (int i = 0; i < WS_MAXSV; ++i) {
+            mbar_init(v_full + i, 1);
+            mbar_init(v_empty + i, 8);
+        }
+        mbar_init(b_full, 1);
+        mbar_init(b_empty, 1);
+        *abort_flag = 0;
+        for (int i = 0; i < 8; ++i) counters[i] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // registers move from the producer/split warpgroup to the two epilogue warpgroups; the launch
+    // grants at least WS_REG_LAUNCH per thread (checked on the host before the first launch), so
+    // 128 x WS_REG_LO + 256 x WS_REG_HI fits the block's allocation
+    if (warp < 4)
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(WS_REG_LO));
+    else
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(WS_REG_HI));
+
+    // every segment of this CTA, in order: unit u, tiles [ta, tb) of the unit
+    auto seg_of = [&](long long g, long long &u, int &ta, int &tb) {
+        u = g / Tu;
+        ta = (int)(g - u * Tu);
+        const long long left = rg.g1 - g;
+        tb = (int)min((long long)Tu, ta + left);
+    };
+
+    if (warp == 0) {
+        // ==================================== producer ===========================================
+        int kt = 0, vt = 0, seg = 0, bseg = 0;
+        ws_griddep_wait();
+        if (lane == 0) {
+            bool ok = true;
+            for (long long g = rg.g0; g < rg.g1 && ok;) {
+                long long u;
+                int ta, tb;
+                seg_of(g, u, ta, tb);
+                const int seq = (int)(u / a.H), h = (int)(u % a.H);
+                // queries of this unit's q-heads
+                const int qs = seg & 1;
+                ok = wait_ab(q_empty + qs, ((seg >> 1) & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                mbar_arrive_expect_tx(q_full + qs, (uint32_t)(G * D * 4));
+                bulk_load(sQ + qs * G * D, a.q + ((size_t)seq * a.H * G + (size_t)h * G) * D,
+                          (uint32_t)(G * D * 4), q_full + qs);
+                ++seg;
+                counters[0] = seg;
+                if (!BF && ta < Tc) {
+                    // B_K of this unit (one buffer; free once the previous segment's MMAs are done)
+                    ok = wait_ab(b_empty, (bseg & 1) ^ 1, abort_flag);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(b_full, WS_BLK);
+                    tma_load_2d(sm + L.bh, &tmB, 0, x.brow0 + (int)u * D, b_full);
+                    ++bseg;
+                    counters[1] = bseg;
+                }
+                for (int tl = ta; tl < tb && ok; ++tl) {
+                    const bool comp = tl < Tc;
+                    long long t0;
+                    int rows;
+                    if (comp) {
+                        t0 = (long long)tl * DEC_TILE;
+                        rows = (int)min((long long)DEC_TILE, a.n_c - t0);
+                        const int ks = kt % WS_NSK;
+                        ok = wait_ab(k_empty + ks, ((kt / WS_NSK) & 1) ^ 1, abort_flag);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(k_full + ks, WS_BLK);
+                        tma_load_2d(sm + L.kst + ks * L.kstage, &tmC, 0,
+                                    (int)(x.row0 + u * a.n_max + t0), k_full + ks);
+                        ++kt;
+                        counters[2] = kt;
+                    } else {
+                        t0 = a.n_c + (long long)(tl - Tc) * DEC_TILE;
+                        rows = (int)min((long long)DEC_TILE, a.t - t0);
+                    }
+                    const int vs = vt % NSV;
+                    ok = wait_ab(v_empty + vs, ((vt / NSV) & 1) ^ 1, abort_flag);
+                    if (!ok) break;
+                    uint8_t *dst = sm + L.vst + vs * L.vstage;
+                    if (comp) {
+                        const uint32_t fsz = BF ? 2u : 4u;
+                        const uint32_t nb = (uint32_t)rows * rV * fsz;
+                        mbar_arrive_expect_tx(v_full + vs, nb);
+                        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.coords[1]) +
+                                             ((size_t)u * a.n_max + t0) * rV * fsz;
+                        bulk_load(dst, src, nb, v_full + vs);
+                    } else {
+                        const int s0 = (int)(t0 % a.R);
+                        const int n1 = min(rows, a.R - s0);
+                        const uint32_t rb = D * esz;
+                        const char *ring = static_cast<const char *>(a.ring[1]) +
+                                           (size_t)u * a.R * D * esz;
+                        mbar_arrive_expect_tx(v_full + vs, (uint32_t)rows * rb);
+                        bulk_load(dst, ring + (size_t)s0 * rb, (uint32_t)n1 * rb, v_full + vs);
+                        if (n1 < rows)
+                            bulk_load(dst + (size_t)n1 * rb, ring, (uint32_t)(rows - n1) * rb,
+                                      v_full + vs);
+                    }
+                    ++vt;
+                    counters[3] = vt;
+                }
+                g += tb - ta;
+            }
+        }
+    } else if (warp < 4) {
+        // =============================== split + MMA issue =======================================
+        const int st = tid - 32;                        // 0 .. 95
+        int kt = 0, at = 0, bseg = 0;
+        ws_griddep_wait();
+        bool ok = true;
+        const uint32_t idesc = BF ? idesc_bf16(128, 128) : idesc_tf32(128, 128);
+        for (long long g = rg.g0; g < rg.g1 && ok;) {
+            long long u;
+            int ta, tb;
+            seg_of(g, u, ta, tb);
+            g += tb - ta;
+            if (ta >= Tc) continue;
+            bool w;
+            if (BF) {
+                // three bf16 terms of this unit's fp32 basis, written in the 128-byte-swizzled
+                // K-major layout, once the previous segment's MMAs no longer read them
+                w = wait_ab(b_empty, (bseg & 1) ^ 1, abort_flag);
+                if (w) {
+                    build_b_terms(sm + L.bh, sm + L.bl, sm + L.bl + WS_BLK,
+                                  a.basis[0] + (size_t)u * D * a.r[0], a.r[0], st, 96);
+                    fence_proxy_async_smem();
+                }
+            } else {
+                w = wait_ab(b_full, bseg & 1, abort_flag);
+                if (w) {
+                    split_tf32_range(sm + L.bh, sm + L.bl, WS_BLK, st, 96);
+                    fence_proxy_async_smem();
+                }
+            }
+            ok = bar_and(BAR_SPLIT, 96, w);
+            if (!ok) break;
+            ++bseg;
+            const int te = min(tb, Tc);
+            for (int tl = ta; tl < te; ++tl) {
+                const int ks = kt % WS_NSK;
+                uint8_t *A = sm + L.kst + ks * L.kstage;
+                w = wait_ab(k_full + ks, (kt / WS_NSK) & 1, abort_flag);
+                if (!BF && w) {
+                    split_tf32_range(A, A + WS_BLK, WS_BLK, st, 96);
+                    fence_proxy_async_smem();
+                }
+                ok = bar_and(BAR_SPLIT, 96, w);
+                if (!ok) break;
+                if (st == 0) {
+                    const int buf = at & 1;
+                    bool e = wait_ab(acc_empty + buf, ((at >> 1) & 1) ^ 1, abort_flag);
+                    if (e) {
+                        tc_fence_after();
+                        const uint32_t d = tmem + 128u * buf;
+                        const uint32_t aH = smem_u32(A), bH = smem_u32(sm + L.bh);
+                        if (BF) {
+                            // C (exact bf16) times the three terms of B; K steps of 16 columns
+                            const int nk = (a.r[0] + 15) >> 4;
+                            const uint32_t bM = smem_u32(sm + L.bl), bL = bM + WS_BLK;
+                            for (int kk = 0; kk < nk; ++kk) {
+                                const uint32_t off = kk * 32;
+                                mma_bf16(d, sw128_kmajor_desc(aH + off), sw128_kmajor_desc(bH + off),
+                                         idesc, kk > 0);
+                                mma_bf16(d, sw128_kmajor_desc(aH + off), sw128_kmajor_desc(bM + off),
+                                         idesc, 1);
+                                mma_bf16(d, sw128_kmajor_desc(aH + off), sw128_kmajor_desc(bL + off),
+                                         idesc, 1);
+                            }
+                        } else {
+                            const uint32_t aL = aH + WS_BLK, bL = smem_u32(sm + L.bl);
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t off = kk * 32;
+                                mma_tf32(d, sw128_kmajor_desc(aH + off), sw128_kmajor_desc(bH + off),
+                                         idesc, kk > 0);
+                                mma_tf32(d, sw128_kmajor_desc(aH + off), sw128_kmajor_desc(bL + off),
+                                         idesc, 1);
+                                mma_tf32(d, sw128_kmajor_desc(aL + off), sw128_kmajor_desc(bH + off),
+                                         idesc, 1);
+                            }
+                        }
+                        mma_commit(acc_full + buf);
+                        mma_commit(k_empty + ks);
+                        if (tl + 1 == te) mma_commit(b_empty);
+                        counters[4] = at + 1;
+                        counters[5] = kt + 1;
+                    }
+                    // on a failed wait the abort flag is raised: every thread's next wait gives up
+                    // and the next split barrier ends the loop for the whole group
+                }
+                __syncwarp();
+                ++kt;
+                ++at;
+            }
+        }
+    } else {
+        // ==================================== epilogue ===========================================
+        const int et = tid - 128;                       // 0 .. 255
+        const int ew = warp - 4, qw = warp & 3, hf = ew >> 2;
+        const int tau = 32 * qw + lane;
+        const int jb = 32 * hf;                         // first RoPE pair of this thread
+        // this row's rotation e^{i w_j tau} for the thread's 32 pairs (fixed for the kernel)
+        float tc_[32], ts_[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            tc_[i] = 1.f;
+            ts_[i] = 0.f;
+        }
+        if (a.rope_cs != nullptr && tau < x.rope_rows) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float2 c = a.rope_cs[(size_t)tau * DH + jb + i];
+                tc_[i] = c.x;
+                ts_[i] = c.y;
+            }
+        }
+        ws_griddep_wait();
+        const float qscale = a.scale * LOG2E;           // scores in log2 units
+        // value-sum layout: thread = (quad qd, slice sl); compressed tiles use kV's quads,
+        // window tiles the 32 channel quads
+        const int nqr = (rV + 3) >> 2;
+        const int nqpr = nqr <= 8 ? 8 : nqr <= 16 ? 16 : 32;
+        const int qdr = et & (nqpr - 1), slr = et / nqpr, nslr = WS_EPI / nqpr;
+        const int qdw = et & 31, slw = et >> 5;
+        bool ok = true;
+        int at = 0, vt = 0, seg = 0, it = 0;
+
+        // q~ = (q rotated by -w_j t0) * scale * log2(e) for tile start t0, into qt buffer `b`
+        auto make_qt = [&](const float *q, long long t0, int b) {
+            for (int o = et; o < G * DH; o += WS_EPI) {
+                const int g = o / DH, j = o % DH;
+                float c = 1.f, s = 0.f;
+                if (a.rope_cs != nullptr) {
+                    const float2 cs = a.rope_cs[(size_t)t0 * DH + j];
+                    c = cs.x;
+                    s = cs.y;
+                }
+                const float qr = q[g * D + j], qi = q[g * D + DH + j];
+                sQt[(b * G + g) * D + j] = qscale * fmaf(qr, c, qi * s);
+                sQt[(b * G + g) * D + DH + j] = qscale * fmaf(qi, c, -qr * s);
+            }
+        };
+
+        for (long long g = rg.g0; g < rg.g1 && ok;) {
+            long long u;
+            int ta, tb;
+            seg_of(g, u, ta, tb);
+            g += tb - ta;
+            const int jseg = (int)(u - u_first);
+            const int qs = seg & 1;
+            bool w = wait_ab(q_full + qs, (seg >> 1) & 1, abort_flag);
+            const float *q = sQ + qs * G * D;
+            float mrun[GT], lrun[GT];
+            float4 vr[GT], vw[GT];
+#pragma unroll
+            for (int gg = 0; gg < GT; ++gg) {
+                mrun[gg] = -CUDART_INF_F;
+                lrun[gg] = 0.f;
+                vr[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
+                vw[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            const long long t0a = ta < Tc ? (long long)ta * DEC_TILE
+                                          : a.n_c + (long long)(ta - Tc) * DEC_TILE;
+            if (w) make_qt(q, t0a, it & 1);
+            ok = bar_and(BAR_EPI, WS_EPI, w);
+            if (!ok) break;
+            bool good = true;                       // this thread's waits of the segment so far
+            const bool has_c = ta < Tc, has_w = tb > Tc;
+            for (int tl = ta; tl < tb; ++tl) {
+                const int b = it & 1;
+                const bool comp = tl < Tc;
+                const long long t0 = comp ? (long long)tl * DEC_TILE
+                                          : a.n_c + (long long)(tl - Tc) * DEC_TILE;
+                const int rows = (int)min((long long)DEC_TILE, (comp ? a.n_c : a.t) - t0);
+                const bool valid = tau < rows;
+                const long long pos = t0 + tau;
+                // ---- this row's key: pairs (j, j + 64), j in [jb, jb + 32), chunks of 8 pairs,
+                //      rotated by e^{i w_j tau} and dotted with the rotated queries ----------------
+                float2 acc2[GT];
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg) acc2[gg] = make_float2(0.f, 0.f);
+                bool wk = true;
+                if (comp) wk = wait_ab(acc_full + (at & 1), (at >> 1) & 1, abort_flag);
+                // the tensor-memory loads below are warp-collective: decide per warp
+                wk = __all_sync(0xffffffffu, wk);
+                good = good && wk;
+                tc_fence_after();
+                const uint32_t trow = tmem + 128u * (at & 1) + ((uint32_t)(qw * 32) << 16);
+                const bool fresh = !comp && pos == a.new_pos;
+                const void *ksrc = fresh ? a.new_row[0] : a.ring[0];
+                const size_t kbase = fresh ? (size_t)u * D
+                                           : ((size_t)u * a.R + (size_t)(pos % a.R)) * D;
+                const float *qt = sQt + (size_t)b * G * D;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int j0 = jb + 8 * ch;
+                    float lo[8], hi[8];
+                    if (comp) {
+                        if (wk) {
+                            tmem_ld8x(trow + j0, lo);
+                            tmem_ld8x(trow + DH + j0, hi);
+                            tmem_wait_ld();
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) lo[i] = hi[i] = 0.f;
+                        }
+                    } else if (valid) {
+                        load_row8(ksrc, kbase + j0, a.kv_dtype, lo);
+                        load_row8(ksrc, kbase + DH + j0, a.kv_dtype, hi);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) lo[i] = hi[i] = 0.f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 k1 = make_float2(lo[2 * i], lo[2 * i + 1]);
+                        const float2 k2 = make_float2(hi[2 * i], hi[2 * i + 1]);
+                        const float2 c2 = make_float2(tc_[8 * ch + 2 * i], tc_[8 * ch + 2 * i + 1]);
+                        const float2 s2 = make_float2(ts_[8 * ch + 2 * i], ts_[8 * ch + 2 * i + 1]);
+                        const float2 t1 = __fmul2_rn(k2, s2);
+                        const float2 zr = __ffma2_rn(k1, c2, make_float2(-t1.x, -t1.y));
+                        const float2 zi = __ffma2_rn(k1, s2, __fmul2_rn(k2, c2));
+#pragma unroll
+                        for (int gg = 0; gg < GT; ++gg) {
+                            const float2 qr = *reinterpret_cast<const float2 *>(qt + gg * D + j0 + 2 * i);
+                            const float2 qi = *reinterpret_cast<const float2 *>(qt + gg * D + DH + j0 + 2 * i);
+                            acc2[gg] = __ffma2_rn(qr, zr, acc2[gg]);
+                            acc2[gg] = __ffma2_rn(qi, zi, acc2[gg]);
+                        }
+                    }
+                }
+                if (comp) {
+                    // the accumulator is read: let the MMA warp reuse it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0 && wk) mbar_arrive(acc_empty + (at & 1));
+                    ++at;
+                }
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg)
+                    sS[((b * 2 + hf) * G + gg) * 128 + tau] = acc2[gg].x + acc2[gg].y;
+                ok = bar_and(BAR_EPI, WS_EPI, good);                     // barrier 1
+                if (!ok) break;
+                // ---- full scores; tile maxima per quarter; next tile's queries ---------------
+                float sc[GT];
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg) {
+                    sc[gg] = valid ? sS[((b * 2 + 0) * G + gg) * 128 + tau] +
+                                         sS[((b * 2 + 1) * G + gg) * 128 + tau]
+                                   : -CUDART_INF_F;
+                    float m = sc[gg];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                    if (hf == 0 && lane == 0) sMax[(b * 4 + qw) * 4 + gg] = m;
+                }
+                if (tl + 1 < tb) {
+                    const int tn = tl + 1;
+                    const long long t0n = tn < Tc ? (long long)tn * DEC_TILE
+                                                  : a.n_c + (long long)(tn - Tc) * DEC_TILE;
+                    make_qt(q, t0n, b ^ 1);
+                }
+                bar_named(BAR_EPI, WS_EPI);                              // barrier 2
+                float alpha[GT];
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg) {
+                    const float mt = fmaxf(fmaxf(sMax[(b * 4 + 0) * 4 + gg], sMax[(b * 4 + 1) * 4 + gg]),
+                                           fmaxf(sMax[(b * 4 + 2) * 4 + gg], sMax[(b * 4 + 3) * 4 + gg]));
+                    const float mn = fmaxf(mrun[gg], mt);
+                    alpha[gg] = ex2(mrun[gg] - mn);
+                    mrun[gg] = mn;
+                    if (GT == 1 ? hf == 0 : (gg & 1) == hf) {
+                        const float p = valid ? ex2(sc[gg] - mn) : 0.f;
+                        sP[(b * 128 + tau) * G + gg] = p;
+                        float s = p;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                        if (lane == 0) sSum[(b * 4 + qw) * 4 + gg] = s;
+                    }
+                }
+                bar_named(BAR_EPI, WS_EPI);                              // barrier 3
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg) {
+                    const float s = (sSum[(b * 4 + 0) * 4 + gg] + sSum[(b * 4 + 1) * 4 + gg]) +
+                                    (sSum[(b * 4 + 2) * 4 + gg] + sSum[(b * 4 + 3) * 4 + gg]);
+                    lrun[gg] = fmaf(lrun[gg], alpha[gg], s);
+                    const float2 al = make_float2(alpha[gg], alpha[gg]);
+                    float2 x01 = __fmul2_rn(al, make_float2(vr[gg].x, vr[gg].y));
+                    float2 x23 = __fmul2_rn(al, make_float2(vr[gg].z, vr[gg].w));
+                    vr[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
+                    x01 = __fmul2_rn(al, make_float2(vw[gg].x, vw[gg].y));
+                    x23 = __fmul2_rn(al, make_float2(vw[gg].z, vw[gg].w));
+                    vw[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
+                }
+                // ---- value sums: v_g += sum_i p[g][i] V[i][quad] ----------------------------
+                const int vs = vt % NSV;
+                const bool wv = wait_ab(v_full + vs, (vt / NSV) & 1, abort_flag);
+                good = good && wv;
+                const uint8_t *V = sm + L.vst + vs * L.vstage;
+                const float *P = sP + (size_t)b * 128 * G;
+                if (wv) {
+                    if (comp) {
+                        const int vld = rV * (BF ? 2 : 4);
+#pragma unroll 4
+                        for (int i = slr; i < rows; i += nslr) {
+                            const float4 v = load_v4s(V + (size_t)i * vld, 4 * qdr, BF ? 2 : 4);
+                            const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
+#pragma unroll
+                            for (int gg = 0; gg < GT; ++gg) {
+                                const float pg = P[i * G + gg];
+                                const float2 p2 = make_float2(pg, pg);
+                                const float2 x01 = __ffma2_rn(p2, v01, make_float2(vr[gg].x, vr[gg].y));
+                                const float2 x23 = __ffma2_rn(p2, v23, make_float2(vr[gg].z, vr[gg].w));
+                                vr[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
+                            }
+                        }
+                    } else {
+                        const int vld = D * esz;
+                        const int inew = (a.new_pos >= t0 && a.new_pos < t0 + rows)
+                                             ? (int)(a.new_pos - t0) : -1;
+#pragma unroll 4
+                        for (int i = slw; i < rows; i += 8) {
+                            float4 v;
+                            if (i == inew) {
+                                float t8[8];
+                                load_row8(a.new_row[1], (size_t)u * D + (4 * qdw & ~7), a.kv_dtype, t8);
+                                const int o4 = (4 * qdw) & 7;
+                                v = make_float4(t8[o4], t8[o4 + 1], t8[o4 + 2], t8[o4 + 3]);
+                            } else {
+                                v = load_v4s(V + (size_t)i * vld, 4 * qdw, esz);
+                            }
+                            const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
+#pragma unroll
+                            for (int gg = 0; gg < GT; ++gg) {
+                                const float pg = P[i * G + gg];
+                                const float2 p2 = make_float2(pg, pg);
+                                const float2 x01 = __ffma2_rn(p2, v01, make_float2(vw[gg].x, vw[gg].y));
+                                const float2 x23 = __ffma2_rn(p2, v23, make_float2(vw[gg].z, vw[gg].w));
+                                vw[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
+                            }
+                        }
+                        if (inew >= 0 && et < D) {
+                            // fused append: store the new position's K and V rows in the ring
+                            const size_t slot = ((size_t)u * a.R + (size_t)(a.new_pos % a.R)) * D + et;
+                            if (a.kv_dtype == ISKV_BF16) {
+                                const __nv_bfloat16 *nk = static_cast<const __nv_bfloat16 *>(a.new_row[0]) + (size_t)u * D;
+                                const __nv_bfloat16 *nv = static_cast<const __nv_bfloat16 *>(a.new_row[1]) + (size_t)u * D;
+                                const_cast<__nv_bfloat16 *>(static_cast<const __nv_bfloat16 *>(a.ring[0]))[slot] = nk[et];
+                                const_cast<__nv_bfloat16 *>(static_cast<const __nv_bfloat16 *>(a.ring[1]))[slot] = nv[et];
+                            } else {
+                                const float *nk = static_cast<const float *>(a.new_row[0]) + (size_t)u * D;
+                                const float *nv = static_cast<const float *>(a.new_row[1]) + (size_t)u * D;
+                                const_cast<float *>(static_cast<const float *>(a.ring[0]))[slot] = nk[et];
+                                const_cast<float *>(static_cast<const float *>(a.ring[1]))[slot] = nv[et];
+                            }
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(v_empty + vs);
+                ++vt;
+                ++it;
+            }
+            // q slot consumed (every q~ of the segment is built)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_empty + qs);
+            ++seg;
+            ok = bar_and(BAR_EPI, WS_EPI, ok && good);    // tiles done: the reduction area is free
+            if (!ok) break;
+            // ---- partial record: [m, l, acc_rank[rV], acc_chan[D]] per q-head ---------------------
+            float *rec = a.ws + ((size_t)blockIdx.x * x.maxseg + jseg) * G * (2 + rV + D);
+            if (has_c) {
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg) {
+                    for (int o = nqpr; o < 32; o <<= 1) {
+                        vr[gg].x += __shfl_xor_sync(0xffffffffu, vr[gg].x, o);
+                        vr[gg].y += __shfl_xor_sync(0xffffffffu, vr[gg].y, o);
+                        vr[gg].z += __shfl_xor_sync(0xffffffffu, vr[gg].z, o);
+                        vr[gg].w += __shfl_xor_sync(0xffffffffu, vr[gg].w, o);
+                    }
+                    if (lane < nqpr) sRed[(ew * G + gg) * 32 + qdr] = vr[gg];
+                }
+                bar_named(BAR_EPI, WS_EPI);
+                for (int o = et; o < G * rV; o += WS_EPI) {
+                    const int gg = o / rV, c = o % rV;
+                    float s = 0.f;
+#pragma unroll
+                    for (int w8 = 0; w8 < 8; ++w8)
+                        s += reinterpret_cast<const float *>(sRed)[((w8 * G + gg) * 32) * 4 + c];
+                    rec[gg * (2 + rV + D) + 2 + c] = s;
+                }
+                bar_named(BAR_EPI, WS_EPI);
+            } else {
+                for (int o = et; o < G * rV; o += WS_EPI)
+                    rec[(o / rV) * (2 + rV + D) + 2 + o % rV] = 0.f;
+            }
+            if (has_w) {
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg) sRed[(ew * G + gg) * 32 + qdw] = vw[gg];
+                bar_named(BAR_EPI, WS_EPI);
+                for (int o = et; o < G * D; o += WS_EPI) {
+                    const int gg = o / D, c = o % D;
+                    float s = 0.f;
+#pragma unroll
+                    for (int w8 = 0; w8 < 8; ++w8)
+                        s += reinterpret_cast<const float *>(sRed)[((w8 * G + gg) * 32) * 4 + c];
+                    rec[gg * (2 + rV + D) + 2 + rV + c] = s;
+                }
+                bar_named(BAR_EPI, WS_EPI);
+            } else {
+                for (int o = et; o < G * D; o += WS_EPI)
+                    rec[(o / D) * (2 + rV + D) + 2 + rV + o % D] = 0.f;
+            }
+            if (et < G) {
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg)
+                    if (gg == et) {
+                        rec[gg * (2 + rV + D)] = mrun[gg];
+                        rec[gg * (2 + rV + D) + 1] = lrun[gg];
+                    }
+            }
+        }
+        if (et == 0) {
+            counters[6] = at;
+            counters[7] = vt;
+        }
+    }
+
+    // ---- teardown: after an abort, wait (bounded) for this CTA's own copies and MMAs ------------
+    ws_griddep_launch();
+    __syncthreads();
+    if (*abort_flag && tid == 0) {
+        set_status(x.status, ISKV_ERR_TIMEOUT);
+        // loads issued but never consumed, and MMAs committed but never read
+        const int kt_p = counters[2], kt_m = counters[5];
+        for (int n = kt_m; n < kt_p; ++n) mbar_wait(k_full + n % WS_NSK, (n / WS_NSK) & 1);
+        const int at_m = counters[4], at_e = counters[6];
+        for (int n = at_e; n < at_m; ++n) mbar_wait(acc_full + (n & 1), (n >> 1) & 1);
+        if (at_m > 0) mbar_wait(acc_full + ((at_m - 1) & 1), ((at_m - 1) >> 1) & 1);
+        const int vt_p = counters[3], vt_e = counters[7];
+        for (int n = vt_e; n < vt_p; ++n) mbar_wait(v_full + n % NSV, (n / NSV) & 1);
+        const int q_p = counters[0];
+        if (q_p > 0) mbar_wait(q_full + ((q_p - 1) & 1), ((q_p - 1) >> 1) & 1);
+        const int b_p = counters[1];
+        if (b_p > 0) mbar_wait(b_full, (b_p - 1) & 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ---- merge: one CTA per unit; thread j owns output channel j of every q-head -------------------
+template <int GT>
+__global__ void __launch_bounds__(128) decode_ws_merge_kernel(DecodeArgs a, WsExtra x) {
+    extern __shared__ float msm[];
+    const int G = GT, rV = a.r[1], kV = a.k[1];
+    const int ldb = kV | 1;
+    float *sBV = msm;                                   // [D][ldb]
+    float *sAcc = sBV + D * ldb;                        // [G][rV]
+    const int u = blockIdx.x;
+    const int seq = u / a.H, h = u % a.H;
+    const int j = threadIdx.x;
+    ws_griddep_launch();
+    if (kV > 0) {
+        const float *B = a.basis[1] + (size_t)u * D * rV;
+        for (int o = j; o < D * kV; o += 128) sBV[(o / kV) * ldb + o % kV] = B[(size_t)(o / kV) * rV + o % kV];
+    }
+    ws_griddep_wait();
+    // CTAs whose tile ranges touch this unit, and the unit's segment index in each
+    const long long x0 = (long long)u * x.Tu, x1 = (long long)(u + 1) * x.Tu - 1;
+    const int c_lo = (int)(((x0 + 1) * x.P + x.N - 1) / x.N) - 1;
+    const int c_hi = (int)(((x1 + 1) * x.P + x.N - 1) / x.N) - 1;
+    const size_t stride = (size_t)G * (2 + rV + D);
+    float M[GT], Lw[GT], accw[GT];
+#pragma unroll
+    for (int g = 0; g < GT; ++g) {
+        M[g] = -CUDART_INF_F;
+        Lw[g] = 0.f;
+        accw[g] = 0.f;
+    }
+    for (int c = c_lo; c <= c_hi; ++c) {
+        const long long g0 = (long long)c * x.N / x.P;
+        const int js = (int)(u - g0 / x.Tu);
+        const float *rec = a.ws + ((size_t)c * x.maxseg + js) * stride;
+#pragma unroll
+        for (int g = 0; g < GT; ++g) M[g] = fmaxf(M[g], __ldcg(rec + g * (2 + rV + D)));
+    }
+    float accr[GT];
+#pragma unroll
+    for (int g = 0; g < GT; ++g) accr[g] = 0.f;
+    for (int c = c_lo; c <= c_hi; ++c) {
+        const long long g0 = (long long)c * x.N / x.P;
+        const int js = (int)(u - g0 / x.Tu);
+        const float *rec = a.ws + ((size_t)c * x.maxseg + js) * stride;
+#pragma unroll
+        for (int g = 0; g < GT; ++g) {
+            const float *r = rec + g * (2 + rV + D);
+            const float w = ex2(__ldcg(r) - M[g]);
+            Lw[g] = fmaf(w, __ldcg(r + 1), Lw[g]);
+            if (j < kV) accr[g] = fmaf(w, __ldcg(r + 2 + j), accr[g]);
+            accw[g] = fmaf(w, __ldcg(r + 2 + rV + j), accw[g]);
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < GT; ++g)
+        if (j < kV) sAcc[g * rV + j] = accr[g];
+    __syncthreads();
+    const float *br = sBV + j * ldb;
+#pragma unroll
+    for (int g = 0; g < GT; ++g) {
+        float o = accw[g];
+        for (int c = 0; c < kV; ++c) o = fmaf(sAcc[g * rV + c], br[c], o);
+        a.out[((size_t)seq * a.H * G + (size_t)h * G + g) * D + j] = o / Lw[g];
+    }
+}
+
+size_t ws_partial_floats(int units, int sms, int G, int rV) {
+    return ((size_t)units + 2 * (size_t)sms) * G * (2 + rV + D);
+}
+
+// The register split inside the kernel waits for registers that the launch must have granted:
+// refuse to launch a build whose register count is below WS_REG_LAUNCH.
+template <bool BF, int GT>
+static bool ws_regs_ok() {
+    static int ok = -1;
+    if (ok < 0) {
+        cudaFuncAttributes fa;
+        ok = (cudaFuncGetAttributes(&fa, decode_ws_kernel<BF, GT>) == cudaSuccess &&
+              ((fa.numRegs + 7) & ~7) >= WS_REG_LAUNCH)
+                 ? 1
+                 : 0;
+        if (!ok) cudaGetLastError();
+    }
+    return ok == 1;
+}
+
+template <bool BF, int GT>
+static cudaError_t launch_ws_t(const CUtensorMap *tmC, const CUtensorMap *tmB, const DecodeArgs &a,
+                               const WsExtra &x, cudaStream_t s, size_t smem, size_t msmem) {
+    static size_t attr[64] = {0}, mattr[64] = {0};
+    if (!ws_regs_ok<BF, GT>()) return cudaErrorInvalidConfiguration;
+    cudaError_t e = ensure_smem((const void *)decode_ws_kernel<BF, GT>, smem, attr);
+    if (e != cudaSuccess) return e;
+    e = ensure_smem((const void *)decode_ws_merge_kernel<GT>, msmem, mattr);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr1[1];
+    attr1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr1[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(x.P);
+    cfg.blockDim = dim3(WS_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr1;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_ws_kernel<BF, GT>, *tmC, *tmB, a, x);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(x.UL);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = msmem;
+    return cudaLaunchKernelEx(&cfg, decode_ws_merge_kernel<GT>, a, x);
+}
+
+cudaError_t launch_decode_ws(const CUtensorMap *tmC, const CUtensorMap *tmB, const DecodeArgs &a,
+                             const WsExtra &x, cudaStream_t s) {
+    const int esz = a.kv_dtype == ISKV_BF16 ? 2 : 4;
+    const size_t smem = ws_smem_bytes(x.factor_bf16, a.r[1], esz, a.G);
+    const size_t msmem = ((size_t)D * (a.k[1] | 1) + (size_t)a.G * a.r[1]) * sizeof(float);
+    const bool bf = x.factor_bf16 != 0;
+    switch (a.G) {
+    case 1: return bf ? launch_ws_t<true, 1>(tmC, tmB, a, x, s, smem, msmem)
+                      : launch_ws_t<false, 1>(tmC, tmB, a, x, s, smem, msmem);
+    case 2: return bf ? launch_ws_t<true, 2>(tmC, tmB, a, x, s, smem, msmem)
+                      : launch_ws_t<false, 2>(tmC, tmB, a, x, s, smem, msmem);
+    case 4: return bf ? launch_ws_t<true, 4>(tmC, tmB, a, x, s, smem, msmem)
+                      : launch_ws_t<false, 4>(tmC, tmB, a, x, s, smem, msmem);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace iskv

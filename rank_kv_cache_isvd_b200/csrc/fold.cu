@@ -890,53 +890,114 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
     __syncthreads();
     // ---- new rows' coordinates C[n_c + i] = F[i] B+ --------------------------------------------
     if (a.skip_new_rows) return;
-    float *Cn = P.coords + ((size_t)unit * a.n_max + a.n_c) * r;
+    const size_t cn0 = ((size_t)unit * a.n_max + a.n_c) * r;
     tile_gemm<2, 4>(b, kp, D, [&](int i, int jj) { return sA[i * LDS + jj]; },
                     [&](int jj, int c) { return sBp[c * LDS + jj]; },
-                    [&](int i, int c, float v) { Cn[(size_t)i * r + c] = v; });
+                    [&](int i, int c, float v) { store_coord(P.coords, cn0 + (size_t)i * r + c, v, a.cbf); });
     for (int o = tid; o < b * (r - kp); o += FT)
-        Cn[(size_t)(o / (r - kp)) * r + kp + o % (r - kp)] = 0.f;
+        store_coord(P.coords, cn0 + (size_t)(o / (r - kp)) * r + kp + o % (r - kp), 0.f, a.cbf);
 }
 
 // History rotation: old coordinates move with the basis, C[0:n] <- C[0:n] H[:k] (iS-KV summary,
 // "Block-Incremental Decoding Updates", U+ = diag(U, I_b) G, so the old rows of U+ Sigma+ are
 // U Sigma H[:k]). Stale mode keeps the old coordinates (zero-padded to the new rank).
-constexpr int ROT_ROWS = 64;
-constexpr int ROT_THREADS = 256;
+constexpr int ROT_ROWS = 64;                  // rows per tile
+constexpr int ROT_THREADS = 256;              // 16 row groups (4 rows) x 16 column groups
+constexpr int ROT_XS = ROT_ROWS + 4;          // stride of the transposed row tile
+constexpr int ROT_HS = 128;                   // stride of H_top in shared memory
+constexpr int ROT_GX = 24;                    // CTAs per (unit, path); each takes every 24th tile
 
-__global__ void __launch_bounds__(ROT_THREADS) rotate_kernel(RotArgs a) {
+// One tile: acc[rr][cc] = sum_l X[4 rg + rr][l] H[l][CW cg + cc]; X^T and H in shared memory.
+// Each thread keeps a 4 x CW block of outputs in registers, so every shared-memory load feeds
+// 4 or CW fused multiply-adds.
+template <int CW>
+__device__ __forceinline__ void rot_tile(const float *sXt, const float *sH, int k, int rg, int cg,
+                                         float (&acc)[4][8]) {
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) acc[rr][cc] = 0.f;
+#pragma unroll 4
+    for (int l = 0; l < k; ++l) {
+        const float4 x = *reinterpret_cast<const float4 *>(sXt + l * ROT_XS + 4 * rg);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+        float hv[CW];
+#pragma unroll
+        for (int cc = 0; cc < CW; ++cc) hv[cc] = sH[l * ROT_HS + CW * cg + cc];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+            for (int cc = 0; cc < CW; ++cc) acc[rr][cc] = fmaf(xs[rr], hv[cc], acc[rr][cc]);
+    }
+}
+
+__global__ void __launch_bounds__(ROT_THREADS, 2) rotate_kernel(RotArgs a) {
     extern __shared__ float smem[];
     const RotPath P = (a.path_lo + (int)blockIdx.z) ? a.path[1] : a.path[0];
     const int unit = a.unit0 + blockIdx.y;
-    const long long row0 = (long long)blockIdx.x * ROT_ROWS;
-    if (row0 >= a.n_old) return;
-    const int rows = (int)min((long long)ROT_ROWS, a.n_old - row0);
     const int k = P.k, kp = P.kp, r = P.r;
-    float *sH = smem;                         // k x kp
-    float *sX = sH + r * r;                   // ROT_ROWS x (k + 1)
-    float *C = P.coords + ((size_t)unit * a.n_max + row0) * r;
-    if (!a.stale) {
-        const float *ht = P.htop + (size_t)unit * r * r;
-        for (int o = threadIdx.x; o < k * kp; o += ROT_THREADS) {
-            const int l = o / kp, c = o % kp;
-            sH[l * kp + c] = ht[(size_t)l * r + c];
+    const int tid = threadIdx.x;
+    const long long tiles = (a.n_old + ROT_ROWS - 1) / ROT_ROWS;
+    const size_t cu = (size_t)unit * a.n_max * r;
+    if (a.stale) {
+        // stale coordinates: kept as they are, columns k .. kp - 1 zero
+        for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
+            const long long row0 = t * ROT_ROWS;
+            const int rows = (int)min((long long)ROT_ROWS, a.n_old - row0);
+            for (int o = tid; o < rows * (r - k); o += ROT_THREADS) {
+                const int i = o / (r - k), c = k + o % (r - k);
+                store_coord(P.coords, cu + (size_t)(row0 + i) * r + c, 0.f, a.cbf);
+            }
         }
+        return;
     }
-    for (int o = threadIdx.x; o < rows * k; o += ROT_THREADS) {
-        const int i = o / k, l = o % k;
-        sX[i * (k + 1) + l] = C[(size_t)i * r + l];
+    float *sH = smem;                         // [k][ROT_HS], zero past kp
+    float *sXt = sH + k * ROT_HS;             // [k][ROT_XS]: column l of the row tile
+    const float *ht = P.htop + (size_t)unit * r * r;
+    for (int o = tid; o < k * ROT_HS; o += ROT_THREADS) {
+        const int l = o / ROT_HS, c = o % ROT_HS;
+        sH[o] = c < kp ? ht[(size_t)l * r + c] : 0.f;
     }
-    __syncthreads();
-    for (int o = threadIdx.x; o < rows * r; o += ROT_THREADS) {
-        const int i = o / r, c = o % r;
-        float s = 0.f;
-        if (a.stale) {
-            s = c < k ? sX[i * (k + 1) + c] : 0.f;
-        } else if (c < kp) {
-            const float *x = sX + i * (k + 1);
-            for (int l = 0; l < k; ++l) s = fmaf(x[l], sH[l * kp + c], s);
+    const int rg = tid >> 4, cg = tid & 15;
+    const int cw = (kp + 15) >> 4;            // columns per thread (1 .. 8)
+    for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const long long row0 = t * ROT_ROWS;
+        const int rows = (int)min((long long)ROT_ROWS, a.n_old - row0);
+        __syncthreads();                      // previous tile's reads of sXt are done
+        for (int o = tid; o < ROT_ROWS * k; o += ROT_THREADS) {
+            const int i = o / k, l = o % k;
+            sXt[l * ROT_XS + i] = i < rows ? load_coord(P.coords, cu + (size_t)(row0 + i) * r + l, a.cbf) : 0.f;
         }
-        C[(size_t)i * r + c] = s;
+        __syncthreads();
+        float acc[4][8];
+        switch (cw) {
+            case 1: rot_tile<1>(sXt, sH, k, rg, cg, acc); break;
+            case 2: rot_tile<2>(sXt, sH, k, rg, cg, acc); break;
+            case 3: rot_tile<3>(sXt, sH, k, rg, cg, acc); break;
+            case 4: rot_tile<4>(sXt, sH, k, rg, cg, acc); break;
+            case 5: rot_tile<5>(sXt, sH, k, rg, cg, acc); break;
+            case 6: rot_tile<6>(sXt, sH, k, rg, cg, acc); break;
+            case 7: rot_tile<7>(sXt, sH, k, rg, cg, acc); break;
+            default: rot_tile<8>(sXt, sH, k, rg, cg, acc); break;
+        }
+        // rows 4 rg .. 4 rg + 3, columns cw cg .. ; the columns kp .. r - 1 are cleared by the
+        // column groups past kp (their H columns are zero)
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            const int i = 4 * rg + rr;
+            if (i >= rows) continue;
+            const size_t base = cu + (size_t)(row0 + i) * r;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                const int c = cw * cg + cc;
+                if (cc < cw && c < r) store_coord(P.coords, base + c, acc[rr][cc], a.cbf);
+            }
+        }
+        // columns past 16 cw (only when kp < r and 16 cw < r): zero
+        for (int o = tid; o < rows * r; o += ROT_THREADS) {
+            const int i = o / r, c = o % r;
+            if (c >= 16 * cw) store_coord(P.coords, cu + (size_t)(row0 + i) * r + c, 0.f, a.cbf);
+        }
     }
 }
 
@@ -952,12 +1013,14 @@ cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s) {
 
 cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s) {
     if (a.n_old <= 0 || a.path_hi <= a.path_lo || n_units <= 0) return cudaSuccess;
-    const int rmax = a.path[0].r > a.path[1].r ? a.path[0].r : a.path[1].r;
-    const size_t smem = (size_t)(rmax * rmax + ROT_ROWS * (rmax + 1)) * sizeof(float);
+    int kmax = 0;
+    for (int x = a.path_lo; x < a.path_hi; ++x) kmax = a.path[x].k > kmax ? a.path[x].k : kmax;
+    const size_t smem = (size_t)kmax * (ROT_HS + ROT_XS) * sizeof(float) + 16;
     static size_t attr[64] = {0};
     const cudaError_t e = ensure_smem((const void *)rotate_kernel, smem, attr);
     if (e != cudaSuccess) return e;
-    const unsigned gx = (unsigned)((a.n_old + ROT_ROWS - 1) / ROT_ROWS);
+    const long long tiles = (a.n_old + ROT_ROWS - 1) / ROT_ROWS;
+    const unsigned gx = (unsigned)(tiles < ROT_GX ? tiles : ROT_GX);
     rotate_kernel<<<dim3(gx, n_units, a.path_hi - a.path_lo), ROT_THREADS, smem, s>>>(a);
     return cudaGetLastError();
 }

@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(RF_THREADS) newrows_kernel(NewRowsArgs a) {
                 const float *f = sF + i * (D + 1);
                 for (int j = 0; j < D; ++j) s = fmaf(f[j], sB[j * ldb + c], s);
             }
-            P.coords[((size_t)unit * a.n_max + a.n_c + c0 + s0 + i) * r + c] = s;
+            store_coord(P.coords, ((size_t)unit * a.n_max + a.n_c + c0 + s0 + i) * r + c, s, a.cbf);
         }
     }
 }

@@ -24,7 +24,9 @@ struct iskv_handle {
     long long n_max = 0;  // coordinate rows per unit
     int max_splits = 0;
     size_t esz = 2;
-    float *coords[2] = {nullptr, nullptr};
+    void *coords[2] = {nullptr, nullptr};  // fp32, or bf16 with coord_bf16
+    int cbf = 0;                          // coordinates stored in bf16
+    size_t csz = 4;                       // bytes per stored coordinate
     float *basis[2] = {nullptr, nullptr};   // [NB][U][D][r]
     float *sigma[2] = {nullptr, nullptr};   // [NB][U][r]
     float *htop[2] = {nullptr, nullptr};    // [NB][U][r][r]
@@ -36,6 +38,7 @@ struct iskv_handle {
     int *status = nullptr;
     unsigned long long *stats = nullptr;  // fold statistics (3 counters)
     bool tc = false;                      // tensor-core decode available for this shape
+    bool ws_ok = false;                   // warp-specialised persistent decode for this shape
     CUtensorMap tmC;                      // key coordinates [U * n_max][r_K], 32 x 128 boxes
     CUtensorMap tmB;                      // key bases [NB * U * D][r_K]
     // per layer
@@ -117,17 +120,19 @@ EncodeTiledFn encode_tiled() {
     return fn;
 }
 
-// 2-D fp32 tensor [rows][cols] (row stride cols), boxes of 32 columns x 128 rows, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const float *base, int cols, long long rows) {
+// 2-D tensor [rows][cols] (row stride cols) of fp32 or bf16 elements, boxes of 128 bytes (32 fp32
+// or 64 bf16 columns; columns past `cols` read as zero) x 128 rows, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, int cols, long long rows, bool bf16 = false) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn || rows < 1 || rows > 0x7fffffffLL) return false;
+    const size_t esz = bf16 ? 2 : 4;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(float)};
-    cuuint32_t box[2] = {32, 128};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * esz};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 128};
     cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -204,6 +209,7 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
     fa.kv_dtype = c.kv_dtype;
     fa.status = h->status;
     fa.stats = h->stats;
+    fa.cbf = h->cbf;
     // coordinates of the block's real rows in the new basis (large blocks) or, for frozen paths,
     // in the frozen basis
     NewRowsArgs nr;
@@ -222,6 +228,7 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
     nr.kv_dtype = c.kv_dtype;
     nr.n_c = nc;
     nr.n_max = h->n_max;
+    nr.cbf = h->cbf;
     if (c.block > BMAX) {
         // large block: fold the 128-row triangular factor of the block (same Sigma+, H and basis),
         // then the coordinates of the block's real rows
@@ -320,6 +327,7 @@ int apply_fold(iskv_handle *h, int l0, int nl, cudaStream_t s) {
         ra.n_old = nc;
         ra.n_max = h->n_max;
         ra.stale = c.rotate_history ? 0 : 1;
+        ra.cbf = h->cbf;
         if (launch_rotate(ra, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
         h->launches += 1;
     }
@@ -426,6 +434,8 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         h->G = c.n_q_heads / c.n_kv_heads;
         h->n_max = ncomp(c.max_tokens, c.block, c.window);
         h->esz = c.kv_dtype == ISKV_BF16 ? 2 : 4;
+        h->cbf = c.coord_bf16 ? 1 : 0;
+        h->csz = h->cbf ? 2 : 4;
         const long long ctiles = (h->n_max + DEC_TILE - 1) / DEC_TILE;
         h->max_splits = (int)(ctiles + (h->R + DEC_TILE - 1) / DEC_TILE + 1);
         // folds in flight ahead of their trigger: at most window / block + 1 (look-ahead only)
@@ -457,7 +467,7 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
     for (int x = 0; x < 2; ++x) {
         const size_t r = (size_t)rank_of(h, x);
         const size_t nb = (size_t)h->NB;
-        alloc((void **)&h->coords[x], U * (size_t)h->n_max * r * sizeof(float));
+        alloc((void **)&h->coords[x], U * (size_t)h->n_max * r * h->csz);
         alloc((void **)&h->basis[x], nb * U * D * r * sizeof(float));
         alloc((void **)&h->sigma[x], nb * U * r * sizeof(float));
         alloc(&h->ring[x], U * (size_t)h->R * D * h->esz);
@@ -466,7 +476,12 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
     }
     if (c.rope) alloc((void **)&h->rope_cs, (size_t)c.max_tokens * DH * sizeof(float2));
     if (c.rope) alloc((void **)&h->rope_t, (size_t)c.max_tokens * DH * sizeof(float2));
-    alloc((void **)&h->ws, (size_t)h->UL * h->max_splits * h->G * (2 + D) * sizeof(float));
+    {
+        // split partials: the larger of the split-kernel layout and the persistent decode's
+        const size_t a1 = (size_t)h->UL * h->max_splits * h->G * (2 + D);
+        const size_t a2 = ws_partial_floats(h->UL, h->sms, h->G, c.rank_v);
+        alloc((void **)&h->ws, (a1 > a2 ? a1 : a2) * sizeof(float));
+    }
     alloc((void **)&h->status, sizeof(int));
     alloc((void **)&h->stats, 4 * sizeof(unsigned long long));
     if (ok) {
@@ -499,14 +514,32 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, h->device);
     memset(&h->tmC, 0, sizeof(h->tmC));
     memset(&h->tmB, 0, sizeof(h->tmB));
-    if (major == 10 && c.rank_k % 4 == 0 && c.rank_k <= 64 && c.rank_v % 4 == 0 &&
-        tc_smem_bytes((c.rank_k + 31) / 32, c.rank_v, (int)h->esz, h->G) <= 227 * 1024) {
+    if (h->cbf) {
+        // bf16 coordinates are read by the persistent decode only: one 64-column box of key
+        // coordinates, 16-byte rows of value coordinates
+        bool m_ok = major == 10 && c.rank_k % 8 == 0 && c.rank_k <= 64 && c.rank_v % 8 == 0 &&
+                    (h->G == 1 || h->G == 2 || h->G == 4) &&
+                    ws_smem_bytes(1, c.rank_v, (int)h->esz, h->G) <= 227 * 1024;
+        if (m_ok && h->n_max > 0)
+            m_ok = make_map(&h->tmC, h->coords[0], c.rank_k, (long long)h->U * h->n_max, true);
+        if (!m_ok) {
+            free_all(h);
+            delete h;
+            return ISKV_ERR_UNSUPPORTED;
+        }
+        h->tc = h->ws_ok = true;
+    } else if (major == 10 && c.rank_k % 4 == 0 && c.rank_k <= 64 && c.rank_v % 4 == 0 &&
+               tc_smem_bytes((c.rank_k + 31) / 32, c.rank_v, (int)h->esz, h->G) <= 227 * 1024) {
         bool m_ok = true;
         if (h->n_max > 0) {
             m_ok = make_map(&h->tmC, h->coords[0], c.rank_k, (long long)h->U * h->n_max) &&
                    make_map(&h->tmB, h->basis[0], c.rank_k, (long long)h->NB * h->U * D);
         }
         h->tc = m_ok;
+        // persistent warp-specialised decode: fp32 key coordinates in one 32-column box, GQA
+        // groups of 1, 2 or 4, value rows in 16-byte units
+        h->ws_ok = m_ok && c.rank_k <= 32 && (h->G == 1 || h->G == 2 || h->G == 4) &&
+                   ws_smem_bytes(0, c.rank_v, (int)h->esz, h->G) <= 227 * 1024;
     }
     *out = h;
     return ISKV_OK;
@@ -584,7 +617,7 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
     for (int x = 0; x < 2; ++x) {
         const size_t r = (size_t)rank_of(h, x);
         const size_t u0 = (size_t)layer * h->UL;
-        da.coords[x] = h->coords[x] + u0 * (size_t)h->n_max * r;
+        da.coords[x] = static_cast<const char *>(h->coords[x]) + u0 * (size_t)h->n_max * r * h->csz;
         da.basis[x] = basis_buf(h, x, cur) + u0 * D * r;
         da.ring[x] = static_cast<const char *>(h->ring[x]) + u0 * (size_t)h->R * D * h->esz;
         da.r[x] = (int)r;
@@ -603,6 +636,7 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
     da.new_row[0] = new_k;
     da.new_row[1] = new_v;
     da.new_pos = new_k ? da.t - 1 : -1;
+    da.cbf = h->cbf;
     // compressed splits: at most one wave of CTAs over all units of the layer (two per SM when
     // two fit in shared memory), the compressed tiles of a unit spread evenly over its splits
     const long long ctiles = (da.n_c + DEC_TILE - 1) / DEC_TILE;
@@ -619,6 +653,33 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
     da.max_splits = h->max_splits;
     da.kv_dtype = c.kv_dtype;
     da.scale = 1.0f / sqrtf((float)D);
+    if (h->ws_ok) {
+        if (reinterpret_cast<uintptr_t>(q) % 16 != 0) return ISKV_ERR_INVALID_ARG;
+        WsExtra x;
+        memset(&x, 0, sizeof(x));
+        x.rope_rows = c.max_tokens;
+        x.row0 = (long long)layer * h->UL * h->n_max;
+        x.brow0 = (cur * h->U + layer * h->UL) * D;
+        x.Tc = (int)ctiles;
+        x.Tw = (int)((e + DEC_TILE - 1) / DEC_TILE);
+        x.Tu = x.Tc + x.Tw;
+        x.UL = h->UL;
+        x.N = (long long)h->UL * x.Tu;
+        x.P = (int)(x.N < h->sms ? x.N : h->sms);
+        x.maxseg = h->UL / x.P + 2;
+        x.factor_bf16 = h->cbf;
+        x.status = h->status;
+        if (x.N < 1) return ISKV_ERR_INVALID_ARG;
+        const cudaError_t e = launch_decode_ws(&h->tmC, &h->tmB, da, x, s);
+        if (e == cudaSuccess) {
+            h->launches += 2;
+            return ISKV_OK;
+        }
+        // a build whose register allocation cannot hold the kernel's register split is never
+        // launched: use the split-kernel decode from now on (fp32 coordinates only)
+        if (e != cudaErrorInvalidConfiguration || h->cbf) return ISKV_ERR_CUDA;
+        h->ws_ok = false;
+    }
     if (da.n_split > h->max_splits) return ISKV_ERR_INVALID_ARG;
     if (h->tc) {
         if (reinterpret_cast<uintptr_t>(q) % 16 != 0) return ISKV_ERR_INVALID_ARG;
@@ -684,7 +745,9 @@ int iskv_reconstruct(iskv_handle *h, int layer, int which, int apply_rope, float
     const size_t r = (size_t)rank_of(h, which);
     const size_t u0 = (size_t)layer * h->UL;
     ReconArgs ra;
-    ra.coords = h->coords[which] + u0 * (size_t)h->n_max * r;
+    memset(&ra, 0, sizeof(ra));
+    ra.coords = static_cast<const char *>(h->coords[which]) + u0 * (size_t)h->n_max * r * h->csz;
+    ra.cbf = h->cbf;
     ra.basis = basis_buf(h, which, current_buffer(h, layer)) + u0 * D * r;
     ra.ring = static_cast<const char *>(h->ring[which]) + u0 * (size_t)h->R * D * h->esz;
     ra.rope_cs = h->rope_cs;
@@ -714,10 +777,14 @@ int iskv_get_factors(iskv_handle *h, int layer, int seq, int kv_head, int which,
     const size_t r = (size_t)rank_of(h, which);
     const size_t u = ((size_t)layer * h->cfg.batch + seq) * h->cfg.n_kv_heads + kv_head;
     const long long nc = h->nc[layer];
-    if (coords && nc > 0 &&
-        cudaMemcpyAsync(coords, h->coords[which] + u * (size_t)h->n_max * r,
-                        (size_t)nc * r * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-        return ISKV_ERR_CUDA;
+    if (coords && nc > 0) {
+        const void *src = static_cast<const char *>(h->coords[which]) + u * (size_t)h->n_max * r * h->csz;
+        const cudaError_t e = h->cbf ? launch_coords_to_f32(coords, src, (size_t)nc * r, s)
+                                     : cudaMemcpyAsync(coords, src, (size_t)nc * r * sizeof(float),
+                                                       cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return ISKV_ERR_CUDA;
+        h->launches += h->cbf ? 1 : 0;
+    }
     const int cur = current_buffer(h, layer);
     if (basis && cudaMemcpyAsync(basis, basis_buf(h, which, cur) + u * D * r,
                                  D * r * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
@@ -788,8 +855,9 @@ int iskv_storage_bytes(const iskv_handle *h, int layer, long long *bytes_out) {
     if (!h || !bytes_out || !valid_layer(h, layer)) return ISKV_ERR_INVALID_ARG;
     const long long n = h->nc[layer], e = h->t[layer] - n;
     long long f = 0;
-    for (int x = 0; x < 2; ++x) f += (long long)h->kcur[x][layer] * (n + D + 1);
-    *bytes_out = (long long)h->UL * (4LL * f + (long long)h->esz * D * 2LL * e);
+    for (int x = 0; x < 2; ++x)
+        f += (long long)h->kcur[x][layer] * ((long long)h->csz * n + 4LL * (D + 1));
+    *bytes_out = (long long)h->UL * (f + (long long)h->esz * D * 2LL * e);
     return ISKV_OK;
 }
 

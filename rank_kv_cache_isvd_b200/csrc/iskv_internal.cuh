@@ -27,7 +27,7 @@ struct FoldPath {
     float *basis_out;       // [units][D][r]
     const float *sigma_in;  // [units][r] Sigma before the fold (read when k > 0)
     float *sigma_out;       // [units][r] Sigma after the fold
-    float *coords;          // [units][n_max][r]
+    void *coords;           // [units][n_max][r] fp32, or bf16 when the args' cbf is set
     float *htop;            // [units][r][r]
     int r, k, p, kp;        // rank budget, rank before, residual basis size, rank after
 };
@@ -45,6 +45,7 @@ struct FoldArgs {
     unsigned long long *stats;  // [0] max sweeps, [1] total sweeps, [2] cores solved
     int skip_new_rows;      // 1: leave the new rows' coordinates to newrows_kernel (large blocks)
     int path_lo, path_hi;   // paths folded: path_lo .. path_hi - 1 (0 = keys, 1 = values)
+    int cbf;                // 1: coordinates stored in bf16 (rounded to nearest even)
 };
 
 // ---- large blocks (b > BMAX): triangular factor of the block, then the real rows' coordinates -
@@ -60,7 +61,7 @@ struct RFactorArgs {
 struct NewRowsPath {
     const void *ring;       // [units][R][D] kv dtype
     const float *basis;     // [units][D][r] basis after the fold
-    float *coords;          // [units][n_max][r]
+    void *coords;           // [units][n_max][r] fp32 or bf16
     int r, kp;
 };
 struct NewRowsArgs {
@@ -68,11 +69,12 @@ struct NewRowsArgs {
     int unit0, slot0, R, b, kv_dtype;
     long long n_c, n_max;
     int path_lo, path_hi;   // paths processed: path_lo .. path_hi - 1
+    int cbf;                // 1: coordinates stored in bf16
 };
 
 // ---- history rotation C[0:n] <- C[0:n] H_top (or stale zero-padding) ---------------------------
 struct RotPath {
-    float *coords;          // [units][n_max][r]
+    void *coords;           // [units][n_max][r] fp32 or bf16
     const float *htop;      // [units][r][r]
     int r, k, kp;
 };
@@ -83,6 +85,7 @@ struct RotArgs {
     long long n_max;
     int stale;              // 1: keep old coordinates (zero columns k..kp-1)
     int path_lo, path_hi;   // paths rotated: path_lo .. path_hi - 1
+    int cbf;                // 1: coordinates stored in bf16 (results rounded to nearest even)
 };
 
 // ---- window append ----------------------------------------------------------------------------
@@ -100,7 +103,7 @@ struct AppendArgs {
 
 // ---- decode -------------------------------------------------------------------------------------
 struct DecodeArgs {
-    const float *coords[2]; // [units][n_max][r] (units offset to the layer)
+    const void *coords[2];  // [units][n_max][r] fp32, or bf16 with cbf (units offset to the layer)
     const float *basis[2];  // [units][D][r]
     const void *ring[2];    // [units][R][D]
     const float2 *rope_cs;  // [max_tokens][DH] (cos, sin) or nullptr
@@ -121,11 +124,12 @@ struct DecodeArgs {
     // its K and V come from new_row[] ([units][D] kv dtype) and the kernel stores them in the ring
     const void *new_row[2];
     long long new_pos;      // -1: no fused append
+    int cbf;                // 1: coordinates stored in bf16 (persistent decode only)
 };
 
 // ---- reconstruct ------------------------------------------------------------------------------
 struct ReconArgs {
-    const float *coords;
+    const void *coords;     // fp32, or bf16 with cbf
     const float *basis;
     const void *ring;
     const float2 *rope_cs;
@@ -133,6 +137,7 @@ struct ReconArgs {
     int r, k;
     long long n_c, t, n_max;
     int R, kv_dtype, apply_rope;
+    int cbf;
 };
 
 // extra state of the tensor-core decode kernel
@@ -145,6 +150,20 @@ struct TcExtra {
     int *status;
 };
 
+// extra state of the warp-specialised persistent decode (decode_ws.cu)
+struct WsExtra {
+    long long rope_rows;    // rows of the (cos, sin) table a.rope_cs
+    long long row0;         // first coordinate row of this layer in the coordinate tensor map
+    int brow0;              // first basis row of this layer (current buffer) in the basis map
+    int Tc, Tw, Tu;         // tiles per unit: compressed, window, total
+    long long N;            // tiles of the layer: units * Tu
+    int P;                  // CTAs (one per SM, at most N)
+    int maxseg;             // partial records per CTA (units / P + 2)
+    int UL;                 // units of the layer
+    int factor_bf16;        // 1: coordinates and bases stored in bf16
+    int *status;
+};
+
 cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_rfactor(const RFactorArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_newrows(const NewRowsArgs &a, int n_units, cudaStream_t s);
@@ -152,13 +171,30 @@ cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_append(const AppendArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_reconstruct(const ReconArgs &a, int n_units, cudaStream_t s);
+cudaError_t launch_coords_to_f32(float *dst, const void *src, size_t n, cudaStream_t s);
 cudaError_t launch_rope_table(float2 *table, long long max_tokens, double theta, cudaStream_t s);
 cudaError_t launch_rope_table_t(float4 *table_t, long long max_tokens, double theta,
                                 cudaStream_t s);
 cudaError_t launch_decode_tc(const CUtensorMap *tmC, const CUtensorMap *tmB, const DecodeArgs &a,
                              const TcExtra &x, int n_units, cudaStream_t s);
+cudaError_t launch_decode_ws(const CUtensorMap *tmC, const CUtensorMap *tmB, const DecodeArgs &a,
+                             const WsExtra &x, cudaStream_t s);
+size_t ws_smem_bytes(int bf, int rV, int esz, int G);
+size_t ws_partial_floats(int units, int sms, int G, int rV);
 size_t fold_smem_bytes();
 size_t tc_smem_bytes(int kblocks, int rV, int esz, int G);
+
+// Stored coordinates: fp32, or bf16 rounded to nearest even from the fp32 result.
+__device__ __forceinline__ float load_coord(const void *base, size_t idx, int cbf) {
+    if (cbf) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[idx]);
+    return reinterpret_cast<const float *>(base)[idx];
+}
+__device__ __forceinline__ void store_coord(void *base, size_t idx, float v, int cbf) {
+    if (cbf)
+        reinterpret_cast<__nv_bfloat16 *>(base)[idx] = __float2bfloat16_rn(v);
+    else
+        reinterpret_cast<float *>(base)[idx] = v;
+}
 
 __device__ __forceinline__ float load_row_elem(const void *base, size_t idx, int kv_dtype) {
     if (kv_dtype == ISKV_BF16)

@@ -86,9 +86,9 @@ __global__ void reconstruct_kernel(ReconArgs a) {
         if (pos >= a.t) break;
         float x;
         if (pos < a.n_c) {
-            const float *c = a.coords + ((size_t)unit * a.n_max + pos) * r;
+            const size_t ci = ((size_t)unit * a.n_max + pos) * r;
             float s = 0.f;
-            for (int l = 0; l < k; ++l) s = fmaf(c[l], sB[j * ks + l], s);
+            for (int l = 0; l < k; ++l) s = fmaf(load_coord(a.coords, ci + l, a.cbf), sB[j * ks + l], s);
             x = s;
         } else {
             const int slot = (int)(pos % a.R);
@@ -116,6 +116,24 @@ cudaError_t launch_reconstruct(const ReconArgs &a, int n_units, cudaStream_t s) 
     if (e != cudaSuccess) return e;
     const unsigned gx = (unsigned)((a.t + 63) / 64);
     reconstruct_kernel<<<dim3(gx, n_units), D, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace iskv
+
+namespace iskv {
+
+// bf16 coordinates -> fp32 (the inspection copy of iskv_get_factors).
+__global__ void coords_to_f32_kernel(float *dst, const __nv_bfloat16 *src, size_t n) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x)
+        dst[i] = __bfloat162float(src[i]);
+}
+
+cudaError_t launch_coords_to_f32(float *dst, const void *src, size_t n, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    coords_to_f32_kernel<<<grid, 256, 0, s>>>(dst, static_cast<const __nv_bfloat16 *>(src), n);
     return cudaGetLastError();
 }
 

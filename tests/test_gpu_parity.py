@@ -41,10 +41,11 @@ def make_cache(wl, **kw):
     return IsKVCache(**args)
 
 
-def make_oracle(wl, rotate=True, fixed_basis=False):
+def make_oracle(wl, rotate=True, fixed_basis=False, coord_bf16=False):
     return OracleCache(wl.batch, wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim,
                        wl.rank_k, wl.rank_v, wl.block, wl.window, rope=wl.rope,
-                       rope_theta=wl.rope_theta, rotate=rotate, fixed_basis=fixed_basis)
+                       rope_theta=wl.rope_theta, rotate=rotate, fixed_basis=fixed_basis,
+                       coord_bf16=coord_bf16)
 
 
 def sub(wl, **kw):
@@ -130,6 +131,98 @@ def test_fold_one_step_parity(variant, wl_id):
     assert worst["proj"] <= PROJ_TOL
     assert worst["recon"] <= SIG_TOL
     assert cache.status() == 0
+
+
+@pytest.mark.parametrize("variant,wl_id", [("gapped", 1), ("literal", 1), ("gapped", 3),
+                                            ("gapped", 4)])
+def test_bf16_coordinates_fold_one_step_parity(variant, wl_id):
+    """bf16 coordinates: each GPU fold, started from the GPU's own state, stores the oracle's
+    rounded coordinates (at most one bf16 step apart, equal almost everywhere where the subspace
+    is gapped); Sigma and the basis (fp32) match as in the fp32 mode."""
+    from oracle import round_bf16
+    base = syn.WORKLOADS[wl_id]
+    T = 1100 if wl_id != 4 else 2100
+    wl = sub(base, batch=1, n_layers=1, n_kv_heads=2, n_q_heads=8, tokens=T, prefill=0)
+    kd, kv, vd, vv = workload_arrays(wl, variant=variant)
+    cache = make_cache(wl, coord_bf16=True)
+    t, folds = 0, 0
+    worst = {"sigma": 0.0, "proj": 0.0, "mismatch": 0.0, "steps": 0.0}
+    while True:
+        nc = n_compressed(t, wl.block, wl.window)
+        t_fold = nc + wl.window + wl.block
+        if t_fold > wl.tokens:
+            break
+        before = _snapshot(cache, wl)
+        cache.append(0, to_device(kd[0][:, :, t:t_fold]), to_device(vd[0][:, :, t:t_fold]))
+        t = t_fold
+        after = _snapshot(cache, wl)
+        folds += 1
+        for (s_, h, x), (C0, B0, S0, k0, n0) in before.items():
+            r = wl.rank_k if x == 0 else wl.rank_v
+            F = (kv if x == 0 else vv)[0][s_, h, n0:n0 + wl.block]
+            assert np.array_equal(C0, round_bf16(C0))           # stored values are bf16
+            Cr, Sr, Br, _ = fold_from_coords(C0[:, :k0], S0[:k0], B0[:, :k0], F, r)
+            C1, B1, S1, k1, n1 = after[s_, h, x]
+            assert n1 == n0 + wl.block and k1 == Sr.size
+            worst["sigma"] = max(worst["sigma"], float((np.abs(S1[:k1] - Sr) / Sr).max()))
+            M = np.vstack([C0[:, :k0] @ B0[:, :k0].T, F]) if n0 else F
+            sv = np.linalg.svd(M, compute_uv=False)
+            if k1 < sv.size and (sv[k1 - 1] - sv[k1]) / sv[0] > GAP:
+                worst["proj"] = max(worst["proj"], projector_err(B1[:, :k1], Br))
+                E = round_bf16(Cr)
+                got = C1[:, :k1]
+                step = np.maximum(np.abs(E), np.abs(got)) * 2.0 ** -7 + 1e-30
+                worst["steps"] = max(worst["steps"], float((np.abs(got - E) / step).max()))
+                worst["mismatch"] = max(worst["mismatch"], float(np.mean(got != E)))
+    print(f"\nbf16 coordinates {variant} cfg {wl_id}: {folds} folds, worst {worst}")
+    assert worst["sigma"] <= SIG_TOL and worst["proj"] <= PROJ_TOL
+    assert worst["steps"] <= 1.0 and worst["mismatch"] <= 2e-2
+    assert cache.status() == 0
+
+
+@pytest.mark.parametrize("wl_id,tokens,key_scale", [(1, 4096, 1.0), (1, 4096, 8.0), (3, 1500, 1.0),
+                                                    (4, 2148, 1.0), (2, 1500, 1.0)])
+def test_bf16_coordinates_decode_parity(wl_id, tokens, key_scale):
+    """bf16 coordinates: streamed decode (fused append + decode, look-ahead folds) against the
+    oracle's bf16-coordinate stream at several lengths, on the shapes of the workloads."""
+    base = syn.WORKLOADS[wl_id]
+    wl = sub(base, batch=1, n_layers=1, n_kv_heads=2, n_q_heads=8, tokens=tokens, prefill=0)
+    kd, kv, vd, vv = workload_arrays(wl, key_scale=key_scale)
+    cache = make_cache(wl, coord_bf16=True, lookahead_folds=True)
+    orc = make_oracle(wl, coord_bf16=True)
+    K, V = to_device(kd[0]), to_device(vd[0])
+    n0 = min(tokens - 200, 1000)
+    append_both(cache, orc, 0, kd[0], kv[0], vd[0], vv[0], 0, n0)
+    worst = 0.0
+    for t in range(n0, tokens):
+        q = syn.queries(5000 + t, (1, wl.n_q_heads, 128))
+        out = cache.append_decode(0, K[:, :, t:t + 1].contiguous(), V[:, :, t:t + 1].contiguous(),
+                                  torch.from_numpy(q).cuda())
+        orc.append(0, kv[0][:, :, t:t + 1], vv[0][:, :, t:t + 1])
+        if t % 37 == 0 or t == tokens - 1:
+            worst = max(worst, max_head_rel_err(out.cpu().numpy(), orc.decode(0, q.astype(np.float64))))
+    print(f"\nbf16 coordinates cfg {wl_id} x{key_scale}: worst attention rel err {worst:.3e}")
+    assert worst <= ATTN_TOL
+    for x in (0, 1):
+        rec = cache.reconstruct(0, x).cpu().numpy()[0, 0]
+        u = orc.unit(0, 0, 0, x)
+        assert rel_err(rec[u.n:], u.reconstruct()[u.n:]) == 0.0     # window rows exact
+    assert cache.status() == 0
+
+
+def test_bf16_coordinates_storage_bytes():
+    """The storage count uses 2-byte coordinates and fp32 bases and Sigma."""
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=900)
+    kd, kv, vd, vv = workload_arrays(wl)
+    a, b = make_cache(wl), make_cache(wl, coord_bf16=True)
+    orc = make_oracle(wl, coord_bf16=True)
+    for c in (a, b):
+        c.append(0, to_device(kd[0]), to_device(vd[0]))
+    orc.append(0, kv[0], vv[0])
+    expect = sum(orc.unit(0, 0, h, x).storage_bytes(2) for h in range(2) for x in (0, 1))
+    assert b.storage_bytes(0) == expect
+    n = orc.unit(0, 0, 0, 0).n
+    assert a.storage_bytes(0) - b.storage_bytes(0) == 2 * 2 * n * (wl.rank_k + wl.rank_v)
 
 
 # ------------------------------------------------------------------------------------------------
@@ -409,14 +502,15 @@ def test_lookahead_stream_captures_into_a_graph():
     assert cache.status(s) == 0
 
 
-def test_long_context_layer_sampled_units():
+@pytest.mark.parametrize("cbf", [False, True])
+def test_long_context_layer_sampled_units(cbf):
     """Full-size Qwen3-8B-shaped layer as the benchmark's long-context decode runs it (batch 8 x
     8 kv-heads, 32 q-heads, b=128, w=256, r_K=32, r_V=64, 32768 tokens in one append, rows drawn
     on the GPU): every output is finite and the q-heads of three sampled (sequence, kv-head)
     units match the oracle run on those units' rows alone."""
     wl = syn.WORKLOADS[3]
     S, H, T, QH, G = wl.batch, wl.n_kv_heads, wl.tokens, wl.n_q_heads, wl.group
-    cache = make_cache(sub(wl, n_layers=1))
+    cache = make_cache(sub(wl, n_layers=1), coord_bf16=cbf)
     K = torch.empty((S, H, T, 128), dtype=torch.bfloat16, device="cuda")
     V = torch.empty_like(K)
     for sq in range(S):
@@ -432,7 +526,7 @@ def test_long_context_layer_sampled_units():
     assert cache.tokens(0) == T
     units = []
     for sq, h in ((0, 0), (3, 5), (7, 7)):
-        err, (orc,) = _sampled_unit_check(wl, q, out, [(sq, h, K[sq, h], V[sq, h])])
+        err, (orc,) = _sampled_unit_check(wl, q, out, [(sq, h, K[sq, h], V[sq, h])], cbf)
         print(f"\nunit (seq {sq}, kv-head {h}): attention rel err {err:.3e}")
         assert err <= ATTN_TOL
         units.append((sq, h, K[sq, h], V[sq, h], orc))
@@ -443,8 +537,9 @@ def test_long_context_layer_sampled_units():
     cache.close()
 
 
-@pytest.mark.parametrize("lookahead,window", [(False, 256), (True, 256), (False, 0)])
-def test_fused_append_decode_equals_separate_calls(lookahead, window):
+@pytest.mark.parametrize("lookahead,window,cbf", [(False, 256, False), (True, 256, False),
+                                                  (False, 0, False), (True, 256, True)])
+def test_fused_append_decode_equals_separate_calls(lookahead, window, cbf):
     """iskv_append_decode (the decode kernel reads the new rows itself and stores them in the
     ring) gives bit-for-bit the outputs, factors and reconstructions of iskv_append_block +
     iskv_decode_attn, across fold triggers; with window 0 it falls back to the two calls."""
@@ -454,7 +549,7 @@ def test_fused_append_decode_equals_separate_calls(lookahead, window):
     Q = torch.from_numpy(syn.queries(31, (wl.tokens, 1, 8, 128))).cuda()
     outs = []
     for fused in (False, True):
-        cache = make_cache(wl, lookahead_folds=lookahead)
+        cache = make_cache(wl, lookahead_folds=lookahead, coord_bf16=cbf)
         out = torch.empty_like(Q)
         for t in range(wl.tokens):
             kr = K[:, :, t:t + 1].contiguous()
@@ -555,23 +650,23 @@ def test_large_blocks_fold_through_their_triangular_factor(variant):
     assert cache.status() == 0
 
 
-def _unit_oracle(wl, K, V):
+def _unit_oracle(wl, K, V, cbf=False):
     """Float64 oracle of one (sequence, kv-head) unit fed the unit's rows as they are on the device
     (bf16 values, exact in float64)."""
     orc = OracleCache(1, 1, 1, wl.group, 128, wl.rank_k, wl.rank_v, wl.block, wl.window,
-                      rope=True, rope_theta=wl.rope_theta)
+                      rope=True, rope_theta=wl.rope_theta, coord_bf16=cbf)
     orc.append(0, K.float().cpu().numpy().astype(np.float64)[None, None],
                V.float().cpu().numpy().astype(np.float64)[None, None])
     return orc
 
 
-def _sampled_unit_check(wl, q, out, units):
+def _sampled_unit_check(wl, q, out, units, cbf=False):
     """Oracle run on single (sequence, kv-head) units of a full-size cache, compared on their
     q-heads. Returns (worst error, the units' oracles)."""
     G = wl.group
     worst, oracles = 0.0, []
     for sq, h, K, V in units:
-        orc = _unit_oracle(wl, K, V)
+        orc = _unit_oracle(wl, K, V, cbf)
         qs = q[sq, h * G:(h + 1) * G].cpu().numpy().astype(np.float64)[None]
         err = max_head_rel_err(out[sq, h * G:(h + 1) * G].cpu().numpy()[None], orc.decode(0, qs))
         worst = max(worst, err)
@@ -664,13 +759,14 @@ def test_32_layer_workload_full_size_sampled_units():
     cache.close()
 
 
-def test_long_prefill_full_size_sampled_unit():
+@pytest.mark.parametrize("cbf", [False, True])
+def test_long_prefill_full_size_sampled_unit(cbf):
     """The long-context layer at its full prefill (batch 4 x 8 kv-heads, 65536 rows in one
     append, b = 512, w = 512, r_K = 64, r_V = 96): one sampled unit of the decode matches the
     oracle run on its rows alone."""
     wl = syn.WORKLOADS[4]
     S, H, T0 = wl.batch, wl.n_kv_heads, wl.prefill
-    cache = make_cache(sub(wl, n_layers=1))
+    cache = make_cache(sub(wl, n_layers=1), coord_bf16=cbf)
     K = torch.empty((S, H, T0, 128), dtype=torch.bfloat16, device="cuda")
     V = torch.empty_like(K)
     for sq in range(S):
@@ -683,7 +779,7 @@ def test_long_prefill_full_size_sampled_unit():
     q = torch.randn((S, wl.n_q_heads, 128), generator=gen, device="cuda")
     out = cache.decode(0, q)
     assert cache.status() == 0 and bool(torch.isfinite(out).all())
-    err, (orc,) = _sampled_unit_check(wl, q, out, [(2, 5, K[2, 5], V[2, 5])])
+    err, (orc,) = _sampled_unit_check(wl, q, out, [(2, 5, K[2, 5], V[2, 5])], cbf)
     # sharp attention on compressed rows past 60K (n_c = 65024) and on a window row
     sa, sb = _sharp_checks(cache, wl, 0, [(2, 5, K[2, 5], V[2, 5], orc)],
                            [60001, 62500, 64999, 65300], 4343)
