@@ -42,6 +42,14 @@ Readings taken where the page is silent (each also stated at its definition):
   bf16 (nearest even, through float32, as a kernel rounding its fp32 results) after every fold,
   and the next fold starts from the rounded values; ``B`` and ``Sigma`` stay unrounded, because
   the update's core assumes an orthonormal ``B``;
+* prefill with protection (section "Prefill Compression", steps 1-3): over the prefill rows that
+  the window does not hold, keys are cut into chunks of ``chunk`` consecutive positions; chunk
+  ``c`` scores ``min_{i in c} cos(k_i^rot, mean_c k^rot)`` (keys rotated at their positions; a
+  zero vector's cosine counts as 1); the ``m`` lowest-scoring chunks (ties by chunk index) plus
+  the last ``suffix`` prefill positions are the protected key positions ``P_K``; ``P_V`` is every
+  position within ``rho`` of ``P_K``. Protected rows stay exact for good; the remaining rows of the
+  prefill (outside the window) get one truncated SVD; later blocks fold from the window as usual.
+  Compressed rows keep their positions (the index map ``C_X`` of "Reconstruction and Storage");
 * the "fixed basis" variant (``fixed_basis=True``, section "Ablation Study": bases kept fixed)
   runs the regular update for the first ``ceil(min(r, d) / block)`` blocks, which fill the rank
   budget, and then freezes ``B`` and ``Sigma``: every later block is stored as its coordinates
@@ -68,6 +76,9 @@ __all__ = [
     "rope",
     "attention",
     "round_bf16",
+    "chunk_scores",
+    "protected_positions",
+    "value_protected",
 ]
 
 
@@ -202,11 +213,14 @@ class OracleUnit:
         self.U = np.zeros((0, 0))
         self.sigma = np.zeros(0)
         self.B = np.zeros((d, 0))
-        self.C_stale = np.zeros((0, 0))      # stored coordinates (stale or fixed-basis modes)
+        self.C_stale = np.zeros((0, 0))      # stored coordinates C (U Sigma, or as the mode keeps them)
         self._exact: list[np.ndarray] = []
         self.t = 0
         self.n = 0
         self.folds = 0
+        self.comp_pos = np.zeros(0, dtype=np.int64)   # position of each compressed row
+        self.prot_pos = np.zeros(0, dtype=np.int64)   # protected positions (exact for good)
+        self.prot_rows = np.zeros((0, d))
 
     # -- state ---------------------------------------------------------------------------------
     @property
@@ -218,25 +232,48 @@ class OracleUnit:
         return np.asarray(self._exact, dtype=np.float64).reshape(len(self._exact), self.d)
 
     def coords(self) -> np.ndarray:
-        """Stored history coordinates ``U Sigma`` (``n x k``)."""
-        if not self.rotate or self.fixed_basis or self.coord_bf16:
-            return self.C_stale
-        return self.U * self.sigma
+        """Stored history coordinates ``U Sigma`` (``n x k``; unrotated in the stale mode)."""
+        return self.C_stale
 
     def storage_scalars(self) -> int:
         """Persistent scalars of this path: ``k (n + d + 1)`` factors plus ``d e`` exact values.
 
         iS-KV summary, section "Reconstruction and Storage" (storage formula, per path).
         """
-        return self.k * (self.n + self.d + 1) + self.d * len(self._exact)
+        return self.k * (self.n + self.d + 1) + self.d * (len(self._exact) + self.prot_pos.size)
 
     def storage_bytes(self, beta_e: int) -> int:
         """Persistent bytes of this path: the storage formula with bf16 (2 bytes) or fp32 (4 bytes)
         coordinates, fp32 basis and Sigma, and ``beta_e`` bytes per exact scalar."""
         beta_c = 2 if self.coord_bf16 else 4
-        return beta_c * self.k * self.n + 4 * self.k * (self.d + 1) + beta_e * self.d * len(self._exact)
+        return (beta_c * self.k * self.n + 4 * self.k * (self.d + 1)
+                + beta_e * self.d * (len(self._exact) + self.prot_pos.size))
 
     # -- updates -------------------------------------------------------------------------------
+    def prefill(self, X: np.ndarray, protected) -> None:
+        """Prefill of an empty unit ("Prefill Compression", step 3): rows ``X`` take positions
+        ``0 .. T0-1``; the last ``window`` of them form the exact window, ``protected`` positions
+        before it stay exact for good, and the remaining rows get one truncated SVD."""
+        if self.t:
+            raise ValueError("prefill needs an empty unit")
+        X = np.asarray(X, dtype=np.float64)
+        T0 = X.shape[0]
+        end = max(0, T0 - self.window)
+        prot = np.asarray(sorted(set(np.asarray(protected).tolist()) & set(range(end))),
+                          dtype=np.int64)
+        comp = np.asarray(sorted(set(range(end)) - set(prot.tolist())), dtype=np.int64)
+        self.prot_pos, self.prot_rows = prot, X[prot]
+        self.comp_pos = comp
+        if comp.size:
+            U, s, B = svd_r(X[comp], self.rank)
+            self.U, self.sigma, self.B = U, s, B
+            rnd = round_bf16 if self.coord_bf16 else (lambda x: x)
+            self.C_stale = rnd(U * s)
+            self.n = comp.size
+            self.folds = 1                      # the initial factorisation counts as an update
+        self._exact = [row.copy() for row in X[end:]]
+        self.t = T0
+
     def append(self, rows: np.ndarray) -> int:
         """Append rows one by one; fold the oldest ``block`` exact rows whenever the window holds
         ``window + block`` rows. Returns the number of folds done."""
@@ -246,8 +283,10 @@ class OracleUnit:
             self.t += 1
             while len(self._exact) >= self.window + self.block:
                 F = np.asarray(self._exact[: self.block])
+                p0 = self.t - len(self._exact)          # position of the oldest window row
                 del self._exact[: self.block]
                 self._fold(F)
+                self.comp_pos = np.concatenate([self.comp_pos, np.arange(p0, p0 + self.block)])
                 done += 1
         return done
 
@@ -278,10 +317,10 @@ class OracleUnit:
             self.folds += 1
             return
         U_new, s, B_new, H, _ = fold(self.U, self.sigma, self.B, F, self.rank)
-        if self.fixed_basis:
-            # still adapting: coordinates rotate with the basis, as in the regular update
+        if self.rotate:
+            # the regular update (also while a fixed basis is still adapting): C+ = U+ Sigma+
             self.C_stale = U_new * s
-        elif not self.rotate:
+        else:
             kp = s.size
             C = np.zeros((self.n, kp))
             m = min(k_old, kp)
@@ -293,9 +332,15 @@ class OracleUnit:
 
     # -- reading -------------------------------------------------------------------------------
     def reconstruct(self) -> np.ndarray:
-        """``X~``: compressed rows ``(U Sigma B^T)[i]`` for ``i < n``, exact rows after."""
-        hist = self.coords() @ self.B.T if self.n else np.zeros((0, self.d))
-        return np.vstack([hist, self.exact])
+        """``X~`` in position order ("Reconstruction and Storage"): the compressed row ``j`` at
+        position ``C_X[j]`` is ``(U Sigma B^T)[j]``, protected and window rows are exact."""
+        out = np.zeros((self.t, self.d))
+        if self.n:
+            out[self.comp_pos] = self.coords() @ self.B.T
+        out[self.prot_pos] = self.prot_rows
+        e = len(self._exact)
+        out[self.t - e:] = self.exact
+        return out
 
 
 # ----------------------------------------------------------------------------------------------
@@ -323,6 +368,53 @@ def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
     return p @ np.asarray(V, dtype=np.float64)
 
 
+# ----------------------------------------------------------------------------------------------
+# Prefill Compression (protection of outlier keys and their value neighbourhoods)
+# ----------------------------------------------------------------------------------------------
+def chunk_scores(K_rot: np.ndarray, chunk: int) -> np.ndarray:
+    """Step 1 score of every chunk of ``chunk`` consecutive rows (the last one may be shorter):
+    the smallest cosine between a rotated key of the chunk and the chunk's mean rotated key."""
+    K_rot = np.asarray(K_rot, dtype=np.float64)
+    out = []
+    for c0 in range(0, K_rot.shape[0], chunk):
+        blk = K_rot[c0:c0 + chunk]
+        mean = blk.mean(axis=0)
+        nm = np.linalg.norm(mean)
+        nr = np.linalg.norm(blk, axis=1)
+        cos = np.ones(blk.shape[0])
+        ok = (nr > 0) & (nm > 0)
+        cos[ok] = (blk[ok] @ mean) / (nr[ok] * nm)
+        out.append(cos.min())
+    return np.asarray(out)
+
+
+def protected_positions(K: np.ndarray, positions: np.ndarray, chunk: int, m: int, suffix: int,
+                        rope_theta: float | None) -> np.ndarray:
+    """Step 1: protected key positions ``P_K`` (sorted) among the rows ``K`` at ``positions``
+    (consecutive): the ``m`` lowest-scoring chunks plus the last ``suffix`` positions. Keys are
+    rotated at their positions first when ``rope_theta`` is given."""
+    positions = np.asarray(positions)
+    if K.shape[0] == 0:
+        return np.zeros(0, dtype=np.int64)
+    K_rot = rope(K, positions, rope_theta) if rope_theta is not None else np.asarray(K, float)
+    sc = chunk_scores(K_rot, chunk)
+    order = np.argsort(sc, kind="stable")[:min(m, sc.size)]
+    prot = set()
+    for c in order:
+        prot.update(positions[c * chunk:(c + 1) * chunk].tolist())
+    if suffix > 0:
+        prot.update(positions[-suffix:].tolist())
+    return np.asarray(sorted(prot), dtype=np.int64)
+
+
+def value_protected(P_K: np.ndarray, rho: int, lo: int, hi: int) -> np.ndarray:
+    """Step 2: every position in ``[lo, hi)`` within ``rho`` tokens of a position of ``P_K``."""
+    out = set()
+    for p in np.asarray(P_K).tolist():
+        out.update(range(max(lo, p - rho), min(hi, p + rho + 1)))
+    return np.asarray(sorted(out), dtype=np.int64)
+
+
 class OracleCache:
     """All units of a cache: ``[layer][sequence][kv-head]`` for the K and V paths."""
 
@@ -342,6 +434,22 @@ class OracleCache:
 
     def tokens(self, layer: int) -> int:
         return self.units[layer][0][0][0].t
+
+    def prefill(self, layer: int, K: np.ndarray, V: np.ndarray, chunk: int, m: int, suffix: int,
+                rho: int) -> None:
+        """Prefill with protection ("Prefill Compression"): ``K``, ``V``: ``[batch][n_kv][T0][d]``
+        (pre-RoPE keys) of an empty layer. Per kv-head, ``P_K`` from the rotated keys of the rows
+        outside the window, ``P_V`` within ``rho`` of ``P_K``; then each unit's prefill."""
+        T0 = K.shape[2]
+        end = max(0, T0 - self.units[layer][0][0][0].window)
+        pos = np.arange(end)
+        for s in range(self.batch):
+            for h in range(self.n_kv):
+                PK = protected_positions(K[s, h, :end], pos, chunk, m, suffix,
+                                         self.theta if self.rope else None)
+                PV = value_protected(PK, rho, 0, end)
+                self.units[layer][s][h][0].prefill(K[s, h], PK)
+                self.units[layer][s][h][1].prefill(V[s, h], PV)
 
     def append(self, layer: int, K: np.ndarray, V: np.ndarray) -> None:
         """``K``, ``V``: ``[batch][n_kv][m][d]`` rows (pre-RoPE keys)."""

@@ -138,8 +138,32 @@ def _pin_bf16_coordinates(m):
     return True
 
 
+def _pin_prefill(m):
+    """Prefill protection: a planted reversed key protects its chunk; the value neighbourhood
+    is the brute-force dilation; the initial factorisation is the library SVD of the rows left."""
+    d, chunk = 8, 4
+    rng = np.random.default_rng(2)
+    base = rng.standard_normal(d)
+    K = np.tile(base, (40, 1)) + 1e-3 * rng.standard_normal((40, d))
+    K[13] = -base
+    if m.protected_positions(K, np.arange(40), chunk, 1, 0, None).tolist() != [12, 13, 14, 15]:
+        return False
+    PK = np.array([0, 5, 17])
+    if m.value_protected(PK, 2, 0, 30).tolist() != [i for i in range(30)
+                                                     if any(abs(i - p) <= 2 for p in PK)]:
+        return False
+    X = _stream(40, d, 9)
+    unit = m.OracleUnit(d, 3, 4, 5)
+    unit.prefill(X, [1, 2, 9])
+    comp = [i for i in range(35) if i not in (1, 2, 9)]
+    u, sv, vt = np.linalg.svd(X[comp], full_matrices=False)
+    rec = unit.reconstruct()
+    return (np.allclose(rec[comp], (u[:, :3] * sv[:3]) @ vt[:3], atol=1e-10)
+            and np.array_equal(rec[[1, 2, 9]], X[[1, 2, 9]]))
+
+
 PINS = [_pin_stacked_svd, _pin_no_truncation, _pin_rope, _pin_attention, _pin_schedule,
-        _pin_stale_two_folds, _pin_fixed_basis, _pin_bf16_coordinates]
+        _pin_stale_two_folds, _pin_fixed_basis, _pin_bf16_coordinates, _pin_prefill]
 
 MUTANTS = {
     "new-row identity block negated": ("Ublk[n:, k:] = np.eye(b)", "Ublk[n:, k:] = -np.eye(b)"),
@@ -167,6 +191,13 @@ MUTANTS = {
                                           "self.folds > self.adapt_folds"),
     "bf16: rotated coordinates left unrounded": ("                self.C_stale = rnd(C_new)",
                                                  "                self.C_stale = C_new"),
+    "prefill: chunk score takes the largest cosine": ("        out.append(cos.min())",
+                                                       "        out.append(cos.max())"),
+    "prefill: value neighbourhood one short": ("range(max(lo, p - rho), min(hi, p + rho + 1))",
+                                               "range(max(lo, p - rho), min(hi, p + rho))"),
+    "prefill: protected rows factorised too": (
+        "comp = np.asarray(sorted(set(range(end)) - set(prot.tolist())), dtype=np.int64)",
+        "comp = np.asarray(sorted(set(range(end))), dtype=np.int64)"),
     "bf16: rounding to 7 significant bits": ("u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16\n    return (u.astype(np.uint32) << 16)",
                                              "u = (u + 0xFFFF + ((u >> 17) & 1)) >> 17\n    return (u.astype(np.uint32) << 17)"),
 }
