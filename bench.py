@@ -78,7 +78,7 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true", help="headline line only")
-    p.add_argument("--coords", choices=["bf16", "f32"], default="bf16",
+    p.add_argument("--coords", choices=["bf16", "f32"], default="f32",
                    help="storage of the coordinates C = U Sigma (bases and Sigma stay fp32)")
     p.add_argument("--profile-case", choices=["short", "long", "prefill"], nargs="?",
                    const="short",
@@ -707,6 +707,7 @@ def long_prefill(args, dev, flush, calls: int = 5):
         if i >= args.warmup:
             ms.append(e0.elapsed_time(e1))
     assert cache.status(sh) == 0 and bool(torch.isfinite(out).all())
+    stored = cache.storage_bytes(0)
     cache.close()
     hbm, _ = peaks()
     folds = wl.n_c(T0) // wl.block
@@ -717,6 +718,7 @@ def long_prefill(args, dev, flush, calls: int = 5):
             "prefill_ms": pre_ms, "head_block_updates": folds * S * H * 2,
             "head_block_updates_per_s": folds * S * H * 2 / (pre_ms / 1e3),
             "prefill_tflops": fold_flops(wl, T0, units=S * H) / (pre_ms / 1e3) / 1e12,
+            "storage_bytes": stored, "compression_vs_bf16_cache": S * H * 2 * T0 * D * 2 / stored,
             "decode_us": dec_us, "decode_bytes": nbytes,
             "decode_achieved_gbs": nbytes / (dec_us / 1e6) / 1e9,
             "decode_frac_of_hbm": nbytes / (dec_us / 1e6) / 1e9 / hbm}
@@ -755,11 +757,13 @@ def layer_decode(args, dev, flush, coords: str, calls: int = 10):
         if i >= args.warmup:
             ms.append(e0.elapsed_time(e1))
     assert cache.status(sh) == 0 and bool(torch.isfinite(out).all())
+    stored = cache.storage_bytes(0)
     cache.close()
     hbm, _ = peaks()
     us = 1e3 * float(np.median(ms))
     nbytes = decode_bytes(T, wl, csz=2 if coords == "bf16" else 4)
     return {"coords": coords, "launch_us": us, "bytes": nbytes,
+            "storage_bytes": stored, "compression_vs_bf16_cache": S * H * 2 * T * D * 2 / stored,
             "achieved_gbs": nbytes / (us / 1e6) / 1e9, "frac": nbytes / (us / 1e6) / 1e9 / hbm,
             "frac_of_nominal": nbytes / (us / 1e6) / 1e9 / HBM_NOMINAL_GBS}
 

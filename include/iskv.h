@@ -90,7 +90,19 @@ typedef struct {
                           /*    Sigma stay fp32 ("Reconstruction and Storage": beta_f = 2 for C). */
                           /*    Needs rank_k <= 64, rank_k and rank_v multiples of 8 and a GQA   */
                           /*    group of 1, 2 or 4 (else ISKV_ERR_UNSUPPORTED). 0: fp32.         */
+    int prot_cap;         /* 0: iskv_prefill() is not available. >= 1: it is, and the protected */
+                          /*    stores hold up to prot_cap exact rows per unit and path        */
+                          /*    ("Prefill Compression"; more set ISKV_ERR_CAPACITY, sticky).   */
 } iskv_config;
+
+/* Key/value protection of iskv_prefill() ("Prefill Compression", steps 1-2). */
+typedef struct {
+    int chunk;            /* positions per key chunk (>= 1)                                   */
+    int m;                /* outlier chunks protected per kv-head: the m lowest min-cosine     */
+                          /*    scores (ties by chunk index) (>= 0)                            */
+    int suffix;           /* positions just before the window that are protected too (>= 0)   */
+    int rho;              /* value protection radius: P_V = positions within rho of P_K (>= 0) */
+} iskv_protect;
 
 /*
  * Creates a cache for `cfg` on the current CUDA device. Allocates every device buffer
@@ -121,6 +133,25 @@ int iskv_destroy(iskv_handle *h);
  */
 int iskv_append_block(iskv_handle *h, int layer, const void *k_rows_dev, const void *v_rows_dev,
                       int m, iskv_stream_t stream);
+
+/*
+ * Prefill of an empty layer with T0 rows per (sequence, kv-head) ("Prefill Compression"): the
+ * last `window` rows form the exact window; of the rows before it, the protected positions (keys:
+ * P_K of step 1; values: P_V of step 2; none when protect is NULL) stay exact for good and the
+ * others are factorised by one truncated SVD of rank r (step 3), computed from the rows'
+ * triangular factor (Householder QR over 128-row chunks) and a one-sided Jacobi SVD of it; the
+ * coordinates of protected positions are zero and decode reads their exact rows. Later appends
+ * fold blocks from the window as usual. Chunk scores use keys rotated at their positions.
+ *   k_rows_dev, v_rows_dev: kv_dtype [batch][n_kv_heads][T0][head_dim] (keys pre-RoPE).
+ *   protect: host pointer or NULL.
+ * Synchronises `stream` when protect is given (the largest protected count sizes the decode's
+ * protected tiles). Needs cfg.prot_cap >= 1 (else ISKV_ERR_UNSUPPORTED); protection also needs
+ * the persistent decode (coordinates in one 32-column box for fp32, G of 1, 2 or 4).
+ * Errors: ISKV_ERR_INVALID_ARG (layer not empty, bad protect values, T0 < 1),
+ *         ISKV_ERR_CAPACITY (T0 > max_tokens), ISKV_ERR_UNSUPPORTED, ISKV_ERR_CUDA.
+ */
+int iskv_prefill(iskv_handle *h, int layer, const void *k_rows_dev, const void *v_rows_dev,
+                 long long T0, const iskv_protect *protect, iskv_stream_t stream);
 
 /*
  * Decode attention of `layer` over all t cached positions 0 .. t-1: compressed rows are

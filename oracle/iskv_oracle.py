@@ -46,7 +46,8 @@ Readings taken where the page is silent (each also stated at its definition):
   the window does not hold, keys are cut into chunks of ``chunk`` consecutive positions; chunk
   ``c`` scores ``min_{i in c} cos(k_i^rot, mean_c k^rot)`` (keys rotated at their positions; a
   zero vector's cosine counts as 1); the ``m`` lowest-scoring chunks (ties by chunk index) plus
-  the last ``suffix`` prefill positions are the protected key positions ``P_K``; ``P_V`` is every
+  the ``suffix`` positions just before the window (the local suffix of the rows that would be
+  compressed) are the protected key positions ``P_K``; ``P_V`` is every
   position within ``rho`` of ``P_K``. Protected rows stay exact for good; the remaining rows of the
   prefill (outside the window) get one truncated SVD; later blocks fold from the window as usual.
   Compressed rows keep their positions (the index map ``C_X`` of "Reconstruction and Storage");

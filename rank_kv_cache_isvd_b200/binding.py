@@ -22,6 +22,7 @@ __all__ = [
     "iskv_sync_status", "iskv_strerror", "iskv_reset", "iskv_launch_count", "iskv_fold_stats",
     "iskv_join", "iskv_append_decode",
     "iskv_decode_view", "iskv_decode_attn_noalloc", "ISKV_NOALLOC_SCRATCH_FLOATS",
+    "iskv_protect", "iskv_prefill",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libiskv.so")
@@ -57,6 +58,17 @@ class iskv_config(ctypes.Structure):
         ("lookahead_folds", ctypes.c_int),
         ("fixed_basis", ctypes.c_int),
         ("coord_bf16", ctypes.c_int),
+        ("prot_cap", ctypes.c_int),
+    ]
+
+
+class iskv_protect(ctypes.Structure):
+    """Key/value protection of iskv_prefill (mirrors the C struct)."""
+    _fields_ = [
+        ("chunk", ctypes.c_int),
+        ("m", ctypes.c_int),
+        ("suffix", ctypes.c_int),
+        ("rho", ctypes.c_int),
     ]
 
 
@@ -120,6 +132,7 @@ _SIGNATURES = {
     "iskv_fold_stats": (_i, [_vp, _vp, ctypes.POINTER(_i), ctypes.POINTER(_ll),
                              ctypes.POINTER(_ll)]),
     "iskv_decode_attn_noalloc": (_i, [ctypes.POINTER(iskv_decode_view), _vp, _vp, _vp]),
+    "iskv_prefill": (_i, [_vp, _i, _vp, _vp, _ll, ctypes.POINTER(iskv_protect), _vp]),
 }
 
 
@@ -258,3 +271,9 @@ def iskv_join(handle, stream=None) -> int:
 
 def iskv_sync_status(handle, stream=None) -> int:
     return lib.iskv_sync_status(handle, _stream(stream))
+
+
+def iskv_prefill(handle, layer: int, k_rows, v_rows, T0: int, protect=None, stream=None) -> int:
+    """``protect``: an :class:`iskv_protect` or ``None`` (no protection)."""
+    return lib.iskv_prefill(handle, layer, _ptr(k_rows), _ptr(v_rows), T0,
+                            None if protect is None else ctypes.byref(protect), _stream(stream))

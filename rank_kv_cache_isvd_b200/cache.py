@@ -19,12 +19,12 @@ class IsKVCache:
                  kv_dtype: str = "bf16", rope: bool = True, rope_theta: float = 5e5,
                  rotate_history: bool = True, head_dim: int = 128,
                  lookahead_folds: bool = False, fixed_basis: bool = False,
-                 coord_bf16: bool = False):
+                 coord_bf16: bool = False, prot_cap: int = 0):
         self.cfg = iskv_config(batch, n_layers, n_kv_heads, n_q_heads, head_dim, rank_k, rank_v,
                                block, window, max_tokens,
                                ISKV_BF16 if kv_dtype == "bf16" else ISKV_F32, int(rope),
                                float(rope_theta), int(rotate_history), int(lookahead_folds),
-                               int(fixed_basis), int(coord_bf16))
+                               int(fixed_basis), int(coord_bf16), int(prot_cap))
         self.dtype = torch.bfloat16 if kv_dtype == "bf16" else torch.float32
         self.handle = 0
         code, h = iskv_create(self.cfg)
@@ -51,6 +51,16 @@ class IsKVCache:
         assert k_rows.is_contiguous() and v_rows.is_contiguous()
         check(iskv_append_block(self.handle, layer, k_rows, v_rows, k_rows.shape[-2], stream),
               "iskv_append_block")
+
+    def prefill(self, layer: int, k_rows: torch.Tensor, v_rows: torch.Tensor, protect=None,
+                stream=None) -> None:
+        """Prefill of an empty layer (``[batch][n_kv][T0][d]`` rows): exact window, protected
+        rows, truncated SVD of the rest. ``protect``: ``(chunk, m, suffix, rho)`` or ``None``."""
+        from .binding import iskv_prefill, iskv_protect
+        assert k_rows.dtype == self.dtype and k_rows.is_contiguous() and v_rows.is_contiguous()
+        pr = None if protect is None else iskv_protect(*protect)
+        check(iskv_prefill(self.handle, layer, k_rows, v_rows, k_rows.shape[-2], pr, stream),
+              "iskv_prefill")
 
     def decode(self, layer: int, q: torch.Tensor, out: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:

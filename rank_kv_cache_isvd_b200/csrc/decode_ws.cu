@@ -46,7 +46,7 @@ static_assert(128 * WS_REG_LO + 256 * WS_REG_HI <= WS_THREADS * WS_REG_LAUNCH,
               "register split exceeds the launch allocation");
 
 struct WsLayout {
-    uint32_t bh, bl, kst, vst, q, qt, ss, sp, smax, ssum, bars, total;
+    uint32_t bh, bl, kst, vst, q, qt, ss, sp, smax, ssum, sfl, sidx, bars, total;
     uint32_t kstage, vstage;
     int nsv;
 };
@@ -69,6 +69,7 @@ __host__ __device__ inline WsLayout ws_layout(int bf, int rV, int esz, int G, ui
     const uint32_t misc = (uint32_t)G * 512u * 2u            // q, two segment slots
                           + (uint32_t)G * 512u * 8u          // qt[2], ss[2][2], sp[2]
                           + 2u * 2u * 4u * 4u * 4u           // smax, ssum
+                          + 2u * 128u * 5u                   // per-row flags and store indices
                           + 256u + 1024u;                    // barriers, alignment slack
     int nsv = WS_MAXSV;
     while (nsv > 2 && o + nsv * L.vstage + misc > limit) --nsv;
@@ -80,6 +81,8 @@ __host__ __device__ inline WsLayout ws_layout(int bf, int rV, int esz, int G, ui
     L.sp = o; o += G * 512u * 2u;
     L.smax = o; o += 2u * 4u * 4u * 4u;
     L.ssum = o; o += 2u * 4u * 4u * 4u;
+    L.sfl = o; o += 2u * 128u;                              // protection flags of the tile's rows
+    L.sidx = o; o += 2u * 128u * 4u;                        // their value-store indices
     L.bars = o; o += 256u;
     L.total = o + 1024u;
     return L;
@@ -241,6 +244,36 @@ __device__ __forceinline__ void load_row8(const void *base, size_t idx, int kv_d
     }
 }
 
+// Index of `key` in the ascending array a[0 .. n), or -1.
+__device__ __forceinline__ int find_sorted(const int *a, int n, int key) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (a[mid] < key) lo = mid + 1;
+        else hi = mid;
+    }
+    return (lo < n && a[lo] == key) ? lo : -1;
+}
+
+// The G probabilities of one row (vector loads: rows are 4 G bytes apart, 16-byte aligned for G = 4).
+template <int GT>
+__device__ __forceinline__ void load_p(const float *p, float (&v)[GT]) {
+    if constexpr (GT == 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(p);
+        v[0] = x.x;
+        v[1] = x.y;
+        v[2] = x.z;
+        v[3] = x.w;
+    } else if constexpr (GT == 2) {
+        const float2 x = *reinterpret_cast<const float2 *>(p);
+        v[0] = x.x;
+        v[1] = x.y;
+    } else {
+#pragma unroll
+        for (int g = 0; g < GT; ++g) v[g] = p[g];
+    }
+}
+
 // Four consecutive values of a staged value row: fmt 2 = bf16, 4 = fp32.
 __device__ __forceinline__ float4 load_v4s(const uint8_t *row, int c, int fmt) {
     if (fmt == 2) {
@@ -288,6 +321,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
     float *sP = reinterpret_cast<float *>(sm + L.sp);       // [2][128][G]
     float *sMax = reinterpret_cast<float *>(sm + L.smax);   // [2][4][4]
     float *sSum = reinterpret_cast<float *>(sm + L.ssum);   // [2][4][4]
+    unsigned char *sFl = sm + L.sfl;                        // [2][128] row flags (protection)
+    int *sIdx = reinterpret_cast<int *>(sm + L.sidx);       // [2][128] value-store index per row
     float4 *sRed = reinterpret_cast<float4 *>(sm + L.qt);   // [8 warps][G][32] (aliases qt..sp)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -366,6 +401,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 }
                 for (int tl = ta; tl < tb && ok; ++tl) {
                     const bool comp = tl < Tc;
+                    if (!comp && tl < Tc + x.Tp) continue;     // protected rows: read by the epilogue
                     long long t0;
                     int rows;
                     if (comp) {
@@ -380,7 +416,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         ++kt;
                         counters[2] = kt;
                     } else {
-                        t0 = a.n_c + (long long)(tl - Tc) * DEC_TILE;
+                        t0 = a.n_c + (long long)(tl - Tc - x.Tp) * DEC_TILE;
                         rows = (int)min((long long)DEC_TILE, a.t - t0);
                     }
                     const int vs = vt % NSV;
@@ -535,19 +571,25 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
         bool ok = true;
         int at = 0, vt = 0, seg = 0, it = 0;
 
+        // start position of tile tl of a unit: compressed, protected (queries unrotated: each
+        // protected row carries its own angle), window
+        auto tile_t0 = [&](int tl) -> long long {
+            if (tl < Tc) return (long long)tl * DEC_TILE;
+            if (tl < Tc + x.Tp) return 0;
+            return a.n_c + (long long)(tl - Tc - x.Tp) * DEC_TILE;
+        };
         // q~ = (q rotated by -w_j t0) * scale * log2(e) for tile start t0, into qt buffer `b`
-        auto make_qt = [&](const float *q, long long t0, int b) {
-            for (int o = et; o < G * DH; o += WS_EPI) {
-                const int g = o / DH, j = o % DH;
-                float c = 1.f, s = 0.f;
-                if (a.rope_cs != nullptr) {
-                    const float2 cs = a.rope_cs[(size_t)t0 * DH + j];
-                    c = cs.x;
-                    s = cs.y;
-                }
+        // this thread's pair of q~ is j = et mod 64 (threads et < G 64 build one element each)
+        auto load_cs = [&](long long t0) -> float2 {
+            if (a.rope_cs == nullptr || et >= G * DH) return make_float2(1.f, 0.f);
+            return a.rope_cs[(size_t)t0 * DH + (et & (DH - 1))];
+        };
+        auto make_qt = [&](const float *q, float2 cs, int b) {
+            if (et < G * DH) {
+                const int g = et / DH, j = et & (DH - 1);
                 const float qr = q[g * D + j], qi = q[g * D + DH + j];
-                sQt[(b * G + g) * D + j] = qscale * fmaf(qr, c, qi * s);
-                sQt[(b * G + g) * D + DH + j] = qscale * fmaf(qi, c, -qr * s);
+                sQt[(b * G + g) * D + j] = qscale * fmaf(qr, cs.x, qi * cs.y);
+                sQt[(b * G + g) * D + DH + j] = qscale * fmaf(qi, cs.x, -qr * cs.y);
             }
         };
 
@@ -569,21 +611,42 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 vr[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
                 vw[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            const long long t0a = ta < Tc ? (long long)ta * DEC_TILE
-                                          : a.n_c + (long long)(ta - Tc) * DEC_TILE;
-            if (w) make_qt(q, t0a, it & 1);
+            const long long t0a = tile_t0(ta);
+            if (w) make_qt(q, load_cs(t0a), it & 1);
             ok = bar_and(BAR_EPI, WS_EPI, w);
             if (!ok) break;
             bool good = true;                       // this thread's waits of the segment so far
-            const bool has_c = ta < Tc, has_w = tb > Tc;
+            // channel-space sums: window or protected tiles, or value-protected compressed rows
+            const bool has_c = ta < Tc, has_w = tb > Tc || (x.pflags != nullptr && ta < Tc);
+            const int npk = x.pflags != nullptr ? x.pcount[0][u] : 0;
+            const int npv = x.pflags != nullptr ? x.pcount[1][u] : 0;
             for (int tl = ta; tl < tb; ++tl) {
                 const int b = it & 1;
                 const bool comp = tl < Tc;
-                const long long t0 = comp ? (long long)tl * DEC_TILE
-                                          : a.n_c + (long long)(tl - Tc) * DEC_TILE;
-                const int rows = (int)min((long long)DEC_TILE, (comp ? a.n_c : a.t) - t0);
-                const bool valid = tau < rows;
-                const long long pos = t0 + tau;
+                const bool prot = !comp && tl < Tc + x.Tp;       // protected exact keys
+                const long long t0 = tile_t0(tl);
+                // the next tile's query rotation: fetched now, used after the first barrier
+                const float2 cs_next = tl + 1 < tb ? load_cs(tile_t0(tl + 1)) : make_float2(1.f, 0.f);
+                int rows;
+                long long pos;
+                unsigned char fl = 0;
+                int vidx = -1;
+                if (prot) {
+                    const int pi = (tl - Tc) * DEC_TILE;
+                    rows = max(0, min(DEC_TILE, npk - pi));
+                    pos = tau < rows ? x.ppos[0][(size_t)u * x.pcap + pi + tau] : 0;
+                    if (tau < rows) vidx = find_sorted(x.ppos[1] + (size_t)u * x.pcap, npv, (int)pos);
+                } else {
+                    rows = (int)min((long long)DEC_TILE, (comp ? a.n_c : a.t) - t0);
+                    pos = t0 + tau;
+                    if (comp && x.pflags != nullptr && tau < rows) {
+                        fl = x.pflags[(size_t)u * x.fstride + pos];
+                        if ((fl & 2) && !(fl & 1))
+                            vidx = find_sorted(x.ppos[1] + (size_t)u * x.pcap, npv, (int)pos);
+                    }
+                }
+                // rows whose key is protected are attended in the protected tiles
+                const bool valid = tau < rows && !(fl & 1);
                 // ---- this row's key: pairs (j, j + 64), j in [jb, jb + 32), chunks of 8 pairs,
                 //      rotated by e^{i w_j tau} and dotted with the rotated queries ----------------
                 float2 acc2[GT];
@@ -596,23 +659,36 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 good = good && wk;
                 tc_fence_after();
                 const uint32_t trow = tmem + 128u * (at & 1) + ((uint32_t)(qw * 32) << 16);
-                const bool fresh = !comp && pos == a.new_pos;
-                const void *ksrc = fresh ? a.new_row[0] : a.ring[0];
-                const size_t kbase = fresh ? (size_t)u * D
-                                           : ((size_t)u * a.R + (size_t)(pos % a.R)) * D;
+                const bool fresh = !comp && !prot && pos == a.new_pos;
+                const void *ksrc = prot ? x.pstore[0] : fresh ? a.new_row[0] : a.ring[0];
+                const size_t kbase =
+                    prot ? ((size_t)u * x.pcap + (tl - Tc) * DEC_TILE + tau) * D
+                         : fresh ? (size_t)u * D : ((size_t)u * a.R + (size_t)(pos % a.R)) * D;
                 const float *qt = sQt + (size_t)b * G * D;
+                // key values of chunks (ch, ch + 1) are loaded from tensor memory together
+                float klo[2][8], khi[2][8];
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
                     const int j0 = jb + 8 * ch;
                     float lo[8], hi[8];
                     if (comp) {
-                        if (wk) {
-                            tmem_ld8x(trow + j0, lo);
-                            tmem_ld8x(trow + DH + j0, hi);
-                            tmem_wait_ld();
-                        } else {
+                        if ((ch & 1) == 0) {
+                            if (wk) {
+                                tmem_ld8x(trow + j0, klo[0]);
+                                tmem_ld8x(trow + DH + j0, khi[0]);
+                                tmem_ld8x(trow + j0 + 8, klo[1]);
+                                tmem_ld8x(trow + DH + j0 + 8, khi[1]);
+                                tmem_wait_ld();
+                            } else {
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) lo[i] = hi[i] = 0.f;
+                                for (int i = 0; i < 8; ++i)
+                                    klo[0][i] = khi[0][i] = klo[1][i] = khi[1][i] = 0.f;
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            lo[i] = klo[ch & 1][i];
+                            hi[i] = khi[ch & 1][i];
                         }
                     } else if (valid) {
                         load_row8(ksrc, kbase + j0, a.kv_dtype, lo);
@@ -621,21 +697,45 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
 #pragma unroll
                         for (int i = 0; i < 8; ++i) lo[i] = hi[i] = 0.f;
                     }
+                    // a protected row's angle is its full position's (its queries are unrotated)
+                    float pc[8], ps[8];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 k1 = make_float2(lo[2 * i], lo[2 * i + 1]);
-                        const float2 k2 = make_float2(hi[2 * i], hi[2 * i + 1]);
-                        const float2 c2 = make_float2(tc_[8 * ch + 2 * i], tc_[8 * ch + 2 * i + 1]);
-                        const float2 s2 = make_float2(ts_[8 * ch + 2 * i], ts_[8 * ch + 2 * i + 1]);
-                        const float2 t1 = __fmul2_rn(k2, s2);
-                        const float2 zr = __ffma2_rn(k1, c2, make_float2(-t1.x, -t1.y));
-                        const float2 zi = __ffma2_rn(k1, s2, __fmul2_rn(k2, c2));
+                    for (int i = 0; i < 8; ++i) {
+                        pc[i] = tc_[8 * ch + i];
+                        ps[i] = ts_[8 * ch + i];
+                    }
+                    if (prot) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            float2 cs = make_float2(1.f, 0.f);
+                            if (a.rope_cs != nullptr && valid) cs = a.rope_cs[(size_t)pos * DH + j0 + i];
+                            pc[i] = cs.x;
+                            ps[i] = cs.y;
+                        }
+                    }
+#pragma unroll
+                    for (int i4 = 0; i4 < 2; ++i4) {
+                        // four pairs: rotate the key by e^{i w tau}, then dot with each rotated query
+                        float2 zr[2], zi[2];
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            const int i = 2 * i4 + h2;
+                            const float2 k1 = make_float2(lo[2 * i], lo[2 * i + 1]);
+                            const float2 k2 = make_float2(hi[2 * i], hi[2 * i + 1]);
+                            const float2 c2 = make_float2(pc[2 * i], pc[2 * i + 1]);
+                            const float2 s2 = make_float2(ps[2 * i], ps[2 * i + 1]);
+                            const float2 t1 = __fmul2_rn(k2, s2);
+                            zr[h2] = __ffma2_rn(k1, c2, make_float2(-t1.x, -t1.y));
+                            zi[h2] = __ffma2_rn(k1, s2, __fmul2_rn(k2, c2));
+                        }
 #pragma unroll
                         for (int gg = 0; gg < GT; ++gg) {
-                            const float2 qr = *reinterpret_cast<const float2 *>(qt + gg * D + j0 + 2 * i);
-                            const float2 qi = *reinterpret_cast<const float2 *>(qt + gg * D + DH + j0 + 2 * i);
-                            acc2[gg] = __ffma2_rn(qr, zr, acc2[gg]);
-                            acc2[gg] = __ffma2_rn(qi, zi, acc2[gg]);
+                            const float4 qr = *reinterpret_cast<const float4 *>(qt + gg * D + j0 + 4 * i4);
+                            const float4 qi = *reinterpret_cast<const float4 *>(qt + gg * D + DH + j0 + 4 * i4);
+                            acc2[gg] = __ffma2_rn(make_float2(qr.x, qr.y), zr[0], acc2[gg]);
+                            acc2[gg] = __ffma2_rn(make_float2(qi.x, qi.y), zi[0], acc2[gg]);
+                            acc2[gg] = __ffma2_rn(make_float2(qr.z, qr.w), zr[1], acc2[gg]);
+                            acc2[gg] = __ffma2_rn(make_float2(qi.z, qi.w), zi[1], acc2[gg]);
                         }
                     }
                 }
@@ -663,11 +763,10 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
                     if (hf == 0 && lane == 0) sMax[(b * 4 + qw) * 4 + gg] = m;
                 }
-                if (tl + 1 < tb) {
-                    const int tn = tl + 1;
-                    const long long t0n = tn < Tc ? (long long)tn * DEC_TILE
-                                                  : a.n_c + (long long)(tn - Tc) * DEC_TILE;
-                    make_qt(q, t0n, b ^ 1);
+                if (tl + 1 < tb) make_qt(q, cs_next, b ^ 1);
+                if (hf == 0) {
+                    sFl[b * 128 + tau] = (unsigned char)((fl & 2) && !(fl & 1) && vidx >= 0 ? 2 : 0);
+                    sIdx[b * 128 + tau] = vidx;
                 }
                 bar_named(BAR_EPI, WS_EPI);                              // barrier 2
                 float alpha[GT];
@@ -676,7 +775,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     const float mt = fmaxf(fmaxf(sMax[(b * 4 + 0) * 4 + gg], sMax[(b * 4 + 1) * 4 + gg]),
                                            fmaxf(sMax[(b * 4 + 2) * 4 + gg], sMax[(b * 4 + 3) * 4 + gg]));
                     const float mn = fmaxf(mrun[gg], mt);
-                    alpha[gg] = ex2(mrun[gg] - mn);
+                    // a tile without rows leaves the running state as it is
+                    alpha[gg] = mn == -CUDART_INF_F ? 1.f : ex2(mrun[gg] - mn);
                     mrun[gg] = mn;
                     if (GT == 1 ? hf == 0 : (gg & 1) == hf) {
                         const float p = valid ? ex2(sc[gg] - mn) : 0.f;
@@ -703,20 +803,62 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 }
                 // ---- value sums: v_g += sum_i p[g][i] V[i][quad] ----------------------------
                 const int vs = vt % NSV;
-                const bool wv = wait_ab(v_full + vs, (vt / NSV) & 1, abort_flag);
+                const bool wv = prot ? true : wait_ab(v_full + vs, (vt / NSV) & 1, abort_flag);
                 good = good && wv;
                 const uint8_t *V = sm + L.vst + vs * L.vstage;
                 const float *P = sP + (size_t)b * 128 * G;
-                if (wv) {
+                if (prot) {
+                    // protected rows: exact values from the value store (channel sums)
+                    for (int i = slw; i < rows; i += 8) {
+                        const int vi = sIdx[b * 128 + i];
+                        if (vi < 0) continue;
+                        float t8[8];
+                        load_row8(x.pstore[1], ((size_t)u * x.pcap + vi) * D + (4 * qdw & ~7), a.kv_dtype, t8);
+                        const int o4 = (4 * qdw) & 7;
+                        const float2 v01 = make_float2(t8[o4], t8[o4 + 1]), v23 = make_float2(t8[o4 + 2], t8[o4 + 3]);
+                        float pv[GT];
+                        load_p(P + i * G, pv);
+#pragma unroll
+                        for (int gg = 0; gg < GT; ++gg) {
+                            const float2 p2 = make_float2(pv[gg], pv[gg]);
+                            const float2 x01 = __ffma2_rn(p2, v01, make_float2(vw[gg].x, vw[gg].y));
+                            const float2 x23 = __ffma2_rn(p2, v23, make_float2(vw[gg].z, vw[gg].w));
+                            vw[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
+                        }
+                    }
+                } else if (wv) {
+                    if (comp && x.pflags != nullptr) {
+                        // value-protected rows of a compressed tile: their coordinates are zero;
+                        // the exact value row enters the channel sums
+                        for (int i = slw; i < rows; i += 8) {
+                            if (!(sFl[b * 128 + i] & 2)) continue;
+                            const int vi = sIdx[b * 128 + i];
+                            float t8[8];
+                            load_row8(x.pstore[1], ((size_t)u * x.pcap + vi) * D + (4 * qdw & ~7), a.kv_dtype, t8);
+                            const int o4 = (4 * qdw) & 7;
+                            const float2 v01 = make_float2(t8[o4], t8[o4 + 1]), v23 = make_float2(t8[o4 + 2], t8[o4 + 3]);
+                            float pv[GT];
+                            load_p(P + i * G, pv);
+#pragma unroll
+                            for (int gg = 0; gg < GT; ++gg) {
+                                const float2 p2 = make_float2(pv[gg], pv[gg]);
+                                const float2 x01 = __ffma2_rn(p2, v01, make_float2(vw[gg].x, vw[gg].y));
+                                const float2 x23 = __ffma2_rn(p2, v23, make_float2(vw[gg].z, vw[gg].w));
+                                vw[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
+                            }
+                        }
+                    }
                     if (comp) {
                         const int vld = rV * (BF ? 2 : 4);
 #pragma unroll 4
                         for (int i = slr; i < rows; i += nslr) {
                             const float4 v = load_v4s(V + (size_t)i * vld, 4 * qdr, BF ? 2 : 4);
                             const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
+                            float pv[GT];
+                            load_p(P + i * G, pv);
 #pragma unroll
                             for (int gg = 0; gg < GT; ++gg) {
-                                const float pg = P[i * G + gg];
+                                const float pg = pv[gg];
                                 const float2 p2 = make_float2(pg, pg);
                                 const float2 x01 = __ffma2_rn(p2, v01, make_float2(vr[gg].x, vr[gg].y));
                                 const float2 x23 = __ffma2_rn(p2, v23, make_float2(vr[gg].z, vr[gg].w));
@@ -739,9 +881,11 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                                 v = load_v4s(V + (size_t)i * vld, 4 * qdw, esz);
                             }
                             const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
+                            float pv[GT];
+                            load_p(P + i * G, pv);
 #pragma unroll
                             for (int gg = 0; gg < GT; ++gg) {
-                                const float pg = P[i * G + gg];
+                                const float pg = pv[gg];
                                 const float2 p2 = make_float2(pg, pg);
                                 const float2 x01 = __ffma2_rn(p2, v01, make_float2(vw[gg].x, vw[gg].y));
                                 const float2 x23 = __ffma2_rn(p2, v23, make_float2(vw[gg].z, vw[gg].w));
@@ -766,8 +910,10 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(v_empty + vs);
-                ++vt;
+                if (!prot) {
+                    if (lane == 0) mbar_arrive(v_empty + vs);
+                    ++vt;
+                }
                 ++it;
             }
             // q slot consumed (every q~ of the segment is built)

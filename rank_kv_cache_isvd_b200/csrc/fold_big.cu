@@ -43,8 +43,15 @@ __global__ void __launch_bounds__(RF_THREADS) rfactor_kernel(RFactorArgs a) {
             const int i = o / D, j = o % D;
             float v = 0.f;
             if (i < rows) {
-                const int slot = (a.slot0 + c0 + i) % a.R;
-                v = load_row_elem(P.ring, ring_base + (size_t)slot * D + j, a.kv_dtype);
+                if (P.src != nullptr) {
+                    // prefill: the caller's rows; protected rows do not enter the factor
+                    const long long p = c0 + i;
+                    if (!(P.fbit && (a.flags[(size_t)unit * a.flag_stride + p] & P.fbit)))
+                        v = load_row_elem(P.src, ((size_t)blockIdx.x * a.src_rows + p) * D + j, a.kv_dtype);
+                } else {
+                    const int slot = (a.slot0 + c0 + i) % a.R;
+                    v = load_row_elem(P.ring, ring_base + (size_t)slot * D + j, a.kv_dtype);
+                }
             }
             M[j * RF_LDM + DEC_TILE + i] = v;
         }
@@ -148,8 +155,15 @@ __global__ void __launch_bounds__(RF_THREADS) newrows_kernel(NewRowsArgs a) {
             const int i = o / D, j = o % D;
             float v = 0.f;
             if (i < sr) {
-                const int slot = (a.slot0 + c0 + s0 + i) % a.R;
-                v = load_row_elem(P.ring, ring_base + (size_t)slot * D + j, a.kv_dtype);
+                if (P.src != nullptr) {
+                    // prefill: the caller's rows; protected rows get zero coordinates
+                    const long long p = c0 + s0 + i;
+                    if (!(P.fbit && (a.flags[(size_t)unit * a.flag_stride + p] & P.fbit)))
+                        v = load_row_elem(P.src, ((size_t)blockIdx.y * a.src_rows + p) * D + j, a.kv_dtype);
+                } else {
+                    const int slot = (a.slot0 + c0 + s0 + i) % a.R;
+                    v = load_row_elem(P.ring, ring_base + (size_t)slot * D + j, a.kv_dtype);
+                }
             }
             sF[i * (D + 1) + j] = v;
         }

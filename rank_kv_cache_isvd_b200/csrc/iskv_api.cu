@@ -44,7 +44,18 @@ struct iskv_handle {
     // per layer
     std::vector<long long> t, nc;
     std::vector<int> kcur[2];             // ranks as of the last applied fold (what decode reads)
-    std::vector<long long> nf;            // folds launched (applied folds: nc / block)
+    std::vector<long long> nf;            // folds launched
+    std::vector<long long> pbase;         // rows compressed by the layer's prefill (0: none)
+    std::vector<int> pfold;               // 1 if the layer's prefill counts as its first update
+    std::vector<int> ptiles;              // 128-row tiles of the largest protected key store
+    std::vector<unsigned char> pact;      // the layer's prefill protected some positions
+    // prefill protection (prot_cap > 0): per-position flags, protected stores, counts, scores
+    int pcap = 0;
+    unsigned char *pflags = nullptr;      // [U][n_max]: bit 0 key protected, bit 1 value protected
+    int *ppos[2] = {nullptr, nullptr};    // [U][pcap] positions, ascending
+    void *pstore[2] = {nullptr, nullptr}; // [U][pcap][D] rows (kv dtype)
+    int *pcount[2] = {nullptr, nullptr};  // [U]
+    float *pscores = nullptr;             // [UL][n_max] chunk scores of one layer
     std::vector<int> kf[2];               // ranks after the last launched fold
     std::vector<int> fk;                  // [layer][NB][4]: k_K, kp_K, k_V, kp_V of fold j % NB
     std::vector<unsigned char> on_side;   // [layer][NB]: fold j % NB ran on an internal stream
@@ -88,6 +99,13 @@ void free_all(iskv_handle *h) {
     }
     cudaFree(h->rope_cs);
     cudaFree(h->rope_t);
+    cudaFree(h->pflags);
+    cudaFree(h->pscores);
+    for (int x = 0; x < 2; ++x) {
+        cudaFree(h->ppos[x]);
+        cudaFree(h->pstore[x]);
+        cudaFree(h->pcount[x]);
+    }
     cudaFree(h->ws);
     cudaFree(h->status);
     cudaFree(h->stats);
@@ -158,9 +176,19 @@ bool frozen(const iskv_handle *h, int x, long long j) {
     return j >= (r + h->cfg.block - 1) / h->cfg.block;
 }
 
+// Fold index of a layer holding nc compressed positions, and the first position of fold j's block.
+// Without a prefill the folds take blocks 0, b, 2b, ...; after a prefill of pbase rows (which
+// counts as update 0) fold j takes the block at pbase + (j - 1) b.
+long long fold_of(const iskv_handle *h, int layer, long long nc) {
+    return h->pfold[layer] + (nc - h->pbase[layer]) / h->cfg.block;
+}
+long long block_start(const iskv_handle *h, int layer, long long j) {
+    return h->pbase[layer] + (j - h->pfold[layer]) * (long long)h->cfg.block;
+}
+
 // buffer of the basis / Sigma produced by the last applied fold
 int current_buffer(const iskv_handle *h, int layer) {
-    return (int)((h->nc[layer] / h->cfg.block) % h->NB);
+    return (int)(fold_of(h, layer, h->nc[layer]) % h->NB);
 }
 int *fold_ranks(iskv_handle *h, int layer, long long j) {
     return &h->fk[((size_t)layer * h->NB + (size_t)(j % h->NB)) * 4];
@@ -171,8 +199,9 @@ int *fold_ranks(iskv_handle *h, int layer, long long j) {
 // into j % NB and the new rows' coordinates. The history is rotated when the fold is applied.
 int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
     const iskv_config &c = h->cfg;
-    // the new rows' coordinates go to rows j*b .. j*b+b-1, which must lie within n_max
-    if ((j + 1) * c.block > h->n_max) return ISKV_ERR_CAPACITY;
+    // the new rows' coordinates go to the block's rows, which must lie within n_max
+    const long long nc = block_start(h, l0, j);
+    if (nc + c.block > h->n_max) return ISKV_ERR_CAPACITY;
     const int bi = (int)(j % h->NB), bo = (int)((j + 1) % h->NB);
     // paths that run the regular update (a contiguous range: frozen paths are a prefix or suffix)
     const bool fz[2] = {frozen(h, 0, j), frozen(h, 1, j)};
@@ -199,7 +228,6 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
         fp.p = p;
         fp.kp = kp;
     }
-    const long long nc = j * c.block;
     fa.unit0 = l0 * h->UL;
     fa.n_c = nc;
     fa.n_max = h->n_max;
@@ -295,7 +323,7 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
 // advances n_c, the ranks and the current buffer.
 int apply_fold(iskv_handle *h, int l0, int nl, cudaStream_t s) {
     const iskv_config &c = h->cfg;
-    const long long j = h->nc[l0] / c.block;
+    const long long j = fold_of(h, l0, h->nc[l0]);
     const int bi = (int)(j % h->NB);
     if (h->nf[l0] <= j) {
         const int rc = launch_fold_j(h, l0, nl, j, s);
@@ -347,8 +375,9 @@ int launch_ahead(iskv_handle *h, int l0, int nl, cudaStream_t s) {
     const iskv_config &c = h->cfg;
     cudaStream_t side = h->side[l0 % iskv_handle::NS];
     bool forked = false;
-    while ((h->nf[l0] + 1) * c.block <= h->t[l0] && (h->nf[l0] + 1) * c.block <= h->n_max &&
-           h->nf[l0] <= h->nc[l0] / c.block + h->NB - 2) {
+    while (block_start(h, l0, h->nf[l0]) + c.block <= h->t[l0] &&
+           block_start(h, l0, h->nf[l0]) + c.block <= h->n_max &&
+           h->nf[l0] <= fold_of(h, l0, h->nc[l0]) + h->NB - 2) {
         const long long j = h->nf[l0];
         const int bi = (int)(j % h->NB);
         if (!forked) {
@@ -416,7 +445,8 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         c.n_q_heads % c.n_kv_heads != 0 || c.n_q_heads / c.n_kv_heads > GMAX || c.head_dim != D ||
         c.rank_k < 1 || c.rank_k > D || c.rank_v < 1 || c.rank_v > D || c.block < 1 ||
         c.window < 0 || c.max_tokens < 1 || (c.kv_dtype != ISKV_BF16 && c.kv_dtype != ISKV_F32) ||
-        (c.rope && !(c.rope_theta > 0.0)) || (c.fixed_basis && !c.rotate_history))
+        (c.rope && !(c.rope_theta > 0.0)) || (c.fixed_basis && !c.rotate_history) ||
+        c.prot_cap < 0)
         return ISKV_ERR_INVALID_ARG;
     if (c.block > BMAX_LARGE) return ISKV_ERR_UNSUPPORTED;
     iskv_handle *h = new (std::nothrow) iskv_handle();
@@ -432,7 +462,10 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         h->U = c.n_layers * h->UL;
         h->R = c.window + c.block;
         h->G = c.n_q_heads / c.n_kv_heads;
-        h->n_max = ncomp(c.max_tokens, c.block, c.window);
+        // compressed positions: up to max_tokens - window (a prefill's end need not be a
+        // multiple of the block)
+        h->n_max = c.max_tokens > c.window ? c.max_tokens - c.window : 0;
+        h->pcap = c.prot_cap;
         h->esz = c.kv_dtype == ISKV_BF16 ? 2 : 4;
         h->cbf = c.coord_bf16 ? 1 : 0;
         h->csz = h->cbf ? 2 : 4;
@@ -443,6 +476,10 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         h->t.assign(c.n_layers, 0);
         h->nc.assign(c.n_layers, 0);
         h->nf.assign(c.n_layers, 0);
+        h->pbase.assign(c.n_layers, 0);
+        h->pfold.assign(c.n_layers, 0);
+        h->ptiles.assign(c.n_layers, 0);
+        h->pact.assign(c.n_layers, 0);
         for (int x = 0; x < 2; ++x) {
             h->kcur[x].assign(c.n_layers, 0);
             h->kf[x].assign(c.n_layers, 0);
@@ -472,7 +509,13 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         alloc((void **)&h->sigma[x], nb * U * r * sizeof(float));
         alloc(&h->ring[x], U * (size_t)h->R * D * h->esz);
         alloc((void **)&h->htop[x], nb * U * r * r * sizeof(float));
-        if (c.block > BMAX) alloc((void **)&h->rbig[x], U * DEC_TILE * D * sizeof(float));
+        if (c.block > BMAX || c.prot_cap > 0)
+            alloc((void **)&h->rbig[x], U * DEC_TILE * D * sizeof(float));
+        if (c.prot_cap > 0) {
+            alloc((void **)&h->ppos[x], U * (size_t)c.prot_cap * sizeof(int));
+            alloc(&h->pstore[x], U * (size_t)c.prot_cap * D * h->esz);
+            alloc((void **)&h->pcount[x], U * sizeof(int));
+        }
     }
     if (c.rope) alloc((void **)&h->rope_cs, (size_t)c.max_tokens * DH * sizeof(float2));
     if (c.rope) alloc((void **)&h->rope_t, (size_t)c.max_tokens * DH * sizeof(float2));
@@ -483,6 +526,10 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         alloc((void **)&h->ws, (a1 > a2 ? a1 : a2) * sizeof(float));
     }
     alloc((void **)&h->status, sizeof(int));
+    if (c.prot_cap > 0) {
+        alloc((void **)&h->pflags, U * (size_t)(h->n_max > 0 ? h->n_max : 1));
+        alloc((void **)&h->pscores, (size_t)h->UL * (size_t)(h->n_max > 0 ? h->n_max : 1) * sizeof(float));
+    }
     alloc((void **)&h->stats, 4 * sizeof(unsigned long long));
     if (ok) {
         for (int x = 0; x < 2; ++x) {
@@ -491,6 +538,11 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
             ok = ok && cudaMemset(h->sigma[x], 0, nb * U * r * sizeof(float)) == cudaSuccess;
         }
         ok = ok && cudaMemset(h->status, 0, sizeof(int)) == cudaSuccess;
+        if (ok && c.prot_cap > 0) {
+            ok = cudaMemset(h->pflags, 0, U * (size_t)(h->n_max > 0 ? h->n_max : 1)) == cudaSuccess &&
+                 cudaMemset(h->pcount[0], 0, U * sizeof(int)) == cudaSuccess &&
+                 cudaMemset(h->pcount[1], 0, U * sizeof(int)) == cudaSuccess;
+        }
         ok = ok && cudaMemset(h->stats, 0, 4 * sizeof(unsigned long long)) == cudaSuccess;
         for (int i = 0; ok && i < iskv_handle::NS; ++i)
             ok = cudaStreamCreateWithFlags(&h->side[i], cudaStreamNonBlocking) == cudaSuccess;
@@ -653,7 +705,12 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
     da.max_splits = h->max_splits;
     da.kv_dtype = c.kv_dtype;
     da.scale = 1.0f / sqrtf((float)D);
-    if (h->ws_ok) {
+    // the persistent decode pays off once every SM streams many tiles; smaller calls (fp32
+    // coordinates, no protection) use the split-kernel decode
+    const long long tiles_ws = (long long)h->UL * (ctiles + (e + DEC_TILE - 1) / DEC_TILE);
+    const bool use_ws = h->ws_ok && (h->cbf || h->pact[layer] || !h->tc ||
+                                     tiles_ws >= 8LL * h->sms);
+    if (use_ws) {
         if (reinterpret_cast<uintptr_t>(q) % 16 != 0) return ISKV_ERR_INVALID_ARG;
         WsExtra x;
         memset(&x, 0, sizeof(x));
@@ -669,6 +726,22 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
         x.maxseg = h->UL / x.P + 2;
         x.factor_bf16 = h->cbf;
         x.status = h->status;
+        if (h->pact[layer]) {
+            const size_t u0 = (size_t)layer * h->UL;
+            x.pflags = h->pflags + u0 * (size_t)h->n_max;
+            x.fstride = h->n_max;
+            for (int p = 0; p < 2; ++p) {
+                x.ppos[p] = h->ppos[p] + u0 * h->pcap;
+                x.pstore[p] = static_cast<const char *>(h->pstore[p]) + u0 * h->pcap * D * h->esz;
+                x.pcount[p] = h->pcount[p] + u0;
+            }
+            x.pcap = h->pcap;
+            x.Tp = h->ptiles[layer];
+            x.Tu = x.Tc + x.Tp + x.Tw;
+            x.N = (long long)h->UL * x.Tu;
+            x.P = (int)(x.N < h->sms ? x.N : h->sms);
+            x.maxseg = h->UL / x.P + 2;
+        }
         if (x.N < 1) return ISKV_ERR_INVALID_ARG;
         const cudaError_t e = launch_decode_ws(&h->tmC, &h->tmB, da, x, s);
         if (e == cudaSuccess) {
@@ -676,8 +749,8 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
             return ISKV_OK;
         }
         // a build whose register allocation cannot hold the kernel's register split is never
-        // launched: use the split-kernel decode from now on (fp32 coordinates only)
-        if (e != cudaErrorInvalidConfiguration || h->cbf) return ISKV_ERR_CUDA;
+        // launched: use the split-kernel decode from now on (fp32 coordinates, no protection)
+        if (e != cudaErrorInvalidConfiguration || h->cbf || h->pact[layer]) return ISKV_ERR_CUDA;
         h->ws_ok = false;
     }
     if (da.n_split > h->max_splits) return ISKV_ERR_INVALID_ARG;
@@ -704,6 +777,173 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
 }  // namespace
 
 extern "C" {
+
+int iskv_prefill(iskv_handle *h, int layer, const void *k_rows, const void *v_rows, long long T0,
+                 const iskv_protect *prot, iskv_stream_t stream) {
+    if (!h || !k_rows || !v_rows || !valid_layer(h, layer) || T0 < 1) return ISKV_ERR_INVALID_ARG;
+    const iskv_config &c = h->cfg;
+    if (h->t[layer] != 0 || h->nf[layer] != 0) return ISKV_ERR_INVALID_ARG;
+    if (prot && (prot->chunk < 1 || prot->m < 0 || prot->suffix < 0 || prot->rho < 0))
+        return ISKV_ERR_INVALID_ARG;
+    if (T0 > c.max_tokens) return ISKV_ERR_CAPACITY;
+    if (h->pcap <= 0) return ISKV_ERR_UNSUPPORTED;
+    const long long end = T0 - c.window;
+    if (end <= 0) return iskv_append_block(h, layer, k_rows, v_rows, (int)T0, stream);
+    if (end > 0x7fffffffLL) return ISKV_ERR_UNSUPPORTED;
+    if (prot && !h->ws_ok) return ISKV_ERR_UNSUPPORTED;
+    DeviceGuard g(h->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int UL = h->UL, u0 = layer * UL;
+    // 1-2. protected positions and stores (step 1 for keys, step 2 for values)
+    if (prot) {
+        ProtArgs pa;
+        memset(&pa, 0, sizeof(pa));
+        pa.keys = k_rows;
+        pa.src[0] = k_rows;
+        pa.src[1] = v_rows;
+        pa.src_rows = T0;
+        pa.end = end;
+        pa.T0 = T0;
+        pa.chunk = prot->chunk;
+        pa.m = prot->m;
+        pa.suffix = prot->suffix;
+        pa.rho = prot->rho;
+        pa.n_chunks = (int)((end + prot->chunk - 1) / prot->chunk);
+        pa.n_chunks_cap = (int)h->n_max;
+        pa.scores = h->pscores;
+        pa.flags = h->pflags;
+        pa.flag_stride = h->n_max;
+        pa.unit0 = u0;
+        pa.cap = h->pcap;
+        for (int x = 0; x < 2; ++x) {
+            pa.ppos[x] = h->ppos[x];
+            pa.store[x] = h->pstore[x];
+            pa.pcount[x] = h->pcount[x];
+        }
+        pa.rope_cs = c.rope ? h->rope_cs : nullptr;
+        pa.kv_dtype = c.kv_dtype;
+        pa.status = h->status;
+        if (launch_protect(pa, UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+        h->launches += 2;
+    }
+    // 3. truncated SVD of the remaining rows: their triangular factor, then its fold from rank 0
+    RFactorArgs rf;
+    memset(&rf, 0, sizeof(rf));
+    for (int x = 0; x < 2; ++x) {
+        rf.path[x].rout = h->rbig[x];
+        rf.path[x].src = x ? v_rows : k_rows;
+        rf.path[x].fbit = prot ? (1 << x) : 0;
+    }
+    rf.unit0 = u0;
+    rf.R = 1;
+    rf.b = (int)end;
+    rf.kv_dtype = c.kv_dtype;
+    rf.path_lo = 0;
+    rf.path_hi = 2;
+    rf.src_rows = T0;
+    rf.flags = h->pflags;
+    rf.flag_stride = h->n_max;
+    if (!prot) rf.flags = nullptr;
+    if (launch_rfactor(rf, UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+    FoldArgs fa;
+    memset(&fa, 0, sizeof(fa));
+    int kp[2];
+    for (int x = 0; x < 2; ++x) {
+        const int r = rank_of(h, x);
+        kp[x] = r < DEC_TILE ? r : DEC_TILE;
+        FoldPath &fp = fa.path[x];
+        fp.ring = h->rbig[x];
+        fp.basis_in = basis_buf(h, x, 0);
+        fp.basis_out = basis_buf(h, x, 1);
+        fp.sigma_in = sigma_buf(h, x, 0);
+        fp.sigma_out = sigma_buf(h, x, 1);
+        fp.coords = h->coords[x];
+        fp.htop = htop_buf(h, x, 0);
+        fp.r = r;
+        fp.k = 0;
+        fp.p = DEC_TILE;
+        fp.kp = kp[x];
+    }
+    fa.unit0 = u0;
+    fa.n_c = 0;
+    fa.n_max = h->n_max;
+    fa.slot0 = 0;
+    fa.R = DEC_TILE;
+    fa.b = DEC_TILE;
+    fa.kv_dtype = ISKV_F32;
+    fa.status = h->status;
+    fa.stats = h->stats;
+    fa.skip_new_rows = 1;
+    fa.path_lo = 0;
+    fa.path_hi = 2;
+    fa.cbf = h->cbf;
+    if (launch_fold(fa, UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+    // coordinates of every row before the window (zero for protected rows)
+    NewRowsArgs nr;
+    memset(&nr, 0, sizeof(nr));
+    for (int x = 0; x < 2; ++x) {
+        nr.path[x].basis = basis_buf(h, x, 1);
+        nr.path[x].coords = h->coords[x];
+        nr.path[x].r = rank_of(h, x);
+        nr.path[x].kp = kp[x];
+        nr.path[x].src = x ? v_rows : k_rows;
+        nr.path[x].fbit = prot ? (1 << x) : 0;
+    }
+    nr.unit0 = u0;
+    nr.R = 1;
+    nr.b = (int)end;
+    nr.kv_dtype = c.kv_dtype;
+    nr.n_c = 0;
+    nr.n_max = h->n_max;
+    nr.path_lo = 0;
+    nr.path_hi = 2;
+    nr.cbf = h->cbf;
+    nr.src_rows = T0;
+    nr.flags = prot ? h->pflags : nullptr;
+    nr.flag_stride = h->n_max;
+    if (launch_newrows(nr, UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+    // the window: rows end .. T0 - 1
+    AppendArgs aa;
+    aa.src[0] = k_rows;
+    aa.src[1] = v_rows;
+    aa.ring[0] = h->ring[0];
+    aa.ring[1] = h->ring[1];
+    aa.unit0 = u0;
+    aa.m_total = (int)T0;
+    aa.row0 = (int)end;
+    aa.rows = (int)(T0 - end);
+    aa.pos0 = end;
+    aa.R = h->R;
+    aa.kv_dtype = c.kv_dtype;
+    if (launch_append(aa, UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+    h->launches += 4;
+    // host state: the prefill is update 0 of the layer
+    h->t[layer] = T0;
+    h->nc[layer] = end;
+    h->pbase[layer] = end;
+    h->pfold[layer] = 1;
+    h->nf[layer] = 1;
+    for (int x = 0; x < 2; ++x) h->kcur[x][layer] = h->kf[x][layer] = kp[x];
+    int *f = fold_ranks(h, layer, 0);
+    f[0] = 0;
+    f[1] = kp[0];
+    f[2] = 0;
+    f[3] = kp[1];
+    if (prot) {
+        // the largest protected key count sizes the decode's protected tiles
+        std::vector<int> cnt(UL);
+        if (cudaMemcpyAsync(cnt.data(), h->pcount[0] + u0, UL * sizeof(int), cudaMemcpyDeviceToHost,
+                            s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return ISKV_ERR_CUDA;
+        int mx = 0;
+        for (int v : cnt) mx = v > mx ? v : mx;
+        h->ptiles[layer] = (mx + DEC_TILE - 1) / DEC_TILE;
+        h->pact[layer] = 1;
+    }
+    if (c.lookahead_folds) return launch_ahead(h, layer, 1, s);
+    return ISKV_OK;
+}
 
 int iskv_decode_attn(iskv_handle *h, int layer, const float *q, float *out, iskv_stream_t stream) {
     if (!h || !q || !out || !valid_layer(h, layer)) return ISKV_ERR_INVALID_ARG;
@@ -760,6 +1000,15 @@ int iskv_reconstruct(iskv_handle *h, int layer, int which, int apply_rope, float
     ra.R = h->R;
     ra.kv_dtype = h->cfg.kv_dtype;
     ra.apply_rope = (which == 0 && apply_rope && h->cfg.rope) ? 1 : 0;
+    if (h->pact[layer]) {
+        ra.pflags = h->pflags + u0 * (size_t)h->n_max;
+        ra.fstride = h->n_max;
+        ra.fbit = which ? 2 : 1;
+        ra.ppos = h->ppos[which] + u0 * h->pcap;
+        ra.pstore = static_cast<const char *>(h->pstore[which]) + u0 * h->pcap * D * h->esz;
+        ra.pcount = h->pcount[which] + u0;
+        ra.pcap = h->pcap;
+    }
     if (launch_reconstruct(ra, h->UL, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return ISKV_ERR_CUDA;
     h->launches += ra.t > 0 ? 1 : 0;
@@ -812,11 +1061,23 @@ int iskv_reset(iskv_handle *h, iskv_stream_t stream) {
         h->t[l] = 0;
         h->nc[l] = 0;
         h->nf[l] = 0;
+        h->pbase[l] = 0;
+        h->pfold[l] = 0;
+        h->ptiles[l] = 0;
+        h->pact[l] = 0;
         for (int x = 0; x < 2; ++x) h->kcur[x][l] = h->kf[x][l] = 0;
     }
     if (cudaMemsetAsync(h->status, 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)) !=
         cudaSuccess)
         return ISKV_ERR_CUDA;
+    if (h->pcap > 0) {
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        if (cudaMemsetAsync(h->pflags, 0, (size_t)h->U * (size_t)(h->n_max > 0 ? h->n_max : 1), s) !=
+                cudaSuccess ||
+            cudaMemsetAsync(h->pcount[0], 0, (size_t)h->U * sizeof(int), s) != cudaSuccess ||
+            cudaMemsetAsync(h->pcount[1], 0, (size_t)h->U * sizeof(int), s) != cudaSuccess)
+            return ISKV_ERR_CUDA;
+    }
     if (cudaMemsetAsync(h->stats, 0, 4 * sizeof(unsigned long long),
                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return ISKV_ERR_CUDA;

@@ -52,17 +52,24 @@ struct FoldArgs {
 struct RFactorPath {
     const void *ring;       // [units][R][D] kv dtype
     float *rout;            // [units][128][D] fp32 pseudo-block (R of the block)
+    const void *src;        // prefill: rows [call units][src_rows][D] read instead of the ring
+    int fbit;               // prefill: rows whose flag has this bit read as zero
 };
 struct RFactorArgs {
     RFactorPath path[2];
     int unit0, slot0, R, b, kv_dtype;
     int path_lo, path_hi;   // paths processed: path_lo .. path_hi - 1
+    long long src_rows;     // prefill: rows per unit of src
+    const unsigned char *flags;   // prefill: per-position protection flags [units][flag_stride]
+    long long flag_stride;
 };
 struct NewRowsPath {
     const void *ring;       // [units][R][D] kv dtype
     const float *basis;     // [units][D][r] basis after the fold
     void *coords;           // [units][n_max][r] fp32 or bf16
     int r, kp;
+    const void *src;        // prefill: rows [call units][src_rows][D] read instead of the ring
+    int fbit;               // prefill: rows whose flag has this bit get zero coordinates
 };
 struct NewRowsArgs {
     NewRowsPath path[2];
@@ -70,6 +77,31 @@ struct NewRowsArgs {
     long long n_c, n_max;
     int path_lo, path_hi;   // paths processed: path_lo .. path_hi - 1
     int cbf;                // 1: coordinates stored in bf16
+    long long src_rows;
+    const unsigned char *flags;
+    long long flag_stride;
+};
+
+// ---- prefill protection ------------------------------------------------------------------------
+struct ProtArgs {
+    const void *keys;       // [call units][src_rows][D] pre-RoPE key rows
+    const void *src[2];     // key and value rows, same layout
+    long long src_rows;     // rows per unit in the caller's arrays (the prefill length T0)
+    long long end;          // rows considered for protection and compression: 0 .. end - 1
+    long long T0;
+    int chunk, m, suffix, rho;
+    int n_chunks, n_chunks_cap;
+    float *scores;          // [call units][n_chunks_cap]
+    unsigned char *flags;   // [units][flag_stride]: bit 0 key protected, bit 1 value protected
+    long long flag_stride;
+    int unit0;              // first unit of the call
+    int cap;                // protected rows kept per unit and path
+    int *ppos[2];           // [units][cap] positions of the protected rows, ascending
+    void *store[2];         // [units][cap][D] the protected rows (kv dtype)
+    int *pcount[2];         // [units] protected rows stored
+    const float2 *rope_cs;  // [max_tokens][DH] (cos, sin) or nullptr (no RoPE)
+    int kv_dtype;
+    int *status;
 };
 
 // ---- history rotation C[0:n] <- C[0:n] H_top (or stale zero-padding) ---------------------------
@@ -138,6 +170,14 @@ struct ReconArgs {
     long long n_c, t, n_max;
     int R, kv_dtype, apply_rope;
     int cbf;
+    // prefill protection of this path (pflags nullptr: none); pointers start at the layer's units
+    const unsigned char *pflags;
+    long long fstride;
+    int fbit;               // 1 keys, 2 values
+    const int *ppos;        // [units][pcap]
+    const void *pstore;     // [units][pcap][D]
+    const int *pcount;      // [units]
+    int pcap;
 };
 
 // extra state of the tensor-core decode kernel
@@ -160,8 +200,16 @@ struct WsExtra {
     int P;                  // CTAs (one per SM, at most N)
     int maxseg;             // partial records per CTA (units / P + 2)
     int UL;                 // units of the layer
-    int factor_bf16;        // 1: coordinates and bases stored in bf16
+    int factor_bf16;        // 1: coordinates stored in bf16
     int *status;
+    // prefill protection (nullptr / 0 when the layer has none); pointers start at the layer's units
+    const unsigned char *pflags;  // [units][fstride]: bit 0 key protected, bit 1 value protected
+    long long fstride;
+    const int *ppos[2];     // [units][pcap] positions of the protected rows, ascending
+    const void *pstore[2];  // [units][pcap][D] protected rows (kv dtype)
+    const int *pcount[2];   // [units]
+    int pcap;
+    int Tp;                 // 128-row tiles of protected keys per unit (after the compressed tiles)
 };
 
 cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s);
@@ -172,6 +220,7 @@ cudaError_t launch_append(const AppendArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_reconstruct(const ReconArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_coords_to_f32(float *dst, const void *src, size_t n, cudaStream_t s);
+cudaError_t launch_protect(const ProtArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_rope_table(float2 *table, long long max_tokens, double theta, cudaStream_t s);
 cudaError_t launch_rope_table_t(float4 *table_t, long long max_tokens, double theta,
                                 cudaStream_t s);

@@ -85,7 +85,21 @@ __global__ void reconstruct_kernel(ReconArgs a) {
         const long long pos = p0 + i;
         if (pos >= a.t) break;
         float x;
-        if (pos < a.n_c) {
+        const bool protd = pos < a.n_c && a.pflags != nullptr &&
+                           (a.pflags[(size_t)unit * a.fstride + pos] & a.fbit);
+        if (protd) {
+            // a protected position: the exact row from the path's store
+            const int *pp = a.ppos + (size_t)unit * a.pcap;
+            int lo = 0, hi = a.pcount[unit];
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (pp[mid] < pos) lo = mid + 1;
+                else hi = mid;
+            }
+            x = (lo < a.pcount[unit] && pp[lo] == pos)
+                    ? load_row_elem(a.pstore, ((size_t)unit * a.pcap + lo) * D + j, a.kv_dtype)
+                    : 0.f;
+        } else if (pos < a.n_c) {
             const size_t ci = ((size_t)unit * a.n_max + pos) * r;
             float s = 0.f;
             for (int l = 0; l < k; ++l) s = fmaf(load_coord(a.coords, ci + l, a.cbf), sB[j * ks + l], s);
