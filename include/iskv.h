@@ -146,7 +146,7 @@ int iskv_append_block(iskv_handle *h, int layer, const void *k_rows_dev, const v
  *   protect: host pointer or NULL.
  * Synchronises `stream` when protect is given (the largest protected count sizes the decode's
  * protected tiles). Needs cfg.prot_cap >= 1 (else ISKV_ERR_UNSUPPORTED); protection also needs
- * the persistent decode (coordinates in one 32-column box for fp32, G of 1, 2 or 4).
+ * the persistent decode (rank_k <= 32 with fp32 coordinates, <= 64 with bf16; G of 1, 2 or 4).
  * Errors: ISKV_ERR_INVALID_ARG (layer not empty, bad protect values, T0 < 1),
  *         ISKV_ERR_CAPACITY (T0 > max_tokens), ISKV_ERR_UNSUPPORTED, ISKV_ERR_CUDA.
  */

@@ -791,6 +791,10 @@ int iskv_prefill(iskv_handle *h, int layer, const void *k_rows, const void *v_ro
     if (end <= 0) return iskv_append_block(h, layer, k_rows, v_rows, (int)T0, stream);
     if (end > 0x7fffffffLL) return ISKV_ERR_UNSUPPORTED;
     if (prot && !h->ws_ok) return ISKV_ERR_UNSUPPORTED;
+    const int n_chunks = prot ? (int)((end + prot->chunk - 1) / prot->chunk) : 0;
+    if (prot && (prot_select_smem(n_chunks, prot->m < n_chunks ? prot->m : n_chunks) > 227 * 1024 ||
+                 prot_score_smem(prot->chunk) > 227 * 1024))
+        return ISKV_ERR_UNSUPPORTED;               // too many chunks (or too long a chunk) for one CTA
     DeviceGuard g(h->device);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int UL = h->UL, u0 = layer * UL;
@@ -805,10 +809,10 @@ int iskv_prefill(iskv_handle *h, int layer, const void *k_rows, const void *v_ro
         pa.end = end;
         pa.T0 = T0;
         pa.chunk = prot->chunk;
-        pa.m = prot->m;
+        pa.n_chunks = (int)((end + prot->chunk - 1) / prot->chunk);
+        pa.m = prot->m < pa.n_chunks ? prot->m : pa.n_chunks;      // "up to m" chunks
         pa.suffix = prot->suffix;
         pa.rho = prot->rho;
-        pa.n_chunks = (int)((end + prot->chunk - 1) / prot->chunk);
         pa.n_chunks_cap = (int)h->n_max;
         pa.scores = h->pscores;
         pa.flags = h->pflags;

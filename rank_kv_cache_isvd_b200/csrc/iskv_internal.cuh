@@ -221,6 +221,8 @@ cudaError_t launch_decode(const DecodeArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_reconstruct(const ReconArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_coords_to_f32(float *dst, const void *src, size_t n, cudaStream_t s);
 cudaError_t launch_protect(const ProtArgs &a, int n_units, cudaStream_t s);
+size_t prot_select_smem(int n_chunks, int m);
+size_t prot_score_smem(int chunk);
 cudaError_t launch_rope_table(float2 *table, long long max_tokens, double theta, cudaStream_t s);
 cudaError_t launch_rope_table_t(float4 *table_t, long long max_tokens, double theta,
                                 cudaStream_t s);

@@ -502,8 +502,16 @@ def test_decode_parity_ranks_below_one_tensor_map_box():
                                             ("gapped", 4)])
 def test_bf16_coordinates_fold_one_step_parity(variant, wl_id):
     """bf16 coordinates: each GPU fold, started from the GPU's own state, stores the oracle's
-    rounded coordinates (at most one bf16 step apart, equal almost everywhere where the subspace
-    is gapped); Sigma and the basis (fp32) match as in the fp32 mode."""
+    rounded coordinates where the subspace is gapped; Sigma and the basis (fp32) match as in the
+    fp32 mode.
+
+    The device rounds its fp32 coordinates c_dev to nearest even, and c_dev differs from the exact
+    coordinates c by the fp32 fold error, at most a subspace-angle error times the row norm. So
+    |stored - c| <= 2^-8 |stored| + PROJ_TOL * |row of c|: the first term is half a bf16 step,
+    the second the fp32 error. Truncation or a one-step rounding error breaks the first term for
+    about half of all entries. Rounding decisions can still differ where c_dev and c fall on the
+    two sides of a rounding midpoint. The expected fraction of such entries is about the fp32
+    error over the bf16 step (a few percent), and it is bounded at 10 %."""
     from oracle import round_bf16
     base = syn.WORKLOADS[wl_id]
     T = 1100 if wl_id != 4 else 2100
@@ -511,7 +519,7 @@ def test_bf16_coordinates_fold_one_step_parity(variant, wl_id):
     kd, kv, vd, vv = workload_arrays(wl, variant=variant)
     cache = make_cache(wl, coord_bf16=True)
     t, folds = 0, 0
-    worst = {"sigma": 0.0, "proj": 0.0, "mismatch": 0.0, "steps": 0.0}
+    worst = {"sigma": 0.0, "proj": 0.0, "mismatch": 0.0, "excess": 0.0, "bias": 0.0}
     while True:
         nc = n_compressed(t, wl.block, wl.window)
         t_fold = nc + wl.window + wl.block
@@ -540,12 +548,16 @@ def test_bf16_coordinates_fold_one_step_parity(variant, wl_id):
                 for c in range(k0, k1):
                     if float(got[:, c] @ E[:, c]) < 0:
                         got[:, c] = -got[:, c]
-                step = np.maximum(np.abs(E), np.abs(got)) * 2.0 ** -7 + 1e-30
-                worst["steps"] = max(worst["steps"], float((np.abs(got - E) / step).max()))
+                row = np.linalg.norm(Cr, axis=1, keepdims=True)
+                bound = 2.0 ** -8 * np.abs(got) + PROJ_TOL * row + 1e-30
+                worst["excess"] = max(worst["excess"], float((np.abs(got - Cr) / bound).max()))
                 worst["mismatch"] = max(worst["mismatch"], float(np.mean(got != E)))
+                # round to nearest leaves no sign bias relative to the bf16 step
+                rel = np.sign(got) * (got - Cr) / (2.0 ** -8 * np.abs(got) + 1e-30)
+                worst["bias"] = max(worst["bias"], abs(float(rel[np.abs(got) > 0].mean())))
     print(f"\nbf16 coordinates {variant} cfg {wl_id}: {folds} folds, worst {worst}")
     assert worst["sigma"] <= SIG_TOL and worst["proj"] <= PROJ_TOL
-    assert worst["steps"] <= 1.0 and worst["mismatch"] <= 2e-2
+    assert worst["excess"] <= 1.0 and worst["mismatch"] <= 0.1 and worst["bias"] <= 0.1
     assert cache.status() == 0
 
 
@@ -848,12 +860,14 @@ def _prefill_rows(wl, planted_chunks, chunk, variant="literal"):
 
 @pytest.mark.parametrize("cbf,variant", [(False, "gapped"), (False, "literal"), (True, "literal")])
 def test_prefill_with_protection_matches_oracle(cbf, variant):
-    """Prefill Compression on the long-context shapes (b = 512, w = 512, r_K = 64, r_V = 96):
+    """Prefill Compression on the long-context shapes (b = 512, w = 512, r_V = 96; r_K = 64 with
+    bf16 coordinates, 32 with fp32 coordinates, whose protected decode takes r_K <= 32):
     protected key chunks and their value neighbourhoods stay exact, the other rows before the
     window get one truncated SVD, later tokens fold from the window; reconstructions and decode
     match the oracle's prefill."""
     base = syn.WORKLOADS[4]
-    wl = sub(base, batch=1, n_layers=1, n_kv_heads=2, n_q_heads=8, tokens=4300, prefill=3000)
+    wl = sub(base, batch=1, n_layers=1, n_kv_heads=2, n_q_heads=8, tokens=4300, prefill=3000,
+             rank_k=base.rank_k if cbf else 32)
     chunk, m, suffix, rho = 32, 3, 40, 2
     kd, kv, vd, vv = _prefill_rows(wl, [5, 31, 60], chunk, variant)
     T0 = wl.prefill
