@@ -65,8 +65,8 @@ WL_SINGLE = syn.WORKLOADS[0]
 
 FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12    # fp32 FMA peak of the B200 at its max SM clock
 HBM_NOMINAL_GBS = 7700.0                              # HBM3e nominal bandwidth (HGX figure), context
-DECODE_SRC = os.path.join(ROOT, "rank_kv_cache_isvd_b200", "csrc", "decode_tc.cu")
-PROFILE_DECODE = os.path.join(ROOT, "profiles", "decode_split_qwen3-8b-layer_t32768.md")
+DECODE_SRC = os.path.join(ROOT, "rank_kv_cache_isvd_b200", "csrc", "decode_ws.cu")
+PROFILE_DECODE = os.path.join(ROOT, "profiles", "decode_ws_qwen3-8b-layer_t32768.md")
 
 
 # ---------------------------------------------------------------------------------------------

@@ -7,8 +7,8 @@
 // afterwards. RoPE at position t0 + tau (tile start t0, row tau) is split into two rotations:
 //   score_g = sum_j Re( conj(Q_gj e^{-i w_j t0}) * (k_j e^{i w_j tau}) ),  k_j = K~_j + i K~_{j+64},
 // so the queries are rotated once per tile (by t0) and every row by an angle that depends only on
-// tau, whose cosines and sines each thread keeps in registers for the whole kernel (no per-row
-// table reads). Values are accumulated in rank space (sum_i p_i C_V[i]) and expanded once through
+// tau. The cosines and sines of row tau are written once into the row's tensor-memory lane and
+// read back next to the row's key values (no per-row global table reads). Values are accumulated in rank space (sum_i p_i C_V[i]) and expanded once through
 // B_V^T by the merge kernel.
 //
 // Work split: the (unit, tile) pairs of all units of the layer - each unit's compressed tiles
@@ -39,6 +39,10 @@ constexpr int WS_MAXSV = 4;                  // value stages (at most)
 constexpr uint32_t WS_BLK = 128u * 128u;     // 128 rows x 128 bytes
 constexpr int BAR_EPI = 1, BAR_SPLIT = 2;    // named barriers
 constexpr float LOG2E = 1.4426950408889634f;
+// Lazy softmax reference: probabilities are 2^(s - m_ref) with m_ref a CTA-uniform running
+// reference that moves only when a score exceeds it by more than WS_LAZY (log2 units), so that
+// p <= 2^WS_LAZY and sums over a unit stay far inside the fp32 range.
+constexpr float WS_LAZY = 20.f;
 // register split: producer/split warpgroup, epilogue warpgroups, and the per-thread count the
 // launch must grant for it (128 x 64 + 256 x 200 = 384 x 154.7)
 constexpr int WS_REG_LO = 64, WS_REG_HI = 200, WS_REG_LAUNCH = 160;
@@ -46,7 +50,7 @@ static_assert(128 * WS_REG_LO + 256 * WS_REG_HI <= WS_THREADS * WS_REG_LAUNCH,
               "register split exceeds the launch allocation");
 
 struct WsLayout {
-    uint32_t bh, bl, kst, vst, q, qt, ss, sp, smax, ssum, sfl, sidx, bars, total;
+    uint32_t bh, bl, kst, vst, q, qt, ss, sp, smax, ssum, sfl, sidx, cs, bars, total;
     uint32_t kstage, vstage;
     int nsv;
 };
@@ -70,6 +74,7 @@ __host__ __device__ inline WsLayout ws_layout(int bf, int rV, int esz, int G, ui
                           + (uint32_t)G * 512u * 8u          // qt[2], ss[2][2], sp[2]
                           + 2u * 2u * 4u * 4u * 4u           // smax, ssum
                           + 2u * 128u * 5u                   // per-row flags and store indices
+                          + (uint32_t)G * DH * 8u            // next tile's (cos, sin) of the queries
                           + 256u + 1024u;                    // barriers, alignment slack
     int nsv = WS_MAXSV;
     while (nsv > 2 && o + nsv * L.vstage + misc > limit) --nsv;
@@ -83,6 +88,7 @@ __host__ __device__ inline WsLayout ws_layout(int bf, int rV, int esz, int G, ui
     L.ssum = o; o += 2u * 4u * 4u * 4u;
     L.sfl = o; o += 2u * 128u;                              // protection flags of the tile's rows
     L.sidx = o; o += 2u * 128u * 4u;                        // their value-store indices
+    L.cs = o; o += (uint32_t)G * DH * 8u;                   // (cos, sin) for the next q~
     L.bars = o; o += 256u;
     L.total = o + 1024u;
     return L;
@@ -137,6 +143,20 @@ __device__ __forceinline__ bool bar_and(int id, int n, bool v) {
     return r != 0;
 }
 
+// Named barrier that also returns the OR of `v` over the participating threads.
+__device__ __forceinline__ bool bar_or(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -147,6 +167,29 @@ __device__ __forceinline__ void ws_griddep_wait() { asm volatile("griddepcontrol
 __device__ __forceinline__ void ws_griddep_launch() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+
+// Tensor-memory columns: two key accumulators of 128 columns, then the per-row RoPE table (cos of
+// the 64 pairs, then their sin), 384 of the 512 allocated.
+constexpr uint32_t WS_TMEM_COLS = 512, WS_TAB = 256;
+
+// 8 consecutive fp32 columns of this thread's TMEM lane <- v (visible after tmem_wait_st).
+__device__ __forceinline__ void tmem_st8x(uint32_t taddr, const float (&v)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 8-byte asynchronous copy global -> shared (this thread waits for its own copies).
+__device__ __forceinline__ void cp_async8(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // 8 consecutive fp32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld8x(uint32_t taddr, float (&v)[8]) {
@@ -244,6 +287,16 @@ __device__ __forceinline__ void load_row8(const void *base, size_t idx, int kv_d
     }
 }
 
+// 4 consecutive channels (idx a multiple of 4) of an exact row (bf16 or fp32) as fp32.
+__device__ __forceinline__ float4 load_row4(const void *base, size_t idx, int kv_dtype) {
+    if (kv_dtype == ISKV_BF16) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(base) + idx);
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                           __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+    }
+    return *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(base) + idx);
+}
+
 // Index of `key` in the ascending array a[0 .. n), or -1.
 __device__ __forceinline__ int find_sorted(const int *a, int n, int key) {
     int lo = 0, hi = n;
@@ -320,9 +373,10 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
     float *sS = reinterpret_cast<float *>(sm + L.ss);       // [2][2 halves][G][128]
     float *sP = reinterpret_cast<float *>(sm + L.sp);       // [2][128][G]
     float *sMax = reinterpret_cast<float *>(sm + L.smax);   // [2][4][4]
-    float *sSum = reinterpret_cast<float *>(sm + L.ssum);   // [2][4][4]
+    float *sSum = reinterpret_cast<float *>(sm + L.ssum);   // [8 warps][4] probability sums
     unsigned char *sFl = sm + L.sfl;                        // [2][128] row flags (protection)
     int *sIdx = reinterpret_cast<int *>(sm + L.sidx);       // [2][128] value-store index per row
+    float2 *sCs = reinterpret_cast<float2 *>(sm + L.cs);    // [G * 64] (cos, sin) of the next tile
     float4 *sRed = reinterpret_cast<float4 *>(sm + L.qt);   // [8 warps][G][32] (aliases qt..sp)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -349,7 +403,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
         for (int i = 0; i < 8; ++i) counters[i] = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(tmem_slot, 256);
+    if (warp == 1) tmem_alloc(tmem_slot, WS_TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -545,21 +599,27 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
         const int ew = warp - 4, qw = warp & 3, hf = ew >> 2;
         const int tau = 32 * qw + lane;
         const int jb = 32 * hf;                         // first RoPE pair of this thread
-        // this row's rotation e^{i w_j tau} for the thread's 32 pairs (fixed for the kernel)
-        float tc_[32], ts_[32];
+        // this row's rotation e^{i w_j tau} for the thread's 32 pairs, fixed for the kernel, kept in
+        // the row's tensor-memory lane (cos at WS_TAB + j, sin at WS_TAB + 64 + j)
+        const uint32_t lrow = (uint32_t)(qw * 32) << 16;
+        const uint32_t ttab = tmem + WS_TAB + lrow;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            tc_[i] = 1.f;
-            ts_[i] = 0.f;
-        }
-        if (a.rope_cs != nullptr && tau < x.rope_rows) {
+        for (int c8 = 0; c8 < 4; ++c8) {
+            float cv[8], sv[8];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float2 c = a.rope_cs[(size_t)tau * DH + jb + i];
-                tc_[i] = c.x;
-                ts_[i] = c.y;
+            for (int i = 0; i < 8; ++i) {
+                cv[i] = 1.f;
+                sv[i] = 0.f;
+                if (a.rope_cs != nullptr && tau < x.rope_rows) {
+                    const float2 c = a.rope_cs[(size_t)tau * DH + jb + 8 * c8 + i];
+                    cv[i] = c.x;
+                    sv[i] = c.y;
+                }
             }
+            tmem_st8x(ttab + jb + 8 * c8, cv);
+            tmem_st8x(ttab + DH + jb + 8 * c8, sv);
         }
+        tmem_wait_st();
         ws_griddep_wait();
         const float qscale = a.scale * LOG2E;           // scores in log2 units
         // value-sum layout: thread = (quad qd, slice sl); compressed tiles use kV's quads,
@@ -602,12 +662,14 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
             const int qs = seg & 1;
             bool w = wait_ab(q_full + qs, (seg >> 1) & 1, abort_flag);
             const float *q = sQ + qs * G * D;
-            float mrun[GT], lrun[GT];
+            // m_ref (uniform), this thread's share of the probability sums (its q-heads), and the
+            // value sums, all relative to 2^m_ref
+            float mref[GT], lth[GT];
             float4 vr[GT], vw[GT];
 #pragma unroll
             for (int gg = 0; gg < GT; ++gg) {
-                mrun[gg] = -CUDART_INF_F;
-                lrun[gg] = 0.f;
+                mref[gg] = -CUDART_INF_F;
+                lth[gg] = 0.f;
                 vr[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
                 vw[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
@@ -625,8 +687,9 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 const bool comp = tl < Tc;
                 const bool prot = !comp && tl < Tc + x.Tp;       // protected exact keys
                 const long long t0 = tile_t0(tl);
-                // the next tile's query rotation: fetched now, used after the first barrier
-                const float2 cs_next = tl + 1 < tb ? load_cs(tile_t0(tl + 1)) : make_float2(1.f, 0.f);
+                // the next tile's query rotation: copied now, used after the first barrier
+                if (tl + 1 < tb && a.rope_cs != nullptr && et < G * DH)
+                    cp_async8(sCs + et, a.rope_cs + (size_t)tile_t0(tl + 1) * DH + (et & (DH - 1)));
                 int rows;
                 long long pos;
                 unsigned char fl = 0;
@@ -658,37 +721,36 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 wk = __all_sync(0xffffffffu, wk);
                 good = good && wk;
                 tc_fence_after();
-                const uint32_t trow = tmem + 128u * (at & 1) + ((uint32_t)(qw * 32) << 16);
+                const uint32_t trow = tmem + 128u * (at & 1) + lrow;
                 const bool fresh = !comp && !prot && pos == a.new_pos;
                 const void *ksrc = prot ? x.pstore[0] : fresh ? a.new_row[0] : a.ring[0];
                 const size_t kbase =
                     prot ? ((size_t)u * x.pcap + (tl - Tc) * DEC_TILE + tau) * D
                          : fresh ? (size_t)u * D : ((size_t)u * a.R + (size_t)(pos % a.R)) * D;
                 const float *qt = sQt + (size_t)b * G * D;
-                // key values of chunks (ch, ch + 1) are loaded from tensor memory together
-                float klo[2][8], khi[2][8];
+                // pairs [j0, j0 + 8) per step: key values and the row's rotation from tensor memory
+                // (collective loads: comp, prot and wk are uniform over the warp)
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int j0 = jb + 8 * ch;
-                    float lo[8], hi[8];
+                for (int cp = 0; cp < 4; ++cp) {
+                    const int j0 = jb + 8 * cp;
+                    float lo[8], hi[8], pc[8], ps[8];
+                    if (!prot) {
+                        tmem_ld8x(ttab + j0, pc);
+
+                        tmem_ld8x(ttab + DH + j0, ps);
+
+                    }
+                    if (comp && wk) {
+                        tmem_ld8x(trow + j0, lo);
+
+                        tmem_ld8x(trow + DH + j0, hi);
+
+                    }
+                    if (!prot || (comp && wk)) tmem_wait_ld();
                     if (comp) {
-                        if ((ch & 1) == 0) {
-                            if (wk) {
-                                tmem_ld8x(trow + j0, klo[0]);
-                                tmem_ld8x(trow + DH + j0, khi[0]);
-                                tmem_ld8x(trow + j0 + 8, klo[1]);
-                                tmem_ld8x(trow + DH + j0 + 8, khi[1]);
-                                tmem_wait_ld();
-                            } else {
+                        if (!wk) {
 #pragma unroll
-                                for (int i = 0; i < 8; ++i)
-                                    klo[0][i] = khi[0][i] = klo[1][i] = khi[1][i] = 0.f;
-                            }
-                        }
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            lo[i] = klo[ch & 1][i];
-                            hi[i] = khi[ch & 1][i];
+                            for (int i = 0; i < 8; ++i) lo[i] = hi[i] = 0.f;
                         }
                     } else if (valid) {
                         load_row8(ksrc, kbase + j0, a.kv_dtype, lo);
@@ -697,14 +759,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
 #pragma unroll
                         for (int i = 0; i < 8; ++i) lo[i] = hi[i] = 0.f;
                     }
-                    // a protected row's angle is its full position's (its queries are unrotated)
-                    float pc[8], ps[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        pc[i] = tc_[8 * ch + i];
-                        ps[i] = ts_[8 * ch + i];
-                    }
                     if (prot) {
+                        // a protected row's angle is its full position's (its queries are unrotated)
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             float2 cs = make_float2(1.f, 0.f);
@@ -751,56 +807,70 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     sS[((b * 2 + hf) * G + gg) * 128 + tau] = acc2[gg].x + acc2[gg].y;
                 ok = bar_and(BAR_EPI, WS_EPI, good);                     // barrier 1
                 if (!ok) break;
-                // ---- full scores; tile maxima per quarter; next tile's queries ---------------
+                // ---- full scores; next tile's queries; probabilities against m_ref ---------------
                 float sc[GT];
 #pragma unroll
-                for (int gg = 0; gg < GT; ++gg) {
+                for (int gg = 0; gg < GT; ++gg)
                     sc[gg] = valid ? sS[((b * 2 + 0) * G + gg) * 128 + tau] +
                                          sS[((b * 2 + 1) * G + gg) * 128 + tau]
                                    : -CUDART_INF_F;
-                    float m = sc[gg];
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                    if (hf == 0 && lane == 0) sMax[(b * 4 + qw) * 4 + gg] = m;
+                if (tl + 1 < tb) {
+                    float2 cs = make_float2(1.f, 0.f);
+                    if (a.rope_cs != nullptr && et < G * DH) {
+                        cp_async_wait_all();
+                        cs = sCs[et];
+                    }
+                    make_qt(q, cs, b ^ 1);
                 }
-                if (tl + 1 < tb) make_qt(q, cs_next, b ^ 1);
                 if (hf == 0) {
                     sFl[b * 128 + tau] = (unsigned char)((fl & 2) && !(fl & 1) && vidx >= 0 ? 2 : 0);
                     sIdx[b * 128 + tau] = vidx;
                 }
-                bar_named(BAR_EPI, WS_EPI);                              // barrier 2
-                float alpha[GT];
+                // each thread owns the q-heads gg with (gg & 1) == hf (both for G = 1, half 0)
+                float pv[GT];
+                bool over = false;
 #pragma unroll
                 for (int gg = 0; gg < GT; ++gg) {
-                    const float mt = fmaxf(fmaxf(sMax[(b * 4 + 0) * 4 + gg], sMax[(b * 4 + 1) * 4 + gg]),
-                                           fmaxf(sMax[(b * 4 + 2) * 4 + gg], sMax[(b * 4 + 3) * 4 + gg]));
-                    const float mn = fmaxf(mrun[gg], mt);
-                    // a tile without rows leaves the running state as it is
-                    alpha[gg] = mn == -CUDART_INF_F ? 1.f : ex2(mrun[gg] - mn);
-                    mrun[gg] = mn;
-                    if (GT == 1 ? hf == 0 : (gg & 1) == hf) {
-                        const float p = valid ? ex2(sc[gg] - mn) : 0.f;
-                        sP[(b * 128 + tau) * G + gg] = p;
-                        float s = p;
+                    const float dlt = sc[gg] - mref[gg];          // +inf or NaN while m_ref is unset
+                    over = over || (valid && !(dlt <= WS_LAZY));
+                    pv[gg] = valid ? ex2(dlt) : 0.f;
+                    if (GT == 1 ? hf == 0 : (gg & 1) == hf) sP[(b * 128 + tau) * G + gg] = pv[gg];
+                }
+                if (bar_or(BAR_EPI, WS_EPI, over)) {                      // barrier 2
+                    // some score is above m_ref + WS_LAZY (or m_ref is unset): m_ref <- the running
+                    // maximum, rescale the sums, recompute this tile's probabilities
 #pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                        if (lane == 0) sSum[(b * 4 + qw) * 4 + gg] = s;
+                    for (int gg = 0; gg < GT; ++gg) {
+                        float m = sc[gg];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                        if (hf == 0 && lane == 0) sMax[(b * 4 + qw) * 4 + gg] = m;
                     }
-                }
-                bar_named(BAR_EPI, WS_EPI);                              // barrier 3
+                    bar_named(BAR_EPI, WS_EPI);
 #pragma unroll
-                for (int gg = 0; gg < GT; ++gg) {
-                    const float s = (sSum[(b * 4 + 0) * 4 + gg] + sSum[(b * 4 + 1) * 4 + gg]) +
-                                    (sSum[(b * 4 + 2) * 4 + gg] + sSum[(b * 4 + 3) * 4 + gg]);
-                    lrun[gg] = fmaf(lrun[gg], alpha[gg], s);
-                    const float2 al = make_float2(alpha[gg], alpha[gg]);
-                    float2 x01 = __fmul2_rn(al, make_float2(vr[gg].x, vr[gg].y));
-                    float2 x23 = __fmul2_rn(al, make_float2(vr[gg].z, vr[gg].w));
-                    vr[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
-                    x01 = __fmul2_rn(al, make_float2(vw[gg].x, vw[gg].y));
-                    x23 = __fmul2_rn(al, make_float2(vw[gg].z, vw[gg].w));
-                    vw[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
+                    for (int gg = 0; gg < GT; ++gg) {
+                        const float mt = fmaxf(fmaxf(sMax[(b * 4 + 0) * 4 + gg], sMax[(b * 4 + 1) * 4 + gg]),
+                                               fmaxf(sMax[(b * 4 + 2) * 4 + gg], sMax[(b * 4 + 3) * 4 + gg]));
+                        const float mn = fmaxf(mref[gg], mt);
+                        // a tile without rows leaves the running state as it is
+                        const float alpha = mn == -CUDART_INF_F ? 1.f : ex2(mref[gg] - mn);
+                        mref[gg] = mn;
+                        lth[gg] *= alpha;
+                        const float2 al = make_float2(alpha, alpha);
+                        float2 x01 = __fmul2_rn(al, make_float2(vr[gg].x, vr[gg].y));
+                        float2 x23 = __fmul2_rn(al, make_float2(vr[gg].z, vr[gg].w));
+                        vr[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
+                        x01 = __fmul2_rn(al, make_float2(vw[gg].x, vw[gg].y));
+                        x23 = __fmul2_rn(al, make_float2(vw[gg].z, vw[gg].w));
+                        vw[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
+                        pv[gg] = valid ? ex2(sc[gg] - mn) : 0.f;
+                        if (GT == 1 ? hf == 0 : (gg & 1) == hf) sP[(b * 128 + tau) * G + gg] = pv[gg];
+                    }
+                    bar_named(BAR_EPI, WS_EPI);
                 }
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg)
+                    if (GT == 1 ? hf == 0 : (gg & 1) == hf) lth[gg] += pv[gg];
                 // ---- value sums: v_g += sum_i p[g][i] V[i][quad] ----------------------------
                 const int vs = vt % NSV;
                 const bool wv = prot ? true : wait_ab(v_full + vs, (vt / NSV) & 1, abort_flag);
@@ -812,10 +882,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     for (int i = slw; i < rows; i += 8) {
                         const int vi = sIdx[b * 128 + i];
                         if (vi < 0) continue;
-                        float t8[8];
-                        load_row8(x.pstore[1], ((size_t)u * x.pcap + vi) * D + (4 * qdw & ~7), a.kv_dtype, t8);
-                        const int o4 = (4 * qdw) & 7;
-                        const float2 v01 = make_float2(t8[o4], t8[o4 + 1]), v23 = make_float2(t8[o4 + 2], t8[o4 + 3]);
+                        const float4 v4 = load_row4(x.pstore[1], ((size_t)u * x.pcap + vi) * D + 4 * qdw, a.kv_dtype);
+                        const float2 v01 = make_float2(v4.x, v4.y), v23 = make_float2(v4.z, v4.w);
                         float pv[GT];
                         load_p(P + i * G, pv);
 #pragma unroll
@@ -833,10 +901,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         for (int i = slw; i < rows; i += 8) {
                             if (!(sFl[b * 128 + i] & 2)) continue;
                             const int vi = sIdx[b * 128 + i];
-                            float t8[8];
-                            load_row8(x.pstore[1], ((size_t)u * x.pcap + vi) * D + (4 * qdw & ~7), a.kv_dtype, t8);
-                            const int o4 = (4 * qdw) & 7;
-                            const float2 v01 = make_float2(t8[o4], t8[o4 + 1]), v23 = make_float2(t8[o4 + 2], t8[o4 + 3]);
+                            const float4 v4 = load_row4(x.pstore[1], ((size_t)u * x.pcap + vi) * D + 4 * qdw, a.kv_dtype);
+                            const float2 v01 = make_float2(v4.x, v4.y), v23 = make_float2(v4.z, v4.w);
                             float pv[GT];
                             load_p(P + i * G, pv);
 #pragma unroll
@@ -873,10 +939,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         for (int i = slw; i < rows; i += 8) {
                             float4 v;
                             if (i == inew) {
-                                float t8[8];
-                                load_row8(a.new_row[1], (size_t)u * D + (4 * qdw & ~7), a.kv_dtype, t8);
-                                const int o4 = (4 * qdw) & 7;
-                                v = make_float4(t8[o4], t8[o4 + 1], t8[o4 + 2], t8[o4 + 3]);
+                                v = load_row4(a.new_row[1], (size_t)u * D + 4 * qdw, a.kv_dtype);
                             } else {
                                 v = load_v4s(V + (size_t)i * vld, 4 * qdw, esz);
                             }
@@ -966,12 +1029,24 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 for (int o = et; o < G * D; o += WS_EPI)
                     rec[(o / D) * (2 + rV + D) + 2 + rV + o % D] = 0.f;
             }
+            // probability sums: per warp, then over the 8 epilogue warps
+#pragma unroll
+            for (int gg = 0; gg < GT; ++gg) {
+                float sl = lth[gg];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) sl += __shfl_xor_sync(0xffffffffu, sl, o);
+                if (lane == 0) sSum[ew * 4 + gg] = sl;
+            }
+            bar_named(BAR_EPI, WS_EPI);
             if (et < G) {
 #pragma unroll
                 for (int gg = 0; gg < GT; ++gg)
                     if (gg == et) {
-                        rec[gg * (2 + rV + D)] = mrun[gg];
-                        rec[gg * (2 + rV + D) + 1] = lrun[gg];
+                        float l = 0.f;
+#pragma unroll
+                        for (int w8 = 0; w8 < 8; ++w8) l += sSum[w8 * 4 + gg];
+                        rec[gg * (2 + rV + D)] = mref[gg];
+                        rec[gg * (2 + rV + D) + 1] = l;
                     }
             }
         }
@@ -1003,7 +1078,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, WS_TMEM_COLS);
     }
 }
 

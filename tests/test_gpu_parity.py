@@ -552,12 +552,13 @@ def test_bf16_coordinates_fold_one_step_parity(variant, wl_id):
                 bound = 2.0 ** -8 * np.abs(got) + PROJ_TOL * row + 1e-30
                 worst["excess"] = max(worst["excess"], float((np.abs(got - Cr) / bound).max()))
                 worst["mismatch"] = max(worst["mismatch"], float(np.mean(got != E)))
-                # round to nearest leaves no sign bias relative to the bf16 step
-                rel = np.sign(got) * (got - Cr) / (2.0 ** -8 * np.abs(got) + 1e-30)
-                worst["bias"] = max(worst["bias"], abs(float(rel[np.abs(got) > 0].mean())))
+                # round to nearest leaves no bias toward zero relative to the bf16 step; truncation
+                # would give about -0.7 here (error uniform over one step, toward zero)
+                bias = float(np.sum(np.sign(got) * (got - Cr)) / (2.0 ** -8 * np.sum(np.abs(got))))
+                worst["bias"] = max(worst["bias"], abs(bias))
     print(f"\nbf16 coordinates {variant} cfg {wl_id}: {folds} folds, worst {worst}")
     assert worst["sigma"] <= SIG_TOL and worst["proj"] <= PROJ_TOL
-    assert worst["excess"] <= 1.0 and worst["mismatch"] <= 0.1 and worst["bias"] <= 0.1
+    assert worst["excess"] <= 1.0 and worst["mismatch"] <= 0.1 and worst["bias"] <= 0.25
     assert cache.status() == 0
 
 
