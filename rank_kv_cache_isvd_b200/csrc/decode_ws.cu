@@ -111,11 +111,15 @@ __device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// Bounded wait that also gives up as soon as another role raised the abort flag.
-__device__ __forceinline__ bool wait_ab(uint64_t *bar, uint32_t parity, volatile int *abort) {
+// Bounded wait that also gives up as soon as another role raised the abort flag. The producer and
+// MMA warps (nap) sleep briefly between polls, leaving issue slots to the epilogue warps that share
+// their schedulers.
+__device__ __forceinline__ bool wait_ab(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                        bool nap = false) {
     for (uint32_t i = 0; i < MBAR_SPIN_LIMIT; ++i) {
         if (mbar_try(bar, parity)) return true;
         if (*abort) return false;
+        if (nap) __nanosleep(64);
     }
     *abort = 1;
     return false;
@@ -427,6 +431,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
     if (warp == 0) {
         // ==================================== producer ===========================================
         int kt = 0, vt = 0, seg = 0, bseg = 0;
+        int vs = 0;                                     // V stage of tile vt, and its pass parity
+        uint32_t vph = 0;
         ws_griddep_wait();
         if (lane == 0) {
             bool ok = true;
@@ -437,7 +443,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 const int seq = (int)(u / a.H), h = (int)(u % a.H);
                 // queries of this unit's q-heads
                 const int qs = seg & 1;
-                ok = wait_ab(q_empty + qs, ((seg >> 1) & 1) ^ 1, abort_flag);
+                ok = wait_ab(q_empty + qs, ((seg >> 1) & 1) ^ 1, abort_flag, true);
                 if (!ok) break;
                 mbar_arrive_expect_tx(q_full + qs, (uint32_t)(G * D * 4));
                 bulk_load(sQ + qs * G * D, a.q + ((size_t)seq * a.H * G + (size_t)h * G) * D,
@@ -446,7 +452,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 counters[0] = seg;
                 if (!BF && ta < Tc) {
                     // B_K of this unit (one buffer; free once the previous segment's MMAs are done)
-                    ok = wait_ab(b_empty, (bseg & 1) ^ 1, abort_flag);
+                    ok = wait_ab(b_empty, (bseg & 1) ^ 1, abort_flag, true);
                     if (!ok) break;
                     mbar_arrive_expect_tx(b_full, WS_BLK);
                     tma_load_2d(sm + L.bh, &tmB, 0, x.brow0 + (int)u * D, b_full);
@@ -462,7 +468,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         t0 = (long long)tl * DEC_TILE;
                         rows = (int)min((long long)DEC_TILE, a.n_c - t0);
                         const int ks = kt % WS_NSK;
-                        ok = wait_ab(k_empty + ks, ((kt / WS_NSK) & 1) ^ 1, abort_flag);
+                        ok = wait_ab(k_empty + ks, ((kt / WS_NSK) & 1) ^ 1, abort_flag, true);
                         if (!ok) break;
                         mbar_arrive_expect_tx(k_full + ks, WS_BLK);
                         tma_load_2d(sm + L.kst + ks * L.kstage, &tmC, 0,
@@ -473,8 +479,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         t0 = a.n_c + (long long)(tl - Tc - x.Tp) * DEC_TILE;
                         rows = (int)min((long long)DEC_TILE, a.t - t0);
                     }
-                    const int vs = vt % NSV;
-                    ok = wait_ab(v_empty + vs, ((vt / NSV) & 1) ^ 1, abort_flag);
+                    ok = wait_ab(v_empty + vs, vph ^ 1, abort_flag, true);
                     if (!ok) break;
                     uint8_t *dst = sm + L.vst + vs * L.vstage;
                     if (comp) {
@@ -497,6 +502,10 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                                       v_full + vs);
                     }
                     ++vt;
+                    if (++vs == NSV) {
+                        vs = 0;
+                        vph ^= 1;
+                    }
                     counters[3] = vt;
                 }
                 g += tb - ta;
@@ -519,14 +528,14 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
             if (BF) {
                 // three bf16 terms of this unit's fp32 basis, written in the 128-byte-swizzled
                 // K-major layout, once the previous segment's MMAs no longer read them
-                w = wait_ab(b_empty, (bseg & 1) ^ 1, abort_flag);
+                w = wait_ab(b_empty, (bseg & 1) ^ 1, abort_flag, true);
                 if (w) {
                     build_b_terms(sm + L.bh, sm + L.bl, sm + L.bl + WS_BLK,
                                   a.basis[0] + (size_t)u * D * a.r[0], a.r[0], st, 96);
                     fence_proxy_async_smem();
                 }
             } else {
-                w = wait_ab(b_full, bseg & 1, abort_flag);
+                w = wait_ab(b_full, bseg & 1, abort_flag, true);
                 if (w) {
                     split_tf32_range(sm + L.bh, sm + L.bl, WS_BLK, st, 96);
                     fence_proxy_async_smem();
@@ -539,7 +548,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
             for (int tl = ta; tl < te; ++tl) {
                 const int ks = kt % WS_NSK;
                 uint8_t *A = sm + L.kst + ks * L.kstage;
-                w = wait_ab(k_full + ks, (kt / WS_NSK) & 1, abort_flag);
+                w = wait_ab(k_full + ks, (kt / WS_NSK) & 1, abort_flag, true);
                 if (!BF && w) {
                     split_tf32_range(A, A + WS_BLK, WS_BLK, st, 96);
                     fence_proxy_async_smem();
@@ -548,7 +557,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 if (!ok) break;
                 if (st == 0) {
                     const int buf = at & 1;
-                    bool e = wait_ab(acc_empty + buf, ((at >> 1) & 1) ^ 1, abort_flag);
+                    bool e = wait_ab(acc_empty + buf, ((at >> 1) & 1) ^ 1, abort_flag, true);
                     if (e) {
                         tc_fence_after();
                         const uint32_t d = tmem + 128u * buf;
@@ -630,6 +639,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
         const int qdw = et & 31, slw = et >> 5;
         bool ok = true;
         int at = 0, vt = 0, seg = 0, it = 0;
+        int vs = 0;                                     // V stage of tile vt, and its pass parity
+        uint32_t vph = 0;
 
         // start position of tile tl of a unit: compressed, protected (queries unrotated: each
         // protected row carries its own angle), window
@@ -722,15 +733,20 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 good = good && wk;
                 tc_fence_after();
                 const uint32_t trow = tmem + 128u * (at & 1) + lrow;
-                const bool fresh = !comp && !prot && pos == a.new_pos;
-                const void *ksrc = prot ? x.pstore[0] : fresh ? a.new_row[0] : a.ring[0];
-                const size_t kbase =
-                    prot ? ((size_t)u * x.pcap + (tl - Tc) * DEC_TILE + tau) * D
-                         : fresh ? (size_t)u * D : ((size_t)u * a.R + (size_t)(pos % a.R)) * D;
-                const float *qt = sQt + (size_t)b * G * D;
+                // exact key rows (protected or window tiles): source and first element
+                const void *ksrc = nullptr;
+                size_t kbase = 0;
+                if (!comp) {
+                    const bool fresh = !prot && pos == a.new_pos;
+                    ksrc = prot ? x.pstore[0] : fresh ? a.new_row[0] : a.ring[0];
+                    kbase = prot ? ((size_t)u * x.pcap + (tl - Tc) * DEC_TILE + tau) * D
+                                 : fresh ? (size_t)u * D
+                                         : ((size_t)u * a.R + (unsigned)pos % (unsigned)a.R) * D;
+                }
+                const float *qt = sQt + b * G * D;
                 // pairs [j0, j0 + 8) per step: key values and the row's rotation from tensor memory
                 // (collective loads: comp, prot and wk are uniform over the warp)
-#pragma unroll
+#pragma unroll 1
                 for (int cp = 0; cp < 4; ++cp) {
                     const int j0 = jb + 8 * cp;
                     float lo[8], hi[8], pc[8], ps[8];
@@ -872,8 +888,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 for (int gg = 0; gg < GT; ++gg)
                     if (GT == 1 ? hf == 0 : (gg & 1) == hf) lth[gg] += pv[gg];
                 // ---- value sums: v_g += sum_i p[g][i] V[i][quad] ----------------------------
-                const int vs = vt % NSV;
-                const bool wv = prot ? true : wait_ab(v_full + vs, (vt / NSV) & 1, abort_flag);
+                const bool wv = prot ? true : wait_ab(v_full + vs, vph, abort_flag);
                 good = good && wv;
                 const uint8_t *V = sm + L.vst + vs * L.vstage;
                 const float *P = sP + (size_t)b * 128 * G;
@@ -976,6 +991,10 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 if (!prot) {
                     if (lane == 0) mbar_arrive(v_empty + vs);
                     ++vt;
+                    if (++vs == NSV) {
+                        vs = 0;
+                        vph ^= 1;
+                    }
                 }
                 ++it;
             }
