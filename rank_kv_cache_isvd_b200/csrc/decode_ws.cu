@@ -111,15 +111,30 @@ __device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// Bounded wait that also gives up as soon as another role raised the abort flag. The producer and
-// MMA warps (nap) sleep briefly between polls, leaving issue slots to the epilogue warps that share
-// their schedulers.
+// try_wait that may suspend the thread for up to `ns` nanoseconds while the phase is incomplete
+// (the thread resumes as soon as it completes), so that waiting warps issue almost nothing.
+__device__ __forceinline__ bool mbar_try_for(uint64_t *bar, uint32_t parity, uint32_t ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return done != 0;
+}
+
+// Polls of a suspending wait before it gives up: each poll suspends for at most WS_SUSPEND_NS, and
+// 2^18 polls of even a microsecond are far longer than any launch.
+constexpr uint32_t WS_POLL_LIMIT = 1u << 18, WS_SUSPEND_NS = 20000;
+
+// Bounded wait that also gives up as soon as another role raised the abort flag.
 __device__ __forceinline__ bool wait_ab(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                        bool nap = false) {
-    for (uint32_t i = 0; i < MBAR_SPIN_LIMIT; ++i) {
-        if (mbar_try(bar, parity)) return true;
+                                        bool = false) {
+    for (uint32_t i = 0; i < WS_POLL_LIMIT; ++i) {
+        if (mbar_try_for(bar, parity, WS_SUSPEND_NS)) return true;
         if (*abort) return false;
-        if (nap) __nanosleep(64);
     }
     *abort = 1;
     return false;
@@ -187,6 +202,25 @@ __device__ __forceinline__ void tmem_st8x(uint32_t taddr, const float (&v)[8]) {
 }
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// One 16-lane x 8-column block of tensor memory in the 16x256b fragment: thread t holds (lane
+// t/4, columns 2(t%4) and 2(t%4)+1) in v[0], v[1] and (lane t/4 + 8, the same columns) in v[2],
+// v[3]; taddr addresses the block's first lane and column.
+__device__ __forceinline__ void tmem_ld4f(uint32_t taddr, float (&v)[4]) {
+    uint32_t r[4];
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st4f(uint32_t taddr, const float (&v)[4]) {
+    asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
+                 "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                 "r"(__float_as_uint(v[3]))
+                 : "memory");
 }
 
 // 8-byte asynchronous copy global -> shared (this thread waits for its own copies).
@@ -606,27 +640,35 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
         // ==================================== epilogue ===========================================
         const int et = tid - 128;                       // 0 .. 255
         const int ew = warp - 4, qw = warp & 3, hf = ew >> 2;
-        const int tau = 32 * qw + lane;
-        const int jb = 32 * hf;                         // first RoPE pair of this thread
-        // this row's rotation e^{i w_j tau} for the thread's 32 pairs, fixed for the kernel, kept in
-        // the row's tensor-memory lane (cos at WS_TAB + j, sin at WS_TAB + 64 + j)
-        const uint32_t lrow = (uint32_t)(qw * 32) << 16;
-        const uint32_t ttab = tmem + WS_TAB + lrow;
+        // Key phase: the warp covers its lane quarter's 32 rows and the pairs [jb, jb + 32); thread
+        // t = (r0, q4) handles rows 32 qw + r0 + 8 m (m = 0 .. 3) and, in every 8-pair group
+        // [j0, j0 + 8), the pairs j0 + 2 q4 and j0 + 2 q4 + 1 (the 16x256b fragment), so each query
+        // value read from shared memory serves four rows. After a quad reduction the thread owns
+        // row tau = 32 qw + r0 + 8 q4 for the softmax.
+        const int q4 = lane & 3, r0 = lane >> 2;
+        const int tau = 32 * qw + r0 + 8 * q4;
+        const int jb = 32 * hf;                         // first RoPE pair of this warp
+        const uint32_t lane0 = (uint32_t)(qw * 32) << 16, lane16 = (uint32_t)(qw * 32 + 16) << 16;
+        // row m's rotation e^{i w_j tau_m} for the thread's pairs, fixed for the kernel, kept in
+        // tensor memory next to the key accumulators (cos at WS_TAB + j, sin at WS_TAB + 64 + j)
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-            float cv[8], sv[8];
+        for (int lh = 0; lh < 2; ++lh) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                cv[i] = 1.f;
-                sv[i] = 0.f;
-                if (a.rope_cs != nullptr && tau < x.rope_rows) {
-                    const float2 c = a.rope_cs[(size_t)tau * DH + jb + 8 * c8 + i];
-                    cv[i] = c.x;
-                    sv[i] = c.y;
+            for (int k = 0; k < 4; ++k) {
+                float cv[4], sv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int row = 32 * qw + 16 * lh + r0 + 8 * (e >> 1);
+                    const int j = jb + 8 * k + 2 * q4 + (e & 1);
+                    float2 c = make_float2(1.f, 0.f);
+                    if (a.rope_cs != nullptr && row < x.rope_rows) c = a.rope_cs[(size_t)row * DH + j];
+                    cv[e] = c.x;
+                    sv[e] = c.y;
                 }
+                const uint32_t tl0 = tmem + WS_TAB + (lh ? lane16 : lane0) + jb + 8 * k;
+                tmem_st4f(tl0, cv);
+                tmem_st4f(tl0 + DH, sv);
             }
-            tmem_st8x(ttab + jb + 8 * c8, cv);
-            tmem_st8x(ttab + DH + jb + 8 * c8, sv);
         }
         tmem_wait_st();
         ws_griddep_wait();
@@ -723,91 +765,112 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 const bool valid = tau < rows && !(fl & 1);
                 // ---- this row's key: pairs (j, j + 64), j in [jb, jb + 32), chunks of 8 pairs,
                 //      rotated by e^{i w_j tau} and dotted with the rotated queries ----------------
-                float2 acc2[GT];
+                // partial scores of the thread's four rows over its pairs (float2: two pairs)
+                float2 acc[4][GT];
 #pragma unroll
-                for (int gg = 0; gg < GT; ++gg) acc2[gg] = make_float2(0.f, 0.f);
+                for (int m = 0; m < 4; ++m)
+#pragma unroll
+                    for (int gg = 0; gg < GT; ++gg) acc[m][gg] = make_float2(0.f, 0.f);
                 bool wk = true;
                 if (comp) wk = wait_ab(acc_full + (at & 1), (at >> 1) & 1, abort_flag);
                 // the tensor-memory loads below are warp-collective: decide per warp
                 wk = __all_sync(0xffffffffu, wk);
                 good = good && wk;
                 tc_fence_after();
-                const uint32_t trow = tmem + 128u * (at & 1) + lrow;
-                // exact key rows (protected or window tiles): source and first element
-                const void *ksrc = nullptr;
-                size_t kbase = 0;
-                if (!comp) {
-                    const bool fresh = !prot && pos == a.new_pos;
-                    ksrc = prot ? x.pstore[0] : fresh ? a.new_row[0] : a.ring[0];
-                    kbase = prot ? ((size_t)u * x.pcap + (tl - Tc) * DEC_TILE + tau) * D
-                                 : fresh ? (size_t)u * D
-                                         : ((size_t)u * a.R + (unsigned)pos % (unsigned)a.R) * D;
-                }
                 const float *qt = sQt + b * G * D;
-                // pairs [j0, j0 + 8) per step: key values and the row's rotation from tensor memory
-                // (collective loads: comp, prot and wk are uniform over the warp)
+                // exact key rows (protected or window tiles): the thread's four rows
+                int xrows = 0;
+                if (!comp) {
+                    const int pi = prot ? (tl - Tc) * DEC_TILE : 0;
+                    xrows = prot ? max(0, min(DEC_TILE, npk - pi)) : (int)min((long long)DEC_TILE, a.t - t0);
+                }
 #pragma unroll 1
-                for (int cp = 0; cp < 4; ++cp) {
-                    const int j0 = jb + 8 * cp;
-                    float lo[8], hi[8], pc[8], ps[8];
-                    if (!prot) {
-                        tmem_ld8x(ttab + j0, pc);
-
-                        tmem_ld8x(ttab + DH + j0, ps);
-
-                    }
-                    if (comp && wk) {
-                        tmem_ld8x(trow + j0, lo);
-
-                        tmem_ld8x(trow + DH + j0, hi);
-
-                    }
-                    if (!prot || (comp && wk)) tmem_wait_ld();
+                for (int k = 0; k < 4; ++k) {
+                    const int j0 = jb + 8 * k;
+                    // [m][two pairs]: key real parts, imaginary parts, cos, sin
+                    float kr[4][2], ki[4][2], cc[4][2], ss[4][2];
                     if (comp) {
+                        float t4[4];
+                        const uint32_t acc0 = tmem + 128u * (at & 1);
+#pragma unroll
+                        for (int lh = 0; lh < 2; ++lh) {
+                            const uint32_t ln = lh ? lane16 : lane0;
+                            tmem_ld4f(tmem + WS_TAB + ln + j0, t4);
+                            cc[2 * lh][0] = t4[0]; cc[2 * lh][1] = t4[1]; cc[2 * lh + 1][0] = t4[2]; cc[2 * lh + 1][1] = t4[3];
+                            tmem_ld4f(tmem + WS_TAB + ln + DH + j0, t4);
+                            ss[2 * lh][0] = t4[0]; ss[2 * lh][1] = t4[1]; ss[2 * lh + 1][0] = t4[2]; ss[2 * lh + 1][1] = t4[3];
+                            if (wk) {
+                                tmem_ld4f(acc0 + ln + j0, t4);
+                                kr[2 * lh][0] = t4[0]; kr[2 * lh][1] = t4[1]; kr[2 * lh + 1][0] = t4[2]; kr[2 * lh + 1][1] = t4[3];
+                                tmem_ld4f(acc0 + ln + DH + j0, t4);
+                                ki[2 * lh][0] = t4[0]; ki[2 * lh][1] = t4[1]; ki[2 * lh + 1][0] = t4[2]; ki[2 * lh + 1][1] = t4[3];
+                            }
+                        }
+                        tmem_wait_ld();
                         if (!wk) {
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) lo[i] = hi[i] = 0.f;
+                            for (int m = 0; m < 4; ++m) kr[m][0] = kr[m][1] = ki[m][0] = ki[m][1] = 0.f;
                         }
-                    } else if (valid) {
-                        load_row8(ksrc, kbase + j0, a.kv_dtype, lo);
-                        load_row8(ksrc, kbase + DH + j0, a.kv_dtype, hi);
                     } else {
+                        // rows from the exact stores; protected rows rotate by their full position
+                        // (their queries are unrotated), window rows by their offset in the tile
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) lo[i] = hi[i] = 0.f;
-                    }
-                    if (prot) {
-                        // a protected row's angle is its full position's (its queries are unrotated)
+                        for (int m = 0; m < 4; ++m) {
+                            const int row = 32 * qw + r0 + 8 * m;
+                            kr[m][0] = kr[m][1] = ki[m][0] = ki[m][1] = 0.f;
+                            cc[m][0] = cc[m][1] = 1.f;
+                            ss[m][0] = ss[m][1] = 0.f;
+                            if (row < xrows) {
+                                const void *src;
+                                size_t base;
+                                long long apos;
+                                if (prot) {
+                                    const size_t pidx = (size_t)u * x.pcap + (tl - Tc) * DEC_TILE + row;
+                                    src = x.pstore[0];
+                                    base = pidx * D;
+                                    apos = x.ppos[0][pidx];
+                                } else {
+                                    const long long p = t0 + row;
+                                    const bool fresh = p == a.new_pos;
+                                    src = fresh ? a.new_row[0] : a.ring[0];
+                                    base = fresh ? (size_t)u * D
+                                                 : ((size_t)u * a.R + (unsigned)p % (unsigned)a.R) * D;
+                                    apos = row;
+                                }
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            float2 cs = make_float2(1.f, 0.f);
-                            if (a.rope_cs != nullptr && valid) cs = a.rope_cs[(size_t)pos * DH + j0 + i];
-                            pc[i] = cs.x;
-                            ps[i] = cs.y;
+                                for (int e = 0; e < 2; ++e) {
+                                    const int j = j0 + 2 * q4 + e;
+                                    kr[m][e] = load_row_elem(src, base + j, a.kv_dtype);
+                                    ki[m][e] = load_row_elem(src, base + DH + j, a.kv_dtype);
+                                    if (a.rope_cs != nullptr) {
+                                        const float2 c = a.rope_cs[(size_t)apos * DH + j];
+                                        cc[m][e] = c.x;
+                                        ss[m][e] = c.y;
+                                    }
+                                }
+                            }
                         }
                     }
+                    // queries of the two pairs, then rotate each row's key and dot
+                    float2 qre[GT], qim[GT];
 #pragma unroll
-                    for (int i4 = 0; i4 < 2; ++i4) {
-                        // four pairs: rotate the key by e^{i w tau}, then dot with each rotated query
-                        float2 zr[2], zi[2];
+                    for (int gg = 0; gg < GT; ++gg) {
+                        qre[gg] = *reinterpret_cast<const float2 *>(qt + gg * D + j0 + 2 * q4);
+                        qim[gg] = *reinterpret_cast<const float2 *>(qt + gg * D + DH + j0 + 2 * q4);
+                    }
 #pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) {
-                            const int i = 2 * i4 + h2;
-                            const float2 k1 = make_float2(lo[2 * i], lo[2 * i + 1]);
-                            const float2 k2 = make_float2(hi[2 * i], hi[2 * i + 1]);
-                            const float2 c2 = make_float2(pc[2 * i], pc[2 * i + 1]);
-                            const float2 s2 = make_float2(ps[2 * i], ps[2 * i + 1]);
-                            const float2 t1 = __fmul2_rn(k2, s2);
-                            zr[h2] = __ffma2_rn(k1, c2, make_float2(-t1.x, -t1.y));
-                            zi[h2] = __ffma2_rn(k1, s2, __fmul2_rn(k2, c2));
-                        }
+                    for (int m = 0; m < 4; ++m) {
+                        const float2 k1 = make_float2(kr[m][0], kr[m][1]);
+                        const float2 k2 = make_float2(ki[m][0], ki[m][1]);
+                        const float2 c2 = make_float2(cc[m][0], cc[m][1]);
+                        const float2 s2 = make_float2(ss[m][0], ss[m][1]);
+                        const float2 t1 = __fmul2_rn(k2, s2);
+                        const float2 zr = __ffma2_rn(k1, c2, make_float2(-t1.x, -t1.y));
+                        const float2 zi = __ffma2_rn(k1, s2, __fmul2_rn(k2, c2));
 #pragma unroll
                         for (int gg = 0; gg < GT; ++gg) {
-                            const float4 qr = *reinterpret_cast<const float4 *>(qt + gg * D + j0 + 4 * i4);
-                            const float4 qi = *reinterpret_cast<const float4 *>(qt + gg * D + DH + j0 + 4 * i4);
-                            acc2[gg] = __ffma2_rn(make_float2(qr.x, qr.y), zr[0], acc2[gg]);
-                            acc2[gg] = __ffma2_rn(make_float2(qi.x, qi.y), zi[0], acc2[gg]);
-                            acc2[gg] = __ffma2_rn(make_float2(qr.z, qr.w), zr[1], acc2[gg]);
-                            acc2[gg] = __ffma2_rn(make_float2(qi.z, qi.w), zi[1], acc2[gg]);
+                            acc[m][gg] = __ffma2_rn(qre[gg], zr, acc[m][gg]);
+                            acc[m][gg] = __ffma2_rn(qim[gg], zi, acc[m][gg]);
                         }
                     }
                 }
@@ -818,9 +881,27 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     if (lane == 0 && wk) mbar_arrive(acc_empty + (at & 1));
                     ++at;
                 }
+                // quad reduction: thread q4 ends with row m = q4 (tile row tau) summed over the
+                // warp's 32 pairs
+                {
+                    float s1[2][GT];
+                    const bool hi2 = (q4 & 2) != 0;
 #pragma unroll
-                for (int gg = 0; gg < GT; ++gg)
-                    sS[((b * 2 + hf) * G + gg) * 128 + tau] = acc2[gg].x + acc2[gg].y;
+                    for (int i = 0; i < 2; ++i)
+#pragma unroll
+                        for (int gg = 0; gg < GT; ++gg) {
+                            const float lo_s = acc[i][gg].x + acc[i][gg].y;
+                            const float hi_s = acc[2 + i][gg].x + acc[2 + i][gg].y;
+                            const float keep = hi2 ? hi_s : lo_s, send = hi2 ? lo_s : hi_s;
+                            s1[i][gg] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                        }
+                    const bool odd = (q4 & 1) != 0;
+#pragma unroll
+                    for (int gg = 0; gg < GT; ++gg) {
+                        const float keep = odd ? s1[1][gg] : s1[0][gg], send = odd ? s1[0][gg] : s1[1][gg];
+                        sS[((b * 2 + hf) * G + gg) * 128 + tau] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                    }
+                }
                 ok = bar_and(BAR_EPI, WS_EPI, good);                     // barrier 1
                 if (!ok) break;
                 // ---- full scores; next tile's queries; probabilities against m_ref ---------------
