@@ -37,7 +37,7 @@ constexpr int WS_EPI = 256;                  // epilogue threads (warps 4 .. 11)
 constexpr int WS_NSK = 2;                    // key-coordinate stages
 constexpr int WS_MAXSV = 4;                  // value stages (at most)
 constexpr uint32_t WS_BLK = 128u * 128u;     // 128 rows x 128 bytes
-constexpr int BAR_EPI = 1, BAR_SPLIT = 2;    // named barriers
+constexpr int BAR_EPI = 1, BAR_SPLIT = 3, BAR_ALL = 4;   // named barriers (groups: 1 and 2)
 constexpr float LOG2E = 1.4426950408889634f;
 // Lazy softmax reference: probabilities are 2^(s - m_ref) with m_ref a CTA-uniform running
 // reference that moves only when a score exceeds it by more than WS_LAZY (log2 units), so that
@@ -50,14 +50,14 @@ static_assert(128 * WS_REG_LO + 256 * WS_REG_HI <= WS_THREADS * WS_REG_LAUNCH,
               "register split exceeds the launch allocation");
 
 struct WsLayout {
-    uint32_t bh, bl, kst, vst, q, qt, ss, sp, smax, ssum, sfl, sidx, cs, bars, total;
+    uint32_t bh, bl, kst, vst, q, eg, smax, ssum, sfl, sidx, cs, bars, total;
     uint32_t kstage, vstage;
     int nsv;
 };
 
 // Shared-memory plan. fp32 coordinates: a K stage holds the tile's tf32 hi part (in place) and its
-// lo part; bf16 coordinates: the tile only (exact bf16 operands). The reduction area of the partial records aliases the
-// per-tile buffers qt, ss and sp (free at the end of a segment).
+// lo part; bf16 coordinates: the tile only (exact bf16 operands). Each epilogue group owns an area
+// of q~ [2][G][128] and p [2][128][G] floats (its segment-end reduction aliases it).
 __host__ __device__ inline WsLayout ws_layout(int bf, int rV, int esz, int G, uint32_t limit) {
     WsLayout L;
     uint32_t o = 0;
@@ -71,25 +71,23 @@ __host__ __device__ inline WsLayout ws_layout(int bf, int rV, int esz, int G, ui
     L.vstage = ((vc > vw ? vc : vw) + 1023u) & ~1023u;
     L.vst = o;
     const uint32_t misc = (uint32_t)G * 512u * 2u            // q, two segment slots
-                          + (uint32_t)G * 512u * 8u          // qt[2], ss[2][2], sp[2]
-                          + 2u * 2u * 4u * 4u * 4u           // smax, ssum
-                          + 2u * 128u * 5u                   // per-row flags and store indices
-                          + (uint32_t)G * DH * 8u            // next tile's (cos, sin) of the queries
-                          + 256u + 1024u;                    // barriers, alignment slack
+                          + (uint32_t)G * 4096u              // the two groups' areas
+                          + 64u * 4u + 32u * 4u              // smax, ssum
+                          + 2u * 2u * 128u * 5u              // per-row flags and store indices
+                          + 2u * (uint32_t)G * DH * 8u       // next tiles' (cos, sin) of the queries
+                          + 512u + 1024u;                    // barriers, alignment slack
     int nsv = WS_MAXSV;
     while (nsv > 2 && o + nsv * L.vstage + misc > limit) --nsv;
     L.nsv = nsv;
     o += nsv * L.vstage;
     L.q = o; o += G * 512u * 2u;
-    L.qt = o; o += G * 512u * 2u;
-    L.ss = o; o += G * 512u * 4u;
-    L.sp = o; o += G * 512u * 2u;
-    L.smax = o; o += 2u * 4u * 4u * 4u;
-    L.ssum = o; o += 2u * 4u * 4u * 4u;
-    L.sfl = o; o += 2u * 128u;                              // protection flags of the tile's rows
-    L.sidx = o; o += 2u * 128u * 4u;                        // their value-store indices
-    L.cs = o; o += (uint32_t)G * DH * 8u;                   // (cos, sin) for the next q~
-    L.bars = o; o += 256u;
+    L.eg = o; o += G * 4096u;
+    L.smax = o; o += 64u * 4u;
+    L.ssum = o; o += 32u * 4u;
+    L.sfl = o; o += 2u * 2u * 128u;                         // protection flags of the tiles' rows
+    L.sidx = o; o += 2u * 2u * 128u * 4u;                   // their value-store indices
+    L.cs = o; o += 2u * (uint32_t)G * DH * 8u;              // (cos, sin) for the groups' next q~
+    L.bars = o; o += 512u;
     L.total = o + 1024u;
     return L;
 }
@@ -365,6 +363,20 @@ __device__ __forceinline__ void load_p(const float *p, float (&v)[GT]) {
     }
 }
 
+// The G probabilities of one row, stored (the row's G floats are 4 G bytes apart: 16-byte aligned
+// for G = 4).
+template <int GT>
+__device__ __forceinline__ void store_p(float *p, const float (&v)[GT]) {
+    if constexpr (GT == 4) {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    } else if constexpr (GT == 2) {
+        *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+    } else {
+#pragma unroll
+        for (int g = 0; g < GT; ++g) p[g] = v[g];
+    }
+}
+
 // Four consecutive values of a staged value row: fmt 2 = bf16, 4 = fp32.
 __device__ __forceinline__ float4 load_v4s(const uint8_t *row, int c, int fmt) {
     if (fmt == 2) {
@@ -407,15 +419,11 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 23);
     int *counters = reinterpret_cast<int *>(bars + 24);    // [8] progress, read at teardown
     float *sQ = reinterpret_cast<float *>(sm + L.q);        // [2 slots][G][128]
-    float *sQt = reinterpret_cast<float *>(sm + L.qt);      // [2][G][128] rotated, scaled
-    float *sS = reinterpret_cast<float *>(sm + L.ss);       // [2][2 halves][G][128]
-    float *sP = reinterpret_cast<float *>(sm + L.sp);       // [2][128][G]
-    float *sMax = reinterpret_cast<float *>(sm + L.smax);   // [2][4][4]
-    float *sSum = reinterpret_cast<float *>(sm + L.ssum);   // [8 warps][4] probability sums
-    unsigned char *sFl = sm + L.sfl;                        // [2][128] row flags (protection)
-    int *sIdx = reinterpret_cast<int *>(sm + L.sidx);       // [2][128] value-store index per row
-    float2 *sCs = reinterpret_cast<float2 *>(sm + L.cs);    // [G * 64] (cos, sin) of the next tile
-    float4 *sRed = reinterpret_cast<float4 *>(sm + L.qt);   // [8 warps][G][32] (aliases qt..sp)
+    float *sMax = reinterpret_cast<float *>(sm + L.smax);   // [2 groups][2][4][4]
+    float *sSum = reinterpret_cast<float *>(sm + L.ssum);   // [2 groups][4 warps][4] probability sums
+    unsigned char *sFl = sm + L.sfl;                        // [2 groups][2][128] row flags
+    int *sIdx = reinterpret_cast<int *>(sm + L.sidx);       // [2 groups][2][128] value-store indices
+    float2 *sCs = reinterpret_cast<float2 *>(sm + L.cs);    // [2 groups][G * 64] (cos, sin)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const WsRange rg = ws_range(x, blockIdx.x);
@@ -427,13 +435,13 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
             mbar_init(k_full + i, 1);
             mbar_init(k_empty + i, 1);
             mbar_init(acc_full + i, 1);
-            mbar_init(acc_empty + i, 8);
+            mbar_init(acc_empty + i, 4);
             mbar_init(q_full + i, 1);
             mbar_init(q_empty + i, 8);
         }
         for (int i = 0; i < WS_MAXSV; ++i) {
             mbar_init(v_full + i, 1);
-            mbar_init(v_empty + i, 8);
+            mbar_init(v_empty + i, 4);
         }
         mbar_init(b_full, 1);
         mbar_init(b_empty, 1);
@@ -638,49 +646,66 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
         }
     } else {
         // ==================================== epilogue ===========================================
-        const int et = tid - 128;                       // 0 .. 255
-        const int ew = warp - 4, qw = warp & 3, hf = ew >> 2;
-        // Key phase: the warp covers its lane quarter's 32 rows and the pairs [jb, jb + 32); thread
-        // t = (r0, q4) handles rows 32 qw + r0 + 8 m (m = 0 .. 3) and, in every 8-pair group
+        // Two groups of four warps (one warp per tensor-memory lane quarter) take alternate tiles of
+        // the CTA's range, so that one group's key phase (FMA pipe) overlaps the other's softmax and
+        // value sums. Key phase: warp qw covers rows 32 qw .. 32 qw + 31 and all 64 RoPE pairs;
+        // thread t = (r0, q4) handles rows 32 qw + r0 + 8 m (m = 0 .. 3) and, in every 8-pair group
         // [j0, j0 + 8), the pairs j0 + 2 q4 and j0 + 2 q4 + 1 (the 16x256b fragment), so each query
-        // value read from shared memory serves four rows. After a quad reduction the thread owns
-        // row tau = 32 qw + r0 + 8 q4 for the softmax.
+        // value read from shared memory serves four rows; a quad reduction leaves thread t with the
+        // full score of row tau = 32 qw + r0 + 8 q4 for every q-head.
+        const int et = tid - 128;                       // 0 .. 255
+        const int ew = warp - 4, qw = warp & 3, gid = ew >> 2;
+        const int gt = et & 127;                        // thread within the group
+        const int bar_g = BAR_EPI + gid;                // the group's named barrier
         const int q4 = lane & 3, r0 = lane >> 2;
         const int tau = 32 * qw + r0 + 8 * q4;
-        const int jb = 32 * hf;                         // first RoPE pair of this warp
         const uint32_t lane0 = (uint32_t)(qw * 32) << 16, lane16 = (uint32_t)(qw * 32 + 16) << 16;
         // row m's rotation e^{i w_j tau_m} for the thread's pairs, fixed for the kernel, kept in
-        // tensor memory next to the key accumulators (cos at WS_TAB + j, sin at WS_TAB + 64 + j)
+        // tensor memory next to the key accumulators (cos at WS_TAB + j, sin at WS_TAB + 64 + j);
+        // group 0 writes it, both groups read it
+        if (gid == 0) {
 #pragma unroll
-        for (int lh = 0; lh < 2; ++lh) {
+            for (int lh = 0; lh < 2; ++lh) {
+#pragma unroll 1
+                for (int k = 0; k < 8; ++k) {
+                    float cv[4], sv[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                float cv[4], sv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int row = 32 * qw + 16 * lh + r0 + 8 * (e >> 1);
-                    const int j = jb + 8 * k + 2 * q4 + (e & 1);
-                    float2 c = make_float2(1.f, 0.f);
-                    if (a.rope_cs != nullptr && row < x.rope_rows) c = a.rope_cs[(size_t)row * DH + j];
-                    cv[e] = c.x;
-                    sv[e] = c.y;
+                    for (int e = 0; e < 4; ++e) {
+                        const int row = 32 * qw + 16 * lh + r0 + 8 * (e >> 1);
+                        const int j = 8 * k + 2 * q4 + (e & 1);
+                        float2 c = make_float2(1.f, 0.f);
+                        if (a.rope_cs != nullptr && row < x.rope_rows) c = a.rope_cs[(size_t)row * DH + j];
+                        cv[e] = c.x;
+                        sv[e] = c.y;
+                    }
+                    const uint32_t tl0 = tmem + WS_TAB + (lh ? lane16 : lane0) + 8 * k;
+                    tmem_st4f(tl0, cv);
+                    tmem_st4f(tl0 + DH, sv);
                 }
-                const uint32_t tl0 = tmem + WS_TAB + (lh ? lane16 : lane0) + jb + 8 * k;
-                tmem_st4f(tl0, cv);
-                tmem_st4f(tl0 + DH, sv);
             }
+            tmem_wait_st();
         }
-        tmem_wait_st();
+        tc_fence_before();
+        bar_named(BAR_ALL, WS_EPI);
+        tc_fence_after();
         ws_griddep_wait();
         const float qscale = a.scale * LOG2E;           // scores in log2 units
-        // value-sum layout: thread = (quad qd, slice sl); compressed tiles use kV's quads,
-        // window tiles the 32 channel quads
+        // group areas: q~ [2][G][128], p [2][128][G]; the segment-end reduction aliases them
+        float *sQt = reinterpret_cast<float *>(sm + L.eg) + (size_t)gid * 4 * G * 128;
+        float *sP = sQt + 2 * G * 128;
+        float4 *sRed = reinterpret_cast<float4 *>(sQt);          // [4 warps][G][32]
+        float *sMaxg = sMax + gid * 32, *sSumg = sSum + gid * 16;
+        unsigned char *sFlg = sFl + gid * 256;
+        int *sIdxg = sIdx + gid * 256;
+        float2 *sCsg = sCs + gid * G * DH;
+        // value-sum layout of the group: thread = (quad qd, slice sl); compressed tiles use kV's
+        // quads, exact rows the 32 channel quads
         const int nqr = (rV + 3) >> 2;
         const int nqpr = nqr <= 8 ? 8 : nqr <= 16 ? 16 : 32;
-        const int qdr = et & (nqpr - 1), slr = et / nqpr, nslr = WS_EPI / nqpr;
-        const int qdw = et & 31, slw = et >> 5;
+        const int qdr = gt & (nqpr - 1), slr = gt / nqpr, nslr = 128 / nqpr;
+        const int qdw = gt & 31, slw = gt >> 5;
         bool ok = true;
-        int at = 0, vt = 0, seg = 0, it = 0;
+        int at = 0, vt = 0, seg = 0, it = 0, own = 0;
         int vs = 0;                                     // V stage of tile vt, and its pass parity
         uint32_t vph = 0;
 
@@ -691,18 +716,20 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
             if (tl < Tc + x.Tp) return 0;
             return a.n_c + (long long)(tl - Tc - x.Tp) * DEC_TILE;
         };
-        // q~ = (q rotated by -w_j t0) * scale * log2(e) for tile start t0, into qt buffer `b`
-        // this thread's pair of q~ is j = et mod 64 (threads et < G 64 build one element each)
-        auto load_cs = [&](long long t0) -> float2 {
-            if (a.rope_cs == nullptr || et >= G * DH) return make_float2(1.f, 0.f);
-            return a.rope_cs[(size_t)t0 * DH + (et & (DH - 1))];
-        };
-        auto make_qt = [&](const float *q, float2 cs, int b) {
-            if (et < G * DH) {
-                const int g = et / DH, j = et & (DH - 1);
-                const float qr = q[g * D + j], qi = q[g * D + DH + j];
-                sQt[(b * G + g) * D + j] = qscale * fmaf(qr, cs.x, qi * cs.y);
-                sQt[(b * G + g) * D + DH + j] = qscale * fmaf(qi, cs.x, -qr * cs.y);
+        // q~ = (q rotated by -w_j t0) * scale * log2(e) for tile start t0, into the group's q~ buffer
+        // b; thread gt builds pairs gt and gt + 128 of the G x 64 pairs
+        auto make_qt = [&](const float *q, long long t0, int b, bool from_cs) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int e = gt + 128 * h;
+                if (e < G * DH) {
+                    const int g = e / DH, j = e & (DH - 1);
+                    float2 cs = make_float2(1.f, 0.f);
+                    if (a.rope_cs != nullptr) cs = from_cs ? sCsg[e] : a.rope_cs[(size_t)t0 * DH + j];
+                    const float qr = q[g * D + j], qi = q[g * D + DH + j];
+                    sQt[(b * G + g) * D + j] = qscale * fmaf(qr, cs.x, qi * cs.y);
+                    sQt[(b * G + g) * D + DH + j] = qscale * fmaf(qi, cs.x, -qr * cs.y);
+                }
             }
         };
 
@@ -715,8 +742,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
             const int qs = seg & 1;
             bool w = wait_ab(q_full + qs, (seg >> 1) & 1, abort_flag);
             const float *q = sQ + qs * G * D;
-            // m_ref (uniform), this thread's share of the probability sums (its q-heads), and the
-            // value sums, all relative to 2^m_ref
+            // m_ref (uniform over the group), this thread's probability sums and the value sums,
+            // all relative to 2^m_ref
             float mref[GT], lth[GT];
             float4 vr[GT], vw[GT];
 #pragma unroll
@@ -726,9 +753,10 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 vr[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
                 vw[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            const long long t0a = tile_t0(ta);
-            if (w) make_qt(q, load_cs(t0a), it & 1);
-            ok = bar_and(BAR_EPI, WS_EPI, w);
+            // this group's first tile of the segment
+            const int tf = ta + ((it & 1) != gid ? 1 : 0);
+            if (w && tf < tb) make_qt(q, tile_t0(tf), own & 1, false);
+            ok = bar_and(bar_g, 128, w);
             if (!ok) break;
             bool good = true;                       // this thread's waits of the segment so far
             // channel-space sums: window or protected tiles, or value-protected compressed rows
@@ -736,13 +764,33 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
             const int npk = x.pflags != nullptr ? x.pcount[0][u] : 0;
             const int npv = x.pflags != nullptr ? x.pcount[1][u] : 0;
             for (int tl = ta; tl < tb; ++tl) {
-                const int b = it & 1;
                 const bool comp = tl < Tc;
                 const bool prot = !comp && tl < Tc + x.Tp;       // protected exact keys
+                if ((it & 1) != gid) {
+                    // the other group's tile: keep the ring and accumulator counters in step
+                    if (comp) ++at;
+                    if (!prot) {
+                        ++vt;
+                        if (++vs == NSV) {
+                            vs = 0;
+                            vph ^= 1;
+                        }
+                    }
+                    ++it;
+                    continue;
+                }
+                const int b = own & 1;
                 const long long t0 = tile_t0(tl);
-                // the next tile's query rotation: copied now, used after the first barrier
-                if (tl + 1 < tb && a.rope_cs != nullptr && et < G * DH)
-                    cp_async8(sCs + et, a.rope_cs + (size_t)tile_t0(tl + 1) * DH + (et & (DH - 1)));
+                // this group's next tile of the segment (two ahead): its query rotation, copied now
+                const bool nxt = tl + 2 < tb;
+                if (nxt && a.rope_cs != nullptr) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int e = gt + 128 * h;
+                        if (e < G * DH)
+                            cp_async8(sCsg + e, a.rope_cs + (size_t)tile_t0(tl + 2) * DH + (e & (DH - 1)));
+                    }
+                }
                 int rows;
                 long long pos;
                 unsigned char fl = 0;
@@ -763,9 +811,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 }
                 // rows whose key is protected are attended in the protected tiles
                 const bool valid = tau < rows && !(fl & 1);
-                // ---- this row's key: pairs (j, j + 64), j in [jb, jb + 32), chunks of 8 pairs,
-                //      rotated by e^{i w_j tau} and dotted with the rotated queries ----------------
-                // partial scores of the thread's four rows over its pairs (float2: two pairs)
+                // ---- key phase: partial scores of the thread's four rows (float2: two pairs) ------
                 float2 acc[4][GT];
 #pragma unroll
                 for (int m = 0; m < 4; ++m)
@@ -778,20 +824,19 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 good = good && wk;
                 tc_fence_after();
                 const float *qt = sQt + b * G * D;
-                // exact key rows (protected or window tiles): the thread's four rows
                 int xrows = 0;
                 if (!comp) {
                     const int pi = prot ? (tl - Tc) * DEC_TILE : 0;
                     xrows = prot ? max(0, min(DEC_TILE, npk - pi)) : (int)min((long long)DEC_TILE, a.t - t0);
                 }
+                const uint32_t acc0 = tmem + 128u * (at & 1);
 #pragma unroll 1
-                for (int k = 0; k < 4; ++k) {
-                    const int j0 = jb + 8 * k;
+                for (int k = 0; k < 8; ++k) {
+                    const int j0 = 8 * k;
                     // [m][two pairs]: key real parts, imaginary parts, cos, sin
                     float kr[4][2], ki[4][2], cc[4][2], ss[4][2];
                     if (comp) {
                         float t4[4];
-                        const uint32_t acc0 = tmem + 128u * (at & 1);
 #pragma unroll
                         for (int lh = 0; lh < 2; ++lh) {
                             const uint32_t ln = lh ? lane16 : lane0;
@@ -881,8 +926,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     if (lane == 0 && wk) mbar_arrive(acc_empty + (at & 1));
                     ++at;
                 }
-                // quad reduction: thread q4 ends with row m = q4 (tile row tau) summed over the
-                // warp's 32 pairs
+                // quad reduction: thread q4 ends with row m = q4 (tile row tau), all 64 pairs
+                float sc[GT];
                 {
                     float s1[2][GT];
                     const bool hi2 = (q4 & 2) != 0;
@@ -899,31 +944,17 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
 #pragma unroll
                     for (int gg = 0; gg < GT; ++gg) {
                         const float keep = odd ? s1[1][gg] : s1[0][gg], send = odd ? s1[0][gg] : s1[1][gg];
-                        sS[((b * 2 + hf) * G + gg) * 128 + tau] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                        const float full = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                        sc[gg] = valid ? full : -CUDART_INF_F;
                     }
                 }
-                ok = bar_and(BAR_EPI, WS_EPI, good);                     // barrier 1
-                if (!ok) break;
-                // ---- full scores; next tile's queries; probabilities against m_ref ---------------
-                float sc[GT];
-#pragma unroll
-                for (int gg = 0; gg < GT; ++gg)
-                    sc[gg] = valid ? sS[((b * 2 + 0) * G + gg) * 128 + tau] +
-                                         sS[((b * 2 + 1) * G + gg) * 128 + tau]
-                                   : -CUDART_INF_F;
-                if (tl + 1 < tb) {
-                    float2 cs = make_float2(1.f, 0.f);
-                    if (a.rope_cs != nullptr && et < G * DH) {
-                        cp_async_wait_all();
-                        cs = sCs[et];
-                    }
-                    make_qt(q, cs, b ^ 1);
+                // ---- the group's next tile's queries; probabilities against m_ref ------------------
+                if (nxt) {
+                    if (a.rope_cs != nullptr) cp_async_wait_all();
+                    make_qt(q, 0, b ^ 1, true);
                 }
-                if (hf == 0) {
-                    sFl[b * 128 + tau] = (unsigned char)((fl & 2) && !(fl & 1) && vidx >= 0 ? 2 : 0);
-                    sIdx[b * 128 + tau] = vidx;
-                }
-                // each thread owns the q-heads gg with (gg & 1) == hf (both for G = 1, half 0)
+                sFlg[b * 128 + tau] = (unsigned char)((fl & 2) && !(fl & 1) && vidx >= 0 ? 2 : 0);
+                sIdxg[b * 128 + tau] = vidx;
                 float pv[GT];
                 bool over = false;
 #pragma unroll
@@ -931,9 +962,9 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     const float dlt = sc[gg] - mref[gg];          // +inf or NaN while m_ref is unset
                     over = over || (valid && !(dlt <= WS_LAZY));
                     pv[gg] = valid ? ex2(dlt) : 0.f;
-                    if (GT == 1 ? hf == 0 : (gg & 1) == hf) sP[(b * 128 + tau) * G + gg] = pv[gg];
                 }
-                if (bar_or(BAR_EPI, WS_EPI, over)) {                      // barrier 2
+                store_p<GT>(sP + (b * 128 + tau) * G, pv);
+                if (bar_or(bar_g, 128, over)) {
                     // some score is above m_ref + WS_LAZY (or m_ref is unset): m_ref <- the running
                     // maximum, rescale the sums, recompute this tile's probabilities
 #pragma unroll
@@ -941,13 +972,13 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         float m = sc[gg];
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                        if (hf == 0 && lane == 0) sMax[(b * 4 + qw) * 4 + gg] = m;
+                        if (lane == 0) sMaxg[(b * 4 + qw) * 4 + gg] = m;
                     }
-                    bar_named(BAR_EPI, WS_EPI);
+                    bar_named(bar_g, 128);
 #pragma unroll
                     for (int gg = 0; gg < GT; ++gg) {
-                        const float mt = fmaxf(fmaxf(sMax[(b * 4 + 0) * 4 + gg], sMax[(b * 4 + 1) * 4 + gg]),
-                                               fmaxf(sMax[(b * 4 + 2) * 4 + gg], sMax[(b * 4 + 3) * 4 + gg]));
+                        const float mt = fmaxf(fmaxf(sMaxg[(b * 4 + 0) * 4 + gg], sMaxg[(b * 4 + 1) * 4 + gg]),
+                                               fmaxf(sMaxg[(b * 4 + 2) * 4 + gg], sMaxg[(b * 4 + 3) * 4 + gg]));
                         const float mn = fmaxf(mref[gg], mt);
                         // a tile without rows leaves the running state as it is
                         const float alpha = mn == -CUDART_INF_F ? 1.f : ex2(mref[gg] - mn);
@@ -961,13 +992,12 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         x23 = __fmul2_rn(al, make_float2(vw[gg].z, vw[gg].w));
                         vw[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
                         pv[gg] = valid ? ex2(sc[gg] - mn) : 0.f;
-                        if (GT == 1 ? hf == 0 : (gg & 1) == hf) sP[(b * 128 + tau) * G + gg] = pv[gg];
                     }
-                    bar_named(BAR_EPI, WS_EPI);
+                    store_p<GT>(sP + (b * 128 + tau) * G, pv);
+                    bar_named(bar_g, 128);
                 }
 #pragma unroll
-                for (int gg = 0; gg < GT; ++gg)
-                    if (GT == 1 ? hf == 0 : (gg & 1) == hf) lth[gg] += pv[gg];
+                for (int gg = 0; gg < GT; ++gg) lth[gg] += pv[gg];
                 // ---- value sums: v_g += sum_i p[g][i] V[i][quad] ----------------------------
                 const bool wv = prot ? true : wait_ab(v_full + vs, vph, abort_flag);
                 good = good && wv;
@@ -975,16 +1005,16 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                 const float *P = sP + (size_t)b * 128 * G;
                 if (prot) {
                     // protected rows: exact values from the value store (channel sums)
-                    for (int i = slw; i < rows; i += 8) {
-                        const int vi = sIdx[b * 128 + i];
+                    for (int i = slw; i < rows; i += 4) {
+                        const int vi = sIdxg[b * 128 + i];
                         if (vi < 0) continue;
                         const float4 v4 = load_row4(x.pstore[1], ((size_t)u * x.pcap + vi) * D + 4 * qdw, a.kv_dtype);
                         const float2 v01 = make_float2(v4.x, v4.y), v23 = make_float2(v4.z, v4.w);
-                        float pv[GT];
-                        load_p(P + i * G, pv);
+                        float pp[GT];
+                        load_p(P + i * G, pp);
 #pragma unroll
                         for (int gg = 0; gg < GT; ++gg) {
-                            const float2 p2 = make_float2(pv[gg], pv[gg]);
+                            const float2 p2 = make_float2(pp[gg], pp[gg]);
                             const float2 x01 = __ffma2_rn(p2, v01, make_float2(vw[gg].x, vw[gg].y));
                             const float2 x23 = __ffma2_rn(p2, v23, make_float2(vw[gg].z, vw[gg].w));
                             vw[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
@@ -994,16 +1024,16 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     if (comp && x.pflags != nullptr) {
                         // value-protected rows of a compressed tile: their coordinates are zero;
                         // the exact value row enters the channel sums
-                        for (int i = slw; i < rows; i += 8) {
-                            if (!(sFl[b * 128 + i] & 2)) continue;
-                            const int vi = sIdx[b * 128 + i];
+                        for (int i = slw; i < rows; i += 4) {
+                            if (!(sFlg[b * 128 + i] & 2)) continue;
+                            const int vi = sIdxg[b * 128 + i];
                             const float4 v4 = load_row4(x.pstore[1], ((size_t)u * x.pcap + vi) * D + 4 * qdw, a.kv_dtype);
                             const float2 v01 = make_float2(v4.x, v4.y), v23 = make_float2(v4.z, v4.w);
-                            float pv[GT];
-                            load_p(P + i * G, pv);
+                            float pp[GT];
+                            load_p(P + i * G, pp);
 #pragma unroll
                             for (int gg = 0; gg < GT; ++gg) {
-                                const float2 p2 = make_float2(pv[gg], pv[gg]);
+                                const float2 p2 = make_float2(pp[gg], pp[gg]);
                                 const float2 x01 = __ffma2_rn(p2, v01, make_float2(vw[gg].x, vw[gg].y));
                                 const float2 x23 = __ffma2_rn(p2, v23, make_float2(vw[gg].z, vw[gg].w));
                                 vw[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
@@ -1016,11 +1046,11 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         for (int i = slr; i < rows; i += nslr) {
                             const float4 v = load_v4s(V + (size_t)i * vld, 4 * qdr, BF ? 2 : 4);
                             const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
-                            float pv[GT];
-                            load_p(P + i * G, pv);
+                            float pp[GT];
+                            load_p(P + i * G, pp);
 #pragma unroll
                             for (int gg = 0; gg < GT; ++gg) {
-                                const float pg = pv[gg];
+                                const float pg = pp[gg];
                                 const float2 p2 = make_float2(pg, pg);
                                 const float2 x01 = __ffma2_rn(p2, v01, make_float2(vr[gg].x, vr[gg].y));
                                 const float2 x23 = __ffma2_rn(p2, v23, make_float2(vr[gg].z, vr[gg].w));
@@ -1032,7 +1062,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         const int inew = (a.new_pos >= t0 && a.new_pos < t0 + rows)
                                              ? (int)(a.new_pos - t0) : -1;
 #pragma unroll 4
-                        for (int i = slw; i < rows; i += 8) {
+                        for (int i = slw; i < rows; i += 4) {
                             float4 v;
                             if (i == inew) {
                                 v = load_row4(a.new_row[1], (size_t)u * D + 4 * qdw, a.kv_dtype);
@@ -1040,30 +1070,30 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                                 v = load_v4s(V + (size_t)i * vld, 4 * qdw, esz);
                             }
                             const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
-                            float pv[GT];
-                            load_p(P + i * G, pv);
+                            float pp[GT];
+                            load_p(P + i * G, pp);
 #pragma unroll
                             for (int gg = 0; gg < GT; ++gg) {
-                                const float pg = pv[gg];
+                                const float pg = pp[gg];
                                 const float2 p2 = make_float2(pg, pg);
                                 const float2 x01 = __ffma2_rn(p2, v01, make_float2(vw[gg].x, vw[gg].y));
                                 const float2 x23 = __ffma2_rn(p2, v23, make_float2(vw[gg].z, vw[gg].w));
                                 vw[gg] = make_float4(x01.x, x01.y, x23.x, x23.y);
                             }
                         }
-                        if (inew >= 0 && et < D) {
+                        if (inew >= 0 && gt < D) {
                             // fused append: store the new position's K and V rows in the ring
-                            const size_t slot = ((size_t)u * a.R + (size_t)(a.new_pos % a.R)) * D + et;
+                            const size_t slot = ((size_t)u * a.R + (size_t)(a.new_pos % a.R)) * D + gt;
                             if (a.kv_dtype == ISKV_BF16) {
                                 const __nv_bfloat16 *nk = static_cast<const __nv_bfloat16 *>(a.new_row[0]) + (size_t)u * D;
                                 const __nv_bfloat16 *nv = static_cast<const __nv_bfloat16 *>(a.new_row[1]) + (size_t)u * D;
-                                const_cast<__nv_bfloat16 *>(static_cast<const __nv_bfloat16 *>(a.ring[0]))[slot] = nk[et];
-                                const_cast<__nv_bfloat16 *>(static_cast<const __nv_bfloat16 *>(a.ring[1]))[slot] = nv[et];
+                                const_cast<__nv_bfloat16 *>(static_cast<const __nv_bfloat16 *>(a.ring[0]))[slot] = nk[gt];
+                                const_cast<__nv_bfloat16 *>(static_cast<const __nv_bfloat16 *>(a.ring[1]))[slot] = nv[gt];
                             } else {
                                 const float *nk = static_cast<const float *>(a.new_row[0]) + (size_t)u * D;
                                 const float *nv = static_cast<const float *>(a.new_row[1]) + (size_t)u * D;
-                                const_cast<float *>(static_cast<const float *>(a.ring[0]))[slot] = nk[et];
-                                const_cast<float *>(static_cast<const float *>(a.ring[1]))[slot] = nv[et];
+                                const_cast<float *>(static_cast<const float *>(a.ring[0]))[slot] = nk[gt];
+                                const_cast<float *>(static_cast<const float *>(a.ring[1]))[slot] = nv[gt];
                             }
                         }
                     }
@@ -1077,16 +1107,18 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         vph ^= 1;
                     }
                 }
+                ++own;
                 ++it;
             }
             // q slot consumed (every q~ of the segment is built)
             __syncwarp();
             if (lane == 0) mbar_arrive(q_empty + qs);
             ++seg;
-            ok = bar_and(BAR_EPI, WS_EPI, ok && good);    // tiles done: the reduction area is free
+            ok = bar_and(bar_g, 128, ok && good);         // tiles done: the reduction area is free
             if (!ok) break;
-            // ---- partial record: [m, l, acc_rank[rV], acc_chan[D]] per q-head ---------------------
-            float *rec = a.ws + ((size_t)blockIdx.x * x.maxseg + jseg) * G * (2 + rV + D);
+            // ---- this group's partial record: [m, l, acc_rank[rV], acc_chan[D]] per q-head ----------
+            float *rec = a.ws + (((size_t)blockIdx.x * x.maxseg + jseg) * 2 + gid) * G * (2 + rV + D);
+            const int gw = ew & 3;                          // warp within the group
             if (has_c) {
 #pragma unroll
                 for (int gg = 0; gg < GT; ++gg) {
@@ -1096,59 +1128,61 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         vr[gg].z += __shfl_xor_sync(0xffffffffu, vr[gg].z, o);
                         vr[gg].w += __shfl_xor_sync(0xffffffffu, vr[gg].w, o);
                     }
-                    if (lane < nqpr) sRed[(ew * G + gg) * 32 + qdr] = vr[gg];
+                    if (lane < nqpr) sRed[(gw * G + gg) * 32 + qdr] = vr[gg];
                 }
-                bar_named(BAR_EPI, WS_EPI);
-                for (int o = et; o < G * rV; o += WS_EPI) {
+                bar_named(bar_g, 128);
+                for (int o = gt; o < G * rV; o += 128) {
                     const int gg = o / rV, c = o % rV;
                     float s = 0.f;
 #pragma unroll
-                    for (int w8 = 0; w8 < 8; ++w8)
-                        s += reinterpret_cast<const float *>(sRed)[((w8 * G + gg) * 32) * 4 + c];
+                    for (int w4 = 0; w4 < 4; ++w4)
+                        s += reinterpret_cast<const float *>(sRed)[((w4 * G + gg) * 32) * 4 + c];
                     rec[gg * (2 + rV + D) + 2 + c] = s;
                 }
-                bar_named(BAR_EPI, WS_EPI);
+                bar_named(bar_g, 128);
             } else {
-                for (int o = et; o < G * rV; o += WS_EPI)
+                for (int o = gt; o < G * rV; o += 128)
                     rec[(o / rV) * (2 + rV + D) + 2 + o % rV] = 0.f;
             }
             if (has_w) {
 #pragma unroll
-                for (int gg = 0; gg < GT; ++gg) sRed[(ew * G + gg) * 32 + qdw] = vw[gg];
-                bar_named(BAR_EPI, WS_EPI);
-                for (int o = et; o < G * D; o += WS_EPI) {
+                for (int gg = 0; gg < GT; ++gg) sRed[(gw * G + gg) * 32 + qdw] = vw[gg];
+                bar_named(bar_g, 128);
+                for (int o = gt; o < G * D; o += 128) {
                     const int gg = o / D, c = o % D;
                     float s = 0.f;
 #pragma unroll
-                    for (int w8 = 0; w8 < 8; ++w8)
-                        s += reinterpret_cast<const float *>(sRed)[((w8 * G + gg) * 32) * 4 + c];
+                    for (int w4 = 0; w4 < 4; ++w4)
+                        s += reinterpret_cast<const float *>(sRed)[((w4 * G + gg) * 32) * 4 + c];
                     rec[gg * (2 + rV + D) + 2 + rV + c] = s;
                 }
-                bar_named(BAR_EPI, WS_EPI);
+                bar_named(bar_g, 128);
             } else {
-                for (int o = et; o < G * D; o += WS_EPI)
+                for (int o = gt; o < G * D; o += 128)
                     rec[(o / D) * (2 + rV + D) + 2 + rV + o % D] = 0.f;
             }
-            // probability sums: per warp, then over the 8 epilogue warps
+            // probability sums: per warp, then over the group's 4 warps
 #pragma unroll
             for (int gg = 0; gg < GT; ++gg) {
                 float sl = lth[gg];
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) sl += __shfl_xor_sync(0xffffffffu, sl, o);
-                if (lane == 0) sSum[ew * 4 + gg] = sl;
+                if (lane == 0) sSumg[gw * 4 + gg] = sl;
             }
-            bar_named(BAR_EPI, WS_EPI);
-            if (et < G) {
+            bar_named(bar_g, 128);
+            if (gt < G) {
 #pragma unroll
                 for (int gg = 0; gg < GT; ++gg)
-                    if (gg == et) {
+                    if (gg == gt) {
                         float l = 0.f;
 #pragma unroll
-                        for (int w8 = 0; w8 < 8; ++w8) l += sSum[w8 * 4 + gg];
+                        for (int w4 = 0; w4 < 4; ++w4) l += sSumg[w4 * 4 + gg];
                         rec[gg * (2 + rV + D)] = mref[gg];
                         rec[gg * (2 + rV + D) + 1] = l;
                     }
             }
+            // the next segment rewrites the group area (aliased by the reduction)
+            bar_named(bar_g, 128);
         }
         if (et == 0) {
             counters[6] = at;
@@ -1211,12 +1245,15 @@ __global__ void __launch_bounds__(128) decode_ws_merge_kernel(DecodeArgs a, WsEx
         Lw[g] = 0.f;
         accw[g] = 0.f;
     }
+    // every CTA whose range touches the unit left one record per epilogue group
     for (int c = c_lo; c <= c_hi; ++c) {
         const long long g0 = (long long)c * x.N / x.P;
         const int js = (int)(u - g0 / x.Tu);
-        const float *rec = a.ws + ((size_t)c * x.maxseg + js) * stride;
+        for (int gr = 0; gr < 2; ++gr) {
+            const float *rec = a.ws + (((size_t)c * x.maxseg + js) * 2 + gr) * stride;
 #pragma unroll
-        for (int g = 0; g < GT; ++g) M[g] = fmaxf(M[g], __ldcg(rec + g * (2 + rV + D)));
+            for (int g = 0; g < GT; ++g) M[g] = fmaxf(M[g], __ldcg(rec + g * (2 + rV + D)));
+        }
     }
     float accr[GT];
 #pragma unroll
@@ -1224,14 +1261,18 @@ __global__ void __launch_bounds__(128) decode_ws_merge_kernel(DecodeArgs a, WsEx
     for (int c = c_lo; c <= c_hi; ++c) {
         const long long g0 = (long long)c * x.N / x.P;
         const int js = (int)(u - g0 / x.Tu);
-        const float *rec = a.ws + ((size_t)c * x.maxseg + js) * stride;
+        for (int gr = 0; gr < 2; ++gr) {
+            const float *rec = a.ws + (((size_t)c * x.maxseg + js) * 2 + gr) * stride;
 #pragma unroll
-        for (int g = 0; g < GT; ++g) {
-            const float *r = rec + g * (2 + rV + D);
-            const float w = ex2(__ldcg(r) - M[g]);
-            Lw[g] = fmaf(w, __ldcg(r + 1), Lw[g]);
-            if (j < kV) accr[g] = fmaf(w, __ldcg(r + 2 + j), accr[g]);
-            accw[g] = fmaf(w, __ldcg(r + 2 + rV + j), accw[g]);
+            for (int g = 0; g < GT; ++g) {
+                const float *r = rec + g * (2 + rV + D);
+                // a group that saw no tile of the unit left m = -inf: weight 0
+                const float m = __ldcg(r);
+                const float w = m == -CUDART_INF_F ? 0.f : ex2(m - M[g]);
+                Lw[g] = fmaf(w, __ldcg(r + 1), Lw[g]);
+                if (j < kV) accr[g] = fmaf(w, __ldcg(r + 2 + j), accr[g]);
+                accw[g] = fmaf(w, __ldcg(r + 2 + rV + j), accw[g]);
+            }
         }
     }
 #pragma unroll
@@ -1248,7 +1289,7 @@ __global__ void __launch_bounds__(128) decode_ws_merge_kernel(DecodeArgs a, WsEx
 }
 
 size_t ws_partial_floats(int units, int sms, int G, int rV) {
-    return ((size_t)units + 2 * (size_t)sms) * G * (2 + rV + D);
+    return ((size_t)units + 2 * (size_t)sms) * 2 * G * (2 + rV + D);
 }
 
 // The register split inside the kernel waits for registers that the launch must have granted:
