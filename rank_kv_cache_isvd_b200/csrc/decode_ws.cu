@@ -221,6 +221,41 @@ __device__ __forceinline__ void tmem_st4f(uint32_t taddr, const float (&v)[4]) {
                  : "memory");
 }
 
+// The key-phase operands of one 8-pair group for the thread's four rows (16x256b fragments):
+// [block][4]: cos lanes 0-15, sin lanes 0-15, key real, key imaginary, then the same at lanes 16-31.
+struct KeyBlk {
+    float v[8][4];
+};
+
+// Loads of one 8-pair group [j0, j0 + 8): the RoPE table and the key accumulator, both lane halves.
+__device__ __forceinline__ void key_blk_load(KeyBlk &kb, uint32_t tab, uint32_t acc, uint32_t ln0,
+                                             uint32_t ln16, int j0) {
+#pragma unroll
+    for (int lh = 0; lh < 2; ++lh) {
+        const uint32_t ln = lh ? ln16 : ln0;
+        tmem_ld4f(tab + ln + j0, kb.v[4 * lh + 0]);
+        tmem_ld4f(tab + ln + DH + j0, kb.v[4 * lh + 1]);
+        tmem_ld4f(acc + ln + j0, kb.v[4 * lh + 2]);
+        tmem_ld4f(acc + ln + DH + j0, kb.v[4 * lh + 3]);
+    }
+}
+
+// Waits for this thread's tensor-memory loads; the loaded registers pass through the wait, so no
+// use of them can be scheduled before it.
+__device__ __forceinline__ void key_blk_wait(KeyBlk &kb) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(kb.v[0][0]), "+f"(kb.v[0][1]), "+f"(kb.v[0][2]), "+f"(kb.v[0][3]),
+                   "+f"(kb.v[1][0]), "+f"(kb.v[1][1]), "+f"(kb.v[1][2]), "+f"(kb.v[1][3]),
+                   "+f"(kb.v[2][0]), "+f"(kb.v[2][1]), "+f"(kb.v[2][2]), "+f"(kb.v[2][3]),
+                   "+f"(kb.v[3][0]), "+f"(kb.v[3][1]), "+f"(kb.v[3][2]), "+f"(kb.v[3][3]),
+                   "+f"(kb.v[4][0]), "+f"(kb.v[4][1]), "+f"(kb.v[4][2]), "+f"(kb.v[4][3]),
+                   "+f"(kb.v[5][0]), "+f"(kb.v[5][1]), "+f"(kb.v[5][2]), "+f"(kb.v[5][3]),
+                   "+f"(kb.v[6][0]), "+f"(kb.v[6][1]), "+f"(kb.v[6][2]), "+f"(kb.v[6][3]),
+                   "+f"(kb.v[7][0]), "+f"(kb.v[7][1]), "+f"(kb.v[7][2]), "+f"(kb.v[7][3])
+                 :
+                 : "memory");
+}
+
 // 8-byte asynchronous copy global -> shared (this thread waits for its own copies).
 __device__ __forceinline__ void cp_async8(void *dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
@@ -830,41 +865,65 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     xrows = prot ? max(0, min(DEC_TILE, npk - pi)) : (int)min((long long)DEC_TILE, a.t - t0);
                 }
                 const uint32_t acc0 = tmem + 128u * (at & 1);
+                // rotate row m's key of the pair group [j0, j0 + 8) and dot it with the queries
+                auto key_math = [&](int j0, const float2 (&kr2)[4], const float2 (&ki2)[4],
+                                    const float2 (&cc2)[4], const float2 (&ss2)[4]) {
+                    float2 qre[GT], qim[GT];
+#pragma unroll
+                    for (int gg = 0; gg < GT; ++gg) {
+                        qre[gg] = *reinterpret_cast<const float2 *>(qt + gg * D + j0 + 2 * q4);
+                        qim[gg] = *reinterpret_cast<const float2 *>(qt + gg * D + DH + j0 + 2 * q4);
+                    }
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float2 k1 = kr2[m], k2 = ki2[m], c2 = cc2[m], s2 = ss2[m];
+                        const float2 t1 = __fmul2_rn(k2, s2);
+                        const float2 zr = __ffma2_rn(k1, c2, make_float2(-t1.x, -t1.y));
+                        const float2 zi = __ffma2_rn(k1, s2, __fmul2_rn(k2, c2));
+#pragma unroll
+                        for (int gg = 0; gg < GT; ++gg) {
+                            acc[m][gg] = __ffma2_rn(qre[gg], zr, acc[m][gg]);
+                            acc[m][gg] = __ffma2_rn(qim[gg], zi, acc[m][gg]);
+                        }
+                    }
+                };
+                auto key_math_blk = [&](int j0, const KeyBlk &kb) {
+                    float2 kr2[4], ki2[4], cc2[4], ss2[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const int lh = m >> 1, o = 2 * (m & 1);
+                        cc2[m] = make_float2(kb.v[4 * lh + 0][o], kb.v[4 * lh + 0][o + 1]);
+                        ss2[m] = make_float2(kb.v[4 * lh + 1][o], kb.v[4 * lh + 1][o + 1]);
+                        kr2[m] = wk ? make_float2(kb.v[4 * lh + 2][o], kb.v[4 * lh + 2][o + 1]) : make_float2(0.f, 0.f);
+                        ki2[m] = wk ? make_float2(kb.v[4 * lh + 3][o], kb.v[4 * lh + 3][o + 1]) : make_float2(0.f, 0.f);
+                    }
+                    key_math(j0, kr2, ki2, cc2, ss2);
+                };
+                if (comp) {
+                    // tensor-memory loads of the next pair group in flight while this one computes
+                    KeyBlk ka, kb;
+                    key_blk_load(ka, tmem + WS_TAB, acc0, lane0, lane16, 0);
+                    key_blk_wait(ka);
 #pragma unroll 1
-                for (int k = 0; k < 8; ++k) {
-                    const int j0 = 8 * k;
-                    // [m][two pairs]: key real parts, imaginary parts, cos, sin
-                    float kr[4][2], ki[4][2], cc[4][2], ss[4][2];
-                    if (comp) {
-                        float t4[4];
-#pragma unroll
-                        for (int lh = 0; lh < 2; ++lh) {
-                            const uint32_t ln = lh ? lane16 : lane0;
-                            tmem_ld4f(tmem + WS_TAB + ln + j0, t4);
-                            cc[2 * lh][0] = t4[0]; cc[2 * lh][1] = t4[1]; cc[2 * lh + 1][0] = t4[2]; cc[2 * lh + 1][1] = t4[3];
-                            tmem_ld4f(tmem + WS_TAB + ln + DH + j0, t4);
-                            ss[2 * lh][0] = t4[0]; ss[2 * lh][1] = t4[1]; ss[2 * lh + 1][0] = t4[2]; ss[2 * lh + 1][1] = t4[3];
-                            if (wk) {
-                                tmem_ld4f(acc0 + ln + j0, t4);
-                                kr[2 * lh][0] = t4[0]; kr[2 * lh][1] = t4[1]; kr[2 * lh + 1][0] = t4[2]; kr[2 * lh + 1][1] = t4[3];
-                                tmem_ld4f(acc0 + ln + DH + j0, t4);
-                                ki[2 * lh][0] = t4[0]; ki[2 * lh][1] = t4[1]; ki[2 * lh + 1][0] = t4[2]; ki[2 * lh + 1][1] = t4[3];
-                            }
-                        }
-                        tmem_wait_ld();
-                        if (!wk) {
-#pragma unroll
-                            for (int m = 0; m < 4; ++m) kr[m][0] = kr[m][1] = ki[m][0] = ki[m][1] = 0.f;
-                        }
-                    } else {
+                    for (int k = 0; k < 8; k += 2) {
+                        key_blk_load(kb, tmem + WS_TAB, acc0, lane0, lane16, 8 * (k + 1));
+                        key_math_blk(8 * k, ka);
+                        key_blk_wait(kb);
+                        if (k + 2 < 8) key_blk_load(ka, tmem + WS_TAB, acc0, lane0, lane16, 8 * (k + 2));
+                        key_math_blk(8 * (k + 1), kb);
+                        if (k + 2 < 8) key_blk_wait(ka);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int k = 0; k < 8; ++k) {
+                        const int j0 = 8 * k;
                         // rows from the exact stores; protected rows rotate by their full position
                         // (their queries are unrotated), window rows by their offset in the tile
+                        float2 kr2[4], ki2[4], cc2[4], ss2[4];
 #pragma unroll
                         for (int m = 0; m < 4; ++m) {
                             const int row = 32 * qw + r0 + 8 * m;
-                            kr[m][0] = kr[m][1] = ki[m][0] = ki[m][1] = 0.f;
-                            cc[m][0] = cc[m][1] = 1.f;
-                            ss[m][0] = ss[m][1] = 0.f;
+                            float kr[2] = {0.f, 0.f}, ki[2] = {0.f, 0.f}, cc[2] = {1.f, 1.f}, ss[2] = {0.f, 0.f};
                             if (row < xrows) {
                                 const void *src;
                                 size_t base;
@@ -885,38 +944,21 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
 #pragma unroll
                                 for (int e = 0; e < 2; ++e) {
                                     const int j = j0 + 2 * q4 + e;
-                                    kr[m][e] = load_row_elem(src, base + j, a.kv_dtype);
-                                    ki[m][e] = load_row_elem(src, base + DH + j, a.kv_dtype);
+                                    kr[e] = load_row_elem(src, base + j, a.kv_dtype);
+                                    ki[e] = load_row_elem(src, base + DH + j, a.kv_dtype);
                                     if (a.rope_cs != nullptr) {
                                         const float2 c = a.rope_cs[(size_t)apos * DH + j];
-                                        cc[m][e] = c.x;
-                                        ss[m][e] = c.y;
+                                        cc[e] = c.x;
+                                        ss[e] = c.y;
                                     }
                                 }
                             }
+                            kr2[m] = make_float2(kr[0], kr[1]);
+                            ki2[m] = make_float2(ki[0], ki[1]);
+                            cc2[m] = make_float2(cc[0], cc[1]);
+                            ss2[m] = make_float2(ss[0], ss[1]);
                         }
-                    }
-                    // queries of the two pairs, then rotate each row's key and dot
-                    float2 qre[GT], qim[GT];
-#pragma unroll
-                    for (int gg = 0; gg < GT; ++gg) {
-                        qre[gg] = *reinterpret_cast<const float2 *>(qt + gg * D + j0 + 2 * q4);
-                        qim[gg] = *reinterpret_cast<const float2 *>(qt + gg * D + DH + j0 + 2 * q4);
-                    }
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const float2 k1 = make_float2(kr[m][0], kr[m][1]);
-                        const float2 k2 = make_float2(ki[m][0], ki[m][1]);
-                        const float2 c2 = make_float2(cc[m][0], cc[m][1]);
-                        const float2 s2 = make_float2(ss[m][0], ss[m][1]);
-                        const float2 t1 = __fmul2_rn(k2, s2);
-                        const float2 zr = __ffma2_rn(k1, c2, make_float2(-t1.x, -t1.y));
-                        const float2 zi = __ffma2_rn(k1, s2, __fmul2_rn(k2, c2));
-#pragma unroll
-                        for (int gg = 0; gg < GT; ++gg) {
-                            acc[m][gg] = __ffma2_rn(qre[gg], zr, acc[m][gg]);
-                            acc[m][gg] = __ffma2_rn(qim[gg], zi, acc[m][gg]);
-                        }
+                        key_math(j0, kr2, ki2, cc2, ss2);
                     }
                 }
                 if (comp) {
