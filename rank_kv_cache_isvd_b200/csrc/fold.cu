@@ -904,12 +904,12 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
 constexpr int ROT_ROWS = 64;                  // rows per tile
 constexpr int ROT_THREADS = 256;              // 16 row groups (4 rows) x 16 column groups
 constexpr int ROT_XS = ROT_ROWS + 4;          // stride of the transposed row tile
-constexpr int ROT_HS = 128;                   // stride of H_top in shared memory
 constexpr int ROT_GX = 24;                    // CTAs per (unit, path); each takes every 24th tile
+constexpr int ROT_HS = 128;                   // stride of H_top in shared memory
 
 // One tile: acc[rr][cc] = sum_l X[4 rg + rr][l] H[l][CW cg + cc]; X^T and H in shared memory.
 // Each thread keeps a 4 x CW block of outputs in registers, so every shared-memory load feeds
-// 4 or CW fused multiply-adds.
+// 4 or CW fused multiply-adds (packed in pairs of columns for even CW).
 template <int CW>
 __device__ __forceinline__ void rot_tile(const float *sXt, const float *sH, int k, int rg, int cg,
                                          float (&acc)[4][8]) {
@@ -917,17 +917,48 @@ __device__ __forceinline__ void rot_tile(const float *sXt, const float *sH, int 
     for (int rr = 0; rr < 4; ++rr)
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) acc[rr][cc] = 0.f;
-#pragma unroll 4
-    for (int l = 0; l < k; ++l) {
-        const float4 x = *reinterpret_cast<const float4 *>(sXt + l * ROT_XS + 4 * rg);
-        const float xs[4] = {x.x, x.y, x.z, x.w};
-        float hv[CW];
-#pragma unroll
-        for (int cc = 0; cc < CW; ++cc) hv[cc] = sH[l * ROT_HS + CW * cg + cc];
+    if constexpr ((CW & 1) == 0) {
+        // even widths: H columns as float2 pairs, packed fused multiply-adds
+        float2 a2[4][CW / 2];
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr)
 #pragma unroll
-            for (int cc = 0; cc < CW; ++cc) acc[rr][cc] = fmaf(xs[rr], hv[cc], acc[rr][cc]);
+            for (int c2 = 0; c2 < CW / 2; ++c2) a2[rr][c2] = make_float2(0.f, 0.f);
+#pragma unroll 4
+        for (int l = 0; l < k; ++l) {
+            const float4 x = *reinterpret_cast<const float4 *>(sXt + l * ROT_XS + 4 * rg);
+            const float xs[4] = {x.x, x.y, x.z, x.w};
+            float2 hv[CW / 2];
+#pragma unroll
+            for (int c2 = 0; c2 < CW / 2; ++c2)
+                hv[c2] = *reinterpret_cast<const float2 *>(sH + l * ROT_HS + CW * cg + 2 * c2);
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const float2 xx = make_float2(xs[rr], xs[rr]);
+#pragma unroll
+                for (int c2 = 0; c2 < CW / 2; ++c2) a2[rr][c2] = __ffma2_rn(xx, hv[c2], a2[rr][c2]);
+            }
+        }
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+            for (int c2 = 0; c2 < CW / 2; ++c2) {
+                acc[rr][2 * c2] = a2[rr][c2].x;
+                acc[rr][2 * c2 + 1] = a2[rr][c2].y;
+            }
+    } else {
+#pragma unroll 4
+        for (int l = 0; l < k; ++l) {
+            const float4 x = *reinterpret_cast<const float4 *>(sXt + l * ROT_XS + 4 * rg);
+            const float xs[4] = {x.x, x.y, x.z, x.w};
+            float hv[CW];
+#pragma unroll
+            for (int cc = 0; cc < CW; ++cc) hv[cc] = sH[l * ROT_HS + CW * cg + cc];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                for (int cc = 0; cc < CW; ++cc) acc[rr][cc] = fmaf(xs[rr], hv[cc], acc[rr][cc]);
+        }
     }
 }
 
@@ -960,15 +991,48 @@ __global__ void __launch_bounds__(ROT_THREADS, 2) rotate_kernel(RotArgs a) {
     }
     const int rg = tid >> 4, cg = tid & 15;
     const int cw = (kp + 15) >> 4;            // columns per thread (1 .. 8)
+    // fp32 coordinates in 16-byte quads: the next tile's rows are loaded into registers while
+    // this tile is computed (thread: row i = o mod 64 of quad q = o / 64 for o = tid + 256 s)
+    const bool vec = !a.cbf && (k & 3) == 0 && (r & 3) == 0;
+    const int nq = vec ? (ROT_ROWS * (k >> 2) + ROT_THREADS - 1) / ROT_THREADS : 0;   // <= 8
+    float4 pre[8];
+    auto prefetch = [&](long long t) {
+        const long long row0 = t * ROT_ROWS;
+        const int rows = (int)min((long long)ROT_ROWS, a.n_old - row0);
+        const float *cf = static_cast<const float *>(P.coords) + cu;
+#pragma unroll
+        for (int sq = 0; sq < 8; ++sq) {
+            const int o = tid + ROT_THREADS * sq, i = o & (ROT_ROWS - 1), q = o >> 6;
+            pre[sq] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (sq < nq && 4 * q < k && i < rows)
+                pre[sq] = *reinterpret_cast<const float4 *>(cf + (size_t)(row0 + i) * r + 4 * q);
+        }
+    };
+    if (vec && blockIdx.x < tiles) prefetch(blockIdx.x);
     for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
         const long long row0 = t * ROT_ROWS;
         const int rows = (int)min((long long)ROT_ROWS, a.n_old - row0);
         __syncthreads();                      // previous tile's reads of sXt are done
-        for (int o = tid; o < ROT_ROWS * k; o += ROT_THREADS) {
-            const int i = o / k, l = o % k;
-            sXt[l * ROT_XS + i] = i < rows ? load_coord(P.coords, cu + (size_t)(row0 + i) * r + l, a.cbf) : 0.f;
+        if (vec) {
+            // transposed store of the prefetched rows (consecutive threads: consecutive rows)
+#pragma unroll
+            for (int sq = 0; sq < 8; ++sq) {
+                const int o = tid + ROT_THREADS * sq, i = o & (ROT_ROWS - 1), q = o >> 6;
+                if (sq < nq && 4 * q < k) {
+                    sXt[(4 * q + 0) * ROT_XS + i] = pre[sq].x;
+                    sXt[(4 * q + 1) * ROT_XS + i] = pre[sq].y;
+                    sXt[(4 * q + 2) * ROT_XS + i] = pre[sq].z;
+                    sXt[(4 * q + 3) * ROT_XS + i] = pre[sq].w;
+                }
+            }
+        } else {
+            for (int o = tid; o < ROT_ROWS * k; o += ROT_THREADS) {
+                const int i = o / k, l = o % k;
+                sXt[l * ROT_XS + i] = i < rows ? load_coord(P.coords, cu + (size_t)(row0 + i) * r + l, a.cbf) : 0.f;
+            }
         }
         __syncthreads();
+        if (vec && t + gridDim.x < tiles) prefetch(t + gridDim.x);
         float acc[4][8];
         switch (cw) {
             case 1: rot_tile<1>(sXt, sH, k, rg, cg, acc); break;
@@ -994,9 +1058,11 @@ __global__ void __launch_bounds__(ROT_THREADS, 2) rotate_kernel(RotArgs a) {
             }
         }
         // columns past 16 cw (only when kp < r and 16 cw < r): zero
-        for (int o = tid; o < rows * r; o += ROT_THREADS) {
-            const int i = o / r, c = o % r;
-            if (c >= 16 * cw) store_coord(P.coords, cu + (size_t)(row0 + i) * r + c, 0.f, a.cbf);
+        if (16 * cw < r) {
+            for (int o = tid; o < rows * r; o += ROT_THREADS) {
+                const int i = o / r, c = o % r;
+                if (c >= 16 * cw) store_coord(P.coords, cu + (size_t)(row0 + i) * r + c, 0.f, a.cbf);
+            }
         }
     }
 }
@@ -1020,8 +1086,8 @@ cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s) {
     const cudaError_t e = ensure_smem((const void *)rotate_kernel, smem, attr);
     if (e != cudaSuccess) return e;
     const long long tiles = (a.n_old + ROT_ROWS - 1) / ROT_ROWS;
-    const unsigned gx = (unsigned)(tiles < ROT_GX ? tiles : ROT_GX);
-    rotate_kernel<<<dim3(gx, n_units, a.path_hi - a.path_lo), ROT_THREADS, smem, s>>>(a);
+    const long long gx = tiles < ROT_GX ? tiles : ROT_GX;
+    rotate_kernel<<<dim3((unsigned)gx, n_units, a.path_hi - a.path_lo), ROT_THREADS, smem, s>>>(a);
     return cudaGetLastError();
 }
 
