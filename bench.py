@@ -67,6 +67,7 @@ FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12    # fp32 FMA peak of the B200 
 HBM_NOMINAL_GBS = 7700.0                              # HBM3e nominal bandwidth (HGX figure), context
 DECODE_SRC = os.path.join(ROOT, "rank_kv_cache_isvd_b200", "csrc", "decode_ws.cu")
 PROFILE_DECODE = os.path.join(ROOT, "profiles", "decode_ws_qwen3-8b-layer_t32768.md")
+PROFILE_DECODE_BYTES = 810811392       # algorithmic bytes of the captured launch (t = 32768)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -133,7 +134,8 @@ def traffic_from_profile():
         return None, "no traffic line in the profile summary"
     if m.group(2) != src:
         return None, "profile summary taken on an older kernel source"
-    return int(m.group(1)), "ncu capture of the one-layer 32768-token launch (same units per launch)"
+    return int(m.group(1)), ("ncu capture of the one-layer launch at t = 32768 (algorithmic "
+                             f"{PROFILE_DECODE_BYTES} B), scaled by the algorithmic bytes of this launch")
 
 
 class Clocks:
@@ -474,6 +476,9 @@ def headline(args, dev, rank: int, world: int, local_rank: int):
     hbm, which = peaks()
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
     traffic, traffic_how = traffic_from_profile()
+    if traffic is not None:
+        # the same units per launch as the capture; traffic grows with the compressed rows read
+        traffic = int(round(traffic * dec_bytes / PROFILE_DECODE_BYTES))
     ms_per_step = total_ms / args.steps
     return {
         "value": job_throughput(world, total_ms, args.steps),
@@ -485,7 +490,7 @@ def headline(args, dev, rank: int, world: int, local_rank: int):
                 "d2h_bytes_per_step": int(per_tok_d2h * TOK_PER_STEP),
                 "how": ("per token: rows and queries of all layers copied from pinned host "
                         "memory, 36 append+decode calls, outputs copied back; same stream")},
-        "roofline": {"bound": "hbm", "kernel": "decode attention (split + merge), one layer call",
+        "roofline": {"bound": "hbm", "kernel": "decode attention (persistent kernel + merge), one layer call",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "frac_of_nominal": achieved / HBM_NOMINAL_GBS,
                      "traffic": traffic, "traffic_source": traffic_how,
