@@ -696,27 +696,27 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
         const int tau = 32 * qw + r0 + 8 * q4;
         const uint32_t lane0 = (uint32_t)(qw * 32) << 16, lane16 = (uint32_t)(qw * 32 + 16) << 16;
         // row m's rotation e^{i w_j tau_m} for the thread's pairs, fixed for the kernel, kept in
-        // tensor memory next to the key accumulators (cos at WS_TAB + j, sin at WS_TAB + 64 + j);
-        // group 0 writes it, both groups read it
-        if (gid == 0) {
+        // tensor memory next to the key accumulators (cos at WS_TAB + j, sin at WS_TAB + 64 + j):
+        // group g writes the rows of lane half g (16-byte loads, all issued before the stores)
+        {
+            const int lh = gid;
+            float4 t[8][2];
 #pragma unroll
-            for (int lh = 0; lh < 2; ++lh) {
-#pragma unroll 1
-                for (int k = 0; k < 8; ++k) {
-                    float cv[4], sv[4];
+            for (int k = 0; k < 8; ++k)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int row = 32 * qw + 16 * lh + r0 + 8 * (e >> 1);
-                        const int j = 8 * k + 2 * q4 + (e & 1);
-                        float2 c = make_float2(1.f, 0.f);
-                        if (a.rope_cs != nullptr && row < x.rope_rows) c = a.rope_cs[(size_t)row * DH + j];
-                        cv[e] = c.x;
-                        sv[e] = c.y;
-                    }
-                    const uint32_t tl0 = tmem + WS_TAB + (lh ? lane16 : lane0) + 8 * k;
-                    tmem_st4f(tl0, cv);
-                    tmem_st4f(tl0 + DH, sv);
+                for (int rs = 0; rs < 2; ++rs) {
+                    const int row = 32 * qw + 16 * lh + r0 + 8 * rs;
+                    t[k][rs] = make_float4(1.f, 0.f, 1.f, 0.f);
+                    if (a.rope_cs != nullptr && row < x.rope_rows)
+                        t[k][rs] = *reinterpret_cast<const float4 *>(a.rope_cs + (size_t)row * DH + 8 * k + 2 * q4);
                 }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float cv[4] = {t[k][0].x, t[k][0].z, t[k][1].x, t[k][1].z};
+                const float sv[4] = {t[k][0].y, t[k][0].w, t[k][1].y, t[k][1].w};
+                const uint32_t tl0 = tmem + WS_TAB + (lh ? lane16 : lane0) + 8 * k;
+                tmem_st4f(tl0, cv);
+                tmem_st4f(tl0 + DH, sv);
             }
             tmem_wait_st();
         }
