@@ -499,7 +499,10 @@ def headline(args, dev, rank: int, world: int, local_rank: int):
                      "at_tokens": t_now,
                      "how": ("36 decode calls back to back on the decode stream after the timed "
                              "steps (same cache state), CUDA events around the batch, median of 3"),
-                     "decode_share_of_step": dec_ms * L * TOK_PER_STEP / ms_per_step},
+                     "decode_share_of_step": dec_ms * L * TOK_PER_STEP / ms_per_step,
+                     # clock-independent size of the launch: microseconds x median SM MHz
+                     "launch_mcycles": (1e3 * dec_ms * clocks["sm_mhz"] / 1e6
+                                        if clocks.get("sm_mhz") else None)},
         "fold": {"head_block_updates_per_step": L * S * H * 2,
                  "fill_head_block_updates_per_s": fill_updates / (fill_ms / 1e3),
                  "fill_ms": fill_ms, "fill_folds_per_unit": wl.n_c(T0) // wl.block,
@@ -729,6 +732,51 @@ def long_prefill(args, dev, flush, calls: int = 5):
             "decode_frac_of_hbm": nbytes / (dec_us / 1e6) / 1e9 / hbm}
 
 
+def long_decode_bf16(args, dev, flush, calls: int = 5):
+    """The long-context layer of `long_prefill` with bf16 coordinates (the storage at which the
+    compressed cache is smaller than the bf16 cache; read by the persistent decode): the 65536-row
+    prefill in one append, then decode calls over the 65024 compressed rows, L2 flushed."""
+    import torch
+    wl = WL_PREFILL
+    S, H, T0, QH = wl.batch, wl.n_kv_heads, wl.prefill, wl.n_q_heads
+    cache = _cache(wl, n_layers=1, coord_bf16=True)
+    s = torch.cuda.Stream(device=dev)
+    sh = s.cuda_stream
+    with torch.cuda.stream(s):
+        Kr = syn.device_rows_batch(wl, range(S), 0, range(H), 0, T=T0, device=dev)
+        Vr = syn.device_rows_batch(wl, range(S), 0, range(H), 1, T=T0, device=dev)
+        cache.append(0, Kr, Vr, sh)
+        del Kr, Vr
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(4242)
+        q = torch.randn((S, QH, D), generator=gen, device=dev)
+        out = torch.empty_like(q)
+    s.synchronize()
+    assert cache.status(sh) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for i in range(args.warmup + calls):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0.record(s)
+            cache.decode(0, q, out, sh)
+            e1.record(s)
+        s.synchronize()
+        if i >= args.warmup:
+            ms.append(e0.elapsed_time(e1))
+    assert cache.status(sh) == 0 and bool(torch.isfinite(out).all())
+    stored = cache.storage_bytes(0)
+    cache.close()
+    hbm, _ = peaks()
+    dec_us = 1e3 * float(np.median(ms))
+    nbytes = decode_bytes(T0, wl, csz=2)
+    return {"workload": f"{wl.name}: one layer after the {T0}-row prefill, bf16 coordinates",
+            "storage_bytes": stored, "compression_vs_bf16_cache": S * H * 2 * T0 * D * 2 / stored,
+            "decode_us": dec_us, "decode_bytes": nbytes,
+            "decode_achieved_gbs": nbytes / (dec_us / 1e6) / 1e9,
+            "decode_frac_of_hbm": nbytes / (dec_us / 1e6) / 1e9 / hbm}
+
+
 def layer_decode(args, dev, flush, coords: str, calls: int = 10):
     """One layer of the headline workload (batch 8 x 8 kv-heads, 32 q-heads) filled to 32768 tokens
     in one append, then decode calls, each after an L2 flush (CUDA events, median): the per-call
@@ -850,6 +898,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         out["llama3_8b_layer_stream"] = llama_layer_stream(args, dev, flush)
         out.update(all_layers_decode_step(args, dev, flush))
         out["long_prefill"] = long_prefill(args, dev, flush)
+        out["long_decode_bf16"] = long_decode_bf16(args, dev, flush)
         del flush
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline()
