@@ -1258,76 +1258,94 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
     }
 }
 
-// ---- merge: one CTA per unit; thread j owns output channel j of every q-head -------------------
+// ---- merge: one CTA of 256 threads per unit -----------------------------------------------------
+// The unit's records (two per CTA whose range touches it) are read in parallel: first their
+// references and sums, then every output element's weighted sum over the records, with the loads
+// of all records independent; the rank-space sum is expanded once through B_V^T.
+constexpr int WM_THREADS = 256;
+
+__host__ __device__ inline int ws_merge_records(int P) { return 2 * P; }
+
 template <int GT>
-__global__ void __launch_bounds__(128) decode_ws_merge_kernel(DecodeArgs a, WsExtra x) {
+__global__ void __launch_bounds__(WM_THREADS) decode_ws_merge_kernel(DecodeArgs a, WsExtra x) {
     extern __shared__ float msm[];
     const int G = GT, rV = a.r[1], kV = a.k[1];
     const int ldb = kV | 1;
+    const int RM = ws_merge_records(x.P);
     float *sBV = msm;                                   // [D][ldb]
-    float *sAcc = sBV + D * ldb;                        // [G][rV]
+    float *sAcc = sBV + D * ldb;                        // [G][rV] rank-space sums
+    float *sCh = sAcc + G * rV;                         // [G][D] channel-space sums
+    float *sW = sCh + G * D;                            // [RM][G] record references, then weights
+    float *sL = sW + RM * G;                            // [RM][G] record sums
+    float *sML = sL + RM * G;                           // [2][G]: reference M, sum L
+    unsigned long long *sOff = reinterpret_cast<unsigned long long *>(sML + 2 * G + 2);   // [RM]
     const int u = blockIdx.x;
     const int seq = u / a.H, h = u % a.H;
-    const int j = threadIdx.x;
+    const int tid = threadIdx.x;
     ws_griddep_launch();
     if (kV > 0) {
         const float *B = a.basis[1] + (size_t)u * D * rV;
-        for (int o = j; o < D * kV; o += 128) sBV[(o / kV) * ldb + o % kV] = B[(size_t)(o / kV) * rV + o % kV];
+        for (int o = tid; o < D * kV; o += WM_THREADS) sBV[(o / kV) * ldb + o % kV] = B[(size_t)(o / kV) * rV + o % kV];
     }
     ws_griddep_wait();
     // CTAs whose tile ranges touch this unit, and the unit's segment index in each
     const long long x0 = (long long)u * x.Tu, x1 = (long long)(u + 1) * x.Tu - 1;
     const int c_lo = (int)(((x0 + 1) * x.P + x.N - 1) / x.N) - 1;
     const int c_hi = (int)(((x1 + 1) * x.P + x.N - 1) / x.N) - 1;
-    const size_t stride = (size_t)G * (2 + rV + D);
-    float M[GT], Lw[GT], accw[GT];
-#pragma unroll
-    for (int g = 0; g < GT; ++g) {
-        M[g] = -CUDART_INF_F;
-        Lw[g] = 0.f;
-        accw[g] = 0.f;
-    }
-    // every CTA whose range touches the unit left one record per epilogue group
-    for (int c = c_lo; c <= c_hi; ++c) {
+    const int R = 2 * (c_hi - c_lo + 1);
+    const int rs = 2 + rV + D;                          // floats per q-head in a record
+    // record r: CTA c_lo + r / 2, group r % 2, at the unit's segment index in that CTA
+    for (int r = tid; r < R; r += WM_THREADS) {
+        const int c = c_lo + (r >> 1);
         const long long g0 = (long long)c * x.N / x.P;
         const int js = (int)(u - g0 / x.Tu);
-        for (int gr = 0; gr < 2; ++gr) {
-            const float *rec = a.ws + (((size_t)c * x.maxseg + js) * 2 + gr) * stride;
-#pragma unroll
-            for (int g = 0; g < GT; ++g) M[g] = fmaxf(M[g], __ldcg(rec + g * (2 + rV + D)));
-        }
+        sOff[r] = (((unsigned long long)c * x.maxseg + js) * 2 + (r & 1)) * (unsigned long long)G * rs;
     }
-    float accr[GT];
-#pragma unroll
-    for (int g = 0; g < GT; ++g) accr[g] = 0.f;
-    for (int c = c_lo; c <= c_hi; ++c) {
-        const long long g0 = (long long)c * x.N / x.P;
-        const int js = (int)(u - g0 / x.Tu);
-        for (int gr = 0; gr < 2; ++gr) {
-            const float *rec = a.ws + (((size_t)c * x.maxseg + js) * 2 + gr) * stride;
-#pragma unroll
-            for (int g = 0; g < GT; ++g) {
-                const float *r = rec + g * (2 + rV + D);
-                // a group that saw no tile of the unit left m = -inf: weight 0
-                const float m = __ldcg(r);
-                const float w = m == -CUDART_INF_F ? 0.f : ex2(m - M[g]);
-                Lw[g] = fmaf(w, __ldcg(r + 1), Lw[g]);
-                if (j < kV) accr[g] = fmaf(w, __ldcg(r + 2 + j), accr[g]);
-                accw[g] = fmaf(w, __ldcg(r + 2 + rV + j), accw[g]);
-            }
-        }
-    }
-#pragma unroll
-    for (int g = 0; g < GT; ++g)
-        if (j < kV) sAcc[g * rV + j] = accr[g];
     __syncthreads();
-    const float *br = sBV + j * ldb;
-#pragma unroll
-    for (int g = 0; g < GT; ++g) {
-        float o = accw[g];
-        for (int c = 0; c < kV; ++c) o = fmaf(sAcc[g * rV + c], br[c], o);
-        a.out[((size_t)seq * a.H * G + (size_t)h * G + g) * D + j] = o / Lw[g];
+    for (int o = tid; o < R * G; o += WM_THREADS) {
+        const float *rp = a.ws + sOff[o / G] + (o % G) * rs;
+        sW[o] = __ldcg(rp);
+        sL[o] = __ldcg(rp + 1);
     }
+    __syncthreads();
+    if (tid < G) {
+        float m = -CUDART_INF_F;
+        for (int r = 0; r < R; ++r) m = fmaxf(m, sW[r * G + tid]);
+        float l = 0.f;
+        for (int r = 0; r < R; ++r) {
+            // a group that saw no tile of the unit left m = -inf: weight 0
+            const float mr = sW[r * G + tid];
+            const float w = mr == -CUDART_INF_F ? 0.f : ex2(mr - m);
+            sW[r * G + tid] = w;
+            l = fmaf(w, sL[r * G + tid], l);
+        }
+        sML[tid] = m;
+        sML[G + tid] = l;
+    }
+    __syncthreads();
+    // weighted sums of the rank-space (c < rV) and channel-space (c >= rV) parts
+    for (int o = tid; o < G * (rV + D); o += WM_THREADS) {
+        const int g = o / (rV + D), c = o % (rV + D);
+        float acc = 0.f;
+#pragma unroll 4
+        for (int r = 0; r < R; ++r) acc = fmaf(sW[r * G + g], __ldcg(a.ws + sOff[r] + g * rs + 2 + c), acc);
+        if (c < rV) sAcc[g * rV + c] = acc;
+        else sCh[g * D + (c - rV)] = acc;
+    }
+    __syncthreads();
+    for (int o = tid; o < G * D; o += WM_THREADS) {
+        const int g = o / D, j = o % D;
+        const float *br = sBV + j * ldb;
+        float v = sCh[g * D + j];
+        for (int c = 0; c < kV; ++c) v = fmaf(sAcc[g * rV + c], br[c], v);
+        a.out[((size_t)seq * a.H * G + (size_t)h * G + g) * D + j] = v / sML[G + g];
+    }
+}
+
+size_t ws_merge_smem_bytes(int kV, int rV, int G, int P) {
+    // floats, two of alignment slack, then the 8-byte record offsets
+    return ((size_t)D * (kV | 1) + (size_t)G * rV + (size_t)G * D + 2 * (size_t)ws_merge_records(P) * G +
+            2 * (size_t)G + 2) * sizeof(float) + (size_t)ws_merge_records(P) * 8 + 8;
 }
 
 size_t ws_partial_floats(int units, int sms, int G, int rV) {
@@ -1372,7 +1390,7 @@ static cudaError_t launch_ws_t(const CUtensorMap *tmC, const CUtensorMap *tmB, c
     e = cudaLaunchKernelEx(&cfg, decode_ws_kernel<BF, GT>, *tmC, *tmB, a, x);
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3(x.UL);
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(WM_THREADS);
     cfg.dynamicSmemBytes = msmem;
     return cudaLaunchKernelEx(&cfg, decode_ws_merge_kernel<GT>, a, x);
 }
@@ -1381,7 +1399,7 @@ cudaError_t launch_decode_ws(const CUtensorMap *tmC, const CUtensorMap *tmB, con
                              const WsExtra &x, cudaStream_t s) {
     const int esz = a.kv_dtype == ISKV_BF16 ? 2 : 4;
     const size_t smem = ws_smem_bytes(x.factor_bf16, a.r[1], esz, a.G);
-    const size_t msmem = ((size_t)D * (a.k[1] | 1) + (size_t)a.G * a.r[1]) * sizeof(float);
+    const size_t msmem = ws_merge_smem_bytes(a.k[1], a.r[1], a.G, x.P);
     const bool bf = x.factor_bf16 != 0;
     switch (a.G) {
     case 1: return bf ? launch_ws_t<true, 1>(tmC, tmB, a, x, s, smem, msmem)
