@@ -57,6 +57,14 @@ Readings taken where the page is silent (each also stated at its definition):
   ``F B`` in the frozen basis (its orthogonal projection onto ``span B``) and old coordinates stay
   as they are (the basis does not move, so nothing drifts).
 
+* joint per-layer factorisation (``joint=True``; "Reconstruction and Storage" counts persistent
+  storage per layer, and the ranks the page reports only compress when all kv-heads of a layer
+  share one factorisation): the rows of all ``n_kv`` kv-heads of one (layer, sequence) at one
+  position are concatenated, head by head, into one row of length ``n_kv d``; one unit per path
+  factorises those rows exactly as above, and kv-head ``h`` reads columns ``h d .. h d + d - 1`` of
+  its reconstruction (RoPE then per head, as in the per-head mode). Its exact window is the same
+  rows, so it is the concatenation of the per-head windows.
+
 Parity: every function here is pinned by ``tests/test_oracle_*.py`` (closed forms, library special
 cases, invariants and brute force); none is "parity unpinned".
 """
@@ -422,25 +430,38 @@ class OracleCache:
     def __init__(self, batch: int, n_layers: int, n_kv_heads: int, n_q_heads: int,
                  head_dim: int, rank_k: int, rank_v: int, block: int, window: int,
                  rope: bool = False, rope_theta: float = 5e5, rotate: bool = True,
-                 fixed_basis: bool = False, coord_bf16: bool = False):
+                 fixed_basis: bool = False, coord_bf16: bool = False, joint: bool = False):
         self.batch, self.n_layers, self.n_kv, self.n_q = batch, n_layers, n_kv_heads, n_q_heads
-        self.d, self.rope, self.theta = head_dim, rope, rope_theta
-        self.units = [[[[OracleUnit(head_dim, rank_k if w == 0 else rank_v, block, window, rotate,
+        self.d, self.rope, self.theta, self.joint = head_dim, rope, rope_theta, joint
+        # joint: one unit per (layer, sequence, path) over rows of length n_kv d, stored as the
+        # single entry [layer][seq][0]
+        d_unit = n_kv_heads * head_dim if joint else head_dim
+        n_units = 1 if joint else n_kv_heads
+        self.units = [[[[OracleUnit(d_unit, rank_k if w == 0 else rank_v, block, window, rotate,
                                     fixed_basis, coord_bf16)
-                         for w in range(2)] for _ in range(n_kv_heads)] for _ in range(batch)]
+                         for w in range(2)] for _ in range(n_units)] for _ in range(batch)]
                       for _ in range(n_layers)]
 
     def unit(self, layer: int, seq: int, head: int, which: int) -> OracleUnit:
-        return self.units[layer][seq][head][which]
+        """The unit that holds kv-head ``head`` (the layer's joint unit when ``joint``)."""
+        return self.units[layer][seq][0 if self.joint else head][which]
 
     def tokens(self, layer: int) -> int:
         return self.units[layer][0][0][0].t
+
+    def _rows(self, X: np.ndarray, head: int) -> np.ndarray:
+        """Kv-head ``head``'s columns of a reconstruction of its unit."""
+        if not self.joint:
+            return X
+        return X[:, head * self.d:(head + 1) * self.d]
 
     def prefill(self, layer: int, K: np.ndarray, V: np.ndarray, chunk: int, m: int, suffix: int,
                 rho: int) -> None:
         """Prefill with protection ("Prefill Compression"): ``K``, ``V``: ``[batch][n_kv][T0][d]``
         (pre-RoPE keys) of an empty layer. Per kv-head, ``P_K`` from the rotated keys of the rows
         outside the window, ``P_V`` within ``rho`` of ``P_K``; then each unit's prefill."""
+        if self.joint:
+            raise ValueError("prefill with protection is per kv-head: not in the joint mode")
         T0 = K.shape[2]
         end = max(0, T0 - self.units[layer][0][0][0].window)
         pos = np.arange(end)
@@ -455,14 +476,19 @@ class OracleCache:
     def append(self, layer: int, K: np.ndarray, V: np.ndarray) -> None:
         """``K``, ``V``: ``[batch][n_kv][m][d]`` rows (pre-RoPE keys)."""
         for s in range(self.batch):
+            if self.joint:
+                # position i's row of the joint unit: the kv-heads' rows side by side
+                self.units[layer][s][0][0].append(np.concatenate(list(K[s]), axis=1))
+                self.units[layer][s][0][1].append(np.concatenate(list(V[s]), axis=1))
+                continue
             for h in range(self.n_kv):
                 self.units[layer][s][h][0].append(K[s, h])
                 self.units[layer][s][h][1].append(V[s, h])
 
     def keys_values(self, layer: int, seq: int, head: int):
         """Reconstructed keys (RoPE applied when enabled) and values of one kv-head."""
-        K = self.units[layer][seq][head][0].reconstruct()
-        V = self.units[layer][seq][head][1].reconstruct()
+        K = self._rows(self.unit(layer, seq, head, 0).reconstruct(), head)
+        V = self._rows(self.unit(layer, seq, head, 1).reconstruct(), head)
         if self.rope:
             K = rope(K, np.arange(K.shape[0]), self.theta)
         return K, V
@@ -486,7 +512,7 @@ class OracleCache:
         for s in range(self.batch):
             row = []
             for h in range(self.n_kv):
-                X = self.units[layer][s][h][which].reconstruct()
+                X = self._rows(self.unit(layer, s, h, which).reconstruct(), h)
                 if apply_rope and which == 0:
                     X = rope(X, np.arange(X.shape[0]), self.theta)
                 row.append(X)

@@ -162,8 +162,30 @@ def _pin_prefill(m):
             and np.array_equal(rec[[1, 2, 9]], X[[1, 2, 9]]))
 
 
+def _pin_joint(m):
+    """Joint per-layer factorisation: after the first fold the layer's compressed rows are the
+    rank-r truncation (library SVD) of the kv-heads' rows side by side, and kv-head h reads its
+    own d columns of it, for keys and values alike."""
+    d, H, r, b, w = 6, 3, 3, 6, 2
+    rng = np.random.default_rng(12)
+    K = rng.standard_normal((1, H, b + w, d)) * np.arange(1, d + 1) ** -0.5
+    V = rng.standard_normal((1, H, b + w, d))
+    c = m.OracleCache(1, 1, H, H, d, r, r, b, w, joint=True)
+    c.append(0, K, V)
+    for which, X in ((0, K), (1, V)):
+        cat = np.concatenate([X[0, h, :b] for h in range(H)], axis=1)
+        u, sv, vt = np.linalg.svd(cat, full_matrices=False)
+        trunc = (u[:, :r] * sv[:r]) @ vt[:r]
+        for h in range(H):
+            got = c.keys_values(0, 0, h)[which]
+            if not (np.allclose(got[:b], trunc[:, h * d:(h + 1) * d], atol=1e-10)
+                    and np.array_equal(got[b:], X[0, h, b:])):
+                return False
+    return True
+
+
 PINS = [_pin_stacked_svd, _pin_no_truncation, _pin_rope, _pin_attention, _pin_schedule,
-        _pin_stale_two_folds, _pin_fixed_basis, _pin_bf16_coordinates, _pin_prefill]
+        _pin_stale_two_folds, _pin_fixed_basis, _pin_bf16_coordinates, _pin_prefill, _pin_joint]
 
 MUTANTS = {
     "new-row identity block negated": ("Ublk[n:, k:] = np.eye(b)", "Ublk[n:, k:] = -np.eye(b)"),
@@ -200,6 +222,11 @@ MUTANTS = {
         "comp = np.asarray(sorted(set(range(end))), dtype=np.int64)"),
     "bf16: rounding to 7 significant bits": ("u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16\n    return (u.astype(np.uint32) << 16)",
                                              "u = (u + 0xFFFF + ((u >> 17) & 1)) >> 17\n    return (u.astype(np.uint32) << 17)"),
+    "joint: kv-heads concatenated in reverse order": (
+        "np.concatenate(list(K[s]), axis=1)", "np.concatenate(list(K[s])[::-1], axis=1)"),
+    "joint: head slice one head late": (
+        "return X[:, head * self.d:(head + 1) * self.d]",
+        "return X[:, ((head + 1) % self.n_kv) * self.d:((head + 1) % self.n_kv + 1) * self.d]"),
 }
 
 
