@@ -549,7 +549,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         if (!ok) break;
                         mbar_arrive_expect_tx(k_full + ks, WS_BLK);
                         tma_load_2d(sm + L.kst + ks * L.kstage, &tmC, 0,
-                                    (int)(x.row0 + u * a.n_max + t0), k_full + ks);
+                                    (int)(x.row0 + coord_unit(u, a.cdiv) * a.n_max + t0), k_full + ks);
                         ++kt;
                         counters[2] = kt;
                     } else {
@@ -564,7 +564,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                         const uint32_t nb = (uint32_t)rows * rV * fsz;
                         mbar_arrive_expect_tx(v_full + vs, nb);
                         const uint8_t *src = reinterpret_cast<const uint8_t *>(a.coords[1]) +
-                                             ((size_t)u * a.n_max + t0) * rV * fsz;
+                                             ((size_t)coord_unit(u, a.cdiv) * a.n_max + t0) * rV * fsz;
                         bulk_load(dst, src, nb, v_full + vs);
                     } else {
                         const int s0 = (int)(t0 % a.R);
@@ -1258,8 +1258,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
     }
 }
 
-// ---- merge: one CTA of 256 threads per unit -----------------------------------------------------
-// The unit's records (two per CTA whose range touches it) are read in parallel: first their
+// ---- merge: one CTA of 256 threads per (unit, q-head) ----------------------------------------------
+// The unit's records (two per CTA whose range touches it) are read in parallel: first the q-head's
 // references and sums, then every output element's weighted sum over the records, with the loads
 // of all records independent; the rank-space sum is expanded once through B_V^T.
 constexpr int WM_THREADS = 256;
@@ -1273,13 +1273,13 @@ __global__ void __launch_bounds__(WM_THREADS) decode_ws_merge_kernel(DecodeArgs 
     const int ldb = kV | 1;
     const int RM = ws_merge_records(x.P);
     float *sBV = msm;                                   // [D][ldb]
-    float *sAcc = sBV + D * ldb;                        // [G][rV] rank-space sums
-    float *sCh = sAcc + G * rV;                         // [G][D] channel-space sums
-    float *sW = sCh + G * D;                            // [RM][G] record references, then weights
-    float *sL = sW + RM * G;                            // [RM][G] record sums
-    float *sML = sL + RM * G;                           // [2][G]: reference M, sum L
-    unsigned long long *sOff = reinterpret_cast<unsigned long long *>(sML + 2 * G + 2);   // [RM]
-    const int u = blockIdx.x;
+    float *sAcc = sBV + D * ldb;                        // [rV] rank-space sums
+    float *sCh = sAcc + rV;                             // [D] channel-space sums
+    float *sW = sCh + D;                                // [RM] record references, then weights
+    float *sL = sW + RM;                                // [RM] record sums
+    float *sML = sL + RM;                               // [2]: reference M, sum L
+    unsigned long long *sOff = reinterpret_cast<unsigned long long *>(sML + 2);   // [RM]
+    const int u = blockIdx.x, g = blockIdx.y;
     const int seq = u / a.H, h = u % a.H;
     const int tid = threadIdx.x;
     ws_griddep_launch();
@@ -1294,58 +1294,64 @@ __global__ void __launch_bounds__(WM_THREADS) decode_ws_merge_kernel(DecodeArgs 
     const int c_hi = (int)(((x1 + 1) * x.P + x.N - 1) / x.N) - 1;
     const int R = 2 * (c_hi - c_lo + 1);
     const int rs = 2 + rV + D;                          // floats per q-head in a record
-    // record r: CTA c_lo + r / 2, group r % 2, at the unit's segment index in that CTA
+    // record r: CTA c_lo + r / 2, group r % 2, at the unit's segment index in that CTA; this
+    // q-head's part of it
     for (int r = tid; r < R; r += WM_THREADS) {
         const int c = c_lo + (r >> 1);
         const long long g0 = (long long)c * x.N / x.P;
         const int js = (int)(u - g0 / x.Tu);
-        sOff[r] = (((unsigned long long)c * x.maxseg + js) * 2 + (r & 1)) * (unsigned long long)G * rs;
+        const unsigned long long off =
+            (((unsigned long long)c * x.maxseg + js) * 2 + (r & 1)) * (unsigned long long)G * rs +
+            (unsigned long long)g * rs;
+        sOff[r] = off;
+        sW[r] = __ldcg(a.ws + off);
+        sL[r] = __ldcg(a.ws + off + 1);
     }
     __syncthreads();
-    for (int o = tid; o < R * G; o += WM_THREADS) {
-        const float *rp = a.ws + sOff[o / G] + (o % G) * rs;
-        sW[o] = __ldcg(rp);
-        sL[o] = __ldcg(rp + 1);
-    }
-    __syncthreads();
-    if (tid < G) {
+    if (tid < 32) {
+        // reference (warp max) and weights; a group that saw no tile of the unit left m = -inf
         float m = -CUDART_INF_F;
-        for (int r = 0; r < R; ++r) m = fmaxf(m, sW[r * G + tid]);
+        for (int r = tid; r < R; r += 32) m = fmaxf(m, sW[r]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         float l = 0.f;
-        for (int r = 0; r < R; ++r) {
-            // a group that saw no tile of the unit left m = -inf: weight 0
-            const float mr = sW[r * G + tid];
+        for (int r = tid; r < R; r += 32) {
+            const float mr = sW[r];
             const float w = mr == -CUDART_INF_F ? 0.f : ex2(mr - m);
-            sW[r * G + tid] = w;
-            l = fmaf(w, sL[r * G + tid], l);
+            sW[r] = w;
+            l = fmaf(w, sL[r], l);
         }
-        sML[tid] = m;
-        sML[G + tid] = l;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (tid == 0) {
+            sML[0] = m;
+            sML[1] = l;
+        }
     }
     __syncthreads();
     // weighted sums of the rank-space (c < rV) and channel-space (c >= rV) parts
-    for (int o = tid; o < G * (rV + D); o += WM_THREADS) {
-        const int g = o / (rV + D), c = o % (rV + D);
+    for (int c = tid; c < rV + D; c += WM_THREADS) {
         float acc = 0.f;
 #pragma unroll 4
-        for (int r = 0; r < R; ++r) acc = fmaf(sW[r * G + g], __ldcg(a.ws + sOff[r] + g * rs + 2 + c), acc);
-        if (c < rV) sAcc[g * rV + c] = acc;
-        else sCh[g * D + (c - rV)] = acc;
+        for (int r = 0; r < R; ++r) acc = fmaf(sW[r], __ldcg(a.ws + sOff[r] + 2 + c), acc);
+        if (c < rV) sAcc[c] = acc;
+        else sCh[c - rV] = acc;
     }
     __syncthreads();
-    for (int o = tid; o < G * D; o += WM_THREADS) {
-        const int g = o / D, j = o % D;
+    for (int j = tid; j < D; j += WM_THREADS) {
         const float *br = sBV + j * ldb;
-        float v = sCh[g * D + j];
-        for (int c = 0; c < kV; ++c) v = fmaf(sAcc[g * rV + c], br[c], v);
-        a.out[((size_t)seq * a.H * G + (size_t)h * G + g) * D + j] = v / sML[G + g];
+        float v = sCh[j];
+        for (int c = 0; c < kV; ++c) v = fmaf(sAcc[c], br[c], v);
+        a.out[((size_t)seq * a.H * G + (size_t)h * G + g) * D + j] = v / sML[1];
     }
 }
 
 size_t ws_merge_smem_bytes(int kV, int rV, int G, int P) {
-    // floats, two of alignment slack, then the 8-byte record offsets
-    return ((size_t)D * (kV | 1) + (size_t)G * rV + (size_t)G * D + 2 * (size_t)ws_merge_records(P) * G +
-            2 * (size_t)G + 2) * sizeof(float) + (size_t)ws_merge_records(P) * 8 + 8;
+    (void)G;
+    // floats (an even count: the 8-byte record offsets follow aligned), then the offsets
+    return ((size_t)D * (kV | 1) + (size_t)rV + (size_t)D + 2 * (size_t)ws_merge_records(P) + 2 + 1) /
+               2 * 2 * sizeof(float) +
+           (size_t)ws_merge_records(P) * 8 + 8;
 }
 
 size_t ws_partial_floats(int units, int sms, int G, int rV) {
@@ -1389,7 +1395,7 @@ static cudaError_t launch_ws_t(const CUtensorMap *tmC, const CUtensorMap *tmB, c
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, decode_ws_kernel<BF, GT>, *tmC, *tmB, a, x);
     if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3(x.UL);
+    cfg.gridDim = dim3(x.UL, GT);
     cfg.blockDim = dim3(WM_THREADS);
     cfg.dynamicSmemBytes = msmem;
     return cudaLaunchKernelEx(&cfg, decode_ws_merge_kernel<GT>, a, x);
