@@ -93,6 +93,17 @@ typedef struct {
     int prot_cap;         /* 0: iskv_prefill() is not available. >= 1: it is, and the protected */
                           /*    stores hold up to prot_cap exact rows per unit and path        */
                           /*    ("Prefill Compression"; more set ISKV_ERR_CAPACITY, sticky).   */
+    int joint_heads;      /* 1: joint per-layer factorisation ("Reconstruction and Storage",     */
+                          /*    persistent storage per layer): the rows of all n_kv_heads of a   */
+                          /*    (layer, sequence) at one position are concatenated, head by    */
+                          /*    head, into one row of length d = n_kv_heads * head_dim, and one  */
+                          /*    factorisation per (layer, sequence, path) folds them: one        */
+                          /*    coordinate row of rank r per position, shared by the kv-heads,   */
+                          /*    and a d x r basis whose rows h*128 .. h*128+127 reconstruct      */
+                          /*    kv-head h. The exact window stays per kv-head. Needs            */
+                          /*    rank + block <= 128 for both paths, fixed_basis = 0 and          */
+                          /*    prot_cap = 0 (else ISKV_ERR_UNSUPPORTED). 0: one factorisation  */
+                          /*    per (layer, sequence, kv-head, path).                           */
 } iskv_config;
 
 /* Key/value protection of iskv_prefill() ("Prefill Compression", steps 1-2). */

@@ -36,6 +36,7 @@ __all__ = [
     "to_bf16",
     "queries",
     "workload_rows",
+    "joint_workload_rows",
     "device_rows",
     "device_rows_batch",
 ]
@@ -175,6 +176,28 @@ def workload_rows(wl: Workload, seq: int, layer: int, head: int, kv: int, T: int
     rank = wl.rank_k if kv == 0 else wl.rank_v
     X = kv_rows(T, wl.head_dim, seed, _decay(wl, seed, kv), channel_sigma=wl.channel_sigma,
                 variant=variant, rank=rank, scale=(key_scale if kv == 0 else 1.0))
+    if wl.kv_dtype == "bf16":
+        return to_bf16(X)
+    f = X.astype(np.float32)
+    return f, f.astype(np.float64)
+
+
+def joint_workload_rows(wl: Workload, seq: int, layer: int, kv: int, T: int | None = None,
+                        variant: str = "literal", key_scale: float = 1.0):
+    """Rows of all kv-heads of one (sequence, layer, path), drawn as ONE low-rank-plus-noise
+    matrix of ``T x (n_kv_heads d)`` rows (the :func:`kv_rows` recipe with ``d = n_kv_heads
+    head_dim``, so the kv-heads share their dominant directions) and split head by head.
+
+    Returns ``(device_array, oracle_values)``, each ``[n_kv_heads][T][head_dim]``, in the
+    workload's dtype as :func:`workload_rows` does.
+    """
+    seed = unit_seed(wl.cfg_id, seq, layer, 1000, kv)
+    T = wl.tokens if T is None else T
+    H, d = wl.n_kv_heads, wl.head_dim
+    rank = wl.rank_k if kv == 0 else wl.rank_v
+    X = kv_rows(T, H * d, seed, _decay(wl, seed, kv), channel_sigma=wl.channel_sigma,
+                variant=variant, rank=rank, scale=(key_scale if kv == 0 else 1.0))
+    X = np.ascontiguousarray(X.reshape(T, H, d).transpose(1, 0, 2))
     if wl.kv_dtype == "bf16":
         return to_bf16(X)
     f = X.astype(np.float32)

@@ -59,6 +59,7 @@ class iskv_config(ctypes.Structure):
         ("fixed_basis", ctypes.c_int),
         ("coord_bf16", ctypes.c_int),
         ("prot_cap", ctypes.c_int),
+        ("joint_heads", ctypes.c_int),
     ]
 
 

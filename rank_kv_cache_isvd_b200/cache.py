@@ -19,12 +19,13 @@ class IsKVCache:
                  kv_dtype: str = "bf16", rope: bool = True, rope_theta: float = 5e5,
                  rotate_history: bool = True, head_dim: int = 128,
                  lookahead_folds: bool = False, fixed_basis: bool = False,
-                 coord_bf16: bool = False, prot_cap: int = 0):
+                 coord_bf16: bool = False, prot_cap: int = 0, joint_heads: bool = False):
         self.cfg = iskv_config(batch, n_layers, n_kv_heads, n_q_heads, head_dim, rank_k, rank_v,
                                block, window, max_tokens,
                                ISKV_BF16 if kv_dtype == "bf16" else ISKV_F32, int(rope),
                                float(rope_theta), int(rotate_history), int(lookahead_folds),
-                               int(fixed_basis), int(coord_bf16), int(prot_cap))
+                               int(fixed_basis), int(coord_bf16), int(prot_cap),
+                               int(joint_heads))
         self.dtype = torch.bfloat16 if kv_dtype == "bf16" else torch.float32
         self.handle = 0
         code, h = iskv_create(self.cfg)

@@ -74,8 +74,9 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(DecodeArgs a)
     float vacc[4] = {0.f, 0.f, 0.f, 0.f};
 
     const int q4 = tid & 3, rp = tid >> 2;     // channel quarter, row pair
-    const float *Ck = static_cast<const float *>(a.coords[0]) + (size_t)ul * a.n_max * rK;
-    const float *Cv = static_cast<const float *>(a.coords[1]) + (size_t)ul * a.n_max * rV;
+    const long long cu = coord_unit(ul, a.cdiv);     // the kv-head's coordinate unit
+    const float *Ck = static_cast<const float *>(a.coords[0]) + (size_t)cu * a.n_max * rK;
+    const float *Cv = static_cast<const float *>(a.coords[1]) + (size_t)cu * a.n_max * rV;
     const size_t ring_base = (size_t)ul * a.R * D;
 
     for (long long t0 = p0; t0 < p1; t0 += DEC_TILE) {

@@ -211,7 +211,8 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
     }
 
     const size_t ring_base = (size_t)ul * a.R * D;
-    const float *Cv = static_cast<const float *>(a.coords[1]) + (size_t)ul * a.n_max * rV;
+    const long long cu = coord_unit(ul, a.cdiv);   // the kv-head's coordinate unit
+    const float *Cv = static_cast<const float *>(a.coords[1]) + (size_t)cu * a.n_max * rV;
     const uint32_t idesc = idesc_tf32(128, 128);
     const uint32_t abytes = x.kblocks * KBLK_BYTES;
 
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) decode_tc_kernel(
     auto tma_a = [&](long long t0) {
         for (int kb = 0; kb < x.kblocks; ++kb)
             tma_load_2d(bAh + kb * KBLK_BYTES, &tmC, kb * 32,
-                        (int)(x.row0 + (long long)ul * a.n_max + t0), bar_a);
+                        (int)(x.row0 + (long long)cu * a.n_max + t0), bar_a);
     };
     auto issue_v = [&](long long t0, int rows) {
         if (comp) {

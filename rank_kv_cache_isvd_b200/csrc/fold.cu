@@ -1091,4 +1091,271 @@ cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// ---- joint per-layer factorisation --------------------------------------------------------------
+// All kv-heads of a (layer, sequence) share one factorisation over rows of length d = H D (the
+// kv-heads' rows side by side). The fold of such a unit reduces to the per-head fold above through
+// a change of coordinates: with k + b <= 128, the basis B (d x k) and the residual basis P (d x b)
+// span at most 128 dimensions, and in the coordinates of [B P] the block is
+// F~ = F [B P] = [F B | F P], the old basis is [I_k; 0] and the core Z, its SVD, H_top and the new
+// rows' coordinates are exactly those of the d-dimensional fold ("Block-Incremental Decoding
+// Updates", steps 1-3). So a joint fold is
+//   1. joint_prep_kernel: S = F B over the kv-heads' slices, E = F - S B^T, and a Householder QR
+//      of A = [B, E^T] (d x n, n = k + b) streamed over the kv-heads: the first head's 128 rows are
+//      factorised directly, every later head's rows together with the triangular factor so far
+//      (tall-skinny QR, one 128-row block per step). With A = [Q1 Q2] [[R11, R12], [0, R22]],
+//      P = Q2, F P = R22^T (Q2 is orthogonal to B = Q1 R11 and to E's part along Q1) and
+//      F B = S + R12^T R11 (what the single projection left along B). Writes F~ as a fp32 pseudo-
+//      block of b rows of 128 and the pseudo-basis [I_k; 0]; keeps every step's Householder vectors;
+//   2. fold_core_kernel on the pseudo-blocks (Sigma+, H_top, the basis B~+ in the coordinates of
+//      [B P], the new rows' coordinates F~ B~+ = F B+);
+//   3. joint_basis_kernel: B+ = [B P] B~+, forming each kv-head's 128 rows of P from the stored
+//      Householder vectors (last head first: the rows of head h are the head's Householder
+//      product applied to [W; 0], W the product of the later heads' top blocks).
+// Both kernels: one CTA (256 threads) per joint unit and path (blockIdx.y = path).
+
+// A 128-row matrix stored by rows (element (i, c) at s[i LDS + c]) whose pivot rows are its own
+// rows: the first kv-head's QR step.
+struct RowMajorRows {
+    float *s;
+    __device__ float *pivot(int j) const { return s + j * LDS; }
+    __device__ int pstride() const { return 1; }
+    __device__ int y0(int j) const { return j + 1; }
+    __device__ int y1() const { return D; }
+    __device__ float &at(int i, int c) const { return s[i * LDS + c]; }
+};
+
+size_t joint_prep_smem(int k, int b) {
+    return ((size_t)2 * D * LDS + D + (size_t)b * (k + 1)) * sizeof(float);
+}
+
+__global__ void __launch_bounds__(FT, 1) joint_prep_kernel(JointArgs a) {
+    extern __shared__ float smem[];
+    const JointPath P = (a.path_lo + (int)blockIdx.y) ? a.path[1] : a.path[0];
+    float *sY = smem;                      // [D][LDS] a kv-head's rows of A: [B_h | E_h^T]
+    float *sR = sY + D * LDS;              // [n][LDS] triangular factor of the rows so far
+    float *sTau = sR + D * LDS;            // [D]
+    float *sS = sTau + D;                  // [b][k + 1] S = F B
+    const int j = a.junit0 + blockIdx.x;
+    const int k = P.k, b = a.b, n = k + b, H = a.H, r = P.r, ks = k + 1;
+    const int tid = threadIdx.x;
+
+    // kv-head h's rows of [B, F^T]: basis rows in columns 0 .. k-1, block rows transposed in
+    // columns k .. n-1 (row i of sY is channel i of the head)
+    auto stage = [&](int h) {
+        const size_t u = (size_t)j * H + h;
+        const float *Bh = P.basis_in + u * D * r;
+        for (int o = tid; o < D * k; o += FT) {
+            const int i = o / k, l = o % k;
+            sY[i * LDS + l] = Bh[(size_t)i * r + l];
+        }
+        for (int o = tid; o < b * D; o += FT) {
+            const int c = o / D, i = o % D;
+            const int slot = (a.slot0 + c) % a.R;
+            sY[i * LDS + k + c] = load_row_elem(P.ring, (u * a.R + slot) * D + i, a.kv_dtype);
+        }
+    };
+
+    // ---- S = F B = sum_h F_h B_h ------------------------------------------------------------
+    for (int o = tid; o < b * ks; o += FT) sS[o] = 0.f;
+    if (k > 0) {
+        for (int h = 0; h < H; ++h) {
+            __syncthreads();
+            stage(h);
+            __syncthreads();
+            tile_gemm<2, 4>(b, k, D, [&](int c, int i) { return sY[i * LDS + k + c]; },
+                            [&](int i, int l) { return sY[i * LDS + l]; },
+                            [&](int c, int l, float v) { sS[c * ks + l] += v; });
+        }
+    }
+    // ---- per kv-head: E_h = F_h - S B_h^T, then one step of the tall-skinny QR of [B, E^T] ----
+    for (int h = 0; h < H; ++h) {
+        __syncthreads();
+        stage(h);
+        __syncthreads();
+        for (int o = tid; o < D * b; o += FT) {
+            const int i = o / b, c = o % b;
+            float v = sY[i * LDS + k + c];
+            for (int l = 0; l < k; ++l) v = fmaf(-sS[c * ks + l], sY[i * LDS + l], v);
+            sY[i * LDS + k + c] = v;
+        }
+        __syncthreads();
+        if (h == 0) {
+            householder_qr(RowMajorRows{sY}, n, sTau);
+            for (int o = tid; o < n * n; o += FT) {
+                const int i = o / n, c = o % n;
+                sR[i * LDS + c] = c >= i ? sY[i * LDS + c] : 0.f;
+            }
+        } else {
+            // pivot rows: the triangular factor so far; body: this head's 128 rows
+            householder_qr(CoreRows{sY, sR, n, D}, n, sTau);
+        }
+        float *rf = P.refl + ((size_t)j * H + h) * D * a.ldr;
+        for (int o = tid; o < D * n; o += FT) {
+            const int i = o / n, c = o % n;
+            rf[(size_t)i * a.ldr + c] = sY[i * LDS + c];
+        }
+        for (int c = tid; c < n; c += FT) P.tau[((size_t)j * H + h) * a.ldr + c] = sTau[c];
+    }
+    __syncthreads();
+    // ---- F B = S + R12^T R11 -------------------------------------------------------------------
+    for (int o = tid; o < b * k; o += FT) {
+        const int c = o / k, l = o % k;
+        float v = 0.f;
+        for (int m = 0; m <= l; ++m) v = fmaf(sR[m * LDS + k + c], sR[m * LDS + l], v);
+        sS[c * ks + l] += v;
+    }
+    __syncthreads();
+    // ---- pseudo-block [F B | R22^T | 0] and pseudo-basis [I_k; 0] ------------------------------
+    float *blk = P.blk + (size_t)j * b * D;
+    for (int o = tid; o < b * D; o += FT) {
+        const int i = o / D, c = o % D;
+        float v = 0.f;
+        if (c < k) v = sS[i * ks + c];
+        else if (c < n && c - k <= i) v = sR[c * LDS + k + i];   // R22[c - k][i]
+        blk[o] = v;
+    }
+    float *pb = P.pbasis + (size_t)j * D * r;
+    for (int o = tid; o < D * r; o += FT) {
+        const int i = o / r, c = o % r;
+        pb[o] = (i == c && c < k) ? 1.f : 0.f;
+    }
+}
+
+size_t joint_basis_smem(int n, int b, int kp) {
+    return ((size_t)D * (LDS + 1) + (size_t)n * (b + 1) + (size_t)n * kp + D) * sizeof(float);
+}
+
+// QB: columns of P per warp (b <= 8 QB)
+template <int QB>
+__global__ void __launch_bounds__(FT, 1) joint_basis_kernel(JointArgs a) {
+    extern __shared__ float smem[];
+    const JointPath P = (a.path_lo + (int)blockIdx.y) ? a.path[1] : a.path[0];
+    const int j = a.junit0 + blockIdx.x;
+    const int k = P.k, b = a.b, n = k + b, H = a.H, r = P.r, kp = P.kp;
+    const int lw = b + 1, lb = k + 1;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float *sY = smem;                      // [D][LDS] one head's Householder vectors; then P_h, B_h
+    float *sW = sY + D * (LDS + 1);        // [n][b + 1] W: the later heads' top blocks times [0; I_b]
+    float *sBp = sW + n * lw;              // [n][kp] B~+ rows 0 .. n-1 (rows n .. 127 are zero)
+    float *sTau = sBp + n * kp;            // [D]
+    for (int o = tid; o < n * b; o += FT) {
+        const int i = o / b, c = o % b;
+        sW[i * lw + c] = (i == k + c) ? 1.f : 0.f;
+    }
+    const float *bo = P.pbasis_out + (size_t)j * D * r;
+    for (int o = tid; o < n * kp; o += FT) sBp[o] = bo[(size_t)(o / kp) * r + o % kp];
+    for (int h = H - 1; h >= 0; --h) {
+        const float *rf = P.refl + ((size_t)j * H + h) * D * a.ldr;
+        __syncthreads();                   // the previous head's P_h and B_h are consumed
+        for (int o = tid; o < D * n; o += FT) sY[(o / n) * LDS + o % n] = rf[(size_t)(o / n) * a.ldr + o % n];
+        for (int c = tid; c < n; c += FT) sTau[c] = P.tau[((size_t)j * H + h) * a.ldr + c];
+        __syncthreads();
+        // X = [W; 0] (head 0: its 128 rows hold W on top), warp w owning columns w + 8 q, lane l
+        // rows l + 32 u; the head's reflectors applied last to first
+        float xb[QB][4];
+#pragma unroll
+        for (int q = 0; q < QB; ++q)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c = warp + FW * q, i = lane + 32 * u;
+                xb[q][u] = (h == 0 && c < b && i < n) ? sW[i * lw + c] : 0.f;
+            }
+        for (int jr = n - 1; jr >= 0; --jr) {
+            const float tau = sTau[jr];
+            if (tau == 0.f) continue;
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = lane + 32 * u;
+                const float y = sY[i * LDS + jr];
+                // later heads: pivot in the top block (row jr of W), all 128 rows in the body;
+                // head 0: unit pivot at row jr, vector below it
+                v[u] = h > 0 ? y : (i > jr ? y : (i == jr ? 1.f : 0.f));
+            }
+            float w[QB], top[QB];
+#pragma unroll
+            for (int q = 0; q < QB; ++q) {
+                w[q] = 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) w[q] = fmaf(v[u], xb[q][u], w[q]);
+                const int c = warp + FW * q;
+                top[q] = (h > 0 && c < b) ? sW[jr * lw + c] : 0.f;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int q = 0; q < QB; ++q) w[q] += __shfl_xor_sync(0xffffffffu, w[q], o);
+            __syncwarp();                  // every lane has read its top entries
+#pragma unroll
+            for (int q = 0; q < QB; ++q) {
+                const int c = warp + FW * q;
+                if (c < b) {
+                    const float wq = (w[q] + top[q]) * tau;
+                    if (h > 0 && lane == 0) sW[jr * lw + c] = top[q] - wq;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) xb[q][u] = fmaf(-wq, v[u], xb[q][u]);
+                }
+            }
+            __syncwarp();
+        }
+        __syncthreads();                   // every warp is done with the Householder vectors
+        float *sP = sY;                    // [D][b + 1] this head's rows of P
+        float *sBh = sY + D * lw;          // [D][k + 1] this head's rows of B
+#pragma unroll
+        for (int q = 0; q < QB; ++q)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c = warp + FW * q;
+                if (c < b) sP[(lane + 32 * u) * lw + c] = xb[q][u];
+            }
+        const size_t uh = (size_t)j * H + h;
+        const float *Bh = P.basis_in + uh * D * r;
+        for (int o = tid; o < D * k; o += FT) sBh[(o / k) * lb + o % k] = Bh[(size_t)(o / k) * r + o % k];
+        __syncthreads();
+        float *Bo = P.basis_out + uh * D * r;
+        tile_gemm<4, 4>(D, kp, n,
+                        [&](int i, int l) { return l < k ? sBh[i * lb + l] : sP[i * lw + l - k]; },
+                        [&](int l, int c) { return sBp[l * kp + c]; },
+                        [&](int i, int c, float v) { Bo[(size_t)i * r + c] = v; });
+        for (int o = tid; o < D * (r - kp); o += FT)
+            Bo[(size_t)(o / (r - kp)) * r + kp + o % (r - kp)] = 0.f;
+    }
+}
+
+cudaError_t launch_joint_prep(const JointArgs &a, int n_junits, cudaStream_t s) {
+    if (a.path_hi <= a.path_lo || n_junits <= 0) return cudaSuccess;
+    size_t smem = 0;
+    for (int x = a.path_lo; x < a.path_hi; ++x) {
+        const size_t v = joint_prep_smem(a.path[x].k, a.b);
+        smem = v > smem ? v : smem;
+    }
+    static size_t attr[64] = {0};
+    const cudaError_t e = ensure_smem((const void *)joint_prep_kernel, smem, attr);
+    if (e != cudaSuccess) return e;
+    joint_prep_kernel<<<dim3(n_junits, a.path_hi - a.path_lo), FT, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_joint_basis(const JointArgs &a, int n_junits, cudaStream_t s) {
+    if (a.path_hi <= a.path_lo || n_junits <= 0) return cudaSuccess;
+    size_t smem = 0;
+    for (int x = a.path_lo; x < a.path_hi; ++x) {
+        const size_t v = joint_basis_smem(a.path[x].k + a.b, a.b, a.path[x].kp);
+        smem = v > smem ? v : smem;
+    }
+    const dim3 grid(n_junits, a.path_hi - a.path_lo);
+    if (a.b <= 8 * 8) {
+        static size_t attr[64] = {0};
+        const cudaError_t e = ensure_smem((const void *)joint_basis_kernel<8>, smem, attr);
+        if (e != cudaSuccess) return e;
+        joint_basis_kernel<8><<<grid, FT, smem, s>>>(a);
+    } else {
+        static size_t attr[64] = {0};
+        const cudaError_t e = ensure_smem((const void *)joint_basis_kernel<16>, smem, attr);
+        if (e != cudaSuccess) return e;
+        joint_basis_kernel<16><<<grid, FT, smem, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace iskv

@@ -31,6 +31,19 @@ struct iskv_handle {
     float *sigma[2] = {nullptr, nullptr};   // [NB][U][r]
     float *htop[2] = {nullptr, nullptr};    // [NB][U][r][r]
     float *rbig[2] = {nullptr, nullptr};    // [U][128][D] triangular factor of a large block
+    // joint per-layer factorisation (joint_heads): joint unit j = layer * batch + seq holds the
+    // coordinates, Sigma and H_top of all kv-heads of that (layer, sequence); its basis is stored
+    // as the kv-heads' slices at units j H + h
+    bool joint = false;
+    int JL = 0;           // joint units per layer (batch)
+    int CU = 0;           // coordinate units per path: U, or n_layers * batch when joint
+    int CL = 0;           // coordinate units per layer: UL, or batch when joint
+    int ldr = 0;          // column stride of jrefl: max over paths of rank + block
+    float *jblk[2] = {nullptr, nullptr};    // [CU][b][D] pseudo-blocks
+    float *jpb[2] = {nullptr, nullptr};     // [CU][D][r] pseudo-bases [I_k; 0]
+    float *jpbo[2] = {nullptr, nullptr};    // [CU][D][r] fold results in pseudo coordinates
+    float *jrefl[2] = {nullptr, nullptr};   // [CU][n_kv][D][ldr] Householder vectors per kv-head
+    float *jtau[2] = {nullptr, nullptr};    // [CU][n_kv][ldr]
     void *ring[2] = {nullptr, nullptr};
     float2 *rope_cs = nullptr;
     float4 *rope_t = nullptr;             // transposed copy for the tensor-core decode
@@ -96,6 +109,11 @@ void free_all(iskv_handle *h) {
         cudaFree(h->ring[x]);
         cudaFree(h->htop[x]);
         cudaFree(h->rbig[x]);
+        cudaFree(h->jblk[x]);
+        cudaFree(h->jpb[x]);
+        cudaFree(h->jpbo[x]);
+        cudaFree(h->jrefl[x]);
+        cudaFree(h->jtau[x]);
     }
     cudaFree(h->rope_cs);
     cudaFree(h->rope_t);
@@ -213,7 +231,8 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
     for (int x = 0; x < 2; ++x) {
         const int r = rank_of(h, x);
         const int k = h->kf[x][l0];
-        const int p = fz[x] ? 0 : (c.block < D - k ? c.block : D - k);
+        const int dj = h->joint ? c.n_kv_heads * D : D;     // columns of the factorised rows
+        const int p = fz[x] ? 0 : (c.block < dj - k ? c.block : dj - k);
         const int kp = r < k + p ? r : k + p;
         FoldPath &fp = fa.path[x];
         fp.ring = h->ring[x];
@@ -257,7 +276,47 @@ int launch_fold_j(iskv_handle *h, int l0, int nl, long long j, cudaStream_t s) {
     nr.n_c = nc;
     nr.n_max = h->n_max;
     nr.cbf = h->cbf;
-    if (c.block > BMAX) {
+    if (h->joint) {
+        // one factorisation per (layer, sequence): the tall-skinny QR over the kv-heads, the fold
+        // in the coordinates of [B P], then the kv-heads' slices of B+ = [B P] B~+
+        JointArgs ja;
+        memset(&ja, 0, sizeof(ja));
+        for (int x = 0; x < 2; ++x) {
+            JointPath &jp = ja.path[x];
+            jp.ring = h->ring[x];
+            jp.basis_in = fa.path[x].basis_in;
+            jp.basis_out = fa.path[x].basis_out;
+            jp.blk = h->jblk[x];
+            jp.pbasis = h->jpb[x];
+            jp.pbasis_out = h->jpbo[x];
+            jp.refl = h->jrefl[x];
+            jp.tau = h->jtau[x];
+            jp.r = fa.path[x].r;
+            jp.k = fa.path[x].k;
+            jp.kp = fa.path[x].kp;
+            fa.path[x].ring = h->jblk[x];
+            fa.path[x].basis_in = h->jpb[x];
+            fa.path[x].basis_out = h->jpbo[x];
+        }
+        ja.junit0 = l0 * h->JL;
+        ja.H = c.n_kv_heads;
+        ja.ldr = h->ldr;
+        ja.slot0 = fa.slot0;
+        ja.R = h->R;
+        ja.b = c.block;
+        ja.kv_dtype = c.kv_dtype;
+        ja.path_lo = 0;
+        ja.path_hi = 2;
+        fa.unit0 = ja.junit0;
+        fa.slot0 = 0;
+        fa.R = c.block;
+        fa.kv_dtype = ISKV_F32;
+        if (launch_joint_prep(ja, nl * h->JL, s) != cudaSuccess ||
+            launch_fold(fa, nl * h->JL, s) != cudaSuccess ||
+            launch_joint_basis(ja, nl * h->JL, s) != cudaSuccess)
+            return ISKV_ERR_CUDA;
+        h->launches += 3;
+    } else if (c.block > BMAX) {
         // large block: fold the 128-row triangular factor of the block (same Sigma+, H and basis),
         // then the coordinates of the block's real rows
         RFactorArgs rf;
@@ -351,12 +410,12 @@ int apply_fold(iskv_handle *h, int l0, int nl, cudaStream_t s) {
             rp.k = f[2 * x];
             rp.kp = f[2 * x + 1];
         }
-        ra.unit0 = l0 * h->UL;
+        ra.unit0 = l0 * h->CL;
         ra.n_old = nc;
         ra.n_max = h->n_max;
         ra.stale = c.rotate_history ? 0 : 1;
         ra.cbf = h->cbf;
-        if (launch_rotate(ra, nl * h->UL, s) != cudaSuccess) return ISKV_ERR_CUDA;
+        if (launch_rotate(ra, nl * h->CL, s) != cudaSuccess) return ISKV_ERR_CUDA;
         h->launches += 1;
     }
     for (int l = l0; l < l0 + nl; ++l) {
@@ -449,6 +508,9 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         c.prot_cap < 0)
         return ISKV_ERR_INVALID_ARG;
     if (c.block > BMAX_LARGE) return ISKV_ERR_UNSUPPORTED;
+    if (c.joint_heads && (c.rank_k + c.block > D || c.rank_v + c.block > D || c.fixed_basis ||
+                          c.prot_cap > 0))
+        return ISKV_ERR_UNSUPPORTED;
     iskv_handle *h = new (std::nothrow) iskv_handle();
     if (!h) return ISKV_ERR_CUDA;
     try {
@@ -460,6 +522,11 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
         cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
         h->UL = c.batch * c.n_kv_heads;
         h->U = c.n_layers * h->UL;
+        h->joint = c.joint_heads != 0;
+        h->JL = c.batch;
+        h->CL = h->joint ? c.batch : h->UL;
+        h->CU = c.n_layers * h->CL;
+        h->ldr = (c.rank_k > c.rank_v ? c.rank_k : c.rank_v) + c.block;
         h->R = c.window + c.block;
         h->G = c.n_q_heads / c.n_kv_heads;
         // compressed positions: up to max_tokens - window (a prefill's end need not be a
@@ -504,7 +571,15 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
     for (int x = 0; x < 2; ++x) {
         const size_t r = (size_t)rank_of(h, x);
         const size_t nb = (size_t)h->NB;
-        alloc((void **)&h->coords[x], U * (size_t)h->n_max * r * h->csz);
+        alloc((void **)&h->coords[x], (size_t)h->CU * (size_t)h->n_max * r * h->csz);
+        if (h->joint) {
+            const size_t J = (size_t)h->CU, Hk = (size_t)c.n_kv_heads;
+            alloc((void **)&h->jblk[x], J * c.block * D * sizeof(float));
+            alloc((void **)&h->jpb[x], J * D * r * sizeof(float));
+            alloc((void **)&h->jpbo[x], J * D * r * sizeof(float));
+            alloc((void **)&h->jrefl[x], J * Hk * D * h->ldr * sizeof(float));
+            alloc((void **)&h->jtau[x], J * Hk * h->ldr * sizeof(float));
+        }
         alloc((void **)&h->basis[x], nb * U * D * r * sizeof(float));
         alloc((void **)&h->sigma[x], nb * U * r * sizeof(float));
         alloc(&h->ring[x], U * (size_t)h->R * D * h->esz);
@@ -573,7 +648,7 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
                     (h->G == 1 || h->G == 2 || h->G == 4) &&
                     ws_smem_bytes(1, c.rank_v, (int)h->esz, h->G) <= 227 * 1024;
         if (m_ok && h->n_max > 0)
-            m_ok = make_map(&h->tmC, h->coords[0], c.rank_k, (long long)h->U * h->n_max, true);
+            m_ok = make_map(&h->tmC, h->coords[0], c.rank_k, (long long)h->CU * h->n_max, true);
         if (!m_ok) {
             free_all(h);
             delete h;
@@ -584,7 +659,7 @@ int iskv_create(const iskv_config *cfg, iskv_handle **out) {
                tc_smem_bytes((c.rank_k + 31) / 32, c.rank_v, (int)h->esz, h->G) <= 227 * 1024) {
         bool m_ok = true;
         if (h->n_max > 0) {
-            m_ok = make_map(&h->tmC, h->coords[0], c.rank_k, (long long)h->U * h->n_max) &&
+            m_ok = make_map(&h->tmC, h->coords[0], c.rank_k, (long long)h->CU * h->n_max) &&
                    make_map(&h->tmB, h->basis[0], c.rank_k, (long long)h->NB * h->U * D);
         }
         h->tc = m_ok;
@@ -668,8 +743,8 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
     const int cur = current_buffer(h, layer);
     for (int x = 0; x < 2; ++x) {
         const size_t r = (size_t)rank_of(h, x);
-        const size_t u0 = (size_t)layer * h->UL;
-        da.coords[x] = static_cast<const char *>(h->coords[x]) + u0 * (size_t)h->n_max * r * h->csz;
+        const size_t u0 = (size_t)layer * h->UL, c0 = (size_t)layer * h->CL;
+        da.coords[x] = static_cast<const char *>(h->coords[x]) + c0 * (size_t)h->n_max * r * h->csz;
         da.basis[x] = basis_buf(h, x, cur) + u0 * D * r;
         da.ring[x] = static_cast<const char *>(h->ring[x]) + u0 * (size_t)h->R * D * h->esz;
         da.r[x] = (int)r;
@@ -689,6 +764,7 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
     da.new_row[1] = new_v;
     da.new_pos = new_k ? da.t - 1 : -1;
     da.cbf = h->cbf;
+    da.cdiv = h->joint ? c.n_kv_heads : 1;
     // compressed splits: at most one wave of CTAs over all units of the layer (two per SM when
     // two fit in shared memory), the compressed tiles of a unit spread evenly over its splits
     const long long ctiles = (da.n_c + DEC_TILE - 1) / DEC_TILE;
@@ -705,17 +781,17 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
     da.max_splits = h->max_splits;
     da.kv_dtype = c.kv_dtype;
     da.scale = 1.0f / sqrtf((float)D);
-    // the persistent decode pays off once every SM streams many tiles; smaller calls (fp32
+    // the persistent decode pays off once every SM streams several tiles; smaller calls (fp32
     // coordinates, no protection) use the split-kernel decode
     const long long tiles_ws = (long long)h->UL * (ctiles + (e + DEC_TILE - 1) / DEC_TILE);
     const bool use_ws = h->ws_ok && (h->cbf || h->pact[layer] || !h->tc ||
-                                     tiles_ws >= 8LL * h->sms);
+                                     tiles_ws >= 6LL * h->sms);
     if (use_ws) {
         if (reinterpret_cast<uintptr_t>(q) % 16 != 0) return ISKV_ERR_INVALID_ARG;
         WsExtra x;
         memset(&x, 0, sizeof(x));
         x.rope_rows = c.max_tokens;
-        x.row0 = (long long)layer * h->UL * h->n_max;
+        x.row0 = (long long)layer * h->CL * h->n_max;
         x.brow0 = (cur * h->U + layer * h->UL) * D;
         x.Tc = (int)ctiles;
         x.Tw = (int)((e + DEC_TILE - 1) / DEC_TILE);
@@ -758,7 +834,7 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
         if (reinterpret_cast<uintptr_t>(q) % 16 != 0) return ISKV_ERR_INVALID_ARG;
         TcExtra x;
         x.kblocks = (c.rank_k + 31) / 32;
-        x.row0 = (long long)layer * h->UL * h->n_max;
+        x.row0 = (long long)layer * h->CL * h->n_max;
         x.brow0 = (cur * h->U + layer * h->UL) * D;
         x.rope_t = c.rope ? h->rope_t : nullptr;
         x.rope_rows = c.max_tokens;
@@ -987,11 +1063,12 @@ int iskv_reconstruct(iskv_handle *h, int layer, int which, int apply_rope, float
         return ISKV_ERR_INVALID_ARG;
     DeviceGuard g(h->device);
     const size_t r = (size_t)rank_of(h, which);
-    const size_t u0 = (size_t)layer * h->UL;
+    const size_t u0 = (size_t)layer * h->UL, c0 = (size_t)layer * h->CL;
     ReconArgs ra;
     memset(&ra, 0, sizeof(ra));
-    ra.coords = static_cast<const char *>(h->coords[which]) + u0 * (size_t)h->n_max * r * h->csz;
+    ra.coords = static_cast<const char *>(h->coords[which]) + c0 * (size_t)h->n_max * r * h->csz;
     ra.cbf = h->cbf;
+    ra.cdiv = h->joint ? h->cfg.n_kv_heads : 1;
     ra.basis = basis_buf(h, which, current_buffer(h, layer)) + u0 * D * r;
     ra.ring = static_cast<const char *>(h->ring[which]) + u0 * (size_t)h->R * D * h->esz;
     ra.rope_cs = h->rope_cs;
@@ -1029,9 +1106,11 @@ int iskv_get_factors(iskv_handle *h, int layer, int seq, int kv_head, int which,
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t r = (size_t)rank_of(h, which);
     const size_t u = ((size_t)layer * h->cfg.batch + seq) * h->cfg.n_kv_heads + kv_head;
+    // coordinates, Sigma: the kv-head's unit, or the (layer, sequence)'s joint unit
+    const size_t cu = h->joint ? (size_t)layer * h->cfg.batch + seq : u;
     const long long nc = h->nc[layer];
     if (coords && nc > 0) {
-        const void *src = static_cast<const char *>(h->coords[which]) + u * (size_t)h->n_max * r * h->csz;
+        const void *src = static_cast<const char *>(h->coords[which]) + cu * (size_t)h->n_max * r * h->csz;
         const cudaError_t e = h->cbf ? launch_coords_to_f32(coords, src, (size_t)nc * r, s)
                                      : cudaMemcpyAsync(coords, src, (size_t)nc * r * sizeof(float),
                                                        cudaMemcpyDeviceToDevice, s);
@@ -1042,7 +1121,7 @@ int iskv_get_factors(iskv_handle *h, int layer, int seq, int kv_head, int which,
     if (basis && cudaMemcpyAsync(basis, basis_buf(h, which, cur) + u * D * r,
                                  D * r * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
         return ISKV_ERR_CUDA;
-    if (sigma && cudaMemcpyAsync(sigma, sigma_buf(h, which, cur) + u * r, r * sizeof(float),
+    if (sigma && cudaMemcpyAsync(sigma, sigma_buf(h, which, cur) + cu * r, r * sizeof(float),
                                  cudaMemcpyDeviceToDevice, s) != cudaSuccess)
         return ISKV_ERR_CUDA;
     if (k_out) *k_out = h->kcur[which][layer];
@@ -1119,10 +1198,12 @@ int iskv_num_tokens(const iskv_handle *h, int layer, long long *t_out) {
 int iskv_storage_bytes(const iskv_handle *h, int layer, long long *bytes_out) {
     if (!h || !bytes_out || !valid_layer(h, layer)) return ISKV_ERR_INVALID_ARG;
     const long long n = h->nc[layer], e = h->t[layer] - n;
+    // factor units of the layer and the length d of their rows
+    const long long fu = h->CL, d = h->joint ? (long long)h->cfg.n_kv_heads * D : D;
     long long f = 0;
     for (int x = 0; x < 2; ++x)
-        f += (long long)h->kcur[x][layer] * ((long long)h->csz * n + 4LL * (D + 1));
-    *bytes_out = (long long)h->UL * (f + (long long)h->esz * D * 2LL * e);
+        f += (long long)h->kcur[x][layer] * ((long long)h->csz * n + 4LL * (d + 1));
+    *bytes_out = fu * f + (long long)h->UL * (long long)h->esz * D * 2LL * e;
     return ISKV_OK;
 }
 

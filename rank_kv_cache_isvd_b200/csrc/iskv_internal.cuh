@@ -82,6 +82,29 @@ struct NewRowsArgs {
     long long flag_stride;
 };
 
+// ---- joint per-layer fold (joint_heads): one factorisation over all kv-heads of a (layer, seq) --
+// Joint unit j = (layer, sequence) owns kv-head units j H .. j H + H - 1; its basis is stored as
+// their per-head slices (d = H D rows in H blocks of D), its coordinates, Sigma and H_top at j.
+struct JointPath {
+    const void *ring;         // [units][R][D] exact rows per kv-head (kv dtype)
+    const float *basis_in;    // [units][D][r] kv-head slices of the joint bases before the fold
+    float *basis_out;         // [units][D][r] after the fold
+    float *blk;               // [junits][b][D] fp32 pseudo-block F [B P] = [F B | R22^T | 0]
+    float *pbasis;            // [junits][D][r] pseudo-basis [I_k; 0]
+    const float *pbasis_out;  // [junits][D][r] the fold's basis in the coordinates of [B P]
+    float *refl;              // [junits][H][D][ldr] Householder vectors of each kv-head's QR step
+    float *tau;               // [junits][H][ldr]
+    int r, k, kp;             // rank budget, rank before, rank after
+};
+struct JointArgs {
+    JointPath path[2];
+    int junit0;               // first joint unit of the call
+    int H;                    // kv-heads per joint unit
+    int ldr;                  // column stride of refl (>= k + b of both paths)
+    int slot0, R, b, kv_dtype;
+    int path_lo, path_hi;     // paths processed: path_lo .. path_hi - 1
+};
+
 // ---- prefill protection ------------------------------------------------------------------------
 struct ProtArgs {
     const void *keys;       // [call units][src_rows][D] pre-RoPE key rows
@@ -157,7 +180,13 @@ struct DecodeArgs {
     const void *new_row[2];
     long long new_pos;      // -1: no fused append
     int cbf;                // 1: coordinates stored in bf16 (persistent decode only)
+    int cdiv;               // kv-heads sharing one coordinate unit (joint factorisation), else 1
 };
+
+// coordinate unit of kv-head unit u (joint factorisation: the kv-heads of a sequence share one)
+__host__ __device__ __forceinline__ long long coord_unit(long long u, int cdiv) {
+    return cdiv > 1 ? u / cdiv : u;
+}
 
 // ---- reconstruct ------------------------------------------------------------------------------
 struct ReconArgs {
@@ -170,6 +199,7 @@ struct ReconArgs {
     long long n_c, t, n_max;
     int R, kv_dtype, apply_rope;
     int cbf;
+    int cdiv;               // kv-heads sharing one coordinate unit (joint factorisation), else 1
     // prefill protection of this path (pflags nullptr: none); pointers start at the layer's units
     const unsigned char *pflags;
     long long fstride;
@@ -216,6 +246,8 @@ cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_rfactor(const RFactorArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_newrows(const NewRowsArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s);
+cudaError_t launch_joint_prep(const JointArgs &a, int n_junits, cudaStream_t s);
+cudaError_t launch_joint_basis(const JointArgs &a, int n_junits, cudaStream_t s);
 cudaError_t launch_append(const AppendArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int n_units, cudaStream_t s);
 cudaError_t launch_reconstruct(const ReconArgs &a, int n_units, cudaStream_t s);

@@ -100,7 +100,7 @@ __global__ void reconstruct_kernel(ReconArgs a) {
                     ? load_row_elem(a.pstore, ((size_t)unit * a.pcap + lo) * D + j, a.kv_dtype)
                     : 0.f;
         } else if (pos < a.n_c) {
-            const size_t ci = ((size_t)unit * a.n_max + pos) * r;
+            const size_t ci = ((size_t)coord_unit(unit, a.cdiv) * a.n_max + pos) * r;
             float s = 0.f;
             for (int l = 0; l < k; ++l) s = fmaf(load_coord(a.coords, ci + l, a.cbf), sB[j * ks + l], s);
             x = s;

@@ -37,6 +37,28 @@ def workload_arrays(wl, T=None, variant="literal", key_scale=1.0, layers=None, s
     return out[0], out[1], out[2], out[3]
 
 
+def joint_workload_arrays(wl, T=None, variant="literal", key_scale=1.0, layers=None, seqs=None):
+    """Like :func:`workload_arrays`, with each (layer, sequence)'s kv-heads drawn jointly
+    (:func:`iskv_synth.joint_workload_rows`): ``(k_dev, k_val, v_dev, v_val)``, each
+    ``[L][S][H][T][D]``."""
+    layers = range(wl.n_layers) if layers is None else layers
+    seqs = range(wl.batch) if seqs is None else seqs
+    out = []
+    for kv in (0, 1):
+        dev, val = [], []
+        for l in layers:
+            dl, vl = [], []
+            for s in seqs:
+                d_, v_ = syn.joint_workload_rows(wl, s, l, kv, T=T, variant=variant,
+                                                 key_scale=key_scale)
+                dl.append(d_)
+                vl.append(v_)
+            dev.append(dl)
+            val.append(vl)
+        out += [np.asarray(dev), np.asarray(val)]
+    return out[0], out[1], out[2], out[3]
+
+
 def to_device(arr: np.ndarray):
     import torch
     if arr.dtype == np.uint16:

@@ -71,6 +71,17 @@ def test_create_reports_unsupported_block():
     assert code == iskv.ISKV_ERR_UNSUPPORTED and h == 0
 
 
+@pytest.mark.parametrize("bad", [
+    dict(joint_heads=1, rank_k=80, block=64),           # rank + block > 128
+    dict(joint_heads=1, rank_v=72, block=64),
+    dict(joint_heads=1, fixed_basis=1),
+    dict(joint_heads=1, prot_cap=16),
+])
+def test_joint_factorisation_limits_are_refused_before_any_cuda_call(bad):
+    code, h = iskv.iskv_create(_cfg(**bad))
+    assert code == iskv.ISKV_ERR_UNSUPPORTED and h == 0
+
+
 def test_null_handle_and_strerror():
     assert iskv.iskv_destroy(None) == 0
     assert iskv.iskv_append_block(None, 0, 1, 1, 1, 0) == iskv.ISKV_ERR_INVALID_ARG
