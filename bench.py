@@ -777,6 +777,79 @@ def long_decode_bf16(args, dev, flush, calls: int = 5):
             "decode_frac_of_hbm": nbytes / (dec_us / 1e6) / 1e9 / hbm}
 
 
+def joint_layer(args, dev, flush, calls: int = 5):
+    """One layer of the headline model (batch 8 x 8 kv-heads, 32 q-heads, 32768 tokens) with the
+    joint per-layer factorisation: the 8 kv-heads of a sequence share one factorisation of rows of
+    d = 1024, at b = 64, r_K = 32, r_V = 64 (rank + block <= 128). All 32768 rows are appended in
+    one call (508 folds per joint unit and path), timed as a graph replay; then decode calls at
+    t = 32768 after an L2 flush (fp32 coordinates)."""
+    import dataclasses
+
+    import torch
+    wl = dataclasses.replace(WL, block=64)
+    S, H, T, QH = wl.batch, wl.n_kv_heads, wl.tokens, wl.n_q_heads
+    cache = _cache(wl, n_layers=1, joint_heads=True)
+    s = torch.cuda.Stream(device=dev)
+    sh = s.cuda_stream
+    with torch.cuda.stream(s):
+        K = syn.device_rows_batch(wl, range(S), 0, range(H), 0, device=dev)
+        V = syn.device_rows_batch(wl, range(S), 0, range(H), 1, device=dev)
+        cache.append(0, K, V, sh)
+    s.synchronize()
+    assert cache.status(sh) == 0
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        cache.reset(sh)
+        cache.append(0, K, V, sh)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    app = []
+    for _ in range(2):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0.record(s)
+            g.replay()
+            e1.record(s)
+        s.synchronize()
+        app.append(e0.elapsed_time(e1))
+    del g, K, V
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(777)
+    q = torch.randn((S, QH, D), generator=gen, device=dev)
+    out = torch.empty_like(q)
+    ms = []
+    for i in range(args.warmup + calls):
+        with torch.cuda.stream(s):
+            flush.zero_()
+            e0.record(s)
+            cache.decode(0, q, out, sh)
+            e1.record(s)
+        s.synchronize()
+        if i >= args.warmup:
+            ms.append(e0.elapsed_time(e1))
+    assert cache.status(sh) == 0 and bool(torch.isfinite(out).all())
+    stored = cache.storage_bytes(0)
+    cache.close()
+    hbm, _ = peaks()
+    folds = wl.n_c(T) // wl.block
+    n = wl.n_c(T)
+    kK, kV = wl.rank_k, wl.rank_v
+    # algorithmic bytes: each sequence's shared coordinates once, every kv-head's basis slice and
+    # window rows, q and out
+    nbytes = S * (4 * n * (kK + kV) + H * (2 * 2 * (T - n) * D + 4 * D * (kK + kV)
+                                           + 2 * 4 * wl.group * D))
+    dec_us = 1e3 * float(np.median(ms))
+    app_ms = float(min(app))
+    return {"workload": (f"{wl.name}, joint factorisation of the 8 kv-heads (d = 1024), b = 64: "
+                         f"one layer, {T} rows appended in one call, then decode"),
+            "append_ms": app_ms, "folds_per_joint_unit": folds,
+            "per_fold_ms": app_ms / folds,
+            "joint_block_updates_per_s": 2 * S * folds / (app_ms / 1e3),
+            "storage_bytes": stored, "compression_vs_bf16_cache": S * H * 2 * T * D * 2 / stored,
+            "decode_us": dec_us, "decode_bytes": nbytes,
+            "decode_achieved_gbs": nbytes / (dec_us / 1e6) / 1e9,
+            "decode_frac_of_hbm": nbytes / (dec_us / 1e6) / 1e9 / hbm}
+
+
 def layer_decode(args, dev, flush, coords: str, calls: int = 10):
     """One layer of the headline workload (batch 8 x 8 kv-heads, 32 q-heads) filled to 32768 tokens
     in one append, then decode calls, each after an L2 flush (CUDA events, median): the per-call
@@ -899,6 +972,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         out.update(all_layers_decode_step(args, dev, flush))
         out["long_prefill"] = long_prefill(args, dev, flush)
         out["long_decode_bf16"] = long_decode_bf16(args, dev, flush)
+        out["joint_layer"] = joint_layer(args, dev, flush)
         del flush
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline()
