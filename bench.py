@@ -81,12 +81,14 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="headline line only")
     p.add_argument("--coords", choices=["bf16", "f32"], default="f32",
                    help="storage of the coordinates C = U Sigma (bases and Sigma stay fp32)")
-    p.add_argument("--profile-case", choices=["short", "long", "prefill"], nargs="?",
+    p.add_argument("--profile-case", choices=["short", "long", "prefill", "joint"], nargs="?",
                    const="short",
                    help="run a short program for profiler captures instead of the bench: "
                         "'short' = the Llama-3-8B layer at 4096 tokens, 'long' = one layer of the "
                         "headline workload filled to 32768 tokens, 'prefill' = one long-context "
-                        "layer (65536 rows in 512-row blocks)")
+                        "layer (65536 rows in 512-row blocks), 'joint' = one Qwen3-8B-shaped layer "
+                        "of 2 sequences with the joint factorisation of its 8 kv-heads (4096 rows, "
+                        "b = 64)")
     return p.parse_args()
 
 
@@ -993,6 +995,20 @@ def run_profile_case(which: str, coords: str = "bf16"):
         Q = torch.from_numpy(q[T - 1]).cuda()
         cache = _cache(wl, coord_bf16=coords == "bf16")
         cache.append(0, K.contiguous()[None], V.contiguous()[None])
+    elif which == "joint":
+        # joint factorisation of a Qwen3-8B-shaped layer's 8 kv-heads (d = 1024, b = 64), two
+        # sequences, 4096 tokens appended in one call (60 folds per joint unit and path)
+        import dataclasses
+        wl = dataclasses.replace(WL, batch=2, tokens=4096, block=64)
+        T = wl.tokens
+        cache = _cache(wl, n_layers=1, coord_bf16=coords == "bf16", joint_heads=True)
+        K = syn.device_rows_batch(wl, range(wl.batch), 0, range(wl.n_kv_heads), 0, T=T, device=dev)
+        V = syn.device_rows_batch(wl, range(wl.batch), 0, range(wl.n_kv_heads), 1, T=T, device=dev)
+        cache.append(0, K, V)
+        del K, V
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(12345)
+        Q = torch.randn((wl.batch, wl.n_q_heads, D), generator=gen, device=dev)
     else:
         wl = WL if which == "long" else WL_PREFILL
         T = wl.tokens if which == "long" else wl.prefill
@@ -1009,7 +1025,8 @@ def run_profile_case(which: str, coords: str = "bf16"):
     torch.cuda.synchronize()
     print(json.dumps({"profile_case": which, "workload": wl.name, "tokens": cache.tokens(0),
                       "coords": coords,
-                      "decode_bytes": decode_bytes(cache.tokens(0), wl, csz=2 if coords == "bf16" else 4),
+                      "decode_bytes": (None if which == "joint" else
+                                       decode_bytes(cache.tokens(0), wl, csz=2 if coords == "bf16" else 4)),
                       "status": cache.status(), "launches": cache.launches(),
                       "out_norm": float(out.norm())}))
     cache.close()

@@ -201,3 +201,59 @@ def test_joint_two_layers_two_sequences_lookahead_and_persistent_decode():
                 ref[s, g] = attention(q[s, g].astype(np.float64), Kr, V)
     assert max_head_rel_err(out, ref) <= ATTN_TOL
     assert c.status() == 0
+
+
+@pytest.mark.parametrize("lookahead", [False, True])
+def test_joint_fused_append_decode_equals_separate_calls(lookahead):
+    """iskv_append_decode in the joint mode gives bit for bit the outputs and reconstructions of
+    iskv_append_block + iskv_decode_attn across fold triggers; the reconstruction (kv-head slices
+    of the shared factorisation) matches the oracle's."""
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=700)
+    kd, kv, vd, vv = joint_workload_arrays(wl, variant="gapped")
+    K, V = to_device(kd[0]), to_device(vd[0])
+    Q = torch.from_numpy(syn.queries(61, (wl.tokens, 1, 8, 128))).cuda()
+    outs = []
+    for fused in (False, True):
+        cache = make_cache(wl, lookahead_folds=lookahead)
+        out = torch.empty_like(Q)
+        for t in range(wl.tokens):
+            kr = K[:, :, t:t + 1].contiguous()
+            vr = V[:, :, t:t + 1].contiguous()
+            if fused:
+                cache.append_decode(0, kr, vr, Q[t], out[t])
+            else:
+                cache.append(0, kr, vr)
+                cache.decode(0, Q[t], out[t])
+        assert cache.status() == 0 and cache.tokens(0) == wl.tokens
+        outs.append((out, [cache.reconstruct(0, x) for x in (0, 1)]))
+        cache.close()
+    (o0, r0), (o1, r1) = outs
+    assert torch.equal(o0, o1)
+    assert torch.equal(r0[0], r1[0]) and torch.equal(r0[1], r1[1])
+    orc = make_oracle(wl)
+    orc.append(0, kv[0], vv[0])
+    for x in (0, 1):
+        assert rel_err(r0[x].cpu().numpy(), orc.reconstruct(0, x)) <= SIG_TOL
+
+
+def test_joint_stale_coordinates_mode_matches_oracle():
+    """The stale-coordinate ablation on a joint factorisation: Sigma and B as the oracle's joint
+    unit with rotate=False, old coordinates unrotated."""
+    wl = sub(W1, n_kv_heads=2, n_q_heads=8, tokens=900)
+    kd, kv, vd, vv = joint_workload_arrays(wl, variant="gapped")
+    cache = make_cache(wl, rotate_history=False)
+    orc = OracleCache(wl.batch, wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim,
+                      wl.rank_k, wl.rank_v, wl.block, wl.window, rope=wl.rope,
+                      rope_theta=wl.rope_theta, rotate=False, joint=True)
+    cache.append(0, to_device(kd[0]), to_device(vd[0]))
+    orc.append(0, kv[0], vv[0])
+    for x in (0, 1):
+        u = orc.unit(0, 0, 0, x)
+        assert rel_err(cache.reconstruct(0, x).cpu().numpy(), orc.reconstruct(0, x)) <= 1e-3
+        _, B, S, k, n = joint_factors(cache, wl, 0, 0, x)
+        assert k == u.k and n == u.n
+        assert np.max(np.abs(S[:k] - u.sigma) / u.sigma) <= SIG_TOL
+    q = syn.queries(71, (1, 8, 128))
+    out = cache.decode(0, torch.from_numpy(q).cuda()).cpu().numpy()
+    assert max_head_rel_err(out, orc.decode(0, q.astype(np.float64))) <= ATTN_TOL
+    assert cache.status() == 0
