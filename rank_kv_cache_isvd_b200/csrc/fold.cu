@@ -81,6 +81,38 @@ __device__ __forceinline__ void jparams(float g, float nx, float ny, float floor
     dc = __fdividef(t * t * ri * ri, 1.f + ri);          // 1 - c
 }
 
+// Dot product of a lane's RPL rows of two columns, two rows per packed fp32x2 FMA.
+template <int RPL>
+__device__ __forceinline__ float jdot(const float (&x)[RPL], const float (&y)[RPL]) {
+    float2 g2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i + 1 < RPL; i += 2)
+        g2 = __ffma2_rn(make_float2(x[i], x[i + 1]), make_float2(y[i], y[i + 1]), g2);
+    if (RPL & 1) g2.x = fmaf(x[RPL - 1], y[RPL - 1], g2.x);
+    return g2.x + g2.y;
+}
+
+// x <- x - dc x - sn y, y <- y - dc y + sn x over a lane's RPL rows (packed fp32x2 FMAs).
+template <int RPL>
+__device__ __forceinline__ void jturn(float (&x)[RPL], float (&y)[RPL], float sn, float dc) {
+    const float2 ndc = make_float2(-dc, -dc), nsn = make_float2(-sn, -sn), psn = make_float2(sn, sn);
+#pragma unroll
+    for (int i = 0; i + 1 < RPL; i += 2) {
+        const float2 xi = make_float2(x[i], x[i + 1]), yi = make_float2(y[i], y[i + 1]);
+        const float2 xo = __ffma2_rn(nsn, yi, __ffma2_rn(ndc, xi, xi));
+        const float2 yo = __ffma2_rn(psn, xi, __ffma2_rn(ndc, yi, yi));
+        x[i] = xo.x;
+        x[i + 1] = xo.y;
+        y[i] = yo.x;
+        y[i + 1] = yo.y;
+    }
+    if (RPL & 1) {
+        const float xi = x[RPL - 1], yi = y[RPL - 1];
+        x[RPL - 1] = fmaf(-sn, yi, fmaf(-dc, xi, xi));
+        y[RPL - 1] = fmaf(sn, xi, fmaf(-dc, yi, yi));
+    }
+}
+
 // Rotates HC disjoint column pairs (x_j, y_(j+S) mod HC) of a lane group at once: the dot
 // products, their reductions and the rotation parameters of all pairs overlap (no branches).
 template <int HC, int RPL, int S>
@@ -88,11 +120,7 @@ __device__ __forceinline__ void jcross(float (&xa)[HC][RPL], float (&xb)[HC][RPL
                                        float (&nb)[HC], float floor2, int &rotated) {
     float g[HC];
 #pragma unroll
-    for (int j = 0; j < HC; ++j) {
-        g[j] = 0.f;
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) g[j] = fmaf(xa[j][i], xb[(j + S) % HC][i], g[j]);
-    }
+    for (int j = 0; j < HC; ++j) g[j] = jdot<RPL>(xa[j], xb[(j + S) % HC]);
 #pragma unroll
     for (int o = 1; o < JL; o <<= 1)
 #pragma unroll
@@ -102,12 +130,7 @@ __device__ __forceinline__ void jcross(float (&xa)[HC][RPL], float (&xb)[HC][RPL
         const int jb = (j + S) % HC;
         float t, sn, dc;
         jparams(g[j], na[j], nb[jb], floor2, t, sn, dc);
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-            const float xi = xa[j][i], yi = xb[jb][i];
-            xa[j][i] = fmaf(-sn, yi, fmaf(-dc, xi, xi));
-            xb[jb][i] = fmaf(sn, xi, fmaf(-dc, yi, yi));
-        }
+        jturn<RPL>(xa[j], xb[jb], sn, dc);
         na[j] = fmaxf(na[j] - t * g[j], 0.f);
         nb[jb] = fmaxf(nb[jb] + t * g[j], 0.f);
         rotated |= (t != 0.f);
@@ -118,18 +141,10 @@ __device__ __forceinline__ void jcross(float (&xa)[HC][RPL], float (&xb)[HC][RPL
 template <int RPL>
 __device__ __forceinline__ void jrot(float (&x)[RPL], float (&y)[RPL], float &nx, float &ny,
                                      float floor2, int &rotated) {
-    float g = 0.f;
-#pragma unroll
-    for (int i = 0; i < RPL; ++i) g = fmaf(x[i], y[i], g);
-    g = group_sum(g);
+    const float g = group_sum(jdot<RPL>(x, y));
     float t, sn, dc;
     jparams(g, nx, ny, floor2, t, sn, dc);
-#pragma unroll
-    for (int i = 0; i < RPL; ++i) {
-        const float xi = x[i], yi = y[i];
-        x[i] = fmaf(-sn, yi, fmaf(-dc, xi, xi));
-        y[i] = fmaf(sn, xi, fmaf(-dc, yi, yi));
-    }
+    jturn<RPL>(x, y, sn, dc);
     nx = fmaxf(nx - t * g, 0.f);
     ny = fmaxf(ny + t * g, 0.f);
     rotated |= (t != 0.f);
