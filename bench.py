@@ -598,7 +598,22 @@ def llama_layer_stream(args, dev, flush):
             "how": "graph replay of reset + 4096 append+decode calls + join, L2 flushed",
             "fold_ms_per_append": float(np.median(fms)),
             "fold_us_per_fold": 1e3 * float(np.median(fms)) / folds,
-            "fold_head_block_updates_per_s": folds * H * 2 / (float(np.median(fms)) / 1e3)}
+            "fold_head_block_updates_per_s": folds * H * 2 / (float(np.median(fms)) / 1e3),
+            **fold_latency_roofline(wl, float(np.median(fms)) * 1e3 / folds)}
+
+
+def fold_latency_roofline(wl, fold_us: float) -> dict:
+    """Latency roofline of one steady-state fold (k = r): the two paths' cores run on separate SMs,
+    so a fold takes at least the slower path's core SVD cost 2 m n^2 + 11 n^3 (m = k + b,
+    n = k + p) at one SM's fp32 FMA rate (128 lanes x 2 flops x 1.965 GHz)."""
+    sm_flops = 128 * 2 * 1.965e9
+    worst = 0.0
+    for r in (wl.rank_k, wl.rank_v):
+        k = min(r, D)
+        p = min(wl.block, D - k)
+        m, n = k + wl.block, k + p
+        worst = max(worst, (2 * m * n * n + 11 * n ** 3) / sm_flops * 1e6)
+    return {"fold_latency_roofline_us": worst, "fold_latency_frac": worst / fold_us}
 
 
 def all_layers_decode_step(args, dev, flush, steps: int = 5):
