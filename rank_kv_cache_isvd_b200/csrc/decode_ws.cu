@@ -426,6 +426,12 @@ __device__ __forceinline__ float4 load_v4s(const uint8_t *row, int c, int fmt) {
 struct WsRange {
     long long g0, g1;
 };
+// First tile of a unit whose partition slot is at or after slot o: the Tc compressed tiles take
+// one slot each, every exact-row tile (protected or window) W slots.
+__host__ __device__ inline int ws_vtile(int o, int Tc, int W) {
+    return o <= Tc ? o : Tc + (o - Tc + W - 1) / W;
+}
+
 __device__ __forceinline__ WsRange ws_range(const WsExtra &x, int c) {
     WsRange r;
     r.g0 = (long long)c * x.N / x.P;
@@ -497,12 +503,15 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
     else
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(WS_REG_HI));
 
-    // every segment of this CTA, in order: unit u, tiles [ta, tb) of the unit
-    auto seg_of = [&](long long g, long long &u, int &ta, int &tb) {
+    // every segment of this CTA, in order: unit u, tiles [ta, tb) of the unit (those whose first
+    // partition slot lies in the CTA's range; possibly none), and the slots it spans
+    auto seg_of = [&](long long g, long long &u, int &ta, int &tb, int &adv) {
         u = g / Tu;
-        ta = (int)(g - u * Tu);
-        const long long left = rg.g1 - g;
-        tb = (int)min((long long)Tu, ta + left);
+        const int o0 = (int)(g - u * Tu);
+        const int o1 = (int)min((long long)Tu, o0 + (rg.g1 - g));
+        ta = ws_vtile(o0, Tc, x.W);
+        tb = ws_vtile(o1, Tc, x.W);
+        adv = o1 - o0;
     };
 
     if (warp == 0) {
@@ -515,8 +524,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
             bool ok = true;
             for (long long g = rg.g0; g < rg.g1 && ok;) {
                 long long u;
-                int ta, tb;
-                seg_of(g, u, ta, tb);
+                int ta, tb, adv;
+                seg_of(g, u, ta, tb, adv);
                 const int seq = (int)(u / a.H), h = (int)(u % a.H);
                 // queries of this unit's q-heads
                 const int qs = seg & 1;
@@ -585,7 +594,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
                     }
                     counters[3] = vt;
                 }
-                g += tb - ta;
+                g += adv;
             }
         }
     } else if (warp < 4) {
@@ -597,9 +606,9 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
         const uint32_t idesc = BF ? idesc_bf16(128, 128) : idesc_tf32(128, 128);
         for (long long g = rg.g0; g < rg.g1 && ok;) {
             long long u;
-            int ta, tb;
-            seg_of(g, u, ta, tb);
-            g += tb - ta;
+            int ta, tb, adv;
+            seg_of(g, u, ta, tb, adv);
+            g += adv;
             if (ta >= Tc) continue;
             bool w;
             if (BF) {
@@ -770,9 +779,9 @@ __global__ void __launch_bounds__(WS_THREADS, 1) decode_ws_kernel(
 
         for (long long g = rg.g0; g < rg.g1 && ok;) {
             long long u;
-            int ta, tb;
-            seg_of(g, u, ta, tb);
-            g += tb - ta;
+            int ta, tb, adv;
+            seg_of(g, u, ta, tb, adv);
+            g += adv;
             const int jseg = (int)(u - u_first);
             const int qs = seg & 1;
             bool w = wait_ab(q_full + qs, (seg >> 1) & 1, abort_flag);

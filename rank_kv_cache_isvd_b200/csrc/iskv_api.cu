@@ -795,7 +795,10 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
         x.brow0 = (cur * h->U + layer * h->UL) * D;
         x.Tc = (int)ctiles;
         x.Tw = (int)((e + DEC_TILE - 1) / DEC_TILE);
-        x.Tu = x.Tc + x.Tw;
+        // an exact-row tile (keys read and rotated on CUDA cores, values summed over 128 channels)
+        // costs about three compressed tiles: it takes three slots of the CTAs' equal shares
+        x.W = 3;
+        x.Tu = x.Tc + x.W * x.Tw;
         x.UL = h->UL;
         x.N = (long long)h->UL * x.Tu;
         x.P = (int)(x.N < h->sms ? x.N : h->sms);
@@ -813,7 +816,7 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
             }
             x.pcap = h->pcap;
             x.Tp = h->ptiles[layer];
-            x.Tu = x.Tc + x.Tp + x.Tw;
+            x.Tu = x.Tc + x.W * (x.Tp + x.Tw);
             x.N = (long long)h->UL * x.Tu;
             x.P = (int)(x.N < h->sms ? x.N : h->sms);
             x.maxseg = h->UL / x.P + 2;

@@ -225,7 +225,8 @@ struct WsExtra {
     long long rope_rows;    // rows of the (cos, sin) table a.rope_cs
     long long row0;         // first coordinate row of this layer in the coordinate tensor map
     int brow0;              // first basis row of this layer (current buffer) in the basis map
-    int Tc, Tw, Tu;         // tiles per unit: compressed, window, total
+    int Tc, Tw, Tu;         // tiles per unit: compressed, window; Tu: partition slots per unit
+    int W;                  // partition slots of an exact-row (window or protected) tile
     long long N;            // tiles of the layer: units * Tu
     int P;                  // CTAs (one per SM, at most N)
     int maxseg;             // partial records per CTA (units / P + 2)
