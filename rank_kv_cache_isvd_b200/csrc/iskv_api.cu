@@ -796,8 +796,9 @@ int decode_layer(iskv_handle *h, int layer, const float *q, float *out, cudaStre
         x.Tc = (int)ctiles;
         x.Tw = (int)((e + DEC_TILE - 1) / DEC_TILE);
         // an exact-row tile (keys read and rotated on CUDA cores, values summed over 128 channels)
-        // costs about three compressed tiles: it takes three slots of the CTAs' equal shares
-        x.W = 3;
+        // costs several compressed tiles: it takes four slots of the CTAs' equal shares (measured
+        // best of 2 .. 6 on the 64-unit 32K-token and the 8-unit 16K-token layer calls)
+        x.W = 4;
         x.Tu = x.Tc + x.W * x.Tw;
         x.UL = h->UL;
         x.N = (long long)h->UL * x.Tu;
