@@ -257,3 +257,35 @@ def test_joint_stale_coordinates_mode_matches_oracle():
     out = cache.decode(0, torch.from_numpy(q).cuda()).cpu().numpy()
     assert max_head_rel_err(out, orc.decode(0, q.astype(np.float64))) <= ATTN_TOL
     assert cache.status() == 0
+
+
+def test_joint_full_size_layer_sampled_sequence():
+    """The bench's joint layer at full size (Qwen3-8B-shaped: batch 8 x 8 kv-heads, 32 q-heads,
+    32768 tokens in one append, b = 64, w = 256, r_K = 32, r_V = 64, rows drawn on the GPU): every
+    output is finite and the 32 q-heads of a sampled sequence match the oracle's joint unit run on
+    that sequence's rows alone."""
+    wl = dataclasses.replace(syn.WORKLOADS[3], block=64)
+    S, H, T, QH = wl.batch, wl.n_kv_heads, wl.tokens, wl.n_q_heads
+    cache = make_cache(sub(wl, n_layers=1))
+    K = syn.device_rows_batch(wl, range(S), 0, range(H), 0)
+    V = syn.device_rows_batch(wl, range(S), 0, range(H), 1)
+    cache.append(0, K, V)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(2024)
+    q = torch.randn((S, QH, 128), generator=gen, device="cuda")
+    out = cache.decode(0, q).cpu().numpy()
+    assert cache.status() == 0 and np.isfinite(out).all() and cache.tokens(0) == T
+    sq = 5
+    orc = OracleCache(1, 1, H, QH, 128, wl.rank_k, wl.rank_v, wl.block, wl.window, rope=wl.rope,
+                      rope_theta=wl.rope_theta, joint=True)
+    orc.append(0, K[sq:sq + 1].float().cpu().numpy().astype(np.float64),
+               V[sq:sq + 1].float().cpu().numpy().astype(np.float64))
+    ref = orc.decode(0, q[sq:sq + 1].cpu().numpy().astype(np.float64))
+    err = max_head_rel_err(out[sq:sq + 1], ref)
+    print(f"\njoint full size, sequence {sq}: attention rel err {err:.3e}")
+    assert err <= ATTN_TOL
+    for x in (0, 1):
+        _, _, _, k, n = cache.factors(0, sq, 0, x)
+        u = orc.unit(0, 0, 0, x)
+        assert n == u.n == wl.n_c(T) and k == u.k
+    cache.close()
