@@ -299,7 +299,9 @@ int iskv_sync_status(iskv_handle *h, iskv_stream_t stream);
  * stream. The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and keeps it; make that first call before any
  * stream capture.
- *   view:    cache description (layouts below), all pointers device pointers owned by the caller;
+ *   view:    cache description (layouts below), all pointers device pointers owned by the caller
+ *            (one coordinate array per kv-head unit: a joint-factorisation cache, whose kv-heads
+ *            share their coordinates, is decoded through iskv_decode_attn instead);
  *   q_dev:   fp32 [batch][n_q_heads][head_dim], already rotated for the query position;
  *   out_dev: fp32 [batch][n_q_heads][head_dim].
  * Errors: ISKV_ERR_INVALID_ARG (NULL pointer, inconsistent sizes), ISKV_ERR_CAPACITY (scratch
