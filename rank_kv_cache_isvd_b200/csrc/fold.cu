@@ -916,80 +916,113 @@ __global__ void __launch_bounds__(FT, 1) fold_core_kernel(FoldArgs a) {
 // History rotation: old coordinates move with the basis, C[0:n] <- C[0:n] H[:k] (iS-KV summary,
 // "Block-Incremental Decoding Updates", U+ = diag(U, I_b) G, so the old rows of U+ Sigma+ are
 // U Sigma H[:k]). Stale mode keeps the old coordinates (zero-padded to the new rank).
-constexpr int ROT_ROWS = 64;                  // rows per tile
-constexpr int ROT_THREADS = 256;              // 16 row groups (4 rows) x 16 column groups
-constexpr int ROT_XS = ROT_ROWS + 4;          // stride of the transposed row tile
+constexpr int ROT_THREADS = 256;              // 16 row groups x 16 column groups
 constexpr int ROT_GX = 24;                    // CTAs per (unit, path); each takes every 24th tile
 constexpr int ROT_HS = 128;                   // stride of H_top in shared memory
 
-// One tile: acc[rr][cc] = sum_l X[4 rg + rr][l] H[l][CW cg + cc]; X^T and H in shared memory.
-// Each thread keeps a 4 x CW block of outputs in registers, so every shared-memory load feeds
-// 4 or CW fused multiply-adds (packed in pairs of columns for even CW).
-template <int CW>
+// One tile: acc[rr][cc] = sum_l X[RPT rg + rr][l] H[l][CW cg + cc] (X^T and H in shared memory,
+// transposed tile stride XS), stored to rows RPT rg + rr < rows, columns CW cg + cc < r of the
+// coordinates. Each thread keeps an RPT x CW block of outputs in registers, so every shared-memory
+// load feeds RPT or CW fused multiply-adds (packed in pairs of columns for even CW).
+template <int CW, int RPT, int XS>
 __device__ __forceinline__ void rot_tile(const float *sXt, const float *sH, int k, int rg, int cg,
-                                         float (&acc)[4][8]) {
-#pragma unroll
-    for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) acc[rr][cc] = 0.f;
+                                         void *coords, size_t cu, long long row0, int rows, int r,
+                                         int cbf) {
+    float acc[RPT][CW];
     if constexpr ((CW & 1) == 0) {
         // even widths: H columns as float2 pairs, packed fused multiply-adds
-        float2 a2[4][CW / 2];
+        float2 a2[RPT][CW / 2];
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr)
+        for (int rr = 0; rr < RPT; ++rr)
 #pragma unroll
             for (int c2 = 0; c2 < CW / 2; ++c2) a2[rr][c2] = make_float2(0.f, 0.f);
 #pragma unroll 4
         for (int l = 0; l < k; ++l) {
-            const float4 x = *reinterpret_cast<const float4 *>(sXt + l * ROT_XS + 4 * rg);
-            const float xs[4] = {x.x, x.y, x.z, x.w};
+            float xs[RPT];
+#pragma unroll
+            for (int q = 0; q < RPT / 4; ++q) {
+                const float4 x = *reinterpret_cast<const float4 *>(sXt + l * XS + RPT * rg + 4 * q);
+                xs[4 * q] = x.x;
+                xs[4 * q + 1] = x.y;
+                xs[4 * q + 2] = x.z;
+                xs[4 * q + 3] = x.w;
+            }
             float2 hv[CW / 2];
 #pragma unroll
             for (int c2 = 0; c2 < CW / 2; ++c2)
                 hv[c2] = *reinterpret_cast<const float2 *>(sH + l * ROT_HS + CW * cg + 2 * c2);
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
+            for (int rr = 0; rr < RPT; ++rr) {
                 const float2 xx = make_float2(xs[rr], xs[rr]);
 #pragma unroll
                 for (int c2 = 0; c2 < CW / 2; ++c2) a2[rr][c2] = __ffma2_rn(xx, hv[c2], a2[rr][c2]);
             }
         }
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr)
+        for (int rr = 0; rr < RPT; ++rr)
 #pragma unroll
             for (int c2 = 0; c2 < CW / 2; ++c2) {
                 acc[rr][2 * c2] = a2[rr][c2].x;
                 acc[rr][2 * c2 + 1] = a2[rr][c2].y;
             }
     } else {
+#pragma unroll
+        for (int rr = 0; rr < RPT; ++rr)
+#pragma unroll
+            for (int cc = 0; cc < CW; ++cc) acc[rr][cc] = 0.f;
 #pragma unroll 4
         for (int l = 0; l < k; ++l) {
-            const float4 x = *reinterpret_cast<const float4 *>(sXt + l * ROT_XS + 4 * rg);
-            const float xs[4] = {x.x, x.y, x.z, x.w};
+            float xs[RPT];
+#pragma unroll
+            for (int q = 0; q < RPT / 4; ++q) {
+                const float4 x = *reinterpret_cast<const float4 *>(sXt + l * XS + RPT * rg + 4 * q);
+                xs[4 * q] = x.x;
+                xs[4 * q + 1] = x.y;
+                xs[4 * q + 2] = x.z;
+                xs[4 * q + 3] = x.w;
+            }
             float hv[CW];
 #pragma unroll
             for (int cc = 0; cc < CW; ++cc) hv[cc] = sH[l * ROT_HS + CW * cg + cc];
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr)
+            for (int rr = 0; rr < RPT; ++rr)
 #pragma unroll
                 for (int cc = 0; cc < CW; ++cc) acc[rr][cc] = fmaf(xs[rr], hv[cc], acc[rr][cc]);
         }
     }
+    // rows RPT rg .. RPT rg + RPT - 1, columns CW cg .. ; the columns kp .. r - 1 are cleared by
+    // the column groups past kp (their H columns are zero)
+#pragma unroll
+    for (int rr = 0; rr < RPT; ++rr) {
+        const int i = RPT * rg + rr;
+        if (i >= rows) continue;
+        const size_t base = cu + (size_t)(row0 + i) * r;
+#pragma unroll
+        for (int cc = 0; cc < CW; ++cc) {
+            const int c = CW * cg + cc;
+            if (c < r) store_coord(coords, base + c, acc[rr][cc], cbf);
+        }
+    }
 }
 
+// RPT rows per thread, tiles of 16 RPT rows (64 or 128).
+template <int RPT>
 __global__ void __launch_bounds__(ROT_THREADS, 2) rotate_kernel(RotArgs a) {
+    constexpr int ROWS = 16 * RPT;
+    constexpr int XS = ROWS + 4;              // stride of the transposed row tile
+    constexpr int LOGR = RPT == 8 ? 7 : 6;
     extern __shared__ float smem[];
     const RotPath P = (a.path_lo + (int)blockIdx.z) ? a.path[1] : a.path[0];
     const int unit = a.unit0 + blockIdx.y;
     const int k = P.k, kp = P.kp, r = P.r;
     const int tid = threadIdx.x;
-    const long long tiles = (a.n_old + ROT_ROWS - 1) / ROT_ROWS;
+    const long long tiles = (a.n_old + ROWS - 1) / ROWS;
     const size_t cu = (size_t)unit * a.n_max * r;
     if (a.stale) {
         // stale coordinates: kept as they are, columns k .. kp - 1 zero
         for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
-            const long long row0 = t * ROT_ROWS;
-            const int rows = (int)min((long long)ROT_ROWS, a.n_old - row0);
+            const long long row0 = t * ROWS;
+            const int rows = (int)min((long long)ROWS, a.n_old - row0);
             for (int o = tid; o < rows * (r - k); o += ROT_THREADS) {
                 const int i = o / (r - k), c = k + o % (r - k);
                 store_coord(P.coords, cu + (size_t)(row0 + i) * r + c, 0.f, a.cbf);
@@ -998,7 +1031,7 @@ __global__ void __launch_bounds__(ROT_THREADS, 2) rotate_kernel(RotArgs a) {
         return;
     }
     float *sH = smem;                         // [k][ROT_HS], zero past kp
-    float *sXt = sH + k * ROT_HS;             // [k][ROT_XS]: column l of the row tile
+    float *sXt = sH + k * ROT_HS;             // [k][XS]: column l of the row tile
     const float *ht = P.htop + (size_t)unit * r * r;
     for (int o = tid; o < k * ROT_HS; o += ROT_THREADS) {
         const int l = o / ROT_HS, c = o % ROT_HS;
@@ -1007,17 +1040,17 @@ __global__ void __launch_bounds__(ROT_THREADS, 2) rotate_kernel(RotArgs a) {
     const int rg = tid >> 4, cg = tid & 15;
     const int cw = (kp + 15) >> 4;            // columns per thread (1 .. 8)
     // fp32 coordinates in 16-byte quads: the next tile's rows are loaded into registers while
-    // this tile is computed (thread: row i = o mod 64 of quad q = o / 64 for o = tid + 256 s)
+    // this tile is computed (thread: row i = o mod ROWS of quad q = o / ROWS for o = tid + 256 s)
     const bool vec = !a.cbf && (k & 3) == 0 && (r & 3) == 0;
-    const int nq = vec ? (ROT_ROWS * (k >> 2) + ROT_THREADS - 1) / ROT_THREADS : 0;   // <= 8
+    const int nq = vec ? (ROWS * (k >> 2) + ROT_THREADS - 1) / ROT_THREADS : 0;   // <= 8
     float4 pre[8];
     auto prefetch = [&](long long t) {
-        const long long row0 = t * ROT_ROWS;
-        const int rows = (int)min((long long)ROT_ROWS, a.n_old - row0);
+        const long long row0 = t * ROWS;
+        const int rows = (int)min((long long)ROWS, a.n_old - row0);
         const float *cf = static_cast<const float *>(P.coords) + cu;
 #pragma unroll
         for (int sq = 0; sq < 8; ++sq) {
-            const int o = tid + ROT_THREADS * sq, i = o & (ROT_ROWS - 1), q = o >> 6;
+            const int o = tid + ROT_THREADS * sq, i = o & (ROWS - 1), q = o >> LOGR;
             pre[sq] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (sq < nq && 4 * q < k && i < rows)
                 pre[sq] = *reinterpret_cast<const float4 *>(cf + (size_t)(row0 + i) * r + 4 * q);
@@ -1025,52 +1058,45 @@ __global__ void __launch_bounds__(ROT_THREADS, 2) rotate_kernel(RotArgs a) {
     };
     if (vec && blockIdx.x < tiles) prefetch(blockIdx.x);
     for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
-        const long long row0 = t * ROT_ROWS;
-        const int rows = (int)min((long long)ROT_ROWS, a.n_old - row0);
+        const long long row0 = t * ROWS;
+        const int rows = (int)min((long long)ROWS, a.n_old - row0);
         __syncthreads();                      // previous tile's reads of sXt are done
         if (vec) {
             // transposed store of the prefetched rows (consecutive threads: consecutive rows)
 #pragma unroll
             for (int sq = 0; sq < 8; ++sq) {
-                const int o = tid + ROT_THREADS * sq, i = o & (ROT_ROWS - 1), q = o >> 6;
+                const int o = tid + ROT_THREADS * sq, i = o & (ROWS - 1), q = o >> LOGR;
                 if (sq < nq && 4 * q < k) {
-                    sXt[(4 * q + 0) * ROT_XS + i] = pre[sq].x;
-                    sXt[(4 * q + 1) * ROT_XS + i] = pre[sq].y;
-                    sXt[(4 * q + 2) * ROT_XS + i] = pre[sq].z;
-                    sXt[(4 * q + 3) * ROT_XS + i] = pre[sq].w;
+                    sXt[(4 * q + 0) * XS + i] = pre[sq].x;
+                    sXt[(4 * q + 1) * XS + i] = pre[sq].y;
+                    sXt[(4 * q + 2) * XS + i] = pre[sq].z;
+                    sXt[(4 * q + 3) * XS + i] = pre[sq].w;
                 }
             }
         } else {
-            for (int o = tid; o < ROT_ROWS * k; o += ROT_THREADS) {
+            for (int o = tid; o < ROWS * k; o += ROT_THREADS) {
                 const int i = o / k, l = o % k;
-                sXt[l * ROT_XS + i] = i < rows ? load_coord(P.coords, cu + (size_t)(row0 + i) * r + l, a.cbf) : 0.f;
+                sXt[l * XS + i] = i < rows ? load_coord(P.coords, cu + (size_t)(row0 + i) * r + l, a.cbf) : 0.f;
             }
         }
         __syncthreads();
         if (vec && t + gridDim.x < tiles) prefetch(t + gridDim.x);
-        float acc[4][8];
+        // (the 8-row variant runs only with kp <= 64: at most 4 columns per thread)
         switch (cw) {
-            case 1: rot_tile<1>(sXt, sH, k, rg, cg, acc); break;
-            case 2: rot_tile<2>(sXt, sH, k, rg, cg, acc); break;
-            case 3: rot_tile<3>(sXt, sH, k, rg, cg, acc); break;
-            case 4: rot_tile<4>(sXt, sH, k, rg, cg, acc); break;
-            case 5: rot_tile<5>(sXt, sH, k, rg, cg, acc); break;
-            case 6: rot_tile<6>(sXt, sH, k, rg, cg, acc); break;
-            case 7: rot_tile<7>(sXt, sH, k, rg, cg, acc); break;
-            default: rot_tile<8>(sXt, sH, k, rg, cg, acc); break;
-        }
-        // rows 4 rg .. 4 rg + 3, columns cw cg .. ; the columns kp .. r - 1 are cleared by the
-        // column groups past kp (their H columns are zero)
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            const int i = 4 * rg + rr;
-            if (i >= rows) continue;
-            const size_t base = cu + (size_t)(row0 + i) * r;
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                const int c = cw * cg + cc;
-                if (cc < cw && c < r) store_coord(P.coords, base + c, acc[rr][cc], a.cbf);
-            }
+            case 1: rot_tile<1, RPT, XS>(sXt, sH, k, rg, cg, P.coords, cu, row0, rows, r, a.cbf); break;
+            case 2: rot_tile<2, RPT, XS>(sXt, sH, k, rg, cg, P.coords, cu, row0, rows, r, a.cbf); break;
+            case 3: rot_tile<3, RPT, XS>(sXt, sH, k, rg, cg, P.coords, cu, row0, rows, r, a.cbf); break;
+            case 4: rot_tile<4, RPT, XS>(sXt, sH, k, rg, cg, P.coords, cu, row0, rows, r, a.cbf); break;
+            default:
+                if constexpr (RPT == 4) {
+                    switch (cw) {
+                        case 5: rot_tile<5, 4, XS>(sXt, sH, k, rg, cg, P.coords, cu, row0, rows, r, a.cbf); break;
+                        case 6: rot_tile<6, 4, XS>(sXt, sH, k, rg, cg, P.coords, cu, row0, rows, r, a.cbf); break;
+                        case 7: rot_tile<7, 4, XS>(sXt, sH, k, rg, cg, P.coords, cu, row0, rows, r, a.cbf); break;
+                        default: rot_tile<8, 4, XS>(sXt, sH, k, rg, cg, P.coords, cu, row0, rows, r, a.cbf); break;
+                    }
+                }
+                break;
         }
         // columns past 16 cw (only when kp < r and 16 cw < r): zero
         if (16 * cw < r) {
@@ -1094,15 +1120,32 @@ cudaError_t launch_fold(const FoldArgs &a, int n_units, cudaStream_t s) {
 
 cudaError_t launch_rotate(const RotArgs &a, int n_units, cudaStream_t s) {
     if (a.n_old <= 0 || a.path_hi <= a.path_lo || n_units <= 0) return cudaSuccess;
-    int kmax = 0;
-    for (int x = a.path_lo; x < a.path_hi; ++x) kmax = a.path[x].k > kmax ? a.path[x].k : kmax;
-    const size_t smem = (size_t)kmax * (ROT_HS + ROT_XS) * sizeof(float) + 16;
-    static size_t attr[64] = {0};
-    const cudaError_t e = ensure_smem((const void *)rotate_kernel, smem, attr);
-    if (e != cudaSuccess) return e;
-    const long long tiles = (a.n_old + ROT_ROWS - 1) / ROT_ROWS;
+    int kmax = 0, kpmax = 0;
+    bool quads = !a.cbf;
+    for (int x = a.path_lo; x < a.path_hi; ++x) {
+        kmax = a.path[x].k > kmax ? a.path[x].k : kmax;
+        kpmax = a.path[x].kp > kpmax ? a.path[x].kp : kpmax;
+        quads = quads && (a.path[x].k & 3) == 0 && (a.path[x].r & 3) == 0;
+    }
+    // 8 rows per thread (128-row tiles) where the prefetch registers allow it (k <= 64) and the
+    // output block stays small (kp <= 64); else 4 rows per thread (64-row tiles)
+    const bool wide = quads && kmax <= 64 && kpmax <= 64;
+    const int rows = wide ? 128 : 64;
+    const size_t smem = (size_t)kmax * (ROT_HS + rows + 4) * sizeof(float) + 16;
+    const long long tiles = (a.n_old + rows - 1) / rows;
     const long long gx = tiles < ROT_GX ? tiles : ROT_GX;
-    rotate_kernel<<<dim3((unsigned)gx, n_units, a.path_hi - a.path_lo), ROT_THREADS, smem, s>>>(a);
+    const dim3 grid((unsigned)gx, n_units, a.path_hi - a.path_lo);
+    if (wide) {
+        static size_t attr[64] = {0};
+        const cudaError_t e = ensure_smem((const void *)rotate_kernel<8>, smem, attr);
+        if (e != cudaSuccess) return e;
+        rotate_kernel<8><<<grid, ROT_THREADS, smem, s>>>(a);
+    } else {
+        static size_t attr[64] = {0};
+        const cudaError_t e = ensure_smem((const void *)rotate_kernel<4>, smem, attr);
+        if (e != cudaSuccess) return e;
+        rotate_kernel<4><<<grid, ROT_THREADS, smem, s>>>(a);
+    }
     return cudaGetLastError();
 }
 
